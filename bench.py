@@ -1,0 +1,409 @@
+#!/usr/bin/env python
+"""Benchmark of the tile-hybrid (dense | 2:4) decode GEMV on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl hyb|reference]
+                    [--workload NAME] [--sweep]
+
+One step = one hyb_spmv call (the whole hot path: stream the packed values and
+masks, decode, fp32 FMA, reduce, store) on the headline workload:
+
+    ffn_down_4096x14336_f0.5_b1 -- the Llama-shaped FFN down projection
+    (n=4096 outputs, k=14336 inputs), bf16 N(0, 0.02) with 1 % x20 outliers,
+    128x128 tiles of which half are 2:4 (seeded shuffle), batch 1.
+
+Inputs are larger than L2: each step uses the next of 16 packed copies of the
+matrix (1.47 GB in total), so every step streams from HBM.  The printed value
+is achieved GB/s over the algorithmic bytes (packed values + masks + tile map +
+x + y).  With N > 1 (torchrun) every rank runs its own replica (the product is
+not sharded; weak scaling) and the time is the max over ranks.
+
+--impl reference times the CPU oracle on a bounded row sample of the same
+workload (rank 0 only).
+"""
+import argparse
+import ctypes
+import hashlib
+import json
+import os
+import re
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from sparse_weight_b200 import hyb, inputs  # noqa: E402
+
+FALLBACK_HBM_GBS = 6650.0
+NOMINAL_HBM_GBS = 8000.0
+ROTATE = 16
+
+WORKLOADS = {
+    # name: (n, k, b1, b2, frac, batch, std, outliers)
+    "ffn_down_4096x14336_f0.5_b1": (4096, 14336, 128, 128, 0.5, 1, 0.02, 0.01),
+    "ffn_up_14336x4096_f0.5_b1": (14336, 4096, 128, 128, 0.5, 1, 0.02, 0.01),
+    "attn_4096x4096_bern0.5_b1": (4096, 4096, 128, 128, None, 1, 0.02, 0.0),
+}
+
+
+# ---------------------------------------------------------------------------
+# environment helpers
+# ---------------------------------------------------------------------------
+
+def dist_env():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def measured_peak():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as fh:
+            d = json.load(fh)
+        return float(d["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def csrc_digest():
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "sparse_weight_b200", "csrc")
+    for name in sorted(os.listdir(csrc)):
+        with open(os.path.join(csrc, name), "rb") as fh:
+            h.update(name.encode())
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic(workload):
+    """DRAM bytes per launch from the committed ncu summary of this workload,
+    if it was taken on the current kernel sources; else None."""
+    path = os.path.join(ROOT, "profiles", f"hybrid_stream_kernel_{workload}.md")
+    try:
+        txt = open(path).read()
+    except OSError:
+        return None
+    src = re.search(r"csrc_sha:\s*([0-9a-f]+)", txt)
+    tr = re.search(r"dram_bytes_per_launch:\s*([0-9]+)", txt)
+    if not src or not tr or src.group(1) != csrc_digest():
+        return None
+    return int(tr.group(1))
+
+
+class ClockSampler:
+    """Samples SM clock and throttle reasons through NVML while running."""
+
+    REASONS = {
+        "gpu_idle": 0x1, "applications_clocks_setting": 0x2, "sw_power_cap": 0x4,
+        "hw_slowdown": 0x8, "sync_boost": 0x10, "sw_thermal_slowdown": 0x20,
+        "hw_thermal_slowdown": 0x40, "hw_power_brake_slowdown": 0x80,
+        "display_clock_setting": 0x100,
+    }
+
+    def __init__(self, index, period=0.005):
+        self.samples = []
+        self.reasons = set()
+        self.max_mhz = None
+        self.ok = False
+        self.period = period
+        self._stop = threading.Event()
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception:
+            self.nv = None
+
+    def _sample(self):
+        mhz = self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM)
+        bits = self.nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+        self.samples.append(mhz)
+        for name, b in self.REASONS.items():
+            if bits & b and name != "gpu_idle":
+                self.reasons.add(name)
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                self._sample()
+            except Exception:
+                return
+            time.sleep(self.period)
+
+    def __enter__(self):
+        if self.ok:
+            self._t = threading.Thread(target=self._run, daemon=True)
+            self._t.start()
+        return self
+
+    def __exit__(self, *exc):
+        if self.ok:
+            self._stop.set()
+            self._t.join()
+
+    def summary(self):
+        if not self.ok or not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons),
+                    "samples": len(self.samples)}
+        return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons), "samples": len(self.samples)}
+
+
+# ---------------------------------------------------------------------------
+# workload
+# ---------------------------------------------------------------------------
+
+def make_matrix(name):
+    n, k, b1, b2, frac, batch, std, outliers = WORKLOADS[name]
+    T = (n // b1) * (k // b2)
+    if frac is None:
+        tmap = inputs.tile_map_bernoulli(T, 0.5, inputs.seed_of(name, "map"))
+    else:
+        tmap = inputs.tile_map_fraction(T, frac, inputs.seed_of(name, "map"))
+    W = inputs.weight(n, k, std, inputs.seed_of(name, "W"), outliers=outliers)
+    return W, tmap
+
+
+class Workload:
+    def __init__(self, name, device, rotate=ROTATE):
+        self.name = name
+        n, k, b1, b2, frac, batch, std, outliers = WORKLOADS[name]
+        self.n, self.k, self.b1, self.b2, self.batch = n, k, b1, b2, batch
+        W, tmap = make_matrix(name)
+        self.W_host, self.tmap = W, tmap
+        Wd = W.to(device)
+        base = hyb.pack(Wd, tmap, b1, b2)
+        self.frac_real = float(tmap.mean())
+        self.mats = [base] + [base.clone() for _ in range(rotate - 1)]
+        self.dense = [Wd] + [Wd.clone() for _ in range(rotate - 1)]
+        self.X = [inputs.activations(batch, k, inputs.seed_of(name, "X", i)).to(device)
+                  for i in range(rotate)]
+        self.Y = [torch.empty(batch, n, dtype=torch.float32, device=device)
+                  for _ in range(rotate)]
+        self.ws = hyb.new_workspace(hyb.workspace_bytes(base, batch), device)
+        self.dws = hyb.new_workspace(hyb.dense_workspace_bytes(n, k, batch), device)
+        # pre-marshalled C-ABI arguments (the timed loop only calls into C)
+        L = hyb.lib()
+        self.fn = L.hyb_spmm_skinny
+        self.dfn = L.hyb_gemv_dense
+        self.structs = [m.struct() for m in self.mats]
+        self.stream = torch.cuda.current_stream(device)
+        s = ctypes.c_void_p(self.stream.cuda_stream)
+        self.args = [(ctypes.byref(self.structs[i]), batch, ctypes.c_void_p(self.X[i].data_ptr()),
+                      k, ctypes.c_void_p(self.Y[i].data_ptr()), n, hyb.HYB_F32, None,
+                      ctypes.c_void_p(self.ws.data_ptr()), self.ws.numel(), s)
+                     for i in range(rotate)]
+        self.dargs = [(n, k, batch, ctypes.c_void_p(self.dense[i].data_ptr()), k,
+                       ctypes.c_void_p(self.X[i].data_ptr()), k,
+                       ctypes.c_void_p(self.Y[i].data_ptr()), n, hyb.HYB_F32,
+                       ctypes.c_void_p(self.dws.data_ptr()), self.dws.numel(), s)
+                      for i in range(rotate)]
+        # algorithmic bytes of one product: packed values + masks, tile map, x, y
+        self.bytes_step = base.nbytes() + base.num_tiles + 2 * batch * k + 4 * batch * n
+        self.dense_bytes_step = 2 * n * k + 2 * batch * k + 4 * batch * n
+
+    def step(self, i):
+        rc = self.fn(*self.args[i % len(self.args)])
+        if rc != 0:
+            raise hyb.HybError("hyb_spmm_skinny", rc)
+
+    def dense_step(self, i):
+        rc = self.dfn(*self.dargs[i % len(self.dargs)])
+        if rc != 0:
+            raise hyb.HybError("hyb_gemv_dense", rc)
+
+
+def timed(fn, steps, warmup, stream, world=1):
+    """Device time of `steps` calls (CUDA events on the launching stream),
+    barrier + synchronize on both sides, max over ranks."""
+    for i in range(warmup):
+        fn(i)
+    torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for i in range(steps):
+        fn(warmup + i)
+    e1.record(stream)
+    e1.synchronize()
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1)
+    if world > 1:
+        t = torch.tensor([ms], dtype=torch.float64, device=torch.device("cuda", torch.cuda.current_device()))
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        ms = float(t.item())
+        torch.distributed.barrier()
+    return ms
+
+
+def e2e_timed(wl, steps, warmup, stream, world=1):
+    """Same metric through the public C ABI with host buffers: per step the
+    pinned host x is copied in, the product runs, and y is copied back."""
+    xh = [wl.X[i].cpu().pin_memory() for i in range(len(wl.X))]
+    yh = torch.empty(wl.batch, wl.n, dtype=torch.float32).pin_memory()
+
+    def one(i):
+        j = i % len(wl.X)
+        wl.X[j].copy_(xh[j], non_blocking=True)
+        wl.step(j)
+        yh.copy_(wl.Y[j], non_blocking=True)
+
+    ms = timed(one, steps, warmup, stream, world)
+    h2d = xh[0].numel() * xh[0].element_size()
+    d2h = yh.numel() * yh.element_size()
+    return ms, h2d, d2h
+
+
+# ---------------------------------------------------------------------------
+# CPU oracle timing (reported baseline)
+# ---------------------------------------------------------------------------
+
+def oracle_sample(wl_name, W_host, tmap, rows_per_step=256):
+    """A bounded sample of the workload for the CPU oracle: the fp64 hybrid
+    product of `rows_per_step` output rows (selection applied on the fly)."""
+    import oracle
+    o = oracle.Oracle()
+    n, k, b1, b2, frac, batch, std, outliers = WORKLOADS[wl_name]
+    Wb = inputs.bits(W_host)
+    X = inputs.bits(inputs.activations(batch, k, inputs.seed_of(wl_name, "X", 0)))
+    rng = np.random.default_rng(0)
+    sparse_frac = float(np.mean(tmap))
+    bytes_per_row = k * (2 * (1 - sparse_frac) + 1.125 * sparse_frac)
+
+    def step(i):
+        rows = np.sort(rng.choice(n, rows_per_step, replace=False)).astype(np.int64)
+        o.rows(Wb, b1, b2, tmap, X, rows)
+    return step, bytes_per_row * rows_per_step + 2 * batch * k + 4 * batch * rows_per_step
+
+
+def cpu_baseline(wl, budget_s=10.0):
+    step, nbytes = oracle_sample(wl.name, wl.W_host, wl.tmap)
+    step(0)
+    t0 = time.perf_counter()
+    reps = 0
+    while time.perf_counter() - t0 < budget_s:
+        step(reps)
+        reps += 1
+    dt = time.perf_counter() - t0
+    return {"value": round(nbytes * reps / dt / 1e9, 4), "unit": "GB/s", "cores": 1,
+            "kind": "oracle",
+            "sample": f"oracle_rows_f64 (fp64, single thread) on 256 random output rows of "
+                      f"{wl.name} per repetition, {reps} repetitions in {dt:.1f} s"}
+
+
+def run_reference(args, world, rank):
+    if rank != 0:
+        return 0
+    name = args.workload
+    W, tmap = make_matrix(name)
+    step, nbytes = oracle_sample(name, W, tmap)
+    for i in range(args.warmup):
+        step(i)
+    t0 = time.perf_counter()
+    for i in range(args.steps):
+        step(args.warmup + i)
+    dt = time.perf_counter() - t0
+    value = nbytes * args.steps / dt / 1e9
+    n, k, b1, b2, frac, batch, std, outliers = WORKLOADS[name]
+    line = {
+        "impl": "reference", "metric": "hybrid 2:4 GEMV achieved HBM GB/s (algorithmic bytes)",
+        "value": round(value, 4), "unit": "GB/s", "n_gpus": args.gpus, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(dt * 1e3 / args.steps, 4),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "config": workload_config(name, frac_real=float(np.mean(tmap))),
+        "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
+                         "sample": "oracle_rows_f64 (fp64, single thread) on 256 random output "
+                                   f"rows of {name} per step"},
+        "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def workload_config(name, frac_real):
+    n, k, b1, b2, frac, batch, std, outliers = WORKLOADS[name]
+    return {"workload": name, "n": n, "k": k, "tile": f"{b1}x{b2}",
+            "sparse_tile_frac": round(frac_real, 4), "batch": batch,
+            "weights": f"bf16 N(0,{std})" + (f" with {outliers:.0%} x20 outliers" if outliers else ""),
+            "l2": f"inputs larger than L2: {ROTATE} rotating packed copies",
+            "parallelism": "replicas"}
+
+
+# ---------------------------------------------------------------------------
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=50)
+    ap.add_argument("--impl", default="hyb", choices=["hyb", "reference"])
+    ap.add_argument("--workload", default="ffn_down_4096x14336_f0.5_b1", choices=list(WORKLOADS))
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    world, rank, local = dist_env()
+    if args.impl == "reference":
+        return run_reference(args, world, rank)
+
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                             device_id=device)
+    wl = Workload(args.workload, device)
+    stream = wl.stream
+
+    with ClockSampler(local) as clocks:
+        ms = timed(wl.step, args.steps, args.warmup, stream, world)
+    dense_ms = timed(wl.dense_step, args.steps, args.warmup, stream, world)
+    e2e_ms, h2d, d2h = e2e_timed(wl, args.steps, args.warmup, stream, world)
+
+    per_step_ms = ms / args.steps
+    value = world * wl.bytes_step * args.steps / (ms * 1e-3) / 1e9
+    achieved = wl.bytes_step / (per_step_ms * 1e-3) / 1e9
+    peak, peak_kind = measured_peak()
+    dense_us = dense_ms / args.steps * 1e3
+    line = {
+        "metric": "hybrid 2:4 GEMV achieved HBM GB/s (algorithmic bytes)",
+        "value": round(value, 2), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(per_step_ms, 6), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": workload_config(args.workload, wl.frac_real),
+        "us_per_matrix": round(per_step_ms * 1e3, 3),
+        "dense_us_per_matrix": round(dense_us, 3),
+        "speedup_vs_dense": round(dense_us / (per_step_ms * 1e3), 4),
+        "frac_of_nominal_8tbs": round(achieved / NOMINAL_HBM_GBS, 4),
+        "roofline": {"bound": "hbm", "achieved": round(achieved, 2), "peak": peak,
+                     "unit": "GB/s", "frac": round(achieved / peak, 4),
+                     "traffic": profiled_traffic(args.workload),
+                     "peak_kind": peak_kind, "kernel": "hybrid_stream_kernel",
+                     "bytes_per_launch": wl.bytes_step},
+        "e2e": {"value": round(world * wl.bytes_step * args.steps / (e2e_ms * 1e-3) / 1e9, 2),
+                "unit": "GB/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "gpu_launches": args.steps,
+        "clocks": clocks.summary(),
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(wl)
+    if world > 1:
+        torch.distributed.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,202 @@
+/*
+ * hyb.h -- C ABI of libhyb: tile-hybrid (dense | 2:4) weight GEMV for decode,
+ * CUDA for NVIDIA B200 (sm_100a).
+ *
+ * What is computed
+ * ----------------
+ * A weight matrix W (n outputs x k inputs, row-major, bf16) is cut into
+ * b1 x b2 tiles (b1 rows along n, b2 columns along k).  Every tile is either
+ * dense or 2:4 sparse: in a 2:4 tile every group of four consecutive
+ * elements along k keeps two.  ("PATCH: Learnable Tile-level Hybrid Sparsity
+ * for LLMs", §2 Methodology, core mechanism; §1 Problem statement for 2:4.)
+ * The kept values of a 2:4 group are stored at a fixed stride with a 4-bit
+ * mask telling which columns they came from ("SparseDecoding: decoding-aware
+ * pruning ...", authors' abstract: bitmask indexing, fixed-stride traversal).
+ * An optional low-rank term adds U (V^T x) ("3BASiL: An Algorithmic
+ * Framework for Sparse plus Low-Rank Compression of LLMs", §1: W ~ S + L).
+ *
+ *   Y[b][i] = sum_k W_hat[i][k] X[b][k]  (+ sum_j U[i][j] sum_k V[k][j] X[b][k])
+ *
+ * with W_hat the masked matrix, bf16 inputs and fp32 accumulation.
+ *
+ * Packed format (produced by hyb_pack)
+ * ------------------------------------
+ *  - Tiles are numbered row-major, t = tr * (k / b2) + tc; tile_map[t] is 1
+ *    for a 2:4 tile and 0 for a dense tile.
+ *  - val_off[t] / meta_off[t] (t = 0..num_tiles) are the element / byte
+ *    offsets of tile t in vals / meta: a dense tile takes b1*b2 values and no
+ *    meta, a 2:4 tile b1*b2/2 values and b1*b2/8 meta bytes.
+ *  - Dense tile: b1 rows of b2 values.  2:4 tile: b1 rows of b2/2 values; the
+ *    two kept values of group g of row i sit at i*(b2/2) + 2g and +1 in
+ *    ascending column order; their mask is the nibble of meta byte
+ *    i*(b2/8) + g/2 (low nibble for even g), bit j set iff column 4g+j kept.
+ *  - Selection keeps the two largest |w| of each group (key = bits & 0x7FFF;
+ *    ties go to the lower column; values are copied bit-exactly).
+ *
+ * Conventions
+ * -----------
+ *  - bf16 crosses the ABI as uint16_t bit patterns.  All data pointers are
+ *    DEVICE pointers unless the argument name ends in _host.  The caller owns
+ *    every buffer; the library never allocates or frees device memory and
+ *    keeps no global mutable state except a per-device SM-count cache.
+ *  - Every call is asynchronous on `stream` (0 = legacy default stream).
+ *    Argument, shape and alignment checks are synchronous: a failing check
+ *    returns a negative hyb_status and launches nothing.  A failed launch
+ *    returns HYB_ERR_CUDA.  Problems only the device can see (a NaN weight,
+ *    a tile_map byte other than 0/1) set a status word in the workspace, read
+ *    and cleared by hyb_check_status.  No device code traps.
+ *  - Workspaces: size them with the *_workspace_bytes queries and zero them
+ *    once (hyb_workspace_init) before first use.  The library leaves them
+ *    ready for the next call.  Two calls that run concurrently must not share
+ *    a workspace.
+ *  - X is [batch][k] bf16 with leading dimension ldx >= k; Y is [batch][n]
+ *    (fp32 or bf16) with ldy >= n.  X, Y and meta must be 16-byte aligned,
+ *    vals 32-byte aligned, workspaces 256-byte aligned; ldx and ldy must keep
+ *    rows 16-byte aligned.
+ *  - Shapes: n % b1 == 0, k % b2 == 0, b2 % 16 == 0, (b1 * b2) % 128 == 0.
+ *    Any batch 1..16.  Tiles of 64 or 128 rows by 64 or 128 columns run the
+ *    tuned streaming kernel; other legal tilings run a simpler CUDA kernel
+ *    (never a CPU fallback).
+ */
+#ifndef HYB_H
+#define HYB_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define HYB_API __attribute__((visibility("default")))
+#else
+#define HYB_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st *hyb_stream_t; /* same type as cudaStream_t */
+
+typedef enum {
+  HYB_OK = 0,
+  HYB_ERR_INVALID_ARG = -1,  /* bad shape, null pointer, bad enum */
+  HYB_ERR_UNSUPPORTED = -2,  /* valid request this build does not handle */
+  HYB_ERR_ALIGNMENT = -3,    /* pointer or leading dimension misaligned */
+  HYB_ERR_WORKSPACE = -4,    /* workspace null or smaller than required */
+  HYB_ERR_CUDA = -5,         /* a CUDA runtime call failed */
+  HYB_ERR_DEVICE_CHECK = -6  /* the device flagged bad data (see above) */
+} hyb_status;
+
+typedef enum { HYB_F32 = 0, HYB_BF16 = 1 } hyb_dtype;
+
+/* A packed hybrid matrix; every pointer is a device pointer. */
+typedef struct {
+  int64_t n, k;          /* outputs, inputs */
+  int32_t b1, b2;        /* tile rows (along n), tile columns (along k) */
+  int64_t num_tiles;     /* (n / b1) * (k / b2) */
+  const uint8_t *tile_map;  /* [num_tiles], 1 = 2:4 tile, 0 = dense tile */
+  const uint16_t *vals;     /* packed values, bf16 bits */
+  const uint8_t *meta;      /* packed 4-bit masks (never NULL: pass any valid
+                               device byte when the map has no 2:4 tile) */
+  const int64_t *val_off;   /* [num_tiles + 1] */
+  const int64_t *meta_off;  /* [num_tiles + 1] */
+  int64_t n_vals;           /* val_off[num_tiles], as given by hyb_packed_sizes */
+  int64_t n_meta_bytes;     /* meta_off[num_tiles], as given by hyb_packed_sizes */
+} hyb_matrix;
+
+/* Low-rank factors of y += U (V^T x): U is [n][rank] (row stride ldu),
+ * V is [k][rank] (row stride ldv), bf16, device pointers.  rank 1..256. */
+typedef struct {
+  int32_t rank;
+  const uint16_t *U;
+  int64_t ldu;
+  const uint16_t *V;
+  int64_t ldv;
+} hyb_lowrank;
+
+/* ---- format ----------------------------------------------------------- */
+
+/* Host-only: number of packed values and meta bytes for a tile map held in
+ * HOST memory (PATCH §2: dense tiles keep b1*b2 values, 2:4 tiles half of
+ * them plus one 4-bit mask per group).  Rejects map bytes other than 0/1. */
+HYB_API int hyb_packed_sizes(int64_t n, int64_t k, int b1, int b2,
+                     const uint8_t *tile_map_host, int64_t *n_vals,
+                     int64_t *n_meta_bytes);
+
+/* Workspace bytes hyb_pack needs (status word only). */
+HYB_API size_t hyb_pack_workspace_bytes(void);
+
+/* Pack W ([n][k] bf16, row stride ldw, device) with the device tile_map into
+ * vals / meta / val_off / meta_off (device buffers of the sizes given by
+ * hyb_packed_sizes; offsets num_tiles + 1 entries each; meta never NULL, a
+ * 1-byte buffer will do when the map has no 2:4 tile).  The selection rule
+ * is the magnitude projection of 3BASiL §2A applied per 2:4 group (two
+ * largest |w|, ties to the lower column).  A group holding a NaN, or a map
+ * byte other than 0/1, sets the workspace status word; the pack still
+ * completes deterministically.  W must be 16-byte aligned with ldw % 8 == 0. */
+HYB_API int hyb_pack(int64_t n, int64_t k, int b1, int b2, const uint16_t *W,
+             int64_t ldw, const uint8_t *tile_map, uint16_t *vals,
+             uint8_t *meta, int64_t *val_off, int64_t *meta_off, void *ws,
+             size_t ws_bytes, hyb_stream_t stream);
+
+/* ---- products ---------------------------------------------------------- */
+
+/* Workspace bytes for hyb_spmv / hyb_spmm_skinny on matrix A with this
+ * batch and low-rank rank (0 = none); 0 if the arguments are invalid.  The
+ * answer depends on the current device (its SM count). */
+HYB_API size_t hyb_workspace_bytes(const hyb_matrix *A, int batch, int rank);
+
+/* Zero a workspace before its first use (asynchronous memset on stream). */
+HYB_API int hyb_workspace_init(void *ws, size_t ws_bytes, hyb_stream_t stream);
+
+/* Y = W_hat x (+ U (V^T x)) for one input vector (batch 1).  The decode-time
+ * sparse matrix-vector product of SparseDecoding (authors' abstract) applied
+ * to PATCH's hybrid tiles, with the sparse-plus-low-rank form of 3BASiL §1.
+ * ydt selects fp32 or bf16 (round-to-nearest-even from fp32) output; lr may
+ * be NULL. */
+HYB_API int hyb_spmv(const hyb_matrix *A, const uint16_t *X, int64_t ldx, void *Y,
+             int64_t ldy, hyb_dtype ydt, const hyb_lowrank *lr, void *ws,
+             size_t ws_bytes, hyb_stream_t stream);
+
+/* Same for a skinny batch of 1..16 input vectors, X [batch][k]. */
+HYB_API int hyb_spmm_skinny(const hyb_matrix *A, int batch, const uint16_t *X,
+                    int64_t ldx, void *Y, int64_t ldy, hyb_dtype ydt,
+                    const hyb_lowrank *lr, void *ws, size_t ws_bytes,
+                    hyb_stream_t stream);
+
+/* Workspace bytes for hyb_lowrank_add. */
+HYB_API size_t hyb_lowrank_workspace_bytes(int64_t k, int batch, int rank);
+
+/* Y[b][i] += sum_j U[i][j] sum_k V[k][j] X[b][k]  (fp32 Y, in place): the
+ * low-rank term of 3BASiL §1 on its own. */
+HYB_API int hyb_lowrank_add(int64_t n, int64_t k, int batch, const hyb_lowrank *lr,
+                    const uint16_t *X, int64_t ldx, float *Y, int64_t ldy,
+                    void *ws, size_t ws_bytes, hyb_stream_t stream);
+
+/* Workspace bytes for hyb_gemv_dense. */
+HYB_API size_t hyb_dense_workspace_bytes(int64_t n, int64_t k, int batch);
+
+/* Plain dense Y = W X for W [n][k] bf16 row-major (row stride ldw), the
+ * dense baseline the pages compare the hybrid format against (PATCH §4,
+ * SparseDecoding abstract).  Same streaming design as hyb_spmv. Needs
+ * n % 8 == 0, k % 16 == 0, ldw % 16 == 0, W 32-byte aligned. */
+HYB_API int hyb_gemv_dense(int64_t n, int64_t k, int batch, const uint16_t *W,
+                   int64_t ldw, const uint16_t *X, int64_t ldx, void *Y,
+                   int64_t ldy, hyb_dtype ydt, void *ws, size_t ws_bytes,
+                   hyb_stream_t stream);
+
+/* ---- status ------------------------------------------------------------ */
+
+/* Synchronise `stream`, read and clear the workspace status word.  Returns
+ * HYB_OK, HYB_ERR_DEVICE_CHECK (a device check fired) or HYB_ERR_CUDA. If
+ * flags is not NULL it receives the raw status bits (1 = NaN weight seen by
+ * hyb_pack, 2 = tile_map byte other than 0/1). */
+HYB_API int hyb_check_status(void *ws, hyb_stream_t stream, uint32_t *flags);
+
+/* Static description of a status code. */
+HYB_API const char *hyb_status_string(int status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* HYB_H */

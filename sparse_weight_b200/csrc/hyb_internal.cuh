@@ -1,0 +1,74 @@
+// hyb_internal.cuh -- device helpers shared by the libhyb CUDA sources.
+//
+// Nothing here is part of the C ABI (include/hyb.h is).  Target: sm_100a.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "hyb.h"
+
+namespace hyb {
+
+// Status bits kept in the first word of every workspace.
+constexpr uint32_t kStatusNaN = 1u;      // hyb_pack saw a NaN weight
+constexpr uint32_t kStatusBadMap = 2u;   // tile_map byte other than 0 / 1
+
+// Workspace header: status word, padded so that what follows is aligned.
+constexpr size_t kHeaderBytes = 256;
+
+__host__ __device__ inline size_t align_up(size_t v, size_t a) {
+  return (v + a - 1) / a * a;
+}
+
+// ---- bf16 <-> fp32 --------------------------------------------------------
+// A bf16 value is the upper half of a binary32: widening is a shift.
+__device__ __forceinline__ float bf16_lo(uint32_t pair) {
+  return __uint_as_float(pair << 16);
+}
+__device__ __forceinline__ float bf16_hi(uint32_t pair) {
+  return __uint_as_float(pair & 0xFFFF0000u);
+}
+// fp32 -> bf16, round-to-nearest-even (CUDA's conversion intrinsic).
+__device__ __forceinline__ uint16_t f32_to_bf16_rne(float f) {
+  return __bfloat16_as_ushort(__float2bfloat16_rn(f));
+}
+
+// ---- streaming loads -------------------------------------------------------
+// Weights are read exactly once per call: read-only path, no L1 allocation;
+// the 32-byte form also carries an L2 evict-first hint so streamed weights do
+// not push the reused operands (X, the low-rank factors, partial sums) out.
+__device__ __forceinline__ uint4 ld_stream16(const void *p) {
+  uint4 r;
+  asm volatile(
+      "ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
+      : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
+      : "l"(p));
+  return r;
+}
+// 32-byte load (sm_100 256-bit global load).
+__device__ __forceinline__ void ld_stream32(const void *p, uint4 &a, uint4 &b) {
+  asm volatile(
+      "ld.global.nc.L1::no_allocate.L2::evict_first.v8.b32 "
+      "{%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+      : "=r"(a.x), "=r"(a.y), "=r"(a.z), "=r"(a.w), "=r"(b.x), "=r"(b.y),
+        "=r"(b.z), "=r"(b.w)
+      : "l"(p));
+}
+__device__ __forceinline__ uint16_t ld_stream_u16(const void *p) {
+  uint16_t r;
+  asm volatile("ld.global.nc.L1::no_allocate.u16 %0, [%1];"
+               : "=h"(r)
+               : "l"(p));
+  return r;
+}
+// Reused operand (X): read-only path, cached in L1.
+__device__ __forceinline__ uint4 ld_keep16(const void *p) {
+  return __ldg(reinterpret_cast<const uint4 *>(p));
+}
+
+// ---- host helpers -----------------------------------------------------------
+int device_sm_count(int *out);  // cached per device
+
+}  // namespace hyb

@@ -1,0 +1,1045 @@
+// hyb_spmv.cu -- Y = W_hat X (+ U (V^T X)) for the tile-hybrid format, plus
+// the dense GEMV baseline and the stand-alone low-rank term.
+//
+// Decode-time products are memory-bound ("SparseDecoding: decoding-aware
+// pruning ...", authors' abstract: the decode phase is limited by memory
+// access and is dominated by sparse matrix-vector products), so the design
+// is a single streaming pass over the packed bytes with no tensor cores:
+//
+//  * Work split: the packed stream is row-major over tiles, so every tile-row
+//    band is contiguous.  CTA c of G takes the tiles whose byte offset falls
+//    in [c, c+1) * total / G -- a split by bytes, not by tiles, because a
+//    dense tile costs 2 B/weight and a 2:4 tile 1.125 B/weight ("PATCH:
+//    Learnable Tile-level Hybrid Sparsity for LLMs", §2: tiles are dense or
+//    2:4).  Each CTA finds its range with two rounds of parallel search over
+//    the tile offsets.
+//  * Inside a tile, warp w owns rows [w*R, (w+1)*R); a lane owns 16 columns of
+//    one row per step: 16 bytes of kept values plus 2 bytes of masks in a 2:4
+//    tile (4 groups), or 32 bytes in a dense tile.  Lanes keep the 16 x values
+//    they need in registers and accumulate in fp32 registers across all the
+//    tiles of a band; the next tile is loaded while the current one computes.
+//  * The mask nibble picks which two of the group's four x values multiply
+//    the two kept values (SparseDecoding: bitmask-indexed, fixed-stride N:M).
+//  * Band results cross CTAs through fp32 partial slots; the last CTA to
+//    arrive at a band (atomic ticket, no spinning) sums the slots in CTA order
+//    -- deterministic -- and applies the epilogue: the low-rank term
+//    ("3BASiL", §1: W ~ S + L) and the fp32 or bf16 store.
+#include <algorithm>
+#include <mutex>
+
+#include "hyb_internal.cuh"
+
+namespace hyb {
+
+int check_tiling(int64_t n, int64_t k, int b1, int b2);  // hyb_pack.cu
+
+namespace {
+
+constexpr int kWarps = 8;
+constexpr int kThreads = kWarps * 32;
+constexpr int kMaxRank = 256;
+
+struct Params {
+  // matrix (packed) or dense W (strided mode)
+  const uint8_t *map;
+  const uint8_t *vals;  // bytes
+  const uint8_t *meta;
+  const int64_t *val_off;
+  const int64_t *meta_off;
+  const uint16_t *Wd;
+  int64_t ldw;
+  int64_t n, k, tpr, T;
+  int R;  // tile-row bands
+  // operands
+  const uint16_t *X;
+  int64_t ldx;
+  int batch;
+  void *Y;
+  int64_t ldy;
+  int ydt;
+  // low rank (t = V^T x already computed into lr_t[batch][rank])
+  const uint16_t *U;
+  int64_t ldu;
+  int rank;
+  const float *lr_t;
+  // split
+  int G;
+  int64_t total;  // packed bytes of the whole matrix
+  float *partials;
+  uint32_t *counters;
+};
+
+// ---------------------------------------------------------------------------
+// helpers
+// ---------------------------------------------------------------------------
+
+template <int BP>
+struct XRegs {
+  uint4 v[BP][2];  // 16 bf16 per batch column
+};
+
+// Select x[p0] and x[p1] of one group from its 4-bit mask (two bits set):
+// p0 is the lowest set bit, p1 the highest.
+__device__ __forceinline__ void pick2(uint32_t nib, float x0, float x1,
+                                      float x2, float x3, float &xa,
+                                      float &xb) {
+  xa = (nib & 1u) ? x0 : ((nib & 2u) ? x1 : x2);
+  xb = (nib & 8u) ? x3 : ((nib & 4u) ? x2 : x1);
+}
+
+__device__ __forceinline__ void unpack16(const uint4 &a, const uint4 &b,
+                                         float f[16]) {
+  const uint32_t w[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    f[2 * i] = bf16_lo(w[i]);
+    f[2 * i + 1] = bf16_hi(w[i]);
+  }
+}
+
+__device__ __forceinline__ int64_t cost_prefix(const Params &p, int64_t t,
+                                               bool strided,
+                                               int64_t tile_cost_dense) {
+  if (strided) return t * tile_cost_dense;
+  return 2 * __ldg(p.val_off + t) + __ldg(p.meta_off + t);
+}
+
+__device__ __forceinline__ int owner_of(int64_t P, const Params &p) {
+  int64_t o = (P * p.G) / p.total;
+  return (int)(o < p.G - 1 ? o : p.G - 1);
+}
+
+// Epilogue for one (row, batch) output: add the low-rank term, store.
+__device__ __forceinline__ void store_out(const Params &p, int64_t row, int b,
+                                          float y) {
+  if (p.rank > 0) {
+    const uint16_t *u = p.U + row * p.ldu;
+    const float *t = p.lr_t + (int64_t)b * p.rank;
+    float s = 0.f;
+    for (int j = 0; j < p.rank; j += 8) {
+      const uint4 uv = __ldg(reinterpret_cast<const uint4 *>(u + j));
+      s = fmaf(bf16_lo(uv.x), t[j + 0], s);
+      s = fmaf(bf16_hi(uv.x), t[j + 1], s);
+      s = fmaf(bf16_lo(uv.y), t[j + 2], s);
+      s = fmaf(bf16_hi(uv.y), t[j + 3], s);
+      s = fmaf(bf16_lo(uv.z), t[j + 4], s);
+      s = fmaf(bf16_hi(uv.z), t[j + 5], s);
+      s = fmaf(bf16_lo(uv.w), t[j + 6], s);
+      s = fmaf(bf16_hi(uv.w), t[j + 7], s);
+    }
+    y += s;
+  }
+  if (p.ydt == HYB_BF16)
+    reinterpret_cast<uint16_t *>(p.Y)[(int64_t)b * p.ldy + row] =
+        f32_to_bf16_rne(y);
+  else
+    reinterpret_cast<float *>(p.Y)[(int64_t)b * p.ldy + row] = y;
+}
+
+// ---------------------------------------------------------------------------
+// the streaming kernel
+// ---------------------------------------------------------------------------
+
+template <int BP, int B1, int B2, bool STRIDED>
+struct Cfg {
+  static constexpr int RW = B1 / kWarps;    // rows per warp per tile
+  static constexpr int CPR = B2 / 16;       // lanes per row (16 columns each)
+  static constexpr int RPS = 32 / CPR;      // rows per warp step
+  static constexpr int JS = RW / RPS;       // steps per warp per tile
+  static constexpr int XB = BP < 4 ? BP : 4;  // batch columns per x sub-block
+  static constexpr int64_t kDenseCost = 2LL * B1 * B2;
+  static constexpr int kMinBlocks = BP <= 1 ? 2 : 1;
+  static_assert(RW * kWarps == B1, "b1 must split over the warps");
+  static_assert(RPS * CPR == 32 && JS * RPS == RW, "tile shape");
+};
+
+// Registers of one tile in flight: per step 16 B (2:4) + 2 B masks, or 32 B.
+template <int JS>
+struct TileRegs {
+  uint4 a[JS];
+  uint4 b[JS];  // dense: second 16 B; 2:4: b[j].x holds the 16 mask bits
+};
+
+template <int BP, int B1, int B2, bool STRIDED>
+__global__ void __launch_bounds__(kThreads, (Cfg<BP, B1, B2, STRIDED>::kMinBlocks))
+    hybrid_stream_kernel(const Params p) {
+  using C = Cfg<BP, B1, B2, STRIDED>;
+  constexpr int JS = C::JS;
+  extern __shared__ int s_owner[];  // [2 * R]: owner CTA of each band's first / last tile
+  __shared__ float s_acc[B1 * BP];
+  __shared__ int64_t s_range[2];
+  __shared__ int s_last;
+
+  const int tid = threadIdx.x;
+  const int warp = tid >> 5, lane = tid & 31;
+  const int cp = lane % C::CPR;  // 16-column part
+  const int rs = lane / C::CPR;  // row inside a step
+  const int c = blockIdx.x;
+  const int G = p.G;
+
+  // ---- 1. this CTA's tile range [t0, t1) -----------------------------------
+  const int64_t tgtA = (int64_t)c * p.total;
+  const int64_t tgtB = (int64_t)(c + 1) * p.total;
+  int64_t t0, t1;
+  if (STRIDED) {
+    // uniform tiles: closed form
+    const int64_t unit = C::kDenseCost * G;
+    t0 = (tgtA + unit - 1) / unit;
+    t1 = (c == G - 1) ? p.T : (tgtB + unit - 1) / unit;
+    for (int i = tid; i < p.R; i += kThreads) {
+      s_owner[2 * i] = owner_of((int64_t)i * p.tpr * C::kDenseCost, p);
+      s_owner[2 * i + 1] =
+          owner_of(((int64_t)(i + 1) * p.tpr - 1) * C::kDenseCost, p);
+    }
+  } else {
+    // round 1: band starts (and owners of every band's first / last tile)
+    int cntA = 0, cntB = 0;
+    for (int base = 0; base <= p.R; base += kThreads) {
+      const int i = base + tid;
+      bool pa = false, pb = false;
+      if (i <= p.R) {
+        const int64_t P0 = cost_prefix(p, (int64_t)i * p.tpr, false, 0);
+        pa = P0 * G < tgtA;
+        pb = P0 * G < tgtB;
+        if (i < p.R) {
+          const int64_t Pl = cost_prefix(p, (int64_t)(i + 1) * p.tpr - 1, false, 0);
+          s_owner[2 * i] = owner_of(P0, p);
+          s_owner[2 * i + 1] = owner_of(Pl, p);
+        }
+      }
+      cntA += __syncthreads_count(pa);
+      cntB += __syncthreads_count(pb);
+    }
+    // round 2: tiles inside the bracketing band
+    const int64_t baseA = cntA > 0 ? (int64_t)(cntA - 1) * p.tpr : 0;
+    const int64_t baseB = cntB > 0 ? (int64_t)(cntB - 1) * p.tpr : 0;
+    int64_t cA = 0, cB = 0;
+    for (int64_t off = 0; off < p.tpr; off += kThreads) {
+      const int64_t o = off + tid;
+      bool pa = false, pb = false;
+      if (o < p.tpr) {
+        if (cntA > 0) pa = cost_prefix(p, baseA + o, false, 0) * G < tgtA;
+        if (cntB > 0) pb = cost_prefix(p, baseB + o, false, 0) * G < tgtB;
+      }
+      cA += __syncthreads_count(pa);
+      cB += __syncthreads_count(pb);
+    }
+    t0 = cntA > 0 ? baseA + cA : 0;
+    t1 = (c == G - 1) ? p.T : (cntB > 0 ? baseB + cB : 0);
+  }
+  if (tid == 0) {
+    s_range[0] = t0;
+    s_range[1] = t1;
+  }
+  __syncthreads();
+  t0 = s_range[0];
+  t1 = s_range[1];
+
+  // ---- 2. stream the tiles --------------------------------------------------
+  float acc[JS][BP];
+#pragma unroll
+  for (int j = 0; j < JS; ++j)
+#pragma unroll
+    for (int b = 0; b < BP; ++b) acc[j][b] = 0.f;
+
+  const int wrow = warp * C::RW;  // first row of this warp inside a tile
+
+  // tile "header": sparse flag and byte offsets (prefetched one tile ahead)
+  struct Head {
+    int64_t vb, mb;
+    bool sparse;
+  };
+  auto head_of = [&](int64_t t) -> Head {
+    Head h;
+    if (STRIDED) {
+      h.vb = 0;
+      h.mb = 0;
+      h.sparse = false;
+    } else {
+      h.sparse = __ldg(p.map + t) == 1;
+      h.vb = 2 * __ldg(p.val_off + t);
+      h.mb = __ldg(p.meta_off + t);
+    }
+    return h;
+  };
+  auto load_tile = [&](int64_t t, const Head &h, TileRegs<JS> &r) {
+    const int64_t tr = t / p.tpr, tc = t - tr * p.tpr;
+    if (STRIDED) {
+      const uint16_t *base =
+          p.Wd + (tr * B1 + wrow + rs) * p.ldw + tc * B2 + 16 * cp;
+#pragma unroll
+      for (int j = 0; j < JS; ++j)
+        ld_stream32(base + (int64_t)j * C::RPS * p.ldw, r.a[j], r.b[j]);
+    } else if (h.sparse) {
+      const uint8_t *vbase = p.vals + h.vb + (int64_t)(wrow + rs) * B2 + 16 * cp;
+      const uint8_t *mbase = p.meta + h.mb + (int64_t)(wrow + rs) * (B2 / 8) + 2 * cp;
+#pragma unroll
+      for (int j = 0; j < JS; ++j) {
+        r.a[j] = ld_stream16(vbase + (int64_t)j * C::RPS * B2);
+        r.b[j].x = ld_stream_u16(mbase + (int64_t)j * C::RPS * (B2 / 8));
+      }
+    } else {
+      const uint8_t *vbase =
+          p.vals + h.vb + (int64_t)(wrow + rs) * 2 * B2 + 32 * cp;
+#pragma unroll
+      for (int j = 0; j < JS; ++j)
+        ld_stream32(vbase + (int64_t)j * C::RPS * 2 * B2, r.a[j], r.b[j]);
+    }
+  };
+  auto load_x = [&](int64_t t, int b0, XRegs<C::XB> &xr) {
+    const int64_t tc = t % p.tpr;
+    const uint16_t *xp = p.X + tc * B2 + 16 * cp;
+#pragma unroll
+    for (int b = 0; b < C::XB; ++b) {
+      if (b0 + b < p.batch) {
+        xr.v[b][0] = ld_keep16(xp + (int64_t)(b0 + b) * p.ldx);
+        xr.v[b][1] = ld_keep16(xp + (int64_t)(b0 + b) * p.ldx + 8);
+      } else {
+        xr.v[b][0] = make_uint4(0, 0, 0, 0);
+        xr.v[b][1] = make_uint4(0, 0, 0, 0);
+      }
+    }
+  };
+
+  // flush the accumulators of band r: lanes -> shared -> slot or epilogue
+  auto flush = [&](int r) {
+#pragma unroll
+    for (int j = 0; j < JS; ++j)
+#pragma unroll
+      for (int b = 0; b < BP; ++b) {
+        float v = acc[j][b];
+#pragma unroll
+        for (int o = 1; o < C::CPR; o <<= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+        acc[j][b] = v;
+      }
+    if (cp == 0) {
+#pragma unroll
+      for (int j = 0; j < JS; ++j)
+#pragma unroll
+        for (int b = 0; b < BP; ++b)
+          s_acc[(wrow + j * C::RPS + rs) * BP + b] = acc[j][b];
+    }
+#pragma unroll
+    for (int j = 0; j < JS; ++j)
+#pragma unroll
+      for (int b = 0; b < BP; ++b) acc[j][b] = 0.f;
+    __syncthreads();
+    const int oA = s_owner[2 * r], oB = s_owner[2 * r + 1];
+    const int64_t row0 = (int64_t)r * B1;
+    if (oA == oB) {
+      // this CTA owns the whole band
+      for (int i = tid; i < B1 * BP; i += kThreads) {
+        const int row = i % B1, b = i / B1;
+        if (b < p.batch) store_out(p, row0 + row, b, s_acc[row * BP + b]);
+      }
+    } else {
+      float *slot = p.partials + (int64_t)(c + r) * (B1 * BP);
+      for (int i = tid; i < B1 * BP; i += kThreads) __stcg(slot + i, s_acc[i]);
+      __threadfence();
+      __syncthreads();
+      if (tid == 0) {
+        const uint32_t prev = atomicAdd(p.counters + r, 1u);
+        s_last = prev == (uint32_t)(oB - oA);
+      }
+      __syncthreads();
+      if (s_last) {
+        __threadfence();
+        for (int i = tid; i < B1 * BP; i += kThreads) {
+          const int row = i % B1, b = i / B1;
+          if (b >= p.batch) continue;
+          float y = 0.f;
+          for (int cc = oA; cc <= oB; ++cc)
+            y += __ldcg(p.partials + (int64_t)(cc + r) * (B1 * BP) + row * BP + b);
+          store_out(p, row0 + row, b, y);
+        }
+        if (tid == 0) p.counters[r] = 0;  // ready for the next call
+      }
+    }
+    __syncthreads();
+  };
+
+  if (t0 < t1) {
+    Head hcur = head_of(t0);
+    Head hnext = hcur;
+    if (t0 + 1 < t1) hnext = head_of(t0 + 1);
+    TileRegs<JS> cur;
+    load_tile(t0, hcur, cur);
+    XRegs<C::XB> xcur;
+    if (BP <= 4) load_x(t0, 0, xcur);
+    for (int64_t t = t0; t < t1; ++t) {
+      Head hnn = hnext;
+      if (t + 2 < t1) hnn = head_of(t + 2);
+      TileRegs<JS> nxt;
+      XRegs<C::XB> xnxt;
+      if (t + 1 < t1) {
+        load_tile(t + 1, hnext, nxt);
+        if (BP <= 4) load_x(t + 1, 0, xnxt);
+      }
+      // ---- compute tile t ----
+#pragma unroll
+      for (int b0 = 0; b0 < BP; b0 += C::XB) {
+        XRegs<C::XB> xs;
+        if (BP <= 4) {
+          xs = xcur;
+        } else {
+          load_x(t, b0, xs);
+        }
+        float xf[C::XB][16];
+#pragma unroll
+        for (int b = 0; b < C::XB; ++b) unpack16(xs.v[b][0], xs.v[b][1], xf[b]);
+        if (hcur.sparse) {
+#pragma unroll
+          for (int j = 0; j < JS; ++j) {
+            const uint32_t w[4] = {cur.a[j].x, cur.a[j].y, cur.a[j].z, cur.a[j].w};
+            const uint32_t m = cur.b[j].x;
+#pragma unroll
+            for (int g = 0; g < 4; ++g) {
+              const uint32_t nib = (m >> (4 * g)) & 0xFu;
+              const float v0 = bf16_lo(w[g]), v1 = bf16_hi(w[g]);
+#pragma unroll
+              for (int b = 0; b < C::XB; ++b) {
+                float xa, xb;
+                pick2(nib, xf[b][4 * g], xf[b][4 * g + 1], xf[b][4 * g + 2],
+                      xf[b][4 * g + 3], xa, xb);
+                acc[j][b0 + b] = fmaf(v0, xa, acc[j][b0 + b]);
+                acc[j][b0 + b] = fmaf(v1, xb, acc[j][b0 + b]);
+              }
+            }
+          }
+        } else {
+#pragma unroll
+          for (int j = 0; j < JS; ++j) {
+            float wf[16];
+            unpack16(cur.a[j], cur.b[j], wf);
+#pragma unroll
+            for (int e = 0; e < 16; ++e)
+#pragma unroll
+              for (int b = 0; b < C::XB; ++b)
+                acc[j][b0 + b] = fmaf(wf[e], xf[b][e], acc[j][b0 + b]);
+          }
+        }
+      }
+      // band boundary or end of range: flush
+      if (t + 1 == t1 || (t + 1) % p.tpr == 0) flush((int)(t / p.tpr));
+      cur = nxt;
+      xcur = xnxt;
+      hcur = hnext;
+      hnext = hnn;
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
+// simple kernel for other legal tilings: one warp per output row
+// ---------------------------------------------------------------------------
+template <int BP, bool STRIDED>
+__global__ void __launch_bounds__(kThreads)
+    hybrid_rowwarp_kernel(const Params p, int b1, int b2) {
+  const int lane = threadIdx.x & 31;
+  const int64_t warps = (int64_t)gridDim.x * kWarps;
+  const int cpr = b2 / 16;  // 16-column chunks per tile row
+  for (int64_t row = (int64_t)blockIdx.x * kWarps + (threadIdx.x >> 5); row < p.n;
+       row += warps) {
+    const int64_t r = row / b1, i = row - r * b1;
+    float acc[BP];
+#pragma unroll
+    for (int b = 0; b < BP; ++b) acc[b] = 0.f;
+    for (int64_t q = lane; q < p.tpr * cpr; q += 32) {
+      const int64_t tc = q / cpr;
+      const int cpart = (int)(q - tc * cpr);
+      const int64_t t = r * p.tpr + tc;
+      float xf[BP][16];
+#pragma unroll
+      for (int b = 0; b < BP; ++b) {
+        if (b < p.batch) {
+          const uint16_t *xp = p.X + (int64_t)b * p.ldx + tc * b2 + 16 * cpart;
+          unpack16(ld_keep16(xp), ld_keep16(xp + 8), xf[b]);
+        } else {
+#pragma unroll
+          for (int e = 0; e < 16; ++e) xf[b][e] = 0.f;
+        }
+      }
+      const bool sparse = !STRIDED && __ldg(p.map + t) == 1;
+      if (sparse) {
+        const uint8_t *vp =
+            p.vals + 2 * __ldg(p.val_off + t) + i * b2 + 16 * cpart;
+        const uint8_t *mp = p.meta + __ldg(p.meta_off + t) + i * (b2 / 8) + 2 * cpart;
+        const uint4 v = ld_stream16(vp);
+        const uint32_t m = ld_stream_u16(mp);
+        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int g = 0; g < 4; ++g) {
+          const uint32_t nib = (m >> (4 * g)) & 0xFu;
+#pragma unroll
+          for (int b = 0; b < BP; ++b) {
+            float xa, xb;
+            pick2(nib, xf[b][4 * g], xf[b][4 * g + 1], xf[b][4 * g + 2],
+                  xf[b][4 * g + 3], xa, xb);
+            acc[b] = fmaf(bf16_lo(w[g]), xa, acc[b]);
+            acc[b] = fmaf(bf16_hi(w[g]), xb, acc[b]);
+          }
+        }
+      } else {
+        const uint8_t *vp =
+            STRIDED ? reinterpret_cast<const uint8_t *>(p.Wd + row * p.ldw + tc * b2 + 16 * cpart)
+                    : p.vals + 2 * __ldg(p.val_off + t) + i * 2 * b2 + 32 * cpart;
+        float wf[16];
+        unpack16(ld_stream16(vp), ld_stream16(vp + 16), wf);
+#pragma unroll
+        for (int e = 0; e < 16; ++e)
+#pragma unroll
+          for (int b = 0; b < BP; ++b) acc[b] = fmaf(wf[e], xf[b][e], acc[b]);
+      }
+    }
+#pragma unroll
+    for (int b = 0; b < BP; ++b)
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) acc[b] += __shfl_xor_sync(0xffffffffu, acc[b], o);
+    if (lane == 0)
+      for (int b = 0; b < p.batch; ++b) store_out(p, row, b, acc[b]);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// low rank: t[b][j] = sum_k V[k][j] x[b][k]  (3BASiL §1: the L = U V^T term)
+// ---------------------------------------------------------------------------
+// CTA c sums k in its slice; partials go to lr_part[c][b][j]; the last CTA to
+// arrive sums them in CTA order into t (deterministic).
+template <int BP>
+__global__ void __launch_bounds__(kThreads)
+    lowrank_t_kernel(const uint16_t *__restrict__ V, int64_t ldv, int rank,
+                     int64_t k, const uint16_t *__restrict__ X, int64_t ldx,
+                     int batch, float *__restrict__ t_out,
+                     float *__restrict__ lr_part, uint32_t *counter) {
+  __shared__ float s_sum[BP * kMaxRank];
+  __shared__ int s_last;
+  const int tid = threadIdx.x;
+  const int jg_count = rank / 8;          // 8 columns of V per thread
+  const int rows_par = kThreads / jg_count;  // k rows in parallel
+  const int jg = tid % jg_count, rg = tid / jg_count;
+  const int G2 = gridDim.x, c = blockIdx.x;
+  const int64_t k0 = k * c / G2, k1 = k * (c + 1) / G2;
+  float acc[BP][8];
+#pragma unroll
+  for (int b = 0; b < BP; ++b)
+#pragma unroll
+    for (int e = 0; e < 8; ++e) acc[b][e] = 0.f;
+  if (rg < rows_par) {
+    for (int64_t kk = k0 + rg; kk < k1; kk += rows_par) {
+      const uint4 v = ld_stream16(V + kk * ldv + 8 * jg);
+      const float vf[8] = {bf16_lo(v.x), bf16_hi(v.x), bf16_lo(v.y), bf16_hi(v.y),
+                           bf16_lo(v.z), bf16_hi(v.z), bf16_lo(v.w), bf16_hi(v.w)};
+#pragma unroll
+      for (int b = 0; b < BP; ++b) {
+        if (b >= batch) break;
+        const float xv = __uint_as_float((uint32_t)__ldg(X + b * ldx + kk) << 16);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) acc[b][e] = fmaf(vf[e], xv, acc[b][e]);
+      }
+    }
+  }
+  // fixed-order reduction over the row groups of this CTA
+  for (int i = tid; i < BP * rank; i += kThreads) s_sum[i] = 0.f;
+  __syncthreads();
+  for (int g = 0; g < rows_par; ++g) {
+    if (rg == g) {
+#pragma unroll
+      for (int b = 0; b < BP; ++b)
+#pragma unroll
+        for (int e = 0; e < 8; ++e) s_sum[b * rank + 8 * jg + e] += acc[b][e];
+    }
+    __syncthreads();
+  }
+  float *mine = lr_part + (int64_t)c * BP * rank;
+  for (int i = tid; i < BP * rank; i += kThreads) __stcg(mine + i, s_sum[i]);
+  __threadfence();
+  __syncthreads();
+  if (tid == 0) s_last = atomicAdd(counter, 1u) == (uint32_t)(G2 - 1);
+  __syncthreads();
+  if (s_last) {
+    __threadfence();
+    for (int i = tid; i < BP * rank; i += kThreads) {
+      float s = 0.f;
+      for (int cc = 0; cc < G2; ++cc) s += __ldcg(lr_part + (int64_t)cc * BP * rank + i);
+      t_out[i] = s;
+    }
+    if (tid == 0) *counter = 0;
+  }
+}
+
+// Y[b][i] += sum_j U[i][j] t[b][j]  (fp32 Y), one thread per row.
+template <int BP>
+__global__ void __launch_bounds__(kThreads)
+    lowrank_apply_kernel(int64_t n, const uint16_t *__restrict__ U, int64_t ldu,
+                         int rank, const float *__restrict__ t, int batch,
+                         float *__restrict__ Y, int64_t ldy) {
+  const int64_t i = (int64_t)blockIdx.x * kThreads + threadIdx.x;
+  if (i >= n) return;
+  float acc[BP];
+#pragma unroll
+  for (int b = 0; b < BP; ++b) acc[b] = 0.f;
+  for (int j = 0; j < rank; j += 8) {
+    const uint4 uv = __ldg(reinterpret_cast<const uint4 *>(U + i * ldu + j));
+    const float uf[8] = {bf16_lo(uv.x), bf16_hi(uv.x), bf16_lo(uv.y), bf16_hi(uv.y),
+                         bf16_lo(uv.z), bf16_hi(uv.z), bf16_lo(uv.w), bf16_hi(uv.w)};
+#pragma unroll
+    for (int b = 0; b < BP; ++b)
+#pragma unroll
+      for (int e = 0; e < 8; ++e) acc[b] = fmaf(uf[e], t[b * rank + j + e], acc[b]);
+  }
+  for (int b = 0; b < batch; ++b) Y[b * ldy + i] += acc[b];
+}
+
+// ---------------------------------------------------------------------------
+// host side
+// ---------------------------------------------------------------------------
+
+int pad_batch(int batch) {
+  if (batch <= 1) return 1;
+  if (batch <= 2) return 2;
+  if (batch <= 4) return 4;
+  if (batch <= 8) return 8;
+  return 16;
+}
+
+enum Shape { kS128x128, kS128x64, kS64x64, kS64x128, kGeneric };
+
+Shape shape_of(int b1, int b2) {
+  if (b1 == 128 && b2 == 128) return kS128x128;
+  if (b1 == 128 && b2 == 64) return kS128x64;
+  if (b1 == 64 && b2 == 64) return kS64x64;
+  if (b1 == 64 && b2 == 128) return kS64x128;
+  return kGeneric;
+}
+
+template <int BP, int B1, int B2, bool STRIDED>
+void *stream_kernel_ptr() {
+  return reinterpret_cast<void *>(&hybrid_stream_kernel<BP, B1, B2, STRIDED>);
+}
+
+template <bool STRIDED>
+void *pick_stream_kernel(int bp, Shape s) {
+#define HYB_CASE(BP_)                                                  \
+  case BP_:                                                            \
+    switch (s) {                                                       \
+      case kS128x128: return stream_kernel_ptr<BP_, 128, 128, STRIDED>(); \
+      case kS128x64: return stream_kernel_ptr<BP_, 128, 64, STRIDED>();   \
+      case kS64x64: return stream_kernel_ptr<BP_, 64, 64, STRIDED>();     \
+      case kS64x128: return stream_kernel_ptr<BP_, 64, 128, STRIDED>();   \
+      default: return nullptr;                                         \
+    }
+  switch (bp) {
+    HYB_CASE(1)
+    HYB_CASE(2)
+    HYB_CASE(4)
+    HYB_CASE(8)
+    HYB_CASE(16)
+    default: return nullptr;
+  }
+#undef HYB_CASE
+}
+
+template <bool STRIDED>
+void *pick_rowwarp_kernel(int bp) {
+  switch (bp) {
+    case 1: return reinterpret_cast<void *>(&hybrid_rowwarp_kernel<1, STRIDED>);
+    case 2: return reinterpret_cast<void *>(&hybrid_rowwarp_kernel<2, STRIDED>);
+    case 4: return reinterpret_cast<void *>(&hybrid_rowwarp_kernel<4, STRIDED>);
+    case 8: return reinterpret_cast<void *>(&hybrid_rowwarp_kernel<8, STRIDED>);
+    default: return reinterpret_cast<void *>(&hybrid_rowwarp_kernel<16, STRIDED>);
+  }
+}
+
+void *pick_lowrank_t(int bp) {
+  switch (bp) {
+    case 1: return reinterpret_cast<void *>(&lowrank_t_kernel<1>);
+    case 2: return reinterpret_cast<void *>(&lowrank_t_kernel<2>);
+    case 4: return reinterpret_cast<void *>(&lowrank_t_kernel<4>);
+    case 8: return reinterpret_cast<void *>(&lowrank_t_kernel<8>);
+    default: return reinterpret_cast<void *>(&lowrank_t_kernel<16>);
+  }
+}
+
+void *pick_lowrank_apply(int bp) {
+  switch (bp) {
+    case 1: return reinterpret_cast<void *>(&lowrank_apply_kernel<1>);
+    case 2: return reinterpret_cast<void *>(&lowrank_apply_kernel<2>);
+    case 4: return reinterpret_cast<void *>(&lowrank_apply_kernel<4>);
+    case 8: return reinterpret_cast<void *>(&lowrank_apply_kernel<8>);
+    default: return reinterpret_cast<void *>(&lowrank_apply_kernel<16>);
+  }
+}
+
+// Resident CTAs per SM of a kernel instance (cached; the answer only depends
+// on the instance and the device).
+int blocks_per_sm(void *fn, size_t dyn_smem) {
+  static std::mutex mu;
+  struct Entry {
+    void *fn;
+    int dev;
+    size_t smem;
+    int blocks;
+  };
+  static Entry cache[256];
+  static int used = 0;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return -1;
+  // dynamic shared memory is small; bucket it so the cache stays tiny
+  const size_t bucket = align_up(dyn_smem, 4096);
+  std::lock_guard<std::mutex> lock(mu);
+  for (int i = 0; i < used; ++i)
+    if (cache[i].fn == fn && cache[i].dev == dev && cache[i].smem == bucket)
+      return cache[i].blocks;
+  int nb = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&nb, fn, kThreads, bucket) !=
+      cudaSuccess)
+    return -1;
+  if (used < 256) cache[used++] = Entry{fn, dev, bucket, nb};
+  return nb;
+}
+
+// Work split and workspace layout of one product call.
+struct Plan {
+  bool stream;     // tuned kernel (else one warp per row)
+  int bp;          // padded batch
+  int b1, b2;
+  int G;           // CTAs of the stream split
+  int R;           // bands
+  int64_t total;   // packed bytes
+  int lr_ctas;     // CTAs of the low-rank reduction
+  size_t off_counters, off_lr_t, off_lr_part, off_lr_counter, off_partials,
+      bytes;
+  size_t dyn_smem;
+};
+
+int make_plan(int64_t n, int64_t k, int b1, int b2, int64_t total_bytes,
+              int batch, int rank, bool strided, Plan *pl) {
+  Plan P{};
+  P.bp = pad_batch(batch);
+  P.b1 = b1;
+  P.b2 = b2;
+  P.R = (int)(n / b1);
+  P.total = total_bytes;
+  const Shape s = shape_of(b1, b2);
+  P.stream = s != kGeneric && P.R <= 8192;
+  int sms = 0;
+  int rc = device_sm_count(&sms);
+  if (rc != HYB_OK) return rc;
+  P.dyn_smem = P.stream ? (size_t)2 * P.R * sizeof(int) : 0;
+  if (P.stream) {
+    void *fn = strided ? pick_stream_kernel<true>(P.bp, s)
+                       : pick_stream_kernel<false>(P.bp, s);
+    if (P.dyn_smem > 48 * 1024) {
+      if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               (int)P.dyn_smem) != cudaSuccess)
+        return HYB_ERR_CUDA;
+    }
+    const int nb = blocks_per_sm(fn, P.dyn_smem);
+    if (nb <= 0) return HYB_ERR_CUDA;
+    const int64_t max_cost = 2LL * b1 * b2;  // a dense tile
+    int64_t G = (int64_t)nb * sms;
+    // every CTA must own at least one tile: total / G >= largest tile
+    const int64_t gcap = std::max<int64_t>(1, total_bytes / max_cost);
+    P.G = (int)std::min(G, gcap);
+  } else {
+    P.G = 0;
+  }
+  P.lr_ctas = rank > 0 ? (int)std::max<int64_t>(1, std::min<int64_t>(sms, k / 64)) : 0;
+  size_t off = kHeaderBytes;
+  P.off_counters = off;
+  if (P.stream) off = align_up(off + (size_t)P.R * sizeof(uint32_t), 256);
+  P.off_lr_t = off;
+  off = align_up(off + (size_t)P.bp * (rank > 0 ? rank : 0) * sizeof(float), 256);
+  P.off_lr_part = off;
+  off = align_up(off + (size_t)P.lr_ctas * P.bp * (rank > 0 ? rank : 0) * sizeof(float), 256);
+  P.off_lr_counter = off;
+  off = align_up(off + sizeof(uint32_t), 256);
+  P.off_partials = off;
+  if (P.stream) off += (size_t)(P.G + P.R) * b1 * P.bp * sizeof(float);
+  P.bytes = align_up(off, 256);
+  *pl = P;
+  return HYB_OK;
+}
+
+int check_lowrank(const hyb_lowrank *lr, int64_t n, int64_t k) {
+  if (!lr) return HYB_OK;
+  if (lr->rank < 0 || lr->rank > kMaxRank) return HYB_ERR_INVALID_ARG;
+  if (lr->rank == 0) return HYB_OK;
+  if (lr->rank % 8 != 0) return HYB_ERR_UNSUPPORTED;
+  if (!lr->U || !lr->V || lr->ldu < lr->rank || lr->ldv < lr->rank)
+    return HYB_ERR_INVALID_ARG;
+  if (((uintptr_t)lr->U | (uintptr_t)lr->V) % 16 != 0 || lr->ldu % 8 != 0 ||
+      lr->ldv % 8 != 0)
+    return HYB_ERR_ALIGNMENT;
+  (void)n;
+  (void)k;
+  return HYB_OK;
+}
+
+int launch_lowrank_t(const Plan &P, const hyb_lowrank *lr, int64_t k,
+                     const uint16_t *X, int64_t ldx, int batch, uint8_t *ws,
+                     cudaStream_t s) {
+  void *fn = pick_lowrank_t(P.bp);
+  const uint16_t *V = lr->V;
+  int64_t ldv = lr->ldv;
+  int rank = lr->rank;
+  float *t_out = reinterpret_cast<float *>(ws + P.off_lr_t);
+  float *part = reinterpret_cast<float *>(ws + P.off_lr_part);
+  uint32_t *counter = reinterpret_cast<uint32_t *>(ws + P.off_lr_counter);
+  void *args[] = {&V, &ldv, &rank, &k, &X, &ldx, &batch, &t_out, &part, &counter};
+  if (cudaLaunchKernel(fn, dim3(P.lr_ctas), dim3(kThreads), args, 0, s) !=
+      cudaSuccess)
+    return HYB_ERR_CUDA;
+  return HYB_OK;
+}
+
+// Shared driver of hyb_spmv / hyb_spmm_skinny / hyb_gemv_dense.
+int run_product(Params prm, int b1, int b2, int batch, const hyb_lowrank *lr,
+                bool strided, void *ws, size_t ws_bytes, cudaStream_t s) {
+  const int rank = (lr && lr->rank > 0) ? lr->rank : 0;
+  Plan P;
+  int rc = make_plan(prm.n, prm.k, b1, b2, prm.total, batch, rank, strided, &P);
+  if (rc != HYB_OK) return rc;
+  if (!ws || ws_bytes < P.bytes) return HYB_ERR_WORKSPACE;
+  if ((uintptr_t)ws % 256 != 0) return HYB_ERR_ALIGNMENT;
+  uint8_t *w = reinterpret_cast<uint8_t *>(ws);
+  prm.R = P.R;
+  prm.G = P.G;
+  prm.partials = reinterpret_cast<float *>(w + P.off_partials);
+  prm.counters = reinterpret_cast<uint32_t *>(w + P.off_counters);
+  prm.rank = rank;
+  prm.U = rank ? lr->U : nullptr;
+  prm.ldu = rank ? lr->ldu : 0;
+  prm.lr_t = reinterpret_cast<const float *>(w + P.off_lr_t);
+  if (rank) {
+    rc = launch_lowrank_t(P, lr, prm.k, prm.X, prm.ldx, batch, w, s);
+    if (rc != HYB_OK) return rc;
+  }
+  void *args[] = {&prm};
+  if (P.stream) {
+    void *fn = strided ? pick_stream_kernel<true>(P.bp, shape_of(b1, b2))
+                       : pick_stream_kernel<false>(P.bp, shape_of(b1, b2));
+    if (cudaLaunchKernel(fn, dim3(P.G), dim3(kThreads), args, P.dyn_smem, s) !=
+        cudaSuccess)
+      return HYB_ERR_CUDA;
+  } else {
+    void *fn = strided ? pick_rowwarp_kernel<true>(P.bp)
+                       : pick_rowwarp_kernel<false>(P.bp);
+    int sms = 0;
+    rc = device_sm_count(&sms);
+    if (rc != HYB_OK) return rc;
+    const int64_t need = (prm.n + kWarps - 1) / kWarps;
+    const int64_t grid = std::min<int64_t>(need, (int64_t)sms * 8);
+    int b1v = b1, b2v = b2;
+    void *args2[] = {&prm, &b1v, &b2v};
+    if (cudaLaunchKernel(fn, dim3((unsigned)grid), dim3(kThreads), args2, 0, s) !=
+        cudaSuccess)
+      return HYB_ERR_CUDA;
+  }
+  return HYB_OK;
+}
+
+int check_io(const uint16_t *X, int64_t ldx, void *Y, int64_t ldy, int64_t n,
+             int64_t k, int batch, int ydt) {
+  if (!X || !Y) return HYB_ERR_INVALID_ARG;
+  if (batch < 1 || batch > 16) return HYB_ERR_INVALID_ARG;
+  if (ydt != HYB_F32 && ydt != HYB_BF16) return HYB_ERR_INVALID_ARG;
+  if (ldx < k || ldy < n) return HYB_ERR_INVALID_ARG;
+  if (((uintptr_t)X | (uintptr_t)Y) % 16 != 0 || ldx % 8 != 0) return HYB_ERR_ALIGNMENT;
+  if ((ldy * (ydt == HYB_F32 ? 4 : 2)) % 16 != 0) return HYB_ERR_ALIGNMENT;
+  return HYB_OK;
+}
+
+int spmm_impl(const hyb_matrix *A, int batch, const uint16_t *X, int64_t ldx,
+              void *Y, int64_t ldy, hyb_dtype ydt, const hyb_lowrank *lr,
+              void *ws, size_t ws_bytes, cudaStream_t s) {
+  if (!A) return HYB_ERR_INVALID_ARG;
+  int rc = check_tiling(A->n, A->k, A->b1, A->b2);
+  if (rc != HYB_OK) return rc;
+  if (A->num_tiles != (A->n / A->b1) * (A->k / A->b2)) return HYB_ERR_INVALID_ARG;
+  if (!A->tile_map || !A->vals || !A->meta || !A->val_off || !A->meta_off)
+    return HYB_ERR_INVALID_ARG;
+  const int64_t te = (int64_t)A->b1 * A->b2;
+  if (A->n_vals < A->num_tiles * te / 2 || A->n_vals > A->num_tiles * te ||
+      A->n_meta_bytes < 0 || A->n_meta_bytes > A->num_tiles * te / 8)
+    return HYB_ERR_INVALID_ARG;
+  if (((uintptr_t)A->vals) % 32 != 0 || ((uintptr_t)A->meta) % 16 != 0)
+    return HYB_ERR_ALIGNMENT;
+  rc = check_io(X, ldx, Y, ldy, A->n, A->k, batch, ydt);
+  if (rc != HYB_OK) return rc;
+  rc = check_lowrank(lr, A->n, A->k);
+  if (rc != HYB_OK) return rc;
+  Params prm{};
+  prm.map = A->tile_map;
+  prm.vals = reinterpret_cast<const uint8_t *>(A->vals);
+  prm.meta = A->meta;
+  prm.val_off = A->val_off;
+  prm.meta_off = A->meta_off;
+  prm.n = A->n;
+  prm.k = A->k;
+  prm.tpr = A->k / A->b2;
+  prm.T = A->num_tiles;
+  prm.X = X;
+  prm.ldx = ldx;
+  prm.batch = batch;
+  prm.Y = Y;
+  prm.ldy = ldy;
+  prm.ydt = ydt;
+  prm.total = 2 * A->n_vals + A->n_meta_bytes;  // packed bytes
+  return run_product(prm, A->b1, A->b2, batch, lr, false, ws, ws_bytes, s);
+}
+
+// Virtual tiling of a plain row-major W for the dense baseline.
+void dense_tiling(int64_t n, int64_t k, int *b1, int *b2) {
+  if (n % 128 == 0 && k % 128 == 0) {
+    *b1 = 128;
+    *b2 = 128;
+  } else if (n % 64 == 0 && k % 64 == 0) {
+    *b1 = 64;
+    *b2 = 64;
+  } else {
+    *b1 = 1;
+    *b2 = 16;
+  }
+}
+
+size_t lowrank_ws_layout(int64_t k, int batch, int rank, size_t *off_t,
+                         size_t *off_part, size_t *off_counter, int *ctas) {
+  int sms = 0;
+  if (device_sm_count(&sms) != HYB_OK) return 0;
+  const int bp = pad_batch(batch);
+  *ctas = (int)std::max<int64_t>(1, std::min<int64_t>(sms, k / 64));
+  size_t off = kHeaderBytes;
+  *off_t = off;
+  off = align_up(off + (size_t)bp * rank * sizeof(float), 256);
+  *off_part = off;
+  off = align_up(off + (size_t)(*ctas) * bp * rank * sizeof(float), 256);
+  *off_counter = off;
+  off = align_up(off + sizeof(uint32_t), 256);
+  return off;
+}
+
+}  // namespace
+}  // namespace hyb
+
+using namespace hyb;
+
+extern "C" {
+
+size_t hyb_workspace_bytes(const hyb_matrix *A, int batch, int rank) {
+  if (!A || check_tiling(A->n, A->k, A->b1, A->b2) != HYB_OK) return 0;
+  if (batch < 1 || batch > 16 || rank < 0 || rank > kMaxRank) return 0;
+  Plan P;
+  if (make_plan(A->n, A->k, A->b1, A->b2, 2 * A->n_vals + A->n_meta_bytes,
+                batch, rank, false, &P) != HYB_OK)
+    return 0;
+  return P.bytes;
+}
+
+int hyb_spmv(const hyb_matrix *A, const uint16_t *X, int64_t ldx, void *Y,
+             int64_t ldy, hyb_dtype ydt, const hyb_lowrank *lr, void *ws,
+             size_t ws_bytes, hyb_stream_t stream) {
+  return spmm_impl(A, 1, X, ldx, Y, ldy, ydt, lr, ws, ws_bytes,
+                   (cudaStream_t)stream);
+}
+
+int hyb_spmm_skinny(const hyb_matrix *A, int batch, const uint16_t *X,
+                    int64_t ldx, void *Y, int64_t ldy, hyb_dtype ydt,
+                    const hyb_lowrank *lr, void *ws, size_t ws_bytes,
+                    hyb_stream_t stream) {
+  return spmm_impl(A, batch, X, ldx, Y, ldy, ydt, lr, ws, ws_bytes,
+                   (cudaStream_t)stream);
+}
+
+size_t hyb_lowrank_workspace_bytes(int64_t k, int batch, int rank) {
+  if (k <= 0 || batch < 1 || batch > 16 || rank < 1 || rank > kMaxRank) return 0;
+  size_t a, b, c;
+  int ctas;
+  return lowrank_ws_layout(k, batch, rank, &a, &b, &c, &ctas);
+}
+
+int hyb_lowrank_add(int64_t n, int64_t k, int batch, const hyb_lowrank *lr,
+                    const uint16_t *X, int64_t ldx, float *Y, int64_t ldy,
+                    void *ws, size_t ws_bytes, hyb_stream_t stream) {
+  if (n <= 0 || k <= 0 || !lr || lr->rank < 1) return HYB_ERR_INVALID_ARG;
+  int rc = check_io(X, ldx, Y, ldy, n, k, batch, HYB_F32);
+  if (rc != HYB_OK) return rc;
+  rc = check_lowrank(lr, n, k);
+  if (rc != HYB_OK) return rc;
+  size_t off_t, off_part, off_counter;
+  int ctas;
+  const size_t need =
+      lowrank_ws_layout(k, batch, lr->rank, &off_t, &off_part, &off_counter, &ctas);
+  if (need == 0) return HYB_ERR_CUDA;
+  if (!ws || ws_bytes < need) return HYB_ERR_WORKSPACE;
+  if ((uintptr_t)ws % 256 != 0) return HYB_ERR_ALIGNMENT;
+  cudaStream_t s = (cudaStream_t)stream;
+  uint8_t *w = reinterpret_cast<uint8_t *>(ws);
+  const int bp = pad_batch(batch);
+  {
+    const uint16_t *V = lr->V;
+    int64_t ldv = lr->ldv, kk = k, ldxx = ldx;
+    int rank = lr->rank, bt = batch;
+    const uint16_t *Xp = X;
+    float *t_out = reinterpret_cast<float *>(w + off_t);
+    float *part = reinterpret_cast<float *>(w + off_part);
+    uint32_t *counter = reinterpret_cast<uint32_t *>(w + off_counter);
+    void *args[] = {&V, &ldv, &rank, &kk, &Xp, &ldxx, &bt, &t_out, &part, &counter};
+    if (cudaLaunchKernel(pick_lowrank_t(bp), dim3(ctas), dim3(kThreads), args, 0, s) !=
+        cudaSuccess)
+      return HYB_ERR_CUDA;
+  }
+  {
+    int64_t nn = n, ldu = lr->ldu, ldyy = ldy;
+    const uint16_t *U = lr->U;
+    int rank = lr->rank, bt = batch;
+    const float *t = reinterpret_cast<const float *>(w + off_t);
+    float *Yp = Y;
+    void *args[] = {&nn, &U, &ldu, &rank, &t, &bt, &Yp, &ldyy};
+    const int64_t grid = (n + kThreads - 1) / kThreads;
+    if (cudaLaunchKernel(pick_lowrank_apply(bp), dim3((unsigned)grid), dim3(kThreads),
+                         args, 0, s) != cudaSuccess)
+      return HYB_ERR_CUDA;
+  }
+  return HYB_OK;
+}
+
+size_t hyb_dense_workspace_bytes(int64_t n, int64_t k, int batch) {
+  if (n <= 0 || k <= 0 || k % 16 != 0 || batch < 1 || batch > 16) return 0;
+  int b1, b2;
+  dense_tiling(n, k, &b1, &b2);
+  Plan P;
+  if (make_plan(n, k, b1, b2, 2 * n * k, batch, 0, true, &P) != HYB_OK) return 0;
+  return P.bytes;
+}
+
+int hyb_gemv_dense(int64_t n, int64_t k, int batch, const uint16_t *W,
+                   int64_t ldw, const uint16_t *X, int64_t ldx, void *Y,
+                   int64_t ldy, hyb_dtype ydt, void *ws, size_t ws_bytes,
+                   hyb_stream_t stream) {
+  if (n <= 0 || k <= 0 || !W || ldw < k) return HYB_ERR_INVALID_ARG;
+  if (k % 16 != 0) return HYB_ERR_INVALID_ARG;
+  int rc = check_io(X, ldx, Y, ldy, n, k, batch, ydt);
+  if (rc != HYB_OK) return rc;
+  if ((uintptr_t)W % 32 != 0 || ldw % 16 != 0) return HYB_ERR_ALIGNMENT;
+  int b1, b2;
+  dense_tiling(n, k, &b1, &b2);
+  Params prm{};
+  prm.Wd = W;
+  prm.ldw = ldw;
+  prm.n = n;
+  prm.k = k;
+  prm.tpr = k / b2;
+  prm.T = (n / b1) * (k / b2);
+  prm.X = X;
+  prm.ldx = ldx;
+  prm.batch = batch;
+  prm.Y = Y;
+  prm.ldy = ldy;
+  prm.ydt = ydt;
+  prm.total = 2 * n * k;
+  return run_product(prm, b1, b2, batch, nullptr, true, ws, ws_bytes,
+                     (cudaStream_t)stream);
+}
+
+}  // extern "C"

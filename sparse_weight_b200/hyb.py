@@ -1,0 +1,345 @@
+"""Thin Python binding of libhyb (include/hyb.h): argument marshalling only.
+
+Every step of the product runs in the CUDA library; PyTorch provides device
+memory and the current stream.  Function names follow the C ABI without the
+``hyb_`` prefix.  bf16 tensors cross as their raw 16-bit patterns.
+
+If ``libhyb.so`` is missing the first call raises; there is no fallback.
+"""
+import ctypes
+import os
+from dataclasses import dataclass
+from typing import Optional
+
+import numpy as np
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libhyb.so")
+
+HYB_OK = 0
+HYB_ERR_INVALID_ARG = -1
+HYB_ERR_UNSUPPORTED = -2
+HYB_ERR_ALIGNMENT = -3
+HYB_ERR_WORKSPACE = -4
+HYB_ERR_CUDA = -5
+HYB_ERR_DEVICE_CHECK = -6
+
+HYB_F32 = 0
+HYB_BF16 = 1
+
+STATUS_NAN = 1
+STATUS_BAD_MAP = 2
+
+_P = ctypes.c_void_p
+_I64 = ctypes.c_int64
+_I = ctypes.c_int
+_SZ = ctypes.c_size_t
+
+
+class HybMatrix(ctypes.Structure):
+    _fields_ = [("n", ctypes.c_int64), ("k", ctypes.c_int64),
+                ("b1", ctypes.c_int32), ("b2", ctypes.c_int32),
+                ("num_tiles", ctypes.c_int64),
+                ("tile_map", _P), ("vals", _P), ("meta", _P),
+                ("val_off", _P), ("meta_off", _P),
+                ("n_vals", ctypes.c_int64), ("n_meta_bytes", ctypes.c_int64)]
+
+
+class HybLowrank(ctypes.Structure):
+    _fields_ = [("rank", ctypes.c_int32), ("U", _P), ("ldu", ctypes.c_int64),
+                ("V", _P), ("ldv", ctypes.c_int64)]
+
+
+class HybError(RuntimeError):
+    def __init__(self, fn, status):
+        self.status = status
+        super().__init__(f"{fn}: {status_string(status)} ({status})")
+
+
+_lib = None
+
+EXPORTS = ["hyb_packed_sizes", "hyb_pack_workspace_bytes", "hyb_pack",
+           "hyb_workspace_bytes", "hyb_workspace_init", "hyb_spmv",
+           "hyb_spmm_skinny", "hyb_lowrank_workspace_bytes", "hyb_lowrank_add",
+           "hyb_dense_workspace_bytes", "hyb_gemv_dense", "hyb_check_status",
+           "hyb_status_string"]
+
+
+def lib():
+    """Load libhyb.so (raises if it has not been built)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise RuntimeError(f"libhyb.so not built ({LIB_PATH}); run "
+                           "`python -m sparse_weight_b200.build`")
+    L = ctypes.CDLL(LIB_PATH)
+    L.hyb_packed_sizes.argtypes = [_I64, _I64, _I, _I, _P, _P, _P]
+    L.hyb_packed_sizes.restype = _I
+    L.hyb_pack_workspace_bytes.argtypes = []
+    L.hyb_pack_workspace_bytes.restype = _SZ
+    L.hyb_pack.argtypes = [_I64, _I64, _I, _I, _P, _I64, _P, _P, _P, _P, _P, _P, _SZ, _P]
+    L.hyb_pack.restype = _I
+    L.hyb_workspace_bytes.argtypes = [ctypes.POINTER(HybMatrix), _I, _I]
+    L.hyb_workspace_bytes.restype = _SZ
+    L.hyb_workspace_init.argtypes = [_P, _SZ, _P]
+    L.hyb_workspace_init.restype = _I
+    L.hyb_spmv.argtypes = [ctypes.POINTER(HybMatrix), _P, _I64, _P, _I64, _I,
+                           ctypes.POINTER(HybLowrank), _P, _SZ, _P]
+    L.hyb_spmv.restype = _I
+    L.hyb_spmm_skinny.argtypes = [ctypes.POINTER(HybMatrix), _I, _P, _I64, _P, _I64, _I,
+                                  ctypes.POINTER(HybLowrank), _P, _SZ, _P]
+    L.hyb_spmm_skinny.restype = _I
+    L.hyb_lowrank_workspace_bytes.argtypes = [_I64, _I, _I]
+    L.hyb_lowrank_workspace_bytes.restype = _SZ
+    L.hyb_lowrank_add.argtypes = [_I64, _I64, _I, ctypes.POINTER(HybLowrank), _P, _I64,
+                                  _P, _I64, _P, _SZ, _P]
+    L.hyb_lowrank_add.restype = _I
+    L.hyb_dense_workspace_bytes.argtypes = [_I64, _I64, _I]
+    L.hyb_dense_workspace_bytes.restype = _SZ
+    L.hyb_gemv_dense.argtypes = [_I64, _I64, _I, _P, _I64, _P, _I64, _P, _I64, _I, _P,
+                                 _SZ, _P]
+    L.hyb_gemv_dense.restype = _I
+    L.hyb_check_status.argtypes = [_P, _P, ctypes.POINTER(ctypes.c_uint32)]
+    L.hyb_check_status.restype = _I
+    L.hyb_status_string.argtypes = [_I]
+    L.hyb_status_string.restype = ctypes.c_char_p
+    _lib = L
+    return L
+
+
+def status_string(status: int) -> str:
+    return lib().hyb_status_string(int(status)).decode()
+
+
+def _check(fn, rc):
+    if rc != HYB_OK:
+        raise HybError(fn, rc)
+
+
+def _stream(stream=None):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _bits(t: torch.Tensor) -> torch.Tensor:
+    """View a bf16 (or int16/uint16) tensor as its 16-bit patterns."""
+    if t.dtype == torch.bfloat16:
+        return t.view(torch.int16)
+    if t.dtype in (torch.int16, torch.uint16):
+        return t
+    raise TypeError(f"expected bf16 data, got {t.dtype}")
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+# ---------------------------------------------------------------------------
+# format
+# ---------------------------------------------------------------------------
+
+def packed_sizes(n: int, k: int, b1: int, b2: int, tile_map) -> tuple:
+    """(n_vals, n_meta_bytes) for a host tile map (numpy/torch CPU uint8)."""
+    m = np.ascontiguousarray(np.asarray(tile_map.cpu() if torch.is_tensor(tile_map)
+                                        else tile_map, dtype=np.uint8).reshape(-1))
+    nv, nm = _I64(), _I64()
+    _check("hyb_packed_sizes", lib().hyb_packed_sizes(
+        n, k, b1, b2, m.ctypes.data_as(_P), ctypes.byref(nv), ctypes.byref(nm)))
+    return nv.value, nm.value
+
+
+@dataclass
+class Packed:
+    """A packed tile-hybrid matrix on the device (tensors own the memory)."""
+    n: int
+    k: int
+    b1: int
+    b2: int
+    tile_map: torch.Tensor   # uint8 [T], device
+    vals: torch.Tensor       # int16 [n_vals] (bf16 bits), device
+    meta: torch.Tensor       # uint8 [max(n_meta, 1)], device
+    val_off: torch.Tensor    # int64 [T+1], device
+    meta_off: torch.Tensor   # int64 [T+1], device
+    n_vals: int
+    n_meta: int
+
+    @property
+    def num_tiles(self) -> int:
+        return self.tile_map.numel()
+
+    def struct(self) -> HybMatrix:
+        return HybMatrix(self.n, self.k, self.b1, self.b2, self.num_tiles,
+                         self.tile_map.data_ptr(), self.vals.data_ptr(),
+                         self.meta.data_ptr(), self.val_off.data_ptr(),
+                         self.meta_off.data_ptr(), self.n_vals, self.n_meta)
+
+    def nbytes(self) -> int:
+        """Packed bytes the product streams (values + masks)."""
+        return 2 * self.n_vals + self.n_meta
+
+    def clone(self) -> "Packed":
+        return Packed(self.n, self.k, self.b1, self.b2, self.tile_map.clone(),
+                      self.vals.clone(), self.meta.clone(), self.val_off.clone(),
+                      self.meta_off.clone(), self.n_vals, self.n_meta)
+
+
+def pack_workspace_bytes() -> int:
+    return int(lib().hyb_pack_workspace_bytes())
+
+
+def workspace_init(ws: torch.Tensor, stream=None):
+    _check("hyb_workspace_init", lib().hyb_workspace_init(_ptr(ws), ws.numel(), _stream(stream)))
+
+
+def new_workspace(nbytes: int, device) -> torch.Tensor:
+    """Zeroed device workspace (uint8), 256-byte aligned by the allocator."""
+    ws = torch.zeros(max(int(nbytes), 256), dtype=torch.uint8, device=device)
+    assert ws.data_ptr() % 256 == 0
+    return ws
+
+
+def pack(W: torch.Tensor, tile_map, b1: int, b2: int, ws: torch.Tensor = None,
+         stream=None, check: bool = True) -> Packed:
+    """hyb_pack: dense bf16 W [n][k] (device) + tile map -> Packed.
+
+    With ``check`` the call synchronises and raises HybError on a NaN weight or
+    a bad map byte (the pack itself is complete either way)."""
+    Wb = _bits(W)
+    assert Wb.is_cuda and Wb.dim() == 2
+    n, k = Wb.shape
+    tm_host = tile_map.cpu().numpy() if torch.is_tensor(tile_map) else np.asarray(tile_map)
+    tm_host = np.ascontiguousarray(tm_host, dtype=np.uint8).reshape(-1)
+    nv, nm = packed_sizes(n, k, b1, b2, tm_host)
+    dev = Wb.device
+    tm = torch.from_numpy(tm_host).to(dev)
+    T = tm.numel()
+    vals = torch.empty(nv, dtype=torch.int16, device=dev)
+    meta = torch.empty(max(nm, 1), dtype=torch.uint8, device=dev)
+    vo = torch.empty(T + 1, dtype=torch.int64, device=dev)
+    mo = torch.empty(T + 1, dtype=torch.int64, device=dev)
+    own_ws = ws is None
+    if own_ws:
+        ws = new_workspace(pack_workspace_bytes(), dev)
+    _check("hyb_pack", lib().hyb_pack(n, k, b1, b2, _ptr(Wb), Wb.stride(0), _ptr(tm),
+                                      _ptr(vals), _ptr(meta), _ptr(vo), _ptr(mo),
+                                      _ptr(ws), ws.numel(), _stream(stream)))
+    if check:
+        check_status(ws, stream)
+    return Packed(n, k, b1, b2, tm, vals, meta, vo, mo, nv, nm)
+
+
+def check_status(ws: torch.Tensor, stream=None) -> int:
+    """hyb_check_status: sync, read + clear the status word; raise on a flag."""
+    flags = ctypes.c_uint32(0)
+    rc = lib().hyb_check_status(_ptr(ws), _stream(stream), ctypes.byref(flags))
+    if rc != HYB_OK:
+        err = HybError("hyb_check_status", rc)
+        err.flags = flags.value
+        raise err
+    return flags.value
+
+
+# ---------------------------------------------------------------------------
+# products
+# ---------------------------------------------------------------------------
+
+def workspace_bytes(A: Packed, batch: int = 1, rank: int = 0) -> int:
+    s = A.struct()
+    nbytes = int(lib().hyb_workspace_bytes(ctypes.byref(s), batch, rank))
+    if nbytes == 0:
+        raise HybError("hyb_workspace_bytes", HYB_ERR_INVALID_ARG)
+    return nbytes
+
+
+def _lowrank_struct(lowrank):
+    if lowrank is None:
+        return None, None
+    U, V = (_bits(t) for t in lowrank)
+    lr = HybLowrank(U.shape[1], U.data_ptr(), U.stride(0), V.data_ptr(), V.stride(0))
+    return lr, (U, V)
+
+
+def _out(n, batch, ydt, device, Y):
+    if Y is not None:
+        return Y
+    dt = torch.float32 if ydt == HYB_F32 else torch.bfloat16
+    return torch.empty(batch, n, dtype=dt, device=device)
+
+
+def spmm_skinny(A: Packed, X: torch.Tensor, Y: torch.Tensor = None, ydt: int = HYB_F32,
+                lowrank=None, ws: torch.Tensor = None, stream=None) -> torch.Tensor:
+    """hyb_spmm_skinny: Y[batch][n] = W_hat X (+ U (V^T X)); X bf16 [batch][k]."""
+    Xb = _bits(X)
+    if Xb.dim() == 1:
+        Xb = Xb.view(1, -1)
+    batch = Xb.shape[0]
+    Y = _out(A.n, batch, ydt, Xb.device, Y)
+    lr, keep = _lowrank_struct(lowrank)
+    if ws is None:
+        ws = new_workspace(workspace_bytes(A, batch, lr.rank if lr else 0), Xb.device)
+    s = A.struct()
+    _check("hyb_spmm_skinny", lib().hyb_spmm_skinny(
+        ctypes.byref(s), batch, _ptr(Xb), Xb.stride(0), _ptr(Y), Y.stride(0), ydt,
+        ctypes.byref(lr) if lr else None, _ptr(ws), ws.numel(), _stream(stream)))
+    return Y
+
+
+def spmv(A: Packed, x: torch.Tensor, y: torch.Tensor = None, ydt: int = HYB_F32,
+         lowrank=None, ws: torch.Tensor = None, stream=None) -> torch.Tensor:
+    """hyb_spmv: y[1][n] = W_hat x (+ U (V^T x)); x bf16 [k] or [1][k]."""
+    xb = _bits(x).reshape(1, -1)
+    y = _out(A.n, 1, ydt, xb.device, y)
+    lr, keep = _lowrank_struct(lowrank)
+    if ws is None:
+        ws = new_workspace(workspace_bytes(A, 1, lr.rank if lr else 0), xb.device)
+    s = A.struct()
+    _check("hyb_spmv", lib().hyb_spmv(
+        ctypes.byref(s), _ptr(xb), xb.stride(0), _ptr(y), y.stride(0), ydt,
+        ctypes.byref(lr) if lr else None, _ptr(ws), ws.numel(), _stream(stream)))
+    return y
+
+
+def lowrank_workspace_bytes(k: int, batch: int, rank: int) -> int:
+    return int(lib().hyb_lowrank_workspace_bytes(k, batch, rank))
+
+
+def lowrank_add(U: torch.Tensor, V: torch.Tensor, X: torch.Tensor, Y: torch.Tensor,
+                ws: torch.Tensor = None, stream=None) -> torch.Tensor:
+    """hyb_lowrank_add: Y (fp32 [batch][n]) += U (V^T X), in place."""
+    Xb = _bits(X)
+    if Xb.dim() == 1:
+        Xb = Xb.view(1, -1)
+    batch, k = Xb.shape
+    n = Y.shape[-1]
+    lr, keep = _lowrank_struct((U, V))
+    if ws is None:
+        ws = new_workspace(lowrank_workspace_bytes(k, batch, lr.rank), Xb.device)
+    _check("hyb_lowrank_add", lib().hyb_lowrank_add(
+        n, k, batch, ctypes.byref(lr), _ptr(Xb), Xb.stride(0), _ptr(Y), Y.stride(0),
+        _ptr(ws), ws.numel(), _stream(stream)))
+    return Y
+
+
+def dense_workspace_bytes(n: int, k: int, batch: int = 1) -> int:
+    return int(lib().hyb_dense_workspace_bytes(n, k, batch))
+
+
+def gemv_dense(W: torch.Tensor, X: torch.Tensor, Y: torch.Tensor = None,
+               ydt: int = HYB_F32, ws: torch.Tensor = None, stream=None) -> torch.Tensor:
+    """hyb_gemv_dense: Y[batch][n] = W X for a plain row-major bf16 W [n][k]."""
+    Wb = _bits(W)
+    Xb = _bits(X)
+    if Xb.dim() == 1:
+        Xb = Xb.view(1, -1)
+    n, k = Wb.shape
+    batch = Xb.shape[0]
+    Y = _out(n, batch, ydt, Xb.device, Y)
+    if ws is None:
+        ws = new_workspace(dense_workspace_bytes(n, k, batch), Xb.device)
+    _check("hyb_gemv_dense", lib().hyb_gemv_dense(
+        n, k, batch, _ptr(Wb), Wb.stride(0), _ptr(Xb), Xb.stride(0), _ptr(Y), Y.stride(0),
+        ydt, _ptr(ws), ws.numel(), _stream(stream)))
+    return Y

@@ -1,0 +1,151 @@
+"""The C ABI without a GPU: the library loads, exports every entry point
+declared in include/hyb.h, and rejects bad arguments synchronously (these
+checks run before any CUDA call, so they are safe on a machine with no GPU)."""
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+from sparse_weight_b200 import hyb
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def declared_symbols():
+    txt = open(os.path.join(ROOT, "include", "hyb.h")).read()
+    return sorted(set(re.findall(r"HYB_API\s+[\w\s\*]*?\b(hyb_\w+)\s*\(", txt)))
+
+
+@pytest.fixture(scope="module")
+def L():
+    from sparse_weight_b200 import build
+    build.build()
+    return hyb.lib()
+
+
+def test_exports_every_declared_symbol(L):
+    names = declared_symbols()
+    assert len(names) >= 13
+    for name in names:
+        assert hasattr(L, name), name
+    assert set(hyb.EXPORTS) == set(names)
+
+
+def test_status_strings(L):
+    for code in range(0, -7, -1):
+        assert hyb.status_string(code)
+    assert "unknown" in hyb.status_string(-99)
+
+
+def _sizes(n, k, b1, b2, m):
+    m = np.ascontiguousarray(m, np.uint8)
+    nv, nm = ctypes.c_int64(), ctypes.c_int64()
+    rc = hyb.lib().hyb_packed_sizes(n, k, b1, b2, m.ctypes.data_as(ctypes.c_void_p),
+                                    ctypes.byref(nv), ctypes.byref(nm))
+    return rc, nv.value, nm.value
+
+
+def test_packed_sizes_closed_form(L, orc):
+    rng = np.random.default_rng(0)
+    for (n, k, b1, b2) in [(256, 256, 64, 64), (4096, 4096, 128, 128), (1024, 4096, 128, 64),
+                           (64, 96, 16, 32)]:
+        T = (n // b1) * (k // b2)
+        m = (rng.random(T) < 0.5).astype(np.uint8)
+        rc, nv, nm = _sizes(n, k, b1, b2, m)
+        assert rc == hyb.HYB_OK
+        assert (nv, nm) == orc.packed_sizes(n, k, b1, b2, m)
+        s = int(m.sum())
+        assert nv == (T - s) * b1 * b2 + s * b1 * b2 // 2 and nm == s * b1 * b2 // 8
+
+
+@pytest.mark.parametrize("shape", [(0, 64, 16, 16), (64, 64, 16, 8), (60, 64, 16, 16),
+                                   (64, 60, 16, 16), (8, 16, 1, 16)])
+def test_packed_sizes_rejects_bad_tiling(L, shape):
+    n, k, b1, b2 = shape
+    T = max(1, (n // max(b1, 1)) * (k // max(b2, 1)))
+    rc, _, _ = _sizes(n, k, b1, b2, np.zeros(T, np.uint8))
+    assert rc == hyb.HYB_ERR_INVALID_ARG
+
+
+def test_packed_sizes_rejects_bad_map_byte(L):
+    m = np.zeros(16, np.uint8)
+    m[3] = 2
+    rc, _, _ = _sizes(256, 256, 64, 64, m)
+    assert rc == hyb.HYB_ERR_INVALID_ARG
+
+
+def test_pack_argument_checks(L):
+    P = ctypes.c_void_p
+    good = P(0x10000)
+    odd = P(0x10008)
+    # null W
+    assert L.hyb_pack(64, 64, 16, 16, None, 64, good, good, good, good, good, good, 256,
+                      None) == hyb.HYB_ERR_INVALID_ARG
+    # ldw < k
+    assert L.hyb_pack(64, 64, 16, 16, good, 32, good, good, good, good, good, good, 256,
+                      None) == hyb.HYB_ERR_INVALID_ARG
+    # no workspace
+    assert L.hyb_pack(64, 64, 16, 16, good, 64, good, good, good, good, good, None, 0,
+                      None) == hyb.HYB_ERR_WORKSPACE
+    # misaligned W
+    assert L.hyb_pack(64, 64, 16, 16, odd, 64, good, good, good, good, good, good, 256,
+                      None) == hyb.HYB_ERR_ALIGNMENT
+
+
+def _matrix(**kw):
+    d = dict(n=256, k=256, b1=64, b2=64, num_tiles=16, tile_map=0x10000, vals=0x20000,
+             meta=0x30000, val_off=0x40000, meta_off=0x50000, n_vals=256 * 256,
+             n_meta_bytes=0)
+    d.update(kw)
+    return hyb.HybMatrix(**d)
+
+
+def test_spmv_argument_checks(L):
+    P = ctypes.c_void_p
+    X, Y, ws = P(0x60000), P(0x70000), P(0x80000)
+    A = _matrix()
+    call = lambda A, X=X, ldx=256, Y=Y, ldy=256, ydt=0, lr=None: L.hyb_spmv(
+        ctypes.byref(A), X, ldx, Y, ldy, ydt, lr, ws, 1 << 20, None)
+    assert L.hyb_spmv(None, X, 256, Y, 256, 0, None, ws, 1 << 20, None) == hyb.HYB_ERR_INVALID_ARG
+    assert call(_matrix(num_tiles=15)) == hyb.HYB_ERR_INVALID_ARG
+    assert call(_matrix(vals=None)) == hyb.HYB_ERR_INVALID_ARG
+    assert call(_matrix(meta=None)) == hyb.HYB_ERR_INVALID_ARG
+    assert call(_matrix(n_vals=5)) == hyb.HYB_ERR_INVALID_ARG
+    assert call(_matrix(vals=0x20010)) == hyb.HYB_ERR_ALIGNMENT
+    assert call(A, X=None) == hyb.HYB_ERR_INVALID_ARG
+    assert call(A, ldx=100) == hyb.HYB_ERR_INVALID_ARG
+    assert call(A, ldx=260) == hyb.HYB_ERR_ALIGNMENT
+    assert call(A, X=P(0x60002)) == hyb.HYB_ERR_ALIGNMENT
+    assert call(A, ydt=7) == hyb.HYB_ERR_INVALID_ARG
+    lr = hyb.HybLowrank(12, 0x90000, 16, 0xA0000, 16)
+    assert call(A, lr=ctypes.byref(lr)) == hyb.HYB_ERR_UNSUPPORTED
+    lr = hyb.HybLowrank(16, None, 16, 0xA0000, 16)
+    assert call(A, lr=ctypes.byref(lr)) == hyb.HYB_ERR_INVALID_ARG
+    lr = hyb.HybLowrank(512, 0x90000, 512, 0xA0000, 512)
+    assert call(A, lr=ctypes.byref(lr)) == hyb.HYB_ERR_INVALID_ARG
+    # batch out of range
+    assert L.hyb_spmm_skinny(ctypes.byref(A), 17, X, 256, Y, 256, 0, None, ws, 1 << 20,
+                             None) == hyb.HYB_ERR_INVALID_ARG
+    assert L.hyb_spmm_skinny(ctypes.byref(A), 0, X, 256, Y, 256, 0, None, ws, 1 << 20,
+                             None) == hyb.HYB_ERR_INVALID_ARG
+
+
+def test_dense_and_lowrank_argument_checks(L):
+    P = ctypes.c_void_p
+    W, X, Y, ws = P(0x10000), P(0x60000), P(0x70000), P(0x80000)
+    assert L.hyb_gemv_dense(64, 40, 1, W, 40, X, 40, Y, 64, 0, ws, 1 << 20,
+                            None) == hyb.HYB_ERR_INVALID_ARG  # k % 16
+    assert L.hyb_gemv_dense(64, 64, 1, P(0x10010), 64, X, 64, Y, 64, 0, ws, 1 << 20,
+                            None) == hyb.HYB_ERR_ALIGNMENT
+    assert L.hyb_gemv_dense(64, 64, 1, W, 72, X, 64, Y, 64, 0, ws, 1 << 20,
+                            None) == hyb.HYB_ERR_ALIGNMENT
+    lr = hyb.HybLowrank(0, P(0x90000), 8, P(0xA0000), 8)
+    assert L.hyb_lowrank_add(64, 64, 1, ctypes.byref(lr), X, 64, Y, 64, ws, 1 << 20,
+                             None) == hyb.HYB_ERR_INVALID_ARG
+    assert L.hyb_workspace_bytes(None, 1, 0) == 0
+    A = _matrix(b2=8)
+    assert L.hyb_workspace_bytes(ctypes.byref(A), 1, 0) == 0
+    assert L.hyb_workspace_init(None, 0, None) == hyb.HYB_ERR_WORKSPACE
+    assert L.hyb_check_status(None, None, None) == hyb.HYB_ERR_WORKSPACE

@@ -1,0 +1,167 @@
+"""hyb_spmv / hyb_spmm_skinny on the GPU against the fp64 CPU oracle.
+
+Bound (spec tolerance, fp32 accumulation of bf16 products):
+|y - y_ref|_i <= 2e-3 * (|W_hat| |x| + |U| (|V|^T |x|))_i, per output."""
+import numpy as np
+import pytest
+import torch
+
+from sparse_weight_b200 import hyb, inputs
+from gpu_cases import assert_within, bf16_within_one_ulp, case, dev
+
+pytestmark = pytest.mark.gpu
+
+
+def _full_check(orc, n, k, b1, b2, tmap, batch, name, rank=0, ydt_bf16=True):
+    W, tmap, X, UV = case(n, k, b1, b2, tmap, batch=batch, name=name, rank=rank)
+    P = hyb.pack(W.to(dev()), tmap, b1, b2)
+    Xd = X.to(dev())
+    lr = tuple(t.to(dev()) for t in UV) if UV else None
+    Y = hyb.spmm_skinny(P, Xd, lowrank=lr)
+    torch.cuda.synchronize()
+    ref = orc.pack(inputs.bits(W), b1, b2, tmap)
+    U = inputs.bits(UV[0]) if UV else None
+    V = inputs.bits(UV[1]) if UV else None
+    y_ref, env = orc.spmv(n, k, b1, b2, tmap, ref, inputs.bits(X), U, V)
+    assert_within(Y.cpu().numpy(), y_ref, env, what=f"{name} {n}x{k} b={batch}")
+    if ydt_bf16:
+        Yb = hyb.spmm_skinny(P, Xd, ydt=hyb.HYB_BF16, lowrank=lr)
+        bf16_within_one_ulp(Yb, Y)
+    return P, Xd, Y
+
+
+def test_tiny_256(orc):
+    tmap = inputs.tile_map_exact(16, 8, inputs.seed_of("tiny_256", "map"))
+    _full_check(orc, 256, 256, 64, 64, tmap, 1, "tiny_256")
+
+
+def test_attn_4096(orc):
+    _full_check(orc, 4096, 4096, 128, 128, inputs.attn_map(1024), 1, "attn_4096")
+
+
+def test_spmv_entry_point_batch1(orc):
+    """hyb_spmv (batch-1 entry point) equals hyb_spmm_skinny at batch 1."""
+    tmap = inputs.attn_map(1024)
+    W, tmap, X, _ = case(4096, 4096, 128, 128, tmap, name="attn_4096")
+    P = hyb.pack(W.to(dev()), tmap, 128, 128)
+    y1 = hyb.spmv(P, X.to(dev()).view(-1))
+    y2 = hyb.spmm_skinny(P, X.to(dev()))
+    assert torch.equal(y1, y2)
+
+
+@pytest.mark.parametrize("tiling", [(128, 128), (128, 64), (64, 64), (64, 128)])
+@pytest.mark.parametrize("batch", [1, 2, 3, 4, 5, 8, 13, 16])
+def test_multi_tile_ragged(orc, tiling, batch):
+    """Shapes that span several tiles and bands, with byte splits that end
+    mid-band: every batch specialisation (and non-power-of-2 batches)."""
+    b1, b2 = tiling
+    n, k = b1 * 5, b2 * 11
+    T = 55
+    tmap = inputs.tile_map_bernoulli(T, 0.4, inputs.seed_of("ragged", b1, b2))
+    _full_check(orc, n, k, b1, b2, tmap, batch, f"ragged{b1}x{b2}")
+
+
+@pytest.mark.parametrize("tiling", [(16, 16), (32, 32), (8, 16), (1, 128), (128, 16), (256, 64)])
+@pytest.mark.parametrize("batch", [1, 3, 16])
+def test_other_tilings(orc, tiling, batch):
+    b1, b2 = tiling
+    n, k = b1 * 6, b2 * 5
+    tmap = inputs.tile_map_bernoulli(30, 0.5, inputs.seed_of("tilings", b1, b2))
+    _full_check(orc, n, k, b1, b2, tmap, batch, f"tilings{b1}x{b2}")
+
+
+@pytest.mark.parametrize("frac", [0.0, 1.0])
+def test_degenerate_maps(orc, frac):
+    """All-dense and all-2:4 maps (0 % and 50 % sparsity)."""
+    T = 32 * 32
+    tmap = np.full(T, int(frac), np.uint8)
+    _full_check(orc, 4096, 4096, 128, 128, tmap, 4, f"degenerate{frac}")
+
+
+def test_single_tile(orc):
+    _full_check(orc, 128, 128, 128, 128, np.array([1], np.uint8), 1, "single")
+    _full_check(orc, 64, 64, 64, 64, np.array([0], np.uint8), 2, "single0")
+
+
+def test_zero_input(orc):
+    """x = 0 gives exactly zero output."""
+    tmap = inputs.attn_map(1024)
+    W, tmap, X, _ = case(4096, 4096, 128, 128, tmap, name="attn_4096")
+    P = hyb.pack(W.to(dev()), tmap, 128, 128)
+    y = hyb.spmv(P, torch.zeros(4096, dtype=torch.bfloat16, device=dev()))
+    assert torch.count_nonzero(y).item() == 0
+
+
+def test_deterministic():
+    """Fixed split and fixed-order reductions: identical bits run to run."""
+    tmap = inputs.attn_map(1024)
+    W, tmap, X, _ = case(4096, 4096, 128, 128, tmap, batch=4, name="attn_4096")
+    P = hyb.pack(W.to(dev()), tmap, 128, 128)
+    Xd = X.to(dev())
+    ws = hyb.new_workspace(hyb.workspace_bytes(P, 4), dev())
+    first = hyb.spmm_skinny(P, Xd, ws=ws).clone()
+    for _ in range(10):
+        assert torch.equal(hyb.spmm_skinny(P, Xd, ws=ws), first)
+
+
+def _sampled_rows(n, b1, count, seed):
+    rng = np.random.default_rng(seed)
+    fixed = [0, 1, b1 - 1, b1, n // 2, n - b1, n - 2, n - 1]
+    return np.unique(np.concatenate([fixed, rng.integers(0, n, size=count)])).astype(np.int64)
+
+
+@pytest.mark.parametrize("shape", [(14336, 4096), (4096, 14336)])
+@pytest.mark.parametrize("frac", [0.0, 0.25, 0.5, 0.75, 1.0])
+def test_ffn_sweep_full_size(orc, shape, frac):
+    """Full FFN shapes with 1 % x20 outliers, the 2:4-tile fraction sweep, batch
+    {1, 4, 8, 16}: sampled output rows against the oracle's per-row product."""
+    n, k = shape
+    T = (n // 128) * (k // 128)
+    tmap = inputs.tile_map_fraction(T, frac, inputs.seed_of("ffn_sweep", n, k, frac))
+    W, tmap, X, _ = case(n, k, 128, 128, tmap, batch=16, outliers=0.01, name="ffn_sweep")
+    P = hyb.pack(W.to(dev()), tmap, 128, 128)
+    rows = _sampled_rows(n, 128, 120, 17)
+    Wb = inputs.bits(W)
+    for batch in (1, 4, 8, 16):
+        Xb = X[:batch]
+        Y = hyb.spmm_skinny(P, Xb.to(dev())).cpu().numpy()
+        y_ref, env = orc.rows(Wb, 128, 128, tmap, inputs.bits(Xb), rows)
+        assert_within(Y[:, rows], y_ref, env, what=f"ffn {n}x{k} f={frac} b={batch}")
+
+
+def test_llama8b_layer_full_size(orc):
+    """One 32-layer-chain layer (128x64 tiles, per-layer fraction), batch 1."""
+    layer = 3
+    f = inputs.chain_fraction(layer)
+    for role, n, k in inputs.LLAMA8B_LAYER:
+        T = (n // 128) * (k // 64)
+        tmap = inputs.tile_map_fraction(T, f, inputs.seed_of("llama8b_chain", layer, role, "map"))
+        W, tmap, X, _ = case(n, k, 128, 64, tmap, name=f"llama8b/{layer}/{role}")
+        P = hyb.pack(W.to(dev()), tmap, 128, 64)
+        rows = _sampled_rows(n, 128, 64, 5)
+        Y = hyb.spmv(P, X.to(dev())).cpu().numpy()
+        y_ref, env = orc.rows(inputs.bits(W), 128, 64, tmap, inputs.bits(X), rows)
+        assert_within(Y[:, rows], y_ref, env, what=f"llama8b {role}")
+
+
+def test_llama70b_ffn_lowrank_full_size(orc):
+    """All-2:4 70B-shaped FFN plus rank-128 low-rank term, fused; batch {1,8,16}."""
+    for role, n, k in inputs.LLAMA70B_FFN:
+        T = (n // 128) * (k // 128)
+        W, tmap, X, UV = case(n, k, 128, 128, np.ones(T, np.uint8), batch=16, std=0.015,
+                              name=f"llama70b/{role}", rank=128)
+        P = hyb.pack(W.to(dev()), tmap, 128, 128)
+        lr = tuple(t.to(dev()) for t in UV)
+        rows = _sampled_rows(n, 128, 48, 9)
+        for batch in (1, 8, 16):
+            Y = hyb.spmm_skinny(P, X[:batch].to(dev()), lowrank=lr).cpu().numpy()
+            y_ref, env = orc.rows(inputs.bits(W), 128, 128, tmap, inputs.bits(X[:batch]),
+                                  rows, inputs.bits(UV[0]), inputs.bits(UV[1]))
+            assert_within(Y[:, rows], y_ref, env, what=f"70b {role} b={batch}")
+        del P, W
+
+
+@pytest.mark.parametrize("batch", [1, 5, 16])
+def test_lowrank_fused_small(orc, batch):
+    tmap = inputs.tile_map_bernoulli(40, 0.6, inputs.seed_of("lrsmall"))
+    _full_check(orc, 640, 1024, 128, 128, tmap, batch, "lrsmall", rank=64)
