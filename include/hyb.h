@@ -50,9 +50,9 @@
  *    ready for the next call.  Two calls that run concurrently must not share
  *    a workspace.
  *  - X is [batch][k] bf16 with leading dimension ldx >= k; Y is [batch][n]
- *    (fp32 or bf16) with ldy >= n.  X, Y and meta must be 16-byte aligned,
- *    vals 32-byte aligned, workspaces 256-byte aligned; ldx and ldy must keep
- *    rows 16-byte aligned.
+ *    (fp32 or bf16) with ldy >= n.  X and meta must be 16-byte aligned and
+ *    ldx a multiple of 8 (rows of X 16-byte aligned); vals 32-byte aligned;
+ *    Y aligned to its element size; workspaces 256-byte aligned.
  *  - Shapes: n % b1 == 0, k % b2 == 0, b2 % 16 == 0, (b1 * b2) % 128 == 0.
  *    Any batch 1..16.  Tiles of 64 or 128 rows by 64 or 128 columns run the
  *    tuned streaming kernel; other legal tilings run a simpler CUDA kernel
@@ -177,8 +177,10 @@ HYB_API size_t hyb_dense_workspace_bytes(int64_t n, int64_t k, int batch);
 
 /* Plain dense Y = W X for W [n][k] bf16 row-major (row stride ldw), the
  * dense baseline the pages compare the hybrid format against (PATCH §4,
- * SparseDecoding abstract).  Same streaming design as hyb_spmv. Needs
- * n % 8 == 0, k % 16 == 0, ldw % 16 == 0, W 32-byte aligned. */
+ * SparseDecoding abstract).  Same streaming design as hyb_spmv.  Needs
+ * k % 16 == 0.  When n and k are both multiples of 64 the tuned kernel runs
+ * and W must be 32-byte aligned with ldw % 16 == 0; otherwise a one-warp-
+ * per-row kernel runs and W must be 16-byte aligned with ldw % 8 == 0. */
 HYB_API int hyb_gemv_dense(int64_t n, int64_t k, int batch, const uint16_t *W,
                    int64_t ldw, const uint16_t *X, int64_t ldx, void *Y,
                    int64_t ldy, hyb_dtype ydt, void *ws, size_t ws_bytes,

@@ -118,6 +118,7 @@ def test_spmv_argument_checks(L):
     assert call(A, ldx=100) == hyb.HYB_ERR_INVALID_ARG
     assert call(A, ldx=260) == hyb.HYB_ERR_ALIGNMENT
     assert call(A, X=P(0x60002)) == hyb.HYB_ERR_ALIGNMENT
+    assert call(A, Y=P(0x70002)) == hyb.HYB_ERR_ALIGNMENT  # fp32 Y needs 4 bytes
     assert call(A, ydt=7) == hyb.HYB_ERR_INVALID_ARG
     lr = hyb.HybLowrank(12, 0x90000, 16, 0xA0000, 16)
     assert call(A, lr=ctypes.byref(lr)) == hyb.HYB_ERR_UNSUPPORTED
@@ -140,6 +141,8 @@ def test_dense_and_lowrank_argument_checks(L):
     assert L.hyb_gemv_dense(64, 64, 1, P(0x10010), 64, X, 64, Y, 64, 0, ws, 1 << 20,
                             None) == hyb.HYB_ERR_ALIGNMENT
     assert L.hyb_gemv_dense(64, 64, 1, W, 72, X, 64, Y, 64, 0, ws, 1 << 20,
+                            None) == hyb.HYB_ERR_ALIGNMENT
+    assert L.hyb_gemv_dense(60, 48, 1, W, 52, X, 48, Y, 64, 0, ws, 1 << 20,
                             None) == hyb.HYB_ERR_ALIGNMENT
     lr = hyb.HybLowrank(0, P(0x90000), 8, P(0xA0000), 8)
     assert L.hyb_lowrank_add(64, 64, 1, ctypes.byref(lr), X, 64, Y, 64, ws, 1 << 20,
