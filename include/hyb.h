@@ -186,6 +186,36 @@ HYB_API int hyb_gemv_dense(int64_t n, int64_t k, int batch, const uint16_t *W,
                    int64_t ldy, hyb_dtype ydt, void *ws, size_t ws_bytes,
                    hyb_stream_t stream);
 
+/* ---- product without any allocation ------------------------------------ */
+
+/* hyb_spmv for callers that cannot allocate device memory -- an engine that
+ * hands out all device memory from one arena sized at start-up, code that
+ * runs while a CUDA graph is being captured (cudaMalloc is not allowed
+ * there), a host whose memory pool refuses allocations after set-up.  The
+ * pages have no counterpart of this entry point; it is a library facility.
+ *
+ * Same operation, arguments and output as hyb_spmv with batch 1 and no
+ * low-rank term, but no workspace argument: the scratch (band tickets and
+ * split partial sums) lives in one static device array of
+ * hyb_spmv_noalloc_max_scratch_bytes() bytes (1 MiB), which every GPU that
+ * loads the library holds until the process exits.  The call allocates and
+ * frees nothing.  A matrix whose scratch would exceed the array (with
+ * 128-row tiles: more than about 1,600 tile-row bands) is rejected with
+ * HYB_ERR_WORKSPACE before anything is queued.
+ *  - The first call on each device looks up the array's device address
+ *    (cudaGetSymbolAddress) with that device current; make that first call
+ *    outside any stream capture.
+ *  - All calls on a device share the one array.  Each call clears the part
+ *    that must start at zero, but two calls whose work overlaps on the GPU
+ *    (different streams, no ordering between them) race on it: order them,
+ *    for instance by using one stream. */
+HYB_API int hyb_spmv_noalloc(const hyb_matrix *A, const uint16_t *X,
+                             int64_t ldx, void *Y, int64_t ldy, hyb_dtype ydt,
+                             hyb_stream_t stream);
+
+/* Size in bytes of the static scratch array behind hyb_spmv_noalloc. */
+HYB_API size_t hyb_spmv_noalloc_max_scratch_bytes(void);
+
 /* ---- status ------------------------------------------------------------ */
 
 /* Synchronise `stream`, read and clear the workspace status word.  Returns

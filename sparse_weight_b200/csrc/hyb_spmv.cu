@@ -1047,3 +1047,92 @@ int hyb_gemv_dense(int64_t n, int64_t k, int batch, const uint16_t *W,
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// hyb_spmv_noalloc: the batch-1 product with its scratch in a fixed array.
+//
+// For callers that may not allocate device memory at all: engines that carve
+// every byte out of one arena at start-up, code running while a CUDA graph is
+// being captured (where cudaMalloc is not permitted), or hosts whose memory
+// pool forbids allocation after initialisation.  hyb_spmv needs a workspace
+// from the caller; this variant takes its split partials and band tickets from
+// a file-scope device array instead and allocates nothing.
+// ---------------------------------------------------------------------------
+namespace hyb {
+namespace {
+
+// 1 MiB per device, held from module load until the process exits.
+constexpr size_t kNoAllocScratchBytes = size_t(1) << 20;
+static __device__ __align__(256) uint8_t g_noalloc_scratch[kNoAllocScratchBytes];
+
+// Device address of the array on the current device.  The name of a
+// __device__ variable in host code is only a host-side stand-in, so the
+// address is looked up once per device (with that device current) and
+// cached.
+int noalloc_scratch_ptr(void **out) {
+  static std::mutex mu;
+  static void *addr[64] = {nullptr};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return HYB_ERR_CUDA;
+  if (dev < 0 || dev >= 64) return HYB_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lock(mu);
+  if (addr[dev] == nullptr) {
+    void *p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr)
+      return HYB_ERR_CUDA;
+    addr[dev] = p;
+  }
+  *out = addr[dev];
+  return HYB_OK;
+}
+
+// The argument checks of the batch-1 product, run before anything is queued.
+int noalloc_validate(const hyb_matrix *A, const uint16_t *X, int64_t ldx,
+                     void *Y, int64_t ldy, int ydt) {
+  if (!A) return HYB_ERR_INVALID_ARG;
+  int rc = check_tiling(A->n, A->k, A->b1, A->b2);
+  if (rc != HYB_OK) return rc;
+  if (A->num_tiles != (A->n / A->b1) * (A->k / A->b2)) return HYB_ERR_INVALID_ARG;
+  if (!A->tile_map || !A->vals || !A->meta || !A->val_off || !A->meta_off)
+    return HYB_ERR_INVALID_ARG;
+  const int64_t te = (int64_t)A->b1 * A->b2;
+  if (A->n_vals < A->num_tiles * te / 2 || A->n_vals > A->num_tiles * te ||
+      A->n_meta_bytes < 0 || A->n_meta_bytes > A->num_tiles * te / 8)
+    return HYB_ERR_INVALID_ARG;
+  if (((uintptr_t)A->vals) % 32 != 0 || ((uintptr_t)A->meta) % 16 != 0)
+    return HYB_ERR_ALIGNMENT;
+  return check_io(X, ldx, Y, ldy, A->n, A->k, 1, ydt);
+}
+
+}  // namespace
+}  // namespace hyb
+
+extern "C" {
+
+size_t hyb_spmv_noalloc_max_scratch_bytes(void) {
+  return hyb::kNoAllocScratchBytes;
+}
+
+int hyb_spmv_noalloc(const hyb_matrix *A, const uint16_t *X, int64_t ldx,
+                     void *Y, int64_t ldy, hyb_dtype ydt, hyb_stream_t stream) {
+  int rc = hyb::noalloc_validate(A, X, ldx, Y, ldy, ydt);
+  if (rc != HYB_OK) return rc;
+  hyb::Plan P;
+  rc = hyb::make_plan(A->n, A->k, A->b1, A->b2, 2 * A->n_vals + A->n_meta_bytes,
+                      1, 0, false, &P);
+  if (rc != HYB_OK) return rc;
+  if (P.bytes > hyb::kNoAllocScratchBytes) return HYB_ERR_WORKSPACE;
+  void *scratch = nullptr;
+  rc = hyb::noalloc_scratch_ptr(&scratch);
+  if (rc != HYB_OK) return rc;
+  cudaStream_t s = (cudaStream_t)stream;
+  // The array keeps whatever the previous call left.  The status word and the
+  // band tickets must start at zero (the partial slots are always written
+  // before they are read), so clear everything in front of the slots.
+  if (cudaMemsetAsync(scratch, 0, P.off_partials, s) != cudaSuccess)
+    return HYB_ERR_CUDA;
+  return hyb::spmm_impl(A, 1, X, ldx, Y, ldy, ydt, nullptr, scratch,
+                        hyb::kNoAllocScratchBytes, s);
+}
+
+}  // extern "C"

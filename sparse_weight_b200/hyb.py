@@ -63,7 +63,7 @@ EXPORTS = ["hyb_packed_sizes", "hyb_pack_workspace_bytes", "hyb_pack",
            "hyb_workspace_bytes", "hyb_workspace_init", "hyb_spmv",
            "hyb_spmm_skinny", "hyb_lowrank_workspace_bytes", "hyb_lowrank_add",
            "hyb_dense_workspace_bytes", "hyb_gemv_dense", "hyb_check_status",
-           "hyb_status_string"]
+           "hyb_status_string", "hyb_spmv_noalloc", "hyb_spmv_noalloc_max_scratch_bytes"]
 
 
 def lib():
@@ -103,6 +103,10 @@ def lib():
     L.hyb_gemv_dense.restype = _I
     L.hyb_check_status.argtypes = [_P, _P, ctypes.POINTER(ctypes.c_uint32)]
     L.hyb_check_status.restype = _I
+    L.hyb_spmv_noalloc.argtypes = [ctypes.POINTER(HybMatrix), _P, _I64, _P, _I64, _I, _P]
+    L.hyb_spmv_noalloc.restype = _I
+    L.hyb_spmv_noalloc_max_scratch_bytes.argtypes = []
+    L.hyb_spmv_noalloc_max_scratch_bytes.restype = _SZ
     L.hyb_status_string.argtypes = [_I]
     L.hyb_status_string.restype = ctypes.c_char_p
     _lib = L
@@ -343,3 +347,22 @@ def gemv_dense(W: torch.Tensor, X: torch.Tensor, Y: torch.Tensor = None,
         n, k, batch, _ptr(Wb), Wb.stride(0), _ptr(Xb), Xb.stride(0), _ptr(Y), Y.stride(0),
         ydt, _ptr(ws), ws.numel(), _stream(stream)))
     return Y
+
+
+def spmv_noalloc(A: Packed, x: torch.Tensor, y: torch.Tensor = None, ydt: int = HYB_F32,
+                 stream=None) -> torch.Tensor:
+    """hyb_spmv_noalloc: hyb_spmv (batch 1, no low-rank term) without a caller
+    workspace; the library's own static device array holds the scratch, so the
+    call allocates nothing (``y`` may be passed in to avoid the output
+    allocation here too).  Make the first call on a device outside any stream
+    capture, and do not let two calls overlap on the GPU."""
+    xb = _bits(x).reshape(1, -1)
+    y = _out(A.n, 1, ydt, xb.device, y)
+    s = A.struct()
+    _check("hyb_spmv_noalloc", lib().hyb_spmv_noalloc(
+        ctypes.byref(s), _ptr(xb), xb.stride(0), _ptr(y), y.stride(0), ydt, _stream(stream)))
+    return y
+
+
+def spmv_noalloc_max_scratch_bytes() -> int:
+    return int(lib().hyb_spmv_noalloc_max_scratch_bytes())
