@@ -338,7 +338,7 @@ def workload_config(name, frac_real):
     return {"workload": name, "n": n, "k": k, "tile": f"{b1}x{b2}",
             "sparse_tile_frac": round(frac_real, 4), "batch": batch,
             "weights": f"bf16 N(0,{std})" + (f" with {outliers:.0%} x20 outliers" if outliers else ""),
-            "l2": f"inputs larger than L2: {ROTATE} rotating packed copies",
+            "l2": f"inputs larger than L2: {ROTATE} rotating packed copies (1.47 GB)",
             "parallelism": "replicas"}
 
 
@@ -352,7 +352,15 @@ def main():
     ap.add_argument("--impl", default="hyb", choices=["hyb", "reference"])
     ap.add_argument("--workload", default="ffn_down_4096x14336_f0.5_b1", choices=list(WORKLOADS))
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--rotate", type=int, default=ROTATE,
+                    help="packed copies cycled through (their total must exceed L2)")
+    ap.add_argument("--profile", action="store_true",
+                    help="small case for a profiler: 2 rotating copies (184 MB > L2), "
+                         "hybrid product only, no dense / end-to-end / CPU legs")
     args = ap.parse_args()
+    if args.profile:
+        args.rotate = 2
+        args.no_cpu_baseline = True
     world, rank, local = dist_env()
     if args.impl == "reference":
         return run_reference(args, world, rank)
@@ -363,11 +371,15 @@ def main():
         import datetime
         torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                              device_id=device)
-    wl = Workload(args.workload, device)
+    wl = Workload(args.workload, device, rotate=args.rotate)
     stream = wl.stream
 
     with ClockSampler(local) as clocks:
         ms = timed(wl.step, args.steps, args.warmup, stream, world)
+    if args.profile:
+        if rank == 0:
+            print(json.dumps({"profile_run": args.workload, "ms": ms, "steps": args.steps}))
+        return 0
     dense_ms = timed(wl.dense_step, args.steps, args.warmup, stream, world)
     e2e_ms, h2d, d2h = e2e_timed(wl, args.steps, args.warmup, stream, world)
 
