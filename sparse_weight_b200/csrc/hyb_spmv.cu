@@ -67,6 +67,10 @@ struct Params {
   int64_t total;  // packed bytes of the whole matrix
   float *partials;
   uint32_t *counters;
+  // work units of the TMA kernel: runs of UT tiles inside one band, Ub per band
+  int NU, Ub, UT;
+  uint32_t *sched;   // [0] next unit, [1] CTAs done
+  uint32_t *status;  // workspace status word
 };
 
 // ---------------------------------------------------------------------------
@@ -430,6 +434,408 @@ __global__ void __launch_bounds__(kThreads, (Cfg<BP, B1, B2, STRIDED>::kMinBlock
 }
 
 // ---------------------------------------------------------------------------
+// the TMA-ring kernel for packed hybrid matrices
+// ---------------------------------------------------------------------------
+//
+// One CTA per SM.  A producer warp copies whole tiles (values, masks and the
+// matching slice of X) from HBM into a ring of shared-memory stages with 1-D
+// bulk copies (cp.async.bulk, completion counted on an mbarrier), so the bytes
+// in flight are set by the ring size, not by registers.  B1/8 consumer warps
+// compute from shared memory.  Work is handed out in units -- runs of UT
+// consecutive tiles inside one tile-row band -- from an atomic counter, so a
+// slow SM simply takes fewer units.  A unit's row sums go to its own fp32 slot;
+// the last unit of a band to finish (atomic ticket) sums the band's slots in
+// unit order, so the result does not depend on which CTA ran which unit.
+//
+// Products use the mixed-precision FMA of sm_100 (bf16 x bf16 + fp32 -> fp32,
+// the product is exact) straight on packed bf16 pairs, and PRMT picks the two
+// x values of a 2:4 group from the 4-bit mask through a 16-entry selector
+// table ("SparseDecoding", authors' abstract: bitmask-indexed N:M SpMV).
+
+constexpr uint32_t kStatusTimeout = 4u;  // a pipeline wait ran out
+constexpr uint32_t kWaitLimit = 1u << 22;
+
+__device__ __forceinline__ uint32_t smem_u32(const void *p) {
+  return (uint32_t)__cvta_generic_to_shared(p);
+}
+__device__ __forceinline__ void mbar_init(uint64_t *bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count)
+               : "memory");
+}
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t *bar, uint32_t tx) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)),
+               "r"(tx)
+               : "memory");
+}
+__device__ __forceinline__ void mbar_arrive(uint64_t *bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+// Every wait is bounded: on expiry the caller records kStatusTimeout and
+// leaves the pipeline instead of spinning for ever.
+__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity) {
+  for (uint32_t i = 0; i < kWaitLimit; ++i)
+    if (mbar_try_wait(bar, parity)) return true;
+  return false;
+}
+__device__ __forceinline__ void bulk_g2s(void *dst, const void *src, uint32_t bytes,
+                                         uint64_t *bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::
+          "r"(smem_u32(dst)),
+      "l"(src), "r"(bytes), "r"(smem_u32(bar))
+      : "memory");
+}
+// acc += lo(w) * lo(x) + hi(w) * hi(x) on two packed bf16 pairs.
+__device__ __forceinline__ void fma_bf16x2(float &acc, uint32_t w, uint32_t x) {
+  unsigned short wl, wh, xl, xh;
+  asm("mov.b32 {%0,%1}, %2;" : "=h"(wl), "=h"(wh) : "r"(w));
+  asm("mov.b32 {%0,%1}, %2;" : "=h"(xl), "=h"(xh) : "r"(x));
+  asm("fma.rn.f32.bf16 %0, %1, %2, %0;" : "+f"(acc) : "h"(wl), "h"(xl));
+  asm("fma.rn.f32.bf16 %0, %1, %2, %0;" : "+f"(acc) : "h"(wh), "h"(xh));
+}
+
+template <int BP, int B1, int B2>
+struct TmaCfg {
+  static constexpr int NC = B1 / 8;                 // consumer warps, 8 rows each
+  static constexpr int RW = 8;                      // rows per consumer warp per tile
+  static constexpr int CPR = B2 / 16;               // lanes per row, 16 columns each
+  static constexpr int RPS = 32 / CPR;              // rows per warp step
+  static constexpr int JS = RW / RPS;               // steps per warp per tile
+  static constexpr int XB = BP < 4 ? BP : 4;        // batch columns per pass
+  static constexpr int TPS = (16384 / (B1 * B2)) > 0 ? 16384 / (B1 * B2) : 1;  // tiles per stage
+  static constexpr int kValsBytes = 2 * B1 * B2 * TPS;        // 32 KB
+  static constexpr int kMetaBytes = B1 * B2 / 8 * TPS;        // 2 KB
+  static constexpr int kXRow = 2 * B2 * TPS;                  // bytes of one X row slice
+  static constexpr int kStageBytes = kValsBytes + kMetaBytes + BP * kXRow;
+  static constexpr int kStages =
+      (220 * 1024 / kStageBytes) < 6 ? (220 * 1024 / kStageBytes) : 6;
+  static constexpr int kThreads = (NC + 1) * 32;
+  static constexpr size_t kSmem = (size_t)kStages * kStageBytes + 1024;
+  static_assert(RPS * CPR == 32 && JS * RPS == RW && JS >= 1, "tile shape");
+  static_assert(kStages >= 3, "ring too short");
+};
+
+struct StageDesc {
+  int64_t t0;        // first tile of the stage
+  int32_t unit;      // unit the tiles belong to
+  uint16_t ntiles;   // tiles in the stage (<= TPS)
+  uint8_t sparse;    // bit i: tile i is 2:4
+  uint8_t flags;     // 1: last stage of its unit, 2: end of work
+};
+
+template <int BP, int B1, int B2>
+__global__ void __launch_bounds__(TmaCfg<BP, B1, B2>::kThreads, 1)
+    hybrid_tma_kernel(const Params p) {
+  using C = TmaCfg<BP, B1, B2>;
+  constexpr int S = C::kStages;
+  extern __shared__ __align__(1024) uint8_t smem[];
+  __shared__ __align__(8) uint64_t full_bar[S];
+  __shared__ __align__(8) uint64_t empty_bar[S];
+  __shared__ StageDesc desc[S];
+  __shared__ uint32_t sel_lut[16];
+
+  const int tid = threadIdx.x;
+  const int warp = tid >> 5, lane = tid & 31;
+  if (tid == 0) {
+    for (int s = 0; s < S; ++s) {
+      mbar_init(&full_bar[s], 1);
+      mbar_init(&empty_bar[s], C::NC);
+    }
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  if (tid < 16) {
+    // PRMT selector that moves bf16 x[p0] to the low and x[p1] to the high
+    // half, p0 < p1 the set bits of the mask (x0x1 in bytes 0-3, x2x3 in 4-7)
+    const uint32_t m = tid;
+    uint32_t p0 = 0, p1 = 0;
+    if (m) {
+      p0 = __ffs(m) - 1;
+      p1 = 31 - __clz(m);
+    }
+    sel_lut[m] = (2 * p0) | ((2 * p0 + 1) << 4) | ((2 * p1) << 8) | ((2 * p1 + 1) << 12);
+  }
+  __syncthreads();
+
+  if (warp == C::NC) {
+    // ------------------------------ producer ------------------------------
+    int stage = 0;
+    uint32_t phase = 0;
+    bool ok = true;
+    auto grab = [&]() -> int {
+      int u = 0;
+      if (lane == 0) u = (int)atomicAdd(p.sched, 1u);
+      return __shfl_sync(0xffffffffu, u, 0);
+    };
+    // per-unit offsets, one tile per lane: val_off / meta_off / map of tile ta+lane
+    struct UnitOff {
+      int64_t vo, mo;
+      uint32_t sp;
+      int64_t ta;
+      int nt;
+    };
+    auto unit_off = [&](int u) -> UnitOff {
+      UnitOff o;
+      const int64_t r = u / p.Ub, q = u - r * p.Ub;
+      o.ta = r * p.tpr + q * p.UT;
+      const int64_t tb = min(o.ta + p.UT, (r + 1) * p.tpr);
+      o.nt = (int)(tb - o.ta);
+      o.vo = 0;
+      o.mo = 0;
+      o.sp = 0;
+      if (lane <= o.nt) {
+        o.vo = __ldg(p.val_off + o.ta + lane);
+        o.mo = __ldg(p.meta_off + o.ta + lane);
+      }
+      if (lane < o.nt) o.sp = __ldg(p.map + o.ta + lane) == 1;
+      return o;
+    };
+    uint32_t armed = 0, armed_parity = 0;  // per stage: copies issued / phase parity
+    int u = grab();
+    UnitOff cur{};
+    if (u < p.NU) cur = unit_off(u);
+    int un = grab();
+    while (ok && u < p.NU) {
+      UnitOff nxt{};
+      if (un < p.NU) nxt = unit_off(un);  // loads in flight while this unit issues
+      // the grab after next: its result is only read once this unit is issued
+      uint32_t unn_raw = 0;
+      if (un < p.NU && lane == 0) unn_raw = atomicAdd(p.sched, 1u);
+      const uint32_t spmask = __ballot_sync(0xffffffffu, cur.sp != 0);
+      for (int i = 0; i < cur.nt; i += C::TPS) {
+        const int nt = min(C::TPS, cur.nt - i);
+        const int64_t v0 = __shfl_sync(0xffffffffu, cur.vo, i);
+        const int64_t v1 = __shfl_sync(0xffffffffu, cur.vo, i + nt);
+        const int64_t m0 = __shfl_sync(0xffffffffu, cur.mo, i);
+        const int64_t m1 = __shfl_sync(0xffffffffu, cur.mo, i + nt);
+        if (lane == 0) {
+          if (!mbar_wait(&empty_bar[stage], phase ^ 1u)) {
+            ok = false;
+          } else {
+            uint8_t *st = smem + (size_t)stage * C::kStageBytes;
+            const uint32_t vbytes = (uint32_t)(2 * (v1 - v0));
+            const uint32_t mbytes = (uint32_t)(m1 - m0);
+            const int64_t t = cur.ta + i;
+            const int64_t tc = t % p.tpr;
+            const uint32_t xrow = (uint32_t)(2 * B2 * nt);
+            StageDesc d;
+            d.t0 = t;
+            d.unit = u;
+            d.ntiles = (uint16_t)nt;
+            d.sparse = (uint8_t)((spmask >> i) & ((1u << nt) - 1u));
+            d.flags = (i + nt >= cur.nt) ? 1 : 0;
+            desc[stage] = d;
+            armed |= 1u << stage;
+            armed_parity = (armed_parity & ~(1u << stage)) | (phase << stage);
+            mbar_arrive_expect_tx(&full_bar[stage], vbytes + mbytes + xrow * p.batch);
+            bulk_g2s(st, p.vals + 2 * v0, vbytes, &full_bar[stage]);
+            if (mbytes) bulk_g2s(st + C::kValsBytes, p.meta + m0, mbytes, &full_bar[stage]);
+            for (int b = 0; b < p.batch; ++b)
+              bulk_g2s(st + C::kValsBytes + C::kMetaBytes + b * C::kXRow,
+                       p.X + (int64_t)b * p.ldx + tc * B2, xrow, &full_bar[stage]);
+          }
+        }
+        ok = __shfl_sync(0xffffffffu, ok, 0);
+        if (!ok) break;
+        if (++stage == S) {
+          stage = 0;
+          phase ^= 1u;
+        }
+      }
+      const int unn = (un < p.NU) ? (int)__shfl_sync(0xffffffffu, unn_raw, 0) : un;
+      u = un;
+      un = unn;
+      cur = nxt;
+    }
+    if (lane == 0) {
+      if (ok && mbar_wait(&empty_bar[stage], phase ^ 1u)) {
+        StageDesc d{};
+        d.flags = 2;
+        desc[stage] = d;
+        mbar_arrive(&full_bar[stage]);
+      } else {
+        ok = false;
+      }
+      if (!ok) {
+        atomicOr(p.status, kStatusTimeout);
+        // let every copy already issued land before the CTA's shared memory
+        // goes away (bounded, like every other wait)
+        for (int s = 0; s < S; ++s)
+          if (armed >> s & 1u) mbar_wait(&full_bar[s], armed_parity >> s & 1u);
+      }
+      // the last CTA to finish resets the unit counter for the next call
+      __threadfence();
+      if (atomicAdd(p.sched + 1, 1u) == (uint32_t)gridDim.x - 1) {
+        p.sched[0] = 0;
+        p.sched[1] = 0;
+      }
+    }
+    return;
+  }
+
+  // -------------------------------- consumers --------------------------------
+  const int cp = lane % C::CPR;
+  const int rs = lane / C::CPR;
+  const int wrow = warp * C::RW;
+  float acc[C::JS][BP];
+#pragma unroll
+  for (int j = 0; j < C::JS; ++j)
+#pragma unroll
+    for (int b = 0; b < BP; ++b) acc[j][b] = 0.f;
+
+  int stage = 0;
+  uint32_t phase = 0;
+  for (;;) {
+    if (!mbar_wait(&full_bar[stage], phase)) {
+      if (lane == 0) atomicOr(p.status, kStatusTimeout);
+      break;
+    }
+    const StageDesc d = desc[stage];
+    if (d.flags & 2) break;
+    const uint8_t *st = smem + (size_t)stage * C::kStageBytes;
+    int voff = 0, moff = 0;
+    for (int i = 0; i < d.ntiles; ++i) {
+      const bool sp = (d.sparse >> i) & 1;
+      // a lane covers columns [16cp, 16cp+16) of a 2:4 tile row, and columns
+      // [8cp, 8cp+8) + [B2/2 + 8cp, B2/2 + 8cp + 8) of a dense tile row (so
+      // that 8 lanes read 128 contiguous bytes of shared memory)
+      const uint8_t *xs = st + C::kValsBytes + C::kMetaBytes + i * 2 * B2;
+      const int xo0 = sp ? 32 * cp : 16 * cp;
+      const int xo1 = sp ? 32 * cp + 16 : B2 + 16 * cp;
+#pragma unroll
+      for (int b0 = 0; b0 < BP; b0 += C::XB) {
+        uint32_t xr[C::XB][8];
+#pragma unroll
+        for (int b = 0; b < C::XB; ++b) {
+          const uint4 lo = *reinterpret_cast<const uint4 *>(xs + (b0 + b) * C::kXRow + xo0);
+          const uint4 hi = *reinterpret_cast<const uint4 *>(xs + (b0 + b) * C::kXRow + xo1);
+          xr[b][0] = lo.x; xr[b][1] = lo.y; xr[b][2] = lo.z; xr[b][3] = lo.w;
+          xr[b][4] = hi.x; xr[b][5] = hi.y; xr[b][6] = hi.z; xr[b][7] = hi.w;
+        }
+        if (sp) {
+#pragma unroll
+          for (int j = 0; j < C::JS; ++j) {
+            const int row = wrow + j * C::RPS + rs;
+            const uint4 v = *reinterpret_cast<const uint4 *>(st + voff + row * B2 + 16 * cp);
+            const uint32_t m = *reinterpret_cast<const uint16_t *>(
+                st + C::kValsBytes + moff + row * (B2 / 8) + 2 * cp);
+            const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+            for (int g = 0; g < 4; ++g) {
+              const uint32_t sel = sel_lut[(m >> (4 * g)) & 0xFu];
+#pragma unroll
+              for (int b = 0; b < C::XB; ++b) {
+                const uint32_t xp = __byte_perm(xr[b][2 * g], xr[b][2 * g + 1], sel);
+                fma_bf16x2(acc[j][b0 + b], w[g], xp);
+              }
+            }
+          }
+        } else {
+#pragma unroll
+          for (int j = 0; j < C::JS; ++j) {
+            const int row = wrow + j * C::RPS + rs;
+            const uint4 a = *reinterpret_cast<const uint4 *>(st + voff + row * 2 * B2 + 16 * cp);
+            const uint4 c2 =
+                *reinterpret_cast<const uint4 *>(st + voff + row * 2 * B2 + B2 + 16 * cp);
+            const uint32_t w[8] = {a.x, a.y, a.z, a.w, c2.x, c2.y, c2.z, c2.w};
+#pragma unroll
+            for (int e = 0; e < 8; ++e)
+#pragma unroll
+              for (int b = 0; b < C::XB; ++b) fma_bf16x2(acc[j][b0 + b], w[e], xr[b][e]);
+          }
+        }
+      }
+      voff += sp ? B1 * B2 : 2 * B1 * B2;
+      moff += sp ? B1 * B2 / 8 : 0;
+    }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&empty_bar[stage]);
+    if (++stage == S) {
+      stage = 0;
+      phase ^= 1u;
+    }
+    if (!(d.flags & 1)) continue;
+
+    // ---- end of a unit: row sums to the unit's slot or straight to Y ----
+    const int u = d.unit;
+    const int r = u / p.Ub;
+#pragma unroll
+    for (int j = 0; j < C::JS; ++j)
+#pragma unroll
+      for (int b = 0; b < BP; ++b) {
+        float v = acc[j][b];
+#pragma unroll
+        for (int o = 1; o < C::CPR; o <<= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+        acc[j][b] = v;
+      }
+    const int64_t row0 = (int64_t)r * B1;
+    if (p.Ub == 1) {
+      if (cp == 0) {
+#pragma unroll
+        for (int j = 0; j < C::JS; ++j)
+#pragma unroll
+          for (int b = 0; b < BP; ++b)
+            if (b < p.batch) store_out(p, row0 + wrow + j * C::RPS + rs, b, acc[j][b]);
+      }
+    } else {
+      // Each warp owns the same 8 rows in every unit, so the rows of a band
+      // are complete once all Ub units of the band passed through this warp
+      // slot: a ticket per (band, warp) finds the last one, which sums the
+      // band's slots for its rows in unit order.  No warp waits for another.
+      if (cp == 0) {
+        float *slot = p.partials + (int64_t)u * BP * B1;
+#pragma unroll
+        for (int j = 0; j < C::JS; ++j)
+#pragma unroll
+          for (int b = 0; b < BP; ++b)
+            __stcg(slot + b * B1 + wrow + j * C::RPS + rs, acc[j][b]);
+        __threadfence();
+      }
+      __syncwarp();
+      uint32_t last = 0;
+      if (lane == 0)
+        last = atomicAdd(p.counters + (int64_t)r * C::NC + warp, 1u) == (uint32_t)(p.Ub - 1);
+      last = __shfl_sync(0xffffffffu, last, 0);
+      if (last) {
+        __threadfence();
+        const float *band = p.partials + (int64_t)r * p.Ub * BP * B1;
+        for (int i = lane; i < C::RW * BP; i += 32) {
+          const int row = wrow + i % C::RW, b = i / C::RW;
+          if (b >= p.batch) continue;
+          const float *src = band + b * B1 + row;
+          const int64_t stride = (int64_t)BP * B1;
+          float y0 = 0.f, y1 = 0.f, y2 = 0.f, y3 = 0.f;
+          int q = 0;
+          for (; q + 4 <= p.Ub; q += 4) {
+            y0 += __ldcg(src + (q + 0) * stride);
+            y1 += __ldcg(src + (q + 1) * stride);
+            y2 += __ldcg(src + (q + 2) * stride);
+            y3 += __ldcg(src + (q + 3) * stride);
+          }
+          for (; q < p.Ub; ++q) y0 += __ldcg(src + q * stride);
+          store_out(p, row0 + row, b, (y0 + y1) + (y2 + y3));
+        }
+        if (lane == 0) p.counters[(int64_t)r * C::NC + warp] = 0;  // ready for the next call
+      }
+    }
+#pragma unroll
+    for (int j = 0; j < C::JS; ++j)
+#pragma unroll
+      for (int b = 0; b < BP; ++b) acc[j][b] = 0.f;
+  }
+}
+
+// ---------------------------------------------------------------------------
 // simple kernel for other legal tilings: one warp per output row
 // ---------------------------------------------------------------------------
 template <int BP, bool STRIDED>
@@ -639,6 +1045,41 @@ void *pick_stream_kernel(int bp, Shape s) {
 #undef HYB_CASE
 }
 
+struct TmaKernel {
+  void *fn;
+  int threads;
+  size_t smem;
+  int tps;
+};
+
+template <int BP, int B1, int B2>
+TmaKernel tma_kernel_info() {
+  using C = TmaCfg<BP, B1, B2>;
+  return TmaKernel{reinterpret_cast<void *>(&hybrid_tma_kernel<BP, B1, B2>), C::kThreads,
+                   C::kSmem, C::TPS};
+}
+
+bool pick_tma_kernel(int bp, Shape s, TmaKernel *out) {
+#define HYB_TCASE(BP_)                                                         \
+  case BP_:                                                                    \
+    switch (s) {                                                               \
+      case kS128x128: *out = tma_kernel_info<BP_, 128, 128>(); return true;    \
+      case kS128x64: *out = tma_kernel_info<BP_, 128, 64>(); return true;      \
+      case kS64x64: *out = tma_kernel_info<BP_, 64, 64>(); return true;        \
+      case kS64x128: *out = tma_kernel_info<BP_, 64, 128>(); return true;      \
+      default: return false;                                                   \
+    }
+  switch (bp) {
+    HYB_TCASE(1)
+    HYB_TCASE(2)
+    HYB_TCASE(4)
+    HYB_TCASE(8)
+    HYB_TCASE(16)
+    default: return false;
+  }
+#undef HYB_TCASE
+}
+
 template <bool STRIDED>
 void *pick_rowwarp_kernel(int bp) {
   switch (bp) {
@@ -672,7 +1113,7 @@ void *pick_lowrank_apply(int bp) {
 
 // Resident CTAs per SM of a kernel instance (cached; the answer only depends
 // on the instance and the device).
-int blocks_per_sm(void *fn, size_t dyn_smem) {
+int blocks_per_sm(void *fn, size_t dyn_smem, int threads = kThreads) {
   static std::mutex mu;
   struct Entry {
     void *fn;
@@ -691,8 +1132,11 @@ int blocks_per_sm(void *fn, size_t dyn_smem) {
     if (cache[i].fn == fn && cache[i].dev == dev && cache[i].smem == bucket)
       return cache[i].blocks;
   int nb = 0;
-  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&nb, fn, kThreads, bucket) !=
-      cudaSuccess)
+  if (bucket > 48 * 1024 &&
+      cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bucket) !=
+          cudaSuccess)
+    return -1;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&nb, fn, threads, bucket) != cudaSuccess)
     return -1;
   if (used < 256) cache[used++] = Entry{fn, dev, bucket, nb};
   return nb;
@@ -700,6 +1144,10 @@ int blocks_per_sm(void *fn, size_t dyn_smem) {
 
 // Work split and workspace layout of one product call.
 struct Plan {
+  bool tma;        // TMA-ring kernel (packed hybrid, tuned tile shapes)
+  TmaKernel tk;
+  int NU, Ub, UT;  // work units
+  size_t off_sched;
   bool stream;     // tuned kernel (else one warp per row)
   int bp;          // padded batch
   int b1, b2;
@@ -721,14 +1169,29 @@ int make_plan(int64_t n, int64_t k, int b1, int b2, int64_t total_bytes,
   P.R = (int)(n / b1);
   P.total = total_bytes;
   const Shape s = shape_of(b1, b2);
-  P.stream = s != kGeneric && P.R <= 8192;
   int sms = 0;
   int rc = device_sm_count(&sms);
   if (rc != HYB_OK) return rc;
-  P.dyn_smem = P.stream ? (size_t)2 * P.R * sizeof(int) : 0;
-  if (P.stream) {
-    void *fn = strided ? pick_stream_kernel<true>(P.bp, s)
-                       : pick_stream_kernel<false>(P.bp, s);
+  P.tma = !strided && pick_tma_kernel(P.bp, s, &P.tk);
+  P.stream = !P.tma && s != kGeneric && P.R <= 8192;
+  P.dyn_smem = P.tma ? P.tk.smem : (P.stream ? (size_t)2 * P.R * sizeof(int) : 0);
+  if (P.tma) {
+    const int nb = blocks_per_sm(P.tk.fn, P.tk.smem, P.tk.threads);
+    if (nb <= 0) return HYB_ERR_CUDA;
+    P.G = sms;  // one CTA per SM (the ring takes most of shared memory)
+    const int64_t tpr = k / b2;
+    const int64_t T = (int64_t)P.R * tpr;
+    // about six units per CTA, at most 31 tiles (one producer lane per tile
+    // offset) and never past a band
+    int64_t ut = (T + 6LL * P.G - 1) / (6LL * P.G);
+    ut = std::max<int64_t>(ut, P.tk.tps);
+    ut = (ut + P.tk.tps - 1) / P.tk.tps * P.tk.tps;
+    ut = std::min<int64_t>(ut, std::min<int64_t>(31, tpr));
+    P.UT = (int)std::max<int64_t>(1, ut);
+    P.Ub = (int)((tpr + P.UT - 1) / P.UT);
+    P.NU = P.R * P.Ub;
+  } else if (P.stream) {
+    void *fn = pick_stream_kernel<true>(P.bp, s);
     if (P.dyn_smem > 48 * 1024) {
       if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                (int)P.dyn_smem) != cudaSuccess)
@@ -746,8 +1209,11 @@ int make_plan(int64_t n, int64_t k, int b1, int b2, int64_t total_bytes,
   }
   P.lr_ctas = rank > 0 ? (int)std::max<int64_t>(1, std::min<int64_t>(sms, k / 64)) : 0;
   size_t off = kHeaderBytes;
+  P.off_sched = off;
+  if (P.tma) off = align_up(off + 2 * sizeof(uint32_t), 256);
   P.off_counters = off;
-  if (P.stream) off = align_up(off + (size_t)P.R * sizeof(uint32_t), 256);
+  if (P.tma) off = align_up(off + (size_t)P.R * (b1 / 8) * sizeof(uint32_t), 256);
+  else if (P.stream) off = align_up(off + (size_t)P.R * sizeof(uint32_t), 256);
   P.off_lr_t = off;
   off = align_up(off + (size_t)P.bp * (rank > 0 ? rank : 0) * sizeof(float), 256);
   P.off_lr_part = off;
@@ -755,7 +1221,8 @@ int make_plan(int64_t n, int64_t k, int b1, int b2, int64_t total_bytes,
   P.off_lr_counter = off;
   off = align_up(off + sizeof(uint32_t), 256);
   P.off_partials = off;
-  if (P.stream) off += (size_t)(P.G + P.R) * b1 * P.bp * sizeof(float);
+  if (P.tma) off += (size_t)P.NU * b1 * P.bp * sizeof(float);
+  else if (P.stream) off += (size_t)(P.G + P.R) * b1 * P.bp * sizeof(float);
   P.bytes = align_up(off, 256);
   *pl = P;
   return HYB_OK;
@@ -815,10 +1282,18 @@ int run_product(Params prm, int b1, int b2, int batch, const hyb_lowrank *lr,
     rc = launch_lowrank_t(P, lr, prm.k, prm.X, prm.ldx, batch, w, s);
     if (rc != HYB_OK) return rc;
   }
+  prm.NU = P.NU;
+  prm.Ub = P.Ub;
+  prm.UT = P.UT;
+  prm.sched = reinterpret_cast<uint32_t *>(w + P.off_sched);
+  prm.status = reinterpret_cast<uint32_t *>(w);
   void *args[] = {&prm};
-  if (P.stream) {
-    void *fn = strided ? pick_stream_kernel<true>(P.bp, shape_of(b1, b2))
-                       : pick_stream_kernel<false>(P.bp, shape_of(b1, b2));
+  if (P.tma) {
+    if (cudaLaunchKernel(P.tk.fn, dim3(P.G), dim3(P.tk.threads), args, P.tk.smem, s) !=
+        cudaSuccess)
+      return HYB_ERR_CUDA;
+  } else if (P.stream) {
+    void *fn = pick_stream_kernel<true>(P.bp, shape_of(b1, b2));
     if (cudaLaunchKernel(fn, dim3(P.G), dim3(kThreads), args, P.dyn_smem, s) !=
         cudaSuccess)
       return HYB_ERR_CUDA;
