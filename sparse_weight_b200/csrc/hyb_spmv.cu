@@ -67,9 +67,6 @@ struct Params {
   int64_t total;  // packed bytes of the whole matrix
   float *partials;
   uint32_t *counters;
-  // work units of the TMA kernel: runs of UT tiles inside one band, Ub per band
-  int NU, Ub, UT;
-  uint32_t *sched;   // [0] next unit, [1] CTAs done
   uint32_t *status;  // workspace status word
 };
 
@@ -437,20 +434,26 @@ __global__ void __launch_bounds__(kThreads, (Cfg<BP, B1, B2, STRIDED>::kMinBlock
 // the TMA-ring kernel for packed hybrid matrices
 // ---------------------------------------------------------------------------
 //
-// One CTA per SM.  A producer warp copies whole tiles (values, masks and the
-// matching slice of X) from HBM into a ring of shared-memory stages with 1-D
-// bulk copies (cp.async.bulk, completion counted on an mbarrier), so the bytes
-// in flight are set by the ring size, not by registers.  B1/8 consumer warps
-// compute from shared memory.  Work is handed out in units -- runs of UT
-// consecutive tiles inside one tile-row band -- from an atomic counter, so a
-// slow SM simply takes fewer units.  A unit's row sums go to its own fp32 slot;
-// the last unit of a band to finish (atomic ticket) sums the band's slots in
-// unit order, so the result does not depend on which CTA ran which unit.
+// One CTA per SM.  CTA c owns the tiles whose packed byte offset falls in
+// [c, c+1) * total / G -- a contiguous piece of the packed stream, found by
+// one round of parallel search over the tile offsets at start-up.  A producer
+// warp copies that piece tile by tile (values, masks and the matching slice of
+// X) from HBM into a ring of shared-memory stages with 1-D bulk copies
+// (cp.async.bulk; completion counted on an mbarrier), so the bytes in flight
+// are set by the ring, not by registers.  B1/8 consumer warps, 8 tile rows
+// each, compute from shared memory and keep fp32 row sums in registers until
+// their piece of a tile-row band ends.
+//
+// A band split between CTAs is summed through fp32 slots: CTA c writes its
+// share of band r to slot c + r, and a ticket per (band, warp) finds the last
+// contribution, whose warp sums the band's slots in CTA order (deterministic;
+// nothing spins, and a ticket's answer is only read after the next piece of
+// work, so the atomic's round trip is hidden).
 //
 // Products use the mixed-precision FMA of sm_100 (bf16 x bf16 + fp32 -> fp32,
-// the product is exact) straight on packed bf16 pairs, and PRMT picks the two
-// x values of a 2:4 group from the 4-bit mask through a 16-entry selector
-// table ("SparseDecoding", authors' abstract: bitmask-indexed N:M SpMV).
+// exact product) straight on packed bf16 pairs, and PRMT picks the two x
+// values of a 2:4 group from its 4-bit mask through a 16-entry selector table
+// ("SparseDecoding", authors' abstract: bitmask-indexed N:M SpMV).
 
 constexpr uint32_t kStatusTimeout = 4u;  // a pipeline wait ran out
 constexpr uint32_t kWaitLimit = 1u << 22;
@@ -482,11 +485,17 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
   return ok != 0;
 }
 // Every wait is bounded: on expiry the caller records kStatusTimeout and
-// leaves the pipeline instead of spinning for ever.
+// leaves the pipeline instead of waiting for ever.
 __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity) {
   for (uint32_t i = 0; i < kWaitLimit; ++i)
     if (mbar_try_wait(bar, parity)) return true;
   return false;
+}
+__device__ __forceinline__ uint32_t atom_add_acq_rel(uint32_t *addr, uint32_t v) {
+  uint32_t old;
+  asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], %2;" : "=r"(old) : "l"(addr), "r"(v)
+               : "memory");
+  return old;
 }
 __device__ __forceinline__ void bulk_g2s(void *dst, const void *src, uint32_t bytes,
                                          uint64_t *bar) {
@@ -507,31 +516,34 @@ __device__ __forceinline__ void fma_bf16x2(float &acc, uint32_t w, uint32_t x) {
 
 template <int BP, int B1, int B2>
 struct TmaCfg {
-  static constexpr int NC = B1 / 8;                 // consumer warps, 8 rows each
-  static constexpr int RW = 8;                      // rows per consumer warp per tile
+  // rows per consumer warp: 8, or 16 for wide batches so that the 17-warp
+  // register budget (96 per thread) is not exceeded by the accumulators
+  static constexpr int RW = BP >= 8 ? 16 : 8;
+  static constexpr int NC = B1 / RW;                // consumer warps
   static constexpr int CPR = B2 / 16;               // lanes per row, 16 columns each
   static constexpr int RPS = 32 / CPR;              // rows per warp step
   static constexpr int JS = RW / RPS;               // steps per warp per tile
   static constexpr int XB = BP < 4 ? BP : 4;        // batch columns per pass
   static constexpr int TPS = (16384 / (B1 * B2)) > 0 ? 16384 / (B1 * B2) : 1;  // tiles per stage
+  static constexpr int WIN = 28;                    // tiles per producer offset window
   static constexpr int kValsBytes = 2 * B1 * B2 * TPS;        // 32 KB
   static constexpr int kMetaBytes = B1 * B2 / 8 * TPS;        // 2 KB
   static constexpr int kXRow = 2 * B2 * TPS;                  // bytes of one X row slice
   static constexpr int kStageBytes = kValsBytes + kMetaBytes + BP * kXRow;
   static constexpr int kStages =
-      (220 * 1024 / kStageBytes) < 6 ? (220 * 1024 / kStageBytes) : 6;
+      (200 * 1024 / kStageBytes) < 6 ? (200 * 1024 / kStageBytes) : 6;
   static constexpr int kThreads = (NC + 1) * 32;
   static constexpr size_t kSmem = (size_t)kStages * kStageBytes + 1024;
   static_assert(RPS * CPR == 32 && JS * RPS == RW && JS >= 1, "tile shape");
   static_assert(kStages >= 3, "ring too short");
+  static_assert(WIN % TPS == 0 && WIN < 32, "offset window");
 };
 
 struct StageDesc {
-  int64_t t0;        // first tile of the stage
-  int32_t unit;      // unit the tiles belong to
-  uint16_t ntiles;   // tiles in the stage (<= TPS)
-  uint8_t sparse;    // bit i: tile i is 2:4
-  uint8_t flags;     // 1: last stage of its unit, 2: end of work
+  int64_t t0;       // first tile of the stage
+  uint16_t ntiles;  // tiles in the stage (<= TPS, never across a band)
+  uint8_t sparse;   // bit i: tile i is 2:4
+  uint8_t flags;    // 1: last stage of this CTA's piece of a band, 2: end of work
 };
 
 template <int BP, int B1, int B2>
@@ -544,19 +556,27 @@ __global__ void __launch_bounds__(TmaCfg<BP, B1, B2>::kThreads, 1)
   __shared__ __align__(8) uint64_t empty_bar[S];
   __shared__ StageDesc desc[S];
   __shared__ uint32_t sel_lut[16];
+  __shared__ uint32_t s_cnt[2];
+  __shared__ int64_t s_range[2];
+  __shared__ float s_rows[C::NC][C::RW * BP];  // a warp's row sums, [b][row]
 
   const int tid = threadIdx.x;
   const int warp = tid >> 5, lane = tid & 31;
+  const int c = blockIdx.x;
+  const int G = p.G;
+  const int tpr = (int)p.tpr;
   if (tid == 0) {
     for (int s = 0; s < S; ++s) {
       mbar_init(&full_bar[s], 1);
       mbar_init(&empty_bar[s], C::NC);
     }
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    s_cnt[0] = 0;
+    s_cnt[1] = 0;
   }
   if (tid < 16) {
-    // PRMT selector that moves bf16 x[p0] to the low and x[p1] to the high
-    // half, p0 < p1 the set bits of the mask (x0x1 in bytes 0-3, x2x3 in 4-7)
+    // PRMT selector moving bf16 x[p0] to the low and x[p1] to the high half,
+    // p0 < p1 the set bits of the mask (x0x1 in bytes 0-3, x2x3 in 4-7)
     const uint32_t m = tid;
     uint32_t p0 = 0, p1 = 0;
     if (m) {
@@ -567,96 +587,138 @@ __global__ void __launch_bounds__(TmaCfg<BP, B1, B2>::kThreads, 1)
   }
   __syncthreads();
 
+  // ---- this CTA's tiles [t0, t1): tiles whose packed offset P(t) satisfies
+  // c*total <= P(t)*G < (c+1)*total.  Round 1 brackets both ends between
+  // band starts, round 2 counts inside the bracketing band. ----
+  {
+    const int64_t tgtA = (int64_t)c * p.total, tgtB = (int64_t)(c + 1) * p.total;
+    uint32_t ca = 0, cb = 0;
+    for (int i = tid; i <= p.R; i += blockDim.x) {
+      const int64_t t = (int64_t)i * tpr;
+      const int64_t P = 2 * __ldg(p.val_off + t) + __ldg(p.meta_off + t);
+      ca += P * G < tgtA;
+      cb += P * G < tgtB;
+    }
+    ca = __reduce_add_sync(0xffffffffu, ca);
+    cb = __reduce_add_sync(0xffffffffu, cb);
+    if (lane == 0) {
+      atomicAdd(&s_cnt[0], ca);
+      atomicAdd(&s_cnt[1], cb);
+    }
+    __syncthreads();
+    const uint32_t bA = s_cnt[0], bB = s_cnt[1];  // band starts below each target
+    __syncthreads();
+    if (tid == 0) {
+      s_cnt[0] = 0;
+      s_cnt[1] = 0;
+    }
+    __syncthreads();
+    ca = 0;
+    cb = 0;
+    const int64_t baseA = bA > 0 ? (int64_t)(bA - 1) * tpr : 0;
+    const int64_t baseB = bB > 0 ? (int64_t)(bB - 1) * tpr : 0;
+    for (int i = tid; i < tpr; i += blockDim.x) {
+      if (bA > 0) {
+        const int64_t t = baseA + i;
+        ca += (2 * __ldg(p.val_off + t) + __ldg(p.meta_off + t)) * G < tgtA;
+      }
+      if (bB > 0) {
+        const int64_t t = baseB + i;
+        cb += (2 * __ldg(p.val_off + t) + __ldg(p.meta_off + t)) * G < tgtB;
+      }
+    }
+    ca = __reduce_add_sync(0xffffffffu, ca);
+    cb = __reduce_add_sync(0xffffffffu, cb);
+    if (lane == 0) {
+      atomicAdd(&s_cnt[0], ca);
+      atomicAdd(&s_cnt[1], cb);
+    }
+    __syncthreads();
+    if (tid == 0) {
+      s_range[0] = bA > 0 ? baseA + s_cnt[0] : 0;
+      s_range[1] = (c == G - 1) ? p.T : (bB > 0 ? baseB + s_cnt[1] : 0);
+    }
+    __syncthreads();
+  }
+  const int64_t t0 = s_range[0];
+  const int64_t t1 = s_range[1];
+
   if (warp == C::NC) {
     // ------------------------------ producer ------------------------------
+    // Stages follow a fixed grid: inside a band, stage boundaries sit every
+    // TPS tiles from the band start, so stage g of the whole matrix covers
+    // tiles [band*tpr + (g%spb)*TPS, ...) with spb stages per band.  Lane i
+    // works out stage g0+i of this CTA's piece (tile range, packed offsets,
+    // 2:4 bits) while the previous 32 stages are issued one by one.
+    const int spb = (tpr + C::TPS - 1) / C::TPS;
+    const int64_t g_first = (t0 / tpr) * spb + (t0 % tpr) / C::TPS;
+    const int64_t g_last = t1 > t0 ? ((t1 - 1) / tpr) * spb + ((t1 - 1) % tpr) / C::TPS : g_first - 1;
+    struct StageInfo {
+      int64_t ts, te;         // tiles [ts, te)
+      int64_t vs, ve, ms, me; // packed value / meta offsets
+      uint32_t sp, flags;
+      const uint16_t *xsrc;   // X slice (row 0)
+    };
+    auto stage_info = [&](int64_t g) -> StageInfo {
+      StageInfo o{};
+      if (g > g_last) return o;
+      const int64_t band = g / spb, loc = g - band * spb;
+      const int64_t bs = band * tpr, be = bs + tpr;
+      o.ts = max(t0, bs + loc * C::TPS);
+      o.te = min(min(t1, be), bs + (loc + 1) * C::TPS);
+      o.vs = __ldg(p.val_off + o.ts);
+      o.ve = __ldg(p.val_off + o.te);
+      o.ms = __ldg(p.meta_off + o.ts);
+      o.me = __ldg(p.meta_off + o.te);
+      for (int64_t q = o.ts; q < o.te; ++q) o.sp |= (uint32_t)(__ldg(p.map + q) == 1) << (q - o.ts);
+      o.flags = (o.te == be || o.te == t1) ? 1u : 0u;
+      o.xsrc = p.X + (o.ts - bs) * B2;
+      return o;
+    };
     int stage = 0;
     uint32_t phase = 0;
     bool ok = true;
-    auto grab = [&]() -> int {
-      int u = 0;
-      if (lane == 0) u = (int)atomicAdd(p.sched, 1u);
-      return __shfl_sync(0xffffffffu, u, 0);
-    };
-    // per-unit offsets, one tile per lane: val_off / meta_off / map of tile ta+lane
-    struct UnitOff {
-      int64_t vo, mo;
-      uint32_t sp;
-      int64_t ta;
-      int nt;
-    };
-    auto unit_off = [&](int u) -> UnitOff {
-      UnitOff o;
-      const int64_t r = u / p.Ub, q = u - r * p.Ub;
-      o.ta = r * p.tpr + q * p.UT;
-      const int64_t tb = min(o.ta + p.UT, (r + 1) * p.tpr);
-      o.nt = (int)(tb - o.ta);
-      o.vo = 0;
-      o.mo = 0;
-      o.sp = 0;
-      if (lane <= o.nt) {
-        o.vo = __ldg(p.val_off + o.ta + lane);
-        o.mo = __ldg(p.meta_off + o.ta + lane);
-      }
-      if (lane < o.nt) o.sp = __ldg(p.map + o.ta + lane) == 1;
-      return o;
-    };
     uint32_t armed = 0, armed_parity = 0;  // per stage: copies issued / phase parity
-    int u = grab();
-    UnitOff cur{};
-    if (u < p.NU) cur = unit_off(u);
-    int un = grab();
-    while (ok && u < p.NU) {
-      UnitOff nxt{};
-      if (un < p.NU) nxt = unit_off(un);  // loads in flight while this unit issues
-      // the grab after next: its result is only read once this unit is issued
-      uint32_t unn_raw = 0;
-      if (un < p.NU && lane == 0) unn_raw = atomicAdd(p.sched, 1u);
-      const uint32_t spmask = __ballot_sync(0xffffffffu, cur.sp != 0);
-      for (int i = 0; i < cur.nt; i += C::TPS) {
-        const int nt = min(C::TPS, cur.nt - i);
-        const int64_t v0 = __shfl_sync(0xffffffffu, cur.vo, i);
-        const int64_t v1 = __shfl_sync(0xffffffffu, cur.vo, i + nt);
-        const int64_t m0 = __shfl_sync(0xffffffffu, cur.mo, i);
-        const int64_t m1 = __shfl_sync(0xffffffffu, cur.mo, i + nt);
-        if (lane == 0) {
+    StageInfo cur = stage_info(g_first + lane);
+    for (int64_t gw = g_first; ok && gw <= g_last; gw += 32) {
+      const StageInfo nxt = stage_info(gw + 32 + lane);  // in flight while issuing
+      const int nst = (int)min((int64_t)32, g_last - gw + 1);
+      for (int k = 0; k < nst; ++k) {
+        if (lane == k) {
           if (!mbar_wait(&empty_bar[stage], phase ^ 1u)) {
             ok = false;
           } else {
             uint8_t *st = smem + (size_t)stage * C::kStageBytes;
-            const uint32_t vbytes = (uint32_t)(2 * (v1 - v0));
-            const uint32_t mbytes = (uint32_t)(m1 - m0);
-            const int64_t t = cur.ta + i;
-            const int64_t tc = t % p.tpr;
+            const uint32_t vbytes = (uint32_t)(2 * (cur.ve - cur.vs));
+            const uint32_t mbytes = (uint32_t)(cur.me - cur.ms);
+            const int nt = (int)(cur.te - cur.ts);
             const uint32_t xrow = (uint32_t)(2 * B2 * nt);
             StageDesc d;
-            d.t0 = t;
-            d.unit = u;
+            d.t0 = cur.ts;
             d.ntiles = (uint16_t)nt;
-            d.sparse = (uint8_t)((spmask >> i) & ((1u << nt) - 1u));
-            d.flags = (i + nt >= cur.nt) ? 1 : 0;
+            d.sparse = (uint8_t)cur.sp;
+            d.flags = (uint8_t)cur.flags;
             desc[stage] = d;
             armed |= 1u << stage;
             armed_parity = (armed_parity & ~(1u << stage)) | (phase << stage);
             mbar_arrive_expect_tx(&full_bar[stage], vbytes + mbytes + xrow * p.batch);
-            bulk_g2s(st, p.vals + 2 * v0, vbytes, &full_bar[stage]);
-            if (mbytes) bulk_g2s(st + C::kValsBytes, p.meta + m0, mbytes, &full_bar[stage]);
+            bulk_g2s(st, p.vals + 2 * cur.vs, vbytes, &full_bar[stage]);
+            if (mbytes) bulk_g2s(st + C::kValsBytes, p.meta + cur.ms, mbytes, &full_bar[stage]);
             for (int b = 0; b < p.batch; ++b)
               bulk_g2s(st + C::kValsBytes + C::kMetaBytes + b * C::kXRow,
-                       p.X + (int64_t)b * p.ldx + tc * B2, xrow, &full_bar[stage]);
+                       cur.xsrc + (int64_t)b * p.ldx, xrow, &full_bar[stage]);
           }
         }
-        ok = __shfl_sync(0xffffffffu, ok, 0);
-        if (!ok) break;
+        // every lane keeps the ring position
         if (++stage == S) {
           stage = 0;
           phase ^= 1u;
         }
       }
-      const int unn = (un < p.NU) ? (int)__shfl_sync(0xffffffffu, unn_raw, 0) : un;
-      u = un;
-      un = unn;
+      ok = __all_sync(0xffffffffu, ok);
       cur = nxt;
     }
+    // lanes kept identical ring positions; lane 0 closes the ring
     if (lane == 0) {
       if (ok && mbar_wait(&empty_bar[stage], phase ^ 1u)) {
         StageDesc d{};
@@ -666,19 +728,14 @@ __global__ void __launch_bounds__(TmaCfg<BP, B1, B2>::kThreads, 1)
       } else {
         ok = false;
       }
-      if (!ok) {
-        atomicOr(p.status, kStatusTimeout);
-        // let every copy already issued land before the CTA's shared memory
-        // goes away (bounded, like every other wait)
-        for (int s = 0; s < S; ++s)
-          if (armed >> s & 1u) mbar_wait(&full_bar[s], armed_parity >> s & 1u);
-      }
-      // the last CTA to finish resets the unit counter for the next call
-      __threadfence();
-      if (atomicAdd(p.sched + 1, 1u) == (uint32_t)gridDim.x - 1) {
-        p.sched[0] = 0;
-        p.sched[1] = 0;
-      }
+    }
+    if (!__all_sync(0xffffffffu, ok)) {
+      if (lane == 0) atomicOr(p.status, kStatusTimeout);
+      // let every copy already issued land before the CTA's shared memory
+      // goes away (bounded, like every other wait); each lane drains the
+      // stages it armed
+      for (int s2 = 0; s2 < S; ++s2)
+        if (armed >> s2 & 1u) mbar_wait(&full_bar[s2], armed_parity >> s2 & 1u);
     }
     return;
   }
@@ -692,6 +749,41 @@ __global__ void __launch_bounds__(TmaCfg<BP, B1, B2>::kThreads, 1)
   for (int j = 0; j < C::JS; ++j)
 #pragma unroll
     for (int b = 0; b < BP; ++b) acc[j][b] = 0.f;
+
+  // Deferred ticket of the last band piece this warp sent to a slot, with the
+  // packed offsets of that band's first and last tile (to name its owners).
+  int pend_band = -1;
+  uint32_t pend_ticket = 0;
+  int64_t pend_pa = 0, pend_pb = 0;
+  auto owner_of_p = [&](int64_t P) -> int {
+    const int64_t o = (P * G) / p.total;
+    return (int)(o < G - 1 ? o : G - 1);
+  };
+  auto finish_band = [&]() {
+    const int rb = pend_band;
+    pend_band = -1;
+    const uint32_t ticket = __shfl_sync(0xffffffffu, pend_ticket, 0);
+    const int oA = owner_of_p(__shfl_sync(0xffffffffu, pend_pa, 0));
+    const int oB = owner_of_p(__shfl_sync(0xffffffffu, pend_pb, 0));
+    if (ticket != (uint32_t)(oB - oA)) return;
+    __syncwarp();
+    // this warp was the last contributor: sum slots oA..oB (CTA order) for
+    // its 8 rows; lanes = (output, phase), phases combined in a fixed pattern
+    constexpr int NOUT = C::RW * BP;
+    constexpr int NPH = NOUT >= 32 ? 1 : 32 / NOUT;
+    for (int base = 0; base < NOUT; base += 32 / NPH) {
+      const int o = base + lane / NPH, ph = lane % NPH;
+      const int row = wrow + o % C::RW, b = o / C::RW;
+      float y = 0.f;
+      if (o < NOUT && b < p.batch)
+        for (int cc = oA + ph; cc <= oB; cc += NPH)
+          y += __ldcg(p.partials + ((int64_t)(cc + rb) * BP + b) * B1 + row);
+#pragma unroll
+      for (int m = 1; m < NPH; m <<= 1) y += __shfl_xor_sync(0xffffffffu, y, m);
+      if (ph == 0 && o < NOUT && b < p.batch) store_out(p, (int64_t)rb * B1 + row, b, y);
+    }
+    if (lane == 0) p.counters[(int64_t)rb * C::NC + warp] = 0;  // ready for the next call
+  };
 
   int stage = 0;
   uint32_t phase = 0;
@@ -766,9 +858,11 @@ __global__ void __launch_bounds__(TmaCfg<BP, B1, B2>::kThreads, 1)
     }
     if (!(d.flags & 1)) continue;
 
-    // ---- end of a unit: row sums to the unit's slot or straight to Y ----
-    const int u = d.unit;
-    const int r = u / p.Ub;
+    // ---- end of this CTA's piece of band r: row sums to Y or to a slot ----
+    // Reduce over the lanes of each row, park the 8 x BP sums of this warp in
+    // shared memory, then let all 32 lanes store them (o = b * RW + row).
+    const int r = (int)(d.t0 / tpr);
+    float *rows_s = s_rows[warp];
 #pragma unroll
     for (int j = 0; j < C::JS; ++j)
 #pragma unroll
@@ -776,63 +870,37 @@ __global__ void __launch_bounds__(TmaCfg<BP, B1, B2>::kThreads, 1)
         float v = acc[j][b];
 #pragma unroll
         for (int o = 1; o < C::CPR; o <<= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-        acc[j][b] = v;
+        if (cp == 0) rows_s[b * C::RW + j * C::RPS + rs] = v;
+        acc[j][b] = 0.f;
       }
-    const int64_t row0 = (int64_t)r * B1;
-    if (p.Ub == 1) {
-      if (cp == 0) {
-#pragma unroll
-        for (int j = 0; j < C::JS; ++j)
-#pragma unroll
-          for (int b = 0; b < BP; ++b)
-            if (b < p.batch) store_out(p, row0 + wrow + j * C::RPS + rs, b, acc[j][b]);
+    __syncwarp();
+    const bool whole = t0 <= (int64_t)r * tpr && t1 >= (int64_t)(r + 1) * tpr;
+    if (whole) {
+      for (int o = lane; o < C::RW * BP; o += 32) {
+        const int row = o % C::RW, b = o / C::RW;
+        if (b < p.batch) store_out(p, (int64_t)r * B1 + wrow + row, b, rows_s[o]);
       }
     } else {
-      // Each warp owns the same 8 rows in every unit, so the rows of a band
-      // are complete once all Ub units of the band passed through this warp
-      // slot: a ticket per (band, warp) finds the last one, which sums the
-      // band's slots for its rows in unit order.  No warp waits for another.
-      if (cp == 0) {
-        float *slot = p.partials + (int64_t)u * BP * B1;
-#pragma unroll
-        for (int j = 0; j < C::JS; ++j)
-#pragma unroll
-          for (int b = 0; b < BP; ++b)
-            __stcg(slot + b * B1 + wrow + j * C::RPS + rs, acc[j][b]);
-        __threadfence();
+      if (pend_band >= 0) finish_band();
+      float *slot = p.partials + (int64_t)(c + r) * BP * B1;
+      for (int o = lane; o < C::RW * BP; o += 32) {
+        const int row = o % C::RW, b = o / C::RW;
+        __stcg(slot + b * B1 + wrow + row, rows_s[o]);
       }
       __syncwarp();
-      uint32_t last = 0;
-      if (lane == 0)
-        last = atomicAdd(p.counters + (int64_t)r * C::NC + warp, 1u) == (uint32_t)(p.Ub - 1);
-      last = __shfl_sync(0xffffffffu, last, 0);
-      if (last) {
-        __threadfence();
-        const float *band = p.partials + (int64_t)r * p.Ub * BP * B1;
-        for (int i = lane; i < C::RW * BP; i += 32) {
-          const int row = wrow + i % C::RW, b = i / C::RW;
-          if (b >= p.batch) continue;
-          const float *src = band + b * B1 + row;
-          const int64_t stride = (int64_t)BP * B1;
-          float y0 = 0.f, y1 = 0.f, y2 = 0.f, y3 = 0.f;
-          int q = 0;
-          for (; q + 4 <= p.Ub; q += 4) {
-            y0 += __ldcg(src + (q + 0) * stride);
-            y1 += __ldcg(src + (q + 1) * stride);
-            y2 += __ldcg(src + (q + 2) * stride);
-            y3 += __ldcg(src + (q + 3) * stride);
-          }
-          for (; q < p.Ub; ++q) y0 += __ldcg(src + q * stride);
-          store_out(p, row0 + row, b, (y0 + y1) + (y2 + y3));
-        }
-        if (lane == 0) p.counters[(int64_t)r * C::NC + warp] = 0;  // ready for the next call
+      if (lane == 0) {
+        // release: the slot rows above (written by this warp, ordered by the
+        // warp barrier) are visible before the ticket moves
+        pend_ticket = atom_add_acq_rel(p.counters + (int64_t)r * C::NC + warp, 1u);
+        const int64_t ta = (int64_t)r * tpr, tb = ta + tpr - 1;
+        pend_pa = 2 * __ldg(p.val_off + ta) + __ldg(p.meta_off + ta);
+        pend_pb = 2 * __ldg(p.val_off + tb) + __ldg(p.meta_off + tb);
       }
+      pend_band = r;
     }
-#pragma unroll
-    for (int j = 0; j < C::JS; ++j)
-#pragma unroll
-      for (int b = 0; b < BP; ++b) acc[j][b] = 0.f;
+    __syncwarp();
   }
+  if (pend_band >= 0) finish_band();
 }
 
 // ---------------------------------------------------------------------------
@@ -1146,8 +1214,6 @@ int blocks_per_sm(void *fn, size_t dyn_smem, int threads = kThreads) {
 struct Plan {
   bool tma;        // TMA-ring kernel (packed hybrid, tuned tile shapes)
   TmaKernel tk;
-  int NU, Ub, UT;  // work units
-  size_t off_sched;
   bool stream;     // tuned kernel (else one warp per row)
   int bp;          // padded batch
   int b1, b2;
@@ -1178,18 +1244,10 @@ int make_plan(int64_t n, int64_t k, int b1, int b2, int64_t total_bytes,
   if (P.tma) {
     const int nb = blocks_per_sm(P.tk.fn, P.tk.smem, P.tk.threads);
     if (nb <= 0) return HYB_ERR_CUDA;
-    P.G = sms;  // one CTA per SM (the ring takes most of shared memory)
-    const int64_t tpr = k / b2;
-    const int64_t T = (int64_t)P.R * tpr;
-    // about six units per CTA, at most 31 tiles (one producer lane per tile
-    // offset) and never past a band
-    int64_t ut = (T + 6LL * P.G - 1) / (6LL * P.G);
-    ut = std::max<int64_t>(ut, P.tk.tps);
-    ut = (ut + P.tk.tps - 1) / P.tk.tps * P.tk.tps;
-    ut = std::min<int64_t>(ut, std::min<int64_t>(31, tpr));
-    P.UT = (int)std::max<int64_t>(1, ut);
-    P.Ub = (int)((tpr + P.UT - 1) / P.UT);
-    P.NU = P.R * P.Ub;
+    // one CTA per SM (the ring takes most of shared memory); every CTA must
+    // own at least one tile: total / G >= the largest tile
+    const int64_t gcap = std::max<int64_t>(1, total_bytes / (2LL * b1 * b2));
+    P.G = (int)std::min<int64_t>(sms, gcap);
   } else if (P.stream) {
     void *fn = pick_stream_kernel<true>(P.bp, s);
     if (P.dyn_smem > 48 * 1024) {
@@ -1209,8 +1267,6 @@ int make_plan(int64_t n, int64_t k, int b1, int b2, int64_t total_bytes,
   }
   P.lr_ctas = rank > 0 ? (int)std::max<int64_t>(1, std::min<int64_t>(sms, k / 64)) : 0;
   size_t off = kHeaderBytes;
-  P.off_sched = off;
-  if (P.tma) off = align_up(off + 2 * sizeof(uint32_t), 256);
   P.off_counters = off;
   if (P.tma) off = align_up(off + (size_t)P.R * (b1 / 8) * sizeof(uint32_t), 256);
   else if (P.stream) off = align_up(off + (size_t)P.R * sizeof(uint32_t), 256);
@@ -1221,8 +1277,7 @@ int make_plan(int64_t n, int64_t k, int b1, int b2, int64_t total_bytes,
   P.off_lr_counter = off;
   off = align_up(off + sizeof(uint32_t), 256);
   P.off_partials = off;
-  if (P.tma) off += (size_t)P.NU * b1 * P.bp * sizeof(float);
-  else if (P.stream) off += (size_t)(P.G + P.R) * b1 * P.bp * sizeof(float);
+  if (P.tma || P.stream) off += (size_t)(P.G + P.R) * b1 * P.bp * sizeof(float);
   P.bytes = align_up(off, 256);
   *pl = P;
   return HYB_OK;
@@ -1282,10 +1337,6 @@ int run_product(Params prm, int b1, int b2, int batch, const hyb_lowrank *lr,
     rc = launch_lowrank_t(P, lr, prm.k, prm.X, prm.ldx, batch, w, s);
     if (rc != HYB_OK) return rc;
   }
-  prm.NU = P.NU;
-  prm.Ub = P.Ub;
-  prm.UT = P.UT;
-  prm.sched = reinterpret_cast<uint32_t *>(w + P.off_sched);
   prm.status = reinterpret_cast<uint32_t *>(w);
   void *args[] = {&prm};
   if (P.tma) {
