@@ -101,6 +101,9 @@ typedef struct {
   const int64_t *meta_off;  /* [num_tiles + 1] */
   int64_t n_vals;           /* val_off[num_tiles], as given by hyb_packed_sizes */
   int64_t n_meta_bytes;     /* meta_off[num_tiles], as given by hyb_packed_sizes */
+  const int64_t *plan;      /* optional (may be NULL): work split made by
+                               hyb_make_plan for this matrix on this device;
+                               saves the products a search at every call */
 } hyb_matrix;
 
 /* Low-rank factors of y += U (V^T x): U is [n][rank] (row stride ldu),
@@ -137,6 +140,19 @@ HYB_API int hyb_pack(int64_t n, int64_t k, int b1, int b2, const uint16_t *W,
              int64_t ldw, const uint8_t *tile_map, uint16_t *vals,
              uint8_t *meta, int64_t *val_off, int64_t *meta_off, void *ws,
              size_t ws_bytes, hyb_stream_t stream);
+
+/* ---- work split -------------------------------------------------------- */
+
+/* Entries of a plan buffer (int64_t) for hyb_make_plan on the current device. */
+HYB_API size_t hyb_plan_entries(void);
+
+/* Write into `plan` (device, hyb_plan_entries() int64_t) the split of A's
+ * packed bytes over the streaming kernel's CTAs on the current device: CTA c
+ * takes the tiles whose packed byte offset falls in [c, c+1) * total / G.
+ * The products find the same split by searching val_off / meta_off when
+ * A->plan is NULL; a plan only saves that search.  A plan made on another
+ * device (another SM count) is detected and ignored. */
+HYB_API int hyb_make_plan(const hyb_matrix *A, int64_t *plan, hyb_stream_t stream);
 
 /* ---- products ---------------------------------------------------------- */
 

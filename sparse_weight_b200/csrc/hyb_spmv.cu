@@ -68,6 +68,7 @@ struct Params {
   float *partials;
   uint32_t *counters;
   uint32_t *status;  // workspace status word
+  const int64_t *plan;  // optional precomputed split: [G, t0(0), ..., t0(G)]
 };
 
 // ---------------------------------------------------------------------------
@@ -117,16 +118,26 @@ __device__ __forceinline__ void store_out(const Params &p, int64_t row, int b,
     const uint16_t *u = p.U + row * p.ldu;
     const float *t = p.lr_t + (int64_t)b * p.rank;
     float s = 0.f;
-    for (int j = 0; j < p.rank; j += 8) {
-      const uint4 uv = __ldg(reinterpret_cast<const uint4 *>(u + j));
-      s = fmaf(bf16_lo(uv.x), t[j + 0], s);
-      s = fmaf(bf16_hi(uv.x), t[j + 1], s);
-      s = fmaf(bf16_lo(uv.y), t[j + 2], s);
-      s = fmaf(bf16_hi(uv.y), t[j + 3], s);
-      s = fmaf(bf16_lo(uv.z), t[j + 4], s);
-      s = fmaf(bf16_hi(uv.z), t[j + 5], s);
-      s = fmaf(bf16_lo(uv.w), t[j + 6], s);
-      s = fmaf(bf16_hi(uv.w), t[j + 7], s);
+    // 64 factor entries per round: their loads are issued together
+    for (int j0 = 0; j0 < p.rank; j0 += 64) {
+      uint4 uv[8];
+#pragma unroll
+      for (int q = 0; q < 8; ++q)
+        uv[q] = j0 + 8 * q < p.rank ? __ldg(reinterpret_cast<const uint4 *>(u + j0 + 8 * q))
+                                    : make_uint4(0, 0, 0, 0);
+#pragma unroll
+      for (int q = 0; q < 8; ++q) {
+        if (j0 + 8 * q >= p.rank) break;
+        const float *tq = t + j0 + 8 * q;
+        s = fmaf(bf16_lo(uv[q].x), tq[0], s);
+        s = fmaf(bf16_hi(uv[q].x), tq[1], s);
+        s = fmaf(bf16_lo(uv[q].y), tq[2], s);
+        s = fmaf(bf16_hi(uv[q].y), tq[3], s);
+        s = fmaf(bf16_lo(uv[q].z), tq[4], s);
+        s = fmaf(bf16_hi(uv[q].z), tq[5], s);
+        s = fmaf(bf16_lo(uv[q].w), tq[6], s);
+        s = fmaf(bf16_hi(uv[q].w), tq[7], s);
+      }
     }
     y += s;
   }
@@ -532,7 +543,7 @@ struct TmaCfg {
   static constexpr int kStageBytes = kValsBytes + kMetaBytes + BP * kXRow;
   static constexpr int kStages =
       (200 * 1024 / kStageBytes) < 6 ? (200 * 1024 / kStageBytes) : 6;
-  static constexpr int kThreads = (NC + 1) * 32;
+  static constexpr int kThreads = (NC + 2) * 32;  // consumers, producer, epilogue
   static constexpr size_t kSmem = (size_t)kStages * kStageBytes + 1024;
   static_assert(RPS * CPR == 32 && JS * RPS == RW && JS >= 1, "tile shape");
   static_assert(kStages >= 3, "ring too short");
@@ -558,7 +569,11 @@ __global__ void __launch_bounds__(TmaCfg<BP, B1, B2>::kThreads, 1)
   __shared__ uint32_t sel_lut[16];
   __shared__ uint32_t s_cnt[2];
   __shared__ int64_t s_range[2];
-  __shared__ float s_rows[C::NC][C::RW * BP];  // a warp's row sums, [b][row]
+  // a CTA's piece of a band: row sums handed from the consumer warps to the
+  // epilogue warp through a 2-slot ring, [slot][warp][b * RW + row]
+  __shared__ float s_rows[2][C::NC][C::RW * BP];
+  __shared__ __align__(8) uint64_t piece_full[2];
+  __shared__ __align__(8) uint64_t piece_empty[2];
 
   const int tid = threadIdx.x;
   const int warp = tid >> 5, lane = tid & 31;
@@ -569,6 +584,10 @@ __global__ void __launch_bounds__(TmaCfg<BP, B1, B2>::kThreads, 1)
     for (int s = 0; s < S; ++s) {
       mbar_init(&full_bar[s], 1);
       mbar_init(&empty_bar[s], C::NC);
+    }
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&piece_full[s], C::NC);
+      mbar_init(&piece_empty[s], 1);
     }
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     s_cnt[0] = 0;
@@ -588,57 +607,72 @@ __global__ void __launch_bounds__(TmaCfg<BP, B1, B2>::kThreads, 1)
   __syncthreads();
 
   // ---- this CTA's tiles [t0, t1): tiles whose packed offset P(t) satisfies
-  // c*total <= P(t)*G < (c+1)*total.  Round 1 brackets both ends between
-  // band starts, round 2 counts inside the bracketing band. ----
-  {
-    const int64_t tgtA = (int64_t)c * p.total, tgtB = (int64_t)(c + 1) * p.total;
-    uint32_t ca = 0, cb = 0;
-    for (int i = tid; i <= p.R; i += blockDim.x) {
-      const int64_t t = (int64_t)i * tpr;
-      const int64_t P = 2 * __ldg(p.val_off + t) + __ldg(p.meta_off + t);
-      ca += P * G < tgtA;
-      cb += P * G < tgtB;
+  // c*total <= P(t)*G < (c+1)*total.  A plan made for this G gives them
+  // directly; otherwise round 1 brackets both ends between band starts and
+  // round 2 counts inside the bracketing band. ----
+  if (tid == 0) {
+    bool planned = false;
+    if (p.plan != nullptr && __ldg(p.plan) == (int64_t)G) {
+      s_range[0] = __ldg(p.plan + 1 + c);
+      s_range[1] = __ldg(p.plan + 2 + c);
+      planned = true;
     }
-    ca = __reduce_add_sync(0xffffffffu, ca);
-    cb = __reduce_add_sync(0xffffffffu, cb);
-    if (lane == 0) {
-      atomicAdd(&s_cnt[0], ca);
-      atomicAdd(&s_cnt[1], cb);
-    }
-    __syncthreads();
-    const uint32_t bA = s_cnt[0], bB = s_cnt[1];  // band starts below each target
-    __syncthreads();
-    if (tid == 0) {
-      s_cnt[0] = 0;
-      s_cnt[1] = 0;
-    }
-    __syncthreads();
-    ca = 0;
-    cb = 0;
-    const int64_t baseA = bA > 0 ? (int64_t)(bA - 1) * tpr : 0;
-    const int64_t baseB = bB > 0 ? (int64_t)(bB - 1) * tpr : 0;
-    for (int i = tid; i < tpr; i += blockDim.x) {
-      if (bA > 0) {
-        const int64_t t = baseA + i;
-        ca += (2 * __ldg(p.val_off + t) + __ldg(p.meta_off + t)) * G < tgtA;
+    s_cnt[0] = planned ? 1u : 0u;
+  }
+  __syncthreads();
+  const bool planned = s_cnt[0] != 0;
+  __syncthreads();
+  if (tid == 0) s_cnt[0] = 0;
+  __syncthreads();
+  if (!planned) {
+      const int64_t tgtA = (int64_t)c * p.total, tgtB = (int64_t)(c + 1) * p.total;
+      uint32_t ca = 0, cb = 0;
+      for (int i = tid; i <= p.R; i += blockDim.x) {
+        const int64_t t = (int64_t)i * tpr;
+        const int64_t P = 2 * __ldg(p.val_off + t) + __ldg(p.meta_off + t);
+        ca += P * G < tgtA;
+        cb += P * G < tgtB;
       }
-      if (bB > 0) {
-        const int64_t t = baseB + i;
-        cb += (2 * __ldg(p.val_off + t) + __ldg(p.meta_off + t)) * G < tgtB;
+      ca = __reduce_add_sync(0xffffffffu, ca);
+      cb = __reduce_add_sync(0xffffffffu, cb);
+      if (lane == 0) {
+        atomicAdd(&s_cnt[0], ca);
+        atomicAdd(&s_cnt[1], cb);
       }
-    }
-    ca = __reduce_add_sync(0xffffffffu, ca);
-    cb = __reduce_add_sync(0xffffffffu, cb);
-    if (lane == 0) {
-      atomicAdd(&s_cnt[0], ca);
-      atomicAdd(&s_cnt[1], cb);
-    }
-    __syncthreads();
-    if (tid == 0) {
-      s_range[0] = bA > 0 ? baseA + s_cnt[0] : 0;
-      s_range[1] = (c == G - 1) ? p.T : (bB > 0 ? baseB + s_cnt[1] : 0);
-    }
-    __syncthreads();
+      __syncthreads();
+      const uint32_t bA = s_cnt[0], bB = s_cnt[1];  // band starts below each target
+      __syncthreads();
+      if (tid == 0) {
+        s_cnt[0] = 0;
+        s_cnt[1] = 0;
+      }
+      __syncthreads();
+      ca = 0;
+      cb = 0;
+      const int64_t baseA = bA > 0 ? (int64_t)(bA - 1) * tpr : 0;
+      const int64_t baseB = bB > 0 ? (int64_t)(bB - 1) * tpr : 0;
+      for (int i = tid; i < tpr; i += blockDim.x) {
+        if (bA > 0) {
+          const int64_t t = baseA + i;
+          ca += (2 * __ldg(p.val_off + t) + __ldg(p.meta_off + t)) * G < tgtA;
+        }
+        if (bB > 0) {
+          const int64_t t = baseB + i;
+          cb += (2 * __ldg(p.val_off + t) + __ldg(p.meta_off + t)) * G < tgtB;
+        }
+      }
+      ca = __reduce_add_sync(0xffffffffu, ca);
+      cb = __reduce_add_sync(0xffffffffu, cb);
+      if (lane == 0) {
+        atomicAdd(&s_cnt[0], ca);
+        atomicAdd(&s_cnt[1], cb);
+      }
+      __syncthreads();
+      if (tid == 0) {
+        s_range[0] = bA > 0 ? baseA + s_cnt[0] : 0;
+        s_range[1] = (c == G - 1) ? p.T : (bB > 0 ? baseB + s_cnt[1] : 0);
+      }
+      __syncthreads();
   }
   const int64_t t0 = s_range[0];
   const int64_t t1 = s_range[1];
@@ -740,6 +774,102 @@ __global__ void __launch_bounds__(TmaCfg<BP, B1, B2>::kThreads, 1)
     return;
   }
 
+  if (warp == C::NC + 1) {
+    // ------------------------------ epilogue ------------------------------
+    // Takes every piece of band this CTA finishes, in band order: a whole
+    // band goes straight to Y (with the low-rank term); a band shared with
+    // other CTAs goes to slot c + r, and a ticket per band finds the last of
+    // its CTAs, which sums the band's slots in CTA order (deterministic).
+    // All global-memory ordering (fence, atomic) happens here, off the
+    // consumer warps' path.
+    auto owner_of_p = [&](int64_t P) -> int {
+      const int64_t o = (P * G) / p.total;
+      return (int)(o < G - 1 ? o : G - 1);
+    };
+    const int r_first = (int)(t0 / tpr), r_last = t1 > t0 ? (int)((t1 - 1) / tpr) : r_first - 1;
+    int piece = 0;
+    for (int r = r_first; r <= r_last; ++r, ++piece) {
+      const int slot = piece & 1;
+      const uint32_t ph = (uint32_t)(piece >> 1) & 1u;
+      const bool whole = t0 <= (int64_t)r * tpr && t1 >= (int64_t)(r + 1) * tpr;
+      // owners of the band's first and last tile, fetched before the wait
+      int64_t pa = 0, pb = 0;
+      if (!whole && lane == 0) {
+        const int64_t ta = (int64_t)r * tpr, tb = ta + tpr - 1;
+        pa = 2 * __ldg(p.val_off + ta) + __ldg(p.meta_off + ta);
+        pb = 2 * __ldg(p.val_off + tb) + __ldg(p.meta_off + tb);
+      }
+      if (!mbar_wait(&piece_full[slot], ph)) {
+        if (lane == 0) atomicOr(p.status, kStatusTimeout);
+        break;
+      }
+      const float(*rows)[C::RW * BP] = s_rows[slot];
+      const int64_t row0 = (int64_t)r * B1;
+      if (whole) {
+        for (int o = lane; o < B1 * BP; o += 32) {
+          const int row = o % B1, b = o / B1;
+          if (b < p.batch) store_out(p, row0 + row, b, rows[row / C::RW][b * C::RW + row % C::RW]);
+        }
+      } else {
+        float *slotp = p.partials + (int64_t)(c + r) * BP * B1;
+        for (int o = lane; o < B1 * BP; o += 32) {
+          const int row = o % B1, b = o / B1;
+          __stcg(slotp + b * B1 + row, rows[row / C::RW][b * C::RW + row % C::RW]);
+        }
+        __threadfence();  // this lane's slot values before the ticket
+        __syncwarp();
+        uint32_t last = 0;
+        int oA = 0, oB = 0;
+        if (lane == 0) {
+          oA = owner_of_p(pa);
+          oB = owner_of_p(pb);
+          last = atomicAdd(p.counters + r, 1u) == (uint32_t)(oB - oA);
+        }
+        last = __shfl_sync(0xffffffffu, last, 0);
+        oA = __shfl_sync(0xffffffffu, oA, 0);
+        oB = __shfl_sync(0xffffffffu, oB, 0);
+        if (last) {
+          __threadfence();
+          // sum the band's slots in CTA order; the loads of 4 outputs x 8
+          // contributors are issued together, then added in a fixed order
+          constexpr int OPL = 4, QMAX = 8;
+          for (int o0 = 0; o0 < B1 * BP; o0 += 32 * OPL) {
+            float y[OPL];
+#pragma unroll
+            for (int u = 0; u < OPL; ++u) y[u] = 0.f;
+            for (int q0 = oA; q0 <= oB; q0 += QMAX) {
+              float v[OPL][QMAX];
+#pragma unroll
+              for (int u = 0; u < OPL; ++u) {
+                const int o = o0 + u * 32 + lane;
+                const int row = o % B1, b = o / B1;
+#pragma unroll
+                for (int q = 0; q < QMAX; ++q)
+                  v[u][q] = (o < B1 * BP && q0 + q <= oB)
+                                ? __ldcg(p.partials + ((int64_t)(q0 + q + r) * BP + b) * B1 + row)
+                                : 0.f;
+              }
+#pragma unroll
+              for (int u = 0; u < OPL; ++u)
+#pragma unroll
+                for (int q = 0; q < QMAX; ++q) y[u] += v[u][q];
+            }
+#pragma unroll
+            for (int u = 0; u < OPL; ++u) {
+              const int o = o0 + u * 32 + lane;
+              const int row = o % B1, b = o / B1;
+              if (o < B1 * BP && b < p.batch) store_out(p, row0 + row, b, y[u]);
+            }
+          }
+          if (lane == 0) p.counters[r] = 0;  // ready for the next call
+        }
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&piece_empty[slot]);
+    }
+    return;
+  }
+
   // -------------------------------- consumers --------------------------------
   const int cp = lane % C::CPR;
   const int rs = lane / C::CPR;
@@ -749,41 +879,7 @@ __global__ void __launch_bounds__(TmaCfg<BP, B1, B2>::kThreads, 1)
   for (int j = 0; j < C::JS; ++j)
 #pragma unroll
     for (int b = 0; b < BP; ++b) acc[j][b] = 0.f;
-
-  // Deferred ticket of the last band piece this warp sent to a slot, with the
-  // packed offsets of that band's first and last tile (to name its owners).
-  int pend_band = -1;
-  uint32_t pend_ticket = 0;
-  int64_t pend_pa = 0, pend_pb = 0;
-  auto owner_of_p = [&](int64_t P) -> int {
-    const int64_t o = (P * G) / p.total;
-    return (int)(o < G - 1 ? o : G - 1);
-  };
-  auto finish_band = [&]() {
-    const int rb = pend_band;
-    pend_band = -1;
-    const uint32_t ticket = __shfl_sync(0xffffffffu, pend_ticket, 0);
-    const int oA = owner_of_p(__shfl_sync(0xffffffffu, pend_pa, 0));
-    const int oB = owner_of_p(__shfl_sync(0xffffffffu, pend_pb, 0));
-    if (ticket != (uint32_t)(oB - oA)) return;
-    __syncwarp();
-    // this warp was the last contributor: sum slots oA..oB (CTA order) for
-    // its 8 rows; lanes = (output, phase), phases combined in a fixed pattern
-    constexpr int NOUT = C::RW * BP;
-    constexpr int NPH = NOUT >= 32 ? 1 : 32 / NOUT;
-    for (int base = 0; base < NOUT; base += 32 / NPH) {
-      const int o = base + lane / NPH, ph = lane % NPH;
-      const int row = wrow + o % C::RW, b = o / C::RW;
-      float y = 0.f;
-      if (o < NOUT && b < p.batch)
-        for (int cc = oA + ph; cc <= oB; cc += NPH)
-          y += __ldcg(p.partials + ((int64_t)(cc + rb) * BP + b) * B1 + row);
-#pragma unroll
-      for (int m = 1; m < NPH; m <<= 1) y += __shfl_xor_sync(0xffffffffu, y, m);
-      if (ph == 0 && o < NOUT && b < p.batch) store_out(p, (int64_t)rb * B1 + row, b, y);
-    }
-    if (lane == 0) p.counters[(int64_t)rb * C::NC + warp] = 0;  // ready for the next call
-  };
+  int piece = 0;
 
   int stage = 0;
   uint32_t phase = 0;
@@ -858,11 +954,14 @@ __global__ void __launch_bounds__(TmaCfg<BP, B1, B2>::kThreads, 1)
     }
     if (!(d.flags & 1)) continue;
 
-    // ---- end of this CTA's piece of band r: row sums to Y or to a slot ----
-    // Reduce over the lanes of each row, park the 8 x BP sums of this warp in
-    // shared memory, then let all 32 lanes store them (o = b * RW + row).
-    const int r = (int)(d.t0 / tpr);
-    float *rows_s = s_rows[warp];
+    // ---- end of this CTA's piece of a band: row sums to the epilogue warp ----
+    const int slot = piece & 1;
+    const uint32_t ph = (uint32_t)(piece >> 1) & 1u;
+    if (!mbar_wait(&piece_empty[slot], ph ^ 1u)) {
+      if (lane == 0) atomicOr(p.status, kStatusTimeout);
+      break;
+    }
+    float *rows_s = s_rows[slot][warp];
 #pragma unroll
     for (int j = 0; j < C::JS; ++j)
 #pragma unroll
@@ -874,33 +973,33 @@ __global__ void __launch_bounds__(TmaCfg<BP, B1, B2>::kThreads, 1)
         acc[j][b] = 0.f;
       }
     __syncwarp();
-    const bool whole = t0 <= (int64_t)r * tpr && t1 >= (int64_t)(r + 1) * tpr;
-    if (whole) {
-      for (int o = lane; o < C::RW * BP; o += 32) {
-        const int row = o % C::RW, b = o / C::RW;
-        if (b < p.batch) store_out(p, (int64_t)r * B1 + wrow + row, b, rows_s[o]);
-      }
-    } else {
-      if (pend_band >= 0) finish_band();
-      float *slot = p.partials + (int64_t)(c + r) * BP * B1;
-      for (int o = lane; o < C::RW * BP; o += 32) {
-        const int row = o % C::RW, b = o / C::RW;
-        __stcg(slot + b * B1 + wrow + row, rows_s[o]);
-      }
-      __syncwarp();
-      if (lane == 0) {
-        // release: the slot rows above (written by this warp, ordered by the
-        // warp barrier) are visible before the ticket moves
-        pend_ticket = atom_add_acq_rel(p.counters + (int64_t)r * C::NC + warp, 1u);
-        const int64_t ta = (int64_t)r * tpr, tb = ta + tpr - 1;
-        pend_pa = 2 * __ldg(p.val_off + ta) + __ldg(p.meta_off + ta);
-        pend_pb = 2 * __ldg(p.val_off + tb) + __ldg(p.meta_off + tb);
-      }
-      pend_band = r;
-    }
-    __syncwarp();
+    if (lane == 0) mbar_arrive(&piece_full[slot]);
+    ++piece;
   }
-  if (pend_band >= 0) finish_band();
+}
+
+// ---------------------------------------------------------------------------
+// work-split plan: plan = [G, t0(0), ..., t0(G)], t0(c) the first tile whose
+// packed offset P satisfies P*G >= c*total (the rule the streaming kernel
+// applies when it has no plan)
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(1024)
+    plan_kernel(const int64_t *__restrict__ val_off, const int64_t *__restrict__ meta_off,
+                int64_t T, int G, int64_t total, int64_t *__restrict__ plan) {
+  auto owner = [&](int64_t t) -> int64_t {
+    const int64_t o = (2 * val_off[t] + meta_off[t]) * G / total;
+    return o < G - 1 ? o : G - 1;
+  };
+  for (int64_t t = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; t < T;
+       t += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t o = owner(t);
+    const int64_t prev = t == 0 ? -1 : owner(t - 1);
+    for (int64_t c = prev + 1; c <= o; ++c) plan[1 + c] = t;
+  }
+  if (blockIdx.x == 0 && threadIdx.x == 0) {
+    plan[0] = G;
+    plan[1 + G] = T;
+  }
 }
 
 // ---------------------------------------------------------------------------
@@ -1413,6 +1512,7 @@ int spmm_impl(const hyb_matrix *A, int batch, const uint16_t *X, int64_t ldx,
   prm.ldy = ldy;
   prm.ydt = ydt;
   prm.total = 2 * A->n_vals + A->n_meta_bytes;  // packed bytes
+  prm.plan = A->plan;
   return run_product(prm, A->b1, A->b2, batch, lr, false, ws, ws_bytes, s);
 }
 
@@ -1452,6 +1552,39 @@ size_t lowrank_ws_layout(int64_t k, int batch, int rank, size_t *off_t,
 using namespace hyb;
 
 extern "C" {
+
+size_t hyb_plan_entries(void) {
+  int sms = 0;
+  if (device_sm_count(&sms) != HYB_OK) return 0;
+  return (size_t)sms + 2;
+}
+
+int hyb_make_plan(const hyb_matrix *A, int64_t *plan, hyb_stream_t stream) {
+  if (!A || !plan) return HYB_ERR_INVALID_ARG;
+  int rc = check_tiling(A->n, A->k, A->b1, A->b2);
+  if (rc != HYB_OK) return rc;
+  if (!A->val_off || !A->meta_off || A->num_tiles != (A->n / A->b1) * (A->k / A->b2))
+    return HYB_ERR_INVALID_ARG;
+  if ((uintptr_t)plan % 8 != 0) return HYB_ERR_ALIGNMENT;
+  int sms = 0;
+  rc = device_sm_count(&sms);
+  if (rc != HYB_OK) return rc;
+  cudaStream_t s = (cudaStream_t)stream;
+  const int64_t total = 2 * A->n_vals + A->n_meta_bytes;
+  if (shape_of(A->b1, A->b2) == kGeneric || total <= 0) {
+    // no streaming kernel for this tiling: an empty plan (G = 0) is ignored
+    return cudaMemsetAsync(plan, 0, sizeof(int64_t), s) == cudaSuccess ? HYB_OK : HYB_ERR_CUDA;
+  }
+  // the same G as make_plan's streaming path: one CTA per SM, each owning
+  // at least one tile
+  const int64_t gcap = std::max<int64_t>(1, total / (2LL * A->b1 * A->b2));
+  const int G = (int)std::min<int64_t>(sms, gcap);
+  const int64_t T = A->num_tiles;
+  const int64_t blocks = std::min<int64_t>((T + 1023) / 1024, 64);
+  plan_kernel<<<(unsigned)std::max<int64_t>(1, blocks), 1024, 0, s>>>(A->val_off, A->meta_off, T,
+                                                                     G, total, plan);
+  return cudaGetLastError() == cudaSuccess ? HYB_OK : HYB_ERR_CUDA;
+}
 
 size_t hyb_workspace_bytes(const hyb_matrix *A, int batch, int rank) {
   if (!A || check_tiling(A->n, A->k, A->b1, A->b2) != HYB_OK) return 0;

@@ -43,7 +43,8 @@ class HybMatrix(ctypes.Structure):
                 ("num_tiles", ctypes.c_int64),
                 ("tile_map", _P), ("vals", _P), ("meta", _P),
                 ("val_off", _P), ("meta_off", _P),
-                ("n_vals", ctypes.c_int64), ("n_meta_bytes", ctypes.c_int64)]
+                ("n_vals", ctypes.c_int64), ("n_meta_bytes", ctypes.c_int64),
+                ("plan", _P)]
 
 
 class HybLowrank(ctypes.Structure):
@@ -63,7 +64,8 @@ EXPORTS = ["hyb_packed_sizes", "hyb_pack_workspace_bytes", "hyb_pack",
            "hyb_workspace_bytes", "hyb_workspace_init", "hyb_spmv",
            "hyb_spmm_skinny", "hyb_lowrank_workspace_bytes", "hyb_lowrank_add",
            "hyb_dense_workspace_bytes", "hyb_gemv_dense", "hyb_check_status",
-           "hyb_status_string", "hyb_spmv_noalloc", "hyb_spmv_noalloc_max_scratch_bytes"]
+           "hyb_status_string", "hyb_spmv_noalloc", "hyb_spmv_noalloc_max_scratch_bytes",
+           "hyb_plan_entries", "hyb_make_plan"]
 
 
 def lib():
@@ -107,6 +109,10 @@ def lib():
     L.hyb_spmv_noalloc.restype = _I
     L.hyb_spmv_noalloc_max_scratch_bytes.argtypes = []
     L.hyb_spmv_noalloc_max_scratch_bytes.restype = _SZ
+    L.hyb_plan_entries.argtypes = []
+    L.hyb_plan_entries.restype = _SZ
+    L.hyb_make_plan.argtypes = [ctypes.POINTER(HybMatrix), _P, _P]
+    L.hyb_make_plan.restype = _I
     L.hyb_status_string.argtypes = [_I]
     L.hyb_status_string.restype = ctypes.c_char_p
     _lib = L
@@ -169,6 +175,7 @@ class Packed:
     meta_off: torch.Tensor   # int64 [T+1], device
     n_vals: int
     n_meta: int
+    plan: Optional[torch.Tensor] = None  # int64 work split (hyb_make_plan), optional
 
     @property
     def num_tiles(self) -> int:
@@ -178,7 +185,8 @@ class Packed:
         return HybMatrix(self.n, self.k, self.b1, self.b2, self.num_tiles,
                          self.tile_map.data_ptr(), self.vals.data_ptr(),
                          self.meta.data_ptr(), self.val_off.data_ptr(),
-                         self.meta_off.data_ptr(), self.n_vals, self.n_meta)
+                         self.meta_off.data_ptr(), self.n_vals, self.n_meta,
+                         None if self.plan is None else self.plan.data_ptr())
 
     def nbytes(self) -> int:
         """Packed bytes the product streams (values + masks)."""
@@ -187,7 +195,8 @@ class Packed:
     def clone(self) -> "Packed":
         return Packed(self.n, self.k, self.b1, self.b2, self.tile_map.clone(),
                       self.vals.clone(), self.meta.clone(), self.val_off.clone(),
-                      self.meta_off.clone(), self.n_vals, self.n_meta)
+                      self.meta_off.clone(), self.n_vals, self.n_meta,
+                      None if self.plan is None else self.plan.clone())
 
 
 def pack_workspace_bytes() -> int:
@@ -205,12 +214,23 @@ def new_workspace(nbytes: int, device) -> torch.Tensor:
     return ws
 
 
+def make_plan(A: "Packed", stream=None) -> torch.Tensor:
+    """hyb_make_plan: the product's work split for A on the current device."""
+    plan = torch.zeros(int(lib().hyb_plan_entries()), dtype=torch.int64,
+                       device=A.val_off.device)
+    s = A.struct()
+    s.plan = None
+    _check("hyb_make_plan", lib().hyb_make_plan(ctypes.byref(s), _ptr(plan), _stream(stream)))
+    return plan
+
+
 def pack(W: torch.Tensor, tile_map, b1: int, b2: int, ws: torch.Tensor = None,
-         stream=None, check: bool = True) -> Packed:
+         stream=None, check: bool = True, plan: bool = True) -> Packed:
     """hyb_pack: dense bf16 W [n][k] (device) + tile map -> Packed.
 
     With ``check`` the call synchronises and raises HybError on a NaN weight or
-    a bad map byte (the pack itself is complete either way)."""
+    a bad map byte (the pack itself is complete either way).  With ``plan`` the
+    product's work split is made once here (hyb_make_plan)."""
     Wb = _bits(W)
     assert Wb.is_cuda and Wb.dim() == 2
     n, k = Wb.shape
@@ -232,7 +252,10 @@ def pack(W: torch.Tensor, tile_map, b1: int, b2: int, ws: torch.Tensor = None,
                                       _ptr(ws), ws.numel(), _stream(stream)))
     if check:
         check_status(ws, stream)
-    return Packed(n, k, b1, b2, tm, vals, meta, vo, mo, nv, nm)
+    P = Packed(n, k, b1, b2, tm, vals, meta, vo, mo, nv, nm)
+    if plan:
+        P.plan = make_plan(P, stream)
+    return P
 
 
 def check_status(ws: torch.Tensor, stream=None) -> int:

@@ -165,3 +165,42 @@ def test_llama70b_ffn_lowrank_full_size(orc):
 def test_lowrank_fused_small(orc, batch):
     tmap = inputs.tile_map_bernoulli(40, 0.6, inputs.seed_of("lrsmall"))
     _full_check(orc, 640, 1024, 128, 128, tmap, batch, "lrsmall", rank=64)
+
+
+def _split_reference(orc, n, k, b1, b2, tmap, G):
+    """CTA c's first tile: the first t with P(t) * G >= c * total, where P is the
+    packed byte offset (2 * val_off + meta_off) -- computed from the oracle's
+    offsets."""
+    vo, mo = orc.offsets(n, k, b1, b2, tmap)
+    P = 2 * vo.astype(np.int64) + mo
+    total = int(P[-1])
+    T = len(tmap)
+    starts = [int(np.sum(P[:T] * G < c * total)) for c in range(G)] + [T]
+    return starts
+
+
+@pytest.mark.parametrize("shape", [(4096, 14336, 128, 128), (14336, 4096, 128, 64),
+                                   (256, 256, 64, 64)])
+def test_plan_matches_definition_and_results(orc, shape):
+    """hyb_make_plan gives the split the kernel would search for, and the product
+    with and without the plan (or with a plan for another SM count) is the same."""
+    n, k, b1, b2 = shape
+    T = (n // b1) * (k // b2)
+    tmap = inputs.tile_map_fraction(T, 0.5, inputs.seed_of("plan", n, k))
+    W, tmap, X, _ = case(n, k, b1, b2, tmap, name="plan")
+    P = hyb.pack(W.to(dev()), tmap, b1, b2)
+    plan = P.plan.cpu().numpy()
+    G = int(plan[0])
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    assert G == min(sms, max(1, (2 * P.n_vals + P.n_meta) // (2 * b1 * b2)))
+    assert plan[1:G + 2].tolist() == _split_reference(orc, n, k, b1, b2, tmap, G)
+    Xd = X.to(dev())
+    y_plan = hyb.spmv(P, Xd)
+    saved = P.plan
+    P.plan = None
+    y_search = hyb.spmv(P, Xd)
+    stale = saved.clone()
+    stale[0] = G + 1  # a plan for another SM count is ignored
+    P.plan = stale
+    y_stale = hyb.spmv(P, Xd)
+    assert torch.equal(y_plan, y_search) and torch.equal(y_plan, y_stale)
