@@ -104,6 +104,7 @@ typedef struct {
   const int64_t *plan;      /* optional (may be NULL): work split made by
                                hyb_make_plan for this matrix on this device;
                                saves the products a search at every call */
+  int32_t plan_ctas;        /* the CTA count hyb_make_plan reported for plan */
 } hyb_matrix;
 
 /* Low-rank factors of y += U (V^T x): U is [n][rank] (row stride ldu),
@@ -147,12 +148,14 @@ HYB_API int hyb_pack(int64_t n, int64_t k, int b1, int b2, const uint16_t *W,
 HYB_API size_t hyb_plan_entries(void);
 
 /* Write into `plan` (device, hyb_plan_entries() int64_t) the split of A's
- * packed bytes over the streaming kernel's CTAs on the current device: CTA c
- * takes the tiles whose packed byte offset falls in [c, c+1) * total / G.
- * The products find the same split by searching val_off / meta_off when
- * A->plan is NULL; a plan only saves that search.  A plan made on another
- * device (another SM count) is detected and ignored. */
-HYB_API int hyb_make_plan(const hyb_matrix *A, int64_t *plan, hyb_stream_t stream);
+ * packed bytes over the streaming kernel's CTAs on the current device (CTA c
+ * takes the tiles whose packed byte offset falls in [c, c+1) * total / G),
+ * together with each CTA's first tile offsets, and store G in *plan_ctas
+ * (0 when the tiling has no streaming kernel).  Set A->plan / A->plan_ctas
+ * from these to let the products skip their start-up search; the products
+ * ignore a plan whose plan_ctas differs from the CTA count they would use. */
+HYB_API int hyb_make_plan(const hyb_matrix *A, int64_t *plan, int32_t *plan_ctas,
+                          hyb_stream_t stream);
 
 /* ---- products ---------------------------------------------------------- */
 

@@ -68,8 +68,15 @@ struct Params {
   float *partials;
   uint32_t *counters;
   uint32_t *status;  // workspace status word
-  const int64_t *plan;  // optional precomputed split: [G, t0(0), ..., t0(G)]
+  const int64_t *plan;  // optional precomputed split (validated by the host)
+  int plan_ctas;
 };
+
+// Plan layout (int64): [0] = G, [1..7] reserved, then one record per CTA:
+// [t0, t1, 2:4 bitmask of tiles t0..t0+30, 0, val_off[t0..t0+31],
+//  meta_off[t0..t0+31]] (offsets clamped at the last tile).
+constexpr int kPlanHead = 8;
+constexpr int kPlanRec = 68;
 
 // ---------------------------------------------------------------------------
 // helpers
@@ -535,11 +542,15 @@ struct TmaCfg {
   static constexpr int RPS = 32 / CPR;              // rows per warp step
   static constexpr int JS = RW / RPS;               // steps per warp per tile
   static constexpr int XB = BP < 4 ? BP : 4;        // batch columns per pass
-  static constexpr int TPS = (16384 / (B1 * B2)) > 0 ? 16384 / (B1 * B2) : 1;  // tiles per stage
-  static constexpr int WIN = 28;                    // tiles per producer offset window
-  static constexpr int kValsBytes = 2 * B1 * B2 * TPS;        // 32 KB
-  static constexpr int kMetaBytes = B1 * B2 / 8 * TPS;        // 2 KB
-  static constexpr int kXRow = 2 * B2 * TPS;                  // bytes of one X row slice
+  // A stage holds 32 KB of values: TPD dense tiles, or up to 2*TPD tiles
+  // when some are 2:4 (a 2:4 tile has half the bytes), so that every stage
+  // in the ring carries about the same number of bytes.
+  static constexpr int TPD = (16384 / (B1 * B2)) > 0 ? 16384 / (B1 * B2) : 1;
+  static constexpr int TPX = 2 * TPD;                         // tiles per stage, at most
+  static constexpr int WIN = 31;                    // tiles per producer offset window
+  static constexpr int kValsBytes = 2 * B1 * B2 * TPD;        // 32 KB
+  static constexpr int kMetaBytes = B1 * B2 / 8 * TPX;        // 4 KB
+  static constexpr int kXRow = 2 * B2 * TPX;                  // bytes of one X row slice
   static constexpr int kStageBytes = kValsBytes + kMetaBytes + BP * kXRow;
   static constexpr int kStages =
       (200 * 1024 / kStageBytes) < 6 ? (200 * 1024 / kStageBytes) : 6;
@@ -547,12 +558,12 @@ struct TmaCfg {
   static constexpr size_t kSmem = (size_t)kStages * kStageBytes + 1024;
   static_assert(RPS * CPR == 32 && JS * RPS == RW && JS >= 1, "tile shape");
   static_assert(kStages >= 3, "ring too short");
-  static_assert(WIN % TPS == 0 && WIN < 32, "offset window");
+  static_assert(TPX <= 8 && WIN < 32, "stage / offset window");
 };
 
 struct StageDesc {
   int64_t t0;       // first tile of the stage
-  uint16_t ntiles;  // tiles in the stage (<= TPS, never across a band)
+  uint16_t ntiles;  // tiles in the stage (<= TPX, never across a band)
   uint8_t sparse;   // bit i: tile i is 2:4
   uint8_t flags;    // 1: last stage of this CTA's piece of a band, 2: end of work
 };
@@ -607,24 +618,12 @@ __global__ void __launch_bounds__(TmaCfg<BP, B1, B2>::kThreads, 1)
   __syncthreads();
 
   // ---- this CTA's tiles [t0, t1): tiles whose packed offset P(t) satisfies
-  // c*total <= P(t)*G < (c+1)*total.  A plan made for this G gives them
-  // directly; otherwise round 1 brackets both ends between band starts and
-  // round 2 counts inside the bracketing band. ----
-  if (tid == 0) {
-    bool planned = false;
-    if (p.plan != nullptr && __ldg(p.plan) == (int64_t)G) {
-      s_range[0] = __ldg(p.plan + 1 + c);
-      s_range[1] = __ldg(p.plan + 2 + c);
-      planned = true;
-    }
-    s_cnt[0] = planned ? 1u : 0u;
-  }
-  __syncthreads();
-  const bool planned = s_cnt[0] != 0;
-  __syncthreads();
-  if (tid == 0) s_cnt[0] = 0;
-  __syncthreads();
-  if (!planned) {
+  // c*total <= P(t)*G < (c+1)*total.  With a plan the producer and the
+  // epilogue warp read them from the CTA's record; otherwise round 1
+  // brackets both ends between band starts and round 2 counts inside the
+  // bracketing band. ----
+  const int64_t *rec = p.plan ? p.plan + kPlanHead + (int64_t)c * kPlanRec : nullptr;
+  if (rec == nullptr) {
       const int64_t tgtA = (int64_t)c * p.total, tgtB = (int64_t)(c + 1) * p.total;
       uint32_t ca = 0, cb = 0;
       for (int i = tid; i <= p.R; i += blockDim.x) {
@@ -674,73 +673,112 @@ __global__ void __launch_bounds__(TmaCfg<BP, B1, B2>::kThreads, 1)
       }
       __syncthreads();
   }
-  const int64_t t0 = s_range[0];
-  const int64_t t1 = s_range[1];
+  // consumers never need the range; the producer and the epilogue warp take
+  // it from the plan record when there is one
+  int64_t t0 = 0, t1 = 0;
+  if (rec == nullptr) {
+    t0 = s_range[0];
+    t1 = s_range[1];
+  } else if (warp >= C::NC) {
+    t0 = __ldg(rec + 0);
+    t1 = __ldg(rec + 1);
+  }
 
   if (warp == C::NC) {
     // ------------------------------ producer ------------------------------
-    // Stages follow a fixed grid: inside a band, stage boundaries sit every
-    // TPS tiles from the band start, so stage g of the whole matrix covers
-    // tiles [band*tpr + (g%spb)*TPS, ...) with spb stages per band.  Lane i
-    // works out stage g0+i of this CTA's piece (tile range, packed offsets,
-    // 2:4 bits) while the previous 32 stages are issued one by one.
-    const int spb = (tpr + C::TPS - 1) / C::TPS;
-    const int64_t g_first = (t0 / tpr) * spb + (t0 % tpr) / C::TPS;
-    const int64_t g_last = t1 > t0 ? ((t1 - 1) / tpr) * spb + ((t1 - 1) % tpr) / C::TPS : g_first - 1;
-    struct StageInfo {
-      int64_t ts, te;         // tiles [ts, te)
-      int64_t vs, ve, ms, me; // packed value / meta offsets
-      uint32_t sp, flags;
-      const uint16_t *xsrc;   // X slice (row 0)
+    // Tiles are taken in windows of WIN: lane i holds the packed offsets of
+    // tile w0 + i (and lane WIN those of the window's end), the next window
+    // is loaded while this one is issued.  Stages are packed greedily inside
+    // a window: a new stage starts at a band start or when the next tile no
+    // longer fits in the 32 KB value buffer; every lane runs the same packing
+    // over the window's 2:4 bitmask, so all agree on the stage starts.
+    struct Win {
+      int64_t vo, mo;
+      uint32_t sp;
     };
-    auto stage_info = [&](int64_t g) -> StageInfo {
-      StageInfo o{};
-      if (g > g_last) return o;
-      const int64_t band = g / spb, loc = g - band * spb;
-      const int64_t bs = band * tpr, be = bs + tpr;
-      o.ts = max(t0, bs + loc * C::TPS);
-      o.te = min(min(t1, be), bs + (loc + 1) * C::TPS);
-      o.vs = __ldg(p.val_off + o.ts);
-      o.ve = __ldg(p.val_off + o.te);
-      o.ms = __ldg(p.meta_off + o.ts);
-      o.me = __ldg(p.meta_off + o.te);
-      for (int64_t q = o.ts; q < o.te; ++q) o.sp |= (uint32_t)(__ldg(p.map + q) == 1) << (q - o.ts);
-      o.flags = (o.te == be || o.te == t1) ? 1u : 0u;
-      o.xsrc = p.X + (o.ts - bs) * B2;
+    auto load_win = [&](int64_t w0) -> Win {
+      Win o{0, 0, 0};
+      const int64_t t = w0 + lane;
+      if (lane <= C::WIN && t <= t1) {
+        o.vo = __ldg(p.val_off + t);
+        o.mo = __ldg(p.meta_off + t);
+      }
+      if (lane < C::WIN && t < t1) o.sp = __ldg(p.map + t) == 1;
       return o;
     };
     int stage = 0;
     uint32_t phase = 0;
     bool ok = true;
     uint32_t armed = 0, armed_parity = 0;  // per stage: copies issued / phase parity
-    StageInfo cur = stage_info(g_first + lane);
-    for (int64_t gw = g_first; ok && gw <= g_last; gw += 32) {
-      const StageInfo nxt = stage_info(gw + 32 + lane);  // in flight while issuing
-      const int nst = (int)min((int64_t)32, g_last - gw + 1);
-      for (int k = 0; k < nst; ++k) {
-        if (lane == k) {
+    Win cur;
+    if (rec != nullptr) {
+      // first window straight from the plan record (same round trip as t0)
+      cur.vo = __ldg(rec + 4 + lane);
+      cur.mo = __ldg(rec + 36 + lane);
+      cur.sp = (uint32_t)(__ldg(rec + 2) >> lane) & 1u;
+    } else {
+      cur = load_win(t0);
+    }
+    for (int64_t w0 = t0; ok && w0 < t1; w0 += C::WIN) {
+      const Win nxt = load_win(w0 + C::WIN);  // in flight while this window issues
+      const int nw = (int)min((int64_t)C::WIN, t1 - w0);
+      const uint32_t spm = __ballot_sync(0xffffffffu, cur.sp != 0);
+      // greedy packing; value bytes in units of a 2:4 tile (dense = 2)
+      uint32_t starts = 0;
+      {
+        int64_t nb = (w0 / tpr) * tpr;  // first band start at or after w0
+        if (nb < w0) nb += tpr;
+        int fill = 2 * C::TPX, cnt = C::TPX;  // force a start at tile 0
+        for (int i = 0; i < nw; ++i) {
+          const int sz = (spm >> i & 1u) ? 1 : 2;
+          const bool band_start = w0 + i == nb;
+          if (band_start) nb += tpr;
+          if (band_start || fill + sz > 2 * C::TPD || cnt == C::TPX) {
+            starts |= 1u << i;
+            fill = 0;
+            cnt = 0;
+          }
+          fill += sz;
+          ++cnt;
+        }
+      }
+      // the stage that starts at this lane: tiles [w0 + lane, w0 + e)
+      const bool is_start = lane < nw && (starts >> lane & 1u);
+      const uint32_t later = lane < 31 ? (starts >> (lane + 1)) : 0u;
+      const int e = later ? lane + 1 + __ffs(later) - 1 : nw;
+      const int64_t v_end = __shfl_sync(0xffffffffu, cur.vo, e & 31);
+      const int64_t m_end = __shfl_sync(0xffffffffu, cur.mo, e & 31);
+      // (e == 32 only when nw == 32, which WIN < 32 rules out)
+      uint32_t todo = starts;
+      while (todo) {
+        const int k = __ffs(todo) - 1;
+        todo &= todo - 1;
+        if (lane == k && is_start) {
           if (!mbar_wait(&empty_bar[stage], phase ^ 1u)) {
             ok = false;
           } else {
             uint8_t *st = smem + (size_t)stage * C::kStageBytes;
-            const uint32_t vbytes = (uint32_t)(2 * (cur.ve - cur.vs));
-            const uint32_t mbytes = (uint32_t)(cur.me - cur.ms);
-            const int nt = (int)(cur.te - cur.ts);
+            const int64_t ts = w0 + k, te = w0 + e;
+            const uint32_t vbytes = (uint32_t)(2 * (v_end - cur.vo));
+            const uint32_t mbytes = (uint32_t)(m_end - cur.mo);
+            const int nt = e - k;
             const uint32_t xrow = (uint32_t)(2 * B2 * nt);
+            const int64_t band = ts / tpr;
             StageDesc d;
-            d.t0 = cur.ts;
+            d.t0 = ts;
             d.ntiles = (uint16_t)nt;
-            d.sparse = (uint8_t)cur.sp;
-            d.flags = (uint8_t)cur.flags;
+            d.sparse = (uint8_t)((spm >> k) & ((1u << nt) - 1u));
+            d.flags = (te == (band + 1) * tpr || te == t1) ? 1 : 0;
             desc[stage] = d;
             armed |= 1u << stage;
             armed_parity = (armed_parity & ~(1u << stage)) | (phase << stage);
             mbar_arrive_expect_tx(&full_bar[stage], vbytes + mbytes + xrow * p.batch);
-            bulk_g2s(st, p.vals + 2 * cur.vs, vbytes, &full_bar[stage]);
-            if (mbytes) bulk_g2s(st + C::kValsBytes, p.meta + cur.ms, mbytes, &full_bar[stage]);
+            bulk_g2s(st, p.vals + 2 * cur.vo, vbytes, &full_bar[stage]);
+            if (mbytes) bulk_g2s(st + C::kValsBytes, p.meta + cur.mo, mbytes, &full_bar[stage]);
+            const uint16_t *xsrc = p.X + (ts - band * tpr) * B2;
             for (int b = 0; b < p.batch; ++b)
               bulk_g2s(st + C::kValsBytes + C::kMetaBytes + b * C::kXRow,
-                       cur.xsrc + (int64_t)b * p.ldx, xrow, &full_bar[stage]);
+                       xsrc + (int64_t)b * p.ldx, xrow, &full_bar[stage]);
           }
         }
         // every lane keeps the ring position
@@ -816,20 +854,23 @@ __global__ void __launch_bounds__(TmaCfg<BP, B1, B2>::kThreads, 1)
           const int row = o % B1, b = o / B1;
           __stcg(slotp + b * B1 + row, rows[row / C::RW][b * C::RW + row % C::RW]);
         }
-        __threadfence();  // this lane's slot values before the ticket
+        // Each lane fences its own slot stores; the warp barrier then orders
+        // them before lane 0's ticket, whose acquire side (acq_rel) covers the
+        // reads of the other CTAs' slots if this CTA turns out to be last.
+        __threadfence();
         __syncwarp();
         uint32_t last = 0;
         int oA = 0, oB = 0;
         if (lane == 0) {
           oA = owner_of_p(pa);
           oB = owner_of_p(pb);
-          last = atomicAdd(p.counters + r, 1u) == (uint32_t)(oB - oA);
+          last = atom_add_acq_rel(p.counters + r, 1u) == (uint32_t)(oB - oA);
         }
         last = __shfl_sync(0xffffffffu, last, 0);
         oA = __shfl_sync(0xffffffffu, oA, 0);
         oB = __shfl_sync(0xffffffffu, oB, 0);
         if (last) {
-          __threadfence();
+          __syncwarp();
           // sum the band's slots in CTA order; the loads of 4 outputs x 8
           // contributors are issued together, then added in a fixed order
           constexpr int OPL = 4, QMAX = 8;
@@ -979,13 +1020,14 @@ __global__ void __launch_bounds__(TmaCfg<BP, B1, B2>::kThreads, 1)
 }
 
 // ---------------------------------------------------------------------------
-// work-split plan: plan = [G, t0(0), ..., t0(G)], t0(c) the first tile whose
-// packed offset P satisfies P*G >= c*total (the rule the streaming kernel
-// applies when it has no plan)
+// work-split plan (layout next to Params): t0(c) is the first tile whose
+// packed offset P satisfies P*G >= c*total, the rule the streaming kernel
+// applies when it has no plan
 // ---------------------------------------------------------------------------
 __global__ void __launch_bounds__(1024)
-    plan_kernel(const int64_t *__restrict__ val_off, const int64_t *__restrict__ meta_off,
-                int64_t T, int G, int64_t total, int64_t *__restrict__ plan) {
+    plan_starts_kernel(const int64_t *__restrict__ val_off,
+                       const int64_t *__restrict__ meta_off, int64_t T, int G,
+                       int64_t total, int64_t *__restrict__ plan) {
   auto owner = [&](int64_t t) -> int64_t {
     const int64_t o = (2 * val_off[t] + meta_off[t]) * G / total;
     return o < G - 1 ? o : G - 1;
@@ -994,11 +1036,30 @@ __global__ void __launch_bounds__(1024)
        t += (int64_t)gridDim.x * blockDim.x) {
     const int64_t o = owner(t);
     const int64_t prev = t == 0 ? -1 : owner(t - 1);
-    for (int64_t c = prev + 1; c <= o; ++c) plan[1 + c] = t;
+    for (int64_t c = prev + 1; c <= o; ++c) plan[kPlanHead + c * kPlanRec] = t;
   }
-  if (blockIdx.x == 0 && threadIdx.x == 0) {
-    plan[0] = G;
-    plan[1 + G] = T;
+  if (blockIdx.x == 0 && threadIdx.x == 0) plan[0] = G;
+}
+
+// One CTA (32 threads) per record: the range end and the first window.
+__global__ void __launch_bounds__(32)
+    plan_records_kernel(const int64_t *__restrict__ val_off,
+                        const int64_t *__restrict__ meta_off,
+                        const uint8_t *__restrict__ map, int64_t T, int G,
+                        int64_t *__restrict__ plan) {
+  const int c = blockIdx.x, lane = threadIdx.x;
+  int64_t *rec = plan + kPlanHead + (int64_t)c * kPlanRec;
+  const int64_t t0 = rec[0];
+  const int64_t t1 = c + 1 < G ? plan[kPlanHead + (int64_t)(c + 1) * kPlanRec] : T;
+  const int64_t t = min(t0 + lane, T);
+  rec[4 + lane] = val_off[t];
+  rec[36 + lane] = meta_off[t];
+  const bool sp = lane < 31 && t0 + lane < t1 && map[t0 + lane] == 1;
+  const uint32_t bits = __ballot_sync(0xffffffffu, sp);
+  if (lane == 0) {
+    rec[1] = t1;
+    rec[2] = (int64_t)bits;
+    rec[3] = 0;
   }
 }
 
@@ -1223,7 +1284,7 @@ template <int BP, int B1, int B2>
 TmaKernel tma_kernel_info() {
   using C = TmaCfg<BP, B1, B2>;
   return TmaKernel{reinterpret_cast<void *>(&hybrid_tma_kernel<BP, B1, B2>), C::kThreads,
-                   C::kSmem, C::TPS};
+                   C::kSmem, C::TPX};
 }
 
 bool pick_tma_kernel(int bp, Shape s, TmaKernel *out) {
@@ -1437,6 +1498,7 @@ int run_product(Params prm, int b1, int b2, int batch, const hyb_lowrank *lr,
     if (rc != HYB_OK) return rc;
   }
   prm.status = reinterpret_cast<uint32_t *>(w);
+  if (!P.tma || prm.plan_ctas != P.G) prm.plan = nullptr;  // stale or foreign plan
   void *args[] = {&prm};
   if (P.tma) {
     if (cudaLaunchKernel(P.tk.fn, dim3(P.G), dim3(P.tk.threads), args, P.tk.smem, s) !=
@@ -1513,6 +1575,7 @@ int spmm_impl(const hyb_matrix *A, int batch, const uint16_t *X, int64_t ldx,
   prm.ydt = ydt;
   prm.total = 2 * A->n_vals + A->n_meta_bytes;  // packed bytes
   prm.plan = A->plan;
+  prm.plan_ctas = A->plan_ctas;
   return run_product(prm, A->b1, A->b2, batch, lr, false, ws, ws_bytes, s);
 }
 
@@ -1556,11 +1619,13 @@ extern "C" {
 size_t hyb_plan_entries(void) {
   int sms = 0;
   if (device_sm_count(&sms) != HYB_OK) return 0;
-  return (size_t)sms + 2;
+  return (size_t)kPlanHead + (size_t)sms * kPlanRec;
 }
 
-int hyb_make_plan(const hyb_matrix *A, int64_t *plan, hyb_stream_t stream) {
-  if (!A || !plan) return HYB_ERR_INVALID_ARG;
+int hyb_make_plan(const hyb_matrix *A, int64_t *plan, int32_t *plan_ctas,
+                  hyb_stream_t stream) {
+  if (!A || !plan || !plan_ctas) return HYB_ERR_INVALID_ARG;
+  *plan_ctas = 0;
   int rc = check_tiling(A->n, A->k, A->b1, A->b2);
   if (rc != HYB_OK) return rc;
   if (!A->val_off || !A->meta_off || A->num_tiles != (A->n / A->b1) * (A->k / A->b2))
@@ -1581,9 +1646,13 @@ int hyb_make_plan(const hyb_matrix *A, int64_t *plan, hyb_stream_t stream) {
   const int G = (int)std::min<int64_t>(sms, gcap);
   const int64_t T = A->num_tiles;
   const int64_t blocks = std::min<int64_t>((T + 1023) / 1024, 64);
-  plan_kernel<<<(unsigned)std::max<int64_t>(1, blocks), 1024, 0, s>>>(A->val_off, A->meta_off, T,
-                                                                     G, total, plan);
-  return cudaGetLastError() == cudaSuccess ? HYB_OK : HYB_ERR_CUDA;
+  plan_starts_kernel<<<(unsigned)std::max<int64_t>(1, blocks), 1024, 0, s>>>(
+      A->val_off, A->meta_off, T, G, total, plan);
+  if (cudaGetLastError() != cudaSuccess) return HYB_ERR_CUDA;
+  plan_records_kernel<<<G, 32, 0, s>>>(A->val_off, A->meta_off, A->tile_map, T, G, plan);
+  if (cudaGetLastError() != cudaSuccess) return HYB_ERR_CUDA;
+  *plan_ctas = G;
+  return HYB_OK;
 }
 
 size_t hyb_workspace_bytes(const hyb_matrix *A, int batch, int rank) {

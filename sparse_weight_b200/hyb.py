@@ -44,7 +44,7 @@ class HybMatrix(ctypes.Structure):
                 ("tile_map", _P), ("vals", _P), ("meta", _P),
                 ("val_off", _P), ("meta_off", _P),
                 ("n_vals", ctypes.c_int64), ("n_meta_bytes", ctypes.c_int64),
-                ("plan", _P)]
+                ("plan", _P), ("plan_ctas", ctypes.c_int32)]
 
 
 class HybLowrank(ctypes.Structure):
@@ -111,7 +111,7 @@ def lib():
     L.hyb_spmv_noalloc_max_scratch_bytes.restype = _SZ
     L.hyb_plan_entries.argtypes = []
     L.hyb_plan_entries.restype = _SZ
-    L.hyb_make_plan.argtypes = [ctypes.POINTER(HybMatrix), _P, _P]
+    L.hyb_make_plan.argtypes = [ctypes.POINTER(HybMatrix), _P, ctypes.POINTER(ctypes.c_int32), _P]
     L.hyb_make_plan.restype = _I
     L.hyb_status_string.argtypes = [_I]
     L.hyb_status_string.restype = ctypes.c_char_p
@@ -176,6 +176,7 @@ class Packed:
     n_vals: int
     n_meta: int
     plan: Optional[torch.Tensor] = None  # int64 work split (hyb_make_plan), optional
+    plan_ctas: int = 0
 
     @property
     def num_tiles(self) -> int:
@@ -186,7 +187,8 @@ class Packed:
                          self.tile_map.data_ptr(), self.vals.data_ptr(),
                          self.meta.data_ptr(), self.val_off.data_ptr(),
                          self.meta_off.data_ptr(), self.n_vals, self.n_meta,
-                         None if self.plan is None else self.plan.data_ptr())
+                         None if self.plan is None else self.plan.data_ptr(),
+                         self.plan_ctas if self.plan is not None else 0)
 
     def nbytes(self) -> int:
         """Packed bytes the product streams (values + masks)."""
@@ -196,7 +198,7 @@ class Packed:
         return Packed(self.n, self.k, self.b1, self.b2, self.tile_map.clone(),
                       self.vals.clone(), self.meta.clone(), self.val_off.clone(),
                       self.meta_off.clone(), self.n_vals, self.n_meta,
-                      None if self.plan is None else self.plan.clone())
+                      None if self.plan is None else self.plan.clone(), self.plan_ctas)
 
 
 def pack_workspace_bytes() -> int:
@@ -214,14 +216,17 @@ def new_workspace(nbytes: int, device) -> torch.Tensor:
     return ws
 
 
-def make_plan(A: "Packed", stream=None) -> torch.Tensor:
-    """hyb_make_plan: the product's work split for A on the current device."""
+def make_plan(A: "Packed", stream=None):
+    """hyb_make_plan: the product's work split for A on the current device;
+    returns (plan tensor, CTA count)."""
     plan = torch.zeros(int(lib().hyb_plan_entries()), dtype=torch.int64,
                        device=A.val_off.device)
     s = A.struct()
     s.plan = None
-    _check("hyb_make_plan", lib().hyb_make_plan(ctypes.byref(s), _ptr(plan), _stream(stream)))
-    return plan
+    ctas = ctypes.c_int32(0)
+    _check("hyb_make_plan", lib().hyb_make_plan(ctypes.byref(s), _ptr(plan), ctypes.byref(ctas),
+                                                _stream(stream)))
+    return plan, ctas.value
 
 
 def pack(W: torch.Tensor, tile_map, b1: int, b2: int, ws: torch.Tensor = None,
@@ -254,7 +259,7 @@ def pack(W: torch.Tensor, tile_map, b1: int, b2: int, ws: torch.Tensor = None,
         check_status(ws, stream)
     P = Packed(n, k, b1, b2, tm, vals, meta, vo, mo, nv, nm)
     if plan:
-        P.plan = make_plan(P, stream)
+        P.plan, P.plan_ctas = make_plan(P, stream)
     return P
 
 

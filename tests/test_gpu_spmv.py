@@ -191,16 +191,24 @@ def test_plan_matches_definition_and_results(orc, shape):
     P = hyb.pack(W.to(dev()), tmap, b1, b2)
     plan = P.plan.cpu().numpy()
     G = int(plan[0])
+    assert G == P.plan_ctas
     sms = torch.cuda.get_device_properties(0).multi_processor_count
     assert G == min(sms, max(1, (2 * P.n_vals + P.n_meta) // (2 * b1 * b2)))
-    assert plan[1:G + 2].tolist() == _split_reference(orc, n, k, b1, b2, tmap, G)
+    starts = _split_reference(orc, n, k, b1, b2, tmap, G)
+    vo, mo = orc.offsets(n, k, b1, b2, tmap)
+    for c in range(G):
+        rec = plan[8 + 68 * c: 8 + 68 * (c + 1)]
+        t0, t1 = starts[c], starts[c + 1]
+        assert (rec[0], rec[1]) == (t0, t1), c
+        idx = np.minimum(t0 + np.arange(32), T)
+        assert np.array_equal(rec[4:36], vo[idx]) and np.array_equal(rec[36:68], mo[idx]), c
+        bits = sum(1 << i for i in range(min(31, t1 - t0)) if tmap[t0 + i] == 1)
+        assert int(rec[2]) == bits, c
     Xd = X.to(dev())
     y_plan = hyb.spmv(P, Xd)
     saved = P.plan
     P.plan = None
     y_search = hyb.spmv(P, Xd)
-    stale = saved.clone()
-    stale[0] = G + 1  # a plan for another SM count is ignored
-    P.plan = stale
+    P.plan, P.plan_ctas = saved, G + 1  # a plan for another CTA count is ignored
     y_stale = hyb.spmv(P, Xd)
     assert torch.equal(y_plan, y_search) and torch.equal(y_plan, y_stale)
