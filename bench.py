@@ -85,7 +85,7 @@ def csrc_digest():
 def profiled_traffic(workload):
     """DRAM bytes per launch from the committed ncu summary of this workload,
     if it was taken on the current kernel sources; else None."""
-    path = os.path.join(ROOT, "profiles", f"hybrid_stream_kernel_{workload}.md")
+    path = os.path.join(ROOT, "profiles", f"hybrid_tma_kernel_{workload}.md")
     try:
         txt = open(path).read()
     except OSError:
@@ -198,7 +198,16 @@ class Workload:
         self.dfn = L.hyb_gemv_dense
         self.structs = [m.struct() for m in self.mats]
         self.stream = torch.cuda.current_stream(device)
-        s = ctypes.c_void_p(self.stream.cuda_stream)
+        self.set_stream(self.stream)
+        # algorithmic bytes of one product: packed values + masks, tile map, x, y
+        self.bytes_step = base.nbytes() + base.num_tiles + 2 * batch * k + 4 * batch * n
+        self.dense_bytes_step = 2 * n * k + 2 * batch * k + 4 * batch * n
+
+    def set_stream(self, stream):
+        """Marshal every call's arguments for launches on `stream`."""
+        s = ctypes.c_void_p(stream.cuda_stream)
+        n, k, batch = self.n, self.k, self.batch
+        rotate = len(self.mats)
         self.args = [(ctypes.byref(self.structs[i]), batch, ctypes.c_void_p(self.X[i].data_ptr()),
                       k, ctypes.c_void_p(self.Y[i].data_ptr()), n, hyb.HYB_F32, None,
                       ctypes.c_void_p(self.ws.data_ptr()), self.ws.numel(), s)
@@ -208,9 +217,6 @@ class Workload:
                        ctypes.c_void_p(self.Y[i].data_ptr()), n, hyb.HYB_F32,
                        ctypes.c_void_p(self.dws.data_ptr()), self.dws.numel(), s)
                       for i in range(rotate)]
-        # algorithmic bytes of one product: packed values + masks, tile map, x, y
-        self.bytes_step = base.nbytes() + base.num_tiles + 2 * batch * k + 4 * batch * n
-        self.dense_bytes_step = 2 * n * k + 2 * batch * k + 4 * batch * n
 
     def step(self, i):
         rc = self.fn(*self.args[i % len(self.args)])
@@ -245,6 +251,46 @@ def timed(fn, steps, warmup, stream, world=1):
         torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
         ms = float(t.item())
         torch.distributed.barrier()
+    return ms
+
+
+def graph_timed(wl, fn, steps, warmup, world=1):
+    """Device time of `steps` calls captured in one CUDA graph and replayed
+    (the launch path of a decode engine): warm-up calls run eagerly first;
+    CUDA events on the replay stream, barrier + synchronize on both sides, max
+    over ranks."""
+    side = torch.cuda.Stream()
+    with torch.cuda.stream(side):
+        wl.set_stream(side)
+        for i in range(warmup):
+            fn(i)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=side):
+        wl.set_stream(torch.cuda.current_stream())
+        for i in range(steps):
+            fn(warmup + i)
+    wl.set_stream(wl.stream)
+    torch.cuda.synchronize()
+    g.replay()  # one untimed replay: first-launch costs of the graph
+    torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(side):
+        e0.record(side)
+        g.replay()
+        e1.record(side)
+    e1.synchronize()
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1)
+    if world > 1:
+        t = torch.tensor([ms], dtype=torch.float64, device=torch.device("cuda", torch.cuda.current_device()))
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        ms = float(t.item())
+        torch.distributed.barrier()
+    del g
     return ms
 
 
@@ -374,13 +420,15 @@ def main():
     wl = Workload(args.workload, device, rotate=args.rotate)
     stream = wl.stream
 
-    with ClockSampler(local) as clocks:
-        ms = timed(wl.step, args.steps, args.warmup, stream, world)
     if args.profile:
+        ms = timed(wl.step, args.steps, args.warmup, stream, world)
         if rank == 0:
             print(json.dumps({"profile_run": args.workload, "ms": ms, "steps": args.steps}))
         return 0
-    dense_ms = timed(wl.dense_step, args.steps, args.warmup, stream, world)
+    with ClockSampler(local) as clocks:
+        ms = graph_timed(wl, wl.step, args.steps, args.warmup, world)
+    eager_ms = timed(wl.step, args.steps, args.warmup, stream, world)
+    dense_ms = graph_timed(wl, wl.dense_step, args.steps, args.warmup, world)
     e2e_ms, h2d, d2h = e2e_timed(wl, args.steps, args.warmup, stream, world)
 
     per_step_ms = ms / args.steps
@@ -395,13 +443,15 @@ def main():
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
         "config": workload_config(args.workload, wl.frac_real),
         "us_per_matrix": round(per_step_ms * 1e3, 3),
+        "launch": "CUDA graph of the K steps (eager launches: %.3f us per matrix)"
+                  % (eager_ms / args.steps * 1e3),
         "dense_us_per_matrix": round(dense_us, 3),
         "speedup_vs_dense": round(dense_us / (per_step_ms * 1e3), 4),
         "frac_of_nominal_8tbs": round(achieved / NOMINAL_HBM_GBS, 4),
         "roofline": {"bound": "hbm", "achieved": round(achieved, 2), "peak": peak,
                      "unit": "GB/s", "frac": round(achieved / peak, 4),
                      "traffic": profiled_traffic(args.workload),
-                     "peak_kind": peak_kind, "kernel": "hybrid_stream_kernel",
+                     "peak_kind": peak_kind, "kernel": "hybrid_tma_kernel",
                      "bytes_per_launch": wl.bytes_step},
         "e2e": {"value": round(world * wl.bytes_step * args.steps / (e2e_ms * 1e-3) / 1e9, 2),
                 "unit": "GB/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},

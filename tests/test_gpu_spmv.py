@@ -212,3 +212,27 @@ def test_plan_matches_definition_and_results(orc, shape):
     P.plan, P.plan_ctas = saved, G + 1  # a plan for another CTA count is ignored
     y_stale = hyb.spmv(P, Xd)
     assert torch.equal(y_plan, y_search) and torch.equal(y_plan, y_stale)
+
+
+def test_cuda_graph_capture_replay():
+    """hyb_spmm_skinny launches nothing but kernels on the given stream, so it
+    can be captured in a CUDA graph; replays give the eager result."""
+    tmap = inputs.attn_map(1024)
+    W, tmap, X, _ = case(4096, 4096, 128, 128, tmap, batch=2, name="attn_4096")
+    P = hyb.pack(W.to(dev()), tmap, 128, 128)
+    Xd = X.to(dev())
+    ws = hyb.new_workspace(hyb.workspace_bytes(P, 2), dev())
+    y_eager = hyb.spmm_skinny(P, Xd, ws=ws).clone()
+    Y = torch.empty_like(y_eager)
+    side = torch.cuda.Stream()
+    with torch.cuda.stream(side):
+        hyb.spmm_skinny(P, Xd, Y=Y, ws=ws)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=side):
+        hyb.spmm_skinny(P, Xd, Y=Y, ws=ws)
+    Y.zero_()
+    for _ in range(3):
+        g.replay()
+    torch.cuda.synchronize()
+    assert torch.equal(Y, y_eager)
