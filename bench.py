@@ -229,6 +229,20 @@ class Workload:
             raise hyb.HybError("hyb_gemv_dense", rc)
 
 
+def max_over_ranks(ms, device, world):
+    """The slowest rank's time (every rank calls this, in the same order)."""
+    if world <= 1:
+        return ms
+    t = torch.tensor([ms], dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def aggregate_gbs(bytes_per_step, steps, ms, world):
+    """Whole-job throughput: every rank streams its own replica."""
+    return world * bytes_per_step * steps / (ms * 1e-3) / 1e9
+
+
 def timed(fn, steps, warmup, stream, world=1):
     """Device time of `steps` calls (CUDA events on the launching stream),
     barrier + synchronize on both sides, max over ranks."""
@@ -247,9 +261,7 @@ def timed(fn, steps, warmup, stream, world=1):
     torch.cuda.synchronize()
     ms = e0.elapsed_time(e1)
     if world > 1:
-        t = torch.tensor([ms], dtype=torch.float64, device=torch.device("cuda", torch.cuda.current_device()))
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        ms = float(t.item())
+        ms = max_over_ranks(ms, torch.device("cuda", torch.cuda.current_device()), world)
         torch.distributed.barrier()
     return ms
 
@@ -286,9 +298,7 @@ def graph_timed(wl, fn, steps, warmup, world=1):
     torch.cuda.synchronize()
     ms = e0.elapsed_time(e1)
     if world > 1:
-        t = torch.tensor([ms], dtype=torch.float64, device=torch.device("cuda", torch.cuda.current_device()))
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        ms = float(t.item())
+        ms = max_over_ranks(ms, torch.device("cuda", torch.cuda.current_device()), world)
         torch.distributed.barrier()
     del g
     return ms
@@ -432,7 +442,7 @@ def main():
     e2e_ms, h2d, d2h = e2e_timed(wl, args.steps, args.warmup, stream, world)
 
     per_step_ms = ms / args.steps
-    value = world * wl.bytes_step * args.steps / (ms * 1e-3) / 1e9
+    value = aggregate_gbs(wl.bytes_step, args.steps, ms, world)
     achieved = wl.bytes_step / (per_step_ms * 1e-3) / 1e9
     peak, peak_kind = measured_peak()
     dense_us = dense_ms / args.steps * 1e3
@@ -453,7 +463,7 @@ def main():
                      "traffic": profiled_traffic(args.workload),
                      "peak_kind": peak_kind, "kernel": "hybrid_tma_kernel",
                      "bytes_per_launch": wl.bytes_step},
-        "e2e": {"value": round(world * wl.bytes_step * args.steps / (e2e_ms * 1e-3) / 1e9, 2),
+        "e2e": {"value": round(aggregate_gbs(wl.bytes_step, args.steps, e2e_ms, world), 2),
                 "unit": "GB/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "gpu_launches": args.steps,
         "clocks": clocks.summary(),
