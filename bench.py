@@ -389,6 +389,200 @@ def run_reference(args, world, rank):
     return 0
 
 
+# ---------------------------------------------------------------------------
+# --sweep: the other measurements (one JSON line each, not the headline)
+# ---------------------------------------------------------------------------
+
+FP32_FMA_PER_SM_PER_CLK = 128   # fp32 lanes per SM (B200)
+
+
+class Calls:
+    """A rotation of pre-marshalled C-ABI calls (for graph_timed)."""
+
+    def __init__(self, fn, make_args, count, name):
+        self.fn, self.make_args, self.count, self.name = fn, make_args, count, name
+        self.stream = torch.cuda.current_stream()
+        self.set_stream(self.stream)
+
+    def set_stream(self, stream):
+        sp = ctypes.c_void_p(stream.cuda_stream)
+        self.args = [self.make_args(i, sp) for i in range(self.count)]
+
+    def step(self, i):
+        rc = self.fn(*self.args[i % self.count])
+        if rc != 0:
+            raise hyb.HybError(self.name, rc)
+
+
+def _alu_roofline(flops, us, sm_mhz):
+    peak = 148 * FP32_FMA_PER_SM_PER_CLK * 2 * sm_mhz * 1e6 / 1e12  # TFLOP/s
+    achieved = flops / (us * 1e-6) / 1e12
+    return {"bound": "alu", "achieved": round(achieved, 2), "peak": round(peak, 1),
+            "unit": "TFLOP/s", "frac": round(achieved / peak, 4),
+            "peak_kind": f"148 SMs x 128 fp32 lanes x 2 x {sm_mhz:.0f} MHz"}
+
+
+def sweep(device, steps=200, warmup=10):
+    """Hybrid vs dense on the FFN shapes across 2:4-tile fractions and batches,
+    the 4096x4096 attention matrix, the 32-layer Llama-3.1-8B chain (224
+    matrices, one CUDA graph) and the Llama-3.3-70B FFN with the fused
+    rank-128 low-rank term."""
+    peak, peak_kind = measured_peak()
+    L = hyb.lib()
+    l2 = 126 << 20
+    sm_mhz = 1965.0
+
+    def rot_count(nbytes):
+        return max(2, int(np.ceil(3 * l2 / nbytes)))
+
+    def emit(d):
+        print(json.dumps(d), flush=True)
+
+    # ---- FFN shapes x fraction x batch, and the attention matrix ----
+    shapes = [("ffn_up", 14336, 4096, [0.0, 0.25, 0.5, 0.75, 1.0]),
+              ("ffn_down", 4096, 14336, [0.0, 0.25, 0.5, 0.75, 1.0]),
+              ("attn", 4096, 4096, ["bern0.5"])]
+    for role, n, k, fracs in shapes:
+        W = inputs.weight(n, k, 0.02, inputs.seed_of("ffn_sweep", n, k, "W"),
+                          outliers=0.01 if role != "attn" else 0.0)
+        Wd = W.to(device)
+        nrot_d = rot_count(2 * n * k)
+        dense = [Wd] + [Wd.clone() for _ in range(nrot_d - 1)]
+        Xs = {b: [inputs.activations(b, k, inputs.seed_of("sweep", n, k, b, i)).to(device)
+                  for i in range(max(nrot_d, 16))] for b in (1, 4, 8, 16)}
+        Ys = {b: [torch.empty(b, n, dtype=torch.float32, device=device)
+                  for _ in range(max(nrot_d, 16))] for b in (1, 4, 8, 16)}
+        dense_us = {}
+        for b in ((1,) if role == "attn" else (1, 4, 8, 16)):
+            dws = hyb.new_workspace(hyb.dense_workspace_bytes(n, k, b), device)
+            c = Calls(L.hyb_gemv_dense, lambda i, sp, b=b, dws=dws: (
+                n, k, b, ctypes.c_void_p(dense[i].data_ptr()), k,
+                ctypes.c_void_p(Xs[b][i].data_ptr()), k, ctypes.c_void_p(Ys[b][i].data_ptr()), n,
+                hyb.HYB_F32, ctypes.c_void_p(dws.data_ptr()), dws.numel(), sp), nrot_d, "dense")
+            dense_us[b] = graph_timed(c, c.step, steps, warmup) / steps * 1e3
+        del dense
+        for f in fracs:
+            T = (n // 128) * (k // 128)
+            if f == "bern0.5":
+                tmap = inputs.attn_map(T)
+            else:
+                tmap = inputs.tile_map_fraction(T, f, inputs.seed_of("ffn_sweep", n, k, f))
+            base = hyb.pack(Wd, tmap, 128, 128)
+            nrot = rot_count(base.nbytes())
+            mats = [base] + [base.clone() for _ in range(nrot - 1)]
+            structs = [m.struct() for m in mats]
+            for b in ((1,) if role == "attn" else (1, 4, 8, 16)):
+                ws = hyb.new_workspace(hyb.workspace_bytes(base, b), device)
+                xs, ys = Xs[b], Ys[b]
+                c = Calls(L.hyb_spmm_skinny, lambda i, sp, b=b, ws=ws, xs=xs, ys=ys: (
+                    ctypes.byref(structs[i]), b, ctypes.c_void_p(xs[i % len(xs)].data_ptr()), k,
+                    ctypes.c_void_p(ys[i % len(ys)].data_ptr()), n, hyb.HYB_F32, None,
+                    ctypes.c_void_p(ws.data_ptr()), ws.numel(), sp), nrot, "hybrid")
+                us = graph_timed(c, c.step, steps, warmup) / steps * 1e3
+                nbytes = base.nbytes() + base.num_tiles + 2 * b * k + 4 * b * n
+                gbs = nbytes / (us * 1e-6) / 1e9
+                kept = base.n_vals  # kept entries = packed values
+                line = {"sweep": "ffn" if role != "attn" else "attn", "shape": f"{n}x{k}",
+                        "tile": "128x128", "sparse_tile_frac": float(np.mean(tmap)), "batch": b,
+                        "us": round(us, 3), "GBps": round(gbs, 1),
+                        "frac_of_measured_hbm": round(gbs / peak, 4),
+                        "frac_of_8tbs": round(gbs / NOMINAL_HBM_GBS, 4),
+                        "dense_us": round(dense_us[b], 3),
+                        "speedup_vs_dense": round(dense_us[b] / us, 4),
+                        "format_bound_speedup": round((2 * n * k) / base.nbytes(), 4)}
+                if b >= 8:
+                    line["alu_roofline"] = _alu_roofline(2 * b * kept, us, sm_mhz)
+                emit(line)
+                del ws
+            del mats, structs, base
+        del Wd, Xs, Ys
+        torch.cuda.empty_cache()
+
+    # ---- 32-layer Llama-3.1-8B chain, 224 matrices in one CUDA graph ----
+    W_role = {role: inputs.weight(n, k, 0.02, inputs.seed_of("llama8b_chain", role, "W")).to(device)
+              for role, n, k in inputs.LLAMA8B_LAYER}
+    mats, shapes8 = [], []
+    for layer in range(32):
+        f = inputs.chain_fraction(layer)
+        for role, n, k in inputs.LLAMA8B_LAYER:
+            T = (n // 128) * (k // 64)
+            tmap = inputs.tile_map_fraction(T, f, inputs.seed_of("llama8b_chain", layer, role, "map"))
+            mats.append(hyb.pack(W_role[role], tmap, 128, 64))
+            shapes8.append((n, k))
+    xs = [inputs.activations(1, k, inputs.seed_of("chain", i)).to(device) for i, (n, k) in enumerate(shapes8)]
+    ys = [torch.empty(1, n, dtype=torch.float32, device=device) for n, k in shapes8]
+    ws = hyb.new_workspace(max(hyb.workspace_bytes(m, 1) for m in mats), device)
+    structs = [m.struct() for m in mats]
+    chain = Calls(L.hyb_spmm_skinny, lambda i, sp: (
+        ctypes.byref(structs[i]), 1, ctypes.c_void_p(xs[i].data_ptr()), shapes8[i][1],
+        ctypes.c_void_p(ys[i].data_ptr()), shapes8[i][0], hyb.HYB_F32, None,
+        ctypes.c_void_p(ws.data_ptr()), ws.numel(), sp), len(mats), "chain")
+    reps = 4
+    ms = graph_timed(chain, chain.step, reps * len(mats), len(mats))
+    packed = sum(m.nbytes() + m.num_tiles for m in mats)
+    nbytes = packed + sum(2 * k + 4 * n for n, k in shapes8)
+    dws = hyb.new_workspace(max(hyb.dense_workspace_bytes(n, k, 1) for n, k in shapes8), device)
+    roles8 = [r for _ in range(32) for r, _, _ in inputs.LLAMA8B_LAYER]
+    dchain = Calls(L.hyb_gemv_dense, lambda i, sp: (
+        shapes8[i][0], shapes8[i][1], 1, ctypes.c_void_p(W_role[roles8[i]].data_ptr()), shapes8[i][1],
+        ctypes.c_void_p(xs[i].data_ptr()), shapes8[i][1], ctypes.c_void_p(ys[i].data_ptr()),
+        shapes8[i][0], hyb.HYB_F32, ctypes.c_void_p(dws.data_ptr()), dws.numel(), sp),
+        len(mats), "dense chain")
+    dms = graph_timed(dchain, dchain.step, reps * len(mats), len(mats))
+    us_chain = ms / reps * 1e3
+    emit({"sweep": "llama8b_chain", "matrices": len(mats), "tile": "128x64", "batch": 1,
+          "us_per_chain": round(us_chain, 2), "us_per_matrix": round(us_chain / len(mats), 3),
+          "GBps": round(nbytes / (us_chain * 1e-6) / 1e9, 1), "packed_GB": round(packed / 1e9, 3),
+          "dense_us_per_chain": round(dms / reps * 1e3, 2),
+          "speedup_vs_dense": round(dms / ms, 4),
+          "note": "one weight draw per role; tile maps drawn per layer (f_l ~ U[0.2,1])"})
+    del mats, structs, W_role, xs, ys, ws, dws
+    torch.cuda.empty_cache()
+
+    # ---- Llama-3.3-70B FFN, all 2:4, rank-128 low-rank term, 8 layers ----
+    mats70, lrs, sh70 = [], [], []
+    for role, n, k in inputs.LLAMA70B_FFN:
+        T = (n // 128) * (k // 128)
+        W = inputs.weight(n, k, 0.015, inputs.seed_of("llama70b", role, "W")).to(device)
+        base = hyb.pack(W, np.ones(T, np.uint8), 128, 128)
+        del W
+        U, V = inputs.lowrank(n, k, 128, 0.01, inputs.seed_of("llama70b", role, "LR"))
+        lr = (U.to(device), V.to(device))
+        for layer in range(8):
+            mats70.append(base if layer == 0 else base.clone())
+            lrs.append(lr)
+            sh70.append((n, k))
+    mats70 = [mats70[(i % 3) * 8 + i // 3] for i in range(24)]
+    lrs = [lrs[(i % 3) * 8 + i // 3] for i in range(24)]
+    sh70 = [sh70[(i % 3) * 8 + i // 3] for i in range(24)]
+    structs = [m.struct() for m in mats70]
+    lrstructs = [hyb.HybLowrank(128, hyb._bits(U).data_ptr(), 128, hyb._bits(V).data_ptr(), 128)
+                 for U, V in lrs]
+    for b in (1, 8, 16):
+        xs = [inputs.activations(b, k, inputs.seed_of("l70", i, b)).to(device) for i, (n, k) in enumerate(sh70)]
+        ys = [torch.empty(b, n, dtype=torch.float32, device=device) for n, k in sh70]
+        ws = hyb.new_workspace(max(hyb.workspace_bytes(m, b, 128) for m in mats70), device)
+        c = Calls(L.hyb_spmm_skinny, lambda i, sp, b=b, ws=ws, xs=xs, ys=ys: (
+            ctypes.byref(structs[i]), b, ctypes.c_void_p(xs[i].data_ptr()), sh70[i][1],
+            ctypes.c_void_p(ys[i].data_ptr()), sh70[i][0], hyb.HYB_F32, ctypes.byref(lrstructs[i]),
+            ctypes.c_void_p(ws.data_ptr()), ws.numel(), sp), 24, "70b")
+        ms = graph_timed(c, c.step, 48, 24)
+        us = ms / 2 * 1e3
+        nbytes = sum(m.nbytes() + m.num_tiles + 2 * b * k + 4 * b * n + 2 * 128 * (n + k)
+                     for m, (n, k) in zip(mats70, sh70))
+        gbs = nbytes / (us * 1e-6) / 1e9
+        line = {"sweep": "llama70b_ffn_lowrank", "matrices": 24, "batch": b, "rank": 128,
+                "us_per_8_layers": round(us, 2), "us_per_matrix": round(us / 24, 3),
+                "GBps": round(gbs, 1), "frac_of_measured_hbm": round(gbs / peak, 4)}
+        if b >= 8:
+            kept = sum(m.n_vals for m in mats70)
+            flops = 2 * b * kept + sum(2 * b * 128 * (n + k) for n, k in sh70)
+            line["alu_roofline"] = _alu_roofline(flops, us, sm_mhz)
+        emit(line)
+        del ws, xs, ys
+    return 0
+
+
 def workload_config(name, frac_real):
     n, k, b1, b2, frac, batch, std, outliers = WORKLOADS[name]
     return {"workload": name, "n": n, "k": k, "tile": f"{b1}x{b2}",
@@ -410,6 +604,9 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--rotate", type=int, default=ROTATE,
                     help="packed copies cycled through (their total must exceed L2)")
+    ap.add_argument("--sweep", action="store_true",
+                    help="print the fraction / batch sweep, the 224-matrix chain and the 70B "
+                         "low-rank lines instead of the headline line")
     ap.add_argument("--profile", action="store_true",
                     help="small case for a profiler: 2 rotating copies (184 MB > L2), "
                          "hybrid product only, no dense / end-to-end / CPU legs")
@@ -427,6 +624,8 @@ def main():
         import datetime
         torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                              device_id=device)
+    if args.sweep:
+        return sweep(device)
     wl = Workload(args.workload, device, rotate=args.rotate)
     stream = wl.stream
 
