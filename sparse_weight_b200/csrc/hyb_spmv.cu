@@ -57,11 +57,13 @@ struct Params {
   void *Y;
   int64_t ldy;
   int ydt;
-  // low rank (t = V^T x already computed into lr_t[batch][rank])
+  // low rank: t = V^T x and then ut = U t (fp32 [batch][n]) are computed by
+  // two small kernels before the product; the product's epilogue adds ut
   const uint16_t *U;
   int64_t ldu;
   int rank;
   const float *lr_t;
+  const float *lr_ut;
   // split
   int G;
   int64_t total;  // packed bytes of the whole matrix
@@ -121,33 +123,7 @@ __device__ __forceinline__ int owner_of(int64_t P, const Params &p) {
 // Epilogue for one (row, batch) output: add the low-rank term, store.
 __device__ __forceinline__ void store_out(const Params &p, int64_t row, int b,
                                           float y) {
-  if (p.rank > 0) {
-    const uint16_t *u = p.U + row * p.ldu;
-    const float *t = p.lr_t + (int64_t)b * p.rank;
-    float s = 0.f;
-    // 64 factor entries per round: their loads are issued together
-    for (int j0 = 0; j0 < p.rank; j0 += 64) {
-      uint4 uv[8];
-#pragma unroll
-      for (int q = 0; q < 8; ++q)
-        uv[q] = j0 + 8 * q < p.rank ? __ldg(reinterpret_cast<const uint4 *>(u + j0 + 8 * q))
-                                    : make_uint4(0, 0, 0, 0);
-#pragma unroll
-      for (int q = 0; q < 8; ++q) {
-        if (j0 + 8 * q >= p.rank) break;
-        const float *tq = t + j0 + 8 * q;
-        s = fmaf(bf16_lo(uv[q].x), tq[0], s);
-        s = fmaf(bf16_hi(uv[q].x), tq[1], s);
-        s = fmaf(bf16_lo(uv[q].y), tq[2], s);
-        s = fmaf(bf16_hi(uv[q].y), tq[3], s);
-        s = fmaf(bf16_lo(uv[q].z), tq[4], s);
-        s = fmaf(bf16_hi(uv[q].z), tq[5], s);
-        s = fmaf(bf16_lo(uv[q].w), tq[6], s);
-        s = fmaf(bf16_hi(uv[q].w), tq[7], s);
-      }
-    }
-    y += s;
-  }
+  if (p.lr_ut != nullptr) y += p.lr_ut[(int64_t)b * p.n + row];
   if (p.ydt == HYB_BF16)
     reinterpret_cast<uint16_t *>(p.Y)[(int64_t)b * p.ldy + row] =
         f32_to_bf16_rne(y);
@@ -1224,6 +1200,36 @@ __global__ void __launch_bounds__(kThreads)
   for (int b = 0; b < batch; ++b) Y[b * ldy + i] += acc[b];
 }
 
+// ut[b][i] = sum_j U[i][j] t[b][j] (fp32), one thread per row; U is read once.
+template <int BP>
+__global__ void __launch_bounds__(kThreads)
+    lowrank_ut_kernel(int64_t n, const uint16_t *__restrict__ U, int64_t ldu, int rank,
+                      const float *__restrict__ t, int batch, float *__restrict__ ut) {
+  const int64_t i = (int64_t)blockIdx.x * kThreads + threadIdx.x;
+  if (i >= n) return;
+  float acc[BP];
+#pragma unroll
+  for (int b = 0; b < BP; ++b) acc[b] = 0.f;
+  for (int j0 = 0; j0 < rank; j0 += 64) {
+    uint4 uv[8];
+#pragma unroll
+    for (int q = 0; q < 8; ++q)
+      uv[q] = j0 + 8 * q < rank ? __ldg(reinterpret_cast<const uint4 *>(U + i * ldu + j0 + 8 * q))
+                                : make_uint4(0, 0, 0, 0);
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+      if (j0 + 8 * q >= rank) break;
+      const float uf[8] = {bf16_lo(uv[q].x), bf16_hi(uv[q].x), bf16_lo(uv[q].y), bf16_hi(uv[q].y),
+                           bf16_lo(uv[q].z), bf16_hi(uv[q].z), bf16_lo(uv[q].w), bf16_hi(uv[q].w)};
+#pragma unroll
+      for (int b = 0; b < BP; ++b)
+#pragma unroll
+        for (int e = 0; e < 8; ++e) acc[b] = fmaf(uf[e], t[b * rank + j0 + 8 * q + e], acc[b]);
+    }
+  }
+  for (int b = 0; b < batch; ++b) ut[(int64_t)b * n + i] = acc[b];
+}
+
 // ---------------------------------------------------------------------------
 // host side
 // ---------------------------------------------------------------------------
@@ -1329,6 +1335,16 @@ void *pick_lowrank_t(int bp) {
   }
 }
 
+void *pick_lowrank_ut(int bp) {
+  switch (bp) {
+    case 1: return reinterpret_cast<void *>(&lowrank_ut_kernel<1>);
+    case 2: return reinterpret_cast<void *>(&lowrank_ut_kernel<2>);
+    case 4: return reinterpret_cast<void *>(&lowrank_ut_kernel<4>);
+    case 8: return reinterpret_cast<void *>(&lowrank_ut_kernel<8>);
+    default: return reinterpret_cast<void *>(&lowrank_ut_kernel<16>);
+  }
+}
+
 void *pick_lowrank_apply(int bp) {
   switch (bp) {
     case 1: return reinterpret_cast<void *>(&lowrank_apply_kernel<1>);
@@ -1381,7 +1397,7 @@ struct Plan {
   int R;           // bands
   int64_t total;   // packed bytes
   int lr_ctas;     // CTAs of the low-rank reduction
-  size_t off_counters, off_lr_t, off_lr_part, off_lr_counter, off_partials,
+  size_t off_counters, off_lr_t, off_lr_part, off_lr_counter, off_lr_ut, off_partials,
       bytes;
   size_t dyn_smem;
 };
@@ -1436,6 +1452,8 @@ int make_plan(int64_t n, int64_t k, int b1, int b2, int64_t total_bytes,
   off = align_up(off + (size_t)P.lr_ctas * P.bp * (rank > 0 ? rank : 0) * sizeof(float), 256);
   P.off_lr_counter = off;
   off = align_up(off + sizeof(uint32_t), 256);
+  P.off_lr_ut = off;
+  off = align_up(off + (size_t)P.bp * (rank > 0 ? n : 0) * sizeof(float), 256);
   P.off_partials = off;
   if (P.tma || P.stream) off += (size_t)(P.G + P.R) * b1 * P.bp * sizeof(float);
   P.bytes = align_up(off, 256);
@@ -1493,9 +1511,21 @@ int run_product(Params prm, int b1, int b2, int batch, const hyb_lowrank *lr,
   prm.U = rank ? lr->U : nullptr;
   prm.ldu = rank ? lr->ldu : 0;
   prm.lr_t = reinterpret_cast<const float *>(w + P.off_lr_t);
+  prm.lr_ut = nullptr;
   if (rank) {
     rc = launch_lowrank_t(P, lr, prm.k, prm.X, prm.ldx, batch, w, s);
     if (rc != HYB_OK) return rc;
+    int64_t nn = prm.n, ldu = lr->ldu;
+    const uint16_t *U = lr->U;
+    int rk = rank, bt = batch;
+    const float *tp = prm.lr_t;
+    float *ut = reinterpret_cast<float *>(w + P.off_lr_ut);
+    void *uargs[] = {&nn, &U, &ldu, &rk, &tp, &bt, &ut};
+    const int64_t grid = (prm.n + kThreads - 1) / kThreads;
+    if (cudaLaunchKernel(pick_lowrank_ut(P.bp), dim3((unsigned)grid), dim3(kThreads), uargs, 0, s) !=
+        cudaSuccess)
+      return HYB_ERR_CUDA;
+    prm.lr_ut = ut;
   }
   prm.status = reinterpret_cast<uint32_t *>(w);
   if (!P.tma || prm.plan_ctas != P.G) prm.plan = nullptr;  // stale or foreign plan
