@@ -82,10 +82,16 @@ def csrc_digest():
     return h.hexdigest()[:16]
 
 
-def profiled_traffic(workload):
+def kernel_of(P):
+    """Streaming kernel the product runs for P: the TMA-ring kernel when the
+    library made a split for it (plan with CTAs), else the generic one."""
+    return "hybrid_tma_kernel" if P.plan is not None and P.plan_ctas > 0 else "hybrid_rowwarp_kernel"
+
+
+def profiled_traffic(workload, kernel):
     """DRAM bytes per launch from the committed ncu summary of this workload,
     if it was taken on the current kernel sources; else None."""
-    path = os.path.join(ROOT, "profiles", f"hybrid_tma_kernel_{workload}.md")
+    path = os.path.join(ROOT, "profiles", f"{kernel}_{workload}.md")
     try:
         txt = open(path).read()
     except OSError:
@@ -645,6 +651,7 @@ def main():
     achieved = wl.bytes_step / (per_step_ms * 1e-3) / 1e9
     peak, peak_kind = measured_peak()
     dense_us = dense_ms / args.steps * 1e3
+    kernel = kernel_of(wl.mats[0])
     line = {
         "metric": "hybrid 2:4 GEMV achieved HBM GB/s (algorithmic bytes)",
         "value": round(value, 2), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
@@ -659,8 +666,8 @@ def main():
         "frac_of_nominal_8tbs": round(achieved / NOMINAL_HBM_GBS, 4),
         "roofline": {"bound": "hbm", "achieved": round(achieved, 2), "peak": peak,
                      "unit": "GB/s", "frac": round(achieved / peak, 4),
-                     "traffic": profiled_traffic(args.workload),
-                     "peak_kind": peak_kind, "kernel": "hybrid_tma_kernel",
+                     "traffic": profiled_traffic(args.workload, kernel),
+                     "peak_kind": peak_kind, "kernel": kernel,
                      "bytes_per_launch": wl.bytes_step},
         "e2e": {"value": round(aggregate_gbs(wl.bytes_step, args.steps, e2e_ms, world), 2),
                 "unit": "GB/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},

@@ -101,9 +101,9 @@ typedef struct {
   const int64_t *meta_off;  /* [num_tiles + 1] */
   int64_t n_vals;           /* val_off[num_tiles], as given by hyb_packed_sizes */
   int64_t n_meta_bytes;     /* meta_off[num_tiles], as given by hyb_packed_sizes */
-  const int64_t *plan;      /* optional (may be NULL): work split made by
-                               hyb_make_plan for this matrix on this device;
-                               saves the products a search at every call */
+  const int64_t *plan;      /* optional, HOST memory (may be NULL): the work
+                               split hyb_make_plan made for this matrix on this
+                               device; saves the products their start-up search */
   int32_t plan_ctas;        /* the CTA count hyb_make_plan reported for plan */
 } hyb_matrix;
 
@@ -144,18 +144,22 @@ HYB_API int hyb_pack(int64_t n, int64_t k, int b1, int b2, const uint16_t *W,
 
 /* ---- work split -------------------------------------------------------- */
 
-/* Entries of a plan buffer (int64_t) for hyb_make_plan on the current device. */
+/* Entries (int64_t) of each of hyb_make_plan's two buffers on the current
+ * device. */
 HYB_API size_t hyb_plan_entries(void);
 
-/* Write into `plan` (device, hyb_plan_entries() int64_t) the split of A's
- * packed bytes over the streaming kernel's CTAs on the current device (CTA c
- * takes the tiles whose packed byte offset falls in [c, c+1) * total / G),
- * together with each CTA's first tile offsets, and store G in *plan_ctas
- * (0 when the tiling has no streaming kernel).  Set A->plan / A->plan_ctas
- * from these to let the products skip their start-up search; the products
- * ignore a plan whose plan_ctas differs from the CTA count they would use. */
-HYB_API int hyb_make_plan(const hyb_matrix *A, int64_t *plan, int32_t *plan_ctas,
-                          hyb_stream_t stream);
+/* Work out, once per matrix, how the streaming kernel splits A's packed bytes
+ * over its CTAs on the current device: CTA c takes the tiles whose packed byte
+ * offset falls in [c, c+1) * total / G.  `scratch` is a device buffer and
+ * `plan_host` a host buffer, both of hyb_plan_entries() int64_t; on return
+ * plan_host holds, for every CTA, its first and end tile, the packed offsets
+ * of its first tile and the 2:4 bits of its first 31 tiles, and *plan_ctas
+ * holds G (0 when the tiling has no streaming kernel).  Synchronises
+ * `stream`.  Point A->plan / A->plan_ctas at the result: the products then
+ * start streaming without any global-memory load, and ignore a plan whose
+ * plan_ctas differs from the CTA count they would use. */
+HYB_API int hyb_make_plan(const hyb_matrix *A, int64_t *scratch, int64_t *plan_host,
+                          int32_t *plan_ctas, hyb_stream_t stream);
 
 /* ---- products ---------------------------------------------------------- */
 

@@ -70,15 +70,23 @@ struct Params {
   float *partials;
   uint32_t *counters;
   uint32_t *status;  // workspace status word
-  const int64_t *plan;  // optional precomputed split (validated by the host)
-  int plan_ctas;
+  int64_t nvb, nmb;  // bytes of the value and mask buffers
 };
 
-// Plan layout (int64): [0] = G, [1..7] reserved, then one record per CTA:
-// [t0, t1, 2:4 bitmask of tiles t0..t0+30, 0, val_off[t0..t0+31],
-//  meta_off[t0..t0+31]] (offsets clamped at the last tile).
+// Work split made once per matrix (hyb_make_plan) and handed to the streaming
+// kernel as launch parameters, so that a CTA issues its first copy without
+// any global-memory load.  Host layout (int64): [0] = G, [1] = kind (1),
+// [2..7] reserved, then G + 1 records {t0, val_off[t0], meta_off[t0], 2:4
+// bits of tiles t0 .. t0 + 30}, t0 being the CTA's first tile; record G
+// holds the end (T).
+constexpr int kMaxCtas = 160;
 constexpr int kPlanHead = 8;
-constexpr int kPlanRec = 68;
+constexpr int32_t kPlanTiles = 1;
+struct LaunchPlan {
+  int32_t kind;  // 0: none (the kernel searches for its range)
+  int32_t ctas;
+  int64_t rec[4 * (kMaxCtas + 1)];
+};
 
 // ---------------------------------------------------------------------------
 // helpers
@@ -546,7 +554,7 @@ struct StageDesc {
 
 template <int BP, int B1, int B2>
 __global__ void __launch_bounds__(TmaCfg<BP, B1, B2>::kThreads, 1)
-    hybrid_tma_kernel(const Params p) {
+    hybrid_tma_kernel(const Params p, const LaunchPlan lp) {
   using C = TmaCfg<BP, B1, B2>;
   constexpr int S = C::kStages;
   extern __shared__ __align__(1024) uint8_t smem[];
@@ -595,11 +603,11 @@ __global__ void __launch_bounds__(TmaCfg<BP, B1, B2>::kThreads, 1)
 
   // ---- this CTA's tiles [t0, t1): tiles whose packed offset P(t) satisfies
   // c*total <= P(t)*G < (c+1)*total.  With a plan the producer and the
-  // epilogue warp read them from the CTA's record; otherwise round 1
+  // epilogue warp take them from the launch parameters; otherwise round 1
   // brackets both ends between band starts and round 2 counts inside the
   // bracketing band. ----
-  const int64_t *rec = p.plan ? p.plan + kPlanHead + (int64_t)c * kPlanRec : nullptr;
-  if (rec == nullptr) {
+  const bool planned = lp.kind == kPlanTiles;
+  if (!planned) {
       const int64_t tgtA = (int64_t)c * p.total, tgtB = (int64_t)(c + 1) * p.total;
       uint32_t ca = 0, cb = 0;
       for (int i = tid; i <= p.R; i += blockDim.x) {
@@ -652,12 +660,12 @@ __global__ void __launch_bounds__(TmaCfg<BP, B1, B2>::kThreads, 1)
   // consumers never need the range; the producer and the epilogue warp take
   // it from the plan record when there is one
   int64_t t0 = 0, t1 = 0;
-  if (rec == nullptr) {
+  if (!planned) {
     t0 = s_range[0];
     t1 = s_range[1];
   } else if (warp >= C::NC) {
-    t0 = __ldg(rec + 0);
-    t1 = __ldg(rec + 1);
+    t0 = lp.rec[4 * c];
+    t1 = lp.rec[4 * (c + 1)];
   }
 
   if (warp == C::NC) {
@@ -687,14 +695,23 @@ __global__ void __launch_bounds__(TmaCfg<BP, B1, B2>::kThreads, 1)
     bool ok = true;
     uint32_t armed = 0, armed_parity = 0;  // per stage: copies issued / phase parity
     Win cur;
-    if (rec != nullptr) {
-      // first window straight from the plan record (same round trip as t0)
-      cur.vo = __ldg(rec + 4 + lane);
-      cur.mo = __ldg(rec + 36 + lane);
-      cur.sp = (uint32_t)(__ldg(rec + 2) >> lane) & 1u;
-    } else {
-      cur = load_win(t0);
+    bool derived = false;
+    if (planned) {
+      // first window from the plan: offsets of tile t0 + lane follow from
+      // those of t0 and the 2:4 bits of the tiles before it
+      constexpr int64_t TE = (int64_t)B1 * B2;
+      const uint32_t bits = (uint32_t)lp.rec[4 * c + 3];
+      const int nb = __popc(bits & ((1u << lane) - 1u));
+      cur.vo = lp.rec[4 * c + 1] + (int64_t)lane * TE - nb * (TE / 2);
+      cur.mo = lp.rec[4 * c + 2] + nb * (TE / 8);
+      cur.sp = lane < C::WIN ? (bits >> lane) & 1u : 0u;
+      // a plan that does not fit the buffers is not used
+      const int nw = (int)min((int64_t)C::WIN, t1 - t0);
+      derived = 2 * __shfl_sync(0xffffffffu, cur.vo, nw) <= p.nvb &&
+                __shfl_sync(0xffffffffu, cur.mo, nw) <= p.nmb && cur.vo >= 0;
+      derived = __all_sync(0xffffffffu, derived);
     }
+    if (!derived) cur = load_win(t0);
     for (int64_t w0 = t0; ok && w0 < t1; w0 += C::WIN) {
       const Win nxt = load_win(w0 + C::WIN);  // in flight while this window issues
       const int nw = (int)min((int64_t)C::WIN, t1 - w0);
@@ -996,47 +1013,40 @@ __global__ void __launch_bounds__(TmaCfg<BP, B1, B2>::kThreads, 1)
 }
 
 // ---------------------------------------------------------------------------
-// work-split plan (layout next to Params): t0(c) is the first tile whose
-// packed offset P satisfies P*G >= c*total, the rule the streaming kernel
-// applies when it has no plan
+// work-split plan: one thread per CTA boundary c in [0, G], by the same rules
+// the streaming kernels apply when they search for their own range
 // ---------------------------------------------------------------------------
-__global__ void __launch_bounds__(1024)
-    plan_starts_kernel(const int64_t *__restrict__ val_off,
-                       const int64_t *__restrict__ meta_off, int64_t T, int G,
-                       int64_t total, int64_t *__restrict__ plan) {
-  auto owner = [&](int64_t t) -> int64_t {
-    const int64_t o = (2 * val_off[t] + meta_off[t]) * G / total;
-    return o < G - 1 ? o : G - 1;
+__global__ void __launch_bounds__(128)
+    plan_kernel(const int64_t *__restrict__ val_off, const int64_t *__restrict__ meta_off,
+                const uint8_t *__restrict__ map, int64_t T, int G, int64_t total,
+                int64_t *__restrict__ plan) {
+  const int c = blockIdx.x * blockDim.x + threadIdx.x;
+  if (c > G) return;
+  auto P = [&](int64_t t) -> int64_t { return 2 * val_off[t] + meta_off[t]; };
+  if (c == 0) {
+    plan[0] = G;
+    plan[1] = kPlanTiles;
+    for (int i = 2; i < kPlanHead; ++i) plan[i] = 0;
+  }
+  auto first_tile = [&](int64_t tg) -> int64_t {  // first t with P(t) G >= tg
+    int64_t lo = 0, hi = T;
+    while (lo < hi) {
+      const int64_t mid = (lo + hi) / 2;
+      if (P(mid) * G < tg) lo = mid + 1;
+      else hi = mid;
+    }
+    return lo;
   };
-  for (int64_t t = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; t < T;
-       t += (int64_t)gridDim.x * blockDim.x) {
-    const int64_t o = owner(t);
-    const int64_t prev = t == 0 ? -1 : owner(t - 1);
-    for (int64_t c = prev + 1; c <= o; ++c) plan[kPlanHead + c * kPlanRec] = t;
-  }
-  if (blockIdx.x == 0 && threadIdx.x == 0) plan[0] = G;
-}
-
-// One CTA (32 threads) per record: the range end and the first window.
-__global__ void __launch_bounds__(32)
-    plan_records_kernel(const int64_t *__restrict__ val_off,
-                        const int64_t *__restrict__ meta_off,
-                        const uint8_t *__restrict__ map, int64_t T, int G,
-                        int64_t *__restrict__ plan) {
-  const int c = blockIdx.x, lane = threadIdx.x;
-  int64_t *rec = plan + kPlanHead + (int64_t)c * kPlanRec;
-  const int64_t t0 = rec[0];
-  const int64_t t1 = c + 1 < G ? plan[kPlanHead + (int64_t)(c + 1) * kPlanRec] : T;
-  const int64_t t = min(t0 + lane, T);
-  rec[4 + lane] = val_off[t];
-  rec[36 + lane] = meta_off[t];
-  const bool sp = lane < 31 && t0 + lane < t1 && map[t0 + lane] == 1;
-  const uint32_t bits = __ballot_sync(0xffffffffu, sp);
-  if (lane == 0) {
-    rec[1] = t1;
-    rec[2] = (int64_t)bits;
-    rec[3] = 0;
-  }
+  const int64_t tgt = (int64_t)c * total;
+  const int64_t t0 = c == G ? T : first_tile(tgt);
+  const int64_t t1 = c >= G - 1 ? T : first_tile(tgt + total);
+  uint32_t bits = 0;
+  for (int i = 0; i < 31 && t0 + i < t1; ++i) bits |= (uint32_t)(map[t0 + i] == 1) << i;
+  int64_t *rec = plan + kPlanHead + 4 * (int64_t)c;
+  rec[0] = t0;
+  rec[1] = val_off[t0];
+  rec[2] = meta_off[t0];
+  rec[3] = bits;
 }
 
 // ---------------------------------------------------------------------------
@@ -1402,6 +1412,14 @@ struct Plan {
   size_t dyn_smem;
 };
 
+// CTAs of the TMA-ring kernels: one per SM (the ring takes most of shared
+// memory), at most kMaxCtas (the size of the launch-parameter plan), and no
+// more than there are dense tiles' worth of bytes.
+int tma_ctas(int sms, int64_t total_bytes, int b1, int b2) {
+  const int64_t gcap = std::max<int64_t>(1, total_bytes / (2LL * b1 * b2));
+  return (int)std::min<int64_t>(std::min(sms, kMaxCtas), gcap);
+}
+
 int make_plan(int64_t n, int64_t k, int b1, int b2, int64_t total_bytes,
               int batch, int rank, bool strided, Plan *pl) {
   Plan P{};
@@ -1414,16 +1432,16 @@ int make_plan(int64_t n, int64_t k, int b1, int b2, int64_t total_bytes,
   int sms = 0;
   int rc = device_sm_count(&sms);
   if (rc != HYB_OK) return rc;
-  P.tma = !strided && pick_tma_kernel(P.bp, s, &P.tk);
+  P.tma = !strided && s != kGeneric;
+  if (P.tma) {
+    P.G = tma_ctas(sms, total_bytes, b1, b2);
+    if (!pick_tma_kernel(P.bp, s, &P.tk)) return HYB_ERR_UNSUPPORTED;
+  }
   P.stream = !P.tma && s != kGeneric && P.R <= 8192;
   P.dyn_smem = P.tma ? P.tk.smem : (P.stream ? (size_t)2 * P.R * sizeof(int) : 0);
   if (P.tma) {
     const int nb = blocks_per_sm(P.tk.fn, P.tk.smem, P.tk.threads);
     if (nb <= 0) return HYB_ERR_CUDA;
-    // one CTA per SM (the ring takes most of shared memory); every CTA must
-    // own at least one tile: total / G >= the largest tile
-    const int64_t gcap = std::max<int64_t>(1, total_bytes / (2LL * b1 * b2));
-    P.G = (int)std::min<int64_t>(sms, gcap);
   } else if (P.stream) {
     void *fn = pick_stream_kernel<true>(P.bp, s);
     if (P.dyn_smem > 48 * 1024) {
@@ -1494,8 +1512,31 @@ int launch_lowrank_t(const Plan &P, const hyb_lowrank *lr, int64_t k,
 }
 
 // Shared driver of hyb_spmv / hyb_spmm_skinny / hyb_gemv_dense.
+// Copies a host plan made for this split into the launch parameters, after
+// checking that its ranges are well formed (a plan for another split, kind or
+// size is ignored and the kernel searches for its own range).
+void fill_launch_plan(const int64_t *plan, int32_t plan_ctas, const Plan &P, const Params &prm,
+                      LaunchPlan *lp) {
+  lp->kind = 0;
+  lp->ctas = 0;
+  const int32_t kind = kPlanTiles;
+  if (!plan || !P.tma || plan_ctas != P.G || plan[0] != P.G || plan[1] != kind) return;
+  const int64_t *rec = plan + kPlanHead;
+  const int64_t end = prm.T;
+  if (rec[0] != 0 || rec[4 * P.G] != end) return;
+  for (int c = 0; c <= P.G; ++c) {
+    const int64_t *r = rec + 4 * c;
+    if (r[0] < 0 || r[0] > end || (c > 0 && r[0] < r[-4])) return;
+    if (r[1] < 0 || 2 * r[1] > prm.nvb || r[2] < 0 || r[2] > prm.nmb) return;
+  }
+  std::copy(rec, rec + 4 * (P.G + 1), lp->rec);
+  lp->kind = kind;
+  lp->ctas = P.G;
+}
+
 int run_product(Params prm, int b1, int b2, int batch, const hyb_lowrank *lr,
-                bool strided, void *ws, size_t ws_bytes, cudaStream_t s) {
+                bool strided, void *ws, size_t ws_bytes, cudaStream_t s,
+                const int64_t *plan = nullptr, int32_t plan_ctas = 0) {
   const int rank = (lr && lr->rank > 0) ? lr->rank : 0;
   Plan P;
   int rc = make_plan(prm.n, prm.k, b1, b2, prm.total, batch, rank, strided, &P);
@@ -1528,10 +1569,12 @@ int run_product(Params prm, int b1, int b2, int batch, const hyb_lowrank *lr,
     prm.lr_ut = ut;
   }
   prm.status = reinterpret_cast<uint32_t *>(w);
-  if (!P.tma || prm.plan_ctas != P.G) prm.plan = nullptr;  // stale or foreign plan
   void *args[] = {&prm};
   if (P.tma) {
-    if (cudaLaunchKernel(P.tk.fn, dim3(P.G), dim3(P.tk.threads), args, P.tk.smem, s) !=
+    LaunchPlan lp;
+    fill_launch_plan(plan, plan_ctas, P, prm, &lp);
+    void *targs[] = {&prm, &lp};
+    if (cudaLaunchKernel(P.tk.fn, dim3(P.G), dim3(P.tk.threads), targs, P.tk.smem, s) !=
         cudaSuccess)
       return HYB_ERR_CUDA;
   } else if (P.stream) {
@@ -1604,9 +1647,10 @@ int spmm_impl(const hyb_matrix *A, int batch, const uint16_t *X, int64_t ldx,
   prm.ldy = ldy;
   prm.ydt = ydt;
   prm.total = 2 * A->n_vals + A->n_meta_bytes;  // packed bytes
-  prm.plan = A->plan;
-  prm.plan_ctas = A->plan_ctas;
-  return run_product(prm, A->b1, A->b2, batch, lr, false, ws, ws_bytes, s);
+  prm.nvb = 2 * A->n_vals;
+  prm.nmb = A->n_meta_bytes;
+  return run_product(prm, A->b1, A->b2, batch, lr, false, ws, ws_bytes, s, A->plan,
+                     A->plan_ctas);
 }
 
 // Virtual tiling of a plain row-major W for the dense baseline.
@@ -1646,41 +1690,34 @@ using namespace hyb;
 
 extern "C" {
 
-size_t hyb_plan_entries(void) {
-  int sms = 0;
-  if (device_sm_count(&sms) != HYB_OK) return 0;
-  return (size_t)kPlanHead + (size_t)sms * kPlanRec;
-}
+size_t hyb_plan_entries(void) { return (size_t)kPlanHead + 4 * (size_t)(kMaxCtas + 1); }
 
-int hyb_make_plan(const hyb_matrix *A, int64_t *plan, int32_t *plan_ctas,
-                  hyb_stream_t stream) {
-  if (!A || !plan || !plan_ctas) return HYB_ERR_INVALID_ARG;
+int hyb_make_plan(const hyb_matrix *A, int64_t *scratch, int64_t *plan_host,
+                  int32_t *plan_ctas, hyb_stream_t stream) {
+  if (!A || !scratch || !plan_host || !plan_ctas) return HYB_ERR_INVALID_ARG;
   *plan_ctas = 0;
   int rc = check_tiling(A->n, A->k, A->b1, A->b2);
   if (rc != HYB_OK) return rc;
-  if (!A->val_off || !A->meta_off || A->num_tiles != (A->n / A->b1) * (A->k / A->b2))
+  if (!A->val_off || !A->meta_off || !A->tile_map ||
+      A->num_tiles != (A->n / A->b1) * (A->k / A->b2))
     return HYB_ERR_INVALID_ARG;
-  if ((uintptr_t)plan % 8 != 0) return HYB_ERR_ALIGNMENT;
+  if ((uintptr_t)scratch % 8 != 0 || (uintptr_t)plan_host % 8 != 0) return HYB_ERR_ALIGNMENT;
   int sms = 0;
   rc = device_sm_count(&sms);
   if (rc != HYB_OK) return rc;
-  cudaStream_t s = (cudaStream_t)stream;
+  std::fill(plan_host, plan_host + hyb_plan_entries(), 0);
   const int64_t total = 2 * A->n_vals + A->n_meta_bytes;
-  if (shape_of(A->b1, A->b2) == kGeneric || total <= 0) {
-    // no streaming kernel for this tiling: an empty plan (G = 0) is ignored
-    return cudaMemsetAsync(plan, 0, sizeof(int64_t), s) == cudaSuccess ? HYB_OK : HYB_ERR_CUDA;
-  }
-  // the same G as make_plan's streaming path: one CTA per SM, each owning
-  // at least one tile
-  const int64_t gcap = std::max<int64_t>(1, total / (2LL * A->b1 * A->b2));
-  const int G = (int)std::min<int64_t>(sms, gcap);
-  const int64_t T = A->num_tiles;
-  const int64_t blocks = std::min<int64_t>((T + 1023) / 1024, 64);
-  plan_starts_kernel<<<(unsigned)std::max<int64_t>(1, blocks), 1024, 0, s>>>(
-      A->val_off, A->meta_off, T, G, total, plan);
+  if (shape_of(A->b1, A->b2) == kGeneric || total <= 0) return HYB_OK;  // no TMA kernel: G = 0
+  // the same split as the products: make_plan's CTA count
+  const int G = tma_ctas(sms, total, A->b1, A->b2);
+  cudaStream_t s = (cudaStream_t)stream;
+  plan_kernel<<<(G + 1 + 127) / 128, 128, 0, s>>>(A->val_off, A->meta_off, A->tile_map,
+                                                  A->num_tiles, G, total, scratch);
   if (cudaGetLastError() != cudaSuccess) return HYB_ERR_CUDA;
-  plan_records_kernel<<<G, 32, 0, s>>>(A->val_off, A->meta_off, A->tile_map, T, G, plan);
-  if (cudaGetLastError() != cudaSuccess) return HYB_ERR_CUDA;
+  const size_t bytes = sizeof(int64_t) * (kPlanHead + 4 * (size_t)(G + 1));
+  if (cudaMemcpyAsync(plan_host, scratch, bytes, cudaMemcpyDeviceToHost, s) != cudaSuccess ||
+      cudaStreamSynchronize(s) != cudaSuccess)
+    return HYB_ERR_CUDA;
   *plan_ctas = G;
   return HYB_OK;
 }

@@ -111,7 +111,8 @@ def lib():
     L.hyb_spmv_noalloc_max_scratch_bytes.restype = _SZ
     L.hyb_plan_entries.argtypes = []
     L.hyb_plan_entries.restype = _SZ
-    L.hyb_make_plan.argtypes = [ctypes.POINTER(HybMatrix), _P, ctypes.POINTER(ctypes.c_int32), _P]
+    L.hyb_make_plan.argtypes = [ctypes.POINTER(HybMatrix), _P, _P, ctypes.POINTER(ctypes.c_int32),
+                                _P]
     L.hyb_make_plan.restype = _I
     L.hyb_status_string.argtypes = [_I]
     L.hyb_status_string.restype = ctypes.c_char_p
@@ -175,7 +176,7 @@ class Packed:
     meta_off: torch.Tensor   # int64 [T+1], device
     n_vals: int
     n_meta: int
-    plan: Optional[torch.Tensor] = None  # int64 work split (hyb_make_plan), optional
+    plan: Optional[torch.Tensor] = None  # int64 work split (hyb_make_plan), host, optional
     plan_ctas: int = 0
 
     @property
@@ -218,14 +219,15 @@ def new_workspace(nbytes: int, device) -> torch.Tensor:
 
 def make_plan(A: "Packed", stream=None):
     """hyb_make_plan: the product's work split for A on the current device;
-    returns (plan tensor, CTA count)."""
-    plan = torch.zeros(int(lib().hyb_plan_entries()), dtype=torch.int64,
-                       device=A.val_off.device)
+    returns (host int64 plan tensor, CTA count).  Synchronises the stream."""
+    entries = int(lib().hyb_plan_entries())
+    scratch = torch.empty(entries, dtype=torch.int64, device=A.val_off.device)
+    plan = torch.zeros(entries, dtype=torch.int64)
     s = A.struct()
     s.plan = None
     ctas = ctypes.c_int32(0)
-    _check("hyb_make_plan", lib().hyb_make_plan(ctypes.byref(s), _ptr(plan), ctypes.byref(ctas),
-                                                _stream(stream)))
+    _check("hyb_make_plan", lib().hyb_make_plan(ctypes.byref(s), _ptr(scratch), _ptr(plan),
+                                                ctypes.byref(ctas), _stream(stream)))
     return plan, ctas.value
 
 

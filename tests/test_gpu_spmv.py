@@ -61,6 +61,19 @@ def test_multi_tile_ragged(orc, tiling, batch):
     _full_check(orc, n, k, b1, b2, tmap, batch, f"ragged{b1}x{b2}")
 
 
+@pytest.mark.parametrize("tiling", [(128, 128), (128, 64), (64, 64), (64, 128)])
+@pytest.mark.parametrize("batch", [1, 2, 3, 4, 5, 8, 13, 16])
+@pytest.mark.parametrize("tpr", [7, 37])
+def test_rows_ragged(orc, tiling, batch, tpr):
+    """2560 output rows with 7 or 37 tiles per band: the byte split puts CTA
+    boundaries mid-band and mid-window (37 tiles span two offset windows)."""
+    b1, b2 = tiling
+    n, k = 2560, b2 * tpr
+    T = (n // b1) * tpr
+    tmap = inputs.tile_map_bernoulli(T, 0.4, inputs.seed_of("rows", b1, b2, tpr))
+    _full_check(orc, n, k, b1, b2, tmap, batch, f"rows{b1}x{b2}", ydt_bf16=batch in (1, 16))
+
+
 @pytest.mark.parametrize("tiling", [(16, 16), (32, 32), (8, 16), (1, 128), (128, 16), (256, 64)])
 @pytest.mark.parametrize("batch", [1, 3, 16])
 def test_other_tilings(orc, tiling, batch):
@@ -167,43 +180,40 @@ def test_lowrank_fused_small(orc, batch):
     _full_check(orc, 640, 1024, 128, 128, tmap, batch, "lrsmall", rank=64)
 
 
-def _split_reference(orc, n, k, b1, b2, tmap, G):
-    """CTA c's first tile: the first t with P(t) * G >= c * total, where P is the
-    packed byte offset (2 * val_off + meta_off) -- computed from the oracle's
-    offsets."""
-    vo, mo = orc.offsets(n, k, b1, b2, tmap)
-    P = 2 * vo.astype(np.int64) + mo
-    total = int(P[-1])
-    T = len(tmap)
-    starts = [int(np.sum(P[:T] * G < c * total)) for c in range(G)] + [T]
-    return starts
+def _tile_split_reference(P, G):
+    """CTA c's first tile is the first t whose packed byte offset P(t)
+    (2 * val_off + meta_off) satisfies P(t) * G >= c * total."""
+    total, T = int(P[-1]), len(P) - 1
+    return [int(np.sum(P[:T] * G < c * total)) for c in range(G)] + [T]
 
 
 @pytest.mark.parametrize("shape", [(4096, 14336, 128, 128), (14336, 4096, 128, 64),
-                                   (256, 256, 64, 64)])
+                                   (256, 256, 64, 64), (1024, 4096, 128, 64)])
 def test_plan_matches_definition_and_results(orc, shape):
-    """hyb_make_plan gives the split the kernel would search for, and the product
-    with and without the plan (or with a plan for another SM count) is the same."""
+    """hyb_make_plan (host records handed to the kernel as launch parameters)
+    gives the split the kernel would search for, and the product with and
+    without the plan (or with a plan for another CTA count) is the same."""
     n, k, b1, b2 = shape
     T = (n // b1) * (k // b2)
     tmap = inputs.tile_map_fraction(T, 0.5, inputs.seed_of("plan", n, k))
     W, tmap, X, _ = case(n, k, b1, b2, tmap, name="plan")
     P = hyb.pack(W.to(dev()), tmap, b1, b2)
-    plan = P.plan.cpu().numpy()
+    plan = P.plan.numpy()
+    assert not P.plan.is_cuda
     G = int(plan[0])
-    assert G == P.plan_ctas
+    assert G == P.plan_ctas and int(plan[1]) == 1
     sms = torch.cuda.get_device_properties(0).multi_processor_count
-    assert G == min(sms, max(1, (2 * P.n_vals + P.n_meta) // (2 * b1 * b2)))
-    starts = _split_reference(orc, n, k, b1, b2, tmap, G)
+    assert G == min(sms, 160, max(1, (2 * P.n_vals + P.n_meta) // (2 * b1 * b2)))
     vo, mo = orc.offsets(n, k, b1, b2, tmap)
+    Pb = 2 * vo.astype(np.int64) + mo
+    rec = plan[8: 8 + 4 * (G + 1)].reshape(G + 1, 4)
+    starts = _tile_split_reference(Pb, G)
+    assert list(rec[:, 0]) == starts
     for c in range(G):
-        rec = plan[8 + 68 * c: 8 + 68 * (c + 1)]
         t0, t1 = starts[c], starts[c + 1]
-        assert (rec[0], rec[1]) == (t0, t1), c
-        idx = np.minimum(t0 + np.arange(32), T)
-        assert np.array_equal(rec[4:36], vo[idx]) and np.array_equal(rec[36:68], mo[idx]), c
+        assert (rec[c, 1], rec[c, 2]) == (vo[t0], mo[t0]), c
         bits = sum(1 << i for i in range(min(31, t1 - t0)) if tmap[t0 + i] == 1)
-        assert int(rec[2]) == bits, c
+        assert int(rec[c, 3]) == bits, c
     Xd = X.to(dev())
     y_plan = hyb.spmv(P, Xd)
     saved = P.plan
@@ -212,6 +222,10 @@ def test_plan_matches_definition_and_results(orc, shape):
     P.plan, P.plan_ctas = saved, G + 1  # a plan for another CTA count is ignored
     y_stale = hyb.spmv(P, Xd)
     assert torch.equal(y_plan, y_search) and torch.equal(y_plan, y_stale)
+    y_ref, env = orc.spmv(n, k, b1, b2, tmap, orc.pack(inputs.bits(W), b1, b2, tmap),
+                          inputs.bits(X))
+    assert_within(y_plan.cpu().numpy().reshape(-1), y_ref.reshape(-1), env.reshape(-1),
+                  what="plan")
 
 
 def test_cuda_graph_capture_replay():
