@@ -77,8 +77,9 @@ struct Params {
 // kernel as launch parameters, so that a CTA issues its first copy without
 // any global-memory load.  Host layout (int64): [0] = G, [1] = kind (1),
 // [2..7] reserved, then G + 1 records {t0, val_off[t0], meta_off[t0], 2:4
-// bits of tiles t0 .. t0 + 30}, t0 being the CTA's first tile; record G
-// holds the end (T).
+// bits of tiles t0 .. t0 + 30 (low word) and the stage starts of that first
+// window (high word)}, t0 being the CTA's first tile; record G holds the end
+// (T).
 constexpr int kMaxCtas = 160;
 constexpr int kPlanHead = 8;
 constexpr int32_t kPlanTiles = 1;
@@ -493,6 +494,16 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity) {
     if (mbar_try_wait(bar, parity)) return true;
   return false;
 }
+__device__ __forceinline__ int64_t ld_volatile_nc64(const int64_t *addr) {
+  int64_t v;
+  asm volatile("ld.global.nc.s64 %0, [%1];" : "=l"(v) : "l"(addr));
+  return v;
+}
+__device__ __forceinline__ uint32_t ld_volatile_nc8(const uint8_t *addr) {
+  uint32_t v;
+  asm volatile("ld.global.nc.u8 %0, [%1];" : "=r"(v) : "l"(addr));
+  return v;
+}
 __device__ __forceinline__ uint32_t atom_add_acq_rel(uint32_t *addr, uint32_t v) {
   uint32_t old;
   asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], %2;" : "=r"(old) : "l"(addr), "r"(v)
@@ -538,12 +549,37 @@ struct TmaCfg {
   static constexpr int kStageBytes = kValsBytes + kMetaBytes + BP * kXRow;
   static constexpr int kStages =
       (200 * 1024 / kStageBytes) < 6 ? (200 * 1024 / kStageBytes) : 6;
-  static constexpr int kThreads = (NC + 2) * 32;  // consumers, producer, epilogue
+  static constexpr int kThreads = (NC + 3) * 32;  // consumers, producer, 2 epilogue warps
   static constexpr size_t kSmem = (size_t)kStages * kStageBytes + 1024;
   static_assert(RPS * CPR == 32 && JS * RPS == RW && JS >= 1, "tile shape");
   static_assert(kStages >= 3, "ring too short");
   static_assert(TPX <= 8 && WIN < 32, "stage / offset window");
 };
+
+// Stage starts of a window of nw tiles beginning at tile w0 (bit i: a stage
+// starts at tile w0 + i): greedy packing by value bytes, in units of a 2:4
+// tile (a dense tile is 2), at most 2 tpd units and tpx tiles per stage, and
+// a new stage at every band start.  Used by the streaming kernel for every
+// window and by the plan for each CTA's first window.
+__device__ __forceinline__ uint32_t stage_starts(uint32_t spm, int nw, int64_t w0, int tpr,
+                                                int tpd, int tpx) {
+  int nb = (int)((tpr - w0 % tpr) % tpr);  // first band start at or after w0, relative
+  uint32_t starts = 0;
+  int fill = 2 * tpx, cnt = tpx;  // force a start at tile 0
+  for (int i = 0; i < nw; ++i) {
+    const int sz = (spm >> i & 1u) ? 1 : 2;
+    const bool band_start = i == nb;
+    if (band_start) nb += tpr;
+    if (band_start || fill + sz > 2 * tpd || cnt == tpx) {
+      starts |= 1u << i;
+      fill = 0;
+      cnt = 0;
+    }
+    fill += sz;
+    ++cnt;
+  }
+  return starts;
+}
 
 struct StageDesc {
   int64_t t0;       // first tile of the stage
@@ -575,6 +611,18 @@ __global__ void __launch_bounds__(TmaCfg<BP, B1, B2>::kThreads, 1)
   const int c = blockIdx.x;
   const int G = p.G;
   const int tpr = (int)p.tpr;
+  // The plan record is read first thing and parked in shared memory before
+  // the first barrier, so that its constant-bank line is fetched while the
+  // barriers are set up rather than when the producer first needs it.
+  __shared__ int64_t s_rec[5];
+  const bool planned = lp.kind == kPlanTiles;
+  if (planned && tid == 32 * C::NC + 1) {
+    s_rec[0] = lp.rec[4 * c];
+    s_rec[1] = lp.rec[4 * (c + 1)];
+    s_rec[2] = lp.rec[4 * c + 1];
+    s_rec[3] = lp.rec[4 * c + 2];
+    s_rec[4] = lp.rec[4 * c + 3];
+  }
   if (tid == 0) {
     for (int s = 0; s < S; ++s) {
       mbar_init(&full_bar[s], 1);
@@ -606,7 +654,6 @@ __global__ void __launch_bounds__(TmaCfg<BP, B1, B2>::kThreads, 1)
   // epilogue warp take them from the launch parameters; otherwise round 1
   // brackets both ends between band starts and round 2 counts inside the
   // bracketing band. ----
-  const bool planned = lp.kind == kPlanTiles;
   if (!planned) {
       const int64_t tgtA = (int64_t)c * p.total, tgtB = (int64_t)(c + 1) * p.total;
       uint32_t ca = 0, cb = 0;
@@ -664,8 +711,8 @@ __global__ void __launch_bounds__(TmaCfg<BP, B1, B2>::kThreads, 1)
     t0 = s_range[0];
     t1 = s_range[1];
   } else if (warp >= C::NC) {
-    t0 = lp.rec[4 * c];
-    t1 = lp.rec[4 * (c + 1)];
+    t0 = s_rec[0];
+    t1 = s_rec[1];
   }
 
   if (warp == C::NC) {
@@ -680,14 +727,16 @@ __global__ void __launch_bounds__(TmaCfg<BP, B1, B2>::kThreads, 1)
       int64_t vo, mo;
       uint32_t sp;
     };
+    // (volatile loads: the compiler may not turn the window load that a
+    // plan makes unnecessary into a speculative load the first window waits on)
     auto load_win = [&](int64_t w0) -> Win {
       Win o{0, 0, 0};
       const int64_t t = w0 + lane;
       if (lane <= C::WIN && t <= t1) {
-        o.vo = __ldg(p.val_off + t);
-        o.mo = __ldg(p.meta_off + t);
+        o.vo = ld_volatile_nc64(p.val_off + t);
+        o.mo = ld_volatile_nc64(p.meta_off + t);
       }
-      if (lane < C::WIN && t < t1) o.sp = __ldg(p.map + t) == 1;
+      if (lane < C::WIN && t < t1) o.sp = ld_volatile_nc8(p.map + t) == 1;
       return o;
     };
     int stage = 0;
@@ -700,10 +749,10 @@ __global__ void __launch_bounds__(TmaCfg<BP, B1, B2>::kThreads, 1)
       // first window from the plan: offsets of tile t0 + lane follow from
       // those of t0 and the 2:4 bits of the tiles before it
       constexpr int64_t TE = (int64_t)B1 * B2;
-      const uint32_t bits = (uint32_t)lp.rec[4 * c + 3];
+      const uint32_t bits = (uint32_t)s_rec[4];
       const int nb = __popc(bits & ((1u << lane) - 1u));
-      cur.vo = lp.rec[4 * c + 1] + (int64_t)lane * TE - nb * (TE / 2);
-      cur.mo = lp.rec[4 * c + 2] + nb * (TE / 8);
+      cur.vo = s_rec[2] + (int64_t)lane * TE - nb * (TE / 2);
+      cur.mo = s_rec[3] + nb * (TE / 8);
       cur.sp = lane < C::WIN ? (bits >> lane) & 1u : 0u;
       // a plan that does not fit the buffers is not used
       const int nw = (int)min((int64_t)C::WIN, t1 - t0);
@@ -716,25 +765,22 @@ __global__ void __launch_bounds__(TmaCfg<BP, B1, B2>::kThreads, 1)
       const Win nxt = load_win(w0 + C::WIN);  // in flight while this window issues
       const int nw = (int)min((int64_t)C::WIN, t1 - w0);
       const uint32_t spm = __ballot_sync(0xffffffffu, cur.sp != 0);
-      // greedy packing; value bytes in units of a 2:4 tile (dense = 2)
+      // stage starts: the plan's for the first window (checked against the
+      // stage limits lane by lane), else the greedy packing
       uint32_t starts = 0;
-      {
-        int64_t nb = (w0 / tpr) * tpr;  // first band start at or after w0
-        if (nb < w0) nb += tpr;
-        int fill = 2 * C::TPX, cnt = C::TPX;  // force a start at tile 0
-        for (int i = 0; i < nw; ++i) {
-          const int sz = (spm >> i & 1u) ? 1 : 2;
-          const bool band_start = w0 + i == nb;
-          if (band_start) nb += tpr;
-          if (band_start || fill + sz > 2 * C::TPD || cnt == C::TPX) {
-            starts |= 1u << i;
-            fill = 0;
-            cnt = 0;
-          }
-          fill += sz;
-          ++cnt;
-        }
+      bool have = false;
+      if (derived && w0 == t0) {
+        starts = (uint32_t)((uint64_t)s_rec[4] >> 32);
+        const uint32_t nxt_s = lane < 31 ? starts >> (lane + 1) : 0u;
+        const int e = nxt_s ? lane + __ffs(nxt_s) : nw;  // end of the stage starting here
+        const uint32_t in = e > lane ? ((e - lane >= 32 ? ~0u : (1u << (e - lane)) - 1u)) : 0u;
+        const int units = 2 * (e - lane) - __popc((spm >> lane) & in);
+        const bool good = lane >= nw || !(starts >> lane & 1u) ||
+                          (e - lane <= C::TPX && units <= 2 * C::TPD);
+        const bool band_ok = lane >= nw || (w0 + lane) % tpr != 0 || (starts >> lane & 1u);
+        have = __all_sync(0xffffffffu, good && band_ok) && (starts & 1u) && (starts >> nw) == 0;
       }
+      if (!have) starts = stage_starts(spm, nw, w0, tpr, C::TPD, C::TPX);
       // the stage that starts at this lane: tiles [w0 + lane, w0 + e)
       const bool is_start = lane < nw && (starts >> lane & 1u);
       const uint32_t later = lane < 31 ? (starts >> (lane + 1)) : 0u;
@@ -805,30 +851,33 @@ __global__ void __launch_bounds__(TmaCfg<BP, B1, B2>::kThreads, 1)
     return;
   }
 
-  if (warp == C::NC + 1) {
+  if (warp >= C::NC + 1) {
     // ------------------------------ epilogue ------------------------------
-    // Takes every piece of band this CTA finishes, in band order: a whole
-    // band goes straight to Y (with the low-rank term); a band shared with
-    // other CTAs goes to slot c + r, and a ticket per band finds the last of
-    // its CTAs, which sums the band's slots in CTA order (deterministic).
-    // All global-memory ordering (fence, atomic) happens here, off the
-    // consumer warps' path.
+    // Takes every piece of band this CTA finishes, in band order, pieces
+    // alternating between the two epilogue warps so that one piece's ticket
+    // round trip does not hold up the next: a whole band goes straight to Y
+    // (with the low-rank term); a band shared with other CTAs goes to slot
+    // c + r, and a ticket per band finds the last of its CTAs, which sums the
+    // band's slots in CTA order (deterministic).  All global-memory ordering
+    // (release, acquire) happens here, off the consumer warps' path.
     auto owner_of_p = [&](int64_t P) -> int {
       const int64_t o = (P * G) / p.total;
       return (int)(o < G - 1 ? o : G - 1);
     };
+    constexpr int OPL = 4, QMAX = 8;  // outputs per lane, contributors per load round
+    const int ew = warp - (C::NC + 1);
     const int r_first = (int)(t0 / tpr), r_last = t1 > t0 ? (int)((t1 - 1) / tpr) : r_first - 1;
-    int piece = 0;
-    for (int r = r_first; r <= r_last; ++r, ++piece) {
+    for (int r = r_first + ew; r <= r_last; r += 2) {
+      const int piece = r - r_first;
       const int slot = piece & 1;
       const uint32_t ph = (uint32_t)(piece >> 1) & 1u;
       const bool whole = t0 <= (int64_t)r * tpr && t1 >= (int64_t)(r + 1) * tpr;
       // owners of the band's first and last tile, fetched before the wait
-      int64_t pa = 0, pb = 0;
+      int oA = 0, oB = 0;
       if (!whole && lane == 0) {
         const int64_t ta = (int64_t)r * tpr, tb = ta + tpr - 1;
-        pa = 2 * __ldg(p.val_off + ta) + __ldg(p.meta_off + ta);
-        pb = 2 * __ldg(p.val_off + tb) + __ldg(p.meta_off + tb);
+        oA = owner_of_p(2 * __ldg(p.val_off + ta) + __ldg(p.meta_off + ta));
+        oB = owner_of_p(2 * __ldg(p.val_off + tb) + __ldg(p.meta_off + tb));
       }
       if (!mbar_wait(&piece_full[slot], ph)) {
         if (lane == 0) atomicOr(p.status, kStatusTimeout);
@@ -847,18 +896,14 @@ __global__ void __launch_bounds__(TmaCfg<BP, B1, B2>::kThreads, 1)
           const int row = o % B1, b = o / B1;
           __stcg(slotp + b * B1 + row, rows[row / C::RW][b * C::RW + row % C::RW]);
         }
-        // Each lane fences its own slot stores; the warp barrier then orders
-        // them before lane 0's ticket, whose acquire side (acq_rel) covers the
-        // reads of the other CTAs' slots if this CTA turns out to be last.
-        __threadfence();
+        // The warp barrier orders every lane's slot stores before lane 0's
+        // ticket; the ticket's release side (acq_rel, cumulative) publishes
+        // them at gpu scope, and its acquire side covers the reads of the
+        // other CTAs' slots if this CTA turns out to be last -- the pattern of
+        // a split-K semaphore, with no full fence per lane.
         __syncwarp();
         uint32_t last = 0;
-        int oA = 0, oB = 0;
-        if (lane == 0) {
-          oA = owner_of_p(pa);
-          oB = owner_of_p(pb);
-          last = atom_add_acq_rel(p.counters + r, 1u) == (uint32_t)(oB - oA);
-        }
+        if (lane == 0) last = atom_add_acq_rel(p.counters + r, 1u) == (uint32_t)(oB - oA);
         last = __shfl_sync(0xffffffffu, last, 0);
         oA = __shfl_sync(0xffffffffu, oA, 0);
         oB = __shfl_sync(0xffffffffu, oB, 0);
@@ -866,7 +911,6 @@ __global__ void __launch_bounds__(TmaCfg<BP, B1, B2>::kThreads, 1)
           __syncwarp();
           // sum the band's slots in CTA order; the loads of 4 outputs x 8
           // contributors are issued together, then added in a fixed order
-          constexpr int OPL = 4, QMAX = 8;
           for (int o0 = 0; o0 < B1 * BP; o0 += 32 * OPL) {
             float y[OPL];
 #pragma unroll
@@ -1018,8 +1062,8 @@ __global__ void __launch_bounds__(TmaCfg<BP, B1, B2>::kThreads, 1)
 // ---------------------------------------------------------------------------
 __global__ void __launch_bounds__(128)
     plan_kernel(const int64_t *__restrict__ val_off, const int64_t *__restrict__ meta_off,
-                const uint8_t *__restrict__ map, int64_t T, int G, int64_t total,
-                int64_t *__restrict__ plan) {
+                const uint8_t *__restrict__ map, int64_t T, int G, int64_t total, int tpr,
+                int tpd, int64_t *__restrict__ plan) {
   const int c = blockIdx.x * blockDim.x + threadIdx.x;
   if (c > G) return;
   auto P = [&](int64_t t) -> int64_t { return 2 * val_off[t] + meta_off[t]; };
@@ -1041,12 +1085,14 @@ __global__ void __launch_bounds__(128)
   const int64_t t0 = c == G ? T : first_tile(tgt);
   const int64_t t1 = c >= G - 1 ? T : first_tile(tgt + total);
   uint32_t bits = 0;
-  for (int i = 0; i < 31 && t0 + i < t1; ++i) bits |= (uint32_t)(map[t0 + i] == 1) << i;
+  const int nw = (int)min((int64_t)31, t1 - t0);
+  for (int i = 0; i < nw; ++i) bits |= (uint32_t)(map[t0 + i] == 1) << i;
+  const uint32_t starts = nw > 0 ? stage_starts(bits, nw, t0, tpr, tpd, 2 * tpd) : 0u;
   int64_t *rec = plan + kPlanHead + 4 * (int64_t)c;
   rec[0] = t0;
   rec[1] = val_off[t0];
   rec[2] = meta_off[t0];
-  rec[3] = bits;
+  rec[3] = (int64_t)(((uint64_t)starts << 32) | bits);
 }
 
 // ---------------------------------------------------------------------------
@@ -1711,8 +1757,11 @@ int hyb_make_plan(const hyb_matrix *A, int64_t *scratch, int64_t *plan_host,
   // the same split as the products: make_plan's CTA count
   const int G = tma_ctas(sms, total, A->b1, A->b2);
   cudaStream_t s = (cudaStream_t)stream;
+  // stage limits of the streaming kernel (a 32 KB value buffer per stage)
+  const int tpd = std::max(1, 16384 / (A->b1 * A->b2));
   plan_kernel<<<(G + 1 + 127) / 128, 128, 0, s>>>(A->val_off, A->meta_off, A->tile_map,
-                                                  A->num_tiles, G, total, scratch);
+                                                  A->num_tiles, G, total,
+                                                  (int)(A->k / A->b2), tpd, scratch);
   if (cudaGetLastError() != cudaSuccess) return HYB_ERR_CUDA;
   const size_t bytes = sizeof(int64_t) * (kPlanHead + 4 * (size_t)(G + 1));
   if (cudaMemcpyAsync(plan_host, scratch, bytes, cudaMemcpyDeviceToHost, s) != cudaSuccess ||

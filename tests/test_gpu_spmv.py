@@ -209,11 +209,26 @@ def test_plan_matches_definition_and_results(orc, shape):
     rec = plan[8: 8 + 4 * (G + 1)].reshape(G + 1, 4)
     starts = _tile_split_reference(Pb, G)
     assert list(rec[:, 0]) == starts
+    tpr, tpd = k // b2, max(1, 16384 // (b1 * b2))
     for c in range(G):
         t0, t1 = starts[c], starts[c + 1]
         assert (rec[c, 1], rec[c, 2]) == (vo[t0], mo[t0]), c
-        bits = sum(1 << i for i in range(min(31, t1 - t0)) if tmap[t0 + i] == 1)
-        assert int(rec[c, 3]) == bits, c
+        nw = min(31, t1 - t0)
+        bits = sum(1 << i for i in range(nw) if tmap[t0 + i] == 1)
+        word = int(rec[c, 3]) & 0xFFFFFFFFFFFFFFFF
+        assert word & 0xFFFFFFFF == bits, c
+        # stage starts of the first window: greedy by value bytes (a 2:4 tile
+        # is one unit, a dense tile two), at most 2 tpd units and 2 tpd tiles
+        # per stage, a new stage at every band start
+        want, fill, cnt = 0, 4 * tpd, 2 * tpd
+        for i in range(nw):
+            sz = 1 if tmap[t0 + i] == 1 else 2
+            if (t0 + i) % tpr == 0 or fill + sz > 2 * tpd or cnt == 2 * tpd:
+                want |= 1 << i
+                fill, cnt = 0, 0
+            fill += sz
+            cnt += 1
+        assert word >> 32 == want, c
     Xd = X.to(dev())
     y_plan = hyb.spmv(P, Xd)
     saved = P.plan
