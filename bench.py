@@ -48,6 +48,8 @@ WORKLOADS = {
     "ffn_down_4096x14336_f0.5_b1": (4096, 14336, 128, 128, 0.5, 1, 0.02, 0.01),
     "ffn_up_14336x4096_f0.5_b1": (14336, 4096, 128, 128, 0.5, 1, 0.02, 0.01),
     "attn_4096x4096_bern0.5_b1": (4096, 4096, 128, 128, None, 1, 0.02, 0.0),
+    "ffn_down_4096x14336_f0.5_b8": (4096, 14336, 128, 128, 0.5, 8, 0.02, 0.01),
+    "ffn_down_4096x14336_f0.5_b16": (4096, 14336, 128, 128, 0.5, 16, 0.02, 0.01),
 }
 
 
@@ -192,6 +194,10 @@ class Workload:
         self.frac_real = float(tmap.mean())
         self.mats = [base] + [base.clone() for _ in range(rotate - 1)]
         self.dense = [Wd] + [Wd.clone() for _ in range(rotate - 1)]
+        # the same W packed with every tile dense, streamed by the same kernel:
+        # the dense reference that differs from the product only in the format
+        dpk = hyb.pack(Wd, np.zeros_like(tmap), b1, b2)
+        self.dense_packed = [dpk] + [dpk.clone() for _ in range(rotate - 1)]
         self.X = [inputs.activations(batch, k, inputs.seed_of(name, "X", i)).to(device)
                   for i in range(rotate)]
         self.Y = [torch.empty(batch, n, dtype=torch.float32, device=device)
@@ -203,6 +209,7 @@ class Workload:
         self.fn = L.hyb_spmm_skinny
         self.dfn = L.hyb_gemv_dense
         self.structs = [m.struct() for m in self.mats]
+        self.dstructs = [m.struct() for m in self.dense_packed]
         self.stream = torch.cuda.current_stream(device)
         self.set_stream(self.stream)
         # algorithmic bytes of one product: packed values + masks, tile map, x, y
@@ -218,6 +225,11 @@ class Workload:
                       k, ctypes.c_void_p(self.Y[i].data_ptr()), n, hyb.HYB_F32, None,
                       ctypes.c_void_p(self.ws.data_ptr()), self.ws.numel(), s)
                      for i in range(rotate)]
+        self.pargs = [(ctypes.byref(self.dstructs[i]), batch,
+                       ctypes.c_void_p(self.X[i].data_ptr()), k,
+                       ctypes.c_void_p(self.Y[i].data_ptr()), n, hyb.HYB_F32, None,
+                       ctypes.c_void_p(self.ws.data_ptr()), self.ws.numel(), s)
+                      for i in range(rotate)]
         self.dargs = [(n, k, batch, ctypes.c_void_p(self.dense[i].data_ptr()), k,
                        ctypes.c_void_p(self.X[i].data_ptr()), k,
                        ctypes.c_void_p(self.Y[i].data_ptr()), n, hyb.HYB_F32,
@@ -233,6 +245,11 @@ class Workload:
         rc = self.dfn(*self.dargs[i % len(self.dargs)])
         if rc != 0:
             raise hyb.HybError("hyb_gemv_dense", rc)
+
+    def dense_packed_step(self, i):
+        rc = self.fn(*self.pargs[i % len(self.pargs)])
+        if rc != 0:
+            raise hyb.HybError("hyb_spmm_skinny", rc)
 
 
 def max_over_ranks(ms, device, world):
@@ -644,6 +661,7 @@ def main():
         ms = graph_timed(wl, wl.step, args.steps, args.warmup, world)
     eager_ms = timed(wl.step, args.steps, args.warmup, stream, world)
     dense_ms = graph_timed(wl, wl.dense_step, args.steps, args.warmup, world)
+    dpk_ms = graph_timed(wl, wl.dense_packed_step, args.steps, args.warmup, world)
     e2e_ms, h2d, d2h = e2e_timed(wl, args.steps, args.warmup, stream, world)
 
     per_step_ms = ms / args.steps
@@ -663,6 +681,9 @@ def main():
                   % (eager_ms / args.steps * 1e3),
         "dense_us_per_matrix": round(dense_us, 3),
         "speedup_vs_dense": round(dense_us / (per_step_ms * 1e3), 4),
+        "dense_packed_us_per_matrix": round(dpk_ms / args.steps * 1e3, 3),
+        "speedup_vs_dense_packed": round(dpk_ms / ms, 4),
+        "format_bound_speedup": round((2 * wl.n * wl.k) / wl.mats[0].nbytes(), 4),
         "frac_of_nominal_8tbs": round(achieved / NOMINAL_HBM_GBS, 4),
         "roofline": {"bound": "hbm", "achieved": round(achieved, 2), "peak": peak,
                      "unit": "GB/s", "frac": round(achieved / peak, 4),
