@@ -152,12 +152,16 @@ HYB_API size_t hyb_plan_entries(void);
  * over its CTAs on the current device: CTA c takes the tiles whose packed byte
  * offset falls in [c, c+1) * total / G.  `scratch` is a device buffer and
  * `plan_host` a host buffer, both of hyb_plan_entries() int64_t; on return
- * plan_host holds, for every CTA, its first and end tile, the packed offsets
- * of its first tile and the 2:4 bits of its first 31 tiles, and *plan_ctas
+ * plan_host holds, for every CTA, its first tile, the packed offsets of that
+ * tile, the 2:4 bits of its first 31 tiles and the stage boundaries of that
+ * first window (and one closing record with the tile count), and *plan_ctas
  * holds G (0 when the tiling has no streaming kernel).  Synchronises
- * `stream`.  Point A->plan / A->plan_ctas at the result: the products then
- * start streaming without any global-memory load, and ignore a plan whose
- * plan_ctas differs from the CTA count they would use. */
+ * `stream`.  Point A->plan / A->plan_ctas at the result: the products copy
+ * it into the kernel's launch parameters and start streaming without any
+ * global-memory load.  A plan whose CTA count differs from the one the
+ * product would use, or whose ranges are malformed, is ignored (the kernel
+ * then finds its range itself); results do not depend on whether a plan is
+ * used. */
 HYB_API int hyb_make_plan(const hyb_matrix *A, int64_t *scratch, int64_t *plan_host,
                           int32_t *plan_ctas, hyb_stream_t stream);
 
