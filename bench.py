@@ -48,6 +48,7 @@ WORKLOADS = {
     "ffn_down_4096x14336_f0.5_b1": (4096, 14336, 128, 128, 0.5, 1, 0.02, 0.01),
     "ffn_up_14336x4096_f0.5_b1": (14336, 4096, 128, 128, 0.5, 1, 0.02, 0.01),
     "attn_4096x4096_bern0.5_b1": (4096, 4096, 128, 128, None, 1, 0.02, 0.0),
+    "ffn_down_4096x14336_f0.5_b4": (4096, 14336, 128, 128, 0.5, 4, 0.02, 0.01),
     "ffn_down_4096x14336_f0.5_b8": (4096, 14336, 128, 128, 0.5, 8, 0.02, 0.01),
     "ffn_down_4096x14336_f0.5_b16": (4096, 14336, 128, 128, 0.5, 16, 0.02, 0.01),
 }

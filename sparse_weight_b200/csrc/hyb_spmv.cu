@@ -24,6 +24,9 @@
 //    arrive at a band (atomic ticket, no spinning) sums the slots in CTA order
 //    -- deterministic -- and applies the epilogue: the low-rank term
 //    ("3BASiL", §1: W ~ S + L) and the fp32 or bf16 store.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
 #include <algorithm>
 #include <mutex>
 
@@ -518,6 +521,16 @@ __device__ __forceinline__ void bulk_g2s(void *dst, const void *src, uint32_t by
       "l"(src), "r"(bytes), "r"(smem_u32(bar))
       : "memory");
 }
+// 2-D tiled TMA load of box (x, y) of the tensor map into shared memory,
+// completion counted on the mbarrier (no multicast).
+__device__ __forceinline__ void tma_load_2d(void *dst, const CUtensorMap *map, int x, int y,
+                                            uint64_t *bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3}], [%4];" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(smem_u32(bar))
+      : "memory");
+}
 // acc += lo(w) * lo(x) + hi(w) * hi(x) on two packed bf16 pairs.
 __device__ __forceinline__ void fma_bf16x2(float &acc, uint32_t w, uint32_t x) {
   unsigned short wl, wh, xl, xh;
@@ -545,8 +558,16 @@ struct TmaCfg {
   static constexpr int WIN = 31;                    // tiles per producer offset window
   static constexpr int kValsBytes = 2 * B1 * B2 * TPD;        // 32 KB
   static constexpr int kMetaBytes = B1 * B2 / 8 * TPX;        // 4 KB
-  static constexpr int kXRow = 2 * B2 * TPX;                  // bytes of one X row slice
-  static constexpr int kStageBytes = kValsBytes + kMetaBytes + BP * kXRow;
+  // X slices of a stage: with XTM (batch >= 4) one 2-D tensor copy fetches
+  // XT tiles' columns for all BP batch rows at once (box [BP][XT B2]);
+  // otherwise one 1-D copy per batch row.  Layout [copy][batch][XT B2].
+  static constexpr bool XTM = BP >= 4;
+  static constexpr int XT0 = 256 / B2 < TPX ? 256 / B2 : TPX;
+  static constexpr int XT = XTM ? XT0 : TPX;                 // tiles per X copy
+  static constexpr int kXBatch = 2 * B2 * XT;                // bytes between batch rows
+  static constexpr int kXCopy = BP * kXBatch;                // bytes of one X copy group
+  static constexpr int kXRegion = (TPX / XT) * kXCopy;       // = BP * 2 * B2 * TPX
+  static constexpr int kStageBytes = kValsBytes + kMetaBytes + kXRegion;
   static constexpr int kStages =
       (200 * 1024 / kStageBytes) < 6 ? (200 * 1024 / kStageBytes) : 6;
   static constexpr int kThreads = (NC + 3) * 32;  // consumers, producer, 2 epilogue warps
@@ -554,6 +575,7 @@ struct TmaCfg {
   static_assert(RPS * CPR == 32 && JS * RPS == RW && JS >= 1, "tile shape");
   static_assert(kStages >= 3, "ring too short");
   static_assert(TPX <= 8 && WIN < 32, "stage / offset window");
+  static_assert(TPX % XT == 0 && (!XTM || XT * B2 <= 256), "X copy groups");
 };
 
 // Stage starts of a window of nw tiles beginning at tile w0 (bit i: a stage
@@ -590,7 +612,7 @@ struct StageDesc {
 
 template <int BP, int B1, int B2>
 __global__ void __launch_bounds__(TmaCfg<BP, B1, B2>::kThreads, 1)
-    hybrid_tma_kernel(const Params p, const LaunchPlan lp) {
+    hybrid_tma_kernel(const Params p, const LaunchPlan lp, const __grid_constant__ CUtensorMap xmap) {
   using C = TmaCfg<BP, B1, B2>;
   constexpr int S = C::kStages;
   extern __shared__ __align__(1024) uint8_t smem[];
@@ -802,6 +824,9 @@ __global__ void __launch_bounds__(TmaCfg<BP, B1, B2>::kThreads, 1)
             const uint32_t mbytes = (uint32_t)(m_end - cur.mo);
             const int nt = e - k;
             const uint32_t xrow = (uint32_t)(2 * B2 * nt);
+            const int ngx = (nt + C::XT - 1) / C::XT;  // X copy groups (tensor path)
+            const uint32_t xbytes =
+                C::XTM ? (uint32_t)(ngx * C::kXCopy) : xrow * (uint32_t)p.batch;
             const int64_t band = ts / tpr;
             StageDesc d;
             d.t0 = ts;
@@ -811,13 +836,22 @@ __global__ void __launch_bounds__(TmaCfg<BP, B1, B2>::kThreads, 1)
             desc[stage] = d;
             armed |= 1u << stage;
             armed_parity = (armed_parity & ~(1u << stage)) | (phase << stage);
-            mbar_arrive_expect_tx(&full_bar[stage], vbytes + mbytes + xrow * p.batch);
+            mbar_arrive_expect_tx(&full_bar[stage], vbytes + mbytes + xbytes);
             bulk_g2s(st, p.vals + 2 * cur.vo, vbytes, &full_bar[stage]);
             if (mbytes) bulk_g2s(st + C::kValsBytes, p.meta + cur.mo, mbytes, &full_bar[stage]);
-            const uint16_t *xsrc = p.X + (ts - band * tpr) * B2;
-            for (int b = 0; b < p.batch; ++b)
-              bulk_g2s(st + C::kValsBytes + C::kMetaBytes + b * C::kXRow,
-                       xsrc + (int64_t)b * p.ldx, xrow, &full_bar[stage]);
+            const int64_t xcol = (ts - band * tpr) * B2;  // first X column of the stage
+            uint8_t *xdst = st + C::kValsBytes + C::kMetaBytes;
+            if constexpr (C::XTM) {
+              // whole boxes: rows past the batch and columns past k are
+              // zero-filled and counted in the transaction bytes
+              for (int q = 0; q < ngx; ++q)
+                tma_load_2d(xdst + q * C::kXCopy, &xmap, (int)(xcol + q * C::XT * B2), 0,
+                            &full_bar[stage]);
+            } else {
+              for (int b = 0; b < p.batch; ++b)
+                bulk_g2s(xdst + b * C::kXBatch, p.X + xcol + (int64_t)b * p.ldx, xrow,
+                         &full_bar[stage]);
+            }
           }
         }
         // every lane keeps the ring position
@@ -975,7 +1009,8 @@ __global__ void __launch_bounds__(TmaCfg<BP, B1, B2>::kThreads, 1)
       // a lane covers columns [16cp, 16cp+16) of a 2:4 tile row, and columns
       // [8cp, 8cp+8) + [B2/2 + 8cp, B2/2 + 8cp + 8) of a dense tile row (so
       // that 8 lanes read 128 contiguous bytes of shared memory)
-      const uint8_t *xs = st + C::kValsBytes + C::kMetaBytes + i * 2 * B2;
+      const uint8_t *xs = st + C::kValsBytes + C::kMetaBytes + (i / C::XT) * C::kXCopy +
+                          (i % C::XT) * 2 * B2;
       const int xo0 = sp ? 32 * cp : 16 * cp;
       const int xo1 = sp ? 32 * cp + 16 : B2 + 16 * cp;
 #pragma unroll
@@ -983,8 +1018,8 @@ __global__ void __launch_bounds__(TmaCfg<BP, B1, B2>::kThreads, 1)
         uint32_t xr[C::XB][8];
 #pragma unroll
         for (int b = 0; b < C::XB; ++b) {
-          const uint4 lo = *reinterpret_cast<const uint4 *>(xs + (b0 + b) * C::kXRow + xo0);
-          const uint4 hi = *reinterpret_cast<const uint4 *>(xs + (b0 + b) * C::kXRow + xo1);
+          const uint4 lo = *reinterpret_cast<const uint4 *>(xs + (b0 + b) * C::kXBatch + xo0);
+          const uint4 hi = *reinterpret_cast<const uint4 *>(xs + (b0 + b) * C::kXBatch + xo1);
           xr[b][0] = lo.x; xr[b][1] = lo.y; xr[b][2] = lo.z; xr[b][3] = lo.w;
           xr[b][4] = hi.x; xr[b][5] = hi.y; xr[b][6] = hi.z; xr[b][7] = hi.w;
         }
@@ -1340,13 +1375,16 @@ struct TmaKernel {
   int threads;
   size_t smem;
   int tps;
+  bool xtm;    // X slices by 2-D tensor copies (box xcols x bp)
+  int xcols;
+  int bp;
 };
 
 template <int BP, int B1, int B2>
 TmaKernel tma_kernel_info() {
   using C = TmaCfg<BP, B1, B2>;
   return TmaKernel{reinterpret_cast<void *>(&hybrid_tma_kernel<BP, B1, B2>), C::kThreads,
-                   C::kSmem, C::TPX};
+                   C::kSmem, C::TPX, C::XTM, C::XT * B2, BP};
 }
 
 bool pick_tma_kernel(int bp, Shape s, TmaKernel *out) {
@@ -1558,6 +1596,34 @@ int launch_lowrank_t(const Plan &P, const hyb_lowrank *lr, int64_t k,
 }
 
 // Shared driver of hyb_spmv / hyb_spmm_skinny / hyb_gemv_dense.
+// Tensor map of X ([batch][k] bf16, row stride ldx) with box [bp][xcols]:
+// rows past the batch and columns past k read as zeros.  The encoder is the
+// driver's, found once through the runtime.
+int encode_x_map(const uint16_t *X, int64_t k, int batch, int64_t ldx, int xcols, int bp,
+                 CUtensorMap *map) {
+  static PFN_cuTensorMapEncodeTiled_v12000 encode = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void *fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+  });
+  if (!encode) return HYB_ERR_CUDA;
+  const cuuint64_t dims[2] = {(cuuint64_t)k, (cuuint64_t)batch};
+  const cuuint64_t strides[1] = {(cuuint64_t)ldx * 2};
+  const cuuint32_t box[2] = {(cuuint32_t)xcols, (cuuint32_t)bp};
+  const cuuint32_t estr[2] = {1, 1};
+  const CUresult r = encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
+                            const_cast<uint16_t *>(X), dims, strides, box, estr,
+                            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                            CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? HYB_OK : HYB_ERR_CUDA;
+}
+
 // Copies a host plan made for this split into the launch parameters, after
 // checking that its ranges are well formed (a plan for another split, kind or
 // size is ignored and the kernel searches for its own range).
@@ -1619,7 +1685,12 @@ int run_product(Params prm, int b1, int b2, int batch, const hyb_lowrank *lr,
   if (P.tma) {
     LaunchPlan lp;
     fill_launch_plan(plan, plan_ctas, P, prm, &lp);
-    void *targs[] = {&prm, &lp};
+    alignas(64) CUtensorMap xmap{};
+    if (P.tk.xtm) {
+      rc = encode_x_map(prm.X, prm.k, batch, prm.ldx, P.tk.xcols, P.tk.bp, &xmap);
+      if (rc != HYB_OK) return rc;
+    }
+    void *targs[] = {&prm, &lp, &xmap};
     if (cudaLaunchKernel(P.tk.fn, dim3(P.G), dim3(P.tk.threads), targs, P.tk.smem, s) !=
         cudaSuccess)
       return HYB_ERR_CUDA;
