@@ -739,6 +739,12 @@ __global__ void __launch_bounds__(TmaCfg<BP, B1, B2>::kThreads, 1)
 
   if (warp == C::NC) {
     // ------------------------------ producer ------------------------------
+    if constexpr (C::XTM) {
+      // bring the X tensor map's descriptor into the TMA unit's cache once
+      if (lane == 0)
+        asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&xmap))
+                     : "memory");
+    }
     // Tiles are taken in windows of WIN: lane i holds the packed offsets of
     // tile w0 + i (and lane WIN those of the window's end), the next window
     // is loaded while this one is issued.  Stages are packed greedily inside

@@ -91,6 +91,34 @@ def test_degenerate_maps(orc, frac):
     _full_check(orc, 4096, 4096, 128, 128, tmap, 4, f"degenerate{frac}")
 
 
+@pytest.mark.parametrize("batch", [1, 3, 5, 16])
+def test_strided_operands(orc, batch):
+    """X rows with a row stride above k and a column offset, Y rows with a row
+    stride above n: the result equals the contiguous call bit for bit, and the
+    padding around Y is left alone (batch >= 4 fetches X by tensor copies whose
+    row stride is ldx)."""
+    n, k, b1, b2 = 1280, 2304, 128, 128
+    T = (n // b1) * (k // b2)
+    tmap = inputs.tile_map_bernoulli(T, 0.5, inputs.seed_of("strided", n, k))
+    W, tmap, X, _ = case(n, k, b1, b2, tmap, batch=batch, name="strided")
+    P = hyb.pack(W.to(dev()), tmap, b1, b2)
+    Xd = X.to(dev())
+    big = torch.zeros(batch, k + 40, dtype=torch.bfloat16, device=dev())
+    big[:, 8:8 + k] = Xd
+    Xs = big[:, 8:8 + k]
+    assert Xs.stride(0) == k + 40 and Xs.data_ptr() % 16 == 0
+    Ybig = torch.full((batch, n + 24), 5.0, device=dev())
+    Ys = Ybig[:, 4:4 + n]
+    hyb.spmm_skinny(P, Xs, Y=Ys)
+    Yc = hyb.spmm_skinny(P, Xd)
+    torch.cuda.synchronize()
+    assert torch.equal(Ys, Yc)
+    assert bool((Ybig[:, :4] == 5.0).all()) and bool((Ybig[:, 4 + n:] == 5.0).all())
+    y_ref, env = orc.spmv(n, k, b1, b2, tmap, orc.pack(inputs.bits(W), b1, b2, tmap),
+                          inputs.bits(X))
+    assert_within(Ys.cpu().numpy(), y_ref, env, what=f"strided b={batch}")
+
+
 def test_single_tile(orc):
     _full_check(orc, 128, 128, 128, 128, np.array([1], np.uint8), 1, "single")
     _full_check(orc, 64, 64, 64, 64, np.array([0], np.uint8), 2, "single0")
