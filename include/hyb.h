@@ -83,7 +83,9 @@ typedef enum {
   HYB_ERR_ALIGNMENT = -3,    /* pointer or leading dimension misaligned */
   HYB_ERR_WORKSPACE = -4,    /* workspace null or smaller than required */
   HYB_ERR_CUDA = -5,         /* a CUDA runtime call failed */
-  HYB_ERR_DEVICE_CHECK = -6  /* the device flagged bad data (see above) */
+  HYB_ERR_DEVICE_CHECK = -6, /* the device flagged bad data (see above) */
+  HYB_ERR_TIMEOUT = -7       /* a bounded wait inside a kernel ran out (status bit 4);
+                                that call's outputs are incomplete, the context is usable */
 } hyb_status;
 
 typedef enum { HYB_F32 = 0, HYB_BF16 = 1 } hyb_dtype;
@@ -246,10 +248,21 @@ HYB_API size_t hyb_spmv_noalloc_max_scratch_bytes(void);
 /* ---- status ------------------------------------------------------------ */
 
 /* Synchronise `stream`, read and clear the workspace status word.  Returns
- * HYB_OK, HYB_ERR_DEVICE_CHECK (a device check fired) or HYB_ERR_CUDA. If
- * flags is not NULL it receives the raw status bits (1 = NaN weight seen by
- * hyb_pack, 2 = tile_map byte other than 0/1). */
+ * HYB_OK, HYB_ERR_TIMEOUT (a pipeline wait gave up), HYB_ERR_DEVICE_CHECK (a
+ * data check fired) or HYB_ERR_CUDA. If flags is not NULL it receives the raw
+ * status bits (1 = NaN weight seen by hyb_pack, 2 = tile_map byte other than
+ * 0/1 or a tile map that does not fit the buffers, 4 = a bounded wait ran
+ * out). */
 HYB_API int hyb_check_status(void *ws, hyb_stream_t stream, uint32_t *flags);
+
+/* Failure-path self test: launch on `stream` a one-CTA kernel whose mbarrier
+ * wait can never complete (nothing arrives), bounded by `wait_limit` tries of
+ * the same wait loop the products use.  The wait runs out, the kernel sets
+ * status bit 4 in the workspace (`ws`, >= 256 bytes, device) and returns; the
+ * next hyb_check_status then returns HYB_ERR_TIMEOUT.  Nothing faults or
+ * traps.  wait_limit must be in [1, 1 << 20]. */
+HYB_API int hyb_selftest_wait_timeout(void *ws, size_t ws_bytes, uint32_t wait_limit,
+                                      hyb_stream_t stream);
 
 /* Static description of a status code. */
 HYB_API const char *hyb_status_string(int status);

@@ -37,6 +37,7 @@ const char *hyb_status_string(int status) {
     case HYB_ERR_WORKSPACE: return "workspace missing or too small";
     case HYB_ERR_CUDA: return "CUDA runtime error";
     case HYB_ERR_DEVICE_CHECK: return "device-side data check failed (NaN weight or bad tile map)";
+    case HYB_ERR_TIMEOUT: return "a bounded wait inside a kernel ran out (outputs incomplete)";
     default: return "unknown status";
   }
 }
@@ -62,6 +63,7 @@ int hyb_check_status(void *ws, hyb_stream_t stream, uint32_t *flags) {
       return HYB_ERR_CUDA;
   }
   if (flags) *flags = host;
+  if (host & hyb::kStatusTimeout) return HYB_ERR_TIMEOUT;
   return host ? HYB_ERR_DEVICE_CHECK : HYB_OK;
 }
 

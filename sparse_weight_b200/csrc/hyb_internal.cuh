@@ -14,6 +14,7 @@ namespace hyb {
 // Status bits kept in the first word of every workspace.
 constexpr uint32_t kStatusNaN = 1u;      // hyb_pack saw a NaN weight
 constexpr uint32_t kStatusBadMap = 2u;   // tile_map byte other than 0 / 1
+constexpr uint32_t kStatusTimeout = 4u;  // a bounded wait inside a kernel ran out
 
 // Workspace header: status word, padded so that what follows is aligned.
 constexpr size_t kHeaderBytes = 256;

@@ -461,7 +461,6 @@ __global__ void __launch_bounds__(kThreads, (Cfg<BP, B1, B2, STRIDED>::kMinBlock
 // values of a 2:4 group from its 4-bit mask through a 16-entry selector table
 // ("SparseDecoding", authors' abstract: bitmask-indexed N:M SpMV).
 
-constexpr uint32_t kStatusTimeout = 4u;  // a pipeline wait ran out
 constexpr uint32_t kWaitLimit = 1u << 22;
 
 __device__ __forceinline__ uint32_t smem_u32(const void *p) {
@@ -492,10 +491,14 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
 }
 // Every wait is bounded: on expiry the caller records kStatusTimeout and
 // leaves the pipeline instead of waiting for ever.
-__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity) {
-  for (uint32_t i = 0; i < kWaitLimit; ++i)
+__device__ __forceinline__ bool mbar_wait_limit(uint64_t *bar, uint32_t parity,
+                                                uint32_t limit) {
+  for (uint32_t i = 0; i < limit; ++i)
     if (mbar_try_wait(bar, parity)) return true;
   return false;
+}
+__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity) {
+  return mbar_wait_limit(bar, parity, kWaitLimit);
 }
 __device__ __forceinline__ int64_t ld_volatile_nc64(const int64_t *addr) {
   int64_t v;
@@ -1328,6 +1331,22 @@ __global__ void __launch_bounds__(kThreads)
 }
 
 // ---------------------------------------------------------------------------
+// failure-path self test: a wait that nothing completes runs out
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(32) selftest_wait_timeout_kernel(uint32_t *status,
+                                                                   uint32_t limit) {
+  __shared__ __align__(8) uint64_t bar;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  __syncwarp();
+  // nothing ever arrives on bar, so phase 0 never completes
+  const bool done = mbar_wait_limit(&bar, 0u, limit);
+  if (!done && threadIdx.x == 0) atomicOr(status, kStatusTimeout);
+}
+
+// ---------------------------------------------------------------------------
 // host side
 // ---------------------------------------------------------------------------
 
@@ -2054,6 +2073,16 @@ int hyb_spmv_noalloc(const hyb_matrix *A, const uint16_t *X, int64_t ldx,
     return HYB_ERR_CUDA;
   return hyb::spmm_impl(A, 1, X, ldx, Y, ldy, ydt, nullptr, scratch,
                         hyb::kNoAllocScratchBytes, s);
+}
+
+int hyb_selftest_wait_timeout(void *ws, size_t ws_bytes, uint32_t wait_limit,
+                              hyb_stream_t stream) {
+  if (ws == nullptr || ws_bytes < hyb::kHeaderBytes) return HYB_ERR_WORKSPACE;
+  if ((uintptr_t)ws % 256 != 0) return HYB_ERR_ALIGNMENT;
+  if (wait_limit < 1 || wait_limit > (1u << 20)) return HYB_ERR_INVALID_ARG;
+  hyb::selftest_wait_timeout_kernel<<<1, 32, 0, (cudaStream_t)stream>>>(
+      reinterpret_cast<uint32_t *>(ws), wait_limit);
+  return cudaGetLastError() == cudaSuccess ? HYB_OK : HYB_ERR_CUDA;
 }
 
 }  // extern "C"

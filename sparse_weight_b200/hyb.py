@@ -24,12 +24,14 @@ HYB_ERR_ALIGNMENT = -3
 HYB_ERR_WORKSPACE = -4
 HYB_ERR_CUDA = -5
 HYB_ERR_DEVICE_CHECK = -6
+HYB_ERR_TIMEOUT = -7
 
 HYB_F32 = 0
 HYB_BF16 = 1
 
 STATUS_NAN = 1
 STATUS_BAD_MAP = 2
+STATUS_TIMEOUT = 4
 
 _P = ctypes.c_void_p
 _I64 = ctypes.c_int64
@@ -65,7 +67,7 @@ EXPORTS = ["hyb_packed_sizes", "hyb_pack_workspace_bytes", "hyb_pack",
            "hyb_spmm_skinny", "hyb_lowrank_workspace_bytes", "hyb_lowrank_add",
            "hyb_dense_workspace_bytes", "hyb_gemv_dense", "hyb_check_status",
            "hyb_status_string", "hyb_spmv_noalloc", "hyb_spmv_noalloc_max_scratch_bytes",
-           "hyb_plan_entries", "hyb_make_plan"]
+           "hyb_plan_entries", "hyb_make_plan", "hyb_selftest_wait_timeout"]
 
 
 def lib():
@@ -105,6 +107,8 @@ def lib():
     L.hyb_gemv_dense.restype = _I
     L.hyb_check_status.argtypes = [_P, _P, ctypes.POINTER(ctypes.c_uint32)]
     L.hyb_check_status.restype = _I
+    L.hyb_selftest_wait_timeout.argtypes = [_P, _SZ, ctypes.c_uint32, _P]
+    L.hyb_selftest_wait_timeout.restype = _I
     L.hyb_spmv_noalloc.argtypes = [ctypes.POINTER(HybMatrix), _P, _I64, _P, _I64, _I, _P]
     L.hyb_spmv_noalloc.restype = _I
     L.hyb_spmv_noalloc_max_scratch_bytes.argtypes = []
@@ -263,6 +267,13 @@ def pack(W: torch.Tensor, tile_map, b1: int, b2: int, ws: torch.Tensor = None,
     if plan:
         P.plan, P.plan_ctas = make_plan(P, stream)
     return P
+
+
+def selftest_wait_timeout(ws: torch.Tensor, wait_limit: int = 2000, stream=None):
+    """hyb_selftest_wait_timeout: launch the failure-path self test (a bounded
+    wait that can never complete); the next check_status reports the timeout."""
+    _check("hyb_selftest_wait_timeout",
+           lib().hyb_selftest_wait_timeout(_ptr(ws), ws.numel(), wait_limit, _stream(stream)))
 
 
 def check_status(ws: torch.Tensor, stream=None) -> int:

@@ -34,9 +34,19 @@ def test_exports_every_declared_symbol(L):
 
 
 def test_status_strings(L):
-    for code in range(0, -7, -1):
-        assert hyb.status_string(code)
+    for code in range(0, -8, -1):
+        assert hyb.status_string(code) and "unknown" not in hyb.status_string(code)
     assert "unknown" in hyb.status_string(-99)
+
+
+def test_selftest_argument_checks(L):
+    """The failure-path self test validates its arguments before any launch."""
+    f = L.hyb_selftest_wait_timeout
+    assert f(None, 256, 10, None) == hyb.HYB_ERR_WORKSPACE
+    assert f(ctypes.c_void_p(256), 255, 10, None) == hyb.HYB_ERR_WORKSPACE
+    assert f(ctypes.c_void_p(256 + 16), 256, 10, None) == hyb.HYB_ERR_ALIGNMENT
+    assert f(ctypes.c_void_p(256), 256, 0, None) == hyb.HYB_ERR_INVALID_ARG
+    assert f(ctypes.c_void_p(256), 256, (1 << 20) + 1, None) == hyb.HYB_ERR_INVALID_ARG
 
 
 def _sizes(n, k, b1, b2, m):
