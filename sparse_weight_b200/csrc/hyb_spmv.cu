@@ -3,23 +3,23 @@
 //
 // Decode-time products are memory-bound ("SparseDecoding: decoding-aware
 // pruning ...", authors' abstract: the decode phase is limited by memory
-// access and is dominated by sparse matrix-vector products), so the design
-// is a single streaming pass over the packed bytes with no tensor cores:
+// access and is dominated by sparse matrix-vector products), so every kernel
+// here is a single streaming pass over the weight bytes with no tensor cores.
 //
-//  * Work split: the packed stream is row-major over tiles, so every tile-row
+//  * hybrid_tma_kernel (packed matrices, tilings 128x128, 128x64, 64x64,
+//    64x128): the packed stream is row-major over tiles, so every tile-row
 //    band is contiguous.  CTA c of G takes the tiles whose byte offset falls
 //    in [c, c+1) * total / G -- a split by bytes, not by tiles, because a
 //    dense tile costs 2 B/weight and a 2:4 tile 1.125 B/weight ("PATCH:
 //    Learnable Tile-level Hybrid Sparsity for LLMs", §2: tiles are dense or
-//    2:4).  Each CTA finds its range with two rounds of parallel search over
-//    the tile offsets.
-//  * Inside a tile, warp w owns rows [w*R, (w+1)*R); a lane owns 16 columns of
-//    one row per step: 16 bytes of kept values plus 2 bytes of masks in a 2:4
-//    tile (4 groups), or 32 bytes in a dense tile.  Lanes keep the 16 x values
-//    they need in registers and accumulate in fp32 registers across all the
-//    tiles of a band; the next tile is loaded while the current one computes.
-//  * The mask nibble picks which two of the group's four x values multiply
-//    the two kept values (SparseDecoding: bitmask-indexed, fixed-stride N:M).
+//    2:4).  A producer warp moves the bytes into a shared-memory ring with
+//    bulk copies; consumer warps compute from it; two epilogue warps finish
+//    the bands.
+//  * hybrid_rowwarp_kernel (any other legal tiling, packed or row-major): one
+//    warp per output row, plain loads.
+//  * dense_gemv_kernel (row-major bf16 W, the baseline the format is measured
+//    against): the same byte split over uniform tiles, register double
+//    buffering instead of a ring.
 //  * Band results cross CTAs through fp32 partial slots; the last CTA to
 //    arrive at a band (atomic ticket, no spinning) sums the slots in CTA order
 //    -- deterministic -- and applies the epilogue: the low-rank term
@@ -120,13 +120,6 @@ __device__ __forceinline__ void unpack16(const uint4 &a, const uint4 &b,
   }
 }
 
-__device__ __forceinline__ int64_t cost_prefix(const Params &p, int64_t t,
-                                               bool strided,
-                                               int64_t tile_cost_dense) {
-  if (strided) return t * tile_cost_dense;
-  return 2 * __ldg(p.val_off + t) + __ldg(p.meta_off + t);
-}
-
 __device__ __forceinline__ int owner_of(int64_t P, const Params &p) {
   int64_t o = (P * p.G) / p.total;
   return (int)(o < p.G - 1 ? o : p.G - 1);
@@ -144,10 +137,13 @@ __device__ __forceinline__ void store_out(const Params &p, int64_t row, int b,
 }
 
 // ---------------------------------------------------------------------------
-// the streaming kernel
+// dense GEMV baseline: row-major bf16 W, CTA c takes tiles
+// [c, c+1) * T / G (all tiles cost the same); warp w owns rows [w*R, (w+1)*R)
+// of a tile and a lane 16 columns of one row per step; the next tile is
+// loaded into registers while the current one computes
 // ---------------------------------------------------------------------------
 
-template <int BP, int B1, int B2, bool STRIDED>
+template <int BP, int B1, int B2>
 struct Cfg {
   static constexpr int RW = B1 / kWarps;    // rows per warp per tile
   static constexpr int CPR = B2 / 16;       // lanes per row (16 columns each)
@@ -160,17 +156,17 @@ struct Cfg {
   static_assert(RPS * CPR == 32 && JS * RPS == RW, "tile shape");
 };
 
-// Registers of one tile in flight: per step 16 B (2:4) + 2 B masks, or 32 B.
+// Registers of one tile in flight: 32 B (16 bf16) per lane per step.
 template <int JS>
 struct TileRegs {
   uint4 a[JS];
-  uint4 b[JS];  // dense: second 16 B; 2:4: b[j].x holds the 16 mask bits
+  uint4 b[JS];
 };
 
-template <int BP, int B1, int B2, bool STRIDED>
-__global__ void __launch_bounds__(kThreads, (Cfg<BP, B1, B2, STRIDED>::kMinBlocks))
-    hybrid_stream_kernel(const Params p) {
-  using C = Cfg<BP, B1, B2, STRIDED>;
+template <int BP, int B1, int B2>
+__global__ void __launch_bounds__(kThreads, (Cfg<BP, B1, B2>::kMinBlocks))
+    dense_gemv_kernel(const Params p) {
+  using C = Cfg<BP, B1, B2>;
   constexpr int JS = C::JS;
   extern __shared__ int s_owner[];  // [2 * R]: owner CTA of each band's first / last tile
   __shared__ float s_acc[B1 * BP];
@@ -187,52 +183,13 @@ __global__ void __launch_bounds__(kThreads, (Cfg<BP, B1, B2, STRIDED>::kMinBlock
   // ---- 1. this CTA's tile range [t0, t1) -----------------------------------
   const int64_t tgtA = (int64_t)c * p.total;
   const int64_t tgtB = (int64_t)(c + 1) * p.total;
-  int64_t t0, t1;
-  if (STRIDED) {
-    // uniform tiles: closed form
-    const int64_t unit = C::kDenseCost * G;
-    t0 = (tgtA + unit - 1) / unit;
-    t1 = (c == G - 1) ? p.T : (tgtB + unit - 1) / unit;
-    for (int i = tid; i < p.R; i += kThreads) {
-      s_owner[2 * i] = owner_of((int64_t)i * p.tpr * C::kDenseCost, p);
-      s_owner[2 * i + 1] =
-          owner_of(((int64_t)(i + 1) * p.tpr - 1) * C::kDenseCost, p);
-    }
-  } else {
-    // round 1: band starts (and owners of every band's first / last tile)
-    int cntA = 0, cntB = 0;
-    for (int base = 0; base <= p.R; base += kThreads) {
-      const int i = base + tid;
-      bool pa = false, pb = false;
-      if (i <= p.R) {
-        const int64_t P0 = cost_prefix(p, (int64_t)i * p.tpr, false, 0);
-        pa = P0 * G < tgtA;
-        pb = P0 * G < tgtB;
-        if (i < p.R) {
-          const int64_t Pl = cost_prefix(p, (int64_t)(i + 1) * p.tpr - 1, false, 0);
-          s_owner[2 * i] = owner_of(P0, p);
-          s_owner[2 * i + 1] = owner_of(Pl, p);
-        }
-      }
-      cntA += __syncthreads_count(pa);
-      cntB += __syncthreads_count(pb);
-    }
-    // round 2: tiles inside the bracketing band
-    const int64_t baseA = cntA > 0 ? (int64_t)(cntA - 1) * p.tpr : 0;
-    const int64_t baseB = cntB > 0 ? (int64_t)(cntB - 1) * p.tpr : 0;
-    int64_t cA = 0, cB = 0;
-    for (int64_t off = 0; off < p.tpr; off += kThreads) {
-      const int64_t o = off + tid;
-      bool pa = false, pb = false;
-      if (o < p.tpr) {
-        if (cntA > 0) pa = cost_prefix(p, baseA + o, false, 0) * G < tgtA;
-        if (cntB > 0) pb = cost_prefix(p, baseB + o, false, 0) * G < tgtB;
-      }
-      cA += __syncthreads_count(pa);
-      cB += __syncthreads_count(pb);
-    }
-    t0 = cntA > 0 ? baseA + cA : 0;
-    t1 = (c == G - 1) ? p.T : (cntB > 0 ? baseB + cB : 0);
+  // uniform tiles: the split is a closed form
+  const int64_t unit = C::kDenseCost * G;
+  int64_t t0 = (tgtA + unit - 1) / unit;
+  int64_t t1 = (c == G - 1) ? p.T : (tgtB + unit - 1) / unit;
+  for (int i = tid; i < p.R; i += kThreads) {
+    s_owner[2 * i] = owner_of((int64_t)i * p.tpr * C::kDenseCost, p);
+    s_owner[2 * i + 1] = owner_of(((int64_t)(i + 1) * p.tpr - 1) * C::kDenseCost, p);
   }
   if (tid == 0) {
     s_range[0] = t0;
@@ -251,47 +208,12 @@ __global__ void __launch_bounds__(kThreads, (Cfg<BP, B1, B2, STRIDED>::kMinBlock
 
   const int wrow = warp * C::RW;  // first row of this warp inside a tile
 
-  // tile "header": sparse flag and byte offsets (prefetched one tile ahead)
-  struct Head {
-    int64_t vb, mb;
-    bool sparse;
-  };
-  auto head_of = [&](int64_t t) -> Head {
-    Head h;
-    if (STRIDED) {
-      h.vb = 0;
-      h.mb = 0;
-      h.sparse = false;
-    } else {
-      h.sparse = __ldg(p.map + t) == 1;
-      h.vb = 2 * __ldg(p.val_off + t);
-      h.mb = __ldg(p.meta_off + t);
-    }
-    return h;
-  };
-  auto load_tile = [&](int64_t t, const Head &h, TileRegs<JS> &r) {
+  // a lane's 16 columns of JS rows of a tile of the row-major W
+  auto load_tile = [&](int64_t t, TileRegs<JS> &r) {
     const int64_t tr = t / p.tpr, tc = t - tr * p.tpr;
-    if (STRIDED) {
-      const uint16_t *base =
-          p.Wd + (tr * B1 + wrow + rs) * p.ldw + tc * B2 + 16 * cp;
+    const uint16_t *base = p.Wd + (tr * B1 + wrow + rs) * p.ldw + tc * B2 + 16 * cp;
 #pragma unroll
-      for (int j = 0; j < JS; ++j)
-        ld_stream32(base + (int64_t)j * C::RPS * p.ldw, r.a[j], r.b[j]);
-    } else if (h.sparse) {
-      const uint8_t *vbase = p.vals + h.vb + (int64_t)(wrow + rs) * B2 + 16 * cp;
-      const uint8_t *mbase = p.meta + h.mb + (int64_t)(wrow + rs) * (B2 / 8) + 2 * cp;
-#pragma unroll
-      for (int j = 0; j < JS; ++j) {
-        r.a[j] = ld_stream16(vbase + (int64_t)j * C::RPS * B2);
-        r.b[j].x = ld_stream_u16(mbase + (int64_t)j * C::RPS * (B2 / 8));
-      }
-    } else {
-      const uint8_t *vbase =
-          p.vals + h.vb + (int64_t)(wrow + rs) * 2 * B2 + 32 * cp;
-#pragma unroll
-      for (int j = 0; j < JS; ++j)
-        ld_stream32(vbase + (int64_t)j * C::RPS * 2 * B2, r.a[j], r.b[j]);
-    }
+    for (int j = 0; j < JS; ++j) ld_stream32(base + (int64_t)j * C::RPS * p.ldw, r.a[j], r.b[j]);
   };
   auto load_x = [&](int64_t t, int b0, XRegs<C::XB> &xr) {
     const int64_t tc = t % p.tpr;
@@ -366,20 +288,15 @@ __global__ void __launch_bounds__(kThreads, (Cfg<BP, B1, B2, STRIDED>::kMinBlock
   };
 
   if (t0 < t1) {
-    Head hcur = head_of(t0);
-    Head hnext = hcur;
-    if (t0 + 1 < t1) hnext = head_of(t0 + 1);
     TileRegs<JS> cur;
-    load_tile(t0, hcur, cur);
+    load_tile(t0, cur);
     XRegs<C::XB> xcur;
     if (BP <= 4) load_x(t0, 0, xcur);
     for (int64_t t = t0; t < t1; ++t) {
-      Head hnn = hnext;
-      if (t + 2 < t1) hnn = head_of(t + 2);
       TileRegs<JS> nxt;
       XRegs<C::XB> xnxt;
       if (t + 1 < t1) {
-        load_tile(t + 1, hnext, nxt);
+        load_tile(t + 1, nxt);
         if (BP <= 4) load_x(t + 1, 0, xnxt);
       }
       // ---- compute tile t ----
@@ -394,44 +311,21 @@ __global__ void __launch_bounds__(kThreads, (Cfg<BP, B1, B2, STRIDED>::kMinBlock
         float xf[C::XB][16];
 #pragma unroll
         for (int b = 0; b < C::XB; ++b) unpack16(xs.v[b][0], xs.v[b][1], xf[b]);
-        if (hcur.sparse) {
 #pragma unroll
-          for (int j = 0; j < JS; ++j) {
-            const uint32_t w[4] = {cur.a[j].x, cur.a[j].y, cur.a[j].z, cur.a[j].w};
-            const uint32_t m = cur.b[j].x;
+        for (int j = 0; j < JS; ++j) {
+          float wf[16];
+          unpack16(cur.a[j], cur.b[j], wf);
 #pragma unroll
-            for (int g = 0; g < 4; ++g) {
-              const uint32_t nib = (m >> (4 * g)) & 0xFu;
-              const float v0 = bf16_lo(w[g]), v1 = bf16_hi(w[g]);
+          for (int e = 0; e < 16; ++e)
 #pragma unroll
-              for (int b = 0; b < C::XB; ++b) {
-                float xa, xb;
-                pick2(nib, xf[b][4 * g], xf[b][4 * g + 1], xf[b][4 * g + 2],
-                      xf[b][4 * g + 3], xa, xb);
-                acc[j][b0 + b] = fmaf(v0, xa, acc[j][b0 + b]);
-                acc[j][b0 + b] = fmaf(v1, xb, acc[j][b0 + b]);
-              }
-            }
-          }
-        } else {
-#pragma unroll
-          for (int j = 0; j < JS; ++j) {
-            float wf[16];
-            unpack16(cur.a[j], cur.b[j], wf);
-#pragma unroll
-            for (int e = 0; e < 16; ++e)
-#pragma unroll
-              for (int b = 0; b < C::XB; ++b)
-                acc[j][b0 + b] = fmaf(wf[e], xf[b][e], acc[j][b0 + b]);
-          }
+            for (int b = 0; b < C::XB; ++b)
+              acc[j][b0 + b] = fmaf(wf[e], xf[b][e], acc[j][b0 + b]);
         }
       }
       // band boundary or end of range: flush
       if (t + 1 == t1 || (t + 1) % p.tpr == 0) flush((int)(t / p.tpr));
       cur = nxt;
       xcur = xnxt;
-      hcur = hnext;
-      hnext = hnn;
     }
   }
 }
@@ -441,20 +335,22 @@ __global__ void __launch_bounds__(kThreads, (Cfg<BP, B1, B2, STRIDED>::kMinBlock
 // ---------------------------------------------------------------------------
 //
 // One CTA per SM.  CTA c owns the tiles whose packed byte offset falls in
-// [c, c+1) * total / G -- a contiguous piece of the packed stream, found by
-// one round of parallel search over the tile offsets at start-up.  A producer
-// warp copies that piece tile by tile (values, masks and the matching slice of
-// X) from HBM into a ring of shared-memory stages with 1-D bulk copies
-// (cp.async.bulk; completion counted on an mbarrier), so the bytes in flight
-// are set by the ring, not by registers.  B1/8 consumer warps, 8 tile rows
-// each, compute from shared memory and keep fp32 row sums in registers until
-// their piece of a tile-row band ends.
+// [c, c+1) * total / G -- a contiguous piece of the packed stream, taken from
+// the launch-parameter plan (or, without one, found by two rounds of parallel
+// search over the tile offsets at start-up).  A producer warp copies that
+// piece stage by stage (the values and masks of one to TPX tiles and the
+// matching slice of X) from HBM into a ring of shared-memory stages with 1-D
+// bulk copies (cp.async.bulk; X through a 2-D tensor map at batch >= 4;
+// completion counted on an mbarrier), so the bytes in flight are set by the
+// ring, not by registers.  B1/RW consumer warps, RW tile rows each, compute
+// from shared memory and keep fp32 row sums in registers until their piece of
+// a tile-row band ends.
 //
-// A band split between CTAs is summed through fp32 slots: CTA c writes its
-// share of band r to slot c + r, and a ticket per (band, warp) finds the last
-// contribution, whose warp sums the band's slots in CTA order (deterministic;
-// nothing spins, and a ticket's answer is only read after the next piece of
-// work, so the atomic's round trip is hidden).
+// A band piece goes to one of two epilogue warps (alternating), which stores
+// a band this CTA owns outright, or writes the piece to fp32 slot c + r; a
+// ticket per band finds the last of its CTAs, whose epilogue warp sums the
+// band's slots in CTA order (deterministic; nothing spins, and the consumers
+// go on with the next piece meanwhile).
 //
 // Products use the mixed-precision FMA of sm_100 (bf16 x bf16 + fp32 -> fp32,
 // exact product) straight on packed bf16 pairs, and PRMT picks the two x
@@ -1368,20 +1264,19 @@ Shape shape_of(int b1, int b2) {
   return kGeneric;
 }
 
-template <int BP, int B1, int B2, bool STRIDED>
-void *stream_kernel_ptr() {
-  return reinterpret_cast<void *>(&hybrid_stream_kernel<BP, B1, B2, STRIDED>);
+template <int BP, int B1, int B2>
+void *dense_kernel_ptr() {
+  return reinterpret_cast<void *>(&dense_gemv_kernel<BP, B1, B2>);
 }
 
-template <bool STRIDED>
-void *pick_stream_kernel(int bp, Shape s) {
+void *pick_dense_kernel(int bp, Shape s) {
 #define HYB_CASE(BP_)                                                  \
   case BP_:                                                            \
     switch (s) {                                                       \
-      case kS128x128: return stream_kernel_ptr<BP_, 128, 128, STRIDED>(); \
-      case kS128x64: return stream_kernel_ptr<BP_, 128, 64, STRIDED>();   \
-      case kS64x64: return stream_kernel_ptr<BP_, 64, 64, STRIDED>();     \
-      case kS64x128: return stream_kernel_ptr<BP_, 64, 128, STRIDED>();   \
+      case kS128x128: return dense_kernel_ptr<BP_, 128, 128>(); \
+      case kS128x64: return dense_kernel_ptr<BP_, 128, 64>();   \
+      case kS64x64: return dense_kernel_ptr<BP_, 64, 64>();     \
+      case kS64x128: return dense_kernel_ptr<BP_, 64, 128>();   \
       default: return nullptr;                                         \
     }
   switch (bp) {
@@ -1546,13 +1441,13 @@ int make_plan(int64_t n, int64_t k, int b1, int b2, int64_t total_bytes,
     P.G = tma_ctas(sms, total_bytes, b1, b2);
     if (!pick_tma_kernel(P.bp, s, &P.tk)) return HYB_ERR_UNSUPPORTED;
   }
-  P.stream = !P.tma && s != kGeneric && P.R <= 8192;
+  P.stream = strided && s != kGeneric && P.R <= 8192;
   P.dyn_smem = P.tma ? P.tk.smem : (P.stream ? (size_t)2 * P.R * sizeof(int) : 0);
   if (P.tma) {
     const int nb = blocks_per_sm(P.tk.fn, P.tk.smem, P.tk.threads);
     if (nb <= 0) return HYB_ERR_CUDA;
   } else if (P.stream) {
-    void *fn = pick_stream_kernel<true>(P.bp, s);
+    void *fn = pick_dense_kernel(P.bp, s);
     if (P.dyn_smem > 48 * 1024) {
       if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                (int)P.dyn_smem) != cudaSuccess)
@@ -1720,7 +1615,7 @@ int run_product(Params prm, int b1, int b2, int batch, const hyb_lowrank *lr,
         cudaSuccess)
       return HYB_ERR_CUDA;
   } else if (P.stream) {
-    void *fn = pick_stream_kernel<true>(P.bp, shape_of(b1, b2));
+    void *fn = pick_dense_kernel(P.bp, shape_of(b1, b2));
     if (cudaLaunchKernel(fn, dim3(P.G), dim3(kThreads), args, P.dyn_smem, s) !=
         cudaSuccess)
       return HYB_ERR_CUDA;
