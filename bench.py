@@ -207,8 +207,9 @@ class Workload:
         self.dws = hyb.new_workspace(hyb.dense_workspace_bytes(n, k, batch), device)
         # pre-marshalled C-ABI arguments (the timed loop only calls into C)
         L = hyb.lib()
-        self.fn = L.hyb_spmm_skinny
-        self.dfn = L.hyb_gemv_dense
+        self.fn = L.hyb_spmm_skinny_ex
+        self.dfn = L.hyb_gemv_dense_ex
+        self.flags = 0  # launch options of every call (hyb_*_ex)
         self.structs = [m.struct() for m in self.mats]
         self.dstructs = [m.struct() for m in self.dense_packed]
         self.stream = torch.cuda.current_stream(device)
@@ -222,18 +223,19 @@ class Workload:
         s = ctypes.c_void_p(stream.cuda_stream)
         n, k, batch = self.n, self.k, self.batch
         rotate = len(self.mats)
+        f = self.flags
         self.args = [(ctypes.byref(self.structs[i]), batch, ctypes.c_void_p(self.X[i].data_ptr()),
-                      k, ctypes.c_void_p(self.Y[i].data_ptr()), n, hyb.HYB_F32, None,
+                      k, ctypes.c_void_p(self.Y[i].data_ptr()), n, hyb.HYB_F32, None, f,
                       ctypes.c_void_p(self.ws.data_ptr()), self.ws.numel(), s)
                      for i in range(rotate)]
         self.pargs = [(ctypes.byref(self.dstructs[i]), batch,
                        ctypes.c_void_p(self.X[i].data_ptr()), k,
-                       ctypes.c_void_p(self.Y[i].data_ptr()), n, hyb.HYB_F32, None,
+                       ctypes.c_void_p(self.Y[i].data_ptr()), n, hyb.HYB_F32, None, f,
                        ctypes.c_void_p(self.ws.data_ptr()), self.ws.numel(), s)
                       for i in range(rotate)]
         self.dargs = [(n, k, batch, ctypes.c_void_p(self.dense[i].data_ptr()), k,
                        ctypes.c_void_p(self.X[i].data_ptr()), k,
-                       ctypes.c_void_p(self.Y[i].data_ptr()), n, hyb.HYB_F32,
+                       ctypes.c_void_p(self.Y[i].data_ptr()), n, hyb.HYB_F32, f,
                        ctypes.c_void_p(self.dws.data_ptr()), self.dws.numel(), s)
                       for i in range(rotate)]
 
@@ -290,11 +292,13 @@ def timed(fn, steps, warmup, stream, world=1):
     return ms
 
 
-def graph_timed(wl, fn, steps, warmup, world=1):
+def graph_timed(wl, fn, steps, warmup, world=1, flags=0):
     """Device time of `steps` calls captured in one CUDA graph and replayed
     (the launch path of a decode engine): warm-up calls run eagerly first;
     CUDA events on the replay stream, barrier + synchronize on both sides, max
-    over ranks."""
+    over ranks.  `flags`: the calls' launch options (HYB_LAUNCH_OVERLAP_PREV:
+    each call a programmatic dependent of the one before it)."""
+    wl.flags = flags
     side = torch.cuda.Stream()
     with torch.cuda.stream(side):
         wl.set_stream(side)
@@ -325,6 +329,8 @@ def graph_timed(wl, fn, steps, warmup, world=1):
         ms = max_over_ranks(ms, torch.device("cuda", torch.cuda.current_device()), world)
         torch.distributed.barrier()
     del g
+    wl.flags = 0
+    wl.set_stream(wl.stream)
     return ms
 
 
@@ -421,16 +427,23 @@ FP32_FMA_PER_SM_PER_CLK = 128   # fp32 lanes per SM (B200)
 
 
 class Calls:
-    """A rotation of pre-marshalled C-ABI calls (for graph_timed)."""
+    """A rotation of pre-marshalled calls of a hyb_*_ex entry point (for
+    graph_timed).  make_args gives each call's arguments without the launch
+    options, which go in front of the trailing (ws, ws_bytes, stream)."""
 
     def __init__(self, fn, make_args, count, name):
         self.fn, self.make_args, self.count, self.name = fn, make_args, count, name
+        self.flags = 0
         self.stream = torch.cuda.current_stream()
         self.set_stream(self.stream)
 
     def set_stream(self, stream):
         sp = ctypes.c_void_p(stream.cuda_stream)
-        self.args = [self.make_args(i, sp) for i in range(self.count)]
+        self.args = []
+        for i in range(self.count):
+            a = list(self.make_args(i, sp))
+            a.insert(len(a) - 3, self.flags)
+            self.args.append(tuple(a))
 
     def step(self, i):
         rc = self.fn(*self.args[i % self.count])
@@ -453,6 +466,7 @@ def sweep(device, steps=200, warmup=10):
     rank-128 low-rank term."""
     peak, peak_kind = measured_peak()
     L = hyb.lib()
+    OV = hyb.LAUNCH_OVERLAP_PREV
     l2 = 126 << 20
     sm_mhz = 1965.0
 
@@ -476,14 +490,15 @@ def sweep(device, steps=200, warmup=10):
                   for i in range(max(nrot_d, 16))] for b in (1, 4, 8, 16)}
         Ys = {b: [torch.empty(b, n, dtype=torch.float32, device=device)
                   for _ in range(max(nrot_d, 16))] for b in (1, 4, 8, 16)}
-        dense_us = {}
+        dense_us, dense_plain_us = {}, {}
         for b in ((1,) if role == "attn" else (1, 4, 8, 16)):
             dws = hyb.new_workspace(hyb.dense_workspace_bytes(n, k, b), device)
-            c = Calls(L.hyb_gemv_dense, lambda i, sp, b=b, dws=dws: (
+            c = Calls(L.hyb_gemv_dense_ex, lambda i, sp, b=b, dws=dws: (
                 n, k, b, ctypes.c_void_p(dense[i].data_ptr()), k,
                 ctypes.c_void_p(Xs[b][i].data_ptr()), k, ctypes.c_void_p(Ys[b][i].data_ptr()), n,
                 hyb.HYB_F32, ctypes.c_void_p(dws.data_ptr()), dws.numel(), sp), nrot_d, "dense")
-            dense_us[b] = graph_timed(c, c.step, steps, warmup) / steps * 1e3
+            dense_us[b] = graph_timed(c, c.step, steps, warmup, flags=OV) / steps * 1e3
+            dense_plain_us[b] = graph_timed(c, c.step, steps, warmup) / steps * 1e3
         del dense
         for f in fracs:
             T = (n // 128) * (k // 128)
@@ -498,11 +513,12 @@ def sweep(device, steps=200, warmup=10):
             for b in ((1,) if role == "attn" else (1, 4, 8, 16)):
                 ws = hyb.new_workspace(hyb.workspace_bytes(base, b), device)
                 xs, ys = Xs[b], Ys[b]
-                c = Calls(L.hyb_spmm_skinny, lambda i, sp, b=b, ws=ws, xs=xs, ys=ys: (
+                c = Calls(L.hyb_spmm_skinny_ex, lambda i, sp, b=b, ws=ws, xs=xs, ys=ys: (
                     ctypes.byref(structs[i]), b, ctypes.c_void_p(xs[i % len(xs)].data_ptr()), k,
                     ctypes.c_void_p(ys[i % len(ys)].data_ptr()), n, hyb.HYB_F32, None,
                     ctypes.c_void_p(ws.data_ptr()), ws.numel(), sp), nrot, "hybrid")
-                us = graph_timed(c, c.step, steps, warmup) / steps * 1e3
+                us = graph_timed(c, c.step, steps, warmup, flags=OV) / steps * 1e3
+                us_plain = graph_timed(c, c.step, steps, warmup) / steps * 1e3
                 nbytes = base.nbytes() + base.num_tiles + 2 * b * k + 4 * b * n
                 gbs = nbytes / (us * 1e-6) / 1e9
                 kept = base.n_vals  # kept entries = packed values
@@ -513,7 +529,9 @@ def sweep(device, steps=200, warmup=10):
                         "frac_of_8tbs": round(gbs / NOMINAL_HBM_GBS, 4),
                         "dense_us": round(dense_us[b], 3),
                         "speedup_vs_dense": round(dense_us[b] / us, 4),
-                        "format_bound_speedup": round((2 * n * k) / base.nbytes(), 4)}
+                        "format_bound_speedup": round((2 * n * k) / base.nbytes(), 4),
+                        "plain_launch": {"us": round(us_plain, 3),
+                                         "dense_us": round(dense_plain_us[b], 3)}}
                 if b >= 8:
                     line["alu_roofline"] = _alu_roofline(2 * b * kept, us, sm_mhz)
                 emit(line)
@@ -537,28 +555,32 @@ def sweep(device, steps=200, warmup=10):
     ys = [torch.empty(1, n, dtype=torch.float32, device=device) for n, k in shapes8]
     ws = hyb.new_workspace(max(hyb.workspace_bytes(m, 1) for m in mats), device)
     structs = [m.struct() for m in mats]
-    chain = Calls(L.hyb_spmm_skinny, lambda i, sp: (
+    chain = Calls(L.hyb_spmm_skinny_ex, lambda i, sp: (
         ctypes.byref(structs[i]), 1, ctypes.c_void_p(xs[i].data_ptr()), shapes8[i][1],
         ctypes.c_void_p(ys[i].data_ptr()), shapes8[i][0], hyb.HYB_F32, None,
         ctypes.c_void_p(ws.data_ptr()), ws.numel(), sp), len(mats), "chain")
     reps = 4
-    ms = graph_timed(chain, chain.step, reps * len(mats), len(mats))
+    ms = graph_timed(chain, chain.step, reps * len(mats), len(mats), flags=OV)
+    ms_plain = graph_timed(chain, chain.step, reps * len(mats), len(mats))
     packed = sum(m.nbytes() + m.num_tiles for m in mats)
     nbytes = packed + sum(2 * k + 4 * n for n, k in shapes8)
     dws = hyb.new_workspace(max(hyb.dense_workspace_bytes(n, k, 1) for n, k in shapes8), device)
     roles8 = [r for _ in range(32) for r, _, _ in inputs.LLAMA8B_LAYER]
-    dchain = Calls(L.hyb_gemv_dense, lambda i, sp: (
+    dchain = Calls(L.hyb_gemv_dense_ex, lambda i, sp: (
         shapes8[i][0], shapes8[i][1], 1, ctypes.c_void_p(W_role[roles8[i]].data_ptr()), shapes8[i][1],
         ctypes.c_void_p(xs[i].data_ptr()), shapes8[i][1], ctypes.c_void_p(ys[i].data_ptr()),
         shapes8[i][0], hyb.HYB_F32, ctypes.c_void_p(dws.data_ptr()), dws.numel(), sp),
         len(mats), "dense chain")
-    dms = graph_timed(dchain, dchain.step, reps * len(mats), len(mats))
+    dms = graph_timed(dchain, dchain.step, reps * len(mats), len(mats), flags=OV)
+    dms_plain = graph_timed(dchain, dchain.step, reps * len(mats), len(mats))
     us_chain = ms / reps * 1e3
     emit({"sweep": "llama8b_chain", "matrices": len(mats), "tile": "128x64", "batch": 1,
           "us_per_chain": round(us_chain, 2), "us_per_matrix": round(us_chain / len(mats), 3),
           "GBps": round(nbytes / (us_chain * 1e-6) / 1e9, 1), "packed_GB": round(packed / 1e9, 3),
           "dense_us_per_chain": round(dms / reps * 1e3, 2),
           "speedup_vs_dense": round(dms / ms, 4),
+          "plain_launch": {"us_per_chain": round(ms_plain / reps * 1e3, 2),
+                           "dense_us_per_chain": round(dms_plain / reps * 1e3, 2)},
           "note": "one weight draw per role; tile maps drawn per layer (f_l ~ U[0.2,1])"})
     del mats, structs, W_role, xs, ys, ws, dws
     torch.cuda.empty_cache()
@@ -586,18 +608,20 @@ def sweep(device, steps=200, warmup=10):
         xs = [inputs.activations(b, k, inputs.seed_of("l70", i, b)).to(device) for i, (n, k) in enumerate(sh70)]
         ys = [torch.empty(b, n, dtype=torch.float32, device=device) for n, k in sh70]
         ws = hyb.new_workspace(max(hyb.workspace_bytes(m, b, 128) for m in mats70), device)
-        c = Calls(L.hyb_spmm_skinny, lambda i, sp, b=b, ws=ws, xs=xs, ys=ys: (
+        c = Calls(L.hyb_spmm_skinny_ex, lambda i, sp, b=b, ws=ws, xs=xs, ys=ys: (
             ctypes.byref(structs[i]), b, ctypes.c_void_p(xs[i].data_ptr()), sh70[i][1],
             ctypes.c_void_p(ys[i].data_ptr()), sh70[i][0], hyb.HYB_F32, ctypes.byref(lrstructs[i]),
             ctypes.c_void_p(ws.data_ptr()), ws.numel(), sp), 24, "70b")
-        ms = graph_timed(c, c.step, 48, 24)
+        ms = graph_timed(c, c.step, 48, 24, flags=OV)
         us = ms / 2 * 1e3
+        us_plain = graph_timed(c, c.step, 48, 24) / 2 * 1e3
         nbytes = sum(m.nbytes() + m.num_tiles + 2 * b * k + 4 * b * n + 2 * 128 * (n + k)
                      for m, (n, k) in zip(mats70, sh70))
         gbs = nbytes / (us * 1e-6) / 1e9
         line = {"sweep": "llama70b_ffn_lowrank", "matrices": 24, "batch": b, "rank": 128,
                 "us_per_8_layers": round(us, 2), "us_per_matrix": round(us / 24, 3),
-                "GBps": round(gbs, 1), "frac_of_measured_hbm": round(gbs / peak, 4)}
+                "GBps": round(gbs, 1), "frac_of_measured_hbm": round(gbs / peak, 4),
+                "plain_launch": {"us_per_8_layers": round(us_plain, 2)}}
         if b >= 8:
             kept = sum(m.n_vals for m in mats70)
             flops = 2 * b * kept + sum(2 * b * 128 * (n + k) for n, k in sh70)
@@ -658,11 +682,20 @@ def main():
         if rank == 0:
             print(json.dumps({"profile_run": args.workload, "ms": ms, "steps": args.steps}))
         return 0
+    # Every leg runs as a decode engine would run a chain of layers: K calls
+    # captured in one CUDA graph, each launched as a programmatic dependent of
+    # the one before (HYB_LAUNCH_OVERLAP_PREV); the same legs launched plainly
+    # (each product starts after the previous one has drained) are reported
+    # beside them.
+    ov = hyb.LAUNCH_OVERLAP_PREV
     with ClockSampler(local) as clocks:
-        ms = graph_timed(wl, wl.step, args.steps, args.warmup, world)
+        ms = graph_timed(wl, wl.step, args.steps, args.warmup, world, flags=ov)
+    plain_ms = graph_timed(wl, wl.step, args.steps, args.warmup, world)
     eager_ms = timed(wl.step, args.steps, args.warmup, stream, world)
-    dense_ms = graph_timed(wl, wl.dense_step, args.steps, args.warmup, world)
-    dpk_ms = graph_timed(wl, wl.dense_packed_step, args.steps, args.warmup, world)
+    dense_ms = graph_timed(wl, wl.dense_step, args.steps, args.warmup, world, flags=ov)
+    dense_plain_ms = graph_timed(wl, wl.dense_step, args.steps, args.warmup, world)
+    dpk_ms = graph_timed(wl, wl.dense_packed_step, args.steps, args.warmup, world, flags=ov)
+    dpk_plain_ms = graph_timed(wl, wl.dense_packed_step, args.steps, args.warmup, world)
     e2e_ms, h2d, d2h = e2e_timed(wl, args.steps, args.warmup, stream, world)
 
     per_step_ms = ms / args.steps
@@ -678,8 +711,13 @@ def main():
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
         "config": workload_config(args.workload, wl.frac_real),
         "us_per_matrix": round(per_step_ms * 1e3, 3),
-        "launch": "CUDA graph of the K steps (eager launches: %.3f us per matrix)"
-                  % (eager_ms / args.steps * 1e3),
+        "launch": "CUDA graph of the K steps, each a programmatic dependent of the one "
+                  "before (HYB_LAUNCH_OVERLAP_PREV)",
+        "plain_launch_us_per_matrix": {
+            "graph": round(plain_ms / args.steps * 1e3, 3),
+            "eager": round(eager_ms / args.steps * 1e3, 3),
+            "dense": round(dense_plain_ms / args.steps * 1e3, 3),
+            "dense_packed": round(dpk_plain_ms / args.steps * 1e3, 3)},
         "dense_us_per_matrix": round(dense_us, 3),
         "speedup_vs_dense": round(dense_us / (per_step_ms * 1e3), 4),
         "dense_packed_us_per_matrix": round(dpk_ms / args.steps * 1e3, 3),

@@ -192,6 +192,29 @@ HYB_API int hyb_spmm_skinny(const hyb_matrix *A, int batch, const uint16_t *X,
                     const hyb_lowrank *lr, void *ws, size_t ws_bytes,
                     hyb_stream_t stream);
 
+/* Launch options of the _ex entry points (bit set; unknown bits are
+ * rejected with HYB_ERR_INVALID_ARG). */
+#define HYB_LAUNCH_OVERLAP_PREV 1u
+/* HYB_LAUNCH_OVERLAP_PREV: launch the streaming kernel as a programmatic
+ * dependent of the kernel queued before it on the stream, so that a chain of
+ * products (one decode step's layers, back to back) does not drain the GPU
+ * between them: while the preceding kernel's last CTAs finish, this product's
+ * CTAs start on the SMs it frees and request their first ring of weight
+ * bytes.  They read X, and read or write Y, the workspace and the low-rank
+ * intermediates, only after the preceding kernel has completed and its
+ * writes are visible (griddepcontrol.wait), so results are identical with
+ * and without the flag.  The caller guarantees that the weights -- A's tile
+ * map, values, masks and offsets (or W for hyb_gemv_dense_ex) -- are not
+ * written by the work queued before the call on the stream that has not
+ * finished by then.  Tilings served by the one-warp-per-row kernel ignore
+ * the flag. */
+
+/* hyb_spmm_skinny with launch options `flags` (0 = hyb_spmm_skinny). */
+HYB_API int hyb_spmm_skinny_ex(const hyb_matrix *A, int batch, const uint16_t *X,
+                               int64_t ldx, void *Y, int64_t ldy, hyb_dtype ydt,
+                               const hyb_lowrank *lr, uint32_t flags, void *ws,
+                               size_t ws_bytes, hyb_stream_t stream);
+
 /* Workspace bytes for hyb_lowrank_add. */
 HYB_API size_t hyb_lowrank_workspace_bytes(int64_t k, int batch, int rank);
 
@@ -214,6 +237,13 @@ HYB_API int hyb_gemv_dense(int64_t n, int64_t k, int batch, const uint16_t *W,
                    int64_t ldw, const uint16_t *X, int64_t ldx, void *Y,
                    int64_t ldy, hyb_dtype ydt, void *ws, size_t ws_bytes,
                    hyb_stream_t stream);
+
+/* hyb_gemv_dense with launch options `flags` (see HYB_LAUNCH_OVERLAP_PREV;
+ * 0 = hyb_gemv_dense). */
+HYB_API int hyb_gemv_dense_ex(int64_t n, int64_t k, int batch, const uint16_t *W,
+                              int64_t ldw, const uint16_t *X, int64_t ldx, void *Y,
+                              int64_t ldy, hyb_dtype ydt, uint32_t flags, void *ws,
+                              size_t ws_bytes, hyb_stream_t stream);
 
 /* ---- product without any allocation ------------------------------------ */
 

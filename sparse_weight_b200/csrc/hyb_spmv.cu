@@ -74,7 +74,23 @@ struct Params {
   uint32_t *counters;
   uint32_t *status;  // workspace status word
   int64_t nvb, nmb;  // bytes of the value and mask buffers
+  // 1: launched as a programmatic dependent of the preceding kernel on the
+  // stream.  The weights (packed matrix or row-major W) may then be read
+  // before that kernel has finished; X, Y, the workspace and the low-rank
+  // intermediates are touched only after griddepcontrol.wait.
+  int pdl;
 };
+
+// Programmatic dependent launch (sm_90+): let the next grid on the stream, if
+// it was launched as a programmatic dependent, start its CTAs as this grid's
+// CTAs exit; and wait until the preceding grid has completed and its memory
+// is visible.  Both are no-ops for a grid launched without the attribute.
+__device__ __forceinline__ void grid_dep_trigger() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+__device__ __forceinline__ void grid_dep_wait() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+}
 
 // Work split made once per matrix (hyb_make_plan) and handed to the streaming
 // kernel as launch parameters, so that a CTA issues its first copy without
@@ -179,6 +195,7 @@ __global__ void __launch_bounds__(kThreads, (Cfg<BP, B1, B2>::kMinBlocks))
   const int rs = lane / C::CPR;  // row inside a step
   const int c = blockIdx.x;
   const int G = p.G;
+  if (p.pdl) grid_dep_trigger();
 
   // ---- 1. this CTA's tile range [t0, t1) -----------------------------------
   const int64_t tgtA = (int64_t)c * p.total;
@@ -290,6 +307,9 @@ __global__ void __launch_bounds__(kThreads, (Cfg<BP, B1, B2>::kMinBlocks))
   if (t0 < t1) {
     TileRegs<JS> cur;
     load_tile(t0, cur);
+    // the first tile of W is on its way; X and everything written below may
+    // belong to the preceding grid
+    if (p.pdl) grid_dep_wait();
     XRegs<C::XB> xcur;
     if (BP <= 4) load_x(t0, 0, xcur);
     for (int64_t t = t0; t < t1; ++t) {
@@ -537,6 +557,7 @@ __global__ void __launch_bounds__(TmaCfg<BP, B1, B2>::kThreads, 1)
   // barriers are set up rather than when the producer first needs it.
   __shared__ int64_t s_rec[5];
   const bool planned = lp.kind == kPlanTiles;
+  if (p.pdl) grid_dep_trigger();
   if (planned && tid == 32 * C::NC + 1) {
     s_rec[0] = lp.rec[4 * c];
     s_rec[1] = lp.rec[4 * (c + 1)];
@@ -670,6 +691,36 @@ __global__ void __launch_bounds__(TmaCfg<BP, B1, B2>::kThreads, 1)
     uint32_t phase = 0;
     bool ok = true;
     uint32_t armed = 0, armed_parity = 0;  // per stage: copies issued / phase parity
+    // X of a stage: whole tensor-map boxes (rows past the batch and columns
+    // past k are zero-filled and counted in the transaction bytes), or one
+    // 1-D copy per batch row
+    auto issue_x = [&](int st_i, int64_t xcol, int nt) {
+      uint8_t *xdst = smem + (size_t)st_i * C::kStageBytes + C::kValsBytes + C::kMetaBytes;
+      if constexpr (C::XTM) {
+        const int ngx = (nt + C::XT - 1) / C::XT;
+        for (int q = 0; q < ngx; ++q)
+          tma_load_2d(xdst + q * C::kXCopy, &xmap, (int)(xcol + q * C::XT * B2), 0,
+                      &full_bar[st_i]);
+      } else {
+        const uint32_t xrow = (uint32_t)(2 * B2 * nt);
+        for (int b = 0; b < p.batch; ++b)
+          bulk_g2s(xdst + b * C::kXBatch, p.X + xcol + (int64_t)b * p.ldx, xrow, &full_bar[st_i]);
+      }
+    };
+    // As a programmatic dependent, the first ring's worth of stages gets its
+    // weight bytes requested at once and its X only after the preceding grid
+    // has finished (it may have written X); the lane that armed a stage keeps
+    // the stage's X request until then.  Warp-uniform: pend, issued.
+    bool pend = p.pdl != 0;
+    int issued = 0;
+    int dx_stage = -1, dx_nt = 0;
+    int64_t dx_col = 0;
+    auto release_x = [&]() {
+      grid_dep_wait();
+      if (dx_stage >= 0) issue_x(dx_stage, dx_col, dx_nt);
+      dx_stage = -1;
+      pend = false;
+    };
     Win cur;
     bool derived = false;
     if (planned) {
@@ -719,6 +770,7 @@ __global__ void __launch_bounds__(TmaCfg<BP, B1, B2>::kThreads, 1)
       while (todo) {
         const int k = __ffs(todo) - 1;
         todo &= todo - 1;
+        if (pend && issued == S) release_x();  // the ring is armed: X can wait no longer
         if (lane == k && is_start) {
           if (!mbar_wait(&empty_bar[stage], phase ^ 1u)) {
             ok = false;
@@ -745,29 +797,27 @@ __global__ void __launch_bounds__(TmaCfg<BP, B1, B2>::kThreads, 1)
             bulk_g2s(st, p.vals + 2 * cur.vo, vbytes, &full_bar[stage]);
             if (mbytes) bulk_g2s(st + C::kValsBytes, p.meta + cur.mo, mbytes, &full_bar[stage]);
             const int64_t xcol = (ts - band * tpr) * B2;  // first X column of the stage
-            uint8_t *xdst = st + C::kValsBytes + C::kMetaBytes;
-            if constexpr (C::XTM) {
-              // whole boxes: rows past the batch and columns past k are
-              // zero-filled and counted in the transaction bytes
-              for (int q = 0; q < ngx; ++q)
-                tma_load_2d(xdst + q * C::kXCopy, &xmap, (int)(xcol + q * C::XT * B2), 0,
-                            &full_bar[stage]);
+            if (pend) {
+              dx_stage = stage;
+              dx_col = xcol;
+              dx_nt = nt;
             } else {
-              for (int b = 0; b < p.batch; ++b)
-                bulk_g2s(xdst + b * C::kXBatch, p.X + xcol + (int64_t)b * p.ldx, xrow,
-                         &full_bar[stage]);
+              issue_x(stage, xcol, nt);
             }
           }
         }
         // every lane keeps the ring position
+        ++issued;
         if (++stage == S) {
           stage = 0;
           phase ^= 1u;
         }
       }
+      if (pend) release_x();  // at the latest after the first window
       ok = __all_sync(0xffffffffu, ok);
       cur = nxt;
     }
+    if (pend) release_x();  // (no window at all)
     // lanes kept identical ring positions; lane 0 closes the ring
     if (lane == 0) {
       if (ok && mbar_wait(&empty_bar[stage], phase ^ 1u)) {
@@ -799,6 +849,9 @@ __global__ void __launch_bounds__(TmaCfg<BP, B1, B2>::kThreads, 1)
     // c + r, and a ticket per band finds the last of its CTAs, which sums the
     // band's slots in CTA order (deterministic).  All global-memory ordering
     // (release, acquire) happens here, off the consumer warps' path.
+    // Y, the slots, the tickets and the low-rank term may belong to the
+    // preceding grid until it has finished.
+    if (p.pdl) grid_dep_wait();
     auto owner_of_p = [&](int64_t P) -> int {
       const int64_t o = (P * G) / p.total;
       return (int)(o < G - 1 ? o : G - 1);
@@ -1566,9 +1619,28 @@ void fill_launch_plan(const int64_t *plan, int32_t plan_ctas, const Plan &P, con
   lp->ctas = P.G;
 }
 
+// A launch, as a programmatic dependent of the preceding kernel on the stream
+// when pdl is set (the kernel then orders its own accesses with
+// griddepcontrol.wait).
+cudaError_t launch_kernel(const void *fn, dim3 grid, dim3 block, void **args, size_t smem,
+                          cudaStream_t s, bool pdl) {
+  if (!pdl) return cudaLaunchKernel(fn, grid, block, args, smem, s);
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelExC(&cfg, fn, args);
+}
+
 int run_product(Params prm, int b1, int b2, int batch, const hyb_lowrank *lr,
                 bool strided, void *ws, size_t ws_bytes, cudaStream_t s,
-                const int64_t *plan = nullptr, int32_t plan_ctas = 0) {
+                const int64_t *plan = nullptr, int32_t plan_ctas = 0, uint32_t flags = 0) {
   const int rank = (lr && lr->rank > 0) ? lr->rank : 0;
   Plan P;
   int rc = make_plan(prm.n, prm.k, b1, b2, prm.total, batch, rank, strided, &P);
@@ -1601,6 +1673,8 @@ int run_product(Params prm, int b1, int b2, int batch, const hyb_lowrank *lr,
     prm.lr_ut = ut;
   }
   prm.status = reinterpret_cast<uint32_t *>(w);
+  const bool pdl = (flags & HYB_LAUNCH_OVERLAP_PREV) != 0 && (P.tma || P.stream);
+  prm.pdl = pdl ? 1 : 0;
   void *args[] = {&prm};
   if (P.tma) {
     LaunchPlan lp;
@@ -1611,13 +1685,12 @@ int run_product(Params prm, int b1, int b2, int batch, const hyb_lowrank *lr,
       if (rc != HYB_OK) return rc;
     }
     void *targs[] = {&prm, &lp, &xmap};
-    if (cudaLaunchKernel(P.tk.fn, dim3(P.G), dim3(P.tk.threads), targs, P.tk.smem, s) !=
+    if (launch_kernel(P.tk.fn, dim3(P.G), dim3(P.tk.threads), targs, P.tk.smem, s, pdl) !=
         cudaSuccess)
       return HYB_ERR_CUDA;
   } else if (P.stream) {
     void *fn = pick_dense_kernel(P.bp, shape_of(b1, b2));
-    if (cudaLaunchKernel(fn, dim3(P.G), dim3(kThreads), args, P.dyn_smem, s) !=
-        cudaSuccess)
+    if (launch_kernel(fn, dim3(P.G), dim3(kThreads), args, P.dyn_smem, s, pdl) != cudaSuccess)
       return HYB_ERR_CUDA;
   } else {
     void *fn = strided ? pick_rowwarp_kernel<true>(P.bp)
@@ -1650,8 +1723,9 @@ int check_io(const uint16_t *X, int64_t ldx, void *Y, int64_t ldy, int64_t n,
 
 int spmm_impl(const hyb_matrix *A, int batch, const uint16_t *X, int64_t ldx,
               void *Y, int64_t ldy, hyb_dtype ydt, const hyb_lowrank *lr,
-              void *ws, size_t ws_bytes, cudaStream_t s) {
+              void *ws, size_t ws_bytes, cudaStream_t s, uint32_t flags = 0) {
   if (!A) return HYB_ERR_INVALID_ARG;
+  if (flags & ~HYB_LAUNCH_OVERLAP_PREV) return HYB_ERR_INVALID_ARG;
   int rc = check_tiling(A->n, A->k, A->b1, A->b2);
   if (rc != HYB_OK) return rc;
   if (A->num_tiles != (A->n / A->b1) * (A->k / A->b2)) return HYB_ERR_INVALID_ARG;
@@ -1687,7 +1761,7 @@ int spmm_impl(const hyb_matrix *A, int batch, const uint16_t *X, int64_t ldx,
   prm.nvb = 2 * A->n_vals;
   prm.nmb = A->n_meta_bytes;
   return run_product(prm, A->b1, A->b2, batch, lr, false, ws, ws_bytes, s, A->plan,
-                     A->plan_ctas);
+                     A->plan_ctas, flags);
 }
 
 // Virtual tiling of a plain row-major W for the dense baseline.
@@ -1787,6 +1861,13 @@ int hyb_spmm_skinny(const hyb_matrix *A, int batch, const uint16_t *X,
                    (cudaStream_t)stream);
 }
 
+int hyb_spmm_skinny_ex(const hyb_matrix *A, int batch, const uint16_t *X, int64_t ldx,
+                       void *Y, int64_t ldy, hyb_dtype ydt, const hyb_lowrank *lr,
+                       uint32_t flags, void *ws, size_t ws_bytes, hyb_stream_t stream) {
+  return spmm_impl(A, batch, X, ldx, Y, ldy, ydt, lr, ws, ws_bytes, (cudaStream_t)stream,
+                   flags);
+}
+
 size_t hyb_lowrank_workspace_bytes(int64_t k, int batch, int rank) {
   if (k <= 0 || batch < 1 || batch > 16 || rank < 1 || rank > kMaxRank) return 0;
   size_t a, b, c;
@@ -1853,6 +1934,13 @@ int hyb_gemv_dense(int64_t n, int64_t k, int batch, const uint16_t *W,
                    int64_t ldw, const uint16_t *X, int64_t ldx, void *Y,
                    int64_t ldy, hyb_dtype ydt, void *ws, size_t ws_bytes,
                    hyb_stream_t stream) {
+  return hyb_gemv_dense_ex(n, k, batch, W, ldw, X, ldx, Y, ldy, ydt, 0, ws, ws_bytes, stream);
+}
+
+int hyb_gemv_dense_ex(int64_t n, int64_t k, int batch, const uint16_t *W, int64_t ldw,
+                      const uint16_t *X, int64_t ldx, void *Y, int64_t ldy, hyb_dtype ydt,
+                      uint32_t flags, void *ws, size_t ws_bytes, hyb_stream_t stream) {
+  if (flags & ~HYB_LAUNCH_OVERLAP_PREV) return HYB_ERR_INVALID_ARG;
   if (n <= 0 || k <= 0 || !W || ldw < k) return HYB_ERR_INVALID_ARG;
   if (k % 16 != 0) return HYB_ERR_INVALID_ARG;
   int rc = check_io(X, ldx, Y, ldy, n, k, batch, ydt);
@@ -1878,7 +1966,7 @@ int hyb_gemv_dense(int64_t n, int64_t k, int batch, const uint16_t *W,
   prm.ydt = ydt;
   prm.total = 2 * n * k;
   return run_product(prm, b1, b2, batch, nullptr, true, ws, ws_bytes,
-                     (cudaStream_t)stream);
+                     (cudaStream_t)stream, nullptr, 0, flags);
 }
 
 }  // extern "C"

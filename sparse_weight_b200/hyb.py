@@ -28,6 +28,7 @@ HYB_ERR_TIMEOUT = -7
 
 HYB_F32 = 0
 HYB_BF16 = 1
+LAUNCH_OVERLAP_PREV = 1  # HYB_LAUNCH_OVERLAP_PREV
 
 STATUS_NAN = 1
 STATUS_BAD_MAP = 2
@@ -67,7 +68,8 @@ EXPORTS = ["hyb_packed_sizes", "hyb_pack_workspace_bytes", "hyb_pack",
            "hyb_spmm_skinny", "hyb_lowrank_workspace_bytes", "hyb_lowrank_add",
            "hyb_dense_workspace_bytes", "hyb_gemv_dense", "hyb_check_status",
            "hyb_status_string", "hyb_spmv_noalloc", "hyb_spmv_noalloc_max_scratch_bytes",
-           "hyb_plan_entries", "hyb_make_plan", "hyb_selftest_wait_timeout"]
+           "hyb_plan_entries", "hyb_make_plan", "hyb_selftest_wait_timeout",
+           "hyb_spmm_skinny_ex", "hyb_gemv_dense_ex"]
 
 
 def lib():
@@ -95,6 +97,9 @@ def lib():
     L.hyb_spmm_skinny.argtypes = [ctypes.POINTER(HybMatrix), _I, _P, _I64, _P, _I64, _I,
                                   ctypes.POINTER(HybLowrank), _P, _SZ, _P]
     L.hyb_spmm_skinny.restype = _I
+    L.hyb_spmm_skinny_ex.argtypes = [ctypes.POINTER(HybMatrix), _I, _P, _I64, _P, _I64, _I,
+                                     ctypes.POINTER(HybLowrank), ctypes.c_uint32, _P, _SZ, _P]
+    L.hyb_spmm_skinny_ex.restype = _I
     L.hyb_lowrank_workspace_bytes.argtypes = [_I64, _I, _I]
     L.hyb_lowrank_workspace_bytes.restype = _SZ
     L.hyb_lowrank_add.argtypes = [_I64, _I64, _I, ctypes.POINTER(HybLowrank), _P, _I64,
@@ -105,6 +110,9 @@ def lib():
     L.hyb_gemv_dense.argtypes = [_I64, _I64, _I, _P, _I64, _P, _I64, _P, _I64, _I, _P,
                                  _SZ, _P]
     L.hyb_gemv_dense.restype = _I
+    L.hyb_gemv_dense_ex.argtypes = [_I64, _I64, _I, _P, _I64, _P, _I64, _P, _I64, _I,
+                                    ctypes.c_uint32, _P, _SZ, _P]
+    L.hyb_gemv_dense_ex.restype = _I
     L.hyb_check_status.argtypes = [_P, _P, ctypes.POINTER(ctypes.c_uint32)]
     L.hyb_check_status.restype = _I
     L.hyb_selftest_wait_timeout.argtypes = [_P, _SZ, ctypes.c_uint32, _P]
@@ -315,8 +323,12 @@ def _out(n, batch, ydt, device, Y):
 
 
 def spmm_skinny(A: Packed, X: torch.Tensor, Y: torch.Tensor = None, ydt: int = HYB_F32,
-                lowrank=None, ws: torch.Tensor = None, stream=None) -> torch.Tensor:
-    """hyb_spmm_skinny: Y[batch][n] = W_hat X (+ U (V^T X)); X bf16 [batch][k]."""
+                lowrank=None, ws: torch.Tensor = None, stream=None,
+                flags: int = 0) -> torch.Tensor:
+    """hyb_spmm_skinny_ex: Y[batch][n] = W_hat X (+ U (V^T X)); X bf16 [batch][k].
+    flags: LAUNCH_OVERLAP_PREV lets the kernel start streaming A before the
+    kernel queued ahead of it on the stream has finished (A must not be
+    written by that kernel)."""
     Xb = _bits(X)
     if Xb.dim() == 1:
         Xb = Xb.view(1, -1)
@@ -326,9 +338,9 @@ def spmm_skinny(A: Packed, X: torch.Tensor, Y: torch.Tensor = None, ydt: int = H
     if ws is None:
         ws = new_workspace(workspace_bytes(A, batch, lr.rank if lr else 0), Xb.device)
     s = A.struct()
-    _check("hyb_spmm_skinny", lib().hyb_spmm_skinny(
+    _check("hyb_spmm_skinny_ex", lib().hyb_spmm_skinny_ex(
         ctypes.byref(s), batch, _ptr(Xb), Xb.stride(0), _ptr(Y), Y.stride(0), ydt,
-        ctypes.byref(lr) if lr else None, _ptr(ws), ws.numel(), _stream(stream)))
+        ctypes.byref(lr) if lr else None, flags, _ptr(ws), ws.numel(), _stream(stream)))
     return Y
 
 
@@ -373,8 +385,10 @@ def dense_workspace_bytes(n: int, k: int, batch: int = 1) -> int:
 
 
 def gemv_dense(W: torch.Tensor, X: torch.Tensor, Y: torch.Tensor = None,
-               ydt: int = HYB_F32, ws: torch.Tensor = None, stream=None) -> torch.Tensor:
-    """hyb_gemv_dense: Y[batch][n] = W X for a plain row-major bf16 W [n][k]."""
+               ydt: int = HYB_F32, ws: torch.Tensor = None, stream=None,
+               flags: int = 0) -> torch.Tensor:
+    """hyb_gemv_dense_ex: Y[batch][n] = W X for a plain row-major bf16 W [n][k]
+    (flags as for spmm_skinny)."""
     Wb = _bits(W)
     Xb = _bits(X)
     if Xb.dim() == 1:
@@ -384,9 +398,9 @@ def gemv_dense(W: torch.Tensor, X: torch.Tensor, Y: torch.Tensor = None,
     Y = _out(n, batch, ydt, Xb.device, Y)
     if ws is None:
         ws = new_workspace(dense_workspace_bytes(n, k, batch), Xb.device)
-    _check("hyb_gemv_dense", lib().hyb_gemv_dense(
+    _check("hyb_gemv_dense_ex", lib().hyb_gemv_dense_ex(
         n, k, batch, _ptr(Wb), Wb.stride(0), _ptr(Xb), Xb.stride(0), _ptr(Y), Y.stride(0),
-        ydt, _ptr(ws), ws.numel(), _stream(stream)))
+        ydt, flags, _ptr(ws), ws.numel(), _stream(stream)))
     return Y
 
 

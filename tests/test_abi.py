@@ -143,6 +143,26 @@ def test_spmv_argument_checks(L):
                              None) == hyb.HYB_ERR_INVALID_ARG
 
 
+def test_launch_flags_checked(L):
+    """The _ex entry points reject unknown launch-option bits before anything
+    is queued (the valid bit, HYB_LAUNCH_OVERLAP_PREV, is exercised on the GPU)."""
+    P = ctypes.c_void_p
+    A = _matrix()
+    X, Y, ws = P(0x60000), P(0x70000), P(0x80000)
+    for flags in (2, 0x80000000, 3):
+        assert L.hyb_spmm_skinny_ex(ctypes.byref(A), 1, X, 256, Y, 256, 0, None, flags, ws,
+                                    1 << 20, None) == hyb.HYB_ERR_INVALID_ARG
+        assert L.hyb_gemv_dense_ex(64, 64, 1, P(0x10000), 64, X, 64, Y, 64, 0, flags, ws,
+                                   1 << 20, None) == hyb.HYB_ERR_INVALID_ARG
+    # the flag does not bypass the other checks
+    assert L.hyb_spmm_skinny_ex(ctypes.byref(A), 17, X, 256, Y, 256, 0, None,
+                                hyb.LAUNCH_OVERLAP_PREV, ws, 1 << 20,
+                                None) == hyb.HYB_ERR_INVALID_ARG
+    assert L.hyb_gemv_dense_ex(64, 40, 1, P(0x10000), 40, X, 40, Y, 64, 0,
+                               hyb.LAUNCH_OVERLAP_PREV, ws, 1 << 20,
+                               None) == hyb.HYB_ERR_INVALID_ARG
+
+
 def test_dense_and_lowrank_argument_checks(L):
     P = ctypes.c_void_p
     W, X, Y, ws = P(0x10000), P(0x60000), P(0x70000), P(0x80000)
