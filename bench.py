@@ -51,6 +51,8 @@ WORKLOADS = {
     "ffn_down_4096x14336_f0.5_b4": (4096, 14336, 128, 128, 0.5, 4, 0.02, 0.01),
     "ffn_down_4096x14336_f0.5_b8": (4096, 14336, 128, 128, 0.5, 8, 0.02, 0.01),
     "ffn_down_4096x14336_f0.5_b16": (4096, 14336, 128, 128, 0.5, 16, 0.02, 0.01),
+    "ffn_down_4096x14336_f0.0_b1": (4096, 14336, 128, 128, 0.0, 1, 0.02, 0.01),
+    "ffn_down_4096x14336_f1.0_b1": (4096, 14336, 128, 128, 1.0, 1, 0.02, 0.01),
 }
 
 

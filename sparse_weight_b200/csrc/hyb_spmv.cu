@@ -374,8 +374,11 @@ __global__ void __launch_bounds__(kThreads, (Cfg<BP, B1, B2>::kMinBlocks))
 //
 // Products use the mixed-precision FMA of sm_100 (bf16 x bf16 + fp32 -> fp32,
 // exact product) straight on packed bf16 pairs, and PRMT picks the two x
-// values of a 2:4 group from its 4-bit mask through a 16-entry selector table
-// ("SparseDecoding", authors' abstract: bitmask-indexed N:M SpMV).
+// values of a 2:4 group from its 4-bit mask ("SparseDecoding", authors'
+// abstract: bitmask-indexed N:M SpMV); the PRMT selector comes from two more
+// PRMTs at batch <= 4 and from a 16-entry shared table above.  Masks are
+// expected to have two bits set (as hyb_pack writes them); any other mask
+// still selects within the group's four values.
 
 constexpr uint32_t kWaitLimit = 1u << 22;
 
@@ -989,9 +992,32 @@ __global__ void __launch_bounds__(TmaCfg<BP, B1, B2>::kThreads, 1)
             const uint32_t m = *reinterpret_cast<const uint16_t *>(
                 st + C::kValsBytes + moff + row * (B2 / 8) + 2 * cp);
             const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+            // PRMT selector of each group: (p0, p1) -- the lowest and highest
+            // kept column -- becomes bytes {2p0, 2p0+1, 2p1, 2p1+1} of the
+            // group's x quad.  Narrow batches, where a selector serves one or
+            // two products, build it in registers: one PRMT looks up (p0, p1)
+            // of two groups at once from a byte table indexed by the low three
+            // bits of each 4-bit mask (distinct for the six masks with two bits
+            // set), a second expands them to byte pairs.  Wide batches reuse a
+            // selector across four columns and take it from the shared table.
+            uint32_t selw[4];
+            if constexpr (BP <= 4) {
+              constexpr uint32_t kPairLo = 0x10313010u, kPairHi = 0x10212032u;
+              const uint32_t s01 = __byte_perm(kPairLo, kPairHi, m & 0x77u);
+              const uint32_t s23 = __byte_perm(kPairLo, kPairHi, (m >> 8) & 0x77u);
+              const uint32_t a01 = __byte_perm(0x76543210u, 0u, s01);
+              const uint32_t a23 = __byte_perm(0x76543210u, 0u, s23);
+              selw[0] = a01;
+              selw[1] = a01 >> 16;
+              selw[2] = a23;
+              selw[3] = a23 >> 16;
+            } else {
+#pragma unroll
+              for (int g = 0; g < 4; ++g) selw[g] = sel_lut[(m >> (4 * g)) & 0xFu];
+            }
 #pragma unroll
             for (int g = 0; g < 4; ++g) {
-              const uint32_t sel = sel_lut[(m >> (4 * g)) & 0xFu];
+              const uint32_t sel = selw[g];
 #pragma unroll
               for (int b = 0; b < C::XB; ++b) {
                 const uint32_t xp = __byte_perm(xr[b][2 * g], xr[b][2 * g + 1], sel);
@@ -1163,15 +1189,20 @@ __global__ void __launch_bounds__(kThreads)
 // low rank: t[b][j] = sum_k V[k][j] x[b][k]  (3BASiL §1: the L = U V^T term)
 // ---------------------------------------------------------------------------
 // CTA c sums k in its slice; partials go to lr_part[c][b][j]; the last CTA to
-// arrive sums them in CTA order into t (deterministic).
+// arrive sums them into t in a fixed order (deterministic).  The kernel lets
+// a programmatic dependent launch at once; with pdl (it is one itself) it
+// waits for its predecessor before touching anything.
 template <int BP>
 __global__ void __launch_bounds__(kThreads)
     lowrank_t_kernel(const uint16_t *__restrict__ V, int64_t ldv, int rank,
                      int64_t k, const uint16_t *__restrict__ X, int64_t ldx,
                      int batch, float *__restrict__ t_out,
-                     float *__restrict__ lr_part, uint32_t *counter) {
+                     float *__restrict__ lr_part, uint32_t *counter, int pdl) {
   __shared__ float s_sum[BP * kMaxRank];
+  __shared__ float4 s_red[kThreads];
   __shared__ int s_last;
+  grid_dep_trigger();  // the U pass that follows may start its U loads
+  if (pdl) grid_dep_wait();
   const int tid = threadIdx.x;
   const int jg_count = rank / 8;          // 8 columns of V per thread
   const int rows_par = kThreads / jg_count;  // k rows in parallel
@@ -1217,10 +1248,47 @@ __global__ void __launch_bounds__(kThreads)
   __syncthreads();
   if (s_last) {
     __threadfence();
-    for (int i = tid; i < BP * rank; i += kThreads) {
-      float s = 0.f;
-      for (int cc = 0; cc < G2; ++cc) s += __ldcg(lr_part + (int64_t)cc * BP * rank + i);
-      t_out[i] = s;
+    // Every thread takes part: a column of four outputs is split over `per`
+    // threads, thread `sub` adding the partials of CTAs sub, sub + per, ...
+    // in ascending order with four loads in flight, and the `per` sums are
+    // then added in sub order.  (BP * rank is a multiple of 8.)
+    const int O4 = BP * rank / 4;
+    const int per = O4 >= kThreads ? 1 : kThreads / O4;
+    const float4 *part4 = reinterpret_cast<const float4 *>(lr_part);
+    float4 *t4 = reinterpret_cast<float4 *>(t_out);
+    auto add4 = [](float4 &a, const float4 &v) {
+      a.x += v.x;
+      a.y += v.y;
+      a.z += v.z;
+      a.w += v.w;
+    };
+    for (int item = tid; item < O4 * per; item += kThreads) {
+      const int col = item % O4, sub = item / O4;
+      float4 a = make_float4(0.f, 0.f, 0.f, 0.f);
+      int cc = sub;
+      for (; cc + 3 * per < G2; cc += 4 * per) {
+        const float4 v0 = __ldcg(part4 + (int64_t)cc * O4 + col);
+        const float4 v1 = __ldcg(part4 + (int64_t)(cc + per) * O4 + col);
+        const float4 v2 = __ldcg(part4 + (int64_t)(cc + 2 * per) * O4 + col);
+        const float4 v3 = __ldcg(part4 + (int64_t)(cc + 3 * per) * O4 + col);
+        add4(a, v0);
+        add4(a, v1);
+        add4(a, v2);
+        add4(a, v3);
+      }
+      for (; cc < G2; cc += per) add4(a, __ldcg(part4 + (int64_t)cc * O4 + col));
+      if (per == 1)
+        t4[col] = a;
+      else
+        s_red[sub * O4 + col] = a;
+    }
+    if (per > 1) {
+      __syncthreads();
+      for (int col = tid; col < O4; col += kThreads) {
+        float4 a = s_red[col];
+        for (int sub = 1; sub < per; ++sub) add4(a, s_red[sub * O4 + col]);
+        t4[col] = a;
+      }
     }
     if (tid == 0) *counter = 0;
   }
@@ -1231,14 +1299,19 @@ template <int BP>
 __global__ void __launch_bounds__(kThreads)
     lowrank_apply_kernel(int64_t n, const uint16_t *__restrict__ U, int64_t ldu,
                          int rank, const float *__restrict__ t, int batch,
-                         float *__restrict__ Y, int64_t ldy) {
+                         float *__restrict__ Y, int64_t ldy, int pdl) {
+  grid_dep_trigger();
   const int64_t i = (int64_t)blockIdx.x * kThreads + threadIdx.x;
+  // the first 16 bytes of this row of U are requested before t and Y, which
+  // the preceding grid writes, may be read
+  const uint4 u0 = i < n ? __ldg(reinterpret_cast<const uint4 *>(U + i * ldu)) : make_uint4(0, 0, 0, 0);
+  if (pdl) grid_dep_wait();
   if (i >= n) return;
   float acc[BP];
 #pragma unroll
   for (int b = 0; b < BP; ++b) acc[b] = 0.f;
   for (int j = 0; j < rank; j += 8) {
-    const uint4 uv = __ldg(reinterpret_cast<const uint4 *>(U + i * ldu + j));
+    const uint4 uv = j == 0 ? u0 : __ldg(reinterpret_cast<const uint4 *>(U + i * ldu + j));
     const float uf[8] = {bf16_lo(uv.x), bf16_hi(uv.x), bf16_lo(uv.y), bf16_hi(uv.y),
                          bf16_lo(uv.z), bf16_hi(uv.z), bf16_lo(uv.w), bf16_hi(uv.w)};
 #pragma unroll
@@ -1253,18 +1326,34 @@ __global__ void __launch_bounds__(kThreads)
 template <int BP>
 __global__ void __launch_bounds__(kThreads)
     lowrank_ut_kernel(int64_t n, const uint16_t *__restrict__ U, int64_t ldu, int rank,
-                      const float *__restrict__ t, int batch, float *__restrict__ ut) {
+                      const float *__restrict__ t, int batch, float *__restrict__ ut, int pdl) {
+  grid_dep_trigger();  // the product that follows may start streaming its weights
   const int64_t i = (int64_t)blockIdx.x * kThreads + threadIdx.x;
-  if (i >= n) return;
+  const bool live = i < n;
+  auto load_chunk = [&](int j0, uint4 (&uv)[8]) {
+#pragma unroll
+    for (int q = 0; q < 8; ++q)
+      uv[q] = live && j0 + 8 * q < rank
+                  ? __ldg(reinterpret_cast<const uint4 *>(U + i * ldu + j0 + 8 * q))
+                  : make_uint4(0, 0, 0, 0);
+  };
+  // the first 128 bytes of this row of U are requested before t, which the
+  // preceding grid writes, may be read
+  uint4 first[8];
+  load_chunk(0, first);
+  if (pdl) grid_dep_wait();
+  if (!live) return;
   float acc[BP];
 #pragma unroll
   for (int b = 0; b < BP; ++b) acc[b] = 0.f;
   for (int j0 = 0; j0 < rank; j0 += 64) {
     uint4 uv[8];
+    if (j0 == 0) {
 #pragma unroll
-    for (int q = 0; q < 8; ++q)
-      uv[q] = j0 + 8 * q < rank ? __ldg(reinterpret_cast<const uint4 *>(U + i * ldu + j0 + 8 * q))
-                                : make_uint4(0, 0, 0, 0);
+      for (int q = 0; q < 8; ++q) uv[q] = first[q];
+    } else {
+      load_chunk(j0, uv);
+    }
 #pragma unroll
     for (int q = 0; q < 8; ++q) {
       if (j0 + 8 * q >= rank) break;
@@ -1551,9 +1640,28 @@ int check_lowrank(const hyb_lowrank *lr, int64_t n, int64_t k) {
   return HYB_OK;
 }
 
+// A launch, as a programmatic dependent of the preceding kernel on the stream
+// when pdl is set (the kernel then orders its own accesses with
+// griddepcontrol.wait).
+cudaError_t launch_kernel(const void *fn, dim3 grid, dim3 block, void **args, size_t smem,
+                          cudaStream_t s, bool pdl) {
+  if (!pdl) return cudaLaunchKernel(fn, grid, block, args, smem, s);
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelExC(&cfg, fn, args);
+}
+
 int launch_lowrank_t(const Plan &P, const hyb_lowrank *lr, int64_t k,
                      const uint16_t *X, int64_t ldx, int batch, uint8_t *ws,
-                     cudaStream_t s) {
+                     cudaStream_t s, bool pdl) {
   void *fn = pick_lowrank_t(P.bp);
   const uint16_t *V = lr->V;
   int64_t ldv = lr->ldv;
@@ -1561,9 +1669,9 @@ int launch_lowrank_t(const Plan &P, const hyb_lowrank *lr, int64_t k,
   float *t_out = reinterpret_cast<float *>(ws + P.off_lr_t);
   float *part = reinterpret_cast<float *>(ws + P.off_lr_part);
   uint32_t *counter = reinterpret_cast<uint32_t *>(ws + P.off_lr_counter);
-  void *args[] = {&V, &ldv, &rank, &k, &X, &ldx, &batch, &t_out, &part, &counter};
-  if (cudaLaunchKernel(fn, dim3(P.lr_ctas), dim3(kThreads), args, 0, s) !=
-      cudaSuccess)
+  int pdl_i = pdl ? 1 : 0;
+  void *args[] = {&V, &ldv, &rank, &k, &X, &ldx, &batch, &t_out, &part, &counter, &pdl_i};
+  if (launch_kernel(fn, dim3(P.lr_ctas), dim3(kThreads), args, 0, s, pdl) != cudaSuccess)
     return HYB_ERR_CUDA;
   return HYB_OK;
 }
@@ -1619,25 +1727,6 @@ void fill_launch_plan(const int64_t *plan, int32_t plan_ctas, const Plan &P, con
   lp->ctas = P.G;
 }
 
-// A launch, as a programmatic dependent of the preceding kernel on the stream
-// when pdl is set (the kernel then orders its own accesses with
-// griddepcontrol.wait).
-cudaError_t launch_kernel(const void *fn, dim3 grid, dim3 block, void **args, size_t smem,
-                          cudaStream_t s, bool pdl) {
-  if (!pdl) return cudaLaunchKernel(fn, grid, block, args, smem, s);
-  cudaLaunchConfig_t cfg{};
-  cfg.gridDim = grid;
-  cfg.blockDim = block;
-  cfg.dynamicSmemBytes = smem;
-  cfg.stream = s;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  return cudaLaunchKernelExC(&cfg, fn, args);
-}
-
 int run_product(Params prm, int b1, int b2, int batch, const hyb_lowrank *lr,
                 bool strided, void *ws, size_t ws_bytes, cudaStream_t s,
                 const int64_t *plan = nullptr, int32_t plan_ctas = 0, uint32_t flags = 0) {
@@ -1657,23 +1746,29 @@ int run_product(Params prm, int b1, int b2, int batch, const hyb_lowrank *lr,
   prm.ldu = rank ? lr->ldu : 0;
   prm.lr_t = reinterpret_cast<const float *>(w + P.off_lr_t);
   prm.lr_ut = nullptr;
+  const bool overlap = (flags & HYB_LAUNCH_OVERLAP_PREV) != 0;
   if (rank) {
-    rc = launch_lowrank_t(P, lr, prm.k, prm.X, prm.ldx, batch, w, s);
+    // V^T x, then U t, then the product: the two later kernels always launch
+    // as programmatic dependents of the one before (their early loads are of
+    // U and the weights, which nothing in this call writes; the first kernel
+    // of the call starts early only when the caller allows it)
+    rc = launch_lowrank_t(P, lr, prm.k, prm.X, prm.ldx, batch, w, s, overlap);
     if (rc != HYB_OK) return rc;
     int64_t nn = prm.n, ldu = lr->ldu;
     const uint16_t *U = lr->U;
     int rk = rank, bt = batch;
     const float *tp = prm.lr_t;
     float *ut = reinterpret_cast<float *>(w + P.off_lr_ut);
-    void *uargs[] = {&nn, &U, &ldu, &rk, &tp, &bt, &ut};
+    int one = 1;
+    void *uargs[] = {&nn, &U, &ldu, &rk, &tp, &bt, &ut, &one};
     const int64_t grid = (prm.n + kThreads - 1) / kThreads;
-    if (cudaLaunchKernel(pick_lowrank_ut(P.bp), dim3((unsigned)grid), dim3(kThreads), uargs, 0, s) !=
-        cudaSuccess)
+    if (launch_kernel(pick_lowrank_ut(P.bp), dim3((unsigned)grid), dim3(kThreads), uargs, 0, s,
+                      true) != cudaSuccess)
       return HYB_ERR_CUDA;
     prm.lr_ut = ut;
   }
   prm.status = reinterpret_cast<uint32_t *>(w);
-  const bool pdl = (flags & HYB_LAUNCH_OVERLAP_PREV) != 0 && (P.tma || P.stream);
+  const bool pdl = (overlap || rank > 0) && (P.tma || P.stream);
   prm.pdl = pdl ? 1 : 0;
   void *args[] = {&prm};
   if (P.tma) {
@@ -1901,7 +1996,8 @@ int hyb_lowrank_add(int64_t n, int64_t k, int batch, const hyb_lowrank *lr,
     float *t_out = reinterpret_cast<float *>(w + off_t);
     float *part = reinterpret_cast<float *>(w + off_part);
     uint32_t *counter = reinterpret_cast<uint32_t *>(w + off_counter);
-    void *args[] = {&V, &ldv, &rank, &kk, &Xp, &ldxx, &bt, &t_out, &part, &counter};
+    int zero = 0;
+    void *args[] = {&V, &ldv, &rank, &kk, &Xp, &ldxx, &bt, &t_out, &part, &counter, &zero};
     if (cudaLaunchKernel(pick_lowrank_t(bp), dim3(ctas), dim3(kThreads), args, 0, s) !=
         cudaSuccess)
       return HYB_ERR_CUDA;
@@ -1912,10 +2008,12 @@ int hyb_lowrank_add(int64_t n, int64_t k, int batch, const hyb_lowrank *lr,
     int rank = lr->rank, bt = batch;
     const float *t = reinterpret_cast<const float *>(w + off_t);
     float *Yp = Y;
-    void *args[] = {&nn, &U, &ldu, &rank, &t, &bt, &Yp, &ldyy};
+    // a programmatic dependent of the V^T x pass, launched plainly just above
+    int one = 1;
+    void *args[] = {&nn, &U, &ldu, &rank, &t, &bt, &Yp, &ldyy, &one};
     const int64_t grid = (n + kThreads - 1) / kThreads;
-    if (cudaLaunchKernel(pick_lowrank_apply(bp), dim3((unsigned)grid), dim3(kThreads),
-                         args, 0, s) != cudaSuccess)
+    if (launch_kernel(pick_lowrank_apply(bp), dim3((unsigned)grid), dim3(kThreads), args, 0, s,
+                      true) != cudaSuccess)
       return HYB_ERR_CUDA;
   }
   return HYB_OK;
