@@ -78,6 +78,9 @@ struct Params {
   // stream.  The weights (packed matrix or row-major W) may then be read
   // before that kernel has finished; X, Y, the workspace and the low-rank
   // intermediates are touched only after griddepcontrol.wait.
+  // 2: the same, behind the low-rank kernels of the same call, which start
+  // only once all work before the call has finished: X may be read at once,
+  // and only the epilogue (Y, workspace, U t) waits.
   int pdl;
 };
 
@@ -714,7 +717,7 @@ __global__ void __launch_bounds__(TmaCfg<BP, B1, B2>::kThreads, 1)
     // weight bytes requested at once and its X only after the preceding grid
     // has finished (it may have written X); the lane that armed a stage keeps
     // the stage's X request until then.  Warp-uniform: pend, issued.
-    bool pend = p.pdl != 0;
+    bool pend = p.pdl == 1;
     int issued = 0;
     int dx_stage = -1, dx_nt = 0;
     int64_t dx_col = 0;
@@ -1189,9 +1192,9 @@ __global__ void __launch_bounds__(kThreads)
 // low rank: t[b][j] = sum_k V[k][j] x[b][k]  (3BASiL §1: the L = U V^T term)
 // ---------------------------------------------------------------------------
 // CTA c sums k in its slice; partials go to lr_part[c][b][j]; the last CTA to
-// arrive sums them into t in a fixed order (deterministic).  The kernel lets
-// a programmatic dependent launch at once; with pdl (it is one itself) it
-// waits for its predecessor before touching anything.
+// arrive sums them into t in a fixed order (deterministic).  With pdl (it is a
+// programmatic dependent itself) it waits for its predecessor before touching
+// anything, and only then lets its own dependents launch.
 template <int BP>
 __global__ void __launch_bounds__(kThreads)
     lowrank_t_kernel(const uint16_t *__restrict__ V, int64_t ldv, int rank,
@@ -1201,8 +1204,10 @@ __global__ void __launch_bounds__(kThreads)
   __shared__ float s_sum[BP * kMaxRank];
   __shared__ float4 s_red[kThreads];
   __shared__ int s_last;
-  grid_dep_trigger();  // the U pass that follows may start its U loads
   if (pdl) grid_dep_wait();
+  // Dependents (the U pass, then the product) may launch from here on: all
+  // work queued before this kernel has finished, so they may read X at once.
+  grid_dep_trigger();
   const int tid = threadIdx.x;
   const int jg_count = rank / 8;          // 8 columns of V per thread
   const int rows_par = kThreads / jg_count;  // k rows in parallel
@@ -1749,9 +1754,11 @@ int run_product(Params prm, int b1, int b2, int batch, const hyb_lowrank *lr,
   const bool overlap = (flags & HYB_LAUNCH_OVERLAP_PREV) != 0;
   if (rank) {
     // V^T x, then U t, then the product: the two later kernels always launch
-    // as programmatic dependents of the one before (their early loads are of
-    // U and the weights, which nothing in this call writes; the first kernel
-    // of the call starts early only when the caller allows it)
+    // as programmatic dependents of the one before.  V^T x lets them launch
+    // only after everything queued before the call has finished (with the
+    // caller's leave it starts early itself, and waits), so their early
+    // loads -- of U, the weights and X -- see finished data; what they wait
+    // for is t, U t and the workspace.
     rc = launch_lowrank_t(P, lr, prm.k, prm.X, prm.ldx, batch, w, s, overlap);
     if (rc != HYB_OK) return rc;
     int64_t nn = prm.n, ldu = lr->ldu;
@@ -1769,7 +1776,7 @@ int run_product(Params prm, int b1, int b2, int batch, const hyb_lowrank *lr,
   }
   prm.status = reinterpret_cast<uint32_t *>(w);
   const bool pdl = (overlap || rank > 0) && (P.tma || P.stream);
-  prm.pdl = pdl ? 1 : 0;
+  prm.pdl = !pdl ? 0 : (rank > 0 ? 2 : 1);
   void *args[] = {&prm};
   if (P.tma) {
     LaunchPlan lp;
