@@ -204,10 +204,14 @@ HYB_API int hyb_spmm_skinny(const hyb_matrix *A, int batch, const uint16_t *X,
  * intermediates, only after the preceding kernel has completed and its
  * writes are visible (griddepcontrol.wait), so results are identical with
  * and without the flag.  The caller guarantees that the weights -- A's tile
- * map, values, masks and offsets (or W for hyb_gemv_dense_ex) -- are not
- * written by the work queued before the call on the stream that has not
- * finished by then.  Tilings served by the one-warp-per-row kernel ignore
- * the flag. */
+ * map, values, masks and offsets, the low-rank factors U and V (or W for
+ * hyb_gemv_dense_ex) -- are not written by the work queued before the call on
+ * the stream that has not finished by then.  Tilings served by the
+ * one-warp-per-row kernel ignore the flag.
+ * With a low-rank term the call runs three kernels (V^T x, U t, the product);
+ * the flag applies to the first, and the later two always start as
+ * programmatic dependents of the one before them, after all work queued
+ * before the call has finished. */
 
 /* hyb_spmm_skinny with launch options `flags` (0 = hyb_spmm_skinny). */
 HYB_API int hyb_spmm_skinny_ex(const hyb_matrix *A, int batch, const uint16_t *X,
