@@ -79,7 +79,7 @@ typedef struct CUstream_st *hyb_stream_t; /* same type as cudaStream_t */
 typedef enum {
   HYB_OK = 0,
   HYB_ERR_INVALID_ARG = -1,  /* bad shape, null pointer, bad enum */
-  HYB_ERR_UNSUPPORTED = -2,  /* valid request this build does not handle */
+  HYB_ERR_UNSUPPORTED = -2,  /* valid request the library does not handle */
   HYB_ERR_ALIGNMENT = -3,    /* pointer or leading dimension misaligned */
   HYB_ERR_WORKSPACE = -4,    /* workspace null or smaller than required */
   HYB_ERR_CUDA = -5,         /* a CUDA runtime call failed */
