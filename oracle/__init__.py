@@ -51,6 +51,15 @@ def load(mutant: int = 0, path: str = None):
     lib.oracle_rows_f64.restype = _I
     lib.oracle_bf16_to_f64.argtypes = [ctypes.c_uint16]
     lib.oracle_bf16_to_f64.restype = ctypes.c_double
+    lib.oracle_offsets_nm.argtypes = [_I64, _I64, _I, _I, _I, _I, _P, _P, _P]
+    lib.oracle_offsets_nm.restype = _I
+    lib.oracle_pack_nm.argtypes = [_I64, _I64, _I, _I, _I, _I, _P, _I64, _P, _P, _P, _P, _P]
+    lib.oracle_pack_nm.restype = _I64
+    lib.oracle_unpack_nm.argtypes = [_I64, _I64, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P]
+    lib.oracle_unpack_nm.restype = _I
+    lib.oracle_spmv_nm_f64.argtypes = [_I64, _I64, _I, _I, _I, _I, _P, _P, _P, _P, _P, _I,
+                                       _P, _I64, _P, _I64, _P, _I64, _I, _P, _I64, _P]
+    lib.oracle_spmv_nm_f64.restype = _I
     _libs[key] = lib
     return lib
 
@@ -185,3 +194,65 @@ class Oracle:
 
     def bf16_to_f64(self, h):
         return self.lib.oracle_bf16_to_f64(int(h))
+
+    # ---- general N:M tiles (nk kept of every m columns) ----
+
+    def offsets_nm(self, n, k, b1, b2, nk, m, tile_map):
+        tile_map = _c(tile_map, np.uint8).reshape(-1)
+        vo = np.zeros(tile_map.size + 1, np.int64)
+        mo = np.zeros(tile_map.size + 1, np.int64)
+        if self.lib.oracle_offsets_nm(n, k, b1, b2, nk, m, _ptr(tile_map), _ptr(vo),
+                                      _ptr(mo)) != 0:
+            raise OracleError("oracle_offsets_nm: bad argument")
+        return vo, mo
+
+    def pack_nm(self, W, b1, b2, tile_map, nk, m):
+        """Returns dict(vals, meta, val_off, meta_off, nan_groups)."""
+        W = _c(W, np.uint16)
+        n, k = W.shape
+        tile_map = _c(tile_map, np.uint8).reshape(-1)
+        vo, mo = self.offsets_nm(n, k, b1, b2, nk, m, tile_map)
+        vals = np.zeros(int(vo[-1]), np.uint16)
+        meta = np.zeros(max(int(mo[-1]), 1), np.uint8)
+        rc = self.lib.oracle_pack_nm(n, k, b1, b2, nk, m, _ptr(W), k, _ptr(tile_map),
+                                     _ptr(vals), _ptr(meta), _ptr(vo), _ptr(mo))
+        if rc < 0:
+            raise OracleError("oracle_pack_nm: bad argument")
+        return dict(vals=vals, meta=meta[:int(mo[-1])], val_off=vo, meta_off=mo,
+                    nan_groups=int(rc))
+
+    def unpack_nm(self, n, k, b1, b2, nk, m, tile_map, packed):
+        tile_map = _c(tile_map, np.uint8).reshape(-1)
+        W_hat = np.zeros((n, k), np.uint16)
+        meta = packed["meta"] if packed["meta"].size else np.zeros(1, np.uint8)
+        rc = self.lib.oracle_unpack_nm(n, k, b1, b2, nk, m, _ptr(tile_map),
+                                       _ptr(_c(packed["vals"], np.uint16)),
+                                       _ptr(_c(meta, np.uint8)),
+                                       _ptr(_c(packed["val_off"], np.int64)),
+                                       _ptr(_c(packed["meta_off"], np.int64)),
+                                       _ptr(W_hat))
+        if rc != 0:
+            raise OracleError("oracle_unpack_nm: bad argument")
+        return W_hat
+
+    def spmv_nm(self, n, k, b1, b2, nk, m, tile_map, packed, X, U=None, V=None):
+        tile_map = _c(tile_map, np.uint8).reshape(-1)
+        X = np.atleast_2d(_c(X, np.uint16))
+        batch = X.shape[0]
+        rank = 0 if U is None else U.shape[1]
+        U = _c(U, np.uint16)
+        V = _c(V, np.uint16)
+        meta = packed["meta"] if packed["meta"].size else np.zeros(1, np.uint8)
+        Y = np.zeros((batch, n), np.float64)
+        env = np.zeros((batch, n), np.float64)
+        rc = self.lib.oracle_spmv_nm_f64(n, k, b1, b2, nk, m, _ptr(tile_map),
+                                         _ptr(_c(packed["vals"], np.uint16)),
+                                         _ptr(_c(meta, np.uint8)),
+                                         _ptr(_c(packed["val_off"], np.int64)),
+                                         _ptr(_c(packed["meta_off"], np.int64)),
+                                         batch, _ptr(X), X.shape[1], _ptr(U),
+                                         rank if rank else 1, _ptr(V), rank if rank else 1,
+                                         rank, _ptr(Y), n, _ptr(env))
+        if rc != 0:
+            raise OracleError("oracle_spmv_nm_f64: bad argument")
+        return Y, env

@@ -403,3 +403,180 @@ int oracle_rows_f64(int64_t n, int64_t k, int b1, int b2, const uint16_t *W,
   free(tabs);
   return ORC_OK;
 }
+
+/* ------------------------------------------------------------------ */
+/* general N:M tiles (N kept of every M consecutive columns)           */
+/* ------------------------------------------------------------------ */
+/*
+ * The pages name other N:M patterns (4:8) as the natural extension of the
+ * tile-level scheme (PATCH, "Future direction"), and SparseDecoding's kernel
+ * is an N:M sparse matrix-vector product with a bitmask and a fixed stride.
+ * Reading used here, which for N = 2, M = 4 is exactly the 2:4 layout above:
+ *  - a sparse tile row keeps N of every M consecutive columns, chosen by the
+ *    same magnitude key, ties to the lower column;
+ *  - its kept values are stored in ascending column order, N per group (group
+ *    g of row i at i*(b2*N/M) + N*g, fixed stride N);
+ *  - its mask is a bit stream of b2 bits, bit c (byte c/8, bit c%8 of the
+ *    row's b2/8 bytes) set iff column c is kept, so a tile costs
+ *    b1*b2*N/M values and b1*b2/8 mask bytes whatever N and M are.
+ * Supported: M in {4, 8, 16}, 0 < N < M, b2 a multiple of M and of 8.
+ */
+
+static int check_nm(int b2, int nk, int m) {
+  if (!(m == 4 || m == 8 || m == 16)) return ORC_BAD_ARG;
+  if (nk <= 0 || nk >= m) return ORC_BAD_ARG;
+  if (b2 % m != 0) return ORC_BAD_ARG;
+  return ORC_OK;
+}
+
+/* Member j of w[0..m-1] is kept iff fewer than nk members rank above it; a
+ * member ranks above j when its key is larger, or equal with a lower column.
+ * Returns the m-bit mask (bit j = column j kept). */
+static unsigned select_n_of_m(const uint16_t *w, int nk, int m) {
+  unsigned mask = 0;
+  for (int j = 0; j < m; ++j) {
+    int above = 0;
+    for (int i = 0; i < m; ++i) {
+      if (i == j) continue;
+#if ORACLE_MUTANT == 7
+      /* planted mistake: among equal keys the higher column ranks above */
+      if (key_of(w[i]) > key_of(w[j]) || (key_of(w[i]) == key_of(w[j]) && i > j))
+        above++;
+#else
+      if (key_of(w[i]) > key_of(w[j]) || (key_of(w[i]) == key_of(w[j]) && i < j))
+        above++;
+#endif
+    }
+    if (above < nk) mask |= 1u << j;
+  }
+  return mask;
+}
+
+/* Byte and bit, inside a sparse tile's mask block, of column c of row i. */
+static int64_t nm_mask_byte(int64_t i, int64_t c, int b2) {
+  return i * (b2 / 8) + c / 8;
+}
+static int nm_mask_bit(int64_t c) {
+#if ORACLE_MUTANT == 8
+  return 7 - (int)(c % 8); /* planted mistake: bits numbered from the top */
+#else
+  return (int)(c % 8);
+#endif
+}
+
+int oracle_offsets_nm(int64_t n, int64_t k, int b1, int b2, int nk, int m,
+                      const uint8_t *tile_map, int64_t *val_off,
+                      int64_t *meta_off) {
+  if (check_shape(n, k, b1, b2, tile_map) != ORC_OK) return ORC_BAD_ARG;
+  if (check_nm(b2, nk, m) != ORC_OK) return ORC_BAD_ARG;
+  int64_t T = (n / b1) * (k / b2);
+  int64_t tile_elems = (int64_t)b1 * b2;
+  val_off[0] = 0;
+  meta_off[0] = 0;
+  for (int64_t t = 0; t < T; ++t) {
+    int sparse = tile_map[t] == 1;
+    val_off[t + 1] = val_off[t] + (sparse ? tile_elems / m * nk : tile_elems);
+    meta_off[t + 1] = meta_off[t] + (sparse ? tile_elems / 8 : 0);
+  }
+  return ORC_OK;
+}
+
+int64_t oracle_pack_nm(int64_t n, int64_t k, int b1, int b2, int nk, int m,
+                       const uint16_t *W, int64_t ldw, const uint8_t *tile_map,
+                       uint16_t *vals, uint8_t *meta, int64_t *val_off,
+                       int64_t *meta_off) {
+  if (oracle_offsets_nm(n, k, b1, b2, nk, m, tile_map, val_off, meta_off) != ORC_OK)
+    return ORC_BAD_ARG;
+  if (W == NULL || ldw < k) return ORC_BAD_ARG;
+  int64_t tiles_per_row = k / b2;
+  int64_t T = (n / b1) * tiles_per_row;
+  int64_t row_vals = (int64_t)b2 / m * nk;
+  int64_t nan_groups = 0;
+  for (int64_t t = 0; t < T; ++t) {
+    int64_t tr = t / tiles_per_row, tc = t % tiles_per_row;
+    const uint16_t *Wt = W + tr * b1 * ldw + tc * b2;
+    uint16_t *vt = vals + val_off[t];
+    if (tile_map[t] == 0) {
+      for (int64_t i = 0; i < b1; ++i)
+        for (int64_t j = 0; j < b2; ++j) vt[i * b2 + j] = Wt[i * ldw + j];
+      continue;
+    }
+    uint8_t *mt = meta + meta_off[t];
+    for (int64_t i = 0; i < (int64_t)b1 * (b2 / 8); ++i) mt[i] = 0;
+    for (int64_t i = 0; i < b1; ++i) {
+      for (int64_t g = 0; g < b2 / m; ++g) {
+        const uint16_t *w = Wt + i * ldw + (int64_t)m * g;
+        unsigned mask = select_n_of_m(w, nk, m);
+        int has_nan = 0;
+        int s = 0;
+        for (int j = 0; j < m; ++j) {
+          if (is_nan_bf16(w[j])) has_nan = 1;
+          if (!((mask >> j) & 1)) continue;
+          int64_t c = (int64_t)m * g + j;
+          vt[i * row_vals + (int64_t)nk * g + s] = w[j];
+          s++;
+          mt[nm_mask_byte(i, c, b2)] |= (uint8_t)(1u << nm_mask_bit(c));
+        }
+        nan_groups += has_nan;
+      }
+    }
+  }
+  return nan_groups;
+}
+
+int oracle_unpack_nm(int64_t n, int64_t k, int b1, int b2, int nk, int m,
+                     const uint8_t *tile_map, const uint16_t *vals,
+                     const uint8_t *meta, const int64_t *val_off,
+                     const int64_t *meta_off, uint16_t *W_hat) {
+  if (check_shape(n, k, b1, b2, tile_map) != ORC_OK) return ORC_BAD_ARG;
+  if (check_nm(b2, nk, m) != ORC_OK) return ORC_BAD_ARG;
+  int64_t tiles_per_row = k / b2;
+  int64_t T = (n / b1) * tiles_per_row;
+  int64_t row_vals = (int64_t)b2 / m * nk;
+  for (int64_t t = 0; t < T; ++t) {
+    int64_t tr = t / tiles_per_row, tc = t % tiles_per_row;
+    uint16_t *Wt = W_hat + tr * b1 * k + tc * b2;
+    const uint16_t *vt = vals + val_off[t];
+    if (tile_map[t] == 0) {
+      for (int64_t i = 0; i < b1; ++i)
+        for (int64_t j = 0; j < b2; ++j) Wt[i * k + j] = vt[i * b2 + j];
+      continue;
+    }
+    const uint8_t *mt = meta + meta_off[t];
+    for (int64_t i = 0; i < b1; ++i) {
+      for (int64_t g = 0; g < b2 / m; ++g) {
+        int s = 0;
+        for (int j = 0; j < m; ++j) {
+          int64_t c = (int64_t)m * g + j;
+          uint16_t v = 0;
+          if ((mt[nm_mask_byte(i, c, b2)] >> nm_mask_bit(c)) & 1) {
+            /* a malformed mask with more than nk bits set reads nothing past
+             * this group's nk slots */
+            v = s < nk ? vt[i * row_vals + (int64_t)nk * g + s] : 0;
+            s++;
+          }
+          Wt[i * k + c] = v;
+        }
+      }
+    }
+  }
+  return ORC_OK;
+}
+
+int oracle_spmv_nm_f64(int64_t n, int64_t k, int b1, int b2, int nk, int m,
+                       const uint8_t *tile_map, const uint16_t *vals,
+                       const uint8_t *meta, const int64_t *val_off,
+                       const int64_t *meta_off, int batch, const uint16_t *X,
+                       int64_t ldx, const uint16_t *U, int64_t ldu,
+                       const uint16_t *V, int64_t ldv, int rank, double *Y,
+                       int64_t ldy, double *env) {
+  uint16_t *W_hat = (uint16_t *)malloc(sizeof(uint16_t) * (size_t)(n * k));
+  if (!W_hat) return ORC_BAD_ARG;
+  int rc = oracle_unpack_nm(n, k, b1, b2, nk, m, tile_map, vals, meta, val_off,
+                            meta_off, W_hat);
+  if (rc == ORC_OK)
+    rc = oracle_matvec_f64(n, k, W_hat, k, batch, X, ldx, U, ldu, V, ldv,
+                           rank, Y, ldy, env);
+  free(W_hat);
+  return rc;
+}

@@ -114,6 +114,31 @@ int oracle_rows_f64(int64_t n, int64_t k, int b1, int b2, const uint16_t *W,
 /* fp64 value of a bf16 bit pattern, exposed for the tests. */
 double oracle_bf16_to_f64(uint16_t h);
 
+/* General N:M tiles (nk kept of every m consecutive columns; m in {4, 8, 16},
+ * 0 < nk < m, b2 a multiple of m and 8).  A sparse tile row stores its kept
+ * values in ascending column order, nk per group, and a b2-bit mask stream
+ * (bit c of the row's b2/8 bytes set iff column c is kept); nk = 2, m = 4 is
+ * the 2:4 layout above, bit for bit.  Same conventions and return codes as
+ * the 2:4 routines. */
+int oracle_offsets_nm(int64_t n, int64_t k, int b1, int b2, int nk, int m,
+                      const uint8_t *tile_map, int64_t *val_off,
+                      int64_t *meta_off);
+int64_t oracle_pack_nm(int64_t n, int64_t k, int b1, int b2, int nk, int m,
+                       const uint16_t *W, int64_t ldw, const uint8_t *tile_map,
+                       uint16_t *vals, uint8_t *meta, int64_t *val_off,
+                       int64_t *meta_off);
+int oracle_unpack_nm(int64_t n, int64_t k, int b1, int b2, int nk, int m,
+                     const uint8_t *tile_map, const uint16_t *vals,
+                     const uint8_t *meta, const int64_t *val_off,
+                     const int64_t *meta_off, uint16_t *W_hat);
+int oracle_spmv_nm_f64(int64_t n, int64_t k, int b1, int b2, int nk, int m,
+                       const uint8_t *tile_map, const uint16_t *vals,
+                       const uint8_t *meta, const int64_t *val_off,
+                       const int64_t *meta_off, int batch, const uint16_t *X,
+                       int64_t ldx, const uint16_t *U, int64_t ldu,
+                       const uint16_t *V, int64_t ldv, int rank, double *Y,
+                       int64_t ldy, double *env);
+
 #ifdef __cplusplus
 }
 #endif

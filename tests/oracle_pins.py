@@ -310,5 +310,146 @@ def pin_special_values(o):
     assert int(pn["meta"][0]) & 0xF == 0b0011  # NaN key outranks -inf
 
 
+# ---------------------------------------------------------------------------
+# general N:M tiles (PATCH, "Future direction": other N:M patterns such as
+# 4:8; SparseDecoding's N:M kernel with a bitmask and a fixed stride)
+
+NM_CASES = [(1, 4), (2, 4), (3, 4), (2, 8), (4, 8), (6, 8)]
+
+
+def brute_force_mask_nm(W_bits, tile_map, b1, b2, nk, m):
+    """Masked dense matrix by enumerating every choice of nk columns out of m
+    in each group of a sparse tile and keeping the one with the largest sum of
+    |w| keys; among equal sums the lexicographically first choice wins."""
+    n, k = W_bits.shape
+    out = np.zeros_like(W_bits)
+    tpr = k // b2
+    key = (W_bits & 0x7FFF).astype(np.int64)
+    choices = list(itertools.combinations(range(m), nk))
+    for i in range(n):
+        for c0 in range(0, k, m):
+            t = (i // b1) * tpr + c0 // b2
+            if tile_map[t] == 0:
+                out[i, c0:c0 + m] = W_bits[i, c0:c0 + m]
+                continue
+            best, best_s = None, -1
+            for ch in choices:
+                s = sum(int(key[i, c0 + j]) for j in ch)
+                if s > best_s:
+                    best, best_s = ch, s
+            for j in best:
+                out[i, c0 + j] = W_bits[i, c0 + j]
+    return out
+
+
+def mask_bits(meta_row):
+    """The bit stream of one tile row's mask bytes, bit c = column c."""
+    return [(int(meta_row[c // 8]) >> (c % 8)) & 1 for c in range(8 * len(meta_row))]
+
+
+def pin_nm_golden(o):
+    """Hand-worked 2x32 example with a 4:8 tile and a dense tile
+    (tests/golden/pack_nm_2x32_4of8.txt)."""
+    g = read_golden("pack_nm_2x32_4of8.txt")
+    n, k, b1, b2, nk, m = (int(g[s][0]) for s in ("n", "k", "b1", "b2", "nk", "m"))
+    tmap = np.array([int(v) for v in g["tile_map"]], np.uint8)
+    W = np.stack([f2bits([float(v) for v in g[f"W{i}"]]) for i in range(n)])
+    p = o.pack_nm(W, b1, b2, tmap, nk, m)
+    assert p["val_off"].tolist() == [int(v) for v in g["val_off"]], p["val_off"]
+    assert p["meta_off"].tolist() == [int(v) for v in g["meta_off"]], p["meta_off"]
+    assert p["vals"].tolist() == f2bits([float(v) for v in g["vals"]]).tolist(), p["vals"]
+    assert p["meta"].tolist() == [int(v, 16) for v in g["meta"]], p["meta"]
+    X = f2bits([[float(v) for v in g["x"]]])
+    Y, _ = o.spmv_nm(n, k, b1, b2, nk, m, tmap, p, X)
+    assert Y[0].tolist() == [float(v) for v in g["y"]], Y
+    Yd, _ = o.spmv_nm(n, k, b1, b2, nk, m, np.zeros_like(tmap),
+                      o.pack_nm(W, b1, b2, np.zeros_like(tmap), nk, m), X)
+    assert Yd[0].tolist() == [float(v) for v in g["y_dense"]], Yd
+
+
+def pin_nm_is_2of4(o):
+    """With N = 2, M = 4 the N:M routines give the 2:4 format bit for bit
+    (values, masks, offsets), on tie-heavy integers and every map of 4 tiles."""
+    rng = np.random.default_rng(99)
+    n, k, b1, b2 = 8, 32, 4, 16
+    for trial in range(3):
+        W = _tie_heavy_ints(rng, (n, k))
+        for bitsmap in itertools.product([0, 1], repeat=4):
+            tmap = np.array(bitsmap, np.uint8)
+            a = o.pack(W, b1, b2, tmap)
+            b = o.pack_nm(W, b1, b2, tmap, 2, 4)
+            for key in ("vals", "meta", "val_off", "meta_off"):
+                assert np.array_equal(a[key], b[key]), (key, bitsmap)
+
+
+def pin_nm_bruteforce(o):
+    """Every (N, M) of NM_CASES on tie-heavy integer inputs and every map of up
+    to 4 tiles: selection against enumeration of the C(M, N) choices, products
+    against exact integer arithmetic."""
+    rng = np.random.default_rng(4321)
+    for (nk, m) in NM_CASES:
+        for (n, k, b1, b2) in [(4, 16, 2, 8), (4, 32, 4, 16)]:
+            if b2 % m:
+                continue
+            T = (n // b1) * (k // b2)
+            W = _tie_heavy_ints(rng, (n, k))
+            X = _tie_heavy_ints(rng, (2, k))
+            for bitsmap in itertools.product([0, 1], repeat=T):
+                tmap = np.array(bitsmap, np.uint8)
+                p = o.pack_nm(W, b1, b2, tmap, nk, m)
+                W_hat = o.unpack_nm(n, k, b1, b2, nk, m, tmap, p)
+                expect = brute_force_mask_nm(W, tmap, b1, b2, nk, m)
+                assert np.array_equal(W_hat, expect), (nk, m, n, k, bitsmap)
+                Y, E = o.spmv_nm(n, k, b1, b2, nk, m, tmap, p, X)
+                Yi, Ei = _ints_exact(expect, X)
+                assert np.array_equal(Y, Yi.astype(np.float64)), (nk, m, bitsmap)
+                assert np.array_equal(E, Ei.astype(np.float64))
+
+
+def pin_nm_invariants(o):
+    """Format invariants on random normal weights: nk mask bits per group of m,
+    offsets and total bytes in closed form, kept values in ascending column
+    order (read back through the mask), all-sparse selection equal to a stable
+    sort of the magnitudes."""
+    rng = np.random.default_rng(11)
+    for (nk, m) in [(4, 8), (2, 8), (8, 16)]:
+        n, k, b1, b2 = 32, 64, 8, 32
+        T = (n // b1) * (k // b2)
+        W = round_bits(rng.normal(0, 1, (n, k)))
+        tmap = (rng.random(T) < 0.5).astype(np.uint8)
+        p = o.pack_nm(W, b1, b2, tmap, nk, m)
+        s = int(tmap.sum())
+        assert p["val_off"][-1] == (T - s) * b1 * b2 + s * b1 * b2 * nk // m
+        assert p["meta_off"][-1] == s * b1 * b2 // 8
+        for t in range(T):
+            size_v = p["val_off"][t + 1] - p["val_off"][t]
+            size_m = p["meta_off"][t + 1] - p["meta_off"][t]
+            assert size_v == (b1 * b2 * nk // m if tmap[t] else b1 * b2)
+            assert size_m == (b1 * b2 // 8 if tmap[t] else 0)
+            if not tmap[t]:
+                continue
+            tr, tc = divmod(t, k // b2)
+            for i in range(b1):
+                mrow = p["meta"][p["meta_off"][t] + i * (b2 // 8):
+                                 p["meta_off"][t] + (i + 1) * (b2 // 8)]
+                bits = mask_bits(mrow)
+                vrow = p["vals"][p["val_off"][t] + i * (b2 * nk // m):
+                                 p["val_off"][t] + (i + 1) * (b2 * nk // m)]
+                w = W[tr * b1 + i, tc * b2:(tc + 1) * b2]
+                kept = [c for c in range(b2) if bits[c]]
+                for g in range(b2 // m):
+                    assert sum(bits[g * m:(g + 1) * m]) == nk
+                assert vrow.tolist() == [int(w[c]) for c in kept]
+        # all-sparse: a stable sort by descending magnitude picks the same columns
+        ones = np.ones(T, np.uint8)
+        W_hat = o.unpack_nm(n, k, b1, b2, nk, m, ones, o.pack_nm(W, b1, b2, ones, nk, m))
+        mag = np.abs(bits2f(W)).reshape(n, k // m, m)
+        order = np.argsort(-mag, axis=2, kind="stable")[:, :, :nk]
+        keep = np.zeros_like(mag, dtype=bool)
+        np.put_along_axis(keep, order, True, axis=2)
+        assert np.array_equal(W_hat, np.where(keep.reshape(n, k), W, 0).astype(np.uint16))
+
+
 ALL_PINS = [pin_golden, pin_bruteforce, pin_invariants, pin_all_dense,
-            pin_all_sparse, pin_lowrank, pin_rows, pin_special_values]
+            pin_all_sparse, pin_lowrank, pin_rows, pin_special_values,
+            pin_nm_golden, pin_nm_is_2of4, pin_nm_bruteforce, pin_nm_invariants]
