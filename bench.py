@@ -77,10 +77,15 @@ def measured_peak():
         return FALLBACK_HBM_GBS, "fallback"
 
 
+# Sources the streaming kernels (hybrid_tma_kernel, dense_gemv_kernel) are
+# compiled from: a profile taken on them stays valid while these are unchanged.
+PROFILED_SOURCES = ("hyb_internal.cuh", "hyb_spmv.cu")
+
+
 def csrc_digest():
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "sparse_weight_b200", "csrc")
-    for name in sorted(os.listdir(csrc)):
+    for name in PROFILED_SOURCES:
         with open(os.path.join(csrc, name), "rb") as fh:
             h.update(name.encode())
             h.update(fh.read())
@@ -433,8 +438,9 @@ class Calls:
     graph_timed).  make_args gives each call's arguments without the launch
     options, which go in front of the trailing (ws, ws_bytes, stream)."""
 
-    def __init__(self, fn, make_args, count, name):
+    def __init__(self, fn, make_args, count, name, with_flags=True):
         self.fn, self.make_args, self.count, self.name = fn, make_args, count, name
+        self.with_flags = with_flags  # False: an entry point without launch options
         self.flags = 0
         self.stream = torch.cuda.current_stream()
         self.set_stream(self.stream)
@@ -444,7 +450,8 @@ class Calls:
         self.args = []
         for i in range(self.count):
             a = list(self.make_args(i, sp))
-            a.insert(len(a) - 3, self.flags)
+            if self.with_flags:
+                a.insert(len(a) - 3, self.flags)
             self.args.append(tuple(a))
 
     def step(self, i):
@@ -633,6 +640,44 @@ def sweep(device, steps=200, warmup=10):
     return 0
 
 
+def sweep_nm(device, steps=200, warmup=10):
+    """General N:M tiles (hyb_spmm_skinny_nm, one warp per output row): the
+    4096x14336 down projection with 4:8 tiles at three fractions, batch 1 and 8,
+    graph replay of rotating copies (larger than L2)."""
+    peak, _ = measured_peak()
+    L = hyb.lib()
+    n, k, b1, b2, nk, m = 4096, 14336, 128, 128, 4, 8
+    W = inputs.weight(n, k, 0.02, inputs.seed_of("nm_sweep", "W"), outliers=0.01).to(device)
+    T = (n // b1) * (k // b2)
+    for f in (0.0, 0.5, 1.0):
+        tmap = inputs.tile_map_fraction(T, f, inputs.seed_of("nm_sweep", f))
+        base = hyb.pack_nm(W, tmap, b1, b2, nk, m)
+        nrot = max(2, int(np.ceil(3 * (126 << 20) / base.nbytes())))
+        mats = [base] + [base.clone() for _ in range(nrot - 1)]
+        structs = [x.struct() for x in mats]
+        ws = hyb.new_workspace(hyb.pack_workspace_bytes(), device)
+        for b in (1, 8):
+            xs = [inputs.activations(b, k, inputs.seed_of("nm_sweep", b, i)).to(device)
+                  for i in range(nrot)]
+            ys = [torch.empty(b, n, dtype=torch.float32, device=device) for _ in range(nrot)]
+            c = Calls(L.hyb_spmm_skinny_nm, lambda i, sp, b=b, xs=xs, ys=ys: (
+                ctypes.byref(structs[i]), nk, m, b, ctypes.c_void_p(xs[i].data_ptr()), k,
+                ctypes.c_void_p(ys[i].data_ptr()), n, hyb.HYB_F32,
+                ctypes.c_void_p(ws.data_ptr()), ws.numel(), sp), nrot, "nm", with_flags=False)
+            us = graph_timed(c, c.step, steps, warmup) / steps * 1e3
+            nbytes = base.nbytes() + base.num_tiles + 2 * b * k + 4 * b * n
+            gbs = nbytes / (us * 1e-6) / 1e9
+            print(json.dumps({"sweep": "nm", "pattern": f"{nk}:{m}", "shape": f"{n}x{k}",
+                              "tile": f"{b1}x{b2}", "sparse_tile_frac": float(np.mean(tmap)),
+                              "batch": b, "us": round(us, 3), "GBps": round(gbs, 1),
+                              "frac_of_measured_hbm": round(gbs / peak, 4),
+                              "kernel": "spmm_nm_kernel (one warp per output row)"}), flush=True)
+        hyb.check_status(ws)
+        del mats, structs, base
+        torch.cuda.empty_cache()
+    return 0
+
+
 def workload_config(name, frac_real):
     n, k, b1, b2, frac, batch, std, outliers = WORKLOADS[name]
     return {"workload": name, "n": n, "k": k, "tile": f"{b1}x{b2}",
@@ -657,6 +702,8 @@ def main():
     ap.add_argument("--sweep", action="store_true",
                     help="print the fraction / batch sweep, the 224-matrix chain and the 70B "
                          "low-rank lines instead of the headline line")
+    ap.add_argument("--nm", action="store_true",
+                    help="print the general N:M (4:8) lines instead of the headline line")
     ap.add_argument("--profile", action="store_true",
                     help="small case for a profiler: 2 rotating copies (184 MB > L2), "
                          "hybrid product only, no dense / end-to-end / CPU legs")
@@ -676,6 +723,8 @@ def main():
                                              device_id=device)
     if args.sweep:
         return sweep(device)
+    if args.nm:
+        return sweep_nm(device)
     wl = Workload(args.workload, device, rotate=args.rotate)
     stream = wl.stream
 

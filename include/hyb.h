@@ -249,6 +249,45 @@ HYB_API int hyb_gemv_dense_ex(int64_t n, int64_t k, int batch, const uint16_t *W
                               int64_t ldy, hyb_dtype ydt, uint32_t flags, void *ws,
                               size_t ws_bytes, hyb_stream_t stream);
 
+/* ---- general N:M tiles ---------------------------------------------------- */
+
+/* Tiles that are dense or N:M sparse for a general N:M: nk kept of every m
+ * consecutive columns, m in {4, 8, 16}, 0 < nk < m, b2 a multiple of m (and
+ * the tiling rules of hyb_pack).  PATCH, "Future direction": the tile-level
+ * scheme extends to other N:M patterns such as 4:8; SparseDecoding (authors'
+ * abstract): N:M with bitmask indexing and fixed-stride traversal.
+ * Layout: a sparse tile row keeps, in every group of m columns, the nk values
+ * with the largest key (bits & 0x7FFF, ties to the lower column), stored in
+ * ascending column order, nk per group (group g at nk*g of the row), and a
+ * b2-bit mask stream, bit c of the row's b2/8 bytes set iff column c is kept.
+ * A sparse tile holds b1*b2*nk/m values and b1*b2/8 mask bytes.  nk = 2,
+ * m = 4 is hyb_pack's layout bit for bit.  Unsupported m returns
+ * HYB_ERR_UNSUPPORTED; other bad arguments HYB_ERR_INVALID_ARG. */
+
+/* hyb_packed_sizes for nk:m tiles (host only). */
+HYB_API int hyb_packed_sizes_nm(int64_t n, int64_t k, int b1, int b2, int nk, int m,
+                                const uint8_t *tile_map_host, int64_t *n_vals,
+                                int64_t *n_meta_bytes);
+
+/* hyb_pack for nk:m tiles: same arguments, buffers, workspace (status word:
+ * NaN weight, bad map byte) and asynchrony as hyb_pack. */
+HYB_API int hyb_pack_nm(int64_t n, int64_t k, int b1, int b2, int nk, int m,
+                        const uint16_t *W, int64_t ldw, const uint8_t *tile_map,
+                        uint16_t *vals, uint8_t *meta, int64_t *val_off,
+                        int64_t *meta_off, void *ws, size_t ws_bytes,
+                        hyb_stream_t stream);
+
+/* Y = W_hat X for a matrix packed by hyb_pack_nm with the same nk, m; X
+ * [batch][k] bf16, batch 1..16, Y [batch][n] fp32 or bf16 (ydt), no low-rank
+ * term.  A->plan is not used.  The workspace needs hyb_pack_workspace_bytes()
+ * bytes (its status word: a tile whose offsets do not fit the buffers is
+ * skipped and flagged, read by hyb_check_status as HYB_ERR_DEVICE_CHECK).
+ * Asynchronous on stream; results are deterministic. */
+HYB_API int hyb_spmm_skinny_nm(const hyb_matrix *A, int nk, int m, int batch,
+                               const uint16_t *X, int64_t ldx, void *Y, int64_t ldy,
+                               hyb_dtype ydt, void *ws, size_t ws_bytes,
+                               hyb_stream_t stream);
+
 /* ---- product without any allocation ------------------------------------ */
 
 /* hyb_spmv for callers that cannot allocate device memory -- an engine that

@@ -69,7 +69,8 @@ EXPORTS = ["hyb_packed_sizes", "hyb_pack_workspace_bytes", "hyb_pack",
            "hyb_dense_workspace_bytes", "hyb_gemv_dense", "hyb_check_status",
            "hyb_status_string", "hyb_spmv_noalloc", "hyb_spmv_noalloc_max_scratch_bytes",
            "hyb_plan_entries", "hyb_make_plan", "hyb_selftest_wait_timeout",
-           "hyb_spmm_skinny_ex", "hyb_gemv_dense_ex"]
+           "hyb_spmm_skinny_ex", "hyb_gemv_dense_ex", "hyb_packed_sizes_nm",
+           "hyb_pack_nm", "hyb_spmm_skinny_nm"]
 
 
 def lib():
@@ -126,6 +127,14 @@ def lib():
     L.hyb_make_plan.argtypes = [ctypes.POINTER(HybMatrix), _P, _P, ctypes.POINTER(ctypes.c_int32),
                                 _P]
     L.hyb_make_plan.restype = _I
+    L.hyb_packed_sizes_nm.argtypes = [_I64, _I64, _I, _I, _I, _I, _P, _P, _P]
+    L.hyb_packed_sizes_nm.restype = _I
+    L.hyb_pack_nm.argtypes = [_I64, _I64, _I, _I, _I, _I, _P, _I64, _P, _P, _P, _P, _P, _P,
+                              _SZ, _P]
+    L.hyb_pack_nm.restype = _I
+    L.hyb_spmm_skinny_nm.argtypes = [ctypes.POINTER(HybMatrix), _I, _I, _I, _P, _I64, _P,
+                                     _I64, _I, _P, _SZ, _P]
+    L.hyb_spmm_skinny_nm.restype = _I
     L.hyb_status_string.argtypes = [_I]
     L.hyb_status_string.restype = ctypes.c_char_p
     _lib = L
@@ -275,6 +284,60 @@ def pack(W: torch.Tensor, tile_map, b1: int, b2: int, ws: torch.Tensor = None,
     if plan:
         P.plan, P.plan_ctas = make_plan(P, stream)
     return P
+
+
+def packed_sizes_nm(n: int, k: int, b1: int, b2: int, nk: int, m: int, tile_map) -> tuple:
+    """(n_vals, n_meta_bytes) of nk:m tiles for a host tile map."""
+    mp = np.ascontiguousarray(np.asarray(tile_map.cpu() if torch.is_tensor(tile_map)
+                                         else tile_map, dtype=np.uint8).reshape(-1))
+    nv, nmb = _I64(), _I64()
+    _check("hyb_packed_sizes_nm", lib().hyb_packed_sizes_nm(
+        n, k, b1, b2, nk, m, mp.ctypes.data_as(_P), ctypes.byref(nv), ctypes.byref(nmb)))
+    return nv.value, nmb.value
+
+
+def pack_nm(W: torch.Tensor, tile_map, b1: int, b2: int, nk: int, m: int,
+            ws: torch.Tensor = None, stream=None, check: bool = True) -> Packed:
+    """hyb_pack_nm: dense bf16 W [n][k] (device) + tile map -> Packed with
+    nk:m sparse tiles (no work-split plan: the N:M product does not use one)."""
+    Wb = _bits(W)
+    assert Wb.is_cuda and Wb.dim() == 2
+    n, k = Wb.shape
+    tm_host = tile_map.cpu().numpy() if torch.is_tensor(tile_map) else np.asarray(tile_map)
+    tm_host = np.ascontiguousarray(tm_host, dtype=np.uint8).reshape(-1)
+    nv, nmb = packed_sizes_nm(n, k, b1, b2, nk, m, tm_host)
+    dev = Wb.device
+    tm = torch.from_numpy(tm_host).to(dev)
+    T = tm.numel()
+    vals = torch.empty(nv, dtype=torch.int16, device=dev)
+    meta = torch.empty(max(nmb, 1), dtype=torch.uint8, device=dev)
+    vo = torch.empty(T + 1, dtype=torch.int64, device=dev)
+    mo = torch.empty(T + 1, dtype=torch.int64, device=dev)
+    if ws is None:
+        ws = new_workspace(pack_workspace_bytes(), dev)
+    _check("hyb_pack_nm", lib().hyb_pack_nm(n, k, b1, b2, nk, m, _ptr(Wb), Wb.stride(0),
+                                            _ptr(tm), _ptr(vals), _ptr(meta), _ptr(vo),
+                                            _ptr(mo), _ptr(ws), ws.numel(), _stream(stream)))
+    if check:
+        check_status(ws, stream)
+    return Packed(n, k, b1, b2, tm, vals, meta, vo, mo, nv, nmb)
+
+
+def spmm_skinny_nm(A: Packed, X: torch.Tensor, nk: int, m: int, Y: torch.Tensor = None,
+                   ydt: int = HYB_F32, ws: torch.Tensor = None, stream=None) -> torch.Tensor:
+    """hyb_spmm_skinny_nm: Y[batch][n] = W_hat X for nk:m tiles; X bf16 [batch][k]."""
+    Xb = _bits(X)
+    if Xb.dim() == 1:
+        Xb = Xb.view(1, -1)
+    batch = Xb.shape[0]
+    Y = _out(A.n, batch, ydt, Xb.device, Y)
+    if ws is None:
+        ws = new_workspace(pack_workspace_bytes(), Xb.device)
+    s = A.struct()
+    _check("hyb_spmm_skinny_nm", lib().hyb_spmm_skinny_nm(
+        ctypes.byref(s), nk, m, batch, _ptr(Xb), Xb.stride(0), _ptr(Y), Y.stride(0), ydt,
+        _ptr(ws), ws.numel(), _stream(stream)))
+    return Y
 
 
 def selftest_wait_timeout(ws: torch.Tensor, wait_limit: int = 2000, stream=None):

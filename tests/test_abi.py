@@ -163,6 +163,47 @@ def test_launch_flags_checked(L):
                                None) == hyb.HYB_ERR_INVALID_ARG
 
 
+def test_nm_sizes_and_argument_checks(L, orc):
+    """hyb_packed_sizes_nm (host only) against the oracle's offsets, and the
+    N:M entry points' synchronous argument checks."""
+    rng = np.random.default_rng(5)
+    for (nk, m) in [(1, 4), (2, 4), (3, 4), (2, 8), (4, 8), (6, 8), (4, 16), (8, 16)]:
+        n, k, b1, b2 = 256, 512, 64, 64
+        tmap = (rng.random((n // b1) * (k // b2)) < 0.5).astype(np.uint8)
+        nv, nmb = hyb.packed_sizes_nm(n, k, b1, b2, nk, m, tmap)
+        vo, mo = orc.offsets_nm(n, k, b1, b2, nk, m, tmap)
+        assert (nv, nmb) == (int(vo[-1]), int(mo[-1])), (nk, m)
+    # 2:4 through the N:M entry point is the 2:4 format
+    assert hyb.packed_sizes_nm(n, k, b1, b2, 2, 4, tmap) == hyb.packed_sizes(n, k, b1, b2, tmap)
+    P = ctypes.c_void_p
+    tm = np.zeros(64, np.uint8)
+    out = (ctypes.c_int64(), ctypes.c_int64())
+    sizes = lambda nk, m: L.hyb_packed_sizes_nm(
+        256, 512, 64, 64, nk, m, tm.ctypes.data_as(P), ctypes.byref(out[0]), ctypes.byref(out[1]))
+    assert sizes(4, 8) == hyb.HYB_OK
+    assert sizes(3, 6) == hyb.HYB_ERR_UNSUPPORTED
+    assert sizes(0, 8) == hyb.HYB_ERR_INVALID_ARG
+    assert sizes(8, 8) == hyb.HYB_ERR_INVALID_ARG
+    W, X, Y, ws = P(0x10000), P(0x60000), P(0x70000), P(0x80000)
+    assert L.hyb_pack_nm(256, 256, 64, 64, 4, 8, W, 256, P(0x20000), P(0x30000), P(0x40000),
+                         P(0x50000), P(0x58000), None, 0, None) == hyb.HYB_ERR_WORKSPACE
+    assert L.hyb_pack_nm(256, 256, 64, 64, 5, 6, W, 256, P(0x20000), P(0x30000), P(0x40000),
+                         P(0x50000), P(0x58000), ws, 1 << 20, None) == hyb.HYB_ERR_UNSUPPORTED
+    A = _matrix(n_vals=256 * 256 // 2, n_meta_bytes=256 * 256 // 8)
+    call = lambda A, nk=4, m=8, batch=1, X=X: L.hyb_spmm_skinny_nm(
+        ctypes.byref(A), nk, m, batch, X, 256, Y, 256, 0, ws, 1 << 20, None)
+    assert call(A, batch=17) == hyb.HYB_ERR_INVALID_ARG
+    assert call(A, nk=9) == hyb.HYB_ERR_INVALID_ARG
+    assert call(A, m=6) == hyb.HYB_ERR_UNSUPPORTED
+    assert call(A, X=None) == hyb.HYB_ERR_INVALID_ARG
+    assert call(A, X=P(0x60008)) == hyb.HYB_ERR_ALIGNMENT
+    assert call(_matrix(n_vals=5)) == hyb.HYB_ERR_INVALID_ARG
+    assert L.hyb_spmm_skinny_nm(None, 4, 8, 1, X, 256, Y, 256, 0, ws, 1 << 20,
+                                None) == hyb.HYB_ERR_INVALID_ARG
+    assert L.hyb_spmm_skinny_nm(ctypes.byref(A), 4, 8, 1, X, 256, Y, 256, 0, None, 0,
+                                None) == hyb.HYB_ERR_WORKSPACE
+
+
 def test_dense_and_lowrank_argument_checks(L):
     P = ctypes.c_void_p
     W, X, Y, ws = P(0x10000), P(0x60000), P(0x70000), P(0x80000)
