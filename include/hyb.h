@@ -304,19 +304,29 @@ HYB_API int hyb_spmm_skinny_nm(const hyb_matrix *A, int nk, int m, int batch,
  * frees nothing.  A matrix whose scratch would exceed the array (with
  * 128-row tiles: more than about 1,600 tile-row bands) is rejected with
  * HYB_ERR_WORKSPACE before anything is queued.
- *  - The first call on each device looks up the array's device address
- *    (cudaGetSymbolAddress) with that device current; make that first call
- *    outside any stream capture.
+ *  - The first call in each CUDA context looks up the array's device address
+ *    (cudaGetSymbolAddress) with that context current and caches it per
+ *    context; make that first call outside any stream capture.
  *  - All calls on a device share the one array.  Each call clears the part
- *    that must start at zero, but two calls whose work overlaps on the GPU
- *    (different streams, no ordering between them) race on it: order them,
- *    for instance by using one stream. */
+ *    that must start at zero (the band tickets), but two calls whose work
+ *    overlaps on the GPU (different streams, no ordering between them) race
+ *    on it: order them, for instance by using one stream.
+ *  - Problems the device detects (a bounded wait that ran out, a tile map
+ *    that does not fit its buffers) set the array's status word, which is
+ *    kept across calls until hyb_spmv_noalloc_check_status reads and clears
+ *    it. */
 HYB_API int hyb_spmv_noalloc(const hyb_matrix *A, const uint16_t *X,
                              int64_t ldx, void *Y, int64_t ldy, hyb_dtype ydt,
                              hyb_stream_t stream);
 
 /* Size in bytes of the static scratch array behind hyb_spmv_noalloc. */
 HYB_API size_t hyb_spmv_noalloc_max_scratch_bytes(void);
+
+/* hyb_check_status for the static array behind hyb_spmv_noalloc on the
+ * current device: synchronise `stream`, read and clear the status word that
+ * the noalloc calls since the last query have set.  Same return values and
+ * flag bits as hyb_check_status.  Allocates nothing. */
+HYB_API int hyb_spmv_noalloc_check_status(hyb_stream_t stream, uint32_t *flags);
 
 /* ---- status ------------------------------------------------------------ */
 

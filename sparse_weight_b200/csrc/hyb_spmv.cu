@@ -2093,24 +2093,54 @@ namespace {
 constexpr size_t kNoAllocScratchBytes = size_t(1) << 20;
 static __device__ __align__(256) uint8_t g_noalloc_scratch[kNoAllocScratchBytes];
 
-// Device address of the array on the current device.  The name of a
+// Device address of the array in the current CUDA context.  The name of a
 // __device__ variable in host code is only a host-side stand-in, so the
-// address is looked up once per device (with that device current) and
-// cached.
+// address is looked up (with the context current) and cached.  The cache is
+// keyed on the context, not on the device ordinal: after cudaDeviceReset, or
+// in another context on the same device, the module is loaded anew and the
+// array lives at another address.
 int noalloc_scratch_ptr(void **out) {
-  static std::mutex mu;
-  static void *addr[64] = {nullptr};
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return HYB_ERR_CUDA;
-  if (dev < 0 || dev >= 64) return HYB_ERR_UNSUPPORTED;
-  std::lock_guard<std::mutex> lock(mu);
-  if (addr[dev] == nullptr) {
+  using GetCtx = CUresult (*)(CUcontext *);
+  static GetCtx get_ctx = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void *fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &fn, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_ctx = reinterpret_cast<GetCtx>(fn);
+  });
+  if (!get_ctx) return HYB_ERR_CUDA;
+  CUcontext ctx = nullptr;
+  if (get_ctx(&ctx) != CUDA_SUCCESS) return HYB_ERR_CUDA;
+  if (ctx == nullptr) {
+    // no context current yet: the runtime's symbol lookup makes the device's
+    // primary context current
     void *p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr)
-      return HYB_ERR_CUDA;
-    addr[dev] = p;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess) return HYB_ERR_CUDA;
+    if (get_ctx(&ctx) != CUDA_SUCCESS || ctx == nullptr) return HYB_ERR_CUDA;
   }
-  *out = addr[dev];
+  static std::mutex mu;
+  struct Entry {
+    CUcontext ctx;
+    void *addr;
+  };
+  static Entry cache[64];
+  static int used = 0, next = 0;
+  std::lock_guard<std::mutex> lock(mu);
+  for (int i = 0; i < used; ++i)
+    if (cache[i].ctx == ctx) {
+      *out = cache[i].addr;
+      return HYB_OK;
+    }
+  void *p = nullptr;
+  if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr)
+    return HYB_ERR_CUDA;
+  // a full table recycles its oldest entry
+  const int slot = used < 64 ? used++ : (next++ % 64);
+  cache[slot] = Entry{ctx, p};
+  *out = p;
   return HYB_OK;
 }
 
@@ -2154,13 +2184,23 @@ int hyb_spmv_noalloc(const hyb_matrix *A, const uint16_t *X, int64_t ldx,
   rc = hyb::noalloc_scratch_ptr(&scratch);
   if (rc != HYB_OK) return rc;
   cudaStream_t s = (cudaStream_t)stream;
-  // The array keeps whatever the previous call left.  The status word and the
-  // band tickets must start at zero (the partial slots are always written
-  // before they are read), so clear everything in front of the slots.
-  if (cudaMemsetAsync(scratch, 0, P.off_partials, s) != cudaSuccess)
+  // The array keeps whatever the previous call left.  The band tickets must
+  // start at zero (the partial slots are always written before they are
+  // read), so clear everything between the header and the slots.  The status
+  // word at the head is not cleared: it collects the flags of every call
+  // until hyb_spmv_noalloc_check_status reads and clears it.
+  if (cudaMemsetAsync(static_cast<uint8_t *>(scratch) + hyb::kHeaderBytes, 0,
+                      P.off_partials - hyb::kHeaderBytes, s) != cudaSuccess)
     return HYB_ERR_CUDA;
   return hyb::spmm_impl(A, 1, X, ldx, Y, ldy, ydt, nullptr, scratch,
                         hyb::kNoAllocScratchBytes, s);
+}
+
+int hyb_spmv_noalloc_check_status(hyb_stream_t stream, uint32_t *flags) {
+  void *scratch = nullptr;
+  const int rc = hyb::noalloc_scratch_ptr(&scratch);
+  if (rc != HYB_OK) return rc;
+  return hyb_check_status(scratch, stream, flags);
 }
 
 int hyb_selftest_wait_timeout(void *ws, size_t ws_bytes, uint32_t wait_limit,

@@ -68,6 +68,7 @@ EXPORTS = ["hyb_packed_sizes", "hyb_pack_workspace_bytes", "hyb_pack",
            "hyb_spmm_skinny", "hyb_lowrank_workspace_bytes", "hyb_lowrank_add",
            "hyb_dense_workspace_bytes", "hyb_gemv_dense", "hyb_check_status",
            "hyb_status_string", "hyb_spmv_noalloc", "hyb_spmv_noalloc_max_scratch_bytes",
+           "hyb_spmv_noalloc_check_status",
            "hyb_plan_entries", "hyb_make_plan", "hyb_selftest_wait_timeout",
            "hyb_spmm_skinny_ex", "hyb_gemv_dense_ex", "hyb_packed_sizes_nm",
            "hyb_pack_nm", "hyb_spmm_skinny_nm"]
@@ -122,6 +123,8 @@ def lib():
     L.hyb_spmv_noalloc.restype = _I
     L.hyb_spmv_noalloc_max_scratch_bytes.argtypes = []
     L.hyb_spmv_noalloc_max_scratch_bytes.restype = _SZ
+    L.hyb_spmv_noalloc_check_status.argtypes = [_P, ctypes.POINTER(ctypes.c_uint32)]
+    L.hyb_spmv_noalloc_check_status.restype = _I
     L.hyb_plan_entries.argtypes = []
     L.hyb_plan_entries.restype = _SZ
     L.hyb_make_plan.argtypes = [ctypes.POINTER(HybMatrix), _P, _P, ctypes.POINTER(ctypes.c_int32),
@@ -484,3 +487,15 @@ def spmv_noalloc(A: Packed, x: torch.Tensor, y: torch.Tensor = None, ydt: int = 
 
 def spmv_noalloc_max_scratch_bytes() -> int:
     return int(lib().hyb_spmv_noalloc_max_scratch_bytes())
+
+
+def spmv_noalloc_check_status(stream=None) -> int:
+    """hyb_spmv_noalloc_check_status: sync, read + clear the status word of the
+    static array behind hyb_spmv_noalloc; raise on a flag."""
+    flags = ctypes.c_uint32(0)
+    rc = lib().hyb_spmv_noalloc_check_status(_stream(stream), ctypes.byref(flags))
+    if rc != HYB_OK:
+        err = HybError("hyb_spmv_noalloc_check_status", rc)
+        err.flags = flags.value
+        raise err
+    return flags.value
