@@ -53,10 +53,10 @@
  *    (fp32 or bf16) with ldy >= n.  X and meta must be 16-byte aligned and
  *    ldx a multiple of 8 (rows of X 16-byte aligned); vals 32-byte aligned;
  *    Y aligned to its element size; workspaces 256-byte aligned.
- *  - Shapes: n % b1 == 0, k % b2 == 0, b2 % 16 == 0, (b1 * b2) % 128 == 0.
+ *  - Shapes: n % b1 == 0, k % b2 == 0, b2 % 8 == 0, (b1 * b2) % 128 == 0.
  *    Any batch 1..16.  Tiles of 64 or 128 rows by 64 or 128 columns run the
- *    tuned streaming kernel; other legal tilings run a simpler CUDA kernel
- *    (never a CPU fallback).
+ *    tuned streaming kernel; other legal tilings (b2 = 8, 16, 24, ...) run a
+ *    simpler one-warp-per-row CUDA kernel (never a CPU fallback).
  */
 #ifndef HYB_H
 #define HYB_H
@@ -208,10 +208,15 @@ HYB_API int hyb_spmm_skinny(const hyb_matrix *A, int batch, const uint16_t *X,
  * hyb_gemv_dense_ex) -- are not written by the work queued before the call on
  * the stream that has not finished by then.  Tilings served by the
  * one-warp-per-row kernel ignore the flag.
- * With a low-rank term the call runs three kernels (V^T x, U t, the product);
- * the flag applies to the first, and the later two always start as
- * programmatic dependents of the one before them, after all work queued
- * before the call has finished. */
+ * Low-rank term: with the tuned tilings the term is computed inside the
+ * streaming kernel (one launch per call).  One warp per CTA computes V^T x
+ * over a slice of V's rows, then t by slices, then U t for a slice of the
+ * output rows.  Bounded grid barriers separate the steps; the CTAs are
+ * never more than the SMs and there is one per SM, so all of them can be
+ * resident.  If other work on the GPU kept some of them from starting for
+ * seconds, the wait runs out and hyb_check_status reports HYB_ERR_TIMEOUT.
+ * Other tilings run three kernels (V^T x, U t, the product) one after
+ * another; the flag applies to the first. */
 
 /* hyb_spmm_skinny with launch options `flags` (0 = hyb_spmm_skinny). */
 HYB_API int hyb_spmm_skinny_ex(const hyb_matrix *A, int batch, const uint16_t *X,
@@ -261,8 +266,9 @@ HYB_API int hyb_gemv_dense_ex(int64_t n, int64_t k, int batch, const uint16_t *W
  * ascending column order, nk per group (group g at nk*g of the row), and a
  * b2-bit mask stream, bit c of the row's b2/8 bytes set iff column c is kept.
  * A sparse tile holds b1*b2*nk/m values and b1*b2/8 mask bytes.  nk = 2,
- * m = 4 is hyb_pack's layout bit for bit.  Unsupported m returns
- * HYB_ERR_UNSUPPORTED; other bad arguments HYB_ERR_INVALID_ARG. */
+ * m = 4 is hyb_pack's layout bit for bit.  Unsupported m, or b2 not a
+ * multiple of 16, returns HYB_ERR_UNSUPPORTED; other bad arguments
+ * HYB_ERR_INVALID_ARG. */
 
 /* hyb_packed_sizes for nk:m tiles (host only). */
 HYB_API int hyb_packed_sizes_nm(int64_t n, int64_t k, int b1, int b2, int nk, int m,
@@ -279,10 +285,15 @@ HYB_API int hyb_pack_nm(int64_t n, int64_t k, int b1, int b2, int nk, int m,
 
 /* Y = W_hat X for a matrix packed by hyb_pack_nm with the same nk, m; X
  * [batch][k] bf16, batch 1..16, Y [batch][n] fp32 or bf16 (ydt), no low-rank
- * term.  A->plan is not used.  The workspace needs hyb_pack_workspace_bytes()
- * bytes (its status word: a tile whose offsets do not fit the buffers is
- * skipped and flagged, read by hyb_check_status as HYB_ERR_DEVICE_CHECK).
- * Asynchronous on stream; results are deterministic. */
+ * term.  2 of 4 and 4 of 8 with 64- or 128-row by 64- or 128-column tiles run
+ * the streaming kernel of hyb_spmm_skinny (the same split, plan -- A->plan is
+ * used -- and stage packing: these patterns keep half of a tile's values
+ * with b1*b2/8 mask bytes); other patterns and tilings run a one-warp-per-row
+ * kernel.  The workspace needs hyb_workspace_bytes(A, batch, 0) bytes and is
+ * zeroed once, as for hyb_spmm_skinny (its status word: a bounded wait that
+ * ran out; a tile whose offsets do not fit the buffers is skipped and
+ * flagged, read by hyb_check_status as HYB_ERR_DEVICE_CHECK).  Asynchronous on
+ * stream; results are deterministic. */
 HYB_API int hyb_spmm_skinny_nm(const hyb_matrix *A, int nk, int m, int batch,
                                const uint16_t *X, int64_t ldx, void *Y, int64_t ldy,
                                hyb_dtype ydt, void *ws, size_t ws_bytes,

@@ -18,6 +18,15 @@ constexpr uint32_t kStatusTimeout = 4u;  // a bounded wait inside a kernel ran o
 
 // Workspace header: status word, padded so that what follows is aligned.
 constexpr size_t kHeaderBytes = 256;
+// At fixed places whatever the call's shape, batch or rank (so that calls of
+// different shapes can share a workspace): in the header, the epoch of the
+// fused low-rank term's grid barriers and the ticket of the separate V^T x
+// kernel; after the header, one barrier flag per CTA of the fused term.
+constexpr size_t kLowrankEpochOffset = 16;
+constexpr size_t kLowrankTicketOffset = 24;
+constexpr size_t kLowrankFlagsOffset = kHeaderBytes;
+constexpr int kLowrankFlags = 256;  // at least the most CTAs a streaming launch has
+constexpr size_t kTicketsOffset = kLowrankFlagsOffset + 4 * kLowrankFlags;
 
 __host__ __device__ inline size_t align_up(size_t v, size_t a) {
   return (v + a - 1) / a * a;
@@ -56,6 +65,19 @@ __device__ __forceinline__ void ld_stream32(const void *p, uint4 &a, uint4 &b) {
       : "=r"(a.x), "=r"(a.y), "=r"(a.z), "=r"(a.w), "=r"(b.x), "=r"(b.y),
         "=r"(b.z), "=r"(b.w)
       : "l"(p));
+}
+// 8-byte load, same hints as ld_stream16.
+__device__ __forceinline__ uint2 ld_stream8(const void *p) {
+  uint2 r;
+  asm volatile("ld.global.nc.L1::no_allocate.v2.u32 {%0,%1}, [%2];"
+               : "=r"(r.x), "=r"(r.y)
+               : "l"(p));
+  return r;
+}
+__device__ __forceinline__ uint32_t ld_stream_u8(const void *p) {
+  uint16_t r;
+  asm volatile("ld.global.nc.L1::no_allocate.u8 %0, [%1];" : "=h"(r) : "l"(p));
+  return r;
 }
 __device__ __forceinline__ uint16_t ld_stream_u16(const void *p) {
   uint16_t r;

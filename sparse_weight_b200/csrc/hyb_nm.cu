@@ -21,6 +21,9 @@
 namespace hyb {
 
 int check_tiling(int64_t n, int64_t k, int b1, int b2);  // hyb_pack.cu
+int stream_product_nm(const hyb_matrix *A, int nk, int m, int batch, const uint16_t *X,
+                      int64_t ldx, void *Y, int64_t ldy, hyb_dtype ydt, void *ws,
+                      size_t ws_bytes, cudaStream_t s);  // hyb_spmv.cu
 
 namespace {
 
@@ -32,6 +35,8 @@ int check_nm(int b2, int nk, int m) {
   if (!(m == 4 || m == 8 || m == 16)) return HYB_ERR_UNSUPPORTED;
   if (nk <= 0 || nk >= m) return HYB_ERR_INVALID_ARG;
   if (b2 % m != 0) return HYB_ERR_INVALID_ARG;
+  // the N:M pack works on 16-column units of a tile row
+  if (b2 % 16 != 0) return HYB_ERR_UNSUPPORTED;
   return HYB_OK;
 }
 
@@ -345,6 +350,10 @@ int hyb_spmm_skinny_nm(const hyb_matrix *A, int nk, int m, int batch, const uint
   if ((uintptr_t)X % 16 != 0 || ldx % 8 != 0) return HYB_ERR_ALIGNMENT;
   if ((uintptr_t)Y % (ydt == HYB_F32 ? 4 : 2) != 0) return HYB_ERR_ALIGNMENT;
   if (!ws || ws_bytes < hyb::kHeaderBytes) return HYB_ERR_WORKSPACE;
+  // 2 of 4 and 4 of 8 with the tuned tilings: the streaming kernel
+  rc = hyb::stream_product_nm(A, nk, m, batch, X, ldx, Y, ldy, ydt, ws, ws_bytes,
+                              (cudaStream_t)stream);
+  if (rc != HYB_ERR_UNSUPPORTED) return rc;
   hyb::NmParams prm{};
   prm.map = A->tile_map;
   prm.vals = A->vals;

@@ -138,7 +138,7 @@ __global__ void __launch_bounds__(kPackThreads)
 int check_tiling(int64_t n, int64_t k, int b1, int b2) {
   if (n <= 0 || k <= 0 || b1 <= 0 || b2 <= 0) return HYB_ERR_INVALID_ARG;
   if (n % b1 != 0 || k % b2 != 0) return HYB_ERR_INVALID_ARG;
-  if (b2 % 16 != 0) return HYB_ERR_INVALID_ARG;
+  if (b2 % 8 != 0) return HYB_ERR_INVALID_ARG;  // whole mask bytes per 2:4 tile row
   if (((int64_t)b1 * b2) % 128 != 0) return HYB_ERR_INVALID_ARG;
   return HYB_OK;
 }

@@ -1,29 +1,29 @@
-// hyb_spmv.cu -- Y = W_hat X (+ U (V^T X)) for the tile-hybrid format, plus
-// the dense GEMV baseline and the stand-alone low-rank term.
+// hyb_spmv.cu -- Y = W_hat X (+ U (V^T X)) for the tile-hybrid format, the
+// dense GEMV baseline and the stand-alone low-rank term.
 //
 // Decode-time products are memory-bound ("SparseDecoding: decoding-aware
 // pruning ...", authors' abstract: the decode phase is limited by memory
 // access and is dominated by sparse matrix-vector products), so every kernel
 // here is a single streaming pass over the weight bytes with no tensor cores.
 //
-//  * hybrid_tma_kernel (packed matrices, tilings 128x128, 128x64, 64x64,
-//    64x128): the packed stream is row-major over tiles, so every tile-row
-//    band is contiguous.  CTA c of G takes the tiles whose byte offset falls
-//    in [c, c+1) * total / G -- a split by bytes, not by tiles, because a
-//    dense tile costs 2 B/weight and a 2:4 tile 1.125 B/weight ("PATCH:
-//    Learnable Tile-level Hybrid Sparsity for LLMs", §2: tiles are dense or
-//    2:4).  A producer warp moves the bytes into a shared-memory ring with
-//    bulk copies; consumer warps compute from it; two epilogue warps finish
-//    the bands.
+//  * hybrid_tma_kernel (tilings 128x128, 128x64, 64x64, 64x128): the packed
+//    stream is row-major over tiles, so every tile-row band is contiguous.
+//    CTA c of G takes the tiles whose byte offset falls in [c, c+1) * total /
+//    G -- a split by bytes, not by tiles, because a dense tile costs
+//    2 B/weight and a 2:4 tile 1.125 B/weight ("PATCH: Learnable Tile-level
+//    Hybrid Sparsity for LLMs", §2: tiles are dense or 2:4).  A producer warp
+//    moves the bytes into a shared-memory ring with bulk copies; consumer
+//    warps compute from it; two epilogue warps finish the bands; a low-rank
+//    warp computes the L = U V^T term ("3BASiL", §1: W ~ S + L) in the same
+//    pass.  The same kernel streams a plain row-major W (every tile dense,
+//    each tile one 2-D tensor copy): the dense baseline the format is
+//    measured against.
 //  * hybrid_rowwarp_kernel (any other legal tiling, packed or row-major): one
 //    warp per output row, plain loads.
-//  * dense_gemv_kernel (row-major bf16 W, the baseline the format is measured
-//    against): the same byte split over uniform tiles, register double
-//    buffering instead of a ring.
 //  * Band results cross CTAs through fp32 partial slots; the last CTA to
 //    arrive at a band (atomic ticket, no spinning) sums the slots in CTA order
-//    -- deterministic -- and applies the epilogue: the low-rank term
-//    ("3BASiL", §1: W ~ S + L) and the fp32 or bf16 store.
+//    -- deterministic -- and applies the epilogue: the low-rank term and the
+//    fp32 or bf16 store.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
@@ -43,7 +43,9 @@ constexpr int kThreads = kWarps * 32;
 constexpr int kMaxRank = 256;
 
 struct Params {
-  // matrix (packed) or dense W (strided mode)
+  // matrix: packed, or (rowmajor) a plain row-major bf16 W read through the
+  // kernel's W tensor map, every b1 x b2 tile dense
+  int rowmajor;
   const uint8_t *map;
   const uint8_t *vals;  // bytes
   const uint8_t *meta;
@@ -60,27 +62,35 @@ struct Params {
   void *Y;
   int64_t ldy;
   int ydt;
-  // low rank: t = V^T x and then ut = U t (fp32 [batch][n]) are computed by
-  // two small kernels before the product; the product's epilogue adds ut
+  // low rank: t = V^T x (fp32 [BP][rank]) and ut = U t (fp32 [BP][n]); the
+  // product's epilogue adds ut.  Fused (streaming kernel): the kernel's
+  // low-rank warp computes both, with lr_part ([G][BP][rank] partials of t),
+  // lr_epoch (the calls' barrier epoch) and lr_flags (one barrier flag per
+  // CTA) in the workspace.  Not fused (other tilings): two small kernels
+  // compute them before the product.
   const uint16_t *U;
   int64_t ldu;
+  const uint16_t *V;
+  int64_t ldv;
   int rank;
-  const float *lr_t;
-  const float *lr_ut;
+  int fused_lr;
+  float *lr_t;
+  float *lr_ut;
+  float *lr_part;
+  uint32_t *lr_epoch;
+  uint32_t *lr_flags;
   // split
   int G;
+  int nst;        // ring stages this launch uses (at most the kernel's compile-time count)
   int64_t total;  // packed bytes of the whole matrix
   float *partials;
   uint32_t *counters;
   uint32_t *status;  // workspace status word
   int64_t nvb, nmb;  // bytes of the value and mask buffers
   // 1: launched as a programmatic dependent of the preceding kernel on the
-  // stream.  The weights (packed matrix or row-major W) may then be read
-  // before that kernel has finished; X, Y, the workspace and the low-rank
-  // intermediates are touched only after griddepcontrol.wait.
-  // 2: the same, behind the low-rank kernels of the same call, which start
-  // only once all work before the call has finished: X may be read at once,
-  // and only the epilogue (Y, workspace, U t) waits.
+  // stream.  The weights (packed matrix or row-major W, and U, V) may then be
+  // read before that kernel has finished; X, Y and the workspace are touched
+  // only after griddepcontrol.wait.
   int pdl;
 };
 
@@ -115,11 +125,6 @@ struct LaunchPlan {
 // helpers
 // ---------------------------------------------------------------------------
 
-template <int BP>
-struct XRegs {
-  uint4 v[BP][2];  // 16 bf16 per batch column
-};
-
 // Select x[p0] and x[p1] of one group from its 4-bit mask (two bits set):
 // p0 is the lowest set bit, p1 the highest.
 __device__ __forceinline__ void pick2(uint32_t nib, float x0, float x1,
@@ -129,228 +134,15 @@ __device__ __forceinline__ void pick2(uint32_t nib, float x0, float x1,
   xb = (nib & 8u) ? x3 : ((nib & 4u) ? x2 : x1);
 }
 
-__device__ __forceinline__ void unpack16(const uint4 &a, const uint4 &b,
-                                         float f[16]) {
-  const uint32_t w[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
-#pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    f[2 * i] = bf16_lo(w[i]);
-    f[2 * i + 1] = bf16_hi(w[i]);
-  }
-}
-
-__device__ __forceinline__ int owner_of(int64_t P, const Params &p) {
-  int64_t o = (P * p.G) / p.total;
-  return (int)(o < p.G - 1 ? o : p.G - 1);
-}
-
 // Epilogue for one (row, batch) output: add the low-rank term, store.
 __device__ __forceinline__ void store_out(const Params &p, int64_t row, int b,
                                           float y) {
-  if (p.lr_ut != nullptr) y += p.lr_ut[(int64_t)b * p.n + row];
+  if (p.lr_ut != nullptr) y += __ldcg(p.lr_ut + (int64_t)b * p.n + row);
   if (p.ydt == HYB_BF16)
     reinterpret_cast<uint16_t *>(p.Y)[(int64_t)b * p.ldy + row] =
         f32_to_bf16_rne(y);
   else
     reinterpret_cast<float *>(p.Y)[(int64_t)b * p.ldy + row] = y;
-}
-
-// ---------------------------------------------------------------------------
-// dense GEMV baseline: row-major bf16 W, CTA c takes tiles
-// [c, c+1) * T / G (all tiles cost the same); warp w owns rows [w*R, (w+1)*R)
-// of a tile and a lane 16 columns of one row per step; the next tile is
-// loaded into registers while the current one computes
-// ---------------------------------------------------------------------------
-
-template <int BP, int B1, int B2>
-struct Cfg {
-  static constexpr int RW = B1 / kWarps;    // rows per warp per tile
-  static constexpr int CPR = B2 / 16;       // lanes per row (16 columns each)
-  static constexpr int RPS = 32 / CPR;      // rows per warp step
-  static constexpr int JS = RW / RPS;       // steps per warp per tile
-  static constexpr int XB = BP < 4 ? BP : 4;  // batch columns per x sub-block
-  static constexpr int64_t kDenseCost = 2LL * B1 * B2;
-  static constexpr int kMinBlocks = BP <= 1 ? 2 : 1;
-  static_assert(RW * kWarps == B1, "b1 must split over the warps");
-  static_assert(RPS * CPR == 32 && JS * RPS == RW, "tile shape");
-};
-
-// Registers of one tile in flight: 32 B (16 bf16) per lane per step.
-template <int JS>
-struct TileRegs {
-  uint4 a[JS];
-  uint4 b[JS];
-};
-
-template <int BP, int B1, int B2>
-__global__ void __launch_bounds__(kThreads, (Cfg<BP, B1, B2>::kMinBlocks))
-    dense_gemv_kernel(const Params p) {
-  using C = Cfg<BP, B1, B2>;
-  constexpr int JS = C::JS;
-  extern __shared__ int s_owner[];  // [2 * R]: owner CTA of each band's first / last tile
-  __shared__ float s_acc[B1 * BP];
-  __shared__ int64_t s_range[2];
-  __shared__ int s_last;
-
-  const int tid = threadIdx.x;
-  const int warp = tid >> 5, lane = tid & 31;
-  const int cp = lane % C::CPR;  // 16-column part
-  const int rs = lane / C::CPR;  // row inside a step
-  const int c = blockIdx.x;
-  const int G = p.G;
-  if (p.pdl) grid_dep_trigger();
-
-  // ---- 1. this CTA's tile range [t0, t1) -----------------------------------
-  const int64_t tgtA = (int64_t)c * p.total;
-  const int64_t tgtB = (int64_t)(c + 1) * p.total;
-  // uniform tiles: the split is a closed form
-  const int64_t unit = C::kDenseCost * G;
-  int64_t t0 = (tgtA + unit - 1) / unit;
-  int64_t t1 = (c == G - 1) ? p.T : (tgtB + unit - 1) / unit;
-  for (int i = tid; i < p.R; i += kThreads) {
-    s_owner[2 * i] = owner_of((int64_t)i * p.tpr * C::kDenseCost, p);
-    s_owner[2 * i + 1] = owner_of(((int64_t)(i + 1) * p.tpr - 1) * C::kDenseCost, p);
-  }
-  if (tid == 0) {
-    s_range[0] = t0;
-    s_range[1] = t1;
-  }
-  __syncthreads();
-  t0 = s_range[0];
-  t1 = s_range[1];
-
-  // ---- 2. stream the tiles --------------------------------------------------
-  float acc[JS][BP];
-#pragma unroll
-  for (int j = 0; j < JS; ++j)
-#pragma unroll
-    for (int b = 0; b < BP; ++b) acc[j][b] = 0.f;
-
-  const int wrow = warp * C::RW;  // first row of this warp inside a tile
-
-  // a lane's 16 columns of JS rows of a tile of the row-major W
-  auto load_tile = [&](int64_t t, TileRegs<JS> &r) {
-    const int64_t tr = t / p.tpr, tc = t - tr * p.tpr;
-    const uint16_t *base = p.Wd + (tr * B1 + wrow + rs) * p.ldw + tc * B2 + 16 * cp;
-#pragma unroll
-    for (int j = 0; j < JS; ++j) ld_stream32(base + (int64_t)j * C::RPS * p.ldw, r.a[j], r.b[j]);
-  };
-  auto load_x = [&](int64_t t, int b0, XRegs<C::XB> &xr) {
-    const int64_t tc = t % p.tpr;
-    const uint16_t *xp = p.X + tc * B2 + 16 * cp;
-#pragma unroll
-    for (int b = 0; b < C::XB; ++b) {
-      if (b0 + b < p.batch) {
-        xr.v[b][0] = ld_keep16(xp + (int64_t)(b0 + b) * p.ldx);
-        xr.v[b][1] = ld_keep16(xp + (int64_t)(b0 + b) * p.ldx + 8);
-      } else {
-        xr.v[b][0] = make_uint4(0, 0, 0, 0);
-        xr.v[b][1] = make_uint4(0, 0, 0, 0);
-      }
-    }
-  };
-
-  // flush the accumulators of band r: lanes -> shared -> slot or epilogue
-  auto flush = [&](int r) {
-#pragma unroll
-    for (int j = 0; j < JS; ++j)
-#pragma unroll
-      for (int b = 0; b < BP; ++b) {
-        float v = acc[j][b];
-#pragma unroll
-        for (int o = 1; o < C::CPR; o <<= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-        acc[j][b] = v;
-      }
-    if (cp == 0) {
-#pragma unroll
-      for (int j = 0; j < JS; ++j)
-#pragma unroll
-        for (int b = 0; b < BP; ++b)
-          s_acc[(wrow + j * C::RPS + rs) * BP + b] = acc[j][b];
-    }
-#pragma unroll
-    for (int j = 0; j < JS; ++j)
-#pragma unroll
-      for (int b = 0; b < BP; ++b) acc[j][b] = 0.f;
-    __syncthreads();
-    const int oA = s_owner[2 * r], oB = s_owner[2 * r + 1];
-    const int64_t row0 = (int64_t)r * B1;
-    if (oA == oB) {
-      // this CTA owns the whole band
-      for (int i = tid; i < B1 * BP; i += kThreads) {
-        const int row = i % B1, b = i / B1;
-        if (b < p.batch) store_out(p, row0 + row, b, s_acc[row * BP + b]);
-      }
-    } else {
-      float *slot = p.partials + (int64_t)(c + r) * (B1 * BP);
-      for (int i = tid; i < B1 * BP; i += kThreads) __stcg(slot + i, s_acc[i]);
-      __threadfence();
-      __syncthreads();
-      if (tid == 0) {
-        const uint32_t prev = atomicAdd(p.counters + r, 1u);
-        s_last = prev == (uint32_t)(oB - oA);
-      }
-      __syncthreads();
-      if (s_last) {
-        __threadfence();
-        for (int i = tid; i < B1 * BP; i += kThreads) {
-          const int row = i % B1, b = i / B1;
-          if (b >= p.batch) continue;
-          float y = 0.f;
-          for (int cc = oA; cc <= oB; ++cc)
-            y += __ldcg(p.partials + (int64_t)(cc + r) * (B1 * BP) + row * BP + b);
-          store_out(p, row0 + row, b, y);
-        }
-        if (tid == 0) p.counters[r] = 0;  // ready for the next call
-      }
-    }
-    __syncthreads();
-  };
-
-  if (t0 < t1) {
-    TileRegs<JS> cur;
-    load_tile(t0, cur);
-    // the first tile of W is on its way; X and everything written below may
-    // belong to the preceding grid
-    if (p.pdl) grid_dep_wait();
-    XRegs<C::XB> xcur;
-    if (BP <= 4) load_x(t0, 0, xcur);
-    for (int64_t t = t0; t < t1; ++t) {
-      TileRegs<JS> nxt;
-      XRegs<C::XB> xnxt;
-      if (t + 1 < t1) {
-        load_tile(t + 1, nxt);
-        if (BP <= 4) load_x(t + 1, 0, xnxt);
-      }
-      // ---- compute tile t ----
-#pragma unroll
-      for (int b0 = 0; b0 < BP; b0 += C::XB) {
-        XRegs<C::XB> xs;
-        if (BP <= 4) {
-          xs = xcur;
-        } else {
-          load_x(t, b0, xs);
-        }
-        float xf[C::XB][16];
-#pragma unroll
-        for (int b = 0; b < C::XB; ++b) unpack16(xs.v[b][0], xs.v[b][1], xf[b]);
-#pragma unroll
-        for (int j = 0; j < JS; ++j) {
-          float wf[16];
-          unpack16(cur.a[j], cur.b[j], wf);
-#pragma unroll
-          for (int e = 0; e < 16; ++e)
-#pragma unroll
-            for (int b = 0; b < C::XB; ++b)
-              acc[j][b0 + b] = fmaf(wf[e], xf[b][e], acc[j][b0 + b]);
-        }
-      }
-      // band boundary or end of range: flush
-      if (t + 1 == t1 || (t + 1) % p.tpr == 0) flush((int)(t / p.tpr));
-      cur = nxt;
-      xcur = xnxt;
-    }
-  }
 }
 
 // ---------------------------------------------------------------------------
@@ -384,6 +176,11 @@ __global__ void __launch_bounds__(kThreads, (Cfg<BP, B1, B2>::kMinBlocks))
 // still selects within the group's four values.
 
 constexpr uint32_t kWaitLimit = 1u << 22;
+// The low-rank warp's chunk buffer after the ring: two halves (16 KB of
+// dynamic shared memory, requested only by launches with a low-rank term;
+// such launches may use one ring stage fewer to make room).
+constexpr int kLrHalf = 8192;
+constexpr int kLrBufBytes = 2 * kLrHalf;
 
 __device__ __forceinline__ uint32_t smem_u32(const void *p) {
   return (uint32_t)__cvta_generic_to_shared(p);
@@ -438,6 +235,60 @@ __device__ __forceinline__ uint32_t atom_add_acq_rel(uint32_t *addr, uint32_t v)
                : "memory");
   return old;
 }
+__device__ __forceinline__ uint32_t ld_acquire_u32(const uint32_t *addr) {
+  uint32_t v;
+  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(addr) : "memory");
+  return v;
+}
+__device__ __forceinline__ void st_release_u32(uint32_t *addr, uint32_t v) {
+  asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(addr), "r"(v) : "memory");
+}
+
+// Grid barrier over the G CTAs of a launch, called by one whole warp per CTA.
+// Every CTA has a flag word; arriving CTA c publishes flags[c] = target with
+// a release store (after a warp barrier, so that it covers everything the
+// warp wrote before), and the warp's lanes then poll all G flags until each
+// has reached target.  No atomics, so arrivals do
+// not queue on one address.  Targets are per call: the call's epoch (read
+// from the workspace at the start) plus the barrier's number, so flags left
+// by earlier calls are always behind.  Needs every CTA of the grid to be
+// resident at some point while the others wait: the streaming kernel runs at
+// most one CTA per SM and no more CTAs than SMs.  The wait is bounded: false
+// when it ran out.
+constexpr uint32_t kGridWaitLimit = 1u << 20;
+__device__ __forceinline__ bool flag_barrier(uint32_t *flags, int G, int c, uint32_t target,
+                                             int lane) {
+  __syncwarp();
+  if (lane == 0) st_release_u32(flags + c, target);
+  // each lane polls the flags of CTAs lane, lane + 32, ... with acquire
+  // loads, so what a CTA published before its flag is visible after the wait
+  bool done = false;
+  for (uint32_t i = 0; i < kGridWaitLimit && !done; ++i) {
+    bool mine = true;
+    for (int q = lane; q < G; q += 32) mine &= (int32_t)(ld_acquire_u32(flags + q) - target) >= 0;
+    done = __all_sync(0xffffffffu, mine);
+    if (!done) __nanosleep(32);
+  }
+  __syncwarp();
+  return done;
+}
+
+// 16-byte asynchronous copy global -> shared through the load/store path
+// (L2 only), completion tracked per thread by commit / wait groups.  Used for
+// the low-rank warp's small chunks so they do not queue in the TMA engine
+// behind the ring's stage copies.
+__device__ __forceinline__ void cp_async16(void *dst, const void *src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(dst)), "l"(src)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() {
+  asm volatile("cp.async.commit_group;" ::: "memory");
+}
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+
 __device__ __forceinline__ void bulk_g2s(void *dst, const void *src, uint32_t bytes,
                                          uint64_t *bar) {
   asm volatile(
@@ -465,10 +316,10 @@ __device__ __forceinline__ void fma_bf16x2(float &acc, uint32_t w, uint32_t x) {
   asm("fma.rn.f32.bf16 %0, %1, %2, %0;" : "+f"(acc) : "h"(wh), "h"(xh));
 }
 
-template <int BP, int B1, int B2>
+template <int BP, int B1, int B2, bool LR = false>
 struct TmaCfg {
-  // rows per consumer warp: 8, or 16 for wide batches so that the 17-warp
-  // register budget (96 per thread) is not exceeded by the accumulators
+  // rows per consumer warp: 8, or 16 for wide batches so that the
+  // accumulators of a warp fit the register budget
   static constexpr int RW = BP >= 8 ? 16 : 8;
   static constexpr int NC = B1 / RW;                // consumer warps
   static constexpr int CPR = B2 / 16;               // lanes per row, 16 columns each
@@ -495,7 +346,10 @@ struct TmaCfg {
   static constexpr int kStageBytes = kValsBytes + kMetaBytes + kXRegion;
   static constexpr int kStages =
       (200 * 1024 / kStageBytes) < 6 ? (200 * 1024 / kStageBytes) : 6;
-  static constexpr int kThreads = (NC + 3) * 32;  // consumers, producer, 2 epilogue warps
+  // consumers, producer, 2 epilogue warps (and, in the instances for calls
+  // with a low-rank term, the low-rank warp: the others carry none of its
+  // code)
+  static constexpr int kThreads = (NC + 3 + (LR ? 1 : 0)) * 32;
   static constexpr size_t kSmem = (size_t)kStages * kStageBytes + 1024;
   static_assert(RPS * CPR == 32 && JS * RPS == RW && JS >= 1, "tile shape");
   static_assert(kStages >= 3, "ring too short");
@@ -535,16 +389,98 @@ struct StageDesc {
   uint8_t flags;    // 1: last stage of this CTA's piece of a band, 2: end of work
 };
 
-template <int BP, int B1, int B2>
-__global__ void __launch_bounds__(TmaCfg<BP, B1, B2>::kThreads, 1)
-    hybrid_tma_kernel(const Params p, const LaunchPlan lp, const __grid_constant__ CUtensorMap xmap) {
-  using C = TmaCfg<BP, B1, B2>;
+// U t for up to `rows` rows of a U chunk in shared memory (rows of r bf16),
+// CPL = r / 8 lanes per row, 32 / CPL rows side by side, one batch column at
+// a time.  Each lane adds its 16-byte chunk's products for CPL rows of its
+// group, then a butterfly over the group's lanes (halving the rows at each
+// step: CPL - 1 shuffles) leaves lane c of the group with the whole dot
+// product of the group's row c, which it stores (consecutive lanes,
+// consecutive rows).  The sum over the lanes has a fixed order.  tv holds
+// the lane's 8 columns of t for LB batch columns.  ut: the chunk's first
+// output row (row stride 1, batch stride n).
+template <int CPL, int LB>
+__device__ __forceinline__ bool ut_block(const uint8_t *src, int rows, int r,
+                                         const float (&tv)[LB][8], int lane, float *ut, int64_t n,
+                                         int b0) {
+  constexpr int RG = 32 / CPL;
+  const int g = lane / CPL, c = lane % CPL;
+  for (int blk = 0; blk < rows; blk += RG * CPL) {
+#pragma unroll
+    for (int b = 0; b < LB; ++b) {
+      float v[CPL];
+#pragma unroll
+      for (int i = 0; i < CPL; ++i) {
+        const int row = blk + g * CPL + i;
+        float part = 0.f;
+        if (row < rows) {
+          const uint4 u = *reinterpret_cast<const uint4 *>(src + (size_t)row * r * 2 + 16 * c);
+          part = fmaf(bf16_lo(u.x), tv[b][0], part);
+          part = fmaf(bf16_hi(u.x), tv[b][1], part);
+          part = fmaf(bf16_lo(u.y), tv[b][2], part);
+          part = fmaf(bf16_hi(u.y), tv[b][3], part);
+          part = fmaf(bf16_lo(u.z), tv[b][4], part);
+          part = fmaf(bf16_hi(u.z), tv[b][5], part);
+          part = fmaf(bf16_lo(u.w), tv[b][6], part);
+          part = fmaf(bf16_hi(u.w), tv[b][7], part);
+        }
+        v[i] = part;
+      }
+      // butterfly: at stride s a lane keeps the half of its 2s rows whose
+      // index has bit s equal to its own and adds its partner's copy of them
+#pragma unroll
+      for (int s = CPL / 2; s >= 1; s /= 2) {
+        const bool hi = (c & s) != 0;
+#pragma unroll
+        for (int i = 0; i < s; ++i) {
+          const float send = hi ? v[i] : v[i + s];
+          const float keep = hi ? v[i + s] : v[i];
+          v[i] = keep + __shfl_xor_sync(0xffffffffu, send, s);
+        }
+      }
+      const int row = blk + g * CPL + c;
+      if (row < rows) __stcg(ut + (int64_t)(b0 + b) * n + row, v[0]);
+    }
+  }
+  return true;
+}
+
+// Selectors of a 4:8 mask byte for the two-PRMT x pairs of the consumers:
+// x[c0], x[c1] through T = PRMT(X0, X1, s1) and PRMT(T, X2, s2); x[c2], x[c3]
+// through T' = PRMT(X2, X3, s3) and PRMT(X1, T', s4).  Entry .x = s1 | s2 << 16,
+// .y = s3 | s4 << 16; 0 for a byte without exactly four bits set.
+__device__ __forceinline__ uint2 lut48_entry(uint32_t m) {
+  if (__popc(m) != 4) return make_uint2(0u, 0u);
+  int c[4], n = 0;
+  for (int i = 0; i < 8; ++i)
+    if ((m >> i) & 1u) c[n++] = i;
+  auto pair = [](int lo, int hi) -> uint32_t {  // nibbles of the bytes lo, lo+1, hi, hi+1
+    return (uint32_t)lo | (uint32_t)(lo + 1) << 4 | (uint32_t)hi << 8 | (uint32_t)(hi + 1) << 12;
+  };
+  // T: x[c0], x[c1] from X0:X1 when below column 4 (bytes 2c, 2c+1)
+  const uint32_t s1 = pair(c[0] < 4 ? 2 * c[0] : 0, c[1] < 4 ? 2 * c[1] : 0);
+  // pair A from T (bytes 0..3) or X2 (bytes 4..7 hold x4, x5)
+  const uint32_t s2 = pair(c[0] < 4 ? 0 : 4 + 2 * (c[0] - 4), c[1] < 4 ? 2 : 4 + 2 * (c[1] - 4));
+  // T': x[c2], x[c3] from X2:X3 when at or above column 4
+  const uint32_t s3 = pair(c[2] >= 4 ? 2 * (c[2] - 4) : 0, c[3] >= 4 ? 2 * (c[3] - 4) : 0);
+  // pair B from X1 (bytes 0..3 hold x2, x3) or T' (bytes 4..7)
+  const uint32_t s4 = pair(c[2] < 4 ? 2 * (c[2] - 2) : 4, c[3] < 4 ? 2 * (c[3] - 2) : 6);
+  return make_uint2(s1 | s2 << 16, s3 | s4 << 16);
+}
+
+// PAT 0: 2:4 tiles (hyb_pack); PAT 1: 4:8 tiles (hyb_pack_nm with 4 of 8).
+// LR: the instance for calls with a low-rank term (an extra warp computes it).
+template <int BP, int B1, int B2, int PAT, bool LR>
+__global__ void __launch_bounds__(TmaCfg<BP, B1, B2, LR>::kThreads, 1)
+    hybrid_tma_kernel(const Params p, const LaunchPlan lp, const __grid_constant__ CUtensorMap xmap,
+                      const __grid_constant__ CUtensorMap wmap) {
+  using C = TmaCfg<BP, B1, B2, LR>;
   constexpr int S = C::kStages;
   extern __shared__ __align__(1024) uint8_t smem[];
   __shared__ __align__(8) uint64_t full_bar[S];
   __shared__ __align__(8) uint64_t empty_bar[S];
   __shared__ StageDesc desc[S];
   __shared__ uint32_t sel_lut[16];
+  __shared__ uint2 lut48[PAT == 1 ? 256 : 1];
   __shared__ uint32_t s_cnt[2];
   __shared__ int64_t s_range[2];
   // a CTA's piece of a band: row sums handed from the consumer warps to the
@@ -552,26 +488,25 @@ __global__ void __launch_bounds__(TmaCfg<BP, B1, B2>::kThreads, 1)
   __shared__ float s_rows[2][C::NC][C::RW * BP];
   __shared__ __align__(8) uint64_t piece_full[2];
   __shared__ __align__(8) uint64_t piece_empty[2];
+  // the low-rank warp's U t is complete (or its wait ran out, which it
+  // records in the status word)
+  __shared__ __align__(8) uint64_t lr_done;
 
   const int tid = threadIdx.x;
   const int warp = tid >> 5, lane = tid & 31;
   const int c = blockIdx.x;
   const int G = p.G;
   const int tpr = (int)p.tpr;
-  // The plan record is read first thing and parked in shared memory before
-  // the first barrier, so that its constant-bank line is fetched while the
-  // barriers are set up rather than when the producer first needs it.
   __shared__ int64_t s_rec[5];
   const bool planned = lp.kind == kPlanTiles;
+  // With a plan, or a row-major W, the CTA's range needs no search.  Then the
+  // producer warp sets up the mbarriers itself, signals the other warps with
+  // a non-blocking arrive on named barrier 1 and goes straight on to request
+  // its first ring of stages; the other warps wait on that barrier.  (Without
+  // a plan every thread takes part in the search, behind __syncthreads.)
+  const bool fast = planned || p.rowmajor;
   if (p.pdl) grid_dep_trigger();
-  if (planned && tid == 32 * C::NC + 1) {
-    s_rec[0] = lp.rec[4 * c];
-    s_rec[1] = lp.rec[4 * (c + 1)];
-    s_rec[2] = lp.rec[4 * c + 1];
-    s_rec[3] = lp.rec[4 * c + 2];
-    s_rec[4] = lp.rec[4 * c + 3];
-  }
-  if (tid == 0) {
+  auto init_barriers = [&]() {
     for (int s = 0; s < S; ++s) {
       mbar_init(&full_bar[s], 1);
       mbar_init(&empty_bar[s], C::NC);
@@ -580,29 +515,63 @@ __global__ void __launch_bounds__(TmaCfg<BP, B1, B2>::kThreads, 1)
       mbar_init(&piece_full[s], C::NC);
       mbar_init(&piece_empty[s], 1);
     }
+    mbar_init(&lr_done, 1);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-    s_cnt[0] = 0;
-    s_cnt[1] = 0;
-  }
-  if (tid < 16) {
-    // PRMT selector moving bf16 x[p0] to the low and x[p1] to the high half,
-    // p0 < p1 the set bits of the mask (x0x1 in bytes 0-3, x2x3 in 4-7)
-    const uint32_t m = tid;
-    uint32_t p0 = 0, p1 = 0;
-    if (m) {
-      p0 = __ffs(m) - 1;
-      p1 = 31 - __clz(m);
+  };
+  if (fast && warp == C::NC) {
+    if (lane == 0) {
+      init_barriers();
+      if (planned) {
+        s_rec[0] = lp.rec[4 * c];
+        s_rec[1] = lp.rec[4 * (c + 1)];
+        s_rec[2] = lp.rec[4 * c + 1];
+        s_rec[3] = lp.rec[4 * c + 2];
+        s_rec[4] = lp.rec[4 * c + 3];
+      } else {
+        // every tile costs the same: CTA c takes tiles [ceil(c T / G), ceil((c+1) T / G))
+        s_range[0] = ((int64_t)c * p.T + G - 1) / G;
+        s_range[1] = ((int64_t)(c + 1) * p.T + G - 1) / G;
+      }
     }
-    sel_lut[m] = (2 * p0) | ((2 * p0 + 1) << 4) | ((2 * p1) << 8) | ((2 * p1 + 1) << 12);
+    __syncwarp();
+    asm volatile("bar.arrive 1, %0;" ::"r"(C::kThreads) : "memory");
+  } else {
+    if (tid == 0 && !fast) {
+      init_barriers();
+      s_cnt[0] = 0;
+      s_cnt[1] = 0;
+      if (planned) {  // (a plan always takes the fast path; kept for robustness)
+        s_rec[0] = lp.rec[4 * c];
+        s_rec[1] = lp.rec[4 * (c + 1)];
+        s_rec[2] = lp.rec[4 * c + 1];
+        s_rec[3] = lp.rec[4 * c + 2];
+        s_rec[4] = lp.rec[4 * c + 3];
+      }
+    }
+    if (tid < 16) {
+      // PRMT selector moving bf16 x[p0] to the low and x[p1] to the high half,
+      // p0 < p1 the set bits of the mask (x0x1 in bytes 0-3, x2x3 in 4-7)
+      const uint32_t m = tid;
+      uint32_t p0 = 0, p1 = 0;
+      if (m) {
+        p0 = __ffs(m) - 1;
+        p1 = 31 - __clz(m);
+      }
+      sel_lut[m] = (2 * p0) | ((2 * p0 + 1) << 4) | ((2 * p1) << 8) | ((2 * p1 + 1) << 12);
+    }
+    if constexpr (PAT == 1) {
+      for (int m = tid; m < 256; m += blockDim.x) lut48[m] = lut48_entry((uint32_t)m);
+    }
+    if (fast) asm volatile("bar.sync 1, %0;" ::"r"(C::kThreads) : "memory");
   }
-  __syncthreads();
+  if (!fast) __syncthreads();
 
   // ---- this CTA's tiles [t0, t1): tiles whose packed offset P(t) satisfies
   // c*total <= P(t)*G < (c+1)*total.  With a plan the producer and the
-  // epilogue warp take them from the launch parameters; otherwise round 1
-  // brackets both ends between band starts and round 2 counts inside the
-  // bracketing band. ----
-  if (!planned) {
+  // epilogue warp take them from the launch parameters; a row-major W has
+  // them in closed form; otherwise round 1 brackets both ends between band
+  // starts and round 2 counts inside the bracketing band. ----
+  if (!fast && !planned) {
       const int64_t tgtA = (int64_t)c * p.total, tgtB = (int64_t)(c + 1) * p.total;
       uint32_t ca = 0, cb = 0;
       for (int i = tid; i <= p.R; i += blockDim.x) {
@@ -618,7 +587,9 @@ __global__ void __launch_bounds__(TmaCfg<BP, B1, B2>::kThreads, 1)
         atomicAdd(&s_cnt[1], cb);
       }
       __syncthreads();
-      const uint32_t bA = s_cnt[0], bB = s_cnt[1];  // band starts below each target
+      // band starts below each target (at most R: the bracketing band is a
+      // real one even when a corrupted matrix puts the end below a target)
+      const uint32_t bA = min(s_cnt[0], (uint32_t)p.R), bB = min(s_cnt[1], (uint32_t)p.R);
       __syncthreads();
       if (tid == 0) {
         s_cnt[0] = 0;
@@ -671,6 +642,9 @@ __global__ void __launch_bounds__(TmaCfg<BP, B1, B2>::kThreads, 1)
         asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&xmap))
                      : "memory");
     }
+    if (p.rowmajor && lane == 1)
+      asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&wmap))
+                   : "memory");
     // Tiles are taken in windows of WIN: lane i holds the packed offsets of
     // tile w0 + i (and lane WIN those of the window's end), the next window
     // is loaded while this one is issued.  Stages are packed greedily inside
@@ -679,18 +653,24 @@ __global__ void __launch_bounds__(TmaCfg<BP, B1, B2>::kThreads, 1)
     // over the window's 2:4 bitmask, so all agree on the stage starts.
     struct Win {
       int64_t vo, mo;
-      uint32_t sp;
+      uint32_t sp;  // the tile's map byte (1: a 2:4 tile)
     };
     // (volatile loads: the compiler may not turn the window load that a
-    // plan makes unnecessary into a speculative load the first window waits on)
+    // plan makes unnecessary into a speculative load the first window waits
+    // on; and nothing here inspects the loaded values, so the next window's
+    // loads stay in flight while this one issues)
     auto load_win = [&](int64_t w0) -> Win {
       Win o{0, 0, 0};
       const int64_t t = w0 + lane;
+      if (p.rowmajor) {  // dense tiles, offsets in closed form, nothing to load
+        o.vo = t * ((int64_t)B1 * B2);
+        return o;
+      }
       if (lane <= C::WIN && t <= t1) {
         o.vo = ld_volatile_nc64(p.val_off + t);
         o.mo = ld_volatile_nc64(p.meta_off + t);
       }
-      if (lane < C::WIN && t < t1) o.sp = ld_volatile_nc8(p.map + t) == 1;
+      if (lane < C::WIN && t < t1) o.sp = ld_volatile_nc8(p.map + t);
       return o;
     };
     int stage = 0;
@@ -748,7 +728,18 @@ __global__ void __launch_bounds__(TmaCfg<BP, B1, B2>::kThreads, 1)
     for (int64_t w0 = t0; ok && w0 < t1; w0 += C::WIN) {
       const Win nxt = load_win(w0 + C::WIN);  // in flight while this window issues
       const int nw = (int)min((int64_t)C::WIN, t1 - w0);
-      const uint32_t spm = __ballot_sync(0xffffffffu, cur.sp != 0);
+      const uint32_t spm = __ballot_sync(0xffffffffu, cur.sp == 1u);
+      if (!p.rowmajor && !(derived && w0 == t0)) {
+        // offsets read from the matrix must step by each tile's size (a
+        // corrupted matrix is flagged; the copies are bounded either way)
+        constexpr int64_t TE = (int64_t)B1 * B2;
+        const int64_t nvo = __shfl_down_sync(0xffffffffu, cur.vo, 1);
+        const int64_t nmo = __shfl_down_sync(0xffffffffu, cur.mo, 1);
+        const bool sp = cur.sp == 1u;
+        const bool bad = lane < nw && (nvo - cur.vo != (sp ? TE / 2 : TE) ||
+                                       nmo - cur.mo != (sp ? TE / 8 : 0));
+        if (__any_sync(0xffffffffu, bad) && lane == 0) atomicOr(p.status, kStatusBadMap);
+      }
       // stage starts: the plan's for the first window (checked against the
       // stage limits lane by lane), else the greedy packing
       uint32_t starts = 0;
@@ -765,44 +756,70 @@ __global__ void __launch_bounds__(TmaCfg<BP, B1, B2>::kThreads, 1)
         have = __all_sync(0xffffffffu, good && band_ok) && (starts & 1u) && (starts >> nw) == 0;
       }
       if (!have) starts = stage_starts(spm, nw, w0, tpr, C::TPD, C::TPX);
-      // the stage that starts at this lane: tiles [w0 + lane, w0 + e)
+      // the stage that starts at this lane: tiles [w0 + lane, w0 + e).  Every
+      // start lane works out its stage here, all at once, so that the serial
+      // part below (one stage after the other, as ring slots free up) only
+      // waits and issues.
       const bool is_start = lane < nw && (starts >> lane & 1u);
       const uint32_t later = lane < 31 ? (starts >> (lane + 1)) : 0u;
       const int e = later ? lane + 1 + __ffs(later) - 1 : nw;
       const int64_t v_end = __shfl_sync(0xffffffffu, cur.vo, e & 31);
       const int64_t m_end = __shfl_sync(0xffffffffu, cur.mo, e & 31);
       // (e == 32 only when nw == 32, which WIN < 32 rules out)
+      const int nt = e - lane;
+      const int64_t ts = w0 + lane, te = w0 + e;
+      // the stage's byte ranges, from the tile offsets: a range that does not
+      // fit the buffers, the stage or 16-byte alignment (a corrupted matrix)
+      // is not copied and is flagged; the consumers then read stale stage
+      // bytes, never outside the stage
+      const int64_t vb = 2 * (v_end - cur.vo), mb = m_end - cur.mo;
+      const bool fits = p.rowmajor || (cur.vo >= 0 && cur.mo >= 0 && vb > 0 && mb >= 0 &&
+                                       vb <= C::kValsBytes && mb <= C::kMetaBytes &&
+                                       2 * cur.vo + vb <= p.nvb && cur.mo + mb <= p.nmb &&
+                                       ((2 * cur.vo) | vb | cur.mo | mb) % 16 == 0);
+      if (__any_sync(0xffffffffu, is_start && !fits) && lane == 0) atomicOr(p.status, kStatusBadMap);
+      const uint32_t vbytes = fits ? (uint32_t)vb : 0u;
+      const uint32_t mbytes = fits ? (uint32_t)mb : 0u;
+      const int ngx = (nt + C::XT - 1) / C::XT;  // X copy groups (tensor path)
+      const uint32_t xbytes =
+          C::XTM ? (uint32_t)(ngx * C::kXCopy) : (uint32_t)(2 * B2 * nt) * (uint32_t)p.batch;
+      const int64_t band = w0 / tpr + (lane + (int)(w0 % tpr)) / tpr;  // = ts / tpr
+      StageDesc dl;
+      dl.t0 = ts;
+      dl.ntiles = (uint16_t)nt;
+      dl.sparse = (uint8_t)((spm >> lane) & ((1u << (nt & 31)) - 1u));
+      dl.flags = (te == (band + 1) * tpr || te == t1) ? 1 : 0;
+      const int64_t xcol = (ts - band * tpr) * B2;  // first X column of the stage
       uint32_t todo = starts;
       while (todo) {
         const int k = __ffs(todo) - 1;
         todo &= todo - 1;
-        if (pend && issued == S) release_x();  // the ring is armed: X can wait no longer
+        if (pend && issued == p.nst) release_x();  // the ring is armed: X can wait no longer
         if (lane == k && is_start) {
           if (!mbar_wait(&empty_bar[stage], phase ^ 1u)) {
             ok = false;
           } else {
             uint8_t *st = smem + (size_t)stage * C::kStageBytes;
-            const int64_t ts = w0 + k, te = w0 + e;
-            const uint32_t vbytes = (uint32_t)(2 * (v_end - cur.vo));
-            const uint32_t mbytes = (uint32_t)(m_end - cur.mo);
-            const int nt = e - k;
-            const uint32_t xrow = (uint32_t)(2 * B2 * nt);
-            const int ngx = (nt + C::XT - 1) / C::XT;  // X copy groups (tensor path)
-            const uint32_t xbytes =
-                C::XTM ? (uint32_t)(ngx * C::kXCopy) : xrow * (uint32_t)p.batch;
-            const int64_t band = ts / tpr;
-            StageDesc d;
-            d.t0 = ts;
-            d.ntiles = (uint16_t)nt;
-            d.sparse = (uint8_t)((spm >> k) & ((1u << nt) - 1u));
-            d.flags = (te == (band + 1) * tpr || te == t1) ? 1 : 0;
-            desc[stage] = d;
+            desc[stage] = dl;
             armed |= 1u << stage;
             armed_parity = (armed_parity & ~(1u << stage)) | (phase << stage);
             mbar_arrive_expect_tx(&full_bar[stage], vbytes + mbytes + xbytes);
-            bulk_g2s(st, p.vals + 2 * cur.vo, vbytes, &full_bar[stage]);
-            if (mbytes) bulk_g2s(st + C::kValsBytes, p.meta + cur.mo, mbytes, &full_bar[stage]);
-            const int64_t xcol = (ts - band * tpr) * B2;  // first X column of the stage
+            if (p.rowmajor) {
+              // one 2-D tensor copy per tile: box [B1 rows][B2 columns] of W,
+              // which lands in the packed dense tile layout
+              int64_t tr = band, tc = ts - band * tpr;
+              for (int q = 0; q < nt; ++q) {
+                tma_load_2d(st + (size_t)q * 2 * B1 * B2, &wmap, (int)(tc * B2), (int)(tr * B1),
+                            &full_bar[stage]);
+                if (++tc == tpr) {
+                  tc = 0;
+                  ++tr;
+                }
+              }
+            } else {
+              if (vbytes) bulk_g2s(st, p.vals + 2 * cur.vo, vbytes, &full_bar[stage]);
+              if (mbytes) bulk_g2s(st + C::kValsBytes, p.meta + cur.mo, mbytes, &full_bar[stage]);
+            }
             if (pend) {
               dx_stage = stage;
               dx_col = xcol;
@@ -814,7 +831,7 @@ __global__ void __launch_bounds__(TmaCfg<BP, B1, B2>::kThreads, 1)
         }
         // every lane keeps the ring position
         ++issued;
-        if (++stage == S) {
+        if (++stage == p.nst) {
           stage = 0;
           phase ^= 1u;
         }
@@ -846,7 +863,238 @@ __global__ void __launch_bounds__(TmaCfg<BP, B1, B2>::kThreads, 1)
     return;
   }
 
-  if (warp >= C::NC + 1) {
+  if (LR && warp == C::NC + 3) {
+    // ------------------------------ low rank ------------------------------
+    // The L = U V^T term of "3BASiL" (§1: W ~ S + L), fused into the pass:
+    // (1) a partial t = V^T x over this CTA's slice of V's rows; (2) once
+    // every CTA has written its partial, elements [E c / G, E (c+1) / G) of
+    // t, each the sum of the G partials in CTA order; (3) once t is whole,
+    // U t for this CTA's slice of the output rows.  A grid barrier separates
+    // the steps; the epilogue warps wait for the last one (lr_done) before
+    // their first final store, and add U t there.  The V and U rows (and the
+    // X slice) come in by bulk copies into two 8 KB halves of a buffer after
+    // the ring, one chunk in flight while the other is used.  Every sum has a
+    // fixed order, so results do not depend on timing.
+    if (!p.fused_lr) return;
+    if (p.pdl) grid_dep_wait();  // X and the workspace may belong to the preceding grid
+    constexpr int LB = BP < 4 ? BP : 4;  // batch columns per pass
+    const uint32_t full = 0xffffffffu;
+    const int r = p.rank;
+    const int cpl = r / 8;                          // 16-byte chunks of a V or U row
+    const int rg = (32 % cpl == 0) ? 32 / cpl : 1;  // rows handled side by side
+    const int chunk = lane % cpl, rgrp = lane / cpl;
+    const bool active = lane < cpl * rg;
+    const int64_t E = (int64_t)BP * r;  // elements of t (padded batch)
+    uint8_t *lrbuf = smem + (size_t)p.nst * C::kStageBytes;
+    bool ok = true;
+    // this call's barrier epoch (every CTA reads it before its first arrival;
+    // CTA 0 advances it after the last barrier)
+    const uint32_t epoch = __shfl_sync(full, lane == 0 ? ld_acquire_u32(p.lr_epoch) : 0u, 0);
+    // Copy chunks [0, nch) through the two halves, calling use(j, half) on
+    // each once it has landed; issue(j, half) has every lane request its
+    // 16-byte pieces of chunk j.  Two chunks in flight, one commit group each.
+    auto pipeline = [&](int nch, auto &&issue, auto &&use) {
+      if (nch > 0) issue(0, lrbuf);
+      cp_async_commit();
+      if (nch > 1) issue(1, lrbuf + kLrHalf);
+      cp_async_commit();
+      for (int j = 0; j < nch; ++j) {
+        cp_async_wait<1>();  // chunk j has landed (at most chunk j + 1 pending)
+        __syncwarp();
+        use(j, lrbuf + (j & 1) * kLrHalf);
+        __syncwarp();
+        if (j + 2 < nch) issue(j + 2, lrbuf + (j & 1) * kLrHalf);
+        cp_async_commit();
+      }
+      cp_async_wait<0>();
+      __syncwarp();
+    };
+    // lanes copy `bytes` contiguous bytes (a multiple of 16) in 16-byte pieces
+    auto copy_span = [&](uint8_t *dst, const void *src, uint32_t bytes) {
+      const uint8_t *g = reinterpret_cast<const uint8_t *>(src);
+      for (uint32_t o = 16u * lane; o < bytes; o += 512u) cp_async16(dst + o, g + o);
+    };
+    // (1) partial t over rows [k0, k1) of V, multiples of 8 so that the X
+    // rows' copies start on 16-byte boundaries; a chunk holds rc rows of V
+    // and the same rows of X for four batch columns
+    {
+      const int64_t k8 = p.k / 8;
+      const int64_t k0 = 8 * (k8 * c / G), k1 = 8 * (k8 * (c + 1) / G);
+      const int rc = max(8, (kLrHalf / (2 * r + 2 * 4)) / 8 * 8);
+      const int nch = (int)((k1 - k0 + rc - 1) / rc);
+      float *mine = p.lr_part + (int64_t)c * E;
+#pragma unroll 1
+      for (int b0 = 0; b0 < BP && ok; b0 += 4) {
+        const int nb = min(4, p.batch - b0);  // batch rows of X in this pass (<= 0: none)
+        float acc[4][8];
+#pragma unroll
+        for (int b = 0; b < 4; ++b)
+#pragma unroll
+          for (int e = 0; e < 8; ++e) acc[b][e] = 0.f;
+        auto issue = [&](int j, uint8_t *dst) {
+          const int64_t row0 = k0 + (int64_t)j * rc;
+          const int rows = (int)min((int64_t)rc, k1 - row0);
+          const uint32_t vb = (uint32_t)rows * r * 2, xb = (uint32_t)rows * 2;
+          if (p.ldv == r)
+            copy_span(dst, p.V + row0 * p.ldv, vb);
+          else
+            for (int i = 0; i < rows; ++i)
+              copy_span(dst + (size_t)i * r * 2, p.V + (row0 + i) * p.ldv, (uint32_t)r * 2);
+          for (int b = 0; b < nb; ++b)
+            copy_span(dst + (size_t)rc * r * 2 + (size_t)b * rc * 2,
+                      p.X + (int64_t)(b0 + b) * p.ldx + row0, xb);
+        };
+        auto use = [&](int j, const uint8_t *src) {
+          const int64_t row0 = k0 + (int64_t)j * rc;
+          const int rows = (int)min((int64_t)rc, k1 - row0);
+          if (!active) return;
+          const uint16_t *xsm = reinterpret_cast<const uint16_t *>(src + (size_t)rc * r * 2);
+          for (int i = rgrp; i < rows; i += rg) {
+            const uint4 v = *reinterpret_cast<const uint4 *>(src + (size_t)i * r * 2 + 16 * chunk);
+            const float vf[8] = {bf16_lo(v.x), bf16_hi(v.x), bf16_lo(v.y), bf16_hi(v.y),
+                                 bf16_lo(v.z), bf16_hi(v.z), bf16_lo(v.w), bf16_hi(v.w)};
+#pragma unroll
+            for (int b = 0; b < 4; ++b) {
+              if (b < nb) {
+                const float xv = __uint_as_float((uint32_t)xsm[b * rc + i] << 16);
+#pragma unroll
+                for (int e = 0; e < 8; ++e) acc[b][e] = fmaf(vf[e], xv, acc[b][e]);
+              }
+            }
+          }
+        };
+        if (nb > 0) pipeline(nch, issue, use);
+        if (rg > 1) {  // lanes chunk + cpl g hold the same columns: a fixed xor tree
+#pragma unroll 1
+          for (int o = cpl; o < 32; o <<= 1)
+#pragma unroll
+            for (int b = 0; b < 4; ++b)
+#pragma unroll
+              for (int e = 0; e < 8; ++e) acc[b][e] += __shfl_xor_sync(full, acc[b][e], o);
+        }
+        if (active && rgrp == 0) {
+#pragma unroll
+          for (int b = 0; b < 4; ++b)
+            if (b0 + b < BP)
+#pragma unroll
+              for (int e = 0; e < 8; ++e) __stcg(mine + (b0 + b) * r + 8 * chunk + e, acc[b][e]);
+        }
+      }
+    }
+    __syncwarp();
+    if (ok) ok = flag_barrier(p.lr_flags, G, c, epoch + 1u, lane);
+    if (ok) {
+      // 8 lanes per element, each adding the partials of CTAs sub, sub + 8,
+      // ... in order (all loads issued first); the 8 sums then combined by a
+      // fixed xor tree
+      const int64_t e0 = E * c / G, e1 = E * (c + 1) / G;
+      const int sub = lane % 8;
+      constexpr int QL = 10;  // partials per lane in flight (two rounds cover 160 CTAs)
+      for (int64_t eb = e0; eb < e1; eb += 4) {
+        const int64_t e = eb + lane / 8;
+        float a = 0.f;
+#pragma unroll 1
+        for (int q0 = 0; q0 < G; q0 += 8 * QL) {
+          float v[QL];
+#pragma unroll
+          for (int q = 0; q < QL; ++q) {
+            const int cq = q0 + sub + 8 * q;
+            v[q] = (e < e1 && cq < G) ? __ldcg(p.lr_part + (int64_t)cq * E + e) : 0.f;
+          }
+#pragma unroll
+          for (int q = 0; q < QL; ++q) a += v[q];
+        }
+        a += __shfl_xor_sync(full, a, 1);
+        a += __shfl_xor_sync(full, a, 2);
+        a += __shfl_xor_sync(full, a, 4);
+        if (e < e1 && sub == 0) __stcg(p.lr_t + e, a);
+      }
+      ok = flag_barrier(p.lr_flags, G, c, epoch + 2u, lane);
+    }
+    if (ok) {
+      // (3) U t for rows [i0, i1); a chunk holds rc3 rows of U
+      const int64_t i0 = p.n * c / G, i1 = p.n * (c + 1) / G;
+      const int rc3 = kLrHalf / (2 * r);
+      const int nch = (int)((i1 - i0 + rc3 - 1) / rc3);
+#pragma unroll 1
+      for (int b0 = 0; b0 < BP && ok; b0 += LB) {
+        float tv[LB][8];
+#pragma unroll
+        for (int b = 0; b < LB; ++b)
+#pragma unroll
+          for (int e = 0; e < 8; ++e)
+            tv[b][e] = active ? __ldcg(p.lr_t + (b0 + b) * r + 8 * chunk + e) : 0.f;
+        auto issue = [&](int j, uint8_t *dst) {
+          const int64_t row0 = i0 + (int64_t)j * rc3;
+          const int rows = (int)min((int64_t)rc3, i1 - row0);
+          if (p.ldu == r)
+            copy_span(dst, p.U + row0 * p.ldu, (uint32_t)rows * r * 2);
+          else
+            for (int i = 0; i < rows; ++i)
+              copy_span(dst + (size_t)i * r * 2, p.U + (row0 + i) * p.ldu, (uint32_t)r * 2);
+        };
+        auto use = [&](int j, const uint8_t *src) {
+          const int64_t row0 = i0 + (int64_t)j * rc3;
+          const int rows = (int)min((int64_t)rc3, i1 - row0);
+          // 16-byte chunks of a row per lane: 4 to 16 (ranks 32 to 128) take
+          // rows a block at a time and a butterfly over the lanes of a row
+          // (ut_block); other ranks one row per lane group and a shuffle sum
+          bool done = false;
+          switch (cpl) {
+            case 4: done = ut_block<4, LB>(src, rows, r, tv, lane, p.lr_ut + row0, p.n, b0); break;
+            case 8: done = ut_block<8, LB>(src, rows, r, tv, lane, p.lr_ut + row0, p.n, b0); break;
+            case 16: done = ut_block<16, LB>(src, rows, r, tv, lane, p.lr_ut + row0, p.n, b0); break;
+            default: break;
+          }
+          if (done) return;
+          for (int ib = 0; ib < rows; ib += rg) {
+            const int i = ib + rgrp;
+            float part[LB];
+#pragma unroll
+            for (int b = 0; b < LB; ++b) part[b] = 0.f;
+            if (active && i < rows) {
+              const uint4 u = *reinterpret_cast<const uint4 *>(src + (size_t)i * r * 2 + 16 * chunk);
+              const float uf[8] = {bf16_lo(u.x), bf16_hi(u.x), bf16_lo(u.y), bf16_hi(u.y),
+                                   bf16_lo(u.z), bf16_hi(u.z), bf16_lo(u.w), bf16_hi(u.w)};
+#pragma unroll
+              for (int b = 0; b < LB; ++b)
+#pragma unroll
+                for (int e = 0; e < 8; ++e) part[b] = fmaf(uf[e], tv[b][e], part[b]);
+            }
+            // the row's cpl lanes: a fixed xor tree, or (cpl not a power of
+            // two, lanes 0 .. cpl-1) a sum in lane order
+#pragma unroll
+            for (int b = 0; b < LB; ++b) {
+              if (rg > 1 || (cpl & (cpl - 1)) == 0) {
+                for (int o = 1; o < cpl; o <<= 1) part[b] += __shfl_xor_sync(full, part[b], o);
+              } else {
+                float t = 0.f;
+                for (int q = 0; q < cpl; ++q) t += __shfl_sync(full, part[b], q);
+                part[b] = t;
+              }
+            }
+            if (active && i < rows && chunk == 0) {
+#pragma unroll
+              for (int b = 0; b < LB; ++b)
+                __stcg(p.lr_ut + (int64_t)(b0 + b) * p.n + row0 + i, part[b]);
+            }
+          }
+        };
+        pipeline(nch, issue, use);
+      }
+      __syncwarp();
+      if (ok) ok = flag_barrier(p.lr_flags, G, c, epoch + 3u, lane);
+      // the next call's epoch: every CTA has read this one (they all arrived)
+      if (ok && c == 0 && lane == 0) st_release_u32(p.lr_epoch, epoch + 3u);
+    }
+    if (lane == 0) {
+      if (!ok) atomicOr(p.status, kStatusTimeout);
+      mbar_arrive(&lr_done);
+    }
+    return;
+  }
+
+  if (warp == C::NC + 1 || warp == C::NC + 2) {
     // ------------------------------ epilogue ------------------------------
     // Takes every piece of band this CTA finishes, in band order, pieces
     // alternating between the two epilogue warps so that one piece's ticket
@@ -858,12 +1106,21 @@ __global__ void __launch_bounds__(TmaCfg<BP, B1, B2>::kThreads, 1)
     // Y, the slots, the tickets and the low-rank term may belong to the
     // preceding grid until it has finished.
     if (p.pdl) grid_dep_wait();
+    // (clamped to [0, G): offsets of a corrupted matrix never index slots
+    // outside the workspace)
     auto owner_of_p = [&](int64_t P) -> int {
       const int64_t o = (P * G) / p.total;
-      return (int)(o < G - 1 ? o : G - 1);
+      return (int)(o < 0 ? 0 : (o < G - 1 ? o : G - 1));
     };
     constexpr int OPL = 4, QMAX = 8;  // outputs per lane, contributors per load round
     const int ew = warp - (C::NC + 1);
+    // the fused low-rank term must be complete before a final store adds it
+    bool lr_wait = LR && p.fused_lr != 0;
+    auto wait_lowrank = [&]() {
+      if (!lr_wait) return;
+      lr_wait = false;
+      if (!mbar_wait(&lr_done, 0u) && lane == 0) atomicOr(p.status, kStatusTimeout);
+    };
     const int r_first = (int)(t0 / tpr), r_last = t1 > t0 ? (int)((t1 - 1) / tpr) : r_first - 1;
     for (int r = r_first + ew; r <= r_last; r += 2) {
       const int piece = r - r_first;
@@ -874,8 +1131,13 @@ __global__ void __launch_bounds__(TmaCfg<BP, B1, B2>::kThreads, 1)
       int oA = 0, oB = 0;
       if (!whole && lane == 0) {
         const int64_t ta = (int64_t)r * tpr, tb = ta + tpr - 1;
-        oA = owner_of_p(2 * __ldg(p.val_off + ta) + __ldg(p.meta_off + ta));
-        oB = owner_of_p(2 * __ldg(p.val_off + tb) + __ldg(p.meta_off + tb));
+        if (p.rowmajor) {
+          oA = owner_of_p(ta * 2 * B1 * B2);
+          oB = owner_of_p(tb * 2 * B1 * B2);
+        } else {
+          oA = owner_of_p(2 * __ldg(p.val_off + ta) + __ldg(p.meta_off + ta));
+          oB = owner_of_p(2 * __ldg(p.val_off + tb) + __ldg(p.meta_off + tb));
+        }
       }
       if (!mbar_wait(&piece_full[slot], ph)) {
         if (lane == 0) atomicOr(p.status, kStatusTimeout);
@@ -884,6 +1146,7 @@ __global__ void __launch_bounds__(TmaCfg<BP, B1, B2>::kThreads, 1)
       const float(*rows)[C::RW * BP] = s_rows[slot];
       const int64_t row0 = (int64_t)r * B1;
       if (whole) {
+        wait_lowrank();
         for (int o = lane; o < B1 * BP; o += 32) {
           const int row = o % B1, b = o / B1;
           if (b < p.batch) store_out(p, row0 + row, b, rows[row / C::RW][b * C::RW + row % C::RW]);
@@ -906,6 +1169,7 @@ __global__ void __launch_bounds__(TmaCfg<BP, B1, B2>::kThreads, 1)
         oA = __shfl_sync(0xffffffffu, oA, 0);
         oB = __shfl_sync(0xffffffffu, oB, 0);
         if (last) {
+          wait_lowrank();
           __syncwarp();
           // sum the band's slots in CTA order; the loads of 4 outputs x 8
           // contributors are issued together, then added in a fixed order
@@ -970,9 +1234,9 @@ __global__ void __launch_bounds__(TmaCfg<BP, B1, B2>::kThreads, 1)
     int voff = 0, moff = 0;
     for (int i = 0; i < d.ntiles; ++i) {
       const bool sp = (d.sparse >> i) & 1;
-      // a lane covers columns [16cp, 16cp+16) of a 2:4 tile row, and columns
-      // [8cp, 8cp+8) + [B2/2 + 8cp, B2/2 + 8cp + 8) of a dense tile row (so
-      // that 8 lanes read 128 contiguous bytes of shared memory)
+      // a lane covers columns [16cp, 16cp+16) of a sparse tile row, and
+      // columns [8cp, 8cp+8) + [B2/2 + 8cp, B2/2 + 8cp + 8) of a dense tile
+      // row (so that 8 lanes read 128 contiguous bytes of shared memory)
       const uint8_t *xs = st + C::kValsBytes + C::kMetaBytes + (i / C::XT) * C::kXCopy +
                           (i % C::XT) * 2 * B2;
       const int xo0 = sp ? 32 * cp : 16 * cp;
@@ -984,8 +1248,14 @@ __global__ void __launch_bounds__(TmaCfg<BP, B1, B2>::kThreads, 1)
         for (int b = 0; b < C::XB; ++b) {
           const uint4 lo = *reinterpret_cast<const uint4 *>(xs + (b0 + b) * C::kXBatch + xo0);
           const uint4 hi = *reinterpret_cast<const uint4 *>(xs + (b0 + b) * C::kXBatch + xo1);
-          xr[b][0] = lo.x; xr[b][1] = lo.y; xr[b][2] = lo.z; xr[b][3] = lo.w;
-          xr[b][4] = hi.x; xr[b][5] = hi.y; xr[b][6] = hi.z; xr[b][7] = hi.w;
+          xr[b][0] = lo.x;
+          xr[b][1] = lo.y;
+          xr[b][2] = lo.z;
+          xr[b][3] = lo.w;
+          xr[b][4] = hi.x;
+          xr[b][5] = hi.y;
+          xr[b][6] = hi.z;
+          xr[b][7] = hi.w;
         }
         if (sp) {
 #pragma unroll
@@ -995,36 +1265,58 @@ __global__ void __launch_bounds__(TmaCfg<BP, B1, B2>::kThreads, 1)
             const uint32_t m = *reinterpret_cast<const uint16_t *>(
                 st + C::kValsBytes + moff + row * (B2 / 8) + 2 * cp);
             const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-            // PRMT selector of each group: (p0, p1) -- the lowest and highest
-            // kept column -- becomes bytes {2p0, 2p0+1, 2p1, 2p1+1} of the
-            // group's x quad.  Narrow batches, where a selector serves one or
-            // two products, build it in registers: one PRMT looks up (p0, p1)
-            // of two groups at once from a byte table indexed by the low three
-            // bits of each 4-bit mask (distinct for the six masks with two bits
-            // set), a second expands them to byte pairs.  Wide batches reuse a
-            // selector across four columns and take it from the shared table.
-            uint32_t selw[4];
-            if constexpr (BP <= 4) {
-              constexpr uint32_t kPairLo = 0x10313010u, kPairHi = 0x10212032u;
-              const uint32_t s01 = __byte_perm(kPairLo, kPairHi, m & 0x77u);
-              const uint32_t s23 = __byte_perm(kPairLo, kPairHi, (m >> 8) & 0x77u);
-              const uint32_t a01 = __byte_perm(0x76543210u, 0u, s01);
-              const uint32_t a23 = __byte_perm(0x76543210u, 0u, s23);
-              selw[0] = a01;
-              selw[1] = a01 >> 16;
-              selw[2] = a23;
-              selw[3] = a23 >> 16;
+            if constexpr (PAT == 1) {
+              // 4:8: two groups of 8 columns, 4 kept each (c0 < c1 < c2 <
+              // c3); (v0, v1) meet x[c0], x[c1] and (v2, v3) x[c2], x[c3].
+              // As c0 <= 4, c1 <= 5, c2 >= 2 and c3 >= 3, each x pair comes
+              // from three of the group's four x registers in two PRMTs,
+              // with selectors from the mask byte's lut48 entry.
+#pragma unroll
+              for (int gb = 0; gb < 2; ++gb) {
+                const uint2 sl = lut48[(m >> (8 * gb)) & 0xFFu];
+                const uint32_t s1 = sl.x, s2 = sl.x >> 16, s3 = sl.y, s4 = sl.y >> 16;
+#pragma unroll
+                for (int b = 0; b < C::XB; ++b) {
+                  const uint32_t *X4 = &xr[b][4 * gb];
+                  const uint32_t pa = __byte_perm(__byte_perm(X4[0], X4[1], s1), X4[2], s2);
+                  const uint32_t pb = __byte_perm(X4[1], __byte_perm(X4[2], X4[3], s3), s4);
+                  fma_bf16x2(acc[j][b0 + b], w[2 * gb], pa);
+                  fma_bf16x2(acc[j][b0 + b], w[2 * gb + 1], pb);
+                }
+              }
             } else {
+              // 2:4: the PRMT selector of each group moves x[p0] to the low
+              // and x[p1] to the high half (p0 < p1 the kept columns).
+              // Narrow batches, where a selector serves one to four products,
+              // build it in registers: one PRMT looks up (p0, p1) of two
+              // groups at once in a byte table indexed by the low three bits
+              // of each 4-bit mask (distinct for the six masks with two bits
+              // set), a second PRMT expands them to byte pairs.  Wide batches
+              // take it from a 16-entry shared table (one load serves eight or
+              // sixteen products).
+              uint32_t selw[4];
+              if constexpr (BP <= 4) {
+                constexpr uint32_t kPairLo = 0x10313010u, kPairHi = 0x10212032u;
+                const uint32_t s01 = __byte_perm(kPairLo, kPairHi, m & 0x77u);
+                const uint32_t s23 = __byte_perm(kPairLo, kPairHi, (m >> 8) & 0x77u);
+                const uint32_t a01 = __byte_perm(0x76543210u, 0u, s01);
+                const uint32_t a23 = __byte_perm(0x76543210u, 0u, s23);
+                selw[0] = a01;
+                selw[1] = a01 >> 16;
+                selw[2] = a23;
+                selw[3] = a23 >> 16;
+              } else {
 #pragma unroll
-              for (int g = 0; g < 4; ++g) selw[g] = sel_lut[(m >> (4 * g)) & 0xFu];
-            }
+                for (int g = 0; g < 4; ++g) selw[g] = sel_lut[(m >> (4 * g)) & 0xFu];
+              }
 #pragma unroll
-            for (int g = 0; g < 4; ++g) {
-              const uint32_t sel = selw[g];
+              for (int g = 0; g < 4; ++g) {
+                const uint32_t sel = selw[g];
 #pragma unroll
-              for (int b = 0; b < C::XB; ++b) {
-                const uint32_t xp = __byte_perm(xr[b][2 * g], xr[b][2 * g + 1], sel);
-                fma_bf16x2(acc[j][b0 + b], w[g], xp);
+                for (int b = 0; b < C::XB; ++b) {
+                  const uint32_t xp = __byte_perm(xr[b][2 * g], xr[b][2 * g + 1], sel);
+                  fma_bf16x2(acc[j][b0 + b], w[g], xp);
+                }
               }
             }
           }
@@ -1048,7 +1340,7 @@ __global__ void __launch_bounds__(TmaCfg<BP, B1, B2>::kThreads, 1)
     }
     __syncwarp();
     if (lane == 0) mbar_arrive(&empty_bar[stage]);
-    if (++stage == S) {
+    if (++stage == p.nst) {
       stage = 0;
       phase ^= 1u;
     }
@@ -1118,14 +1410,17 @@ __global__ void __launch_bounds__(128)
 }
 
 // ---------------------------------------------------------------------------
-// simple kernel for other legal tilings: one warp per output row
+// simple kernel for other legal tilings: one warp per output row.  A lane
+// takes 8-column chunks of the row (b2 is a multiple of 8): 16 bytes of a
+// dense tile row, or 4 kept values (8 bytes) and one mask byte (two groups)
+// of a 2:4 tile row, with the chunk's 8 x values.
 // ---------------------------------------------------------------------------
 template <int BP, bool STRIDED>
 __global__ void __launch_bounds__(kThreads)
     hybrid_rowwarp_kernel(const Params p, int b1, int b2) {
   const int lane = threadIdx.x & 31;
   const int64_t warps = (int64_t)gridDim.x * kWarps;
-  const int cpr = b2 / 16;  // 16-column chunks per tile row
+  const int cpr = b2 / 8;  // 8-column chunks per tile row
   for (int64_t row = (int64_t)blockIdx.x * kWarps + (threadIdx.x >> 5); row < p.n;
        row += warps) {
     const int64_t r = row / b1, i = row - r * b1;
@@ -1136,47 +1431,54 @@ __global__ void __launch_bounds__(kThreads)
       const int64_t tc = q / cpr;
       const int cpart = (int)(q - tc * cpr);
       const int64_t t = r * p.tpr + tc;
-      float xf[BP][16];
+      uint32_t xr[BP][4];
 #pragma unroll
       for (int b = 0; b < BP; ++b) {
         if (b < p.batch) {
-          const uint16_t *xp = p.X + (int64_t)b * p.ldx + tc * b2 + 16 * cpart;
-          unpack16(ld_keep16(xp), ld_keep16(xp + 8), xf[b]);
+          const uint4 xv = ld_keep16(p.X + (int64_t)b * p.ldx + tc * b2 + 8 * cpart);
+          xr[b][0] = xv.x;
+          xr[b][1] = xv.y;
+          xr[b][2] = xv.z;
+          xr[b][3] = xv.w;
         } else {
 #pragma unroll
-          for (int e = 0; e < 16; ++e) xf[b][e] = 0.f;
+          for (int e = 0; e < 4; ++e) xr[b][e] = 0u;
         }
       }
       const bool sparse = !STRIDED && __ldg(p.map + t) == 1;
       if (sparse) {
-        const uint8_t *vp =
-            p.vals + 2 * __ldg(p.val_off + t) + i * b2 + 16 * cpart;
-        const uint8_t *mp = p.meta + __ldg(p.meta_off + t) + i * (b2 / 8) + 2 * cpart;
-        const uint4 v = ld_stream16(vp);
-        const uint32_t m = ld_stream_u16(mp);
-        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+        // groups 2 cpart and 2 cpart + 1 of the row: kept values 4 cpart ..
+        // 4 cpart + 3, mask byte cpart
+        const uint8_t *vp = p.vals + 2 * __ldg(p.val_off + t) + i * b2 + 8 * cpart;
+        const uint8_t *mp = p.meta + __ldg(p.meta_off + t) + i * (b2 / 8) + cpart;
+        const uint2 v = ld_stream8(vp);
+        const uint32_t m = ld_stream_u8(mp);
+        const uint32_t w[2] = {v.x, v.y};
 #pragma unroll
-        for (int g = 0; g < 4; ++g) {
+        for (int g = 0; g < 2; ++g) {
           const uint32_t nib = (m >> (4 * g)) & 0xFu;
 #pragma unroll
           for (int b = 0; b < BP; ++b) {
             float xa, xb;
-            pick2(nib, xf[b][4 * g], xf[b][4 * g + 1], xf[b][4 * g + 2],
-                  xf[b][4 * g + 3], xa, xb);
+            pick2(nib, bf16_lo(xr[b][2 * g]), bf16_hi(xr[b][2 * g]), bf16_lo(xr[b][2 * g + 1]),
+                  bf16_hi(xr[b][2 * g + 1]), xa, xb);
             acc[b] = fmaf(bf16_lo(w[g]), xa, acc[b]);
             acc[b] = fmaf(bf16_hi(w[g]), xb, acc[b]);
           }
         }
       } else {
         const uint8_t *vp =
-            STRIDED ? reinterpret_cast<const uint8_t *>(p.Wd + row * p.ldw + tc * b2 + 16 * cpart)
-                    : p.vals + 2 * __ldg(p.val_off + t) + i * 2 * b2 + 32 * cpart;
-        float wf[16];
-        unpack16(ld_stream16(vp), ld_stream16(vp + 16), wf);
+            STRIDED ? reinterpret_cast<const uint8_t *>(p.Wd + row * p.ldw + tc * b2 + 8 * cpart)
+                    : p.vals + 2 * __ldg(p.val_off + t) + i * 2 * b2 + 16 * cpart;
+        const uint4 wv = ld_stream16(vp);
+        const uint32_t w[4] = {wv.x, wv.y, wv.z, wv.w};
 #pragma unroll
-        for (int e = 0; e < 16; ++e)
+        for (int e = 0; e < 4; ++e)
 #pragma unroll
-          for (int b = 0; b < BP; ++b) acc[b] = fmaf(wf[e], xf[b][e], acc[b]);
+          for (int b = 0; b < BP; ++b) {
+            acc[b] = fmaf(bf16_lo(w[e]), bf16_lo(xr[b][e]), acc[b]);
+            acc[b] = fmaf(bf16_hi(w[e]), bf16_hi(xr[b][e]), acc[b]);
+          }
       }
     }
 #pragma unroll
@@ -1411,67 +1713,59 @@ Shape shape_of(int b1, int b2) {
   return kGeneric;
 }
 
-template <int BP, int B1, int B2>
-void *dense_kernel_ptr() {
-  return reinterpret_cast<void *>(&dense_gemv_kernel<BP, B1, B2>);
-}
-
-void *pick_dense_kernel(int bp, Shape s) {
-#define HYB_CASE(BP_)                                                  \
-  case BP_:                                                            \
-    switch (s) {                                                       \
-      case kS128x128: return dense_kernel_ptr<BP_, 128, 128>(); \
-      case kS128x64: return dense_kernel_ptr<BP_, 128, 64>();   \
-      case kS64x64: return dense_kernel_ptr<BP_, 64, 64>();     \
-      case kS64x128: return dense_kernel_ptr<BP_, 64, 128>();   \
-      default: return nullptr;                                         \
-    }
-  switch (bp) {
-    HYB_CASE(1)
-    HYB_CASE(2)
-    HYB_CASE(4)
-    HYB_CASE(8)
-    HYB_CASE(16)
-    default: return nullptr;
-  }
-#undef HYB_CASE
-}
-
 struct TmaKernel {
   void *fn;
   int threads;
-  size_t smem;
+  size_t smem;       // dynamic shared memory with every stage of the ring
+  int stage_bytes;
+  int stages;        // the ring's compile-time stage count
   int tps;
   bool xtm;    // X slices by 2-D tensor copies (box xcols x bp)
   int xcols;
   int bp;
 };
 
-template <int BP, int B1, int B2>
+template <int BP, int B1, int B2, int PAT, bool LR = false>
 TmaKernel tma_kernel_info() {
-  using C = TmaCfg<BP, B1, B2>;
-  return TmaKernel{reinterpret_cast<void *>(&hybrid_tma_kernel<BP, B1, B2>), C::kThreads,
-                   C::kSmem, C::TPX, C::XTM, C::XT * B2, BP};
+  using C = TmaCfg<BP, B1, B2, LR>;
+  return TmaKernel{reinterpret_cast<void *>(&hybrid_tma_kernel<BP, B1, B2, PAT, LR>), C::kThreads,
+                   C::kSmem, C::kStageBytes, C::kStages, C::TPX, C::XTM, C::XT * B2, BP};
 }
 
-bool pick_tma_kernel(int bp, Shape s, TmaKernel *out) {
-#define HYB_TCASE(BP_)                                                         \
-  case BP_:                                                                    \
-    switch (s) {                                                               \
-      case kS128x128: *out = tma_kernel_info<BP_, 128, 128>(); return true;    \
-      case kS128x64: *out = tma_kernel_info<BP_, 128, 64>(); return true;      \
-      case kS64x64: *out = tma_kernel_info<BP_, 64, 64>(); return true;        \
-      case kS64x128: *out = tma_kernel_info<BP_, 64, 128>(); return true;      \
-      default: return false;                                                   \
+bool pick_tma_kernel(int bp, Shape s, int pat, bool lr, TmaKernel *out) {
+#define HYB_TCASE(BP_, PAT_, LR_)                                                            \
+  case BP_:                                                                                  \
+    switch (s) {                                                                             \
+      case kS128x128: *out = tma_kernel_info<BP_, 128, 128, PAT_, LR_>(); return true;       \
+      case kS128x64: *out = tma_kernel_info<BP_, 128, 64, PAT_, LR_>(); return true;         \
+      case kS64x64: *out = tma_kernel_info<BP_, 64, 64, PAT_, LR_>(); return true;           \
+      case kS64x128: *out = tma_kernel_info<BP_, 64, 128, PAT_, LR_>(); return true;         \
+      default: return false;                                                                 \
     }
-  switch (bp) {
-    HYB_TCASE(1)
-    HYB_TCASE(2)
-    HYB_TCASE(4)
-    HYB_TCASE(8)
-    HYB_TCASE(16)
-    default: return false;
+#define HYB_TSET(PAT_, LR_)  \
+  switch (bp) {              \
+    HYB_TCASE(1, PAT_, LR_)  \
+    HYB_TCASE(2, PAT_, LR_)  \
+    HYB_TCASE(4, PAT_, LR_)  \
+    HYB_TCASE(8, PAT_, LR_)  \
+    HYB_TCASE(16, PAT_, LR_) \
+    default: return false;   \
   }
+  // the low-rank term exists for 2:4 tiles only (the N:M entry point has none)
+  if (pat == 1) {
+    if (lr) return false;
+    HYB_TSET(1, false)
+  }
+  if (lr) {
+    switch (bp) {  // (only narrow batches fuse the low-rank term)
+      HYB_TCASE(1, 0, true)
+      HYB_TCASE(2, 0, true)
+      HYB_TCASE(4, 0, true)
+      default: return false;
+    }
+  }
+  HYB_TSET(0, false)
+#undef HYB_TSET
 #undef HYB_TCASE
 }
 
@@ -1516,8 +1810,47 @@ void *pick_lowrank_apply(int bp) {
   }
 }
 
-// Resident CTAs per SM of a kernel instance (cached; the answer only depends
-// on the instance and the device).
+// Static shared memory of a kernel instance and the dynamic shared memory it
+// may be launched with (the device's opt-in maximum less the static part);
+// the first query for an instance also raises its dynamic limit to that
+// maximum.  Cached per instance and device.
+int kernel_smem_limits(void *fn, size_t *static_bytes, size_t *max_dynamic) {
+  static std::mutex mu;
+  struct Entry {
+    void *fn;
+    int dev;
+    size_t stat, dyn;
+  };
+  static Entry cache[256];
+  static int used = 0;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return HYB_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(mu);
+  for (int i = 0; i < used; ++i)
+    if (cache[i].fn == fn && cache[i].dev == dev) {
+      *static_bytes = cache[i].stat;
+      *max_dynamic = cache[i].dyn;
+      return HYB_OK;
+    }
+  cudaFuncAttributes attr{};
+  int optin = 0;
+  if (cudaFuncGetAttributes(&attr, fn) != cudaSuccess ||
+      cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess)
+    return HYB_ERR_CUDA;
+  if ((size_t)optin <= attr.sharedSizeBytes) return HYB_ERR_UNSUPPORTED;
+  const size_t dyn = (size_t)optin - attr.sharedSizeBytes;
+  if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)dyn) !=
+      cudaSuccess)
+    return HYB_ERR_CUDA;
+  if (used < 256) cache[used++] = Entry{fn, dev, attr.sharedSizeBytes, dyn};
+  *static_bytes = attr.sharedSizeBytes;
+  *max_dynamic = dyn;
+  return HYB_OK;
+}
+
+// Resident CTAs per SM of a kernel instance with this much dynamic shared
+// memory (cached; the answer only depends on the instance, the size and the
+// device).
 int blocks_per_sm(void *fn, size_t dyn_smem, int threads = kThreads) {
   static std::mutex mu;
   struct Entry {
@@ -1530,31 +1863,28 @@ int blocks_per_sm(void *fn, size_t dyn_smem, int threads = kThreads) {
   static int used = 0;
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return -1;
-  // dynamic shared memory is small; bucket it so the cache stays tiny
-  const size_t bucket = align_up(dyn_smem, 4096);
+  size_t stat = 0, maxdyn = 0;
+  if (kernel_smem_limits(fn, &stat, &maxdyn) != HYB_OK || dyn_smem > maxdyn) return -1;
   std::lock_guard<std::mutex> lock(mu);
   for (int i = 0; i < used; ++i)
-    if (cache[i].fn == fn && cache[i].dev == dev && cache[i].smem == bucket)
+    if (cache[i].fn == fn && cache[i].dev == dev && cache[i].smem == dyn_smem)
       return cache[i].blocks;
   int nb = 0;
-  if (bucket > 48 * 1024 &&
-      cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bucket) !=
-          cudaSuccess)
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&nb, fn, threads, dyn_smem) != cudaSuccess)
     return -1;
-  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&nb, fn, threads, bucket) != cudaSuccess)
-    return -1;
-  if (used < 256) cache[used++] = Entry{fn, dev, bucket, nb};
+  if (used < 256) cache[used++] = Entry{fn, dev, dyn_smem, nb};
   return nb;
 }
 
 // Work split and workspace layout of one product call.
 struct Plan {
-  bool tma;        // TMA-ring kernel (packed hybrid, tuned tile shapes)
+  bool tma;        // TMA-ring kernel (tuned tile shapes, packed or row-major)
+  bool fused;      // a low-rank term computed inside the streaming kernel
   TmaKernel tk;
-  bool stream;     // tuned kernel (else one warp per row)
   int bp;          // padded batch
   int b1, b2;
   int G;           // CTAs of the stream split
+  int nst;         // ring stages of the launch
   int R;           // bands
   int64_t total;   // packed bytes
   int lr_ctas;     // CTAs of the low-rank reduction
@@ -1572,7 +1902,7 @@ int tma_ctas(int sms, int64_t total_bytes, int b1, int b2) {
 }
 
 int make_plan(int64_t n, int64_t k, int b1, int b2, int64_t total_bytes,
-              int batch, int rank, bool strided, Plan *pl) {
+              int batch, int rank, bool strided, Plan *pl, int pat = 0) {
   Plan P{};
   P.bp = pad_batch(batch);
   P.b1 = b1;
@@ -1583,48 +1913,53 @@ int make_plan(int64_t n, int64_t k, int b1, int b2, int64_t total_bytes,
   int sms = 0;
   int rc = device_sm_count(&sms);
   if (rc != HYB_OK) return rc;
-  P.tma = !strided && s != kGeneric;
+  (void)strided;  // packed and row-major matrices take the same kernels
+  P.tma = s != kGeneric;
+  // A low-rank term rides in the streaming kernel for narrow batches, where
+  // it is a few percent more bytes and little arithmetic; for batch 8 and 16
+  // its arithmetic (2 batch r (n + k) flops) is better spread over the whole
+  // GPU by the separate kernels than left to one warp of each CTA.
+  P.fused = P.tma && rank > 0 && P.bp <= 4;
   if (P.tma) {
     P.G = tma_ctas(sms, total_bytes, b1, b2);
-    if (!pick_tma_kernel(P.bp, s, &P.tk)) return HYB_ERR_UNSUPPORTED;
-  }
-  P.stream = strided && s != kGeneric && P.R <= 8192;
-  P.dyn_smem = P.tma ? P.tk.smem : (P.stream ? (size_t)2 * P.R * sizeof(int) : 0);
-  if (P.tma) {
-    const int nb = blocks_per_sm(P.tk.fn, P.tk.smem, P.tk.threads);
+    if (!pick_tma_kernel(P.bp, s, pat, P.fused, &P.tk)) return HYB_ERR_UNSUPPORTED;
+    // a low-rank term adds the low-rank warp's chunk buffer after the ring,
+    // and the ring gives up stages if both do not fit
+    size_t stat = 0, maxdyn = 0;
+    rc = kernel_smem_limits(P.tk.fn, &stat, &maxdyn);
+    if (rc != HYB_OK) return rc;
+    const size_t extra = P.tk.smem - (size_t)P.tk.stages * P.tk.stage_bytes;  // alignment slack
+    const size_t lrb = P.fused ? (size_t)kLrBufBytes : 0;
+    const int fit = maxdyn > extra + lrb ? (int)((maxdyn - extra - lrb) / P.tk.stage_bytes) : 0;
+    P.nst = std::min(P.tk.stages, fit);
+    if (P.nst < 3) return HYB_ERR_UNSUPPORTED;
+    P.dyn_smem = (size_t)P.nst * P.tk.stage_bytes + extra + lrb;
+    const int nb = blocks_per_sm(P.tk.fn, P.dyn_smem, P.tk.threads);
     if (nb <= 0) return HYB_ERR_CUDA;
-  } else if (P.stream) {
-    void *fn = pick_dense_kernel(P.bp, s);
-    if (P.dyn_smem > 48 * 1024) {
-      if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               (int)P.dyn_smem) != cudaSuccess)
-        return HYB_ERR_CUDA;
-    }
-    const int nb = blocks_per_sm(fn, P.dyn_smem);
-    if (nb <= 0) return HYB_ERR_CUDA;
-    const int64_t max_cost = 2LL * b1 * b2;  // a dense tile
-    int64_t G = (int64_t)nb * sms;
-    // every CTA must own at least one tile: total / G >= largest tile
-    const int64_t gcap = std::max<int64_t>(1, total_bytes / max_cost);
-    P.G = (int)std::min(G, gcap);
   } else {
     P.G = 0;
+    P.nst = 0;
+    P.dyn_smem = 0;
   }
-  P.lr_ctas = rank > 0 ? (int)std::max<int64_t>(1, std::min<int64_t>(sms, k / 64)) : 0;
-  size_t off = kHeaderBytes;
+  // partials of t: one per CTA of the streaming kernel (fused), else one per
+  // CTA of the separate V^T x kernel
+  P.lr_ctas = rank <= 0 ? 0
+              : P.fused  ? P.G
+                         : (int)std::max<int64_t>(1, std::min<int64_t>(sms, k / 64));
+  size_t off = kTicketsOffset;
   P.off_counters = off;
   if (P.tma) off = align_up(off + (size_t)P.R * (b1 / 8) * sizeof(uint32_t), 256);
-  else if (P.stream) off = align_up(off + (size_t)P.R * sizeof(uint32_t), 256);
   P.off_lr_t = off;
   off = align_up(off + (size_t)P.bp * (rank > 0 ? rank : 0) * sizeof(float), 256);
   P.off_lr_part = off;
   off = align_up(off + (size_t)P.lr_ctas * P.bp * (rank > 0 ? rank : 0) * sizeof(float), 256);
-  P.off_lr_counter = off;
-  off = align_up(off + sizeof(uint32_t), 256);
+  // ticket of the V^T x kernel (the fused term's epoch and flags have their
+  // own fixed places)
+  P.off_lr_counter = kLowrankTicketOffset;
   P.off_lr_ut = off;
   off = align_up(off + (size_t)P.bp * (rank > 0 ? n : 0) * sizeof(float), 256);
   P.off_partials = off;
-  if (P.tma || P.stream) off += (size_t)(P.G + P.R) * b1 * P.bp * sizeof(float);
+  if (P.tma) off += (size_t)(P.G + P.R) * b1 * P.bp * sizeof(float);
   P.bytes = align_up(off, 256);
   *pl = P;
   return HYB_OK;
@@ -1685,8 +2020,7 @@ int launch_lowrank_t(const Plan &P, const hyb_lowrank *lr, int64_t k,
 // Tensor map of X ([batch][k] bf16, row stride ldx) with box [bp][xcols]:
 // rows past the batch and columns past k read as zeros.  The encoder is the
 // driver's, found once through the runtime.
-int encode_x_map(const uint16_t *X, int64_t k, int batch, int64_t ldx, int xcols, int bp,
-                 CUtensorMap *map) {
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
   static PFN_cuTensorMapEncodeTiled_v12000 encode = nullptr;
   static std::once_flag once;
   std::call_once(once, [] {
@@ -1697,6 +2031,12 @@ int encode_x_map(const uint16_t *X, int64_t k, int batch, int64_t ldx, int xcols
         q == cudaDriverEntryPointSuccess)
       encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
   });
+  return encode;
+}
+
+int encode_x_map(const uint16_t *X, int64_t k, int batch, int64_t ldx, int xcols, int bp,
+                 CUtensorMap *map) {
+  PFN_cuTensorMapEncodeTiled_v12000 encode = tensor_map_encoder();
   if (!encode) return HYB_ERR_CUDA;
   const cuuint64_t dims[2] = {(cuuint64_t)k, (cuuint64_t)batch};
   const cuuint64_t strides[1] = {(cuuint64_t)ldx * 2};
@@ -1706,6 +2046,24 @@ int encode_x_map(const uint16_t *X, int64_t k, int batch, int64_t ldx, int xcols
                             const_cast<uint16_t *>(X), dims, strides, box, estr,
                             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
                             CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? HYB_OK : HYB_ERR_CUDA;
+}
+
+// Tensor map of a row-major bf16 W ([n][k], row stride ldw) with box
+// [b1 rows][b2 columns]: one box is one dense tile, in the packed dense
+// tile layout.
+int encode_w_map(const uint16_t *W, int64_t n, int64_t k, int64_t ldw, int b1, int b2,
+                 CUtensorMap *map) {
+  PFN_cuTensorMapEncodeTiled_v12000 encode = tensor_map_encoder();
+  if (!encode) return HYB_ERR_CUDA;
+  const cuuint64_t dims[2] = {(cuuint64_t)k, (cuuint64_t)n};
+  const cuuint64_t strides[1] = {(cuuint64_t)ldw * 2};
+  const cuuint32_t box[2] = {(cuuint32_t)b2, (cuuint32_t)b1};
+  const cuuint32_t estr[2] = {1, 1};
+  const CUresult r = encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<uint16_t *>(W),
+                            dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                            CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS ? HYB_OK : HYB_ERR_CUDA;
 }
@@ -1734,31 +2092,41 @@ void fill_launch_plan(const int64_t *plan, int32_t plan_ctas, const Plan &P, con
 
 int run_product(Params prm, int b1, int b2, int batch, const hyb_lowrank *lr,
                 bool strided, void *ws, size_t ws_bytes, cudaStream_t s,
-                const int64_t *plan = nullptr, int32_t plan_ctas = 0, uint32_t flags = 0) {
+                const int64_t *plan = nullptr, int32_t plan_ctas = 0, uint32_t flags = 0,
+                int pat = 0) {
   const int rank = (lr && lr->rank > 0) ? lr->rank : 0;
   Plan P;
-  int rc = make_plan(prm.n, prm.k, b1, b2, prm.total, batch, rank, strided, &P);
+  int rc = make_plan(prm.n, prm.k, b1, b2, prm.total, batch, rank, strided, &P, pat);
   if (rc != HYB_OK) return rc;
   if (!ws || ws_bytes < P.bytes) return HYB_ERR_WORKSPACE;
   if ((uintptr_t)ws % 256 != 0) return HYB_ERR_ALIGNMENT;
   uint8_t *w = reinterpret_cast<uint8_t *>(ws);
   prm.R = P.R;
   prm.G = P.G;
+  prm.nst = P.nst;
   prm.partials = reinterpret_cast<float *>(w + P.off_partials);
   prm.counters = reinterpret_cast<uint32_t *>(w + P.off_counters);
   prm.rank = rank;
   prm.U = rank ? lr->U : nullptr;
   prm.ldu = rank ? lr->ldu : 0;
-  prm.lr_t = reinterpret_cast<const float *>(w + P.off_lr_t);
+  prm.V = rank ? lr->V : nullptr;
+  prm.ldv = rank ? lr->ldv : 0;
+  prm.lr_t = reinterpret_cast<float *>(w + P.off_lr_t);
+  prm.lr_part = reinterpret_cast<float *>(w + P.off_lr_part);
+  prm.lr_epoch = reinterpret_cast<uint32_t *>(w + kLowrankEpochOffset);
+  prm.lr_flags = reinterpret_cast<uint32_t *>(w + kLowrankFlagsOffset);
   prm.lr_ut = nullptr;
+  prm.fused_lr = 0;
   const bool overlap = (flags & HYB_LAUNCH_OVERLAP_PREV) != 0;
-  if (rank) {
-    // V^T x, then U t, then the product: the two later kernels always launch
-    // as programmatic dependents of the one before.  V^T x lets them launch
-    // only after everything queued before the call has finished (with the
-    // caller's leave it starts early itself, and waits), so their early
-    // loads -- of U, the weights and X -- see finished data; what they wait
-    // for is t, U t and the workspace.
+  if (rank && P.fused) {
+    // the streaming kernel's low-rank warp computes V^T x and U t itself
+    prm.fused_lr = 1;
+    prm.lr_ut = reinterpret_cast<float *>(w + P.off_lr_ut);
+  } else if (rank) {
+    // wide batches and other tilings: V^T x, then U t, then the product,
+    // launched one after the other (the first as a programmatic dependent
+    // with the caller's overlap flag; the one-warp-per-row product ignores
+    // the flag)
     rc = launch_lowrank_t(P, lr, prm.k, prm.X, prm.ldx, batch, w, s, overlap);
     if (rc != HYB_OK) return rc;
     int64_t nn = prm.n, ldu = lr->ldu;
@@ -1766,33 +2134,34 @@ int run_product(Params prm, int b1, int b2, int batch, const hyb_lowrank *lr,
     int rk = rank, bt = batch;
     const float *tp = prm.lr_t;
     float *ut = reinterpret_cast<float *>(w + P.off_lr_ut);
-    int one = 1;
-    void *uargs[] = {&nn, &U, &ldu, &rk, &tp, &bt, &ut, &one};
+    int zero = 0;
+    void *uargs[] = {&nn, &U, &ldu, &rk, &tp, &bt, &ut, &zero};
     const int64_t grid = (prm.n + kThreads - 1) / kThreads;
-    if (launch_kernel(pick_lowrank_ut(P.bp), dim3((unsigned)grid), dim3(kThreads), uargs, 0, s,
-                      true) != cudaSuccess)
+    if (cudaLaunchKernel(pick_lowrank_ut(P.bp), dim3((unsigned)grid), dim3(kThreads), uargs, 0,
+                         s) != cudaSuccess)
       return HYB_ERR_CUDA;
     prm.lr_ut = ut;
   }
   prm.status = reinterpret_cast<uint32_t *>(w);
-  const bool pdl = (overlap || rank > 0) && (P.tma || P.stream);
-  prm.pdl = !pdl ? 0 : (rank > 0 ? 2 : 1);
-  void *args[] = {&prm};
+  const bool pdl = overlap && P.tma;
+  prm.pdl = pdl ? 1 : 0;
+  prm.rowmajor = strided ? 1 : 0;
   if (P.tma) {
     LaunchPlan lp;
-    fill_launch_plan(plan, plan_ctas, P, prm, &lp);
+    fill_launch_plan(strided ? nullptr : plan, plan_ctas, P, prm, &lp);
     alignas(64) CUtensorMap xmap{};
+    alignas(64) CUtensorMap wmap{};
     if (P.tk.xtm) {
       rc = encode_x_map(prm.X, prm.k, batch, prm.ldx, P.tk.xcols, P.tk.bp, &xmap);
       if (rc != HYB_OK) return rc;
     }
-    void *targs[] = {&prm, &lp, &xmap};
-    if (launch_kernel(P.tk.fn, dim3(P.G), dim3(P.tk.threads), targs, P.tk.smem, s, pdl) !=
+    if (strided) {
+      rc = encode_w_map(prm.Wd, prm.n, prm.k, prm.ldw, b1, b2, &wmap);
+      if (rc != HYB_OK) return rc;
+    }
+    void *targs[] = {&prm, &lp, &xmap, &wmap};
+    if (launch_kernel(P.tk.fn, dim3(P.G), dim3(P.tk.threads), targs, P.dyn_smem, s, pdl) !=
         cudaSuccess)
-      return HYB_ERR_CUDA;
-  } else if (P.stream) {
-    void *fn = pick_dense_kernel(P.bp, shape_of(b1, b2));
-    if (launch_kernel(fn, dim3(P.G), dim3(kThreads), args, P.dyn_smem, s, pdl) != cudaSuccess)
       return HYB_ERR_CUDA;
   } else {
     void *fn = strided ? pick_rowwarp_kernel<true>(P.bp)
@@ -1825,7 +2194,7 @@ int check_io(const uint16_t *X, int64_t ldx, void *Y, int64_t ldy, int64_t n,
 
 int spmm_impl(const hyb_matrix *A, int batch, const uint16_t *X, int64_t ldx,
               void *Y, int64_t ldy, hyb_dtype ydt, const hyb_lowrank *lr,
-              void *ws, size_t ws_bytes, cudaStream_t s, uint32_t flags = 0) {
+              void *ws, size_t ws_bytes, cudaStream_t s, uint32_t flags = 0, int pat = 0) {
   if (!A) return HYB_ERR_INVALID_ARG;
   if (flags & ~HYB_LAUNCH_OVERLAP_PREV) return HYB_ERR_INVALID_ARG;
   int rc = check_tiling(A->n, A->k, A->b1, A->b2);
@@ -1863,7 +2232,7 @@ int spmm_impl(const hyb_matrix *A, int batch, const uint16_t *X, int64_t ldx,
   prm.nvb = 2 * A->n_vals;
   prm.nmb = A->n_meta_bytes;
   return run_product(prm, A->b1, A->b2, batch, lr, false, ws, ws_bytes, s, A->plan,
-                     A->plan_ctas, flags);
+                     A->plan_ctas, flags, pat);
 }
 
 // Virtual tiling of a plain row-major W for the dense baseline.
@@ -1891,12 +2260,28 @@ size_t lowrank_ws_layout(int64_t k, int batch, int rank, size_t *off_t,
   off = align_up(off + (size_t)bp * rank * sizeof(float), 256);
   *off_part = off;
   off = align_up(off + (size_t)(*ctas) * bp * rank * sizeof(float), 256);
-  *off_counter = off;
-  off = align_up(off + sizeof(uint32_t), 256);
+  *off_counter = kLowrankTicketOffset;  // in the header, the same place for every call
   return off;
 }
 
 }  // namespace
+
+// The streaming product of a matrix packed by hyb_pack_nm with nk = 2 of
+// m = 4 (hyb_pack's layout) or nk = 4 of m = 8: both keep half of a sparse
+// tile's values with b1 * b2 / 8 mask bytes, so the split, the plan and the
+// stage packing are the 2:4 ones; only the mask decode differs.  Returns
+// HYB_ERR_UNSUPPORTED when the tiling has no streaming kernel.
+int stream_product_nm(const hyb_matrix *A, int nk, int m, int batch, const uint16_t *X,
+                      int64_t ldx, void *Y, int64_t ldy, hyb_dtype ydt, void *ws,
+                      size_t ws_bytes, cudaStream_t s) {
+  if (shape_of(A->b1, A->b2) == kGeneric) return HYB_ERR_UNSUPPORTED;
+  int pat;
+  if (nk == 2 && m == 4) pat = 0;
+  else if (nk == 4 && m == 8) pat = 1;
+  else return HYB_ERR_UNSUPPORTED;
+  return spmm_impl(A, batch, X, ldx, Y, ldy, ydt, nullptr, ws, ws_bytes, s, 0, pat);
+}
+
 }  // namespace hyb
 
 using namespace hyb;
@@ -2052,10 +2437,9 @@ int hyb_gemv_dense_ex(int64_t n, int64_t k, int batch, const uint16_t *W, int64_
   if (rc != HYB_OK) return rc;
   int b1, b2;
   dense_tiling(n, k, &b1, &b2);
-  // the tuned kernel reads 32-byte pieces of W; the row-per-warp one 16
-  const bool wide = b1 > 1;
-  if ((uintptr_t)W % (wide ? 32 : 16) != 0 || ldw % (wide ? 16 : 8) != 0)
-    return HYB_ERR_ALIGNMENT;
+  // the streaming kernel reads W by tensor copies (16-byte aligned start and
+  // row stride), the row-per-warp one in 16-byte pieces
+  if ((uintptr_t)W % 16 != 0 || ldw % 8 != 0) return HYB_ERR_ALIGNMENT;
   Params prm{};
   prm.Wd = W;
   prm.ldw = ldw;

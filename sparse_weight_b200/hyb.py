@@ -300,9 +300,11 @@ def packed_sizes_nm(n: int, k: int, b1: int, b2: int, nk: int, m: int, tile_map)
 
 
 def pack_nm(W: torch.Tensor, tile_map, b1: int, b2: int, nk: int, m: int,
-            ws: torch.Tensor = None, stream=None, check: bool = True) -> Packed:
+            ws: torch.Tensor = None, stream=None, check: bool = True,
+            plan: bool = True) -> Packed:
     """hyb_pack_nm: dense bf16 W [n][k] (device) + tile map -> Packed with
-    nk:m sparse tiles (no work-split plan: the N:M product does not use one)."""
+    nk:m sparse tiles.  With ``plan``, 2:4 and 4:8 matrices (whose products run
+    the streaming kernel) get their work split made once here."""
     Wb = _bits(W)
     assert Wb.is_cuda and Wb.dim() == 2
     n, k = Wb.shape
@@ -323,7 +325,10 @@ def pack_nm(W: torch.Tensor, tile_map, b1: int, b2: int, nk: int, m: int,
                                             _ptr(mo), _ptr(ws), ws.numel(), _stream(stream)))
     if check:
         check_status(ws, stream)
-    return Packed(n, k, b1, b2, tm, vals, meta, vo, mo, nv, nmb)
+    P = Packed(n, k, b1, b2, tm, vals, meta, vo, mo, nv, nmb)
+    if plan and (nk, m) in ((2, 4), (4, 8)):
+        P.plan, P.plan_ctas = make_plan(P, stream)
+    return P
 
 
 def spmm_skinny_nm(A: Packed, X: torch.Tensor, nk: int, m: int, Y: torch.Tensor = None,
@@ -335,7 +340,7 @@ def spmm_skinny_nm(A: Packed, X: torch.Tensor, nk: int, m: int, Y: torch.Tensor 
     batch = Xb.shape[0]
     Y = _out(A.n, batch, ydt, Xb.device, Y)
     if ws is None:
-        ws = new_workspace(pack_workspace_bytes(), Xb.device)
+        ws = new_workspace(workspace_bytes(A, batch), Xb.device)
     s = A.struct()
     _check("hyb_spmm_skinny_nm", lib().hyb_spmm_skinny_nm(
         ctypes.byref(s), nk, m, batch, _ptr(Xb), Xb.stride(0), _ptr(Y), Y.stride(0), ydt,

@@ -60,7 +60,7 @@ def _sizes(n, k, b1, b2, m):
 def test_packed_sizes_closed_form(L, orc):
     rng = np.random.default_rng(0)
     for (n, k, b1, b2) in [(256, 256, 64, 64), (4096, 4096, 128, 128), (1024, 4096, 128, 64),
-                           (64, 96, 16, 32)]:
+                           (64, 96, 16, 32), (64, 128, 16, 8), (128, 96, 64, 24)]:
         T = (n // b1) * (k // b2)
         m = (rng.random(T) < 0.5).astype(np.uint8)
         rc, nv, nm = _sizes(n, k, b1, b2, m)
@@ -70,8 +70,9 @@ def test_packed_sizes_closed_form(L, orc):
         assert nv == (T - s) * b1 * b2 + s * b1 * b2 // 2 and nm == s * b1 * b2 // 8
 
 
-@pytest.mark.parametrize("shape", [(0, 64, 16, 16), (64, 64, 16, 8), (60, 64, 16, 16),
-                                   (64, 60, 16, 16), (8, 16, 1, 16)])
+@pytest.mark.parametrize("shape", [(0, 64, 16, 16), (64, 64, 8, 8), (64, 64, 32, 4),
+                                   (60, 64, 16, 16), (64, 60, 16, 16), (8, 16, 1, 16),
+                                   (64, 60, 16, 12)])
 def test_packed_sizes_rejects_bad_tiling(L, shape):
     n, k, b1, b2 = shape
     T = max(1, (n // max(b1, 1)) * (k // max(b2, 1)))
@@ -209,17 +210,17 @@ def test_dense_and_lowrank_argument_checks(L):
     W, X, Y, ws = P(0x10000), P(0x60000), P(0x70000), P(0x80000)
     assert L.hyb_gemv_dense(64, 40, 1, W, 40, X, 40, Y, 64, 0, ws, 1 << 20,
                             None) == hyb.HYB_ERR_INVALID_ARG  # k % 16
-    assert L.hyb_gemv_dense(64, 64, 1, P(0x10010), 64, X, 64, Y, 64, 0, ws, 1 << 20,
-                            None) == hyb.HYB_ERR_ALIGNMENT
-    assert L.hyb_gemv_dense(64, 64, 1, W, 72, X, 64, Y, 64, 0, ws, 1 << 20,
-                            None) == hyb.HYB_ERR_ALIGNMENT
+    assert L.hyb_gemv_dense(64, 64, 1, P(0x10008), 64, X, 64, Y, 64, 0, ws, 1 << 20,
+                            None) == hyb.HYB_ERR_ALIGNMENT  # W not 16-byte aligned
+    assert L.hyb_gemv_dense(64, 64, 1, W, 68, X, 64, Y, 64, 0, ws, 1 << 20,
+                            None) == hyb.HYB_ERR_ALIGNMENT  # rows not 16-byte aligned
     assert L.hyb_gemv_dense(60, 48, 1, W, 52, X, 48, Y, 64, 0, ws, 1 << 20,
                             None) == hyb.HYB_ERR_ALIGNMENT
     lr = hyb.HybLowrank(0, P(0x90000), 8, P(0xA0000), 8)
     assert L.hyb_lowrank_add(64, 64, 1, ctypes.byref(lr), X, 64, Y, 64, ws, 1 << 20,
                              None) == hyb.HYB_ERR_INVALID_ARG
     assert L.hyb_workspace_bytes(None, 1, 0) == 0
-    A = _matrix(b2=8)
+    A = _matrix(b2=4)
     assert L.hyb_workspace_bytes(ctypes.byref(A), 1, 0) == 0
     assert L.hyb_workspace_init(None, 0, None) == hyb.HYB_ERR_WORKSPACE
     assert L.hyb_check_status(None, None, None) == hyb.HYB_ERR_WORKSPACE

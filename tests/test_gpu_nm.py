@@ -113,17 +113,21 @@ def test_spmm_nm_strided_operands(orc):
     assert bool((Ys[:, :4] == 7.0).all()) and bool((Ys[:, 4 + n:] == 7.0).all())
 
 
-def test_spmm_nm_bad_offsets_are_flagged():
+@pytest.mark.parametrize("nk,m", [(4, 8), (2, 8)])
+def test_spmm_nm_bad_offsets_are_flagged(nk, m):
     """A corrupted offset (past the value buffer) is skipped and reported
-    through the status word; nothing is read out of bounds."""
+    through the status word; nothing is read out of bounds.  4:8 runs the
+    streaming kernel (whose producer checks every stage's byte ranges), 2:8
+    the one-warp-per-row kernel."""
     n, k, b1, b2 = 256, 256, 64, 64
     T = (n // b1) * (k // b2)
     tmap = inputs.tile_map_fraction(T, 0.5, inputs.seed_of("nm_bad"))
     W = inputs.weight(n, k, 0.02, inputs.seed_of("nm_bad", "W")).to(dev())
-    P = hyb.pack_nm(W, tmap, b1, b2, 4, 8)
+    P = hyb.pack_nm(W, tmap, b1, b2, nk, m)
     P.val_off[3] = P.n_vals + 4096  # past the end of the values
-    ws = hyb.new_workspace(hyb.pack_workspace_bytes(), dev())
-    hyb.spmm_skinny_nm(P, torch.ones(1, k, dtype=torch.bfloat16, device=dev()), 4, 8, ws=ws)
+    P.plan, P.plan_ctas = None, 0  # the kernel reads the (corrupted) offsets itself
+    ws = hyb.new_workspace(hyb.workspace_bytes(P, 1), dev())
+    hyb.spmm_skinny_nm(P, torch.ones(1, k, dtype=torch.bfloat16, device=dev()), nk, m, ws=ws)
     with pytest.raises(hyb.HybError) as e:
         hyb.check_status(ws)
     assert e.value.status == hyb.HYB_ERR_DEVICE_CHECK

@@ -57,7 +57,8 @@ def test_pack_llama70b_ffn(orc):
         _pack_and_compare(orc, W, tmap, 128, 128)
 
 
-@pytest.mark.parametrize("tiling", [(16, 16), (32, 32), (8, 16), (1, 128), (128, 16)])
+@pytest.mark.parametrize("tiling", [(16, 16), (32, 32), (8, 16), (1, 128), (128, 16),
+                                    (16, 8), (128, 8), (64, 24)])
 def test_pack_other_tilings(orc, tiling):
     b1, b2 = tiling
     n, k = b1 * 6, b2 * 5

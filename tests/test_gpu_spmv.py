@@ -74,7 +74,8 @@ def test_rows_ragged(orc, tiling, batch, tpr):
     _full_check(orc, n, k, b1, b2, tmap, batch, f"rows{b1}x{b2}", ydt_bf16=batch in (1, 16))
 
 
-@pytest.mark.parametrize("tiling", [(16, 16), (32, 32), (8, 16), (1, 128), (128, 16), (256, 64)])
+@pytest.mark.parametrize("tiling", [(16, 16), (32, 32), (8, 16), (1, 128), (128, 16), (256, 64),
+                                    (16, 8), (128, 8), (64, 24), (32, 40)])
 @pytest.mark.parametrize("batch", [1, 3, 16])
 def test_other_tilings(orc, tiling, batch):
     b1, b2 = tiling
@@ -206,6 +207,44 @@ def test_llama70b_ffn_lowrank_full_size(orc):
 def test_lowrank_fused_small(orc, batch):
     tmap = inputs.tile_map_bernoulli(40, 0.6, inputs.seed_of("lrsmall"))
     _full_check(orc, 640, 1024, 128, 128, tmap, batch, "lrsmall", rank=64)
+
+
+@pytest.mark.parametrize("rank", [8, 24, 40, 128, 256])
+@pytest.mark.parametrize("tiling", [(128, 128), (128, 64), (64, 64)])
+@pytest.mark.parametrize("batch", [1, 3, 16])
+def test_lowrank_fused_ranks(orc, rank, tiling, batch):
+    """The low-rank term computed inside the streaming kernel (V^T x over
+    k-slices, t summed by slices, U t by row slices, grid barriers between):
+    every rank layout (16-byte chunks of a factor row that do and do not
+    divide a warp), tilings whose CTA counts differ, ragged batches."""
+    b1, b2 = tiling
+    n, k = 10 * b1, 24 * b2
+    T = (n // b1) * (k // b2)
+    tmap = inputs.tile_map_bernoulli(T, 0.5, inputs.seed_of("lrranks", b1, b2))
+    _full_check(orc, n, k, b1, b2, tmap, batch, f"lrranks{rank}", rank=rank)
+
+
+def test_lowrank_fused_repeated_calls(orc):
+    """The fused term's grid barrier and partial buffers are left ready for
+    the next call: calls in a row, alternating ranks, on one workspace."""
+    n, k, b1, b2 = 1024, 2048, 128, 128
+    T = (n // b1) * (k // b2)
+    tmap = inputs.tile_map_bernoulli(T, 0.5, inputs.seed_of("lrrep"))
+    W, tmap, X, _ = case(n, k, b1, b2, tmap, batch=4, name="lrrep")
+    P = hyb.pack(W.to(dev()), tmap, b1, b2)
+    ws = hyb.new_workspace(hyb.workspace_bytes(P, 4, 128), dev())
+    ref = orc.pack(inputs.bits(W), b1, b2, tmap)
+    outs = []
+    for i, rank in enumerate([128, 64, 128, 8]):
+        U, V = inputs.lowrank(n, k, rank, 0.01, inputs.seed_of("lrrep", i))
+        Y = hyb.spmm_skinny(P, X.to(dev()), lowrank=(U.to(dev()), V.to(dev())), ws=ws)
+        outs.append((U, V, Y))
+    torch.cuda.synchronize()
+    assert hyb.check_status(ws) == 0
+    for U, V, Y in outs:
+        y_ref, env = orc.spmv(n, k, b1, b2, tmap, ref, inputs.bits(X), inputs.bits(U),
+                              inputs.bits(V))
+        assert_within(Y.cpu().numpy(), y_ref, env, what=f"repeated r={U.shape[1]}")
 
 
 def _tile_split_reference(P, G):
