@@ -53,6 +53,9 @@ WORKLOADS = {
     "ffn_down_4096x14336_f0.5_b16": (4096, 14336, 128, 128, 0.5, 16, 0.02, 0.01),
     "ffn_down_4096x14336_f0.0_b1": (4096, 14336, 128, 128, 0.0, 1, 0.02, 0.01),
     "ffn_down_4096x14336_f1.0_b1": (4096, 14336, 128, 128, 1.0, 1, 0.02, 0.01),
+    "ffn_down_4096x14336_f1.0_b4": (4096, 14336, 128, 128, 1.0, 4, 0.02, 0.01),
+    "ffn_down_4096x14336_f1.0_b16": (4096, 14336, 128, 128, 1.0, 16, 0.02, 0.01),
+    "ffn_down_4096x14336_f0.0_b16": (4096, 14336, 128, 128, 0.0, 16, 0.02, 0.01),
 }
 
 

@@ -316,11 +316,32 @@ __device__ __forceinline__ void fma_bf16x2(float &acc, uint32_t w, uint32_t x) {
   asm("fma.rn.f32.bf16 %0, %1, %2, %0;" : "+f"(acc) : "h"(wh), "h"(xh));
 }
 
-template <int BP, int B1, int B2, bool LR = false>
+// D (16 x 8, fp32) += A (16 x 16, bf16, row-major) B (16 x 8, bf16, "col"):
+// one warp-wide tensor-core product.  Lane (g, c) = (lane / 4, lane % 4)
+// holds A rows g and g + 8 at k = 2c, 2c + 1 (a0, a1) and 2c + 8, 2c + 9
+// (a2, a3), B column g at the same k (b0, b1), and D rows g, g + 8 at
+// columns 2c, 2c + 1.
+__device__ __forceinline__ void mma_bf16_16816(float (&d)[4], uint32_t a0, uint32_t a1,
+                                               uint32_t a2, uint32_t a3, uint32_t b0,
+                                               uint32_t b1) {
+  asm("mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, "
+      "{%4, %5, %6, %7}, {%8, %9}, {%0, %1, %2, %3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+template <int BP, int B1, int B2, bool LR = false, int PAT = 0>
 struct TmaCfg {
-  // rows per consumer warp: 8, or 16 for wide batches so that the
-  // accumulators of a warp fit the register budget
-  static constexpr int RW = BP >= 8 ? 16 : 8;
+  // From batch 4 on, dense and 2:4 tiles go through the tensor cores (the
+  // batch is the product's M side, padded to 16; a 2:4 tile row is expanded
+  // to dense bf16 pairs in registers); narrower batches, and 4:8 tiles, use
+  // scalar FMAs.
+  static constexpr bool MMA = BP >= 4 && PAT == 0;
+  // rows per consumer warp: 8; 16 from batch 4 on (scalar: fewer warps,
+  // each reusing its X registers over more rows; tensor cores: two 8-row
+  // product columns per warp, eight warps for a 128-row tile -- four warps
+  // leave the tensor products too little overlap, sixteen re-read X too often)
+  static constexpr int RW = BP >= 4 ? 16 : 8;
   static constexpr int NC = B1 / RW;                // consumer warps
   static constexpr int CPR = B2 / 16;               // lanes per row, 16 columns each
   static constexpr int RPS = 32 / CPR;              // rows per warp step
@@ -351,7 +372,8 @@ struct TmaCfg {
   // code)
   static constexpr int kThreads = (NC + 3 + (LR ? 1 : 0)) * 32;
   static constexpr size_t kSmem = (size_t)kStages * kStageBytes + 1024;
-  static_assert(RPS * CPR == 32 && JS * RPS == RW && JS >= 1, "tile shape");
+  static_assert(MMA || (RPS * CPR == 32 && JS * RPS == RW && JS >= 1), "tile shape");
+  static_assert(!MMA || (B2 % 64 == 0 && B1 % RW == 0), "tensor-core tile shape");
   static_assert(kStages >= 3, "ring too short");
   static_assert(TPX <= 8 && WIN < 32, "stage / offset window");
   static_assert(TPX % XT == 0 && (!XTM || XT * B2 <= 256), "X copy groups");
@@ -362,9 +384,10 @@ struct TmaCfg {
 // tile (a dense tile is 2), at most 2 tpd units and tpx tiles per stage, and
 // a new stage at every band start.  Used by the streaming kernel for every
 // window and by the plan for each CTA's first window.
-__device__ __forceinline__ uint32_t stage_starts(uint32_t spm, int nw, int64_t w0, int tpr,
+__device__ __forceinline__ uint32_t stage_starts(uint32_t spm, int nw, uint32_t w0_col, int tpr,
                                                 int tpd, int tpx) {
-  int nb = (int)((tpr - w0 % tpr) % tpr);  // first band start at or after w0, relative
+  // (w0_col = w0 mod tpr: the tile column of w0 within its band)
+  int nb = (int)(((uint32_t)tpr - w0_col) % (uint32_t)tpr);  // first band start at or after w0
   uint32_t starts = 0;
   int fill = 2 * tpx, cnt = tpx;  // force a start at tile 0
   for (int i = 0; i < nw; ++i) {
@@ -470,16 +493,17 @@ __device__ __forceinline__ uint2 lut48_entry(uint32_t m) {
 // PAT 0: 2:4 tiles (hyb_pack); PAT 1: 4:8 tiles (hyb_pack_nm with 4 of 8).
 // LR: the instance for calls with a low-rank term (an extra warp computes it).
 template <int BP, int B1, int B2, int PAT, bool LR>
-__global__ void __launch_bounds__(TmaCfg<BP, B1, B2, LR>::kThreads, 1)
+__global__ void __launch_bounds__(TmaCfg<BP, B1, B2, LR, PAT>::kThreads, 1)
     hybrid_tma_kernel(const Params p, const LaunchPlan lp, const __grid_constant__ CUtensorMap xmap,
                       const __grid_constant__ CUtensorMap wmap) {
-  using C = TmaCfg<BP, B1, B2, LR>;
+  using C = TmaCfg<BP, B1, B2, LR, PAT>;
   constexpr int S = C::kStages;
   extern __shared__ __align__(1024) uint8_t smem[];
   __shared__ __align__(8) uint64_t full_bar[S];
   __shared__ __align__(8) uint64_t empty_bar[S];
   __shared__ StageDesc desc[S];
   __shared__ uint32_t sel_lut[16];
+  __shared__ uint32_t sel_dense[16];
   __shared__ uint2 lut48[PAT == 1 ? 256 : 1];
   __shared__ uint32_t s_cnt[2];
   __shared__ int64_t s_range[2];
@@ -558,6 +582,16 @@ __global__ void __launch_bounds__(TmaCfg<BP, B1, B2, LR>::kThreads, 1)
         p1 = 31 - __clz(m);
       }
       sel_lut[m] = (2 * p0) | ((2 * p0 + 1) << 4) | ((2 * p1) << 8) | ((2 * p1 + 1) << 12);
+      // PRMT selectors expanding a kept pair (v_p0 in bytes 0-1, v_p1 in
+      // bytes 2-3, zero bytes 4-7) to the group's dense columns 0-1 (low
+      // half) and 2-3 (high half); a column not kept takes zero bytes
+      uint32_t sd = 0;
+      for (int j = 0; j < 4; ++j) {
+        const uint32_t lo = !m ? 4u : (j == (int)p0 ? 0u : (j == (int)p1 ? 2u : 4u));
+        const uint32_t hi = lo == 4u ? 4u : lo + 1u;
+        sd |= (lo | hi << 4) << (8 * j);
+      }
+      sel_dense[m] = sd;
     }
     if constexpr (PAT == 1) {
       for (int m = tid; m < 256; m += blockDim.x) lut48[m] = lut48_entry((uint32_t)m);
@@ -729,6 +763,9 @@ __global__ void __launch_bounds__(TmaCfg<BP, B1, B2, LR>::kThreads, 1)
       const Win nxt = load_win(w0 + C::WIN);  // in flight while this window issues
       const int nw = (int)min((int64_t)C::WIN, t1 - w0);
       const uint32_t spm = __ballot_sync(0xffffffffu, cur.sp == 1u);
+      // band and tile column of w0 (tile indices fit 32 bits on this path)
+      const uint32_t tpu = (uint32_t)tpr;
+      const uint32_t wband = (uint32_t)w0 / tpu, wcol = (uint32_t)w0 - wband * tpu;
       if (!p.rowmajor && !(derived && w0 == t0)) {
         // offsets read from the matrix must step by each tile's size (a
         // corrupted matrix is flagged; the copies are bounded either way)
@@ -752,10 +789,10 @@ __global__ void __launch_bounds__(TmaCfg<BP, B1, B2, LR>::kThreads, 1)
         const int units = 2 * (e - lane) - __popc((spm >> lane) & in);
         const bool good = lane >= nw || !(starts >> lane & 1u) ||
                           (e - lane <= C::TPX && units <= 2 * C::TPD);
-        const bool band_ok = lane >= nw || (w0 + lane) % tpr != 0 || (starts >> lane & 1u);
+        const bool band_ok = lane >= nw || (wcol + lane) % tpu != 0 || (starts >> lane & 1u);
         have = __all_sync(0xffffffffu, good && band_ok) && (starts & 1u) && (starts >> nw) == 0;
       }
-      if (!have) starts = stage_starts(spm, nw, w0, tpr, C::TPD, C::TPX);
+      if (!have) starts = stage_starts(spm, nw, wcol, tpr, C::TPD, C::TPX);
       // the stage that starts at this lane: tiles [w0 + lane, w0 + e).  Every
       // start lane works out its stage here, all at once, so that the serial
       // part below (one stage after the other, as ring slots free up) only
@@ -783,7 +820,7 @@ __global__ void __launch_bounds__(TmaCfg<BP, B1, B2, LR>::kThreads, 1)
       const int ngx = (nt + C::XT - 1) / C::XT;  // X copy groups (tensor path)
       const uint32_t xbytes =
           C::XTM ? (uint32_t)(ngx * C::kXCopy) : (uint32_t)(2 * B2 * nt) * (uint32_t)p.batch;
-      const int64_t band = w0 / tpr + (lane + (int)(w0 % tpr)) / tpr;  // = ts / tpr
+      const int64_t band = wband + (wcol + lane) / tpu;  // = ts / tpr
       StageDesc dl;
       dl.t0 = ts;
       dl.ntiles = (uint16_t)nt;
@@ -1121,7 +1158,8 @@ __global__ void __launch_bounds__(TmaCfg<BP, B1, B2, LR>::kThreads, 1)
       lr_wait = false;
       if (!mbar_wait(&lr_done, 0u) && lane == 0) atomicOr(p.status, kStatusTimeout);
     };
-    const int r_first = (int)(t0 / tpr), r_last = t1 > t0 ? (int)((t1 - 1) / tpr) : r_first - 1;
+    const int r_first = (int)((uint32_t)t0 / (uint32_t)tpr);
+    const int r_last = t1 > t0 ? (int)((uint32_t)(t1 - 1) / (uint32_t)tpr) : r_first - 1;
     for (int r = r_first + ew; r <= r_last; r += 2) {
       const int piece = r - r_first;
       const int slot = piece & 1;
@@ -1214,11 +1252,21 @@ __global__ void __launch_bounds__(TmaCfg<BP, B1, B2, LR>::kThreads, 1)
   const int cp = lane % C::CPR;
   const int rs = lane / C::CPR;
   const int wrow = warp * C::RW;
-  float acc[C::JS][BP];
+  // scalar consumers: acc[j][b], row j RPS + rs of the warp, batch column b
+  float acc[C::MMA ? 1 : C::JS][BP];
 #pragma unroll
-  for (int j = 0; j < C::JS; ++j)
+  for (int j = 0; j < (C::MMA ? 1 : C::JS); ++j)
 #pragma unroll
     for (int b = 0; b < BP; ++b) acc[j][b] = 0.f;
+  // tensor-core consumers: dacc[nb] is the D fragment of the warp's rows
+  // 8 nb .. 8 nb + 7 (lane (g, c): batch g and g + 8, rows 2c and 2c + 1)
+  constexpr int NB = C::MMA ? C::RW / 8 : 1;
+  float dacc[NB][4];
+#pragma unroll
+  for (int nb = 0; nb < NB; ++nb)
+#pragma unroll
+    for (int q = 0; q < 4; ++q) dacc[nb][q] = 0.f;
+  const int mg = lane >> 2, mc = lane & 3;
   int piece = 0;
 
   int stage = 0;
@@ -1239,99 +1287,154 @@ __global__ void __launch_bounds__(TmaCfg<BP, B1, B2, LR>::kThreads, 1)
       // row (so that 8 lanes read 128 contiguous bytes of shared memory)
       const uint8_t *xs = st + C::kValsBytes + C::kMetaBytes + (i / C::XT) * C::kXCopy +
                           (i % C::XT) * 2 * B2;
-      const int xo0 = sp ? 32 * cp : 16 * cp;
-      const int xo1 = sp ? 32 * cp + 16 : B2 + 16 * cp;
+      if constexpr (C::MMA) {
+        // Columns of a 64-column block are spread over the four products of
+        // the block so that every lane reads contiguous bytes: lane (g, c)
+        // covers columns 16c .. 16c + 15, product j taking 16c + 4j .. 16c +
+        // 4j + 3 as its k = 2c, 2c + 1, 2c + 8, 2c + 9.  A is X (batch rows
+        // g and g + 8, zero past the batch), B the tile rows.
 #pragma unroll
-      for (int b0 = 0; b0 < BP; b0 += C::XB) {
-        uint32_t xr[C::XB][8];
+        for (int kb = 0; kb < B2 / 64; ++kb) {
+          uint32_t xa[2][8];
 #pragma unroll
-        for (int b = 0; b < C::XB; ++b) {
-          const uint4 lo = *reinterpret_cast<const uint4 *>(xs + (b0 + b) * C::kXBatch + xo0);
-          const uint4 hi = *reinterpret_cast<const uint4 *>(xs + (b0 + b) * C::kXBatch + xo1);
-          xr[b][0] = lo.x;
-          xr[b][1] = lo.y;
-          xr[b][2] = lo.z;
-          xr[b][3] = lo.w;
-          xr[b][4] = hi.x;
-          xr[b][5] = hi.y;
-          xr[b][6] = hi.z;
-          xr[b][7] = hi.w;
-        }
-        if (sp) {
+          for (int h = 0; h < 2; ++h) {
+            const int b = mg + 8 * h;
+            if (b < BP) {
+              const uint8_t *xp = xs + b * C::kXBatch + (kb * 64 + 16 * mc) * 2;
+              const uint4 lo = *reinterpret_cast<const uint4 *>(xp);
+              const uint4 hi = *reinterpret_cast<const uint4 *>(xp + 16);
+              xa[h][0] = lo.x; xa[h][1] = lo.y; xa[h][2] = lo.z; xa[h][3] = lo.w;
+              xa[h][4] = hi.x; xa[h][5] = hi.y; xa[h][6] = hi.z; xa[h][7] = hi.w;
+            } else {
 #pragma unroll
-          for (int j = 0; j < C::JS; ++j) {
-            const int row = wrow + j * C::RPS + rs;
-            const uint4 v = *reinterpret_cast<const uint4 *>(st + voff + row * B2 + 16 * cp);
-            const uint32_t m = *reinterpret_cast<const uint16_t *>(
-                st + C::kValsBytes + moff + row * (B2 / 8) + 2 * cp);
-            const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-            if constexpr (PAT == 1) {
-              // 4:8: two groups of 8 columns, 4 kept each (c0 < c1 < c2 <
-              // c3); (v0, v1) meet x[c0], x[c1] and (v2, v3) x[c2], x[c3].
-              // As c0 <= 4, c1 <= 5, c2 >= 2 and c3 >= 3, each x pair comes
-              // from three of the group's four x registers in two PRMTs,
-              // with selectors from the mask byte's lut48 entry.
+              for (int q = 0; q < 8; ++q) xa[h][q] = 0u;
+            }
+          }
 #pragma unroll
-              for (int gb = 0; gb < 2; ++gb) {
-                const uint2 sl = lut48[(m >> (8 * gb)) & 0xFFu];
-                const uint32_t s1 = sl.x, s2 = sl.x >> 16, s3 = sl.y, s4 = sl.y >> 16;
+          for (int nb = 0; nb < NB; ++nb) {
+            const int row = wrow + 8 * nb + mg;
+            uint32_t wv[8];
+            if (sp) {
+              // 8 kept values (4 groups of 4 columns) and their 4 masks
+              const uint4 v = *reinterpret_cast<const uint4 *>(st + voff + row * B2 + kb * 64 +
+                                                              16 * mc);
+              const uint32_t m = *reinterpret_cast<const uint16_t *>(
+                  st + C::kValsBytes + moff + row * (B2 / 8) + kb * 8 + 2 * mc);
+              const uint32_t kv[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
-                for (int b = 0; b < C::XB; ++b) {
-                  const uint32_t *X4 = &xr[b][4 * gb];
-                  const uint32_t pa = __byte_perm(__byte_perm(X4[0], X4[1], s1), X4[2], s2);
-                  const uint32_t pb = __byte_perm(X4[1], __byte_perm(X4[2], X4[3], s3), s4);
-                  fma_bf16x2(acc[j][b0 + b], w[2 * gb], pa);
-                  fma_bf16x2(acc[j][b0 + b], w[2 * gb + 1], pb);
-                }
+              for (int q = 0; q < 4; ++q) {
+                const uint32_t sd = sel_dense[(m >> (4 * q)) & 0xFu];
+                wv[2 * q] = __byte_perm(kv[q], 0u, sd);
+                wv[2 * q + 1] = __byte_perm(kv[q], 0u, sd >> 16);
               }
             } else {
-              // 2:4: the PRMT selector of each group moves x[p0] to the low
-              // and x[p1] to the high half (p0 < p1 the kept columns).
-              // Narrow batches, where a selector serves one to four products,
-              // build it in registers: one PRMT looks up (p0, p1) of two
-              // groups at once in a byte table indexed by the low three bits
-              // of each 4-bit mask (distinct for the six masks with two bits
-              // set), a second PRMT expands them to byte pairs.  Wide batches
-              // take it from a 16-entry shared table (one load serves eight or
-              // sixteen products).
-              uint32_t selw[4];
-              if constexpr (BP <= 4) {
-                constexpr uint32_t kPairLo = 0x10313010u, kPairHi = 0x10212032u;
-                const uint32_t s01 = __byte_perm(kPairLo, kPairHi, m & 0x77u);
-                const uint32_t s23 = __byte_perm(kPairLo, kPairHi, (m >> 8) & 0x77u);
-                const uint32_t a01 = __byte_perm(0x76543210u, 0u, s01);
-                const uint32_t a23 = __byte_perm(0x76543210u, 0u, s23);
-                selw[0] = a01;
-                selw[1] = a01 >> 16;
-                selw[2] = a23;
-                selw[3] = a23 >> 16;
+              const uint8_t *wp = st + voff + row * 2 * B2 + (kb * 64 + 16 * mc) * 2;
+              const uint4 lo = *reinterpret_cast<const uint4 *>(wp);
+              const uint4 hi = *reinterpret_cast<const uint4 *>(wp + 16);
+              wv[0] = lo.x; wv[1] = lo.y; wv[2] = lo.z; wv[3] = lo.w;
+              wv[4] = hi.x; wv[5] = hi.y; wv[6] = hi.z; wv[7] = hi.w;
+            }
+#pragma unroll
+            for (int j = 0; j < 4; ++j)
+              mma_bf16_16816(dacc[nb], xa[0][2 * j], xa[1][2 * j], xa[0][2 * j + 1],
+                             xa[1][2 * j + 1], wv[2 * j], wv[2 * j + 1]);
+          }
+        }
+      } else {
+        const int xo0 = sp ? 32 * cp : 16 * cp;
+        const int xo1 = sp ? 32 * cp + 16 : B2 + 16 * cp;
+#pragma unroll
+        for (int b0 = 0; b0 < BP; b0 += C::XB) {
+          uint32_t xr[C::XB][8];
+#pragma unroll
+          for (int b = 0; b < C::XB; ++b) {
+            const uint4 lo = *reinterpret_cast<const uint4 *>(xs + (b0 + b) * C::kXBatch + xo0);
+            const uint4 hi = *reinterpret_cast<const uint4 *>(xs + (b0 + b) * C::kXBatch + xo1);
+            xr[b][0] = lo.x;
+            xr[b][1] = lo.y;
+            xr[b][2] = lo.z;
+            xr[b][3] = lo.w;
+            xr[b][4] = hi.x;
+            xr[b][5] = hi.y;
+            xr[b][6] = hi.z;
+            xr[b][7] = hi.w;
+          }
+          if (sp) {
+#pragma unroll
+            for (int j = 0; j < C::JS; ++j) {
+              const int row = wrow + j * C::RPS + rs;
+              const uint4 v = *reinterpret_cast<const uint4 *>(st + voff + row * B2 + 16 * cp);
+              const uint32_t m = *reinterpret_cast<const uint16_t *>(
+                  st + C::kValsBytes + moff + row * (B2 / 8) + 2 * cp);
+              const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+              if constexpr (PAT == 1) {
+                // 4:8: two groups of 8 columns, 4 kept each (c0 < c1 < c2 <
+                // c3); (v0, v1) meet x[c0], x[c1] and (v2, v3) x[c2], x[c3].
+                // As c0 <= 4, c1 <= 5, c2 >= 2 and c3 >= 3, each x pair comes
+                // from three of the group's four x registers in two PRMTs,
+                // with selectors from the mask byte's lut48 entry.
+#pragma unroll
+                for (int gb = 0; gb < 2; ++gb) {
+                  const uint2 sl = lut48[(m >> (8 * gb)) & 0xFFu];
+                  const uint32_t s1 = sl.x, s2 = sl.x >> 16, s3 = sl.y, s4 = sl.y >> 16;
+#pragma unroll
+                  for (int b = 0; b < C::XB; ++b) {
+                    const uint32_t *X4 = &xr[b][4 * gb];
+                    const uint32_t pa = __byte_perm(__byte_perm(X4[0], X4[1], s1), X4[2], s2);
+                    const uint32_t pb = __byte_perm(X4[1], __byte_perm(X4[2], X4[3], s3), s4);
+                    fma_bf16x2(acc[j][b0 + b], w[2 * gb], pa);
+                    fma_bf16x2(acc[j][b0 + b], w[2 * gb + 1], pb);
+                  }
+                }
               } else {
+                // 2:4: the PRMT selector of each group moves x[p0] to the low
+                // and x[p1] to the high half (p0 < p1 the kept columns).
+                // Narrow batches, where a selector serves one to four products,
+                // build it in registers: one PRMT looks up (p0, p1) of two
+                // groups at once in a byte table indexed by the low three bits
+                // of each 4-bit mask (distinct for the six masks with two bits
+                // set), a second PRMT expands them to byte pairs.  Wide batches
+                // take it from a 16-entry shared table (one load serves eight or
+                // sixteen products).
+                uint32_t selw[4];
+                if constexpr (BP <= 4) {
+                  constexpr uint32_t kPairLo = 0x10313010u, kPairHi = 0x10212032u;
+                  const uint32_t s01 = __byte_perm(kPairLo, kPairHi, m & 0x77u);
+                  const uint32_t s23 = __byte_perm(kPairLo, kPairHi, (m >> 8) & 0x77u);
+                  const uint32_t a01 = __byte_perm(0x76543210u, 0u, s01);
+                  const uint32_t a23 = __byte_perm(0x76543210u, 0u, s23);
+                  selw[0] = a01;
+                  selw[1] = a01 >> 16;
+                  selw[2] = a23;
+                  selw[3] = a23 >> 16;
+                } else {
 #pragma unroll
-                for (int g = 0; g < 4; ++g) selw[g] = sel_lut[(m >> (4 * g)) & 0xFu];
-              }
+                  for (int g = 0; g < 4; ++g) selw[g] = sel_lut[(m >> (4 * g)) & 0xFu];
+                }
 #pragma unroll
-              for (int g = 0; g < 4; ++g) {
-                const uint32_t sel = selw[g];
+                for (int g = 0; g < 4; ++g) {
+                  const uint32_t sel = selw[g];
 #pragma unroll
-                for (int b = 0; b < C::XB; ++b) {
-                  const uint32_t xp = __byte_perm(xr[b][2 * g], xr[b][2 * g + 1], sel);
-                  fma_bf16x2(acc[j][b0 + b], w[g], xp);
+                  for (int b = 0; b < C::XB; ++b) {
+                    const uint32_t xp = __byte_perm(xr[b][2 * g], xr[b][2 * g + 1], sel);
+                    fma_bf16x2(acc[j][b0 + b], w[g], xp);
+                  }
                 }
               }
             }
-          }
-        } else {
+          } else {
 #pragma unroll
-          for (int j = 0; j < C::JS; ++j) {
-            const int row = wrow + j * C::RPS + rs;
-            const uint4 a = *reinterpret_cast<const uint4 *>(st + voff + row * 2 * B2 + 16 * cp);
-            const uint4 c2 =
-                *reinterpret_cast<const uint4 *>(st + voff + row * 2 * B2 + B2 + 16 * cp);
-            const uint32_t w[8] = {a.x, a.y, a.z, a.w, c2.x, c2.y, c2.z, c2.w};
+            for (int j = 0; j < C::JS; ++j) {
+              const int row = wrow + j * C::RPS + rs;
+              const uint4 a = *reinterpret_cast<const uint4 *>(st + voff + row * 2 * B2 + 16 * cp);
+              const uint4 c2 =
+                  *reinterpret_cast<const uint4 *>(st + voff + row * 2 * B2 + B2 + 16 * cp);
+              const uint32_t w[8] = {a.x, a.y, a.z, a.w, c2.x, c2.y, c2.z, c2.w};
 #pragma unroll
-            for (int e = 0; e < 8; ++e)
+              for (int e = 0; e < 8; ++e)
 #pragma unroll
-              for (int b = 0; b < C::XB; ++b) fma_bf16x2(acc[j][b0 + b], w[e], xr[b][e]);
+                for (int b = 0; b < C::XB; ++b) fma_bf16x2(acc[j][b0 + b], w[e], xr[b][e]);
+            }
           }
         }
       }
@@ -1354,16 +1457,33 @@ __global__ void __launch_bounds__(TmaCfg<BP, B1, B2, LR>::kThreads, 1)
       break;
     }
     float *rows_s = s_rows[slot][warp];
+    if constexpr (C::MMA) {
 #pragma unroll
-    for (int j = 0; j < C::JS; ++j)
+      for (int nb = 0; nb < NB; ++nb) {
+        const int r0 = 8 * nb + 2 * mc;
+        if (mg < BP) {
+          rows_s[mg * C::RW + r0] = dacc[nb][0];
+          rows_s[mg * C::RW + r0 + 1] = dacc[nb][1];
+        }
+        if (mg + 8 < BP) {
+          rows_s[(mg + 8) * C::RW + r0] = dacc[nb][2];
+          rows_s[(mg + 8) * C::RW + r0 + 1] = dacc[nb][3];
+        }
 #pragma unroll
-      for (int b = 0; b < BP; ++b) {
-        float v = acc[j][b];
-#pragma unroll
-        for (int o = 1; o < C::CPR; o <<= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-        if (cp == 0) rows_s[b * C::RW + j * C::RPS + rs] = v;
-        acc[j][b] = 0.f;
+        for (int q = 0; q < 4; ++q) dacc[nb][q] = 0.f;
       }
+    } else {
+#pragma unroll
+      for (int j = 0; j < C::JS; ++j)
+#pragma unroll
+        for (int b = 0; b < BP; ++b) {
+          float v = acc[j][b];
+#pragma unroll
+          for (int o = 1; o < C::CPR; o <<= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+          if (cp == 0) rows_s[b * C::RW + j * C::RPS + rs] = v;
+          acc[j][b] = 0.f;
+        }
+    }
     __syncwarp();
     if (lane == 0) mbar_arrive(&piece_full[slot]);
     ++piece;
@@ -1401,7 +1521,7 @@ __global__ void __launch_bounds__(128)
   uint32_t bits = 0;
   const int nw = (int)min((int64_t)31, t1 - t0);
   for (int i = 0; i < nw; ++i) bits |= (uint32_t)(map[t0 + i] == 1) << i;
-  const uint32_t starts = nw > 0 ? stage_starts(bits, nw, t0, tpr, tpd, 2 * tpd) : 0u;
+  const uint32_t starts = nw > 0 ? stage_starts(bits, nw, (uint32_t)(t0 % tpr), tpr, tpd, 2 * tpd) : 0u;
   int64_t *rec = plan + kPlanHead + 4 * (int64_t)c;
   rec[0] = t0;
   rec[1] = val_off[t0];
@@ -1727,7 +1847,7 @@ struct TmaKernel {
 
 template <int BP, int B1, int B2, int PAT, bool LR = false>
 TmaKernel tma_kernel_info() {
-  using C = TmaCfg<BP, B1, B2, LR>;
+  using C = TmaCfg<BP, B1, B2, LR, PAT>;
   return TmaKernel{reinterpret_cast<void *>(&hybrid_tma_kernel<BP, B1, B2, PAT, LR>), C::kThreads,
                    C::kSmem, C::kStageBytes, C::kStages, C::TPX, C::XTM, C::XT * B2, BP};
 }
@@ -1914,7 +2034,8 @@ int make_plan(int64_t n, int64_t k, int b1, int b2, int64_t total_bytes,
   int rc = device_sm_count(&sms);
   if (rc != HYB_OK) return rc;
   (void)strided;  // packed and row-major matrices take the same kernels
-  P.tma = s != kGeneric;
+  // (tile indices are 32-bit in the streaming kernel's band arithmetic)
+  P.tma = s != kGeneric && (n / b1) * (k / b2) < (int64_t(1) << 31);
   // A low-rank term rides in the streaming kernel for narrow batches, where
   // it is a few percent more bytes and little arithmetic; for batch 8 and 16
   // its arithmetic (2 batch r (n + k) flops) is better spread over the whole
