@@ -56,6 +56,18 @@ WORKLOADS = {
     "ffn_down_4096x14336_f1.0_b4": (4096, 14336, 128, 128, 1.0, 4, 0.02, 0.01),
     "ffn_down_4096x14336_f1.0_b16": (4096, 14336, 128, 128, 1.0, 16, 0.02, 0.01),
     "ffn_down_4096x14336_f0.0_b16": (4096, 14336, 128, 128, 0.0, 16, 0.02, 0.01),
+    # Llama-3.3-70B FFN matrices, all 2:4, with a low-rank term (rank below)
+    "llama70b_down_8192x28672_lr128_b1": (8192, 28672, 128, 128, 1.0, 1, 0.015, 0.0),
+    "llama70b_gate_28672x8192_lr128_b1": (28672, 8192, 128, 128, 1.0, 1, 0.015, 0.0),
+    "llama70b_down_8192x28672_lr64_b1": (8192, 28672, 128, 128, 1.0, 1, 0.015, 0.0),
+    "llama70b_down_8192x28672_lr128_b4": (8192, 28672, 128, 128, 1.0, 4, 0.015, 0.0),
+}
+# workloads with a low-rank term y += U (V^T x): name -> (rank, std of U and V)
+LOWRANK = {
+    "llama70b_down_8192x28672_lr128_b1": (128, 0.01),
+    "llama70b_gate_28672x8192_lr128_b1": (128, 0.01),
+    "llama70b_down_8192x28672_lr64_b1": (64, 0.01),
+    "llama70b_down_8192x28672_lr128_b4": (128, 0.01),
 }
 
 
@@ -203,6 +215,7 @@ class Workload:
         Wd = W.to(device)
         base = hyb.pack(Wd, tmap, b1, b2)
         self.frac_real = float(tmap.mean())
+        rotate = rotation(name, tmap, rotate)
         self.mats = [base] + [base.clone() for _ in range(rotate - 1)]
         self.dense = [Wd] + [Wd.clone() for _ in range(rotate - 1)]
         # the same W packed with every tile dense, streamed by the same kernel:
@@ -213,7 +226,16 @@ class Workload:
                   for i in range(rotate)]
         self.Y = [torch.empty(batch, n, dtype=torch.float32, device=device)
                   for _ in range(rotate)]
-        self.ws = hyb.new_workspace(hyb.workspace_bytes(base, batch), device)
+        self.rank, lr_std = LOWRANK.get(name, (0, 0.0))
+        self.U_host = self.V_host = None
+        self.lr = None
+        if self.rank:
+            self.U_host, self.V_host = inputs.lowrank(n, k, self.rank, lr_std,
+                                                      inputs.seed_of(name, "LR"))
+            self.U, self.V = self.U_host.to(device), self.V_host.to(device)
+            self.lr = hyb.HybLowrank(self.rank, hyb._bits(self.U).data_ptr(), self.rank,
+                                     hyb._bits(self.V).data_ptr(), self.rank)
+        self.ws = hyb.new_workspace(hyb.workspace_bytes(base, batch, self.rank), device)
         self.dws = hyb.new_workspace(hyb.dense_workspace_bytes(n, k, batch), device)
         # pre-marshalled C-ABI arguments (the timed loop only calls into C)
         L = hyb.lib()
@@ -225,7 +247,9 @@ class Workload:
         self.stream = torch.cuda.current_stream(device)
         self.set_stream(self.stream)
         # algorithmic bytes of one product: packed values + masks, tile map, x, y
-        self.bytes_step = base.nbytes() + base.num_tiles + 2 * batch * k + 4 * batch * n
+        # (and U, V for a low-rank term)
+        self.bytes_step = (base.nbytes() + base.num_tiles + 2 * batch * k + 4 * batch * n
+                           + 2 * self.rank * (n + k))
         self.dense_bytes_step = 2 * n * k + 2 * batch * k + 4 * batch * n
 
     def set_stream(self, stream):
@@ -234,8 +258,9 @@ class Workload:
         n, k, batch = self.n, self.k, self.batch
         rotate = len(self.mats)
         f = self.flags
+        lr = ctypes.byref(self.lr) if self.lr is not None else None
         self.args = [(ctypes.byref(self.structs[i]), batch, ctypes.c_void_p(self.X[i].data_ptr()),
-                      k, ctypes.c_void_p(self.Y[i].data_ptr()), n, hyb.HYB_F32, None, f,
+                      k, ctypes.c_void_p(self.Y[i].data_ptr()), n, hyb.HYB_F32, lr, f,
                       ctypes.c_void_p(self.ws.data_ptr()), self.ws.numel(), s)
                      for i in range(rotate)]
         self.pargs = [(ctypes.byref(self.dstructs[i]), batch,
@@ -371,7 +396,7 @@ def e2e_timed(wl, steps, warmup, stream, world=1):
 # CPU oracle timing (reported baseline)
 # ---------------------------------------------------------------------------
 
-def oracle_sample(wl_name, W_host, tmap, rows_per_step=256, threads=1):
+def oracle_sample(wl_name, W_host, tmap, rows_per_step=256, threads=1, U=None, V=None):
     """A bounded sample of the workload for the CPU oracle: the fp64 hybrid
     product of `rows_per_step` output rows (selection applied on the fly),
     split over `threads` host threads (the oracle's C routine runs without the
@@ -382,6 +407,9 @@ def oracle_sample(wl_name, W_host, tmap, rows_per_step=256, threads=1):
     o = oracle.Oracle()
     n, k, b1, b2, frac, batch, std, outliers = WORKLOADS[wl_name]
     Wb = inputs.bits(W_host)
+    Ub = inputs.bits(U) if U is not None else None
+    Vb = inputs.bits(V) if V is not None else None
+    rank = 0 if U is None else U.shape[1]
     X = inputs.bits(inputs.activations(batch, k, inputs.seed_of(wl_name, "X", 0)))
     rng = np.random.default_rng(0)
     sparse_frac = float(np.mean(tmap))
@@ -391,11 +419,13 @@ def oracle_sample(wl_name, W_host, tmap, rows_per_step=256, threads=1):
     def step(i):
         rows = np.sort(rng.choice(n, rows_per_step, replace=False)).astype(np.int64)
         if pool is None:
-            o.rows(Wb, b1, b2, tmap, X, rows)
+            o.rows(Wb, b1, b2, tmap, X, rows, U=Ub, V=Vb)
             return
         parts = np.array_split(rows, threads)
-        list(pool.map(lambda r: o.rows(Wb, b1, b2, tmap, X, r), parts))
-    return step, bytes_per_row * rows_per_step + 2 * batch * k + 4 * batch * rows_per_step
+        list(pool.map(lambda r: o.rows(Wb, b1, b2, tmap, X, r, U=Ub, V=Vb), parts))
+    # (each sampled step recomputes V^T x: its V bytes count once per step)
+    return step, (bytes_per_row + 2 * rank) * rows_per_step + 2 * batch * k \
+        + 4 * batch * rows_per_step + 2 * rank * k
 
 
 def host_cores():
@@ -409,7 +439,7 @@ def host_cores():
 def _cpu_leg(wl, threads, budget_s):
     rows = 256 * threads
     step, nbytes = oracle_sample(wl.name, wl.W_host, wl.tmap, rows_per_step=rows,
-                                 threads=threads)
+                                 threads=threads, U=wl.U_host, V=wl.V_host)
     step(0)
     t0 = time.perf_counter()
     reps = 0
@@ -442,7 +472,12 @@ def run_reference(args, world, rank):
     W, tmap = make_matrix(name)
     cores = host_cores()
     rows = 256 * cores
-    step, nbytes = oracle_sample(name, W, tmap, rows_per_step=rows, threads=cores)
+    rank, lr_std = LOWRANK.get(name, (0, 0.0))
+    U = V = None
+    if rank:
+        n, k = WORKLOADS[name][:2]
+        U, V = inputs.lowrank(n, k, rank, lr_std, inputs.seed_of(name, "LR"))
+    step, nbytes = oracle_sample(name, W, tmap, rows_per_step=rows, threads=cores, U=U, V=V)
     for i in range(args.warmup):
         step(i)
     t0 = time.perf_counter()
@@ -456,7 +491,9 @@ def run_reference(args, world, rank):
         "value": round(value, 4), "unit": "GB/s", "n_gpus": args.gpus, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(dt * 1e3 / args.steps, 4),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-        "data": "synthetic", "config": workload_config(name, frac_real=float(np.mean(tmap))),
+        "data": "synthetic",
+        "config": workload_config(name, float(np.mean(tmap)), rotation(name, tmap),
+                                  packed_bytes(name, tmap)),
         "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": cores,
                          "kind": "oracle",
                          "sample": f"oracle_rows_f64 (fp64) on {rows} random output rows of "
@@ -472,7 +509,6 @@ def run_reference(args, world, rank):
 # --sweep: the other measurements (one JSON line each, not the headline)
 # ---------------------------------------------------------------------------
 
-FP32_FMA_PER_SM_PER_CLK = 128   # fp32 lanes per SM (B200)
 
 
 class Calls:
@@ -502,12 +538,20 @@ class Calls:
             raise hyb.HybError(self.name, rc)
 
 
-def _alu_roofline(flops, us, sm_mhz):
-    peak = 148 * FP32_FMA_PER_SM_PER_CLK * 2 * sm_mhz * 1e6 / 1e12  # TFLOP/s
-    achieved = flops / (us * 1e-6) / 1e12
-    return {"bound": "alu", "achieved": round(achieved, 2), "peak": round(peak, 1),
-            "unit": "TFLOP/s", "frac": round(achieved / peak, 4),
-            "peak_kind": f"148 SMs x 128 fp32 lanes x 2 x {sm_mhz:.0f} MHz"}
+def _tensor_roofline(n, k, us):
+    """Batch >= 4 products run on the tensor cores (bf16 m16n8k16, batch
+    padded to 16 rows, 2:4 tiles expanded to dense): issued tensor FLOPs per
+    second against the measured dense bf16 peak.  A small fraction means the
+    product is not bound by tensor throughput."""
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as fh:
+            peak, kind = float(json.load(fh)["bf16_tflops"]), "measured"
+    except Exception:
+        peak, kind = 1590.0, "fallback"
+    achieved = 2 * 16 * n * k / (us * 1e-6) / 1e12
+    return {"bound": "tensor", "achieved": round(achieved, 2), "peak": peak, "unit": "TFLOP/s",
+            "frac": round(achieved / peak, 4), "peak_kind": f"{kind} cuBLAS bf16 (burst)",
+            "issued": "2 x 16 x n x k per product (mma.sync m16n8k16 bf16 -> fp32)"}
 
 
 def sweep(device, steps=200, warmup=10):
@@ -585,8 +629,8 @@ def sweep(device, steps=200, warmup=10):
                         "format_bound_speedup": round((2 * n * k) / base.nbytes(), 4),
                         "plain_launch": {"us": round(us_plain, 3),
                                          "dense_us": round(dense_plain_us[b], 3)}}
-                if b >= 8:
-                    line["alu_roofline"] = _alu_roofline(2 * b * kept, us, sm_mhz)
+                if b >= 4:
+                    line["tensor_roofline"] = _tensor_roofline(n, k, us)
                 emit(line)
                 del ws
             del mats, structs, base
@@ -641,28 +685,37 @@ def sweep(device, steps=200, warmup=10):
     torch.cuda.empty_cache()
 
     # ---- Llama-3.3-70B FFN, all 2:4, rank-128 low-rank term, 8 layers ----
-    mats70, lrs, sh70 = [], [], []
+    mats70, sh70 = [], []
     for role, n, k in inputs.LLAMA70B_FFN:
         T = (n // 128) * (k // 128)
         W = inputs.weight(n, k, 0.015, inputs.seed_of("llama70b", role, "W")).to(device)
         base = hyb.pack(W, np.ones(T, np.uint8), 128, 128)
         del W
-        U, V = inputs.lowrank(n, k, 128, 0.01, inputs.seed_of("llama70b", role, "LR"))
-        lr = (U.to(device), V.to(device))
         for layer in range(8):
             mats70.append(base if layer == 0 else base.clone())
-            lrs.append(lr)
             sh70.append((n, k))
     mats70 = [mats70[(i % 3) * 8 + i // 3] for i in range(24)]
-    lrs = [lrs[(i % 3) * 8 + i // 3] for i in range(24)]
     sh70 = [sh70[(i % 3) * 8 + i // 3] for i in range(24)]
     structs = [m.struct() for m in mats70]
-    lrstructs = [hyb.HybLowrank(128, hyb._bits(U).data_ptr(), 128, hyb._bits(V).data_ptr(), 128)
-                 for U, V in lrs]
-    for b in (1, 8, 16):
+    for rank, batches in ((128, (1, 4, 8, 16)), (64, (1,))):
+        lr_by_role = {}
+        for role, n, k in inputs.LLAMA70B_FFN:
+            U, V = inputs.lowrank(n, k, rank, 0.01, inputs.seed_of("llama70b", role, "LR", rank))
+            lr_by_role[(n, k)] = (U.to(device), V.to(device))
+        lrs = [lr_by_role[sh] for sh in sh70]
+        lrstructs = [hyb.HybLowrank(rank, hyb._bits(U).data_ptr(), rank,
+                                    hyb._bits(V).data_ptr(), rank) for U, V in lrs]
+        _sweep_70b(L, structs, lrstructs, mats70, sh70, rank, batches, device, peak, emit, sm_mhz)
+        del lrs, lrstructs, lr_by_role
+    return 0
+
+
+def _sweep_70b(L, structs, lrstructs, mats70, sh70, rank, batches, device, peak, emit, sm_mhz):
+    OV = hyb.LAUNCH_OVERLAP_PREV
+    for b in batches:
         xs = [inputs.activations(b, k, inputs.seed_of("l70", i, b)).to(device) for i, (n, k) in enumerate(sh70)]
         ys = [torch.empty(b, n, dtype=torch.float32, device=device) for n, k in sh70]
-        ws = hyb.new_workspace(max(hyb.workspace_bytes(m, b, 128) for m in mats70), device)
+        ws = hyb.new_workspace(max(hyb.workspace_bytes(m, b, rank) for m in mats70), device)
         c = Calls(L.hyb_spmm_skinny_ex, lambda i, sp, b=b, ws=ws, xs=xs, ys=ys: (
             ctypes.byref(structs[i]), b, ctypes.c_void_p(xs[i].data_ptr()), sh70[i][1],
             ctypes.c_void_p(ys[i].data_ptr()), sh70[i][0], hyb.HYB_F32, ctypes.byref(lrstructs[i]),
@@ -671,26 +724,26 @@ def sweep(device, steps=200, warmup=10):
         us = ms / 2 * 1e3
         us_plain = graph_timed(c, c.step, 48, 24) / 2 * 1e3
         hyb.check_status(ws)
-        nbytes = sum(m.nbytes() + m.num_tiles + 2 * b * k + 4 * b * n + 2 * 128 * (n + k)
+        nbytes = sum(m.nbytes() + m.num_tiles + 2 * b * k + 4 * b * n + 2 * rank * (n + k)
                      for m, (n, k) in zip(mats70, sh70))
         gbs = nbytes / (us * 1e-6) / 1e9
-        line = {"sweep": "llama70b_ffn_lowrank", "matrices": 24, "batch": b, "rank": 128,
+        line = {"sweep": "llama70b_ffn_lowrank", "matrices": 24, "batch": b, "rank": rank,
+                "lowrank_path": "fused into the streaming kernel" if b <= 4
+                                else "three kernels (V^T x, U t, product)",
                 "us_per_8_layers": round(us, 2), "us_per_matrix": round(us / 24, 3),
                 "GBps": round(gbs, 1), "frac_of_measured_hbm": round(gbs / peak, 4),
                 "plain_launch": {"us_per_8_layers": round(us_plain, 2)}}
-        if b >= 8:
-            kept = sum(m.n_vals for m in mats70)
-            flops = 2 * b * kept + sum(2 * b * 128 * (n + k) for n, k in sh70)
-            line["alu_roofline"] = _alu_roofline(flops, us, sm_mhz)
+        if b >= 4:
+            line["tensor_roofline"] = _tensor_roofline(sum(n * k for n, k in sh70), 1, us)
         emit(line)
         del ws, xs, ys
-    return 0
 
 
 def sweep_nm(device, steps=200, warmup=10):
-    """General N:M tiles (hyb_spmm_skinny_nm, one warp per output row): the
-    4096x14336 down projection with 4:8 tiles at three fractions, batch 1 and 8,
-    graph replay of rotating copies (larger than L2)."""
+    """General N:M tiles (hyb_spmm_skinny_nm; 4:8 runs in the streaming
+    kernel): the 4096x14336 down projection with 4:8 tiles at three
+    fractions, batch 1 and 8, graph replay of rotating copies (larger than
+    L2)."""
     peak, _ = measured_peak()
     L = hyb.lib()
     n, k, b1, b2, nk, m = 4096, 14336, 128, 128, 4, 8
@@ -718,20 +771,41 @@ def sweep_nm(device, steps=200, warmup=10):
                               "tile": f"{b1}x{b2}", "sparse_tile_frac": float(np.mean(tmap)),
                               "batch": b, "us": round(us, 3), "GBps": round(gbs, 1),
                               "frac_of_measured_hbm": round(gbs / peak, 4),
-                              "kernel": "spmm_nm_kernel (one warp per output row)"}), flush=True)
+                              "kernel": "hybrid_tma_kernel (4:8 tiles: mask-byte PRMT "
+                                        "selectors, scalar fp32 FMAs)"}), flush=True)
         hyb.check_status(ws)
         del mats, structs, base
         torch.cuda.empty_cache()
     return 0
 
 
-def workload_config(name, frac_real):
+def packed_bytes(name, tmap):
+    """Packed values + masks of the workload's matrix (the format's closed form)."""
+    n, k, b1, b2 = WORKLOADS[name][:4]
+    s = int(np.sum(tmap == 1))
+    return (len(tmap) - s) * 2 * b1 * b2 + s * (b1 * b2 + b1 * b2 // 8)
+
+
+def rotation(name, tmap, rotate=ROTATE):
+    """Packed copies cycled through: a matrix larger than L2 needs only a few
+    to stay cold."""
+    nb = packed_bytes(name, tmap)
+    if nb > (126 << 20):
+        rotate = min(rotate, max(2, int(np.ceil(3 * (126 << 20) / nb))))
+    return rotate
+
+
+def workload_config(name, frac_real, rot, nbytes):
     n, k, b1, b2, frac, batch, std, outliers = WORKLOADS[name]
-    return {"workload": name, "n": n, "k": k, "tile": f"{b1}x{b2}",
-            "sparse_tile_frac": round(frac_real, 4), "batch": batch,
-            "weights": f"bf16 N(0,{std})" + (f" with {outliers:.0%} x20 outliers" if outliers else ""),
-            "l2": f"inputs larger than L2: {ROTATE} rotating packed copies (1.47 GB)",
-            "parallelism": "replicas"}
+    cfg = {"workload": name, "n": n, "k": k, "tile": f"{b1}x{b2}",
+           "sparse_tile_frac": round(frac_real, 4), "batch": batch,
+           "weights": f"bf16 N(0,{std})" + (f" with {outliers:.0%} x20 outliers" if outliers else ""),
+           "l2": f"inputs larger than L2: {rot} rotating packed copies ({rot * nbytes / 1e9:.2f} GB)",
+           "parallelism": "replicas"}
+    rank = LOWRANK.get(name, (0, 0.0))[0]
+    if rank:
+        cfg["lowrank"] = {"rank": rank, "U": f"bf16 [{n}][{rank}]", "V": f"bf16 [{k}][{rank}]"}
+    return cfg
 
 
 # ---------------------------------------------------------------------------
@@ -819,7 +893,7 @@ def main():
         "value": round(value, 2), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(per_step_ms, 6), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": workload_config(args.workload, wl.frac_real),
+        "config": workload_config(wl.name, wl.frac_real, len(wl.mats), wl.mats[0].nbytes()),
         "us_per_matrix": round(per_step_ms * 1e3, 3),
         "launch": "CUDA graph of the K steps, each a programmatic dependent of the one "
                   "before (HYB_LAUNCH_OVERLAP_PREV)",
@@ -841,9 +915,15 @@ def main():
                      "bytes_per_launch": wl.bytes_step},
         "e2e": {"value": round(aggregate_gbs(wl.bytes_step, args.steps, e2e_ms, world), 2),
                 "unit": "GB/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
-        "gpu_launches": args.steps,
+        "consumer": ("tensor cores (bf16 m16n8k16, batch padded to 16, fp32 accumulate)"
+                     if wl.batch >= 4 else "scalar fp32 FMAs (PRMT-selected x pairs)"),
+        "lowrank_path": (None if not wl.rank else "fused into the streaming kernel"
+                         if wl.batch <= 4 else "three kernels (V^T x, U t, product)"),
+        "gpu_launches": args.steps * (1 if wl.rank == 0 or wl.batch <= 4 else 3),
         "clocks": clocks.summary(),
     }
+    if wl.batch >= 4:
+        line["tensor_roofline"] = _tensor_roofline(wl.n, wl.k, per_step_ms * 1e3)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(wl)
     if world > 1:

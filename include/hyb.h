@@ -215,14 +215,43 @@ HYB_API int hyb_spmm_skinny(const hyb_matrix *A, int batch, const uint16_t *X,
  * never more than the SMs and there is one per SM, so all of them can be
  * resident.  If other work on the GPU kept some of them from starting for
  * seconds, the wait runs out and hyb_check_status reports HYB_ERR_TIMEOUT.
- * Other tilings run three kernels (V^T x, U t, the product) one after
- * another; the flag applies to the first. */
+ * Batches of 8 and 16, and other tilings, run three kernels (V^T x, U t,
+ * the product) one after another; the flag applies to the first. */
 
 /* hyb_spmm_skinny with launch options `flags` (0 = hyb_spmm_skinny). */
 HYB_API int hyb_spmm_skinny_ex(const hyb_matrix *A, int batch, const uint16_t *X,
                                int64_t ldx, void *Y, int64_t ldy, hyb_dtype ydt,
                                const hyb_lowrank *lr, uint32_t flags, void *ws,
                                size_t ws_bytes, hyb_stream_t stream);
+
+/* ---- gate and up projections sharing one low-rank factor V ---------------
+ * 3BASiL §1-§2: a weight is approximated by S + L with L = U V^T of
+ * rank r.  The gate and up projections of an FFN
+ * read the same input x; when their low-rank terms share V, t = V^T x is one
+ * vector for both:
+ *     Yg = Ag X + Ug (V^T X),   Yu = Au X + Uu (V^T X)
+ * (X [batch][k] bf16, row stride ldx; Yg [batch][Ag->n] and Yu [batch][Au->n]
+ * with row strides ldyg, ldyu, in ydt).  lr_g gives the rank, Ug (ldu) and V
+ * (ldv); Uu ([Au->n][rank] bf16, row stride lduu) is the up projection's U.
+ * The gate product runs as hyb_spmm_skinny_ex would and leaves t in its part
+ * of the workspace; the up product then computes only Uu t (no second pass
+ * over V, no second V^T x reduction).  Ag->k must equal Au->k.  Yg is
+ * bit-identical to a hyb_spmm_skinny_ex call with (Ug, V); Yu differs from a
+ * call with (Uu, V) only by the rounding of t, which the gate product reduces
+ * over its own split of k (identical when both products split over the same
+ * number of CTAs, and always for batches above 4).
+ * flags: as for hyb_spmm_skinny_ex (the up product is a programmatic
+ * dependent of the gate product when HYB_LAUNCH_OVERLAP_PREV is set).
+ * Workspace: at least hyb_gate_up_workspace_bytes(Ag, Au, batch, rank) bytes,
+ * 256-byte aligned; errors as hyb_spmm_skinny. */
+HYB_API size_t hyb_gate_up_workspace_bytes(const hyb_matrix *Ag, const hyb_matrix *Au,
+                                           int batch, int rank);
+HYB_API int hyb_spmm_skinny_gate_up(const hyb_matrix *Ag, const hyb_matrix *Au, int batch,
+                                    const uint16_t *X, int64_t ldx, void *Yg, int64_t ldyg,
+                                    void *Yu, int64_t ldyu, hyb_dtype ydt,
+                                    const hyb_lowrank *lr_g, const uint16_t *Uu, int64_t lduu,
+                                    uint32_t flags, void *ws, size_t ws_bytes,
+                                    hyb_stream_t stream);
 
 /* Workspace bytes for hyb_lowrank_add. */
 HYB_API size_t hyb_lowrank_workspace_bytes(int64_t k, int batch, int rank);

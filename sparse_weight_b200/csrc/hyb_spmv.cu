@@ -75,6 +75,9 @@ struct Params {
   int rank;
   int fused_lr;
   float *lr_t;
+  // t computed by an earlier call that shares V (gate and up of one input):
+  // the fused low-rank warp, or the call's kernels, then compute U t only
+  const float *lr_t_in;
   float *lr_ut;
   float *lr_part;
   uint32_t *lr_epoch;
@@ -954,7 +957,7 @@ __global__ void __launch_bounds__(TmaCfg<BP, B1, B2, LR, PAT>::kThreads, 1)
     // (1) partial t over rows [k0, k1) of V, multiples of 8 so that the X
     // rows' copies start on 16-byte boundaries; a chunk holds rc rows of V
     // and the same rows of X for four batch columns
-    {
+    if (!p.lr_t_in) {  // V^T x here (else t comes from an earlier call)
       const int64_t k8 = p.k / 8;
       const int64_t k0 = 8 * (k8 * c / G), k1 = 8 * (k8 * (c + 1) / G);
       const int rc = max(8, (kLrHalf / (2 * r + 2 * 4)) / 8 * 8);
@@ -1018,38 +1021,41 @@ __global__ void __launch_bounds__(TmaCfg<BP, B1, B2, LR, PAT>::kThreads, 1)
         }
       }
     }
-    __syncwarp();
-    if (ok) ok = flag_barrier(p.lr_flags, G, c, epoch + 1u, lane);
-    if (ok) {
-      // 8 lanes per element, each adding the partials of CTAs sub, sub + 8,
-      // ... in order (all loads issued first); the 8 sums then combined by a
-      // fixed xor tree
-      const int64_t e0 = E * c / G, e1 = E * (c + 1) / G;
-      const int sub = lane % 8;
-      constexpr int QL = 10;  // partials per lane in flight (two rounds cover 160 CTAs)
-      for (int64_t eb = e0; eb < e1; eb += 4) {
-        const int64_t e = eb + lane / 8;
-        float a = 0.f;
+    if (!p.lr_t_in) {
+      __syncwarp();
+      if (ok) ok = flag_barrier(p.lr_flags, G, c, epoch + 1u, lane);
+      if (ok) {
+        // 8 lanes per element, each adding the partials of CTAs sub, sub + 8,
+        // ... in order (all loads issued first); the 8 sums then combined by a
+        // fixed xor tree
+        const int64_t e0 = E * c / G, e1 = E * (c + 1) / G;
+        const int sub = lane % 8;
+        constexpr int QL = 10;  // partials per lane in flight (two rounds cover 160 CTAs)
+        for (int64_t eb = e0; eb < e1; eb += 4) {
+          const int64_t e = eb + lane / 8;
+          float a = 0.f;
 #pragma unroll 1
-        for (int q0 = 0; q0 < G; q0 += 8 * QL) {
-          float v[QL];
+          for (int q0 = 0; q0 < G; q0 += 8 * QL) {
+            float v[QL];
 #pragma unroll
-          for (int q = 0; q < QL; ++q) {
-            const int cq = q0 + sub + 8 * q;
-            v[q] = (e < e1 && cq < G) ? __ldcg(p.lr_part + (int64_t)cq * E + e) : 0.f;
+            for (int q = 0; q < QL; ++q) {
+              const int cq = q0 + sub + 8 * q;
+              v[q] = (e < e1 && cq < G) ? __ldcg(p.lr_part + (int64_t)cq * E + e) : 0.f;
+            }
+#pragma unroll
+            for (int q = 0; q < QL; ++q) a += v[q];
           }
-#pragma unroll
-          for (int q = 0; q < QL; ++q) a += v[q];
+          a += __shfl_xor_sync(full, a, 1);
+          a += __shfl_xor_sync(full, a, 2);
+          a += __shfl_xor_sync(full, a, 4);
+          if (e < e1 && sub == 0) __stcg(p.lr_t + e, a);
         }
-        a += __shfl_xor_sync(full, a, 1);
-        a += __shfl_xor_sync(full, a, 2);
-        a += __shfl_xor_sync(full, a, 4);
-        if (e < e1 && sub == 0) __stcg(p.lr_t + e, a);
+        ok = flag_barrier(p.lr_flags, G, c, epoch + 2u, lane);
       }
-      ok = flag_barrier(p.lr_flags, G, c, epoch + 2u, lane);
     }
     if (ok) {
       // (3) U t for rows [i0, i1); a chunk holds rc3 rows of U
+      const float *tsrc = p.lr_t_in ? p.lr_t_in : p.lr_t;
       const int64_t i0 = p.n * c / G, i1 = p.n * (c + 1) / G;
       const int rc3 = kLrHalf / (2 * r);
       const int nch = (int)((i1 - i0 + rc3 - 1) / rc3);
@@ -1060,7 +1066,7 @@ __global__ void __launch_bounds__(TmaCfg<BP, B1, B2, LR, PAT>::kThreads, 1)
         for (int b = 0; b < LB; ++b)
 #pragma unroll
           for (int e = 0; e < 8; ++e)
-            tv[b][e] = active ? __ldcg(p.lr_t + (b0 + b) * r + 8 * chunk + e) : 0.f;
+            tv[b][e] = active ? __ldcg(tsrc + (b0 + b) * r + 8 * chunk + e) : 0.f;
         auto issue = [&](int j, uint8_t *dst) {
           const int64_t row0 = i0 + (int64_t)j * rc3;
           const int rows = (int)min((int64_t)rc3, i1 - row0);
@@ -2214,7 +2220,7 @@ void fill_launch_plan(const int64_t *plan, int32_t plan_ctas, const Plan &P, con
 int run_product(Params prm, int b1, int b2, int batch, const hyb_lowrank *lr,
                 bool strided, void *ws, size_t ws_bytes, cudaStream_t s,
                 const int64_t *plan = nullptr, int32_t plan_ctas = 0, uint32_t flags = 0,
-                int pat = 0) {
+                int pat = 0, const float *t_in = nullptr, const float **t_out = nullptr) {
   const int rank = (lr && lr->rank > 0) ? lr->rank : 0;
   Plan P;
   int rc = make_plan(prm.n, prm.k, b1, b2, prm.total, batch, rank, strided, &P, pat);
@@ -2236,6 +2242,8 @@ int run_product(Params prm, int b1, int b2, int batch, const hyb_lowrank *lr,
   prm.lr_part = reinterpret_cast<float *>(w + P.off_lr_part);
   prm.lr_epoch = reinterpret_cast<uint32_t *>(w + kLowrankEpochOffset);
   prm.lr_flags = reinterpret_cast<uint32_t *>(w + kLowrankFlagsOffset);
+  prm.lr_t_in = rank ? t_in : nullptr;
+  if (t_out) *t_out = rank && !t_in ? prm.lr_t : nullptr;
   prm.lr_ut = nullptr;
   prm.fused_lr = 0;
   const bool overlap = (flags & HYB_LAUNCH_OVERLAP_PREV) != 0;
@@ -2248,12 +2256,14 @@ int run_product(Params prm, int b1, int b2, int batch, const hyb_lowrank *lr,
     // launched one after the other (the first as a programmatic dependent
     // with the caller's overlap flag; the one-warp-per-row product ignores
     // the flag)
-    rc = launch_lowrank_t(P, lr, prm.k, prm.X, prm.ldx, batch, w, s, overlap);
-    if (rc != HYB_OK) return rc;
+    if (!t_in) {
+      rc = launch_lowrank_t(P, lr, prm.k, prm.X, prm.ldx, batch, w, s, overlap);
+      if (rc != HYB_OK) return rc;
+    }
     int64_t nn = prm.n, ldu = lr->ldu;
     const uint16_t *U = lr->U;
     int rk = rank, bt = batch;
-    const float *tp = prm.lr_t;
+    const float *tp = t_in ? t_in : prm.lr_t;
     float *ut = reinterpret_cast<float *>(w + P.off_lr_ut);
     int zero = 0;
     void *uargs[] = {&nn, &U, &ldu, &rk, &tp, &bt, &ut, &zero};
@@ -2315,7 +2325,8 @@ int check_io(const uint16_t *X, int64_t ldx, void *Y, int64_t ldy, int64_t n,
 
 int spmm_impl(const hyb_matrix *A, int batch, const uint16_t *X, int64_t ldx,
               void *Y, int64_t ldy, hyb_dtype ydt, const hyb_lowrank *lr,
-              void *ws, size_t ws_bytes, cudaStream_t s, uint32_t flags = 0, int pat = 0) {
+              void *ws, size_t ws_bytes, cudaStream_t s, uint32_t flags = 0, int pat = 0,
+              const float *t_in = nullptr, const float **t_out = nullptr) {
   if (!A) return HYB_ERR_INVALID_ARG;
   if (flags & ~HYB_LAUNCH_OVERLAP_PREV) return HYB_ERR_INVALID_ARG;
   int rc = check_tiling(A->n, A->k, A->b1, A->b2);
@@ -2353,7 +2364,7 @@ int spmm_impl(const hyb_matrix *A, int batch, const uint16_t *X, int64_t ldx,
   prm.nvb = 2 * A->n_vals;
   prm.nmb = A->n_meta_bytes;
   return run_product(prm, A->b1, A->b2, batch, lr, false, ws, ws_bytes, s, A->plan,
-                     A->plan_ctas, flags, pat);
+                     A->plan_ctas, flags, pat, t_in, t_out);
 }
 
 // Virtual tiling of a plain row-major W for the dense baseline.
@@ -2474,6 +2485,42 @@ int hyb_spmm_skinny_ex(const hyb_matrix *A, int batch, const uint16_t *X, int64_
                        uint32_t flags, void *ws, size_t ws_bytes, hyb_stream_t stream) {
   return spmm_impl(A, batch, X, ldx, Y, ldy, ydt, lr, ws, ws_bytes, (cudaStream_t)stream,
                    flags);
+}
+
+size_t hyb_gate_up_workspace_bytes(const hyb_matrix *Ag, const hyb_matrix *Au, int batch,
+                                   int rank) {
+  if (rank < 1) return 0;
+  const size_t a = hyb_workspace_bytes(Ag, batch, rank);
+  const size_t b = hyb_workspace_bytes(Au, batch, rank);
+  if (a == 0 || b == 0) return 0;
+  return (a + 255) / 256 * 256 + b;
+}
+
+int hyb_spmm_skinny_gate_up(const hyb_matrix *Ag, const hyb_matrix *Au, int batch,
+                            const uint16_t *X, int64_t ldx, void *Yg, int64_t ldyg, void *Yu,
+                            int64_t ldyu, hyb_dtype ydt, const hyb_lowrank *lr_g,
+                            const uint16_t *Uu, int64_t lduu, uint32_t flags, void *ws,
+                            size_t ws_bytes, hyb_stream_t stream) {
+  if (!Ag || !Au || !lr_g || lr_g->rank < 1 || !Uu) return HYB_ERR_INVALID_ARG;
+  if (Ag->k != Au->k) return HYB_ERR_INVALID_ARG;  // one input x for both
+  const hyb_lowrank lr_u{lr_g->rank, Uu, lduu, lr_g->V, lr_g->ldv};
+  int rc = check_lowrank(&lr_u, Au->n, Au->k);
+  if (rc != HYB_OK) return rc;
+  const size_t need = hyb_gate_up_workspace_bytes(Ag, Au, batch, lr_g->rank);
+  if (need == 0) return HYB_ERR_INVALID_ARG;
+  if (!ws || ws_bytes < need) return HYB_ERR_WORKSPACE;
+  const size_t wa = (hyb_workspace_bytes(Ag, batch, lr_g->rank) + 255) / 256 * 256;
+  uint8_t *w = static_cast<uint8_t *>(ws);
+  cudaStream_t s = (cudaStream_t)stream;
+  // gate: the full product, which leaves t = V^T x in its workspace
+  const float *t = nullptr;
+  rc = hyb::spmm_impl(Ag, batch, X, ldx, Yg, ldyg, ydt, lr_g, w, wa, s, flags, 0, nullptr, &t);
+  if (rc != HYB_OK) return rc;
+  if (!t) return HYB_ERR_CUDA;
+  // up: the same t, only U_up t (launched after the gate product on the
+  // stream; as a programmatic dependent when the caller asked for overlap)
+  return hyb::spmm_impl(Au, batch, X, ldx, Yu, ldyu, ydt, &lr_u, w + wa, ws_bytes - wa, s,
+                        flags, 0, t, nullptr);
 }
 
 size_t hyb_lowrank_workspace_bytes(int64_t k, int batch, int rank) {

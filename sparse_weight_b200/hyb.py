@@ -68,7 +68,8 @@ EXPORTS = ["hyb_packed_sizes", "hyb_pack_workspace_bytes", "hyb_pack",
            "hyb_spmm_skinny", "hyb_lowrank_workspace_bytes", "hyb_lowrank_add",
            "hyb_dense_workspace_bytes", "hyb_gemv_dense", "hyb_check_status",
            "hyb_status_string", "hyb_spmv_noalloc", "hyb_spmv_noalloc_max_scratch_bytes",
-           "hyb_spmv_noalloc_check_status",
+           "hyb_spmv_noalloc_check_status", "hyb_gate_up_workspace_bytes",
+           "hyb_spmm_skinny_gate_up",
            "hyb_plan_entries", "hyb_make_plan", "hyb_selftest_wait_timeout",
            "hyb_spmm_skinny_ex", "hyb_gemv_dense_ex", "hyb_packed_sizes_nm",
            "hyb_pack_nm", "hyb_spmm_skinny_nm"]
@@ -102,6 +103,14 @@ def lib():
     L.hyb_spmm_skinny_ex.argtypes = [ctypes.POINTER(HybMatrix), _I, _P, _I64, _P, _I64, _I,
                                      ctypes.POINTER(HybLowrank), ctypes.c_uint32, _P, _SZ, _P]
     L.hyb_spmm_skinny_ex.restype = _I
+    L.hyb_gate_up_workspace_bytes.argtypes = [ctypes.POINTER(HybMatrix), ctypes.POINTER(HybMatrix),
+                                              _I, _I]
+    L.hyb_gate_up_workspace_bytes.restype = _SZ
+    L.hyb_spmm_skinny_gate_up.argtypes = [ctypes.POINTER(HybMatrix), ctypes.POINTER(HybMatrix), _I,
+                                          _P, _I64, _P, _I64, _P, _I64, _I,
+                                          ctypes.POINTER(HybLowrank), _P, _I64, ctypes.c_uint32,
+                                          _P, _SZ, _P]
+    L.hyb_spmm_skinny_gate_up.restype = _I
     L.hyb_lowrank_workspace_bytes.argtypes = [_I64, _I, _I]
     L.hyb_lowrank_workspace_bytes.restype = _SZ
     L.hyb_lowrank_add.argtypes = [_I64, _I64, _I, ctypes.POINTER(HybLowrank), _P, _I64,
@@ -413,6 +422,34 @@ def spmm_skinny(A: Packed, X: torch.Tensor, Y: torch.Tensor = None, ydt: int = H
         ctypes.byref(s), batch, _ptr(Xb), Xb.stride(0), _ptr(Y), Y.stride(0), ydt,
         ctypes.byref(lr) if lr else None, flags, _ptr(ws), ws.numel(), _stream(stream)))
     return Y
+
+
+def gate_up_workspace_bytes(Ag: Packed, Au: Packed, batch: int, rank: int) -> int:
+    sg, su = Ag.struct(), Au.struct()
+    return int(lib().hyb_gate_up_workspace_bytes(ctypes.byref(sg), ctypes.byref(su), batch, rank))
+
+
+def spmm_skinny_gate_up(Ag: Packed, Au: Packed, X: torch.Tensor, Ug: torch.Tensor,
+                        Uu: torch.Tensor, V: torch.Tensor, ydt: int = HYB_F32,
+                        ws: torch.Tensor = None, stream=None, flags: int = 0):
+    """hyb_spmm_skinny_gate_up: (Yg, Yu) = (Ag X + Ug (V^T X), Au X + Uu (V^T X))
+    with V^T X computed once; X bf16 [batch][k]."""
+    Xb = _bits(X)
+    if Xb.dim() == 1:
+        Xb = Xb.view(1, -1)
+    batch = Xb.shape[0]
+    Yg = _out(Ag.n, batch, ydt, Xb.device, None)
+    Yu = _out(Au.n, batch, ydt, Xb.device, None)
+    lr, keep = _lowrank_struct((Ug, V))
+    Uub = _bits(Uu)
+    if ws is None:
+        ws = new_workspace(gate_up_workspace_bytes(Ag, Au, batch, lr.rank), Xb.device)
+    sg, su = Ag.struct(), Au.struct()
+    _check("hyb_spmm_skinny_gate_up", lib().hyb_spmm_skinny_gate_up(
+        ctypes.byref(sg), ctypes.byref(su), batch, _ptr(Xb), Xb.stride(0), _ptr(Yg),
+        Yg.stride(0), _ptr(Yu), Yu.stride(0), ydt, ctypes.byref(lr), _ptr(Uub), Uub.stride(0),
+        flags, _ptr(ws), ws.numel(), _stream(stream)))
+    return Yg, Yu
 
 
 def spmv(A: Packed, x: torch.Tensor, y: torch.Tensor = None, ydt: int = HYB_F32,

@@ -186,6 +186,36 @@ def test_llama8b_layer_full_size(orc):
         assert_within(Y[:, rows], y_ref, env, what=f"llama8b {role}")
 
 
+def test_llama8b_chain_every_layer(orc):
+    """The 32-layer chain as the bench runs it: one weight draw per role, the
+    tile map drawn per layer at that layer's fraction, all 224 matrices
+    packed at full size and each product checked on sampled rows (the first
+    two bands' edges, the middle, the last band's edges and six seeded random
+    rows per matrix)."""
+    Wr = {role: inputs.weight(n, k, 0.02, inputs.seed_of("llama8b_chain", role, "W"))
+          for role, n, k in inputs.LLAMA8B_LAYER}
+    Wd = {role: W.to(dev()) for role, W in Wr.items()}
+    Wb = {role: inputs.bits(W) for role, W in Wr.items()}
+    checked = 0
+    for layer in range(32):
+        f = inputs.chain_fraction(layer)
+        for role, n, k in inputs.LLAMA8B_LAYER:
+            T = (n // 128) * (k // 64)
+            tmap = inputs.tile_map_fraction(T, f, inputs.seed_of("llama8b_chain", layer, role,
+                                                                  "map"))
+            X = inputs.activations(1, k, inputs.seed_of("chain_parity", layer, role))
+            P = hyb.pack(Wd[role], tmap, 128, 64)
+            # the realised 2:4-tile fraction is the layer's (exact count by seeded shuffle)
+            assert int(tmap.sum()) == round(f * T)
+            rows = _sampled_rows(n, 128, 6, layer)
+            Y = hyb.spmv(P, X.to(dev())).cpu().numpy()
+            y_ref, env = orc.rows(Wb[role], 128, 64, tmap, inputs.bits(X), rows)
+            assert_within(Y[:, rows], y_ref, env, what=f"llama8b layer {layer} {role} f={f:.3f}")
+            checked += 1
+            del P
+    assert checked == 224
+
+
 def test_llama70b_ffn_lowrank_full_size(orc):
     """All-2:4 70B-shaped FFN plus rank-128 low-rank term, fused; batch {1,8,16}."""
     for role, n, k in inputs.LLAMA70B_FFN:
@@ -245,6 +275,49 @@ def test_lowrank_fused_repeated_calls(orc):
         y_ref, env = orc.spmv(n, k, b1, b2, tmap, ref, inputs.bits(X), inputs.bits(U),
                               inputs.bits(V))
         assert_within(Y.cpu().numpy(), y_ref, env, what=f"repeated r={U.shape[1]}")
+
+
+@pytest.mark.parametrize("batch", [1, 3, 8, 16])
+@pytest.mark.parametrize("shape", [(1024, 2048, 128, 128), (1536, 1024, 128, 64)])
+def test_gate_up_shared_lowrank(orc, batch, shape):
+    """Gate and up projections of one input with one shared V (3BASiL §1:
+    W ~ S + U V^T; the same x, so the same V^T x): each output within the
+    oracle's tolerance of (S + U V^T) x; the gate output bit-identical to a
+    separate call, the up output too where a separate up call would reduce t
+    over the same split (same CTA count, or the three-kernel path of batch 8
+    and 16, whose V^T x split depends on k only).  Batch <= 4 takes the fused
+    path."""
+    n, k, b1, b2 = shape
+    T = (n // b1) * (k // b2)
+    rank = 64
+    Wg, tg, X, _ = case(n, k, b1, b2, inputs.tile_map_bernoulli(
+        T, 0.5, inputs.seed_of("gateup", "g", n)), batch=batch, name="gateup_g")
+    Wu, tu, _, _ = case(n, k, b1, b2, inputs.tile_map_bernoulli(
+        T, 0.5, inputs.seed_of("gateup", "u", n)), batch=batch, name="gateup_u")
+    Ug, V = inputs.lowrank(n, k, rank, 0.01, inputs.seed_of("gateup", "lr_g", n))
+    Uu, _ = inputs.lowrank(n, k, rank, 0.01, inputs.seed_of("gateup", "lr_u", n))
+    Pg = hyb.pack(Wg.to(dev()), tg, b1, b2)
+    Pu = hyb.pack(Wu.to(dev()), tu, b1, b2)
+    Xd, Ugd, Uud, Vd = X.to(dev()), Ug.to(dev()), Uu.to(dev()), V.to(dev())
+    ws = hyb.new_workspace(hyb.gate_up_workspace_bytes(Pg, Pu, batch, rank), dev())
+    Yg, Yu = hyb.spmm_skinny_gate_up(Pg, Pu, Xd, Ugd, Uud, Vd, ws=ws)
+    # a second time on the same workspace, as a chain of layers would
+    Yg2, Yu2 = hyb.spmm_skinny_gate_up(Pg, Pu, Xd, Ugd, Uud, Vd, ws=ws,
+                                       flags=hyb.LAUNCH_OVERLAP_PREV)
+    Yg_sep = hyb.spmm_skinny(Pg, Xd, lowrank=(Ugd, Vd))
+    Yu_sep = hyb.spmm_skinny(Pu, Xd, lowrank=(Uud, Vd))
+    torch.cuda.synchronize()
+    assert hyb.check_status(ws) == 0
+    assert torch.equal(Yg, Yg_sep)
+    if batch > 4 or Pg.plan_ctas == Pu.plan_ctas:
+        # t reduced over the same split as in a separate up call
+        assert torch.equal(Yu, Yu_sep)
+    assert torch.equal(Yg, Yg2) and torch.equal(Yu, Yu2)
+    for W, tmap, U, Y, nm in ((Wg, tg, Ug, Yg, "gate"), (Wu, tu, Uu, Yu, "up")):
+        ref = orc.pack(inputs.bits(W), b1, b2, tmap)
+        y_ref, env = orc.spmv(n, k, b1, b2, tmap, ref, inputs.bits(X), inputs.bits(U),
+                              inputs.bits(V))
+        assert_within(Y.cpu().numpy(), y_ref, env, what=f"gate/up shared LR {nm} b={batch}")
 
 
 def _tile_split_reference(P, G):
