@@ -224,6 +224,27 @@ HYB_API int hyb_spmm_skinny_ex(const hyb_matrix *A, int batch, const uint16_t *X
                                const hyb_lowrank *lr, uint32_t flags, void *ws,
                                size_t ws_bytes, hyb_stream_t stream);
 
+/* ---- prefill / large batch on the tensor cores ---------------------------
+ * Y[m][i] = sum_k W_hat[i][k] X[m][k] for a block of M tokens (PATCH: dense
+ * tiles on dense tensor-core kernels, 2:4 tiles on sparse ones, §2 Method):
+ * one tcgen05 pipeline per 128-row band and 128-token block, fp32
+ * accumulators in tensor memory, the tile's operands moved by TMA (dense
+ * tiles as 128-byte-swizzled boxes; a 2:4 tile's kept values and masks
+ * staged and expanded to the dense layout in shared memory, so its tensor
+ * work is a dense tile's while its bytes are the hybrid format's).
+ *   A: 128 x 128 tiles (HYB_ERR_UNSUPPORTED otherwise), k <= 131072.
+ *   X: [m][k] bf16, row stride ldx (>= k, multiple of 8), 16-byte aligned;
+ *      m >= 1 (any; the last block's missing tokens read as zeros).
+ *   Y: [m][n] fp32, row stride ldy >= n, 4-byte aligned; written, not
+ *      accumulated.
+ *   ws: at least hyb_prefill_workspace_bytes() bytes, 256-byte aligned, its
+ *      status word zeroed before the first call (hyb_check_status reads and
+ *      clears it).  Nothing is allocated.  Asynchronous on `stream`. */
+HYB_API size_t hyb_prefill_workspace_bytes(void);
+HYB_API int hyb_spmm_prefill(const hyb_matrix *A, int64_t m, const uint16_t *X, int64_t ldx,
+                             float *Y, int64_t ldy, void *ws, size_t ws_bytes,
+                             hyb_stream_t stream);
+
 /* ---- gate and up projections sharing one low-rank factor V ---------------
  * 3BASiL §1-§2: a weight is approximated by S + L with L = U V^T of
  * rank r.  The gate and up projections of an FFN

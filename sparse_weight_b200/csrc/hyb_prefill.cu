@@ -1,0 +1,442 @@
+// hyb_spmm_prefill: a hybrid (dense | 2:4) weight times a tall block of
+// activations on the 5th-generation tensor cores,
+//
+//     Y[m][i] = sum_k W_hat[i][k] X[m][k]     (m < M tokens, i < n rows)
+//
+// the prefill / large-batch form of the product.  PATCH ("PATCH: Learnable
+// Tile-level Hybrid Sparsity for LLMs", §2 Method) runs its dense tiles on
+// dense tensor-core kernels and its 2:4 tiles on the sparse tensor cores; here
+// both kinds of tile feed one tcgen05 pipeline:
+//
+//   * CTA (band r, token block mb) owns Y[128 mb .. +128][128 r .. +128]: a
+//     128 x 128 fp32 accumulator in tensor memory (TMEM), M = 128 weight rows,
+//     N = 128 tokens, K looped over the band's tiles (128 columns each).
+//   * warp 0 (one lane) moves each tile's operands with TMA: a dense tile as
+//     two 2-D boxes of 64 columns x 128 rows with 128-byte swizzle (the
+//     K-major layout tcgen05.mma reads), X as two such boxes of the token
+//     block; a 2:4 tile's kept values and masks as plain bulk copies into a
+//     staging buffer.
+//   * warps 4-7 expand a staged 2:4 tile into the same swizzled dense layout
+//     (thread i: row i; kept pairs placed by the mask nibble, zeros
+//     elsewhere), fence it for the async proxy and signal the MMA warp.
+//   * warp 1 owns the TMEM allocation; one lane issues 8 tcgen05.mma
+//     (kind::f16, bf16 x bf16 -> fp32, K = 16 each) per tile and frees the
+//     stage with tcgen05.commit.
+//   * warps 4-7 then read the accumulator with tcgen05.ld (warp w: TMEM lanes
+//     32 (w % 4) ..) and store Y (a warp writes 32 consecutive rows of one
+//     token: 128 contiguous bytes).
+//
+// 2:4 tiles take the dense MMA after expansion: the weight bytes moved are
+// the hybrid format's, the tensor work is that of a dense tile.  (The sparse
+// MMA, tcgen05.mma.sp, needs its metadata in a TMEM layout of its own; it is
+// not used.)  Every wait is bounded; one that runs out sets kStatusTimeout in
+// the status word and the CTA leaves its pipeline.
+#include "hyb_internal.cuh"
+
+namespace hyb {
+namespace {
+
+constexpr int kPM = 128;                      // weight rows per CTA (b1), MMA M
+constexpr int kPN = 128;                      // tokens per CTA, MMA N
+constexpr int kPK = 128;                      // columns per tile (b2)
+constexpr int kAtomBytes = 128 * 128;         // 128 rows x 128 bytes (64 bf16), swizzled
+constexpr int kABytes = 2 * kAtomBytes;       // a dense tile: two 64-column atoms
+constexpr int kXBytes = 2 * kAtomBytes;       // 128 tokens x 128 columns
+constexpr int kSValBytes = kPM * kPK;         // 2:4 staging: kept values (bf16)
+constexpr int kSMetaBytes = kPM * kPK / 8;    // and masks
+constexpr int kStageBytes = kABytes + kXBytes + kSValBytes + kSMetaBytes;  // 82 KB
+constexpr int kPStages = 2;
+constexpr int kPThreads = 256;
+constexpr int kTmemCols = 128;                // fp32 accumulator columns (= kPN)
+constexpr int kMaxBandTiles = 1024;           // tiles per band (k <= 131072)
+static_assert(kStageBytes % 1024 == 0, "stages keep the 1024-byte swizzle alignment");
+
+// tcgen05.mma instruction descriptor: D fp32, A and B bf16, both K-major,
+// N = kPN, M = kPM (bit layout of the sm_100 instruction descriptor).
+constexpr uint32_t kIdesc = (1u << 4)                     // D format: f32
+                            | (1u << 7)                   // A format: bf16
+                            | (1u << 10)                  // B format: bf16
+                            | ((uint32_t)(kPN >> 3) << 17)  // N / 8
+                            | ((uint32_t)(kPM >> 4) << 24);  // M / 16
+
+// Shared-memory matrix descriptor of a K-major operand in the 128-byte
+// swizzle layout: rows 128 bytes apart, 8-row groups 1024 bytes apart
+// (stride byte offset), descriptor version 1, layout type 2 (128B swizzle).
+__device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr) {
+  uint64_t d = (uint64_t)((saddr >> 4) & 0x3FFFu);
+  d |= (uint64_t)1 << 16;             // leading byte offset (unused by swizzled K-major)
+  d |= (uint64_t)(1024 >> 4) << 32;   // stride byte offset
+  d |= (uint64_t)1 << 46;             // version
+  d |= (uint64_t)2 << 61;             // 128-byte swizzle
+  return d;
+}
+
+__device__ __forceinline__ void umma_bf16(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc,
+                                          uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %3, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %4, p;\n\t}" ::"r"(tmem_d),
+      "l"(adesc), "l"(bdesc), "r"(accumulate), "r"(kIdesc)
+      : "memory");
+}
+// arrives on the mbarrier once every tcgen05.mma this thread issued before
+// has completed
+__device__ __forceinline__ void umma_commit(uint64_t *bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::
+                   "r"(smem_u32(bar))
+               : "memory");
+}
+__device__ __forceinline__ void tc_fence_after() {
+  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_before() {
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+// 16 consecutive fp32 columns of this thread's TMEM lane
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, float (&v)[16]) {
+  uint32_t r[16];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, "
+      "%11, %12, %13, %14, %15}, [%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+        "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr));
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+  for (int q = 0; q < 16; ++q) v[q] = __uint_as_float(r[q]);
+}
+
+struct PrefillParams {
+  const uint8_t *map;
+  const uint16_t *vals;
+  const uint8_t *meta;
+  const int64_t *val_off;
+  const int64_t *meta_off;
+  int64_t n, k, m;
+  int tpr;
+  int64_t nvb, nmb;  // bytes of the value and mask buffers
+  float *Y;
+  int64_t ldy;
+  uint32_t *status;
+};
+
+__global__ void __launch_bounds__(kPThreads, 1)
+    hybrid_prefill_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap xmap,
+                          const __grid_constant__ CUtensorMap wmap) {
+  extern __shared__ uint8_t smem_raw[];
+  __shared__ __align__(8) uint64_t full_bar[kPStages];
+  __shared__ __align__(8) uint64_t empty_bar[kPStages];
+  // a 2:4 tile's staging copy landed / the tile has been expanded: their
+  // phases advance only on the 2:4 uses of a stage (the MMA warp takes the
+  // tiles in order and waits for every expansion, so neither barrier ever
+  // runs two phases ahead of a thread waiting on it)
+  __shared__ __align__(8) uint64_t sfull_bar[kPStages];
+  __shared__ __align__(8) uint64_t exp_bar[kPStages];
+  __shared__ __align__(8) uint64_t acc_bar;
+  __shared__ uint32_t s_tmem;
+  __shared__ uint32_t sel_dense[16];
+  __shared__ uint8_t s_map[kMaxBandTiles];
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int r = blockIdx.x;                  // tile-row band
+  const int64_t m0 = (int64_t)blockIdx.y * kPN;  // first token
+  const int tpr = p.tpr;
+  // stages at a 1024-byte boundary (the swizzle pattern repeats every 1024)
+  uint8_t *smem =
+      smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+
+  if (tid == 0) {
+    for (int s = 0; s < kPStages; ++s) {
+      mbar_init(&full_bar[s], 1);
+      mbar_init(&empty_bar[s], 1);
+      mbar_init(&sfull_bar[s], 1);
+      mbar_init(&exp_bar[s], 128);
+    }
+    mbar_init(&acc_bar, 1);
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  if (tid < 16) {
+    // PRMT selectors expanding a kept pair (v_p0 in bytes 0-1, v_p1 in bytes
+    // 2-3, zero bytes 4-7) to the group's columns 0-1 (low half) and 2-3
+    // (high half), p0 < p1 the mask's set bits; a column not kept gets zeros
+    const uint32_t msk = tid;
+    const int p0 = msk ? __ffs(msk) - 1 : -1, p1 = msk ? 31 - __clz(msk) : -1;
+    uint32_t sd = 0;
+    for (int j = 0; j < 4; ++j) {
+      const uint32_t lo = j == p0 ? 0u : (j == p1 ? 2u : 4u);
+      const uint32_t hi = lo == 4u ? 4u : lo + 1u;
+      sd |= (lo | hi << 4) << (8 * j);
+    }
+    sel_dense[msk] = sd;
+  }
+  for (int j = tid; j < tpr; j += kPThreads) s_map[j] = p.map[(int64_t)r * tpr + j];
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                     smem_u32(&s_tmem)),
+                 "r"(kTmemCols)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = s_tmem;
+
+  if (warp == 0) {
+    // ------------------------------ producer ------------------------------
+    // lane l holds the offsets of tile w0 + l of the band (a window of 32,
+    // the next window loaded while this one is issued)
+    bool ok = true;
+    const int64_t t_band = (int64_t)r * tpr;
+    auto load = [&](int w0, int64_t &vo, int64_t &mo) {
+      vo = mo = 0;
+      if (w0 + lane < tpr) {
+        vo = __ldg(p.val_off + t_band + w0 + lane);
+        mo = __ldg(p.meta_off + t_band + w0 + lane);
+      }
+    };
+    int64_t vo, mo, nvo, nmo;
+    load(0, vo, mo);
+    for (int w0 = 0; w0 < tpr && ok; w0 += 32) {
+      load(w0 + 32, nvo, nmo);
+      const int nw = min(32, tpr - w0);
+      for (int l = 0; l < nw && ok; ++l) {
+        const int j = w0 + l;
+        const int s = j % kPStages;
+        const uint32_t ph = (uint32_t)(j / kPStages) & 1u;
+        const int64_t tvo = __shfl_sync(0xffffffffu, vo, l);
+        const int64_t tmo = __shfl_sync(0xffffffffu, mo, l);
+        if (lane == 0) {
+          if (!mbar_wait(&empty_bar[s], ph ^ 1u)) {
+            ok = false;
+          } else {
+            uint8_t *st = smem + (size_t)s * kStageBytes;
+            uint8_t *xs = st + kABytes;
+            const bool sp = s_map[j] == 1;
+            // a range outside the buffers (a corrupted matrix) is not copied
+            const bool fits = sp ? (tvo >= 0 && tmo >= 0 && 2 * tvo + kSValBytes <= p.nvb &&
+                                    tmo + kSMetaBytes <= p.nmb && ((2 * tvo) | tmo) % 16 == 0)
+                                 : (tvo >= 0 && 2 * tvo + kABytes <= p.nvb && tvo % kPK == 0);
+            if (!fits) atomicOr(p.status, kStatusBadMap);
+            const uint32_t abytes = fits && !sp ? (uint32_t)kABytes : 0u;
+            mbar_arrive_expect_tx(&full_bar[s], (uint32_t)kXBytes + abytes);
+            // X: tokens m0 .. m0 + 127 (rows past M read as zeros), columns of tile j
+            tma_load_2d(xs, &xmap, j * kPK, (int)m0, &full_bar[s]);
+            tma_load_2d(xs + kAtomBytes, &xmap, j * kPK + 64, (int)m0, &full_bar[s]);
+            if (fits && !sp) {
+              const int row = (int)(tvo / kPK);  // the tile's first row in the 128-wide view
+              tma_load_2d(st, &wmap, 0, row, &full_bar[s]);
+              tma_load_2d(st + kAtomBytes, &wmap, 64, row, &full_bar[s]);
+            } else if (fits) {
+              uint8_t *sv = st + kABytes + kXBytes;
+              mbar_arrive_expect_tx(&sfull_bar[s], (uint32_t)(kSValBytes + kSMetaBytes));
+              bulk_g2s(sv, p.vals + tvo, kSValBytes, &sfull_bar[s]);
+              bulk_g2s(sv + kSValBytes, p.meta + tmo, kSMetaBytes, &sfull_bar[s]);
+            } else if (sp) {
+              mbar_arrive(&sfull_bar[s]);  // nothing copied: the expansion reads stale bytes
+            }
+          }
+        }
+        ok = __shfl_sync(0xffffffffu, ok, 0);
+      }
+      vo = nvo;
+      mo = nmo;
+    }
+    if (!ok && lane == 0) atomicOr(p.status, kStatusTimeout);
+  } else if (warp == 1) {
+    // ------------------------------- MMA --------------------------------
+    bool ok = true;
+    uint32_t exp_ph = 0;  // bit s: parity of stage s's expansion barrier
+    for (int j = 0; j < tpr && ok; ++j) {
+      const int s = j % kPStages;
+      const uint32_t ph = (uint32_t)(j / kPStages) & 1u;
+      if (lane == 0) {
+        const bool sp = s_map[j] == 1;
+        ok = mbar_wait(&full_bar[s], ph);
+        if (ok && sp) {
+          ok = mbar_wait(&exp_bar[s], (exp_ph >> s) & 1u);
+          exp_ph ^= 1u << s;
+        }
+        if (ok) {
+          tc_fence_after();
+          const uint32_t a0 = smem_u32(smem + (size_t)s * kStageBytes);
+          const uint32_t b0 = a0 + kABytes;
+#pragma unroll
+          for (int kb = 0; kb < 2; ++kb)
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk) {
+              // K = 16 columns (32 bytes) at a time inside the 128-byte row
+              const uint32_t off = kb * kAtomBytes + kk * 32;
+              umma_bf16(tmem, sw128_desc(a0 + off), sw128_desc(b0 + off),
+                        (j | kb | kk) != 0 ? 1u : 0u);
+            }
+          umma_commit(&empty_bar[s]);
+        }
+      }
+      ok = __shfl_sync(0xffffffffu, ok, 0);
+    }
+    if (lane == 0) {
+      if (!ok) atomicOr(p.status, kStatusTimeout);
+      // the accumulator is final once every MMA issued above has completed
+      // (also after a timeout, so that nothing is in flight at the end)
+      umma_commit(&acc_bar);
+      if (!mbar_wait(&acc_bar, 0u)) atomicOr(p.status, kStatusTimeout);
+    }
+    __syncwarp();
+  } else if (warp >= 4) {
+    // ------------------- 2:4 expansion, then the epilogue -------------------
+    const int i = tid - 128;  // tile row
+    bool ok = true;
+    uint32_t sp_ph = 0;  // bit s: parity of stage s's next 2:4 use
+    for (int j = 0; j < tpr && ok; ++j) {
+      const int s = j % kPStages;
+      if (s_map[j] != 1) continue;
+      if (!mbar_wait(&sfull_bar[s], (sp_ph >> s) & 1u)) {
+        ok = false;
+        break;
+      }
+      sp_ph ^= 1u << s;
+      uint8_t *st = smem + (size_t)s * kStageBytes;
+      const uint8_t *sv = st + kABytes + kXBytes + i * (kPK);            // 64 kept bf16
+      const uint4 mv = *reinterpret_cast<const uint4 *>(st + kABytes + kXBytes + kSValBytes +
+                                                         i * (kPK / 8));  // 32 mask nibbles
+#pragma unroll
+      for (int q = 0; q < 8; ++q) {
+        // piece pc: groups 4pc .. 4pc + 3 = columns 16pc .. 16pc + 15 (rotated
+        // by row so that the 8 rows of a load phase hit different banks)
+        const int pc = (q + i) & 7;
+        const uint4 v = *reinterpret_cast<const uint4 *>(sv + 16 * pc);
+        const uint32_t w01 = (pc & 2) ? mv.y : mv.x, w23 = (pc & 2) ? mv.w : mv.z;
+        const uint32_t m16 = (((pc & 4) ? w23 : w01) >> (16 * (pc & 1))) & 0xFFFFu;
+        const uint32_t kv[4] = {v.x, v.y, v.z, v.w};
+        uint32_t w[8];
+#pragma unroll
+        for (int g = 0; g < 4; ++g) {
+          const uint32_t sd = sel_dense[(m16 >> (4 * g)) & 0xFu];
+          w[2 * g] = __byte_perm(kv[g], 0u, sd);
+          w[2 * g + 1] = __byte_perm(kv[g], 0u, sd >> 16);
+        }
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          const int c = 2 * pc + h;  // 16-byte chunk of the dense row (8 columns)
+          uint8_t *dst = st + (c >> 3) * kAtomBytes + i * 128 + (((c & 7) ^ (i & 7)) << 4);
+          *reinterpret_cast<uint4 *>(dst) =
+              make_uint4(w[4 * h], w[4 * h + 1], w[4 * h + 2], w[4 * h + 3]);
+        }
+      }
+      // generic-proxy writes, read next by tcgen05.mma (async proxy)
+      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+      mbar_arrive(&exp_bar[s]);
+    }
+    if (!ok && lane == 0) atomicOr(p.status, kStatusTimeout);
+    // epilogue: TMEM lanes 32 (warp % 4) .. + 31 are this warp's weight rows
+    if (mbar_wait(&acc_bar, 0u)) {
+      tc_fence_after();
+      const int q = warp & 3;
+      const int64_t row = (int64_t)r * kPM + 32 * q + lane;
+#pragma unroll 1
+      for (int c0 = 0; c0 < kPN; c0 += 16) {
+        float v[16];
+        tmem_ld16(tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)c0, v);
+#pragma unroll
+        for (int jj = 0; jj < 16; ++jj) {
+          const int64_t tok = m0 + c0 + jj;
+          if (tok < p.m) p.Y[tok * p.ldy + row] = v[jj];
+        }
+      }
+    } else if (lane == 0) {
+      atomicOr(p.status, kStatusTimeout);
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem),
+                 "r"(kTmemCols)
+                 : "memory");
+  }
+}
+
+// 2-D tensor map, bf16, 128-byte swizzle, box 64 columns x 128 rows.
+int encode_sw128(const void *base, uint64_t cols, uint64_t rows, uint64_t row_bytes,
+                 CUtensorMap *map) {
+  PFN_cuTensorMapEncodeTiled_v12000 encode = tensor_map_encoder();
+  if (!encode) return HYB_ERR_CUDA;
+  const cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+  const cuuint64_t strides[1] = {(cuuint64_t)row_bytes};
+  const cuuint32_t box[2] = {64, 128};
+  const cuuint32_t estr[2] = {1, 1};
+  const CUresult res =
+      encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides,
+             box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return res == CUDA_SUCCESS ? HYB_OK : HYB_ERR_CUDA;
+}
+
+}  // namespace
+}  // namespace hyb
+
+using namespace hyb;
+
+size_t hyb_prefill_workspace_bytes(void) { return kHeaderBytes; }
+
+int hyb_spmm_prefill(const hyb_matrix *A, int64_t m, const uint16_t *X, int64_t ldx, float *Y,
+                     int64_t ldy, void *ws, size_t ws_bytes, hyb_stream_t stream) {
+  if (!A || !X || !Y || m < 1) return HYB_ERR_INVALID_ARG;
+  if (A->b1 != kPM || A->b2 != kPK) return HYB_ERR_UNSUPPORTED;
+  if (A->n <= 0 || A->k <= 0 || A->n % kPM != 0 || A->k % kPK != 0)
+    return HYB_ERR_INVALID_ARG;
+  const int64_t tpr = A->k / kPK;
+  if (tpr > kMaxBandTiles || A->n / kPM > INT32_MAX || (m + kPN - 1) / kPN > 65535)
+    return HYB_ERR_UNSUPPORTED;
+  if (A->num_tiles != (A->n / kPM) * tpr) return HYB_ERR_INVALID_ARG;
+  if (!A->tile_map || !A->vals || !A->meta || !A->val_off || !A->meta_off)
+    return HYB_ERR_INVALID_ARG;
+  const int64_t te = (int64_t)kPM * kPK;
+  if (A->n_vals < A->num_tiles * te / 2 || A->n_vals > A->num_tiles * te ||
+      A->n_vals % kPK != 0 || A->n_meta_bytes < 0 || A->n_meta_bytes > A->num_tiles * te / 8)
+    return HYB_ERR_INVALID_ARG;
+  if (ldx < A->k || ldy < A->n) return HYB_ERR_INVALID_ARG;
+  if ((uintptr_t)A->vals % 16 != 0 || (uintptr_t)A->meta % 16 != 0 || (uintptr_t)X % 16 != 0 ||
+      ldx % 8 != 0 || (uintptr_t)Y % 4 != 0)
+    return HYB_ERR_ALIGNMENT;
+  if (!ws || ws_bytes < kHeaderBytes) return HYB_ERR_WORKSPACE;
+  if ((uintptr_t)ws % 256 != 0) return HYB_ERR_ALIGNMENT;
+
+  alignas(64) CUtensorMap xmap{};
+  alignas(64) CUtensorMap wmap{};
+  int rc = encode_sw128(X, (uint64_t)A->k, (uint64_t)m, (uint64_t)ldx * 2, &xmap);
+  if (rc != HYB_OK) return rc;
+  // the value buffer seen as rows of 128 bf16: a dense tile at element offset
+  // vo is rows vo / 128 .. + 127
+  rc = encode_sw128(A->vals, (uint64_t)kPK, (uint64_t)(A->n_vals / kPK), (uint64_t)kPK * 2,
+                    &wmap);
+  if (rc != HYB_OK) return rc;
+
+  PrefillParams prm{};
+  prm.map = A->tile_map;
+  prm.vals = A->vals;
+  prm.meta = A->meta;
+  prm.val_off = A->val_off;
+  prm.meta_off = A->meta_off;
+  prm.n = A->n;
+  prm.k = A->k;
+  prm.m = m;
+  prm.tpr = (int)tpr;
+  prm.nvb = 2 * A->n_vals;
+  prm.nmb = A->n_meta_bytes;
+  prm.Y = Y;
+  prm.ldy = ldy;
+  prm.status = static_cast<uint32_t *>(ws);
+
+  const size_t dyn = (size_t)kPStages * kStageBytes + 1024;
+  if (cudaFuncSetAttribute(hybrid_prefill_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)dyn) != cudaSuccess)
+    return HYB_ERR_CUDA;
+  const dim3 grid((unsigned)(A->n / kPM), (unsigned)((m + kPN - 1) / kPN));
+  hybrid_prefill_kernel<<<grid, kPThreads, dyn, (cudaStream_t)stream>>>(prm, xmap, wmap);
+  return cudaGetLastError() == cudaSuccess ? HYB_OK : HYB_ERR_CUDA;
+}

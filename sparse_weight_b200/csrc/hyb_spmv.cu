@@ -178,50 +178,12 @@ __device__ __forceinline__ void store_out(const Params &p, int64_t row, int b,
 // expected to have two bits set (as hyb_pack writes them); any other mask
 // still selects within the group's four values.
 
-constexpr uint32_t kWaitLimit = 1u << 22;
 // The low-rank warp's chunk buffer after the ring: two halves (16 KB of
 // dynamic shared memory, requested only by launches with a low-rank term;
 // such launches may use one ring stage fewer to make room).
 constexpr int kLrHalf = 8192;
 constexpr int kLrBufBytes = 2 * kLrHalf;
 
-__device__ __forceinline__ uint32_t smem_u32(const void *p) {
-  return (uint32_t)__cvta_generic_to_shared(p);
-}
-__device__ __forceinline__ void mbar_init(uint64_t *bar, uint32_t count) {
-  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count)
-               : "memory");
-}
-__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t *bar, uint32_t tx) {
-  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)),
-               "r"(tx)
-               : "memory");
-}
-__device__ __forceinline__ void mbar_arrive(uint64_t *bar) {
-  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
-}
-__device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
-  uint32_t ok;
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-      "selp.u32 %0, 1, 0, p;\n\t}"
-      : "=r"(ok)
-      : "r"(smem_u32(bar)), "r"(parity)
-      : "memory");
-  return ok != 0;
-}
-// Every wait is bounded: on expiry the caller records kStatusTimeout and
-// leaves the pipeline instead of waiting for ever.
-__device__ __forceinline__ bool mbar_wait_limit(uint64_t *bar, uint32_t parity,
-                                                uint32_t limit) {
-  for (uint32_t i = 0; i < limit; ++i)
-    if (mbar_try_wait(bar, parity)) return true;
-  return false;
-}
-__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity) {
-  return mbar_wait_limit(bar, parity, kWaitLimit);
-}
 __device__ __forceinline__ int64_t ld_volatile_nc64(const int64_t *addr) {
   int64_t v;
   asm volatile("ld.global.nc.s64 %0, [%1];" : "=l"(v) : "l"(addr));
@@ -292,24 +254,6 @@ __device__ __forceinline__ void cp_async_wait() {
   asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
 }
 
-__device__ __forceinline__ void bulk_g2s(void *dst, const void *src, uint32_t bytes,
-                                         uint64_t *bar) {
-  asm volatile(
-      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::
-          "r"(smem_u32(dst)),
-      "l"(src), "r"(bytes), "r"(smem_u32(bar))
-      : "memory");
-}
-// 2-D tiled TMA load of box (x, y) of the tensor map into shared memory,
-// completion counted on the mbarrier (no multicast).
-__device__ __forceinline__ void tma_load_2d(void *dst, const CUtensorMap *map, int x, int y,
-                                            uint64_t *bar) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
-      " [%0], [%1, {%2, %3}], [%4];" ::"r"(smem_u32(dst)),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(smem_u32(bar))
-      : "memory");
-}
 // acc += lo(w) * lo(x) + hi(w) * hi(x) on two packed bf16 pairs.
 __device__ __forceinline__ void fma_bf16x2(float &acc, uint32_t w, uint32_t x) {
   unsigned short wl, wh, xl, xh;
@@ -2145,22 +2089,7 @@ int launch_lowrank_t(const Plan &P, const hyb_lowrank *lr, int64_t k,
 
 // Shared driver of hyb_spmv / hyb_spmm_skinny / hyb_gemv_dense.
 // Tensor map of X ([batch][k] bf16, row stride ldx) with box [bp][xcols]:
-// rows past the batch and columns past k read as zeros.  The encoder is the
-// driver's, found once through the runtime.
-PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
-  static PFN_cuTensorMapEncodeTiled_v12000 encode = nullptr;
-  static std::once_flag once;
-  std::call_once(once, [] {
-    void *fn = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) ==
-            cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
-  });
-  return encode;
-}
-
+// rows past the batch and columns past k read as zeros.
 int encode_x_map(const uint16_t *X, int64_t k, int batch, int64_t ldx, int xcols, int bp,
                  CUtensorMap *map) {
   PFN_cuTensorMapEncodeTiled_v12000 encode = tensor_map_encoder();

@@ -69,7 +69,7 @@ EXPORTS = ["hyb_packed_sizes", "hyb_pack_workspace_bytes", "hyb_pack",
            "hyb_dense_workspace_bytes", "hyb_gemv_dense", "hyb_check_status",
            "hyb_status_string", "hyb_spmv_noalloc", "hyb_spmv_noalloc_max_scratch_bytes",
            "hyb_spmv_noalloc_check_status", "hyb_gate_up_workspace_bytes",
-           "hyb_spmm_skinny_gate_up",
+           "hyb_spmm_skinny_gate_up", "hyb_prefill_workspace_bytes", "hyb_spmm_prefill",
            "hyb_plan_entries", "hyb_make_plan", "hyb_selftest_wait_timeout",
            "hyb_spmm_skinny_ex", "hyb_gemv_dense_ex", "hyb_packed_sizes_nm",
            "hyb_pack_nm", "hyb_spmm_skinny_nm"]
@@ -111,6 +111,11 @@ def lib():
                                           ctypes.POINTER(HybLowrank), _P, _I64, ctypes.c_uint32,
                                           _P, _SZ, _P]
     L.hyb_spmm_skinny_gate_up.restype = _I
+    L.hyb_prefill_workspace_bytes.argtypes = []
+    L.hyb_prefill_workspace_bytes.restype = _SZ
+    L.hyb_spmm_prefill.argtypes = [ctypes.POINTER(HybMatrix), _I64, _P, _I64, _P, _I64, _P, _SZ,
+                                   _P]
+    L.hyb_spmm_prefill.restype = _I
     L.hyb_lowrank_workspace_bytes.argtypes = [_I64, _I, _I]
     L.hyb_lowrank_workspace_bytes.restype = _SZ
     L.hyb_lowrank_add.argtypes = [_I64, _I64, _I, ctypes.POINTER(HybLowrank), _P, _I64,
@@ -421,6 +426,23 @@ def spmm_skinny(A: Packed, X: torch.Tensor, Y: torch.Tensor = None, ydt: int = H
     _check("hyb_spmm_skinny_ex", lib().hyb_spmm_skinny_ex(
         ctypes.byref(s), batch, _ptr(Xb), Xb.stride(0), _ptr(Y), Y.stride(0), ydt,
         ctypes.byref(lr) if lr else None, flags, _ptr(ws), ws.numel(), _stream(stream)))
+    return Y
+
+
+def spmm_prefill(A: Packed, X: torch.Tensor, Y: torch.Tensor = None, ws: torch.Tensor = None,
+                 stream=None) -> torch.Tensor:
+    """hyb_spmm_prefill: Y[m][n] = W_hat X for m tokens (tensor cores); X bf16
+    [m][k], Y fp32 [m][n]."""
+    Xb = _bits(X)
+    m = Xb.shape[0]
+    if Y is None:
+        Y = torch.empty(m, A.n, dtype=torch.float32, device=Xb.device)
+    if ws is None:
+        ws = new_workspace(int(lib().hyb_prefill_workspace_bytes()), Xb.device)
+    s = A.struct()
+    _check("hyb_spmm_prefill", lib().hyb_spmm_prefill(
+        ctypes.byref(s), m, _ptr(Xb), Xb.stride(0), _ptr(Y), Y.stride(0), _ptr(ws), ws.numel(),
+        _stream(stream)))
     return Y
 
 
