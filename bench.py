@@ -557,8 +557,8 @@ def _tensor_roofline(n, k, us):
 def sweep(device, steps=200, warmup=10):
     """Hybrid vs dense on the FFN shapes across 2:4-tile fractions and batches,
     the 4096x4096 attention matrix, the 32-layer Llama-3.1-8B chain (224
-    matrices, one CUDA graph) and the Llama-3.3-70B FFN with the fused
-    rank-128 low-rank term."""
+    matrices, one CUDA graph), the Llama-3.3-70B FFN with a rank-128 (and
+    rank-64) low-rank term, and prefill on the tensor cores."""
     peak, peak_kind = measured_peak()
     L = hyb.lib()
     OV = hyb.LAUNCH_OVERLAP_PREV
@@ -707,7 +707,52 @@ def sweep(device, steps=200, warmup=10):
                                     hyb._bits(V).data_ptr(), rank) for U, V in lrs]
         _sweep_70b(L, structs, lrstructs, mats70, sh70, rank, batches, device, peak, emit, sm_mhz)
         del lrs, lrstructs, lr_by_role
+    del mats70, structs
+    torch.cuda.empty_cache()
+    _sweep_prefill(device, emit)
     return 0
+
+
+def _sweep_prefill(device, emit, steps=20, warmup=3):
+    """Prefill on the tensor cores (hyb_spmm_prefill): the FFN shapes at 512
+    and 2048 tokens and three 2:4-tile fractions, against torch.matmul (cuBLAS
+    bf16, the dense weight) on the same inputs.  Tokens x weight bytes exceed
+    L2, so back-to-back calls are timed (CUDA events, mean of `steps`)."""
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as fh:
+            peak = float(json.load(fh)["bf16_tflops"])
+    except Exception:
+        peak = 1590.0
+    for n, k in ((4096, 14336), (14336, 4096)):
+        W = inputs.weight(n, k, 0.02, inputs.seed_of("prefill_sweep", n, k)).to(device)
+        T = (n // 128) * (k // 128)
+        for m in (512, 2048):
+            X = inputs.activations(m, k, inputs.seed_of("prefill_sweep", "X", m, k)).to(device)
+            Y = torch.empty(m, n, dtype=torch.float32, device=device)
+            stream = torch.cuda.current_stream(device)
+            cub_ms = timed(lambda i: torch.matmul(X, W.t()), steps, warmup, stream)
+            cub_us = cub_ms / steps * 1e3
+            for f in (0.0, 0.5, 1.0):
+                tmap = inputs.tile_map_fraction(T, f, inputs.seed_of("prefill_sweep", f))
+                P = hyb.pack(W, tmap, 128, 128)
+                ws = hyb.new_workspace(hyb.lib().hyb_prefill_workspace_bytes(), device)
+                ms = timed(lambda i: hyb.spmm_prefill(P, X, Y=Y, ws=ws), steps, warmup, stream)
+                hyb.check_status(ws)
+                us = ms / steps * 1e3
+                flops = 2 * m * n * k
+                emit({"sweep": "prefill", "shape": f"{n}x{k}", "tokens": m, "tile": "128x128",
+                      "sparse_tile_frac": float(np.mean(tmap)), "us": round(us, 2),
+                      "tensor_roofline": {"bound": "tensor",
+                                          "achieved": round(flops / (us * 1e-6) / 1e12, 1),
+                                          "peak": peak, "unit": "TFLOP/s",
+                                          "frac": round(flops / (us * 1e-6) / 1e12 / peak, 4),
+                                          "flops": "2 m n k (2:4 tiles expanded to dense)"},
+                      "cublas_bf16_dense_us": round(cub_us, 2),
+                      "speedup_vs_cublas_dense": round(cub_us / us, 4),
+                      "kernel": "hybrid_prefill_kernel (tcgen05.mma kind::f16, TMEM accumulator)"})
+                del P, ws
+        del W
+    torch.cuda.empty_cache()
 
 
 def _sweep_70b(L, structs, lrstructs, mats70, sh70, rank, batches, device, peak, emit, sm_mhz):
@@ -755,7 +800,8 @@ def sweep_nm(device, steps=200, warmup=10):
         nrot = max(2, int(np.ceil(3 * (126 << 20) / base.nbytes())))
         mats = [base] + [base.clone() for _ in range(nrot - 1)]
         structs = [x.struct() for x in mats]
-        ws = hyb.new_workspace(hyb.pack_workspace_bytes(), device)
+        ws = hyb.new_workspace(max(hyb.workspace_bytes(base, 8), hyb.pack_workspace_bytes()),
+                               device)
         for b in (1, 8):
             xs = [inputs.activations(b, k, inputs.seed_of("nm_sweep", b, i)).to(device)
                   for i in range(nrot)]
@@ -825,6 +871,9 @@ def main():
                          "low-rank lines instead of the headline line")
     ap.add_argument("--nm", action="store_true",
                     help="print the general N:M (4:8) lines instead of the headline line")
+    ap.add_argument("--prefill-profile", action="store_true",
+                    help="small prefill case for a profiler: hyb_spmm_prefill on 4096x14336, "
+                         "f = 0.5, 512 tokens, --steps eager calls")
     ap.add_argument("--profile", action="store_true",
                     help="small case for a profiler: 2 rotating copies (184 MB > L2), "
                          "hybrid product only, no dense / end-to-end / CPU legs")
@@ -842,6 +891,22 @@ def main():
         import datetime
         torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                              device_id=device)
+    if args.prefill_profile:
+        n, k, m = 4096, 14336, 512
+        W = inputs.weight(n, k, 0.02, inputs.seed_of("prefill_profile", n, k)).to(device)
+        T = (n // 128) * (k // 128)
+        P = hyb.pack(W, inputs.tile_map_fraction(T, 0.5, inputs.seed_of("prefill_profile", "map")),
+                     128, 128)
+        X = inputs.activations(m, k, inputs.seed_of("prefill_profile", "X")).to(device)
+        Y = torch.empty(m, n, dtype=torch.float32, device=device)
+        ws = hyb.new_workspace(hyb.lib().hyb_prefill_workspace_bytes(), device)
+        ms = timed(lambda i: hyb.spmm_prefill(P, X, Y=Y, ws=ws), args.steps, args.warmup,
+                   torch.cuda.current_stream(device))
+        hyb.check_status(ws)
+        if rank == 0:
+            print(json.dumps({"profile_run": "prefill 4096x14336 f0.5 m512", "ms": ms,
+                              "steps": args.steps}))
+        return 0
     if args.sweep:
         return sweep(device)
     if args.nm:

@@ -11,11 +11,11 @@
 //   * CTA (band r, token block mb) owns Y[128 mb .. +128][128 r .. +128]: a
 //     128 x 128 fp32 accumulator in tensor memory (TMEM), M = 128 weight rows,
 //     N = 128 tokens, K looped over the band's tiles (128 columns each).
-//   * warp 0 (one lane) moves each tile's operands with TMA: a dense tile as
-//     two 2-D boxes of 64 columns x 128 rows with 128-byte swizzle (the
-//     K-major layout tcgen05.mma reads), X as two such boxes of the token
-//     block; a 2:4 tile's kept values and masks as plain bulk copies into a
-//     staging buffer.
+//   * warp 0 (one lane) moves each tile's operands with TMA into a 3-stage
+//     ring: a dense tile as two 2-D boxes of 64 columns x 128 rows with
+//     128-byte swizzle (the K-major layout tcgen05.mma reads), X as two such
+//     boxes of the token block; a 2:4 tile's kept values and masks as plain
+//     bulk copies into one staging buffer outside the ring.
 //   * warps 4-7 expand a staged 2:4 tile into the same swizzled dense layout
 //     (thread i: row i; kept pairs placed by the mask nibble, zeros
 //     elsewhere), fence it for the async proxy and signal the MMA warp.
@@ -44,8 +44,9 @@ constexpr int kABytes = 2 * kAtomBytes;       // a dense tile: two 64-column ato
 constexpr int kXBytes = 2 * kAtomBytes;       // 128 tokens x 128 columns
 constexpr int kSValBytes = kPM * kPK;         // 2:4 staging: kept values (bf16)
 constexpr int kSMetaBytes = kPM * kPK / 8;    // and masks
-constexpr int kStageBytes = kABytes + kXBytes + kSValBytes + kSMetaBytes;  // 82 KB
-constexpr int kPStages = 2;
+constexpr int kStageBytes = kABytes + kXBytes;            // 64 KB
+constexpr int kStagingBytes = kSValBytes + kSMetaBytes;  // 18 KB, one buffer after the ring
+constexpr int kPStages = 3;
 constexpr int kPThreads = 256;
 constexpr int kTmemCols = 128;                // fp32 accumulator columns (= kPN)
 constexpr int kMaxBandTiles = 1024;           // tiles per band (k <= 131072)
@@ -128,11 +129,14 @@ __global__ void __launch_bounds__(kPThreads, 1)
   extern __shared__ uint8_t smem_raw[];
   __shared__ __align__(8) uint64_t full_bar[kPStages];
   __shared__ __align__(8) uint64_t empty_bar[kPStages];
-  // a 2:4 tile's staging copy landed / the tile has been expanded: their
-  // phases advance only on the 2:4 uses of a stage (the MMA warp takes the
-  // tiles in order and waits for every expansion, so neither barrier ever
-  // runs two phases ahead of a thread waiting on it)
-  __shared__ __align__(8) uint64_t sfull_bar[kPStages];
+  // 2:4 tiles: the staging copy landed (sfull) / the staging buffer has been
+  // read (sempty) / stage s's expanded tile is written (exp).  Their phases
+  // advance only on 2:4 tiles: the producer refills the staging buffer only
+  // after the previous 2:4 tile was read, and the MMA warp takes the tiles in
+  // order and waits for every expansion, so none of them ever runs two
+  // phases ahead of a thread waiting on it.
+  __shared__ __align__(8) uint64_t sfull_bar;
+  __shared__ __align__(8) uint64_t sempty_bar;
   __shared__ __align__(8) uint64_t exp_bar[kPStages];
   __shared__ __align__(8) uint64_t acc_bar;
   __shared__ uint32_t s_tmem;
@@ -151,9 +155,10 @@ __global__ void __launch_bounds__(kPThreads, 1)
     for (int s = 0; s < kPStages; ++s) {
       mbar_init(&full_bar[s], 1);
       mbar_init(&empty_bar[s], 1);
-      mbar_init(&sfull_bar[s], 1);
       mbar_init(&exp_bar[s], 128);
     }
+    mbar_init(&sfull_bar, 1);
+    mbar_init(&sempty_bar, 128);
     mbar_init(&acc_bar, 1);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
@@ -198,6 +203,8 @@ __global__ void __launch_bounds__(kPThreads, 1)
       }
     };
     int64_t vo, mo, nvo, nmo;
+    uint32_t nsp = 0;  // 2:4 tiles issued so far
+    uint8_t *staging = smem + (size_t)kPStages * kStageBytes;
     load(0, vo, mo);
     for (int w0 = 0; w0 < tpr && ok; w0 += 32) {
       load(w0 + 32, nvo, nmo);
@@ -229,13 +236,18 @@ __global__ void __launch_bounds__(kPThreads, 1)
               const int row = (int)(tvo / kPK);  // the tile's first row in the 128-wide view
               tma_load_2d(st, &wmap, 0, row, &full_bar[s]);
               tma_load_2d(st + kAtomBytes, &wmap, 64, row, &full_bar[s]);
-            } else if (fits) {
-              uint8_t *sv = st + kABytes + kXBytes;
-              mbar_arrive_expect_tx(&sfull_bar[s], (uint32_t)(kSValBytes + kSMetaBytes));
-              bulk_g2s(sv, p.vals + tvo, kSValBytes, &sfull_bar[s]);
-              bulk_g2s(sv + kSValBytes, p.meta + tmo, kSMetaBytes, &sfull_bar[s]);
             } else if (sp) {
-              mbar_arrive(&sfull_bar[s]);  // nothing copied: the expansion reads stale bytes
+              // the staging buffer is free once the previous 2:4 tile was read
+              if (!mbar_wait(&sempty_bar, (nsp & 1u) ^ 1u)) {
+                ok = false;
+              } else if (fits) {
+                mbar_arrive_expect_tx(&sfull_bar, (uint32_t)kStagingBytes);
+                bulk_g2s(staging, p.vals + tvo, kSValBytes, &sfull_bar);
+                bulk_g2s(staging + kSValBytes, p.meta + tmo, kSMetaBytes, &sfull_bar);
+              } else {
+                mbar_arrive(&sfull_bar);  // nothing copied: the expansion reads stale bytes
+              }
+              ++nsp;
             }
           }
         }
@@ -289,19 +301,20 @@ __global__ void __launch_bounds__(kPThreads, 1)
     // ------------------- 2:4 expansion, then the epilogue -------------------
     const int i = tid - 128;  // tile row
     bool ok = true;
-    uint32_t sp_ph = 0;  // bit s: parity of stage s's next 2:4 use
+    uint32_t nsp = 0;  // 2:4 tiles expanded so far
+    const uint8_t *staging = smem + (size_t)kPStages * kStageBytes;
     for (int j = 0; j < tpr && ok; ++j) {
       const int s = j % kPStages;
       if (s_map[j] != 1) continue;
-      if (!mbar_wait(&sfull_bar[s], (sp_ph >> s) & 1u)) {
+      if (!mbar_wait(&sfull_bar, nsp & 1u)) {
         ok = false;
         break;
       }
-      sp_ph ^= 1u << s;
+      ++nsp;
       uint8_t *st = smem + (size_t)s * kStageBytes;
-      const uint8_t *sv = st + kABytes + kXBytes + i * (kPK);            // 64 kept bf16
-      const uint4 mv = *reinterpret_cast<const uint4 *>(st + kABytes + kXBytes + kSValBytes +
-                                                         i * (kPK / 8));  // 32 mask nibbles
+      const uint8_t *sv = staging + i * kPK;                                   // 64 kept bf16
+      const uint4 mv =
+          *reinterpret_cast<const uint4 *>(staging + kSValBytes + i * (kPK / 8));  // 32 nibbles
 #pragma unroll
       for (int q = 0; q < 8; ++q) {
         // piece pc: groups 4pc .. 4pc + 3 = columns 16pc .. 16pc + 15 (rotated
@@ -326,6 +339,8 @@ __global__ void __launch_bounds__(kPThreads, 1)
               make_uint4(w[4 * h], w[4 * h + 1], w[4 * h + 2], w[4 * h + 3]);
         }
       }
+      // the staging row has been read (every value above is in use)
+      mbar_arrive(&sempty_bar);
       // generic-proxy writes, read next by tcgen05.mma (async proxy)
       asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
       mbar_arrive(&exp_bar[s]);
@@ -432,7 +447,7 @@ int hyb_spmm_prefill(const hyb_matrix *A, int64_t m, const uint16_t *X, int64_t 
   prm.ldy = ldy;
   prm.status = static_cast<uint32_t *>(ws);
 
-  const size_t dyn = (size_t)kPStages * kStageBytes + 1024;
+  const size_t dyn = (size_t)kPStages * kStageBytes + kStagingBytes + 1024;
   if (cudaFuncSetAttribute(hybrid_prefill_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            (int)dyn) != cudaSuccess)
     return HYB_ERR_CUDA;
