@@ -856,6 +856,47 @@ def workload_config(name, frac_real, rot, nbytes):
 
 # ---------------------------------------------------------------------------
 
+def run_tp(args, device, world, rank):
+    """Row-sharded decode: every rank applies its bands of the workload's
+    matrix (hyb_shard_bands) to the full X, then one all-gather assembles Y on
+    every rank.  Eager steps between CUDA events, max over ranks; value = the
+    whole matrix's algorithmic bytes per step / time (strong scaling)."""
+    from sparse_weight_b200 import tp
+    W, tmap = make_matrix(args.workload)
+    n, k, b1, b2, frac, batch, std, outliers = WORKLOADS[args.workload]
+    P = hyb.pack(W.to(device), tmap, b1, b2)
+    # rotating copies (larger than L2 in all), each sharded the same way
+    rot = rotation(args.workload, tmap, args.rotate)
+    shards = [tp.RowShard(m, rank, world) for m in [P] + [P.clone() for _ in range(rot - 1)]]
+    X = inputs.activations(batch, k, inputs.seed_of(args.workload, "X", 0)).to(device)
+    local = shards[0].local
+    ws = (hyb.new_workspace(hyb.workspace_bytes(local, batch), device)
+          if local is not None else None)
+    stream = torch.cuda.current_stream(device)
+    ms = timed(lambda i: shards[i % rot].apply(X, ws=ws), args.steps, args.warmup, stream,
+               world)
+    if ws is not None:
+        hyb.check_status(ws)
+    nbytes = P.nbytes() + P.num_tiles + 2 * batch * k + 4 * batch * n
+    value = nbytes * args.steps / (ms * 1e-3) / 1e9
+    if world > 1:
+        torch.distributed.destroy_process_group()
+    if rank == 0:
+        print(json.dumps({
+            "metric": "hybrid 2:4 GEMV achieved HBM GB/s (algorithmic bytes)",
+            "value": round(value, 2), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": round(ms / args.steps, 6),
+            "higher_is_better": True, "scaling": "strong", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic",
+            "config": dict(workload_config(args.workload, float(np.mean(tmap)), rot, P.nbytes()),
+                           parallelism=f"tp{world} (row shards, NCCL all-gather of Y)",
+                           rows_per_rank=[hi - lo for lo, hi in shards[0].rows],
+                           launch="eager steps (the shard product, the all-gather and the "
+                                  "row reassembly)"),
+            "gpu_launches": args.steps}), flush=True)
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -871,9 +912,13 @@ def main():
                          "low-rank lines instead of the headline line")
     ap.add_argument("--nm", action="store_true",
                     help="print the general N:M (4:8) lines instead of the headline line")
+    ap.add_argument("--tp", action="store_true",
+                    help="row-sharded (tensor-parallel) decode of the workload's matrix over the "
+                         "ranks: each rank its bands, one NCCL all-gather of Y per step "
+                         "(strong scaling; the default is one replica per rank)")
     ap.add_argument("--prefill-profile", action="store_true",
-                    help="small prefill case for a profiler: hyb_spmm_prefill on 4096x14336, "
-                         "f = 0.5, 512 tokens, --steps eager calls")
+                    help="prefill case for a profiler: hyb_spmm_prefill on 4096x14336, "
+                         "f = 0.5, 2048 tokens (512 CTAs), --steps eager calls")
     ap.add_argument("--profile", action="store_true",
                     help="small case for a profiler: 2 rotating copies (184 MB > L2), "
                          "hybrid product only, no dense / end-to-end / CPU legs")
@@ -892,7 +937,7 @@ def main():
         torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                              device_id=device)
     if args.prefill_profile:
-        n, k, m = 4096, 14336, 512
+        n, k, m = 4096, 14336, 2048
         W = inputs.weight(n, k, 0.02, inputs.seed_of("prefill_profile", n, k)).to(device)
         T = (n // 128) * (k // 128)
         P = hyb.pack(W, inputs.tile_map_fraction(T, 0.5, inputs.seed_of("prefill_profile", "map")),
@@ -904,9 +949,11 @@ def main():
                    torch.cuda.current_stream(device))
         hyb.check_status(ws)
         if rank == 0:
-            print(json.dumps({"profile_run": "prefill 4096x14336 f0.5 m512", "ms": ms,
+            print(json.dumps({"profile_run": "prefill 4096x14336 f0.5 m2048", "ms": ms,
                               "steps": args.steps}))
         return 0
+    if args.tp:
+        return run_tp(args, device, world, rank)
     if args.sweep:
         return sweep(device)
     if args.nm:

@@ -224,6 +224,22 @@ HYB_API int hyb_spmm_skinny_ex(const hyb_matrix *A, int batch, const uint16_t *X
                                const hyb_lowrank *lr, uint32_t flags, void *ws,
                                size_t ws_bytes, hyb_stream_t stream);
 
+/* ---- row sharding for tensor-parallel decode ---------------------------
+ * Host only.  The tile-row bands [*band_begin, *band_end) that rank `rank` of
+ * `world` holds when a packed matrix is split by rows for tensor-parallel
+ * decode: contiguous bands, balanced by packed bytes (rank i takes the bands
+ * whose first packed byte b satisfies i * total <= b * world < (i + 1) *
+ * total), every band on exactly one rank; a rank may get none when there are
+ * fewer bands than ranks.  Each rank then applies its bands (rows band_begin
+ * * b1 .. band_end * b1) to the full X and the ranks' outputs are gathered.
+ * The bands of one rank are a contiguous slice of the packed buffers, so a
+ * shard needs no repacking: its values, masks and tile map are views, its
+ * offsets the matrix's minus those of its first tile.  Errors:
+ * HYB_ERR_INVALID_ARG for a bad tiling, map byte, world or rank. */
+HYB_API int hyb_shard_bands(int64_t n, int64_t k, int b1, int b2,
+                            const uint8_t *tile_map_host, int world, int rank,
+                            int64_t *band_begin, int64_t *band_end);
+
 /* ---- prefill / large batch on the tensor cores ---------------------------
  * Y[m][i] = sum_k W_hat[i][k] X[m][k] for a block of M tokens (PATCH: dense
  * tiles on dense tensor-core kernels, 2:4 tiles on sparse ones, §2 Method):

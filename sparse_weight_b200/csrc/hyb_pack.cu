@@ -168,6 +168,36 @@ int hyb_packed_sizes(int64_t n, int64_t k, int b1, int b2,
   return HYB_OK;
 }
 
+int hyb_shard_bands(int64_t n, int64_t k, int b1, int b2, const uint8_t *tile_map_host,
+                    int world, int rank, int64_t *band_begin, int64_t *band_end) {
+  int rc = hyb::check_tiling(n, k, b1, b2);
+  if (rc != HYB_OK) return rc;
+  if (!tile_map_host || !band_begin || !band_end || world < 1 || rank < 0 || rank >= world)
+    return HYB_ERR_INVALID_ARG;
+  const int64_t R = n / b1, tpr = k / b2;
+  const int64_t dense = 2LL * b1 * b2, sparse = (int64_t)b1 * b2 + (int64_t)b1 * b2 / 8;
+  // packed bytes before each band; rank i takes the bands whose first byte
+  // b satisfies i * total <= b * world < (i + 1) * total (contiguous bands,
+  // balanced by bytes, every band on exactly one rank)
+  int64_t total = 0;
+  for (int64_t t = 0; t < R * tpr; ++t) {
+    if (tile_map_host[t] > 1) return HYB_ERR_INVALID_ARG;
+    total += tile_map_host[t] ? sparse : dense;
+  }
+  int64_t before = 0, lo = -1, hi = -1;
+  for (int64_t r = 0; r <= R; ++r) {
+    const int64_t b = r < R ? before : total;
+    if (lo < 0 && (r == R || b * world >= (int64_t)rank * total)) lo = r;
+    if (hi < 0 && (r == R || b * world >= (int64_t)(rank + 1) * total)) hi = r;
+    if (r < R)
+      for (int64_t t = r * tpr; t < (r + 1) * tpr; ++t) before += tile_map_host[t] ? sparse : dense;
+  }
+  if (rank == world - 1) hi = R;
+  *band_begin = lo;
+  *band_end = hi < lo ? lo : hi;
+  return HYB_OK;
+}
+
 int hyb_pack(int64_t n, int64_t k, int b1, int b2, const uint16_t *W,
              int64_t ldw, const uint8_t *tile_map, uint16_t *vals,
              uint8_t *meta, int64_t *val_off, int64_t *meta_off, void *ws,

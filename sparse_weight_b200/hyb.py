@@ -70,6 +70,7 @@ EXPORTS = ["hyb_packed_sizes", "hyb_pack_workspace_bytes", "hyb_pack",
            "hyb_status_string", "hyb_spmv_noalloc", "hyb_spmv_noalloc_max_scratch_bytes",
            "hyb_spmv_noalloc_check_status", "hyb_gate_up_workspace_bytes",
            "hyb_spmm_skinny_gate_up", "hyb_prefill_workspace_bytes", "hyb_spmm_prefill",
+           "hyb_shard_bands",
            "hyb_plan_entries", "hyb_make_plan", "hyb_selftest_wait_timeout",
            "hyb_spmm_skinny_ex", "hyb_gemv_dense_ex", "hyb_packed_sizes_nm",
            "hyb_pack_nm", "hyb_spmm_skinny_nm"]
@@ -111,6 +112,9 @@ def lib():
                                           ctypes.POINTER(HybLowrank), _P, _I64, ctypes.c_uint32,
                                           _P, _SZ, _P]
     L.hyb_spmm_skinny_gate_up.restype = _I
+    L.hyb_shard_bands.argtypes = [_I64, _I64, _I, _I, _P, _I, _I, ctypes.POINTER(ctypes.c_int64),
+                                  ctypes.POINTER(ctypes.c_int64)]
+    L.hyb_shard_bands.restype = _I
     L.hyb_prefill_workspace_bytes.argtypes = []
     L.hyb_prefill_workspace_bytes.restype = _SZ
     L.hyb_spmm_prefill.argtypes = [ctypes.POINTER(HybMatrix), _I64, _P, _I64, _P, _I64, _P, _SZ,
@@ -238,6 +242,38 @@ class Packed:
                       self.vals.clone(), self.meta.clone(), self.val_off.clone(),
                       self.meta_off.clone(), self.n_vals, self.n_meta,
                       None if self.plan is None else self.plan.clone(), self.plan_ctas)
+
+
+def shard_bands(n: int, k: int, b1: int, b2: int, tile_map, world: int, rank: int):
+    """hyb_shard_bands: the tile-row bands [begin, end) rank `rank` of `world`
+    holds (host only)."""
+    tm = tile_map.cpu().numpy() if torch.is_tensor(tile_map) else np.asarray(tile_map)
+    tm = np.ascontiguousarray(tm, dtype=np.uint8).reshape(-1)
+    lo, hi = ctypes.c_int64(0), ctypes.c_int64(0)
+    _check("hyb_shard_bands", lib().hyb_shard_bands(n, k, b1, b2, tm.ctypes.data, world, rank,
+                                                    ctypes.byref(lo), ctypes.byref(hi)))
+    return lo.value, hi.value
+
+
+def shard(A: "Packed", rank: int, world: int, plan: bool = True) -> Optional["Packed"]:
+    """The rows of A that rank `rank` of `world` holds (hyb_shard_bands): its
+    bands' slice of A's packed buffers (views), offsets rebased to the slice,
+    and (with ``plan``, on a GPU) its own work split.  None when the rank
+    holds no band."""
+    r0, r1 = shard_bands(A.n, A.k, A.b1, A.b2, A.tile_map, world, rank)
+    if r1 <= r0:
+        return None
+    tpr = A.k // A.b2
+    t0, t1 = r0 * tpr, r1 * tpr
+    vo, mo = A.val_off[t0:t1 + 1], A.meta_off[t0:t1 + 1]
+    v0, v1, m0, m1 = int(vo[0]), int(vo[-1]), int(mo[0]), int(mo[-1])
+    # a shard without 2:4 tiles still passes a valid, aligned mask pointer
+    meta = A.meta[m0:m1] if m1 > m0 else torch.zeros(16, dtype=torch.uint8, device=A.meta.device)
+    S = Packed((r1 - r0) * A.b1, A.k, A.b1, A.b2, A.tile_map[t0:t1], A.vals[v0:v1], meta,
+               vo - v0, mo - m0, v1 - v0, m1 - m0)
+    if plan and S.val_off.is_cuda:
+        S.plan, S.plan_ctas = make_plan(S)
+    return S
 
 
 def pack_workspace_bytes() -> int:
