@@ -14,17 +14,17 @@
 //   * warp 0 (one lane) moves each tile's operands with TMA into a 3-stage
 //     ring: a dense tile as two 2-D boxes of 64 columns x 128 rows with
 //     128-byte swizzle (the K-major layout tcgen05.mma reads), X as two such
-//     boxes of the token block; a 2:4 tile's kept values and masks as plain
-//     bulk copies into one staging buffer outside the ring.
-//   * warps 4-7 expand a staged 2:4 tile into the same swizzled dense layout
-//     (thread i: row i; kept pairs placed by the mask nibble, zeros
+//     boxes of the token block.
+//   * warps 4-11 expand each 2:4 tile into the same swizzled dense layout in
+//     its stage (two threads per row, half a row each, read from global
+//     memory one 2:4 tile ahead; kept pairs placed by the mask nibble, zeros
 //     elsewhere), fence it for the async proxy and signal the MMA warp.
 //   * warp 1 owns the TMEM allocation; one lane issues 8 tcgen05.mma
 //     (kind::f16, bf16 x bf16 -> fp32, K = 16 each) per tile and frees the
 //     stage with tcgen05.commit.
-//   * warps 4-7 then read the accumulator with tcgen05.ld (warp w: TMEM lanes
-//     32 (w % 4) ..) and store Y (a warp writes 32 consecutive rows of one
-//     token: 128 contiguous bytes).
+//   * warps 4-11 then read the accumulator with tcgen05.ld (warp w: TMEM lanes
+//     32 (w % 4) .., half of the token columns each) and store Y (a warp
+//     writes 32 consecutive rows of one token: 128 contiguous bytes).
 //
 // 2:4 tiles take the dense MMA after expansion: the weight bytes moved are
 // the hybrid format's, the tensor work is that of a dense tile.  (The sparse
@@ -42,12 +42,12 @@ constexpr int kPK = 128;                      // columns per tile (b2)
 constexpr int kAtomBytes = 128 * 128;         // 128 rows x 128 bytes (64 bf16), swizzled
 constexpr int kABytes = 2 * kAtomBytes;       // a dense tile: two 64-column atoms
 constexpr int kXBytes = 2 * kAtomBytes;       // 128 tokens x 128 columns
-constexpr int kSValBytes = kPM * kPK;         // 2:4 staging: kept values (bf16)
+constexpr int kSValBytes = kPM * kPK;         // a 2:4 tile's kept values (bf16)
 constexpr int kSMetaBytes = kPM * kPK / 8;    // and masks
-constexpr int kStageBytes = kABytes + kXBytes;            // 64 KB
-constexpr int kStagingBytes = kSValBytes + kSMetaBytes;  // 18 KB, one buffer after the ring
+constexpr int kStageBytes = kABytes + kXBytes;  // 64 KB
 constexpr int kPStages = 3;
-constexpr int kPThreads = 256;
+constexpr int kPThreads = 384;  // warp 0 TMA, warp 1 MMA + TMEM, warps 4-11 expand + epilogue
+constexpr int kExpThreads = 256;  // two per tile row (columns 0-63, 64-127)
 constexpr int kTmemCols = 128;                // fp32 accumulator columns (= kPN)
 constexpr int kMaxBandTiles = 1024;           // tiles per band (k <= 131072)
 static_assert(kStageBytes % 1024 == 0, "stages keep the 1024-byte swizzle alignment");
@@ -129,19 +129,19 @@ __global__ void __launch_bounds__(kPThreads, 1)
   extern __shared__ uint8_t smem_raw[];
   __shared__ __align__(8) uint64_t full_bar[kPStages];
   __shared__ __align__(8) uint64_t empty_bar[kPStages];
-  // 2:4 tiles: the staging copy landed (sfull) / the staging buffer has been
-  // read (sempty) / stage s's expanded tile is written (exp).  Their phases
-  // advance only on 2:4 tiles: the producer refills the staging buffer only
-  // after the previous 2:4 tile was read, and the MMA warp takes the tiles in
-  // order and waits for every expansion, so none of them ever runs two
-  // phases ahead of a thread waiting on it.
-  __shared__ __align__(8) uint64_t sfull_bar;
-  __shared__ __align__(8) uint64_t sempty_bar;
+  // 2:4 tiles: stage s's A buffer is free for an expansion (go) / the
+  // expanded tile is written (exp).  Their phases advance only on 2:4 uses of
+  // the stage; the producer frees a stage only after the MMAs of its previous
+  // use, which for a 2:4 use waited for that expansion, so neither barrier
+  // runs two phases ahead of a thread waiting on it.
+  __shared__ __align__(8) uint64_t go_bar[kPStages];
   __shared__ __align__(8) uint64_t exp_bar[kPStages];
   __shared__ __align__(8) uint64_t acc_bar;
   __shared__ uint32_t s_tmem;
   __shared__ uint32_t sel_dense[16];
   __shared__ uint8_t s_map[kMaxBandTiles];
+  __shared__ int64_t s_vo[kMaxBandTiles];  // the band's tile offsets (values, masks)
+  __shared__ int64_t s_mo[kMaxBandTiles];
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int r = blockIdx.x;                  // tile-row band
@@ -155,10 +155,9 @@ __global__ void __launch_bounds__(kPThreads, 1)
     for (int s = 0; s < kPStages; ++s) {
       mbar_init(&full_bar[s], 1);
       mbar_init(&empty_bar[s], 1);
-      mbar_init(&exp_bar[s], 128);
+      mbar_init(&go_bar[s], 1);
+      mbar_init(&exp_bar[s], kExpThreads);
     }
-    mbar_init(&sfull_bar, 1);
-    mbar_init(&sempty_bar, 128);
     mbar_init(&acc_bar, 1);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
@@ -176,7 +175,12 @@ __global__ void __launch_bounds__(kPThreads, 1)
     }
     sel_dense[msk] = sd;
   }
-  for (int j = tid; j < tpr; j += kPThreads) s_map[j] = p.map[(int64_t)r * tpr + j];
+  for (int j = tid; j < tpr; j += kPThreads) {
+    const int64_t t = (int64_t)r * tpr + j;
+    s_map[j] = p.map[t];
+    s_vo[j] = p.val_off[t];
+    s_mo[j] = p.meta_off[t];
+  }
   if (warp == 1) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
                      smem_u32(&s_tmem)),
@@ -203,8 +207,6 @@ __global__ void __launch_bounds__(kPThreads, 1)
       }
     };
     int64_t vo, mo, nvo, nmo;
-    uint32_t nsp = 0;  // 2:4 tiles issued so far
-    uint8_t *staging = smem + (size_t)kPStages * kStageBytes;
     load(0, vo, mo);
     for (int w0 = 0; w0 < tpr && ok; w0 += 32) {
       load(w0 + 32, nvo, nmo);
@@ -237,17 +239,7 @@ __global__ void __launch_bounds__(kPThreads, 1)
               tma_load_2d(st, &wmap, 0, row, &full_bar[s]);
               tma_load_2d(st + kAtomBytes, &wmap, 64, row, &full_bar[s]);
             } else if (sp) {
-              // the staging buffer is free once the previous 2:4 tile was read
-              if (!mbar_wait(&sempty_bar, (nsp & 1u) ^ 1u)) {
-                ok = false;
-              } else if (fits) {
-                mbar_arrive_expect_tx(&sfull_bar, (uint32_t)kStagingBytes);
-                bulk_g2s(staging, p.vals + tvo, kSValBytes, &sfull_bar);
-                bulk_g2s(staging + kSValBytes, p.meta + tmo, kSMetaBytes, &sfull_bar);
-              } else {
-                mbar_arrive(&sfull_bar);  // nothing copied: the expansion reads stale bytes
-              }
-              ++nsp;
+              mbar_arrive(&go_bar[s]);  // the expansion warps may now write the A buffer
             }
           }
         }
@@ -299,31 +291,46 @@ __global__ void __launch_bounds__(kPThreads, 1)
     __syncwarp();
   } else if (warp >= 4) {
     // ------------------- 2:4 expansion, then the epilogue -------------------
-    const int i = tid - 128;  // tile row
+    const int e = tid - 128;
+    const int i = e & 127;   // tile row
+    const int hf = e >> 7;   // half of the row: columns 64 hf .. 64 hf + 63
     bool ok = true;
-    uint32_t nsp = 0;  // 2:4 tiles expanded so far
-    const uint8_t *staging = smem + (size_t)kPStages * kStageBytes;
-    for (int j = 0; j < tpr && ok; ++j) {
-      const int s = j % kPStages;
-      if (s_map[j] != 1) continue;
-      if (!mbar_wait(&sfull_bar, nsp & 1u)) {
-        ok = false;
-        break;
-      }
-      ++nsp;
-      uint8_t *st = smem + (size_t)s * kStageBytes;
-      const uint8_t *sv = staging + i * kPK;                                   // 64 kept bf16
-      const uint4 mv =
-          *reinterpret_cast<const uint4 *>(staging + kSValBytes + i * (kPK / 8));  // 32 nibbles
+    uint32_t go_ph = 0;  // bit s: parity of stage s's next 2:4 use
+    // half a row of a 2:4 tile: 32 kept values (4 x 16 B) and 16 mask nibbles
+    // (8 B); a range outside the buffers (a corrupted matrix) reads nothing
+    // and expands zeros (the producer flags it)
+    auto load_row = [&](int j, uint4 (&v)[5]) {
+      const int64_t vo = s_vo[j], mo = s_mo[j];
+      const bool fits = vo >= 0 && mo >= 0 && 2 * vo + kSValBytes <= p.nvb &&
+                        mo + kSMetaBytes <= p.nmb && ((2 * vo) | mo) % 16 == 0;
+      const uint4 *src = reinterpret_cast<const uint4 *>(p.vals + vo + (int64_t)i * (kPK / 2) +
+                                                          hf * (kPK / 4));
+      const uint2 *msk = reinterpret_cast<const uint2 *>(p.meta + mo + (int64_t)i * (kPK / 8) +
+                                                          hf * (kPK / 16));
 #pragma unroll
-      for (int q = 0; q < 8; ++q) {
-        // piece pc: groups 4pc .. 4pc + 3 = columns 16pc .. 16pc + 15 (rotated
-        // by row so that the 8 rows of a load phase hit different banks)
-        const int pc = (q + i) & 7;
-        const uint4 v = *reinterpret_cast<const uint4 *>(sv + 16 * pc);
-        const uint32_t w01 = (pc & 2) ? mv.y : mv.x, w23 = (pc & 2) ? mv.w : mv.z;
-        const uint32_t m16 = (((pc & 4) ? w23 : w01) >> (16 * (pc & 1))) & 0xFFFFu;
-        const uint32_t kv[4] = {v.x, v.y, v.z, v.w};
+      for (int q = 0; q < 4; ++q) v[q] = fits ? __ldg(src + q) : make_uint4(0, 0, 0, 0);
+      const uint2 m = fits ? __ldg(msk) : make_uint2(0, 0);
+      v[4] = make_uint4(m.x, m.y, 0, 0);
+    };
+    auto next_sparse = [&](int j) {
+      int q = j + 1;
+      while (q < tpr && s_map[q] != 1) ++q;
+      return q;
+    };
+    // expand 2:4 tile j (its half-row in v) into its stage's A buffer
+    auto expand = [&](int j, const uint4 (&v)[5]) -> bool {
+      const int s = j % kPStages;
+      if (!mbar_wait(&go_bar[s], (go_ph >> s) & 1u)) return false;
+      go_ph ^= 1u << s;
+      uint8_t *st = smem + (size_t)s * kStageBytes;
+      const uint4 mv = v[4];
+#pragma unroll
+      for (int hp = 0; hp < 4; ++hp) {
+        // piece pc: groups 4pc .. 4pc + 3 = columns 16pc .. 16pc + 15
+        const int pc = 4 * hf + hp;
+        const uint4 w4 = v[hp];
+        const uint32_t m16 = ((hp & 2) ? mv.y : mv.x) >> (16 * (hp & 1)) & 0xFFFFu;
+        const uint32_t kv[4] = {w4.x, w4.y, w4.z, w4.w};
         uint32_t w[8];
 #pragma unroll
         for (int g = 0; g < 4; ++g) {
@@ -333,26 +340,42 @@ __global__ void __launch_bounds__(kPThreads, 1)
         }
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
-          const int c = 2 * pc + h;  // 16-byte chunk of the dense row (8 columns)
+          // 16-byte chunk c of the dense row (8 columns), swizzled by row: the
+          // 8 rows of a store phase land in different banks
+          const int c = 2 * pc + h;
           uint8_t *dst = st + (c >> 3) * kAtomBytes + i * 128 + (((c & 7) ^ (i & 7)) << 4);
           *reinterpret_cast<uint4 *>(dst) =
               make_uint4(w[4 * h], w[4 * h + 1], w[4 * h + 2], w[4 * h + 3]);
         }
       }
-      // the staging row has been read (every value above is in use)
-      mbar_arrive(&sempty_bar);
       // generic-proxy writes, read next by tcgen05.mma (async proxy)
       asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
       mbar_arrive(&exp_bar[s]);
+      return true;
+    };
+    // the next 2:4 tile's half-row is loaded while this one is expanded
+    int j = next_sparse(-1);
+    uint4 cur[5];
+    if (j < tpr) load_row(j, cur);
+    while (j < tpr && ok) {
+      const int jn = next_sparse(j);
+      uint4 nxt[5];
+      if (jn < tpr) load_row(jn, nxt);
+      if (!(ok = expand(j, cur))) break;
+#pragma unroll
+      for (int q = 0; q < 5; ++q) cur[q] = nxt[q];
+      j = jn;
     }
     if (!ok && lane == 0) atomicOr(p.status, kStatusTimeout);
-    // epilogue: TMEM lanes 32 (warp % 4) .. + 31 are this warp's weight rows
+    // epilogue: TMEM lanes 32 (warp % 4) .. + 31 are this warp's weight rows;
+    // warps 4-7 store tokens 0-63 of the block, warps 8-11 tokens 64-127
     if (mbar_wait(&acc_bar, 0u)) {
       tc_fence_after();
       const int q = warp & 3;
       const int64_t row = (int64_t)r * kPM + 32 * q + lane;
+      const int cb = warp >= 8 ? kPN / 2 : 0;
 #pragma unroll 1
-      for (int c0 = 0; c0 < kPN; c0 += 16) {
+      for (int c0 = cb; c0 < cb + kPN / 2; c0 += 16) {
         float v[16];
         tmem_ld16(tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)c0, v);
 #pragma unroll
@@ -447,7 +470,7 @@ int hyb_spmm_prefill(const hyb_matrix *A, int64_t m, const uint16_t *X, int64_t 
   prm.ldy = ldy;
   prm.status = static_cast<uint32_t *>(ws);
 
-  const size_t dyn = (size_t)kPStages * kStageBytes + kStagingBytes + 1024;
+  const size_t dyn = (size_t)kPStages * kStageBytes + 1024;
   if (cudaFuncSetAttribute(hybrid_prefill_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            (int)dyn) != cudaSuccess)
     return HYB_ERR_CUDA;
