@@ -6,31 +6,33 @@
 // the prefill / large-batch form of the product.  PATCH ("PATCH: Learnable
 // Tile-level Hybrid Sparsity for LLMs", §2 Method) runs its dense tiles on
 // dense tensor-core kernels and its 2:4 tiles on the sparse tensor cores; here
-// both kinds of tile feed one tcgen05 pipeline:
+// both kinds of tile feed one tcgen05 pipeline, dense tiles through
+// tcgen05.mma and 2:4 tiles through tcgen05.mma.sp:
 //
 //   * CTA (band r, token block mb) owns Y[128 mb .. +128][128 r .. +128]: a
 //     128 x 128 fp32 accumulator in tensor memory (TMEM), M = 128 weight rows,
 //     N = 128 tokens, K looped over the band's tiles (128 columns each).
 //   * warp 0 (one lane) moves each tile's operands with TMA into a 3-stage
 //     ring: a dense tile as two 2-D boxes of 64 columns x 128 rows with
-//     128-byte swizzle (the K-major layout tcgen05.mma reads), X as two such
-//     boxes of the token block.
-//   * warps 4-11 expand each 2:4 tile into the same swizzled dense layout in
-//     its stage (two threads per row, half a row each, read from global
-//     memory one 2:4 tile ahead; kept pairs placed by the mask nibble, zeros
-//     elsewhere), fence it for the async proxy and signal the MMA warp.
-//   * warp 1 owns the TMEM allocation; one lane issues 8 tcgen05.mma
-//     (kind::f16, bf16 x bf16 -> fp32, K = 16 each) per tile and frees the
-//     stage with tcgen05.commit.
+//     128-byte swizzle (the K-major layout tcgen05.mma reads), a 2:4 tile's
+//     kept values as one box of 64 values x 128 rows (already the sparse
+//     MMA's compressed A operand: 2 kept values per group of 4, ascending),
+//     X as two boxes of the token block.
+//   * warps 4-11 turn each 2:4 tile's masks into the sparse MMA's metadata
+//     (the two kept positions of a group as a nibble, laid out by tensor-
+//     memory lane and column), fence it for the async proxy and signal the
+//     MMA warp.
+//   * warp 1 owns the TMEM allocation; one lane issues per tile 8
+//     tcgen05.mma (dense: kind::f16, bf16 x bf16 -> fp32, K = 16 each) or a
+//     tcgen05.cp of the metadata and 4 tcgen05.mma.sp (K = 32 each), and
+//     frees the stage with tcgen05.commit.
 //   * warps 4-11 then read the accumulator with tcgen05.ld (warp w: TMEM lanes
 //     32 (w % 4) .., half of the token columns each) and store Y (a warp
 //     writes 32 consecutive rows of one token: 128 contiguous bytes).
 //
-// 2:4 tiles take the dense MMA after expansion: the weight bytes moved are
-// the hybrid format's, the tensor work is that of a dense tile.  (The sparse
-// MMA, tcgen05.mma.sp, needs its metadata in a TMEM layout of its own; it is
-// not used.)  Every wait is bounded; one that runs out sets kStatusTimeout in
-// the status word and the CTA leaves its pipeline.
+// A 2:4 tile moves the hybrid format's bytes and costs half a dense tile's
+// tensor work.  Every wait is bounded; one that runs out sets kStatusTimeout
+// in the status word and the CTA leaves its pipeline.
 #include "hyb_internal.cuh"
 
 namespace hyb {
@@ -44,21 +46,37 @@ constexpr int kABytes = 2 * kAtomBytes;       // a dense tile: two 64-column ato
 constexpr int kXBytes = 2 * kAtomBytes;       // 128 tokens x 128 columns
 constexpr int kSValBytes = kPM * kPK;         // a 2:4 tile's kept values (bf16)
 constexpr int kSMetaBytes = kPM * kPK / 8;    // and masks
-constexpr int kStageBytes = kABytes + kXBytes;  // 64 KB
+constexpr int kEBytes = kPM * kPK / 8;      // a 2:4 tile's sparse-MMA metadata, 2 KB
+constexpr int kStageBytes = kABytes + kXBytes + kEBytes;  // 66 KB
 constexpr int kPStages = 3;
 constexpr int kPThreads = 384;  // warp 0 TMA, warp 1 MMA + TMEM, warps 4-11 expand + epilogue
 constexpr int kExpThreads = 256;  // two per tile row (columns 0-63, 64-127)
-constexpr int kTmemCols = 128;                // fp32 accumulator columns (= kPN)
+constexpr int kTmemCols = 256;  // fp32 accumulator (kPN columns), then 4 metadata columns per stage
+constexpr int kTmemE = kPN;     // first metadata column
 constexpr int kMaxBandTiles = 1024;           // tiles per band (k <= 131072)
 static_assert(kStageBytes % 1024 == 0, "stages keep the 1024-byte swizzle alignment");
 
 // tcgen05.mma instruction descriptor: D fp32, A and B bf16, both K-major,
-// N = kPN, M = kPM (bit layout of the sm_100 instruction descriptor).
+// N = kPN, M = kPM (bit layout of the sm_100 instruction descriptor); the
+// sparse form adds bit 2 and selects its metadata half with bits 0-1.
 constexpr uint32_t kIdesc = (1u << 4)                     // D format: f32
                             | (1u << 7)                   // A format: bf16
                             | (1u << 10)                  // B format: bf16
                             | ((uint32_t)(kPN >> 3) << 17)  // N / 8
                             | ((uint32_t)(kPM >> 4) << 24);  // M / 16
+
+constexpr uint32_t kIdescSparse = kIdesc | (1u << 2);
+
+// Shared-memory matrix descriptor of the metadata for tcgen05.cp (128 rows of
+// 16 bytes, no swizzle: 8-row core matrices of 128 contiguous bytes, 128
+// bytes apart).
+__device__ __forceinline__ uint64_t e_desc(uint32_t saddr) {
+  uint64_t d = (uint64_t)((saddr >> 4) & 0x3FFFu);
+  d |= (uint64_t)(128 >> 4) << 16;    // leading byte offset (one 16-byte column: unused)
+  d |= (uint64_t)(128 >> 4) << 32;    // stride byte offset: next 8 rows
+  d |= (uint64_t)1 << 46;             // version; layout type 0 (no swizzle)
+  return d;
+}
 
 // Shared-memory matrix descriptor of a K-major operand in the 128-byte
 // swizzle layout: rows 128 bytes apart, 8-row groups 1024 bytes apart
@@ -80,6 +98,22 @@ __device__ __forceinline__ void umma_bf16(uint32_t tmem_d, uint64_t adesc, uint6
       "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %4, p;\n\t}" ::"r"(tmem_d),
       "l"(adesc), "l"(bdesc), "r"(accumulate), "r"(kIdesc)
       : "memory");
+}
+// D += A (2:4 compressed, K = 32 per instruction, 16 stored) x B, metadata
+// from tensor memory column `tmem_e` (even) and half `id2`
+__device__ __forceinline__ void umma_sp_bf16(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc,
+                                             uint32_t tmem_e, uint32_t id2,
+                                             uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.sp.cta_group::1.kind::f16 [%0], %1, %2, [%3], %5, p;\n\t}" ::"r"(tmem_d),
+      "l"(adesc), "l"(bdesc), "r"(tmem_e), "r"(accumulate), "r"(kIdescSparse | id2)
+      : "memory");
+}
+// copy 128 lanes x 16 bytes of metadata from shared to tensor memory
+__device__ __forceinline__ void tmem_cp_128x128b(uint32_t taddr, uint64_t sdesc) {
+  asm volatile("tcgen05.cp.cta_group::1.128x128b [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
 }
 // arrives on the mbarrier once every tcgen05.mma this thread issued before
 // has completed
@@ -125,7 +159,8 @@ struct PrefillParams {
 
 __global__ void __launch_bounds__(kPThreads, 1)
     hybrid_prefill_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap xmap,
-                          const __grid_constant__ CUtensorMap wmap) {
+                          const __grid_constant__ CUtensorMap wmap,
+                          const __grid_constant__ CUtensorMap spmap) {
   extern __shared__ uint8_t smem_raw[];
   __shared__ __align__(8) uint64_t full_bar[kPStages];
   __shared__ __align__(8) uint64_t empty_bar[kPStages];
@@ -138,10 +173,8 @@ __global__ void __launch_bounds__(kPThreads, 1)
   __shared__ __align__(8) uint64_t exp_bar[kPStages];
   __shared__ __align__(8) uint64_t acc_bar;
   __shared__ uint32_t s_tmem;
-  __shared__ uint32_t sel_dense[16];
   __shared__ uint8_t s_map[kMaxBandTiles];
-  __shared__ int64_t s_vo[kMaxBandTiles];  // the band's tile offsets (values, masks)
-  __shared__ int64_t s_mo[kMaxBandTiles];
+  __shared__ int64_t s_mo[kMaxBandTiles];  // the band's mask offsets
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int r = blockIdx.x;                  // tile-row band
@@ -161,24 +194,9 @@ __global__ void __launch_bounds__(kPThreads, 1)
     mbar_init(&acc_bar, 1);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
-  if (tid < 16) {
-    // PRMT selectors expanding a kept pair (v_p0 in bytes 0-1, v_p1 in bytes
-    // 2-3, zero bytes 4-7) to the group's columns 0-1 (low half) and 2-3
-    // (high half), p0 < p1 the mask's set bits; a column not kept gets zeros
-    const uint32_t msk = tid;
-    const int p0 = msk ? __ffs(msk) - 1 : -1, p1 = msk ? 31 - __clz(msk) : -1;
-    uint32_t sd = 0;
-    for (int j = 0; j < 4; ++j) {
-      const uint32_t lo = j == p0 ? 0u : (j == p1 ? 2u : 4u);
-      const uint32_t hi = lo == 4u ? 4u : lo + 1u;
-      sd |= (lo | hi << 4) << (8 * j);
-    }
-    sel_dense[msk] = sd;
-  }
   for (int j = tid; j < tpr; j += kPThreads) {
     const int64_t t = (int64_t)r * tpr + j;
     s_map[j] = p.map[t];
-    s_vo[j] = p.val_off[t];
     s_mo[j] = p.meta_off[t];
   }
   if (warp == 1) {
@@ -226,10 +244,11 @@ __global__ void __launch_bounds__(kPThreads, 1)
             const bool sp = s_map[j] == 1;
             // a range outside the buffers (a corrupted matrix) is not copied
             const bool fits = sp ? (tvo >= 0 && tmo >= 0 && 2 * tvo + kSValBytes <= p.nvb &&
-                                    tmo + kSMetaBytes <= p.nmb && ((2 * tvo) | tmo) % 16 == 0)
+                                    tmo + kSMetaBytes <= p.nmb && tvo % (kPK / 2) == 0 &&
+                                    tmo % 16 == 0)
                                  : (tvo >= 0 && 2 * tvo + kABytes <= p.nvb && tvo % kPK == 0);
             if (!fits) atomicOr(p.status, kStatusBadMap);
-            const uint32_t abytes = fits && !sp ? (uint32_t)kABytes : 0u;
+            const uint32_t abytes = !fits ? 0u : (sp ? (uint32_t)kSValBytes : (uint32_t)kABytes);
             mbar_arrive_expect_tx(&full_bar[s], (uint32_t)kXBytes + abytes);
             // X: tokens m0 .. m0 + 127 (rows past M read as zeros), columns of tile j
             tma_load_2d(xs, &xmap, j * kPK, (int)m0, &full_bar[s]);
@@ -239,7 +258,10 @@ __global__ void __launch_bounds__(kPThreads, 1)
               tma_load_2d(st, &wmap, 0, row, &full_bar[s]);
               tma_load_2d(st + kAtomBytes, &wmap, 64, row, &full_bar[s]);
             } else if (sp) {
-              mbar_arrive(&go_bar[s]);  // the expansion warps may now write the A buffer
+              // the kept values are the sparse MMA's compressed A operand: one
+              // box of 64 values x 128 rows (the 128-byte swizzle layout)
+              if (fits) tma_load_2d(st, &spmap, 0, (int)(tvo / (kPK / 2)), &full_bar[s]);
+              mbar_arrive(&go_bar[s]);  // the metadata buffer of the stage is free
             }
           }
         }
@@ -267,15 +289,30 @@ __global__ void __launch_bounds__(kPThreads, 1)
           tc_fence_after();
           const uint32_t a0 = smem_u32(smem + (size_t)s * kStageBytes);
           const uint32_t b0 = a0 + kABytes;
+          if (sp) {
+            // metadata to tensor memory (4 columns: one per K = 32 product),
+            // then 4 sparse products, A advancing 16 stored values (32 B) and
+            // B 32 columns (64 B) each
+            const uint32_t te = tmem + kTmemE + 4 * s;
+            tmem_cp_128x128b(te, e_desc(b0 + kXBytes));
 #pragma unroll
-          for (int kb = 0; kb < 2; ++kb)
-#pragma unroll
-            for (int kk = 0; kk < 4; ++kk) {
-              // K = 16 columns (32 bytes) at a time inside the 128-byte row
-              const uint32_t off = kb * kAtomBytes + kk * 32;
-              umma_bf16(tmem, sw128_desc(a0 + off), sw128_desc(b0 + off),
-                        (j | kb | kk) != 0 ? 1u : 0u);
+            for (int kb = 0; kb < 4; ++kb) {
+              const uint32_t ecol = te + kb;
+              umma_sp_bf16(tmem, sw128_desc(a0 + kb * 32),
+                           sw128_desc(b0 + (kb >> 1) * kAtomBytes + (kb & 1) * 64), ecol & ~1u,
+                           ecol & 1u, (j | kb) != 0 ? 1u : 0u);
             }
+          } else {
+#pragma unroll
+            for (int kb = 0; kb < 2; ++kb)
+#pragma unroll
+              for (int kk = 0; kk < 4; ++kk) {
+                // K = 16 columns (32 bytes) at a time inside the 128-byte row
+                const uint32_t off = kb * kAtomBytes + kk * 32;
+                umma_bf16(tmem, sw128_desc(a0 + off), sw128_desc(b0 + off),
+                          (j | kb | kk) != 0 ? 1u : 0u);
+              }
+          }
           umma_commit(&empty_bar[s]);
         }
       }
@@ -290,80 +327,68 @@ __global__ void __launch_bounds__(kPThreads, 1)
     }
     __syncwarp();
   } else if (warp >= 4) {
-    // ------------------- 2:4 expansion, then the epilogue -------------------
+    // ------------- 2:4 metadata for the sparse MMA, then the epilogue -------------
+    // The sparse MMA reads, per K = 32 product kb, a tensor-memory column in
+    // which lane L = r0 + 8 k1 + 16 r2 holds rows r = r0 + 8 r1 + 16 r2
+    // (r1 = 0, 1) in its 16-bit halves r1: the four 4-column chunks c of the
+    // product's columns 16 k1 .. 16 k1 + 15, one nibble each (c = 0 lowest),
+    // a nibble being the two kept positions p0 < p1 as p0 | p1 << 2.  The
+    // buffer is copied to tensor memory by tcgen05.cp (lane L: bytes 16 L ..
+    // 16 L + 15, column kb: bytes 4 kb .. 4 kb + 3).
     const int e = tid - 128;
-    const int i = e & 127;   // tile row
-    const int hf = e >> 7;   // half of the row: columns 64 hf .. 64 hf + 63
+    const int row = e & 127;  // tile row
+    const int hf = e >> 7;    // half of the row: products 2 hf, 2 hf + 1
+    const int r0 = row & 7, r1 = (row >> 3) & 1, r2 = row >> 4;
     bool ok = true;
     uint32_t go_ph = 0;  // bit s: parity of stage s's next 2:4 use
-    // half a row of a 2:4 tile: 32 kept values (4 x 16 B) and 16 mask nibbles
-    // (8 B); a range outside the buffers (a corrupted matrix) reads nothing
-    // and expands zeros (the producer flags it)
-    auto load_row = [&](int j, uint4 (&v)[5]) {
-      const int64_t vo = s_vo[j], mo = s_mo[j];
-      const bool fits = vo >= 0 && mo >= 0 && 2 * vo + kSValBytes <= p.nvb &&
-                        mo + kSMetaBytes <= p.nmb && ((2 * vo) | mo) % 16 == 0;
-      const uint4 *src = reinterpret_cast<const uint4 *>(p.vals + vo + (int64_t)i * (kPK / 2) +
-                                                          hf * (kPK / 4));
-      const uint2 *msk = reinterpret_cast<const uint2 *>(p.meta + mo + (int64_t)i * (kPK / 8) +
-                                                          hf * (kPK / 16));
-#pragma unroll
-      for (int q = 0; q < 4; ++q) v[q] = fits ? __ldg(src + q) : make_uint4(0, 0, 0, 0);
-      const uint2 m = fits ? __ldg(msk) : make_uint2(0, 0);
-      v[4] = make_uint4(m.x, m.y, 0, 0);
+    // the half-row's 16 mask nibbles (8 bytes); a range outside the buffer (a
+    // corrupted matrix) reads nothing (the producer flags it)
+    auto load_masks = [&](int j) -> uint2 {
+      const int64_t mo = s_mo[j];
+      const bool fits = mo >= 0 && mo + kSMetaBytes <= p.nmb && mo % 16 == 0;
+      return fits ? __ldg(reinterpret_cast<const uint2 *>(p.meta + mo + (int64_t)row * (kPK / 8) +
+                                                         hf * (kPK / 16)))
+                  : make_uint2(0, 0);
     };
+    // kept positions of a mask nibble as p0 | p1 << 2 (masks with two bits set;
+    // any other mask gives 0)
+    constexpr uint64_t kIdx = (0x4ull << 12) | (0x8ull << 20) | (0x9ull << 24) | (0xCull << 36) |
+                              (0xDull << 40) | (0xEull << 48);
     auto next_sparse = [&](int j) {
       int q = j + 1;
       while (q < tpr && s_map[q] != 1) ++q;
       return q;
     };
-    // expand 2:4 tile j (its half-row in v) into its stage's A buffer
-    auto expand = [&](int j, const uint4 (&v)[5]) -> bool {
+    int j = next_sparse(-1);
+    uint2 cur = j < tpr ? load_masks(j) : make_uint2(0, 0);
+    while (j < tpr) {
+      const int jn = next_sparse(j);
+      const uint2 nxt = jn < tpr ? load_masks(jn) : make_uint2(0, 0);
       const int s = j % kPStages;
-      if (!mbar_wait(&go_bar[s], (go_ph >> s) & 1u)) return false;
+      if (!mbar_wait(&go_bar[s], (go_ph >> s) & 1u)) {
+        ok = false;
+        break;
+      }
       go_ph ^= 1u << s;
-      uint8_t *st = smem + (size_t)s * kStageBytes;
-      const uint4 mv = v[4];
+      uint8_t *eb = smem + (size_t)s * kStageBytes + kABytes + kXBytes;
 #pragma unroll
-      for (int hp = 0; hp < 4; ++hp) {
-        // piece pc: groups 4pc .. 4pc + 3 = columns 16pc .. 16pc + 15
-        const int pc = 4 * hf + hp;
-        const uint4 w4 = v[hp];
-        const uint32_t m16 = ((hp & 2) ? mv.y : mv.x) >> (16 * (hp & 1)) & 0xFFFFu;
-        const uint32_t kv[4] = {w4.x, w4.y, w4.z, w4.w};
-        uint32_t w[8];
+      for (int kk = 0; kk < 2; ++kk) {
+        const int kb = 2 * hf + kk;
+        const uint32_t w = kk ? cur.y : cur.x;  // chunks 8 kb .. 8 kb + 7 (2 per byte)
 #pragma unroll
-        for (int g = 0; g < 4; ++g) {
-          const uint32_t sd = sel_dense[(m16 >> (4 * g)) & 0xFu];
-          w[2 * g] = __byte_perm(kv[g], 0u, sd);
-          w[2 * g + 1] = __byte_perm(kv[g], 0u, sd >> 16);
-        }
+        for (int k1 = 0; k1 < 2; ++k1) {
+          const uint32_t m16 = (w >> (16 * k1)) & 0xFFFFu;
+          uint32_t v = 0;
 #pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          // 16-byte chunk c of the dense row (8 columns), swizzled by row: the
-          // 8 rows of a store phase land in different banks
-          const int c = 2 * pc + h;
-          uint8_t *dst = st + (c >> 3) * kAtomBytes + i * 128 + (((c & 7) ^ (i & 7)) << 4);
-          *reinterpret_cast<uint4 *>(dst) =
-              make_uint4(w[4 * h], w[4 * h + 1], w[4 * h + 2], w[4 * h + 3]);
+          for (int c = 0; c < 4; ++c) v |= (uint32_t)((kIdx >> (4 * ((m16 >> (4 * c)) & 0xFu))) & 0xFu) << (4 * c);
+          const int L = r0 + 8 * k1 + 16 * r2;
+          *reinterpret_cast<uint16_t *>(eb + L * 16 + 4 * kb + 2 * r1) = (uint16_t)v;
         }
       }
-      // generic-proxy writes, read next by tcgen05.mma (async proxy)
+      // generic-proxy writes, read next by tcgen05.cp (async proxy)
       asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
       mbar_arrive(&exp_bar[s]);
-      return true;
-    };
-    // the next 2:4 tile's half-row is loaded while this one is expanded
-    int j = next_sparse(-1);
-    uint4 cur[5];
-    if (j < tpr) load_row(j, cur);
-    while (j < tpr && ok) {
-      const int jn = next_sparse(j);
-      uint4 nxt[5];
-      if (jn < tpr) load_row(jn, nxt);
-      if (!(ok = expand(j, cur))) break;
-#pragma unroll
-      for (int q = 0; q < 5; ++q) cur[q] = nxt[q];
+      cur = nxt;
       j = jn;
     }
     if (!ok && lane == 0) atomicOr(p.status, kStatusTimeout);
@@ -372,7 +397,7 @@ __global__ void __launch_bounds__(kPThreads, 1)
     if (mbar_wait(&acc_bar, 0u)) {
       tc_fence_after();
       const int q = warp & 3;
-      const int64_t row = (int64_t)r * kPM + 32 * q + lane;
+      const int64_t yrow = (int64_t)r * kPM + 32 * q + lane;
       const int cb = warp >= 8 ? kPN / 2 : 0;
 #pragma unroll 1
       for (int c0 = cb; c0 < cb + kPN / 2; c0 += 16) {
@@ -381,7 +406,7 @@ __global__ void __launch_bounds__(kPThreads, 1)
 #pragma unroll
         for (int jj = 0; jj < 16; ++jj) {
           const int64_t tok = m0 + c0 + jj;
-          if (tok < p.m) p.Y[tok * p.ldy + row] = v[jj];
+          if (tok < p.m) p.Y[tok * p.ldy + yrow] = v[jj];
         }
       }
     } else if (lane == 0) {
@@ -453,6 +478,12 @@ int hyb_spmm_prefill(const hyb_matrix *A, int64_t m, const uint16_t *X, int64_t 
   rc = encode_sw128(A->vals, (uint64_t)kPK, (uint64_t)(A->n_vals / kPK), (uint64_t)kPK * 2,
                     &wmap);
   if (rc != HYB_OK) return rc;
+  // and as rows of 64 bf16: a 2:4 tile's 128 rows of kept values at element
+  // offset vo are rows vo / 64 .. + 127
+  alignas(64) CUtensorMap spmap{};
+  rc = encode_sw128(A->vals, (uint64_t)(kPK / 2), (uint64_t)(A->n_vals / (kPK / 2)),
+                    (uint64_t)kPK, &spmap);
+  if (rc != HYB_OK) return rc;
 
   PrefillParams prm{};
   prm.map = A->tile_map;
@@ -475,6 +506,6 @@ int hyb_spmm_prefill(const hyb_matrix *A, int64_t m, const uint16_t *X, int64_t 
                            (int)dyn) != cudaSuccess)
     return HYB_ERR_CUDA;
   const dim3 grid((unsigned)(A->n / kPM), (unsigned)((m + kPN - 1) / kPN));
-  hybrid_prefill_kernel<<<grid, kPThreads, dyn, (cudaStream_t)stream>>>(prm, xmap, wmap);
+  hybrid_prefill_kernel<<<grid, kPThreads, dyn, (cudaStream_t)stream>>>(prm, xmap, wmap, spmap);
   return cudaGetLastError() == cudaSuccess ? HYB_OK : HYB_ERR_CUDA;
 }
