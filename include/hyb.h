@@ -244,10 +244,11 @@ HYB_API int hyb_shard_bands(int64_t n, int64_t k, int b1, int b2,
  * Y[m][i] = sum_k W_hat[i][k] X[m][k] for a block of M tokens (PATCH: dense
  * tiles on dense tensor-core kernels, 2:4 tiles on sparse ones, §2 Method):
  * one tcgen05 pipeline per 128-row band and 128-token block, fp32
- * accumulators in tensor memory, the tile's operands moved by TMA (dense
- * tiles as 128-byte-swizzled boxes; a 2:4 tile's kept values and masks
- * staged and expanded to the dense layout in shared memory, so its tensor
- * work is a dense tile's while its bytes are the hybrid format's).
+ * accumulators in tensor memory, the tile's operands moved by TMA in the
+ * 128-byte swizzle layout.  Dense tiles run tcgen05.mma; 2:4 tiles run the
+ * sparse tensor cores (tcgen05.mma.sp): their packed kept values are the
+ * compressed operand as stored, and their masks are converted to the sparse
+ * MMA's metadata inside the kernel.
  *   A: 128 x 128 tiles (HYB_ERR_UNSUPPORTED otherwise), k <= 131072.
  *   X: [m][k] bf16, row stride ldx (>= k, multiple of 8), 16-byte aligned;
  *      m >= 1 (any; the last block's missing tokens read as zeros).
