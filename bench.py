@@ -920,6 +920,8 @@ def main():
     ap.add_argument("--prefill-profile", action="store_true",
                     help="prefill case for a profiler: hyb_spmm_prefill on 4096x14336, "
                          "f = 0.5, 2048 tokens (512 CTAs), --steps eager calls")
+    ap.add_argument("--dense", action="store_true",
+                    help="with --profile: run the row-major dense baseline leg instead")
     ap.add_argument("--profile", action="store_true",
                     help="small case for a profiler: 2 rotating copies (184 MB > L2), "
                          "hybrid product only, no dense / end-to-end / CPU legs")
@@ -963,10 +965,12 @@ def main():
     stream = wl.stream
 
     if args.profile:
-        ms = timed(wl.step, args.steps, args.warmup, stream, world)
+        fn = wl.dense_step if args.dense else wl.step
+        ms = timed(fn, args.steps, args.warmup, stream, world)
         wl.check()
         if rank == 0:
-            print(json.dumps({"profile_run": args.workload, "ms": ms, "steps": args.steps}))
+            print(json.dumps({"profile_run": args.workload + (" dense" if args.dense else ""),
+                              "ms": ms, "steps": args.steps}))
         return 0
     # Every leg runs as a decode engine would run a chain of layers: K calls
     # captured in one CUDA graph, each launched as a programmatic dependent of
