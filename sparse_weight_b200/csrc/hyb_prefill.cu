@@ -47,11 +47,12 @@ constexpr int kXBytes = 2 * kAtomBytes;       // 128 tokens x 128 columns
 constexpr int kSValBytes = kPM * kPK;         // a 2:4 tile's kept values (bf16)
 constexpr int kSMetaBytes = kPM * kPK / 8;    // and masks
 constexpr int kEBytes = kPM * kPK / 8;      // a 2:4 tile's sparse-MMA metadata, 2 KB
-constexpr int kStageBytes = kABytes + kXBytes + kEBytes;  // 66 KB
+constexpr int kStageBytes = kABytes + kXBytes;  // 64 KB
+constexpr int kESlots = 8;                      // metadata ring: 2:4 tiles converted ahead
 constexpr int kPStages = 3;
 constexpr int kPThreads = 384;  // warp 0 TMA, warp 1 MMA + TMEM, warps 4-11 expand + epilogue
 constexpr int kExpThreads = 256;  // two per tile row (columns 0-63, 64-127)
-constexpr int kTmemCols = 256;  // fp32 accumulator (kPN columns), then 4 metadata columns per stage
+constexpr int kTmemCols = 256;  // fp32 accumulator (kPN columns), then 4 metadata columns per slot
 constexpr int kTmemE = kPN;     // first metadata column
 constexpr int kMaxBandTiles = 1024;           // tiles per band (k <= 131072)
 static_assert(kStageBytes % 1024 == 0, "stages keep the 1024-byte swizzle alignment");
@@ -164,13 +165,13 @@ __global__ void __launch_bounds__(kPThreads, 1)
   extern __shared__ uint8_t smem_raw[];
   __shared__ __align__(8) uint64_t full_bar[kPStages];
   __shared__ __align__(8) uint64_t empty_bar[kPStages];
-  // 2:4 tiles: stage s's A buffer is free for an expansion (go) / the
-  // expanded tile is written (exp).  Their phases advance only on 2:4 uses of
-  // the stage; the producer frees a stage only after the MMAs of its previous
-  // use, which for a 2:4 use waited for that expansion, so neither barrier
-  // runs two phases ahead of a thread waiting on it.
-  __shared__ __align__(8) uint64_t go_bar[kPStages];
-  __shared__ __align__(8) uint64_t exp_bar[kPStages];
+  // the metadata ring: slot q holds the metadata of every kESlots-th 2:4 tile
+  // of the band (efull: written; eempty: the MMAs that read it completed).
+  // The converting warps and the MMA warp take the 2:4 tiles in the same
+  // order, and each waits for the other's previous use of the slot, so
+  // neither barrier runs two phases ahead of a thread waiting on it.
+  __shared__ __align__(8) uint64_t efull_bar[kESlots];
+  __shared__ __align__(8) uint64_t eempty_bar[kESlots];
   __shared__ __align__(8) uint64_t acc_bar;
   __shared__ uint32_t s_tmem;
   __shared__ uint8_t s_map[kMaxBandTiles];
@@ -188,8 +189,10 @@ __global__ void __launch_bounds__(kPThreads, 1)
     for (int s = 0; s < kPStages; ++s) {
       mbar_init(&full_bar[s], 1);
       mbar_init(&empty_bar[s], 1);
-      mbar_init(&go_bar[s], 1);
-      mbar_init(&exp_bar[s], kExpThreads);
+    }
+    for (int q = 0; q < kESlots; ++q) {
+      mbar_init(&efull_bar[q], kExpThreads);
+      mbar_init(&eempty_bar[q], 1);
     }
     mbar_init(&acc_bar, 1);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -261,7 +264,6 @@ __global__ void __launch_bounds__(kPThreads, 1)
               // the kept values are the sparse MMA's compressed A operand: one
               // box of 64 values x 128 rows (the 128-byte swizzle layout)
               if (fits) tma_load_2d(st, &spmap, 0, (int)(tvo / (kPK / 2)), &full_bar[s]);
-              mbar_arrive(&go_bar[s]);  // the metadata buffer of the stage is free
             }
           }
         }
@@ -274,17 +276,16 @@ __global__ void __launch_bounds__(kPThreads, 1)
   } else if (warp == 1) {
     // ------------------------------- MMA --------------------------------
     bool ok = true;
-    uint32_t exp_ph = 0;  // bit s: parity of stage s's expansion barrier
+    uint32_t nsp = 0;  // 2:4 tiles multiplied so far
+    const uint32_t eb0 = smem_u32(smem + (size_t)kPStages * kStageBytes);  // metadata ring
     for (int j = 0; j < tpr && ok; ++j) {
       const int s = j % kPStages;
       const uint32_t ph = (uint32_t)(j / kPStages) & 1u;
       if (lane == 0) {
         const bool sp = s_map[j] == 1;
+        const int q = (int)(nsp % kESlots);
         ok = mbar_wait(&full_bar[s], ph);
-        if (ok && sp) {
-          ok = mbar_wait(&exp_bar[s], (exp_ph >> s) & 1u);
-          exp_ph ^= 1u << s;
-        }
+        if (ok && sp) ok = mbar_wait(&efull_bar[q], (nsp / kESlots) & 1u);
         if (ok) {
           tc_fence_after();
           const uint32_t a0 = smem_u32(smem + (size_t)s * kStageBytes);
@@ -293,8 +294,8 @@ __global__ void __launch_bounds__(kPThreads, 1)
             // metadata to tensor memory (4 columns: one per K = 32 product),
             // then 4 sparse products, A advancing 16 stored values (32 B) and
             // B 32 columns (64 B) each
-            const uint32_t te = tmem + kTmemE + 4 * s;
-            tmem_cp_128x128b(te, e_desc(b0 + kXBytes));
+            const uint32_t te = tmem + kTmemE + 4 * q;
+            tmem_cp_128x128b(te, e_desc(eb0 + (uint32_t)q * kEBytes));
 #pragma unroll
             for (int kb = 0; kb < 4; ++kb) {
               const uint32_t ecol = te + kb;
@@ -314,6 +315,10 @@ __global__ void __launch_bounds__(kPThreads, 1)
               }
           }
           umma_commit(&empty_bar[s]);
+          if (sp) {
+            umma_commit(&eempty_bar[q]);  // the slot is free once these products completed
+            ++nsp;
+          }
         }
       }
       ok = __shfl_sync(0xffffffffu, ok, 0);
@@ -340,7 +345,7 @@ __global__ void __launch_bounds__(kPThreads, 1)
     const int hf = e >> 7;    // half of the row: products 2 hf, 2 hf + 1
     const int r0 = row & 7, r1 = (row >> 3) & 1, r2 = row >> 4;
     bool ok = true;
-    uint32_t go_ph = 0;  // bit s: parity of stage s's next 2:4 use
+    uint32_t nsp = 0;  // 2:4 tiles converted so far
     // the half-row's 16 mask nibbles (8 bytes); a range outside the buffer (a
     // corrupted matrix) reads nothing (the producer flags it)
     auto load_masks = [&](int j) -> uint2 {
@@ -364,13 +369,14 @@ __global__ void __launch_bounds__(kPThreads, 1)
     while (j < tpr) {
       const int jn = next_sparse(j);
       const uint2 nxt = jn < tpr ? load_masks(jn) : make_uint2(0, 0);
-      const int s = j % kPStages;
-      if (!mbar_wait(&go_bar[s], (go_ph >> s) & 1u)) {
+      const int q = (int)(nsp % kESlots);
+      // the slot's previous tile has been multiplied
+      if (!mbar_wait(&eempty_bar[q], ((nsp / kESlots) & 1u) ^ 1u)) {
         ok = false;
         break;
       }
-      go_ph ^= 1u << s;
-      uint8_t *eb = smem + (size_t)s * kStageBytes + kABytes + kXBytes;
+      ++nsp;
+      uint8_t *eb = smem + (size_t)kPStages * kStageBytes + (size_t)q * kEBytes;
 #pragma unroll
       for (int kk = 0; kk < 2; ++kk) {
         const int kb = 2 * hf + kk;
@@ -387,7 +393,7 @@ __global__ void __launch_bounds__(kPThreads, 1)
       }
       // generic-proxy writes, read next by tcgen05.cp (async proxy)
       asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-      mbar_arrive(&exp_bar[s]);
+      mbar_arrive(&efull_bar[q]);
       cur = nxt;
       j = jn;
     }
@@ -501,7 +507,7 @@ int hyb_spmm_prefill(const hyb_matrix *A, int64_t m, const uint16_t *X, int64_t 
   prm.ldy = ldy;
   prm.status = static_cast<uint32_t *>(ws);
 
-  const size_t dyn = (size_t)kPStages * kStageBytes + 1024;
+  const size_t dyn = (size_t)kPStages * kStageBytes + (size_t)kESlots * kEBytes + 1024;
   if (cudaFuncSetAttribute(hybrid_prefill_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            (int)dyn) != cudaSuccess)
     return HYB_ERR_CUDA;
