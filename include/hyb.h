@@ -243,7 +243,7 @@ HYB_API int hyb_shard_bands(int64_t n, int64_t k, int b1, int b2,
 /* ---- prefill / large batch on the tensor cores ---------------------------
  * Y[m][i] = sum_k W_hat[i][k] X[m][k] for a block of M tokens (PATCH: dense
  * tiles on dense tensor-core kernels, 2:4 tiles on sparse ones, §2 Method):
- * one tcgen05 pipeline per 128-row band and 128-token block, fp32
+ * one tcgen05 pipeline per 128-row band and block of 128 or 256 tokens, fp32
  * accumulators in tensor memory, the tile's operands moved by TMA in the
  * 128-byte swizzle layout.  Dense tiles run tcgen05.mma; 2:4 tiles run the
  * sparse tensor cores (tcgen05.mma.sp): their packed kept values are the
@@ -256,11 +256,21 @@ HYB_API int hyb_shard_bands(int64_t n, int64_t k, int b1, int b2,
  *      accumulated.
  *   ws: at least hyb_prefill_workspace_bytes() bytes, 256-byte aligned, its
  *      status word zeroed before the first call (hyb_check_status reads and
- *      clears it).  Nothing is allocated.  Asynchronous on `stream`. */
+ *      clears it).  Nothing is allocated.  Asynchronous on `stream`.
+ * hyb_spmm_prefill takes the token block hyb_prefill_block_tokens(n, m)
+ * returns; hyb_spmm_prefill_blocked takes it from block_tokens (128 or 256;
+ * 0 = the same choice; anything else is HYB_ERR_INVALID_ARG).  The two
+ * blocks give the same sums in the same order: Y is bit-identical. */
 HYB_API size_t hyb_prefill_workspace_bytes(void);
+/* 256 when (n / 128) x ceil(m / 256) CTAs still cover the current device's
+ * SMs (half the operand bytes per product), else 128; 0 for n or m < 1. */
+HYB_API int hyb_prefill_block_tokens(int64_t n, int64_t m);
 HYB_API int hyb_spmm_prefill(const hyb_matrix *A, int64_t m, const uint16_t *X, int64_t ldx,
                              float *Y, int64_t ldy, void *ws, size_t ws_bytes,
                              hyb_stream_t stream);
+HYB_API int hyb_spmm_prefill_blocked(const hyb_matrix *A, int64_t m, const uint16_t *X,
+                                     int64_t ldx, float *Y, int64_t ldy, int block_tokens,
+                                     void *ws, size_t ws_bytes, hyb_stream_t stream);
 
 /* ---- gate and up projections sharing one low-rank factor V ---------------
  * 3BASiL §1-§2: a weight is approximated by S + L with L = U V^T of

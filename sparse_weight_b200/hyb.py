@@ -70,7 +70,7 @@ EXPORTS = ["hyb_packed_sizes", "hyb_pack_workspace_bytes", "hyb_pack",
            "hyb_status_string", "hyb_spmv_noalloc", "hyb_spmv_noalloc_max_scratch_bytes",
            "hyb_spmv_noalloc_check_status", "hyb_gate_up_workspace_bytes",
            "hyb_spmm_skinny_gate_up", "hyb_prefill_workspace_bytes", "hyb_spmm_prefill",
-           "hyb_shard_bands",
+           "hyb_prefill_block_tokens", "hyb_spmm_prefill_blocked", "hyb_shard_bands",
            "hyb_plan_entries", "hyb_make_plan", "hyb_selftest_wait_timeout",
            "hyb_spmm_skinny_ex", "hyb_gemv_dense_ex", "hyb_packed_sizes_nm",
            "hyb_pack_nm", "hyb_spmm_skinny_nm"]
@@ -120,6 +120,11 @@ def lib():
     L.hyb_spmm_prefill.argtypes = [ctypes.POINTER(HybMatrix), _I64, _P, _I64, _P, _I64, _P, _SZ,
                                    _P]
     L.hyb_spmm_prefill.restype = _I
+    L.hyb_prefill_block_tokens.argtypes = [_I64, _I64]
+    L.hyb_prefill_block_tokens.restype = _I
+    L.hyb_spmm_prefill_blocked.argtypes = [ctypes.POINTER(HybMatrix), _I64, _P, _I64, _P, _I64,
+                                           _I, _P, _SZ, _P]
+    L.hyb_spmm_prefill_blocked.restype = _I
     L.hyb_lowrank_workspace_bytes.argtypes = [_I64, _I, _I]
     L.hyb_lowrank_workspace_bytes.restype = _SZ
     L.hyb_lowrank_add.argtypes = [_I64, _I64, _I, ctypes.POINTER(HybLowrank), _P, _I64,
@@ -466,9 +471,10 @@ def spmm_skinny(A: Packed, X: torch.Tensor, Y: torch.Tensor = None, ydt: int = H
 
 
 def spmm_prefill(A: Packed, X: torch.Tensor, Y: torch.Tensor = None, ws: torch.Tensor = None,
-                 stream=None) -> torch.Tensor:
+                 stream=None, block_tokens: int = None) -> torch.Tensor:
     """hyb_spmm_prefill: Y[m][n] = W_hat X for m tokens (tensor cores); X bf16
-    [m][k], Y fp32 [m][n]."""
+    [m][k], Y fp32 [m][n].  block_tokens (128 or 256) calls
+    hyb_spmm_prefill_blocked with that token block."""
     Xb = _bits(X)
     m = Xb.shape[0]
     if Y is None:
@@ -476,10 +482,20 @@ def spmm_prefill(A: Packed, X: torch.Tensor, Y: torch.Tensor = None, ws: torch.T
     if ws is None:
         ws = new_workspace(int(lib().hyb_prefill_workspace_bytes()), Xb.device)
     s = A.struct()
-    _check("hyb_spmm_prefill", lib().hyb_spmm_prefill(
-        ctypes.byref(s), m, _ptr(Xb), Xb.stride(0), _ptr(Y), Y.stride(0), _ptr(ws), ws.numel(),
-        _stream(stream)))
+    if block_tokens is None:
+        _check("hyb_spmm_prefill", lib().hyb_spmm_prefill(
+            ctypes.byref(s), m, _ptr(Xb), Xb.stride(0), _ptr(Y), Y.stride(0), _ptr(ws),
+            ws.numel(), _stream(stream)))
+    else:
+        _check("hyb_spmm_prefill_blocked", lib().hyb_spmm_prefill_blocked(
+            ctypes.byref(s), m, _ptr(Xb), Xb.stride(0), _ptr(Y), Y.stride(0), block_tokens,
+            _ptr(ws), ws.numel(), _stream(stream)))
     return Y
+
+
+def prefill_block_tokens(n: int, m: int) -> int:
+    """hyb_prefill_block_tokens: the token block hyb_spmm_prefill takes."""
+    return int(lib().hyb_prefill_block_tokens(n, m))
 
 
 def gate_up_workspace_bytes(Ag: Packed, Au: Packed, batch: int, rank: int) -> int:
