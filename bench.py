@@ -732,18 +732,19 @@ def _sweep_prefill(device, emit, steps=20, warmup=3):
             stream = torch.cuda.current_stream(device)
             cub_ms = timed(lambda i: torch.matmul(X, W.t()), steps, warmup, stream)
             cub_us = cub_ms / steps * 1e3
-            chosen = hyb.prefill_block_tokens(n, m)
-            for f, bt in ((f, bt) for f in (0.0, 0.5, 1.0) for bt in (128, 256)):
+            chosen = hyb.prefill_block_shape(n, m)
+            for f, blk in ((f, blk) for f in (0.0, 0.5, 1.0) for blk in hyb.PREFILL_SHAPES):
                 tmap = inputs.tile_map_fraction(T, f, inputs.seed_of("prefill_sweep", f))
                 P = hyb.pack(W, tmap, 128, 128)
                 ws = hyb.new_workspace(hyb.lib().hyb_prefill_workspace_bytes(), device)
-                ms = timed(lambda i: hyb.spmm_prefill(P, X, Y=Y, ws=ws, block_tokens=bt),
+                ms = timed(lambda i: hyb.spmm_prefill(P, X, Y=Y, ws=ws, block=blk),
                            steps, warmup, stream)
                 hyb.check_status(ws)
                 us = ms / steps * 1e3
                 flops = 2 * m * n * k
                 emit({"sweep": "prefill", "shape": f"{n}x{k}", "tokens": m, "tile": "128x128",
-                      "block_tokens": bt, "chosen_by_hyb_spmm_prefill": bt == chosen,
+                      "block_rows": blk[0], "block_tokens": blk[1],
+                      "chosen_by_hyb_spmm_prefill": tuple(blk) == tuple(chosen),
                       "sparse_tile_frac": float(np.mean(tmap)), "us": round(us, 2),
                       "tensor_roofline": {"bound": "tensor",
                                           "achieved": round(flops / (us * 1e-6) / 1e12, 1),
@@ -922,7 +923,7 @@ def main():
                          "(strong scaling; the default is one replica per rank)")
     ap.add_argument("--prefill-profile", action="store_true",
                     help="prefill case for a profiler: hyb_spmm_prefill on 4096x14336, "
-                         "f = 0.5, 2048 tokens (256-token blocks: 256 CTAs), --steps eager calls")
+                         "f = 0.5, 2048 tokens (two bands x 240 tokens: 144 CTAs), --steps eager calls")
     ap.add_argument("--dense", action="store_true",
                     help="with --profile: run the row-major dense baseline leg instead")
     ap.add_argument("--profile", action="store_true",

@@ -243,8 +243,8 @@ HYB_API int hyb_shard_bands(int64_t n, int64_t k, int b1, int b2,
 /* ---- prefill / large batch on the tensor cores ---------------------------
  * Y[m][i] = sum_k W_hat[i][k] X[m][k] for a block of M tokens (PATCH: dense
  * tiles on dense tensor-core kernels, 2:4 tiles on sparse ones, §2 Method):
- * one tcgen05 pipeline per 128-row band and block of 128 or 256 tokens, fp32
- * accumulators in tensor memory, the tile's operands moved by TMA in the
+ * one tcgen05 pipeline per CTA of one or two 128-row bands and a block of
+ * tokens, fp32 accumulators in tensor memory, the tile's operands moved by TMA in the
  * 128-byte swizzle layout.  Dense tiles run tcgen05.mma; 2:4 tiles run the
  * sparse tensor cores (tcgen05.mma.sp): their packed kept values are the
  * compressed operand as stored, and their masks are converted to the sparse
@@ -257,20 +257,26 @@ HYB_API int hyb_shard_bands(int64_t n, int64_t k, int b1, int b2,
  *   ws: at least hyb_prefill_workspace_bytes() bytes, 256-byte aligned, its
  *      status word zeroed before the first call (hyb_check_status reads and
  *      clears it).  Nothing is allocated.  Asynchronous on `stream`.
- * hyb_spmm_prefill takes the token block hyb_prefill_block_tokens(n, m)
- * returns; hyb_spmm_prefill_blocked takes it from block_tokens (128 or 256;
- * 0 = the same choice; anything else is HYB_ERR_INVALID_ARG).  The two
- * blocks give the same sums in the same order: Y is bit-identical. */
+ * hyb_spmm_prefill takes the CTA shape hyb_prefill_block_shape(n, m)
+ * returns; hyb_spmm_prefill_blocked takes it from (block_rows, block_tokens):
+ * (128, 128), (128, 256) or (256, 240) (two bands sharing each X tile); (0, 0)
+ * = the same choice; anything else is HYB_ERR_INVALID_ARG.  Every shape adds
+ * the same products in the same order: Y is bit-identical. */
 HYB_API size_t hyb_prefill_workspace_bytes(void);
-/* 256 when (n / 128) x ceil(m / 256) CTAs still cover the current device's
- * SMs (half the operand bytes per product), else 128; 0 for n or m < 1. */
-HYB_API int hyb_prefill_block_tokens(int64_t n, int64_t m);
+/* The CTA shape for an n-row weight and m tokens on the current device: of
+ * the three above, the one with the fewest modelled bytes per SM (CTAs
+ * stream their operands from L2 at about the same rate, so a launch takes
+ * its waves of CTAs times the bytes one CTA moves per tile).  Writes
+ * *block_rows and *block_tokens; HYB_ERR_INVALID_ARG for n < 128, m < 1 or a
+ * null pointer (both set to 0). */
+HYB_API int hyb_prefill_block_shape(int64_t n, int64_t m, int *block_rows, int *block_tokens);
 HYB_API int hyb_spmm_prefill(const hyb_matrix *A, int64_t m, const uint16_t *X, int64_t ldx,
                              float *Y, int64_t ldy, void *ws, size_t ws_bytes,
                              hyb_stream_t stream);
 HYB_API int hyb_spmm_prefill_blocked(const hyb_matrix *A, int64_t m, const uint16_t *X,
-                                     int64_t ldx, float *Y, int64_t ldy, int block_tokens,
-                                     void *ws, size_t ws_bytes, hyb_stream_t stream);
+                                     int64_t ldx, float *Y, int64_t ldy, int block_rows,
+                                     int block_tokens, void *ws, size_t ws_bytes,
+                                     hyb_stream_t stream);
 
 /* ---- gate and up projections sharing one low-rank factor V ---------------
  * 3BASiL §1-§2: a weight is approximated by S + L with L = U V^T of

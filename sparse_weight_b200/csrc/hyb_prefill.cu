@@ -59,23 +59,31 @@ constexpr int kExpThreads = 256;  // two per tile row (columns 0-63, 64-127)
 constexpr int kMaxBandTiles = 1024;           // tiles per band (k <= 131072)
 static_assert(kSValBytes == kAtomBytes, "a 2:4 tile's kept values fill one swizzle box");
 
-// The shape of one CTA's pipeline at PN tokens.  A ring slot holds HS
-// half-tiles (64 columns each): A's halves (16 KB each), then X's (PN x 128
-// bytes each); a whole tile per slot at N = 128 (3 slots of 64 KB), a half
-// per slot at N = 256 (4 slots of 48 KB).  TMEM holds the PN-column fp32
-// accumulator, then 4 metadata columns per metadata slot.
-template <int PN>
+// The shape of one CTA's pipeline: NB row bands of 128 rows (1 or 2) and PN
+// tokens.  A ring slot holds HS half-tiles (64 columns each), a half-tile
+// being the bands' A halves (16 KB each) and then X's (PN x 128 bytes): a
+// whole tile per slot for one band and 128 tokens (3 slots of 64 KB), a half
+// per slot otherwise (4 slots of 48 KB for one band and 256 tokens, 3 slots of
+// 62 KB for two bands and 240 tokens).  TMEM holds the bands' PN-column fp32
+// accumulators (band b from column 256 b), then 4 metadata columns per
+// metadata slot (8 slots for one band, 4 in the last 16 columns for two).
+template <int PN, int NB>
 struct PrefillShape {
-  static constexpr int HS = PN == 256 ? 1 : 2;  // half-tiles per ring slot
+  static constexpr int HS = (NB == 1 && PN == 128) ? 2 : 1;  // half-tiles per ring slot
   static constexpr int kXHalfBytes = PN * 128;
-  static constexpr int kSlotBytes = HS * (kAtomBytes + kXHalfBytes);
+  static constexpr int kHalfBytes = NB * kAtomBytes + kXHalfBytes;
+  static constexpr int kSlotBytes = HS * kHalfBytes;
   static constexpr int kSlots = kRingBytes / kSlotBytes;
-  static constexpr int kTmemCols = PN == 256 ? 512 : 256;
-  static constexpr int kTmemE = PN;  // first metadata column
-  static_assert(PN == 128 || PN == 256, "N = 128 or 256 tokens per CTA");
+  static constexpr int kAccStride = 256;                         // band b's accumulator: column 256 b
+  static constexpr int kEsl = NB == 1 ? kESlots : 4;             // metadata slots in use
+  static constexpr int kTmemE = NB == 1 ? PN : 512 - 4 * kEsl;  // first metadata column
+  static constexpr int kTmemCols = kTmemE + 4 * kEsl <= 256 ? 256 : 512;
+  static_assert(NB == 1 || NB == 2, "one or two bands per CTA");
+  static_assert(PN % 16 == 0 && PN >= 16 && PN <= 256, "MMA N: a multiple of 16 up to 256");
   static_assert(kSlots >= 3 && kSlots <= kMaxSlots, "ring depth");
-  static_assert(kSlotBytes % 1024 == 0, "slots keep the 1024-byte swizzle alignment");
-  static_assert(kTmemE + 4 * kESlots <= kTmemCols, "metadata columns fit the allocation");
+  static_assert(kHalfBytes % 1024 == 0, "slots keep the 1024-byte swizzle alignment");
+  static_assert((NB - 1) * kAccStride + PN <= kTmemE, "accumulators before the metadata");
+  static_assert(kTmemE + 4 * kEsl <= kTmemCols && kTmemCols <= 512, "TMEM columns");
 };
 
 // tcgen05.mma instruction descriptor: D fp32, A and B bf16, both K-major,
@@ -195,38 +203,42 @@ struct PrefillParams {
   const int64_t *meta_off;
   int64_t n, k, m;
   int tpr;
+  int bands;         // n / 128
   int64_t nvb, nmb;  // bytes of the value and mask buffers
   float *Y;
   int64_t ldy;
   uint32_t *status;
 };
 
-template <int PN>
+constexpr uint32_t kNoMeta = 0xFFFFFFFFu;  // a mask offset that cannot be used
+
+template <int PN, int NB>
 __global__ void __launch_bounds__(kPThreads, 1)
     hybrid_prefill_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap xmap,
                           const __grid_constant__ CUtensorMap wmap,
                           const __grid_constant__ CUtensorMap spmap) {
-  using Sh = PrefillShape<PN>;
+  using Sh = PrefillShape<PN, NB>;
   constexpr int NS = Sh::kSlots, HS = Sh::HS;
   constexpr uint32_t kIdesc = idesc_f16<PN>();
   extern __shared__ uint8_t smem_raw[];
   __shared__ __align__(8) uint64_t full_bar[kMaxSlots];
   __shared__ __align__(8) uint64_t empty_bar[kMaxSlots];
-  // the metadata ring: slot q holds the metadata of every kESlots-th 2:4 tile
-  // of the band (efull: written; eempty: the MMAs that read it completed).
-  // The converting warps and the MMA warp take the 2:4 tiles in the same
-  // order, and each waits for the other's previous use of the slot, so
-  // neither barrier runs two phases ahead of a thread waiting on it.
+  // the metadata ring: slot q holds the metadata of every kEsl-th 2:4 tile
+  // of the CTA, taken in (tile, band) order (efull: written; eempty: the MMAs
+  // that read it completed).  The converting warps and the MMA warp take the
+  // 2:4 tiles in the same order, and each waits for the other's previous use
+  // of the slot, so neither barrier runs two phases ahead of a waiting thread.
   __shared__ __align__(8) uint64_t efull_bar[kESlots];
   __shared__ __align__(8) uint64_t eempty_bar[kESlots];
   __shared__ __align__(8) uint64_t acc_bar;
   __shared__ uint32_t s_tmem;
-  __shared__ uint8_t s_map[kMaxBandTiles];
-  __shared__ int64_t s_mo[kMaxBandTiles];  // the band's mask offsets
+  __shared__ uint8_t s_map[NB][kMaxBandTiles];
+  __shared__ uint32_t s_mo[NB][kMaxBandTiles];  // the bands' mask offsets / 16, or kNoMeta
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int r = blockIdx.x;                  // tile-row band
-  const int64_t m0 = (int64_t)blockIdx.y * PN;  // first token
+  const int r0 = blockIdx.x * NB;                  // first tile-row band
+  const int nb = min(NB, p.bands - r0);            // bands present (the last CTA may have one)
+  const int64_t m0 = (int64_t)blockIdx.y * PN;     // first token
   const int tpr = p.tpr;
   // ring slots at a 1024-byte boundary (the swizzle pattern repeats every 1024)
   uint8_t *smem =
@@ -244,10 +256,19 @@ __global__ void __launch_bounds__(kPThreads, 1)
     mbar_init(&acc_bar, 1);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
-  for (int j = tid; j < tpr; j += kPThreads) {
-    const int64_t t = (int64_t)r * tpr + j;
-    s_map[j] = p.map[t];
-    s_mo[j] = p.meta_off[t];
+  for (int i = tid; i < NB * tpr; i += kPThreads) {
+    const int b = i / tpr, j = i - b * tpr;
+    uint8_t sp = 0;
+    uint32_t mo16 = kNoMeta;
+    if (b < nb) {
+      const int64_t t = (int64_t)(r0 + b) * tpr + j;
+      sp = p.map[t];
+      const int64_t mo = p.meta_off[t];
+      if (mo >= 0 && mo % 16 == 0 && mo + kSMetaBytes <= p.nmb && mo / 16 < (int64_t)kNoMeta)
+        mo16 = (uint32_t)(mo / 16);
+    }
+    s_map[b][j] = sp;
+    s_mo[b][j] = mo16;
   }
   if (warp == 1) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
@@ -263,35 +284,37 @@ __global__ void __launch_bounds__(kPThreads, 1)
 
   if (warp == 0) {
     // ------------------------------ producer ------------------------------
-    // lane l holds the offsets of tile w0 + l of the band (a window of 32,
-    // the next window loaded while this one is issued)
+    // lane l holds the value offsets of tile w0 + l of each band (a window of
+    // 32, the next window loaded while this one is issued)
     bool ok = true;
-    const int64_t t_band = (int64_t)r * tpr;
-    auto load = [&](int w0, int64_t &vo, int64_t &mo) {
-      vo = mo = 0;
-      if (w0 + lane < tpr) {
-        vo = __ldg(p.val_off + t_band + w0 + lane);
-        mo = __ldg(p.meta_off + t_band + w0 + lane);
-      }
+    auto load = [&](int w0, int64_t (&vo)[NB]) {
+#pragma unroll
+      for (int b = 0; b < NB; ++b)
+        vo[b] = (b < nb && w0 + lane < tpr) ? __ldg(p.val_off + (int64_t)(r0 + b) * tpr + w0 + lane)
+                                            : 0;
     };
-    int64_t vo, mo, nvo, nmo;
-    load(0, vo, mo);
+    int64_t vo[NB], nvo[NB];
+    load(0, vo);
     for (int w0 = 0; w0 < tpr && ok; w0 += 32) {
-      load(w0 + 32, nvo, nmo);
+      load(w0 + 32, nvo);
       const int nw = min(32, tpr - w0);
       for (int l = 0; l < nw && ok; ++l) {
         const int j = w0 + l;
-        const int64_t tvo = __shfl_sync(0xffffffffu, vo, l);
-        const int64_t tmo = __shfl_sync(0xffffffffu, mo, l);
+        int64_t tvo[NB];
+#pragma unroll
+        for (int b = 0; b < NB; ++b) tvo[b] = __shfl_sync(0xffffffffu, vo[b], l);
         if (lane == 0) {
-          const bool sp = s_map[j] == 1;
-          // a range outside the buffers (a corrupted matrix) is not copied
-          const bool fits = sp ? (tvo >= 0 && tmo >= 0 && 2 * tvo + kSValBytes <= p.nvb &&
-                                  tmo + kSMetaBytes <= p.nmb && tvo % (kPK / 2) == 0 &&
-                                  tmo % 16 == 0)
-                               : (tvo >= 0 && 2 * tvo + 2 * kAtomBytes <= p.nvb &&
-                                  tvo % kPK == 0);
-          if (!fits) atomicOr(p.status, kStatusBadMap);
+          bool sp[NB], fits[NB];
+#pragma unroll
+          for (int b = 0; b < NB; ++b) {
+            sp[b] = b < nb && s_map[b][j] == 1;
+            // a range outside the buffers (a corrupted matrix) is not copied
+            fits[b] = b < nb && (sp[b] ? (tvo[b] >= 0 && 2 * tvo[b] + kSValBytes <= p.nvb &&
+                                          tvo[b] % (kPK / 2) == 0 && s_mo[b][j] != kNoMeta)
+                                       : (tvo[b] >= 0 && 2 * tvo[b] + 2 * kAtomBytes <= p.nvb &&
+                                          tvo[b] % kPK == 0));
+            if (b < nb && !fits[b]) atomicOr(p.status, kStatusBadMap);
+          }
           for (int h0 = 0; h0 < 2 && ok; h0 += HS) {
             const int idx = (2 * j + h0) / HS;  // ring position of halves h0 .. h0 + HS - 1
             const int s = idx % NS;
@@ -302,26 +325,37 @@ __global__ void __launch_bounds__(kPThreads, 1)
             uint8_t *st = smem + (size_t)s * Sh::kSlotBytes;
             // A's bytes in this slot: a dense tile's halves, or a 2:4 tile's
             // whole compressed operand with its first half
-            const uint32_t abytes =
-                !fits ? 0u : (sp ? (h0 == 0 ? (uint32_t)kAtomBytes : 0u) : (uint32_t)(HS * kAtomBytes));
-            mbar_arrive_expect_tx(&full_bar[s], (uint32_t)(HS * Sh::kXHalfBytes) + abytes);
+            uint32_t bytes = (uint32_t)(HS * Sh::kXHalfBytes);
+#pragma unroll
+            for (int b = 0; b < NB; ++b)
+              if (fits[b])
+                bytes += sp[b] ? (h0 == 0 ? (uint32_t)kAtomBytes : 0u) : (uint32_t)(HS * kAtomBytes);
+            mbar_arrive_expect_tx(&full_bar[s], bytes);
             for (int hh = 0; hh < HS; ++hh) {
               const int h = h0 + hh;
+              uint8_t *hb = st + (size_t)hh * Sh::kHalfBytes;
               // X: tokens m0 .. m0 + PN - 1 (rows past M read as zeros),
               // columns 64 h .. 64 h + 63 of tile j
-              tma_load_2d(st + HS * kAtomBytes + hh * Sh::kXHalfBytes, &xmap, j * kPK + 64 * h,
-                          (int)m0, &full_bar[s]);
-              if (fits && !sp)  // the tile's first row in the 128-wide view of the values
-                tma_load_2d(st + hh * kAtomBytes, &wmap, 64 * h, (int)(tvo / kPK), &full_bar[s]);
+              tma_load_2d(hb + NB * kAtomBytes, &xmap, j * kPK + 64 * h, (int)m0, &full_bar[s]);
+#pragma unroll
+              for (int b = 0; b < NB; ++b)
+                if (fits[b] && !sp[b])  // the tile's first row in the 128-wide view of the values
+                  tma_load_2d(hb + b * kAtomBytes, &wmap, 64 * h, (int)(tvo[b] / kPK),
+                              &full_bar[s]);
             }
-            if (fits && sp && h0 == 0)  // 64 kept values x 128 rows (128-byte swizzle)
-              tma_load_2d(st, &spmap, 0, (int)(tvo / (kPK / 2)), &full_bar[s]);
+            if (h0 == 0) {
+#pragma unroll
+              for (int b = 0; b < NB; ++b)
+                if (fits[b] && sp[b])  // 64 kept values x 128 rows (128-byte swizzle)
+                  tma_load_2d(st + b * kAtomBytes, &spmap, 0, (int)(tvo[b] / (kPK / 2)),
+                              &full_bar[s]);
+            }
           }
         }
         ok = __shfl_sync(0xffffffffu, ok, 0);
       }
-      vo = nvo;
-      mo = nmo;
+#pragma unroll
+      for (int b = 0; b < NB; ++b) vo[b] = nvo[b];
     }
     if (!ok && lane == 0) atomicOr(p.status, kStatusTimeout);
   } else if (warp == 1) {
@@ -331,59 +365,84 @@ __global__ void __launch_bounds__(kPThreads, 1)
     const uint32_t eb0 = smem_u32(smem + (size_t)kRingBytes);  // metadata ring
     for (int j = 0; j < tpr && ok; ++j) {
       if (lane == 0) {
-        const bool sp = s_map[j] == 1;
-        const int q = (int)(nsp % kESlots);
-        const uint32_t te = tmem + Sh::kTmemE + 4 * q;
-        uint32_t a_sp = 0;  // a 2:4 tile's compressed A (in its first half's slot)
+        bool sp[NB];
+        uint32_t qn[NB];  // metadata ring positions of the 2:4 bands
+        uint32_t c = nsp;
+        bool any_sp = false;
+#pragma unroll
+        for (int b = 0; b < NB; ++b) {
+          sp[b] = b < nb && s_map[b][j] == 1;
+          qn[b] = sp[b] ? c++ : 0u;
+          any_sp = any_sp || sp[b];
+        }
+        uint32_t a_sp = 0;  // the 2:4 bands' compressed A (in the first half's slot)
         int s_first = 0;
         for (int h0 = 0; h0 < 2 && ok; h0 += HS) {
           const int idx = (2 * j + h0) / HS;
           const int s = idx % NS;
           ok = ring_wait(&full_bar[s], (uint32_t)(idx / NS) & 1u);
-          if (ok && sp && h0 == 0) ok = ring_wait(&efull_bar[q], (nsp / kESlots) & 1u);
+          if (h0 == 0) {
+#pragma unroll
+            for (int b = 0; b < NB; ++b)
+              if (ok && sp[b])
+                ok = ring_wait(&efull_bar[qn[b] % Sh::kEsl], (qn[b] / Sh::kEsl) & 1u);
+          }
           if (!ok) break;
           tc_fence_after();
           const uint32_t st = smem_u32(smem + (size_t)s * Sh::kSlotBytes);
-          if (sp && h0 == 0) {
+          if (h0 == 0) {
             // metadata to tensor memory (4 columns: one per K = 32 product)
-            tmem_cp_128x128b(te, e_desc(eb0 + (uint32_t)q * kEBytes));
+#pragma unroll
+            for (int b = 0; b < NB; ++b)
+              if (sp[b])
+                tmem_cp_128x128b(tmem + Sh::kTmemE + 4 * (qn[b] % Sh::kEsl),
+                                 e_desc(eb0 + (qn[b] % Sh::kEsl) * kEBytes));
             a_sp = st;
             s_first = s;
           }
 #pragma unroll
           for (int hh = 0; hh < HS; ++hh) {
             const int h = h0 + hh;
-            const uint32_t a0 = st + hh * kAtomBytes;
-            const uint32_t b0 = st + HS * kAtomBytes + hh * Sh::kXHalfBytes;
-            if (sp) {
-              // products 2h, 2h + 1: A advancing 16 stored values (32 B), B 32
-              // columns (64 B) of this half each
+            const uint32_t hb = st + hh * Sh::kHalfBytes;
+            const uint32_t b0 = hb + NB * kAtomBytes;  // X of this half
 #pragma unroll
-              for (int kk = 0; kk < 2; ++kk) {
-                const int kb = 2 * h + kk;
-                const uint32_t ecol = te + kb;
-                umma_sp_bf16(tmem, sw128_desc(a_sp + kb * 32), sw128_desc(b0 + kk * 64),
-                             ecol & ~1u, ecol & 1u, (j | kb) != 0 ? 1u : 0u, kIdesc);
+            for (int b = 0; b < NB; ++b) {
+              if (b >= nb) continue;
+              const uint32_t d = tmem + b * Sh::kAccStride;  // band b's accumulator
+              if (sp[b]) {
+                // products 2h, 2h + 1: A advancing 16 stored values (32 B), B
+                // 32 columns (64 B) of this half each
+                const uint32_t te = tmem + Sh::kTmemE + 4 * (qn[b] % Sh::kEsl);
+#pragma unroll
+                for (int kk = 0; kk < 2; ++kk) {
+                  const int kb = 2 * h + kk;
+                  const uint32_t ecol = te + kb;
+                  umma_sp_bf16(d, sw128_desc(a_sp + b * kAtomBytes + kb * 32),
+                               sw128_desc(b0 + kk * 64), ecol & ~1u, ecol & 1u,
+                               (j | kb) != 0 ? 1u : 0u, kIdesc);
+                }
+              } else {
+#pragma unroll
+                for (int kk = 0; kk < 4; ++kk)
+                  // K = 16 columns (32 bytes) at a time inside the 128-byte row
+                  umma_bf16(d, sw128_desc(hb + b * kAtomBytes + kk * 32), sw128_desc(b0 + kk * 32),
+                            (j | h | kk) != 0 ? 1u : 0u, kIdesc);
               }
-            } else {
-#pragma unroll
-              for (int kk = 0; kk < 4; ++kk)
-                // K = 16 columns (32 bytes) at a time inside the 128-byte row
-                umma_bf16(tmem, sw128_desc(a0 + kk * 32), sw128_desc(b0 + kk * 32),
-                          (j | h | kk) != 0 ? 1u : 0u, kIdesc);
             }
           }
-          // the slot is free once its products completed; a 2:4 tile's first
-          // slot holds A for the second half too
-          if (!sp || HS == 2) {
+          // a slot is free once its products completed; with a 2:4 band, the
+          // first half's slot holds that band's A for the second half too
+          if (!any_sp || HS == 2) {
             umma_commit(&empty_bar[s]);
           } else if (h0 == 1) {
             umma_commit(&empty_bar[s_first]);
             umma_commit(&empty_bar[s]);
           }
-          if (sp && h0 + HS == 2) {
-            umma_commit(&eempty_bar[q]);  // the metadata slot is free once these completed
-            ++nsp;
+          if (h0 + HS == 2) {
+#pragma unroll
+            for (int b = 0; b < NB; ++b)
+              if (sp[b]) umma_commit(&eempty_bar[qn[b] % Sh::kEsl]);  // metadata slot free
+            nsp = c;
           }
         }
       }
@@ -391,7 +450,7 @@ __global__ void __launch_bounds__(kPThreads, 1)
     }
     if (lane == 0) {
       if (!ok) atomicOr(p.status, kStatusTimeout);
-      // the accumulator is final once every MMA issued above has completed
+      // the accumulators are final once every MMA issued above has completed
       // (also after a timeout, so that nothing is in flight at the end)
       umma_commit(&acc_bar);
       if (!ring_wait(&acc_bar, 0u)) atomicOr(p.status, kStatusTimeout);
@@ -409,35 +468,36 @@ __global__ void __launch_bounds__(kPThreads, 1)
     const int e = tid - 128;
     const int row = e & 127;  // tile row
     const int hf = e >> 7;    // half of the row: products 2 hf, 2 hf + 1
-    const int r0 = row & 7, r1 = (row >> 3) & 1, r2 = row >> 4;
+    const int q0 = row & 7, q1 = (row >> 3) & 1, q2 = row >> 4;
     bool ok = true;
     uint32_t nsp = 0;  // 2:4 tiles converted so far
-    // the half-row's 16 mask nibbles (8 bytes); a range outside the buffer (a
-    // corrupted matrix) reads nothing (the producer flags it)
-    auto load_masks = [&](int j) -> uint2 {
-      const int64_t mo = s_mo[j];
-      const bool fits = mo >= 0 && mo + kSMetaBytes <= p.nmb && mo % 16 == 0;
-      return fits ? __ldg(reinterpret_cast<const uint2 *>(p.meta + mo + (int64_t)row * (kPK / 8) +
-                                                         hf * (kPK / 16)))
-                  : make_uint2(0, 0);
+    // the half-row's 16 mask nibbles (8 bytes) of 2:4 tile (position pos =
+    // NB j + b); an offset that is unusable reads nothing (the producer flags it)
+    auto load_masks = [&](int pos) -> uint2 {
+      const uint32_t mo16 = s_mo[pos % NB][pos / NB];
+      return mo16 != kNoMeta
+                 ? __ldg(reinterpret_cast<const uint2 *>(p.meta + (int64_t)mo16 * 16 +
+                                                         (int64_t)row * (kPK / 8) + hf * (kPK / 16)))
+                 : make_uint2(0, 0);
     };
     // kept positions of a mask nibble as p0 | p1 << 2 (masks with two bits set;
     // any other mask gives 0)
     constexpr uint64_t kIdx = (0x4ull << 12) | (0x8ull << 20) | (0x9ull << 24) | (0xCull << 36) |
                               (0xDull << 40) | (0xEull << 48);
-    auto next_sparse = [&](int j) {
-      int q = j + 1;
-      while (q < tpr && s_map[q] != 1) ++q;
+    const int npos = NB * tpr;
+    auto next_sparse = [&](int pos) {
+      int q = pos + 1;
+      while (q < npos && !(q % NB < nb && s_map[q % NB][q / NB] == 1)) ++q;
       return q;
     };
-    int j = next_sparse(-1);
-    uint2 cur = j < tpr ? load_masks(j) : make_uint2(0, 0);
-    while (j < tpr) {
-      const int jn = next_sparse(j);
-      const uint2 nxt = jn < tpr ? load_masks(jn) : make_uint2(0, 0);
-      const int q = (int)(nsp % kESlots);
+    int pos = next_sparse(-1);
+    uint2 cur = pos < npos ? load_masks(pos) : make_uint2(0, 0);
+    while (pos < npos) {
+      const int pn = next_sparse(pos);
+      const uint2 nxt = pn < npos ? load_masks(pn) : make_uint2(0, 0);
+      const int q = (int)(nsp % Sh::kEsl);
       // the slot's previous tile has been multiplied
-      if (!ring_wait(&eempty_bar[q], ((nsp / kESlots) & 1u) ^ 1u)) {
+      if (!ring_wait(&eempty_bar[q], ((nsp / Sh::kEsl) & 1u) ^ 1u)) {
         ok = false;
         break;
       }
@@ -453,32 +513,37 @@ __global__ void __launch_bounds__(kPThreads, 1)
           uint32_t v = 0;
 #pragma unroll
           for (int c = 0; c < 4; ++c) v |= (uint32_t)((kIdx >> (4 * ((m16 >> (4 * c)) & 0xFu))) & 0xFu) << (4 * c);
-          const int L = r0 + 8 * k1 + 16 * r2;
-          *reinterpret_cast<uint16_t *>(eb + L * 16 + 4 * kb + 2 * r1) = (uint16_t)v;
+          const int L = q0 + 8 * k1 + 16 * q2;
+          *reinterpret_cast<uint16_t *>(eb + L * 16 + 4 * kb + 2 * q1) = (uint16_t)v;
         }
       }
       // generic-proxy writes, read next by tcgen05.cp (async proxy)
       asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
       mbar_arrive(&efull_bar[q]);
       cur = nxt;
-      j = jn;
+      pos = pn;
     }
     if (!ok && lane == 0) atomicOr(p.status, kStatusTimeout);
     // epilogue: TMEM lanes 32 (warp % 4) .. + 31 are this warp's weight rows;
-    // warps 4-7 store the block's first PN / 2 tokens, warps 8-11 the rest
+    // one band: warps 4-7 store the block's first PN / 2 tokens, warps 8-11
+    // the rest; two bands: warps 4-7 band 0, warps 8-11 band 1, every token
     if (ring_wait(&acc_bar, 0u)) {
       tc_fence_after();
-      const int q = warp & 3;
-      const int64_t yrow = (int64_t)r * kPM + 32 * q + lane;
-      const int cb = warp >= 8 ? PN / 2 : 0;
+      const int qw = warp & 3;
+      const int b = NB == 2 && warp >= 8 ? 1 : 0;
+      const int cb = NB == 1 && warp >= 8 ? PN / 2 : 0;
+      const int ce = NB == 1 ? cb + PN / 2 : PN;
+      if (b < nb) {
+        const int64_t yrow = (int64_t)(r0 + b) * kPM + 32 * qw + lane;
 #pragma unroll 1
-      for (int c0 = cb; c0 < cb + PN / 2; c0 += 16) {
-        float v[16];
-        tmem_ld16(tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)c0, v);
+        for (int c0 = cb; c0 < ce; c0 += 16) {
+          float v[16];
+          tmem_ld16(tmem + ((uint32_t)(32 * qw) << 16) + (uint32_t)(b * Sh::kAccStride + c0), v);
 #pragma unroll
-        for (int jj = 0; jj < 16; ++jj) {
-          const int64_t tok = m0 + c0 + jj;
-          if (tok < p.m) p.Y[tok * p.ldy + yrow] = v[jj];
+          for (int jj = 0; jj < 16; ++jj) {
+            const int64_t tok = m0 + c0 + jj;
+            if (tok < p.m) p.Y[tok * p.ldy + yrow] = v[jj];
+          }
         }
       }
     } else if (lane == 0) {
@@ -511,17 +576,20 @@ int encode_sw128(const void *base, uint64_t cols, uint64_t rows, uint64_t row_by
   return res == CUDA_SUCCESS ? HYB_OK : HYB_ERR_CUDA;
 }
 
-template <int PN>
+template <int PN, int NB>
 int launch_prefill(const PrefillParams &prm, const CUtensorMap &xmap, const CUtensorMap &wmap,
-                   const CUtensorMap &spmap, int64_t bands, int64_t m, cudaStream_t stream) {
+                   const CUtensorMap &spmap, int64_t m, cudaStream_t stream) {
   const size_t dyn = (size_t)kRingBytes + (size_t)kESlots * kEBytes + 1024;
-  if (cudaFuncSetAttribute(hybrid_prefill_kernel<PN>,
+  if (cudaFuncSetAttribute(hybrid_prefill_kernel<PN, NB>,
                            cudaFuncAttributeMaxDynamicSharedMemorySize, (int)dyn) != cudaSuccess)
     return HYB_ERR_CUDA;
-  const dim3 grid((unsigned)bands, (unsigned)((m + PN - 1) / PN));
-  hybrid_prefill_kernel<PN><<<grid, kPThreads, dyn, stream>>>(prm, xmap, wmap, spmap);
+  const dim3 grid((unsigned)((prm.bands + NB - 1) / NB), (unsigned)((m + PN - 1) / PN));
+  hybrid_prefill_kernel<PN, NB><<<grid, kPThreads, dyn, stream>>>(prm, xmap, wmap, spmap);
   return cudaGetLastError() == cudaSuccess ? HYB_OK : HYB_ERR_CUDA;
 }
+
+// The CTA shapes (rows, tokens) the kernel is built for.
+constexpr int kShapes[3][2] = {{128, 128}, {128, 256}, {256, 240}};
 
 }  // namespace
 }  // namespace hyb
@@ -530,28 +598,50 @@ using namespace hyb;
 
 size_t hyb_prefill_workspace_bytes(void) { return kHeaderBytes; }
 
-int hyb_prefill_block_tokens(int64_t n, int64_t m) {
-  if (n <= 0 || m <= 0) return 0;
+int hyb_prefill_block_shape(int64_t n, int64_t m, int *block_rows, int *block_tokens) {
+  if (!block_rows || !block_tokens) return HYB_ERR_INVALID_ARG;
+  *block_rows = *block_tokens = 0;
+  if (n < kPM || m < 1) return HYB_ERR_INVALID_ARG;
   int sms = 148;
   int dev = 0;
   if (cudaGetDevice(&dev) == cudaSuccess)
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  // 256 tokens per CTA when that grid still gives every SM a CTA
-  const int64_t ctas256 = ((n + kPM - 1) / kPM) * ((m + 255) / 256);
-  return ctas256 >= sms ? 256 : 128;
+  if (sms < 1) sms = 148;
+  // Every shape streams its operands from L2 at about the same rate per SM,
+  // so a CTA's time goes with the bytes it moves per tile (its bands' A and
+  // its tokens' X), and the launch's with that times its waves of CTAs.
+  const int64_t bands = (n + kPM - 1) / kPM;
+  int64_t best = -1;
+  for (const auto &sh : kShapes) {
+    const int nb = sh[0] / kPM, pn = sh[1];
+    if (nb > bands) continue;
+    const int64_t ctas = ((bands + nb - 1) / nb) * ((m + pn - 1) / pn);
+    const int64_t cost = ((ctas + sms - 1) / sms) * ((int64_t)nb * 2 * kAtomBytes + (int64_t)pn * 256);
+    if (best < 0 || cost < best) {
+      best = cost;
+      *block_rows = sh[0];
+      *block_tokens = pn;
+    }
+  }
+  return HYB_OK;
 }
 
 int hyb_spmm_prefill_blocked(const hyb_matrix *A, int64_t m, const uint16_t *X, int64_t ldx,
-                             float *Y, int64_t ldy, int block_tokens, void *ws, size_t ws_bytes,
-                             hyb_stream_t stream) {
+                             float *Y, int64_t ldy, int block_rows, int block_tokens, void *ws,
+                             size_t ws_bytes, hyb_stream_t stream) {
   if (!A || !X || !Y || m < 1) return HYB_ERR_INVALID_ARG;
-  if (block_tokens != 0 && block_tokens != 128 && block_tokens != 256)
-    return HYB_ERR_INVALID_ARG;
   if (A->b1 != kPM || A->b2 != kPK) return HYB_ERR_UNSUPPORTED;
   if (A->n <= 0 || A->k <= 0 || A->n % kPM != 0 || A->k % kPK != 0)
     return HYB_ERR_INVALID_ARG;
+  int rows = block_rows, pn = block_tokens;
+  if (rows == 0 && pn == 0) {
+    const int rc = hyb_prefill_block_shape(A->n, m, &rows, &pn);
+    if (rc != HYB_OK) return rc;
+  }
+  bool known = false;
+  for (const auto &sh : kShapes) known = known || (sh[0] == rows && sh[1] == pn);
+  if (!known) return HYB_ERR_INVALID_ARG;
   const int64_t tpr = A->k / kPK;
-  const int pn = block_tokens ? block_tokens : hyb_prefill_block_tokens(A->n, m);
   if (tpr > kMaxBandTiles || A->n / kPM > INT32_MAX || (m + pn - 1) / pn > 65535 ||
       m > INT32_MAX)
     return HYB_ERR_UNSUPPORTED;
@@ -596,19 +686,20 @@ int hyb_spmm_prefill_blocked(const hyb_matrix *A, int64_t m, const uint16_t *X, 
   prm.k = A->k;
   prm.m = m;
   prm.tpr = (int)tpr;
+  prm.bands = (int)(A->n / kPM);
   prm.nvb = 2 * A->n_vals;
   prm.nmb = A->n_meta_bytes;
   prm.Y = Y;
   prm.ldy = ldy;
   prm.status = static_cast<uint32_t *>(ws);
 
-  const int64_t bands = A->n / kPM;
-  return pn == 256
-             ? launch_prefill<256>(prm, xmap, wmap, spmap, bands, m, (cudaStream_t)stream)
-             : launch_prefill<128>(prm, xmap, wmap, spmap, bands, m, (cudaStream_t)stream);
+  cudaStream_t st = (cudaStream_t)stream;
+  if (rows == 256) return launch_prefill<240, 2>(prm, xmap, wmap, spmap, m, st);
+  return pn == 256 ? launch_prefill<256, 1>(prm, xmap, wmap, spmap, m, st)
+                   : launch_prefill<128, 1>(prm, xmap, wmap, spmap, m, st);
 }
 
 int hyb_spmm_prefill(const hyb_matrix *A, int64_t m, const uint16_t *X, int64_t ldx, float *Y,
                      int64_t ldy, void *ws, size_t ws_bytes, hyb_stream_t stream) {
-  return hyb_spmm_prefill_blocked(A, m, X, ldx, Y, ldy, 0, ws, ws_bytes, stream);
+  return hyb_spmm_prefill_blocked(A, m, X, ldx, Y, ldy, 0, 0, ws, ws_bytes, stream);
 }

@@ -70,7 +70,7 @@ EXPORTS = ["hyb_packed_sizes", "hyb_pack_workspace_bytes", "hyb_pack",
            "hyb_status_string", "hyb_spmv_noalloc", "hyb_spmv_noalloc_max_scratch_bytes",
            "hyb_spmv_noalloc_check_status", "hyb_gate_up_workspace_bytes",
            "hyb_spmm_skinny_gate_up", "hyb_prefill_workspace_bytes", "hyb_spmm_prefill",
-           "hyb_prefill_block_tokens", "hyb_spmm_prefill_blocked", "hyb_shard_bands",
+           "hyb_prefill_block_shape", "hyb_spmm_prefill_blocked", "hyb_shard_bands",
            "hyb_plan_entries", "hyb_make_plan", "hyb_selftest_wait_timeout",
            "hyb_spmm_skinny_ex", "hyb_gemv_dense_ex", "hyb_packed_sizes_nm",
            "hyb_pack_nm", "hyb_spmm_skinny_nm"]
@@ -120,10 +120,10 @@ def lib():
     L.hyb_spmm_prefill.argtypes = [ctypes.POINTER(HybMatrix), _I64, _P, _I64, _P, _I64, _P, _SZ,
                                    _P]
     L.hyb_spmm_prefill.restype = _I
-    L.hyb_prefill_block_tokens.argtypes = [_I64, _I64]
-    L.hyb_prefill_block_tokens.restype = _I
+    L.hyb_prefill_block_shape.argtypes = [_I64, _I64, ctypes.POINTER(_I), ctypes.POINTER(_I)]
+    L.hyb_prefill_block_shape.restype = _I
     L.hyb_spmm_prefill_blocked.argtypes = [ctypes.POINTER(HybMatrix), _I64, _P, _I64, _P, _I64,
-                                           _I, _P, _SZ, _P]
+                                           _I, _I, _P, _SZ, _P]
     L.hyb_spmm_prefill_blocked.restype = _I
     L.hyb_lowrank_workspace_bytes.argtypes = [_I64, _I, _I]
     L.hyb_lowrank_workspace_bytes.restype = _SZ
@@ -471,10 +471,10 @@ def spmm_skinny(A: Packed, X: torch.Tensor, Y: torch.Tensor = None, ydt: int = H
 
 
 def spmm_prefill(A: Packed, X: torch.Tensor, Y: torch.Tensor = None, ws: torch.Tensor = None,
-                 stream=None, block_tokens: int = None) -> torch.Tensor:
+                 stream=None, block=None) -> torch.Tensor:
     """hyb_spmm_prefill: Y[m][n] = W_hat X for m tokens (tensor cores); X bf16
-    [m][k], Y fp32 [m][n].  block_tokens (128 or 256) calls
-    hyb_spmm_prefill_blocked with that token block."""
+    [m][k], Y fp32 [m][n].  block = (rows, tokens) calls
+    hyb_spmm_prefill_blocked with that CTA shape."""
     Xb = _bits(X)
     m = Xb.shape[0]
     if Y is None:
@@ -482,20 +482,26 @@ def spmm_prefill(A: Packed, X: torch.Tensor, Y: torch.Tensor = None, ws: torch.T
     if ws is None:
         ws = new_workspace(int(lib().hyb_prefill_workspace_bytes()), Xb.device)
     s = A.struct()
-    if block_tokens is None:
+    if block is None:
         _check("hyb_spmm_prefill", lib().hyb_spmm_prefill(
             ctypes.byref(s), m, _ptr(Xb), Xb.stride(0), _ptr(Y), Y.stride(0), _ptr(ws),
             ws.numel(), _stream(stream)))
     else:
         _check("hyb_spmm_prefill_blocked", lib().hyb_spmm_prefill_blocked(
-            ctypes.byref(s), m, _ptr(Xb), Xb.stride(0), _ptr(Y), Y.stride(0), block_tokens,
+            ctypes.byref(s), m, _ptr(Xb), Xb.stride(0), _ptr(Y), Y.stride(0), block[0], block[1],
             _ptr(ws), ws.numel(), _stream(stream)))
     return Y
 
 
-def prefill_block_tokens(n: int, m: int) -> int:
-    """hyb_prefill_block_tokens: the token block hyb_spmm_prefill takes."""
-    return int(lib().hyb_prefill_block_tokens(n, m))
+PREFILL_SHAPES = ((128, 128), (128, 256), (256, 240))
+
+
+def prefill_block_shape(n: int, m: int):
+    """hyb_prefill_block_shape: the (rows, tokens) CTA shape hyb_spmm_prefill takes."""
+    r, t = ctypes.c_int(0), ctypes.c_int(0)
+    _check("hyb_prefill_block_shape",
+           lib().hyb_prefill_block_shape(n, m, ctypes.byref(r), ctypes.byref(t)))
+    return r.value, t.value
 
 
 def gate_up_workspace_bytes(Ag: Packed, Au: Packed, batch: int, rank: int) -> int:

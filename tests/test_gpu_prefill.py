@@ -11,11 +11,14 @@ from gpu_cases import assert_within, case, dev
 pytestmark = pytest.mark.gpu
 
 
-def _check(orc, n, k, m, tmap, name, rows=None, bt=None):
+SHAPES = list(hyb.PREFILL_SHAPES)
+
+
+def _check(orc, n, k, m, tmap, name, rows=None, block=None):
     W, tmap, X, _ = case(n, k, 128, 128, tmap, batch=m, name=name)
     P = hyb.pack(W.to(dev()), tmap, 128, 128)
     ws = hyb.new_workspace(hyb.lib().hyb_prefill_workspace_bytes(), dev())
-    Y = hyb.spmm_prefill(P, X.to(dev()), ws=ws, block_tokens=bt)
+    Y = hyb.spmm_prefill(P, X.to(dev()), ws=ws, block=block)
     torch.cuda.synchronize()
     assert hyb.check_status(ws) == 0
     Yh = Y.cpu().numpy()
@@ -29,42 +32,44 @@ def _check(orc, n, k, m, tmap, name, rows=None, bt=None):
     return P, X, Y
 
 
-@pytest.mark.parametrize("bt", [128, 256])
+@pytest.mark.parametrize("block", SHAPES)
 @pytest.mark.parametrize("frac", [0.0, 0.5, 1.0])
 @pytest.mark.parametrize("m", [64, 128, 200, 300])
-def test_prefill_fractions(orc, frac, m, bt):
+def test_prefill_fractions(orc, frac, m, block):
     """Every tile dense, half and half, every tile 2:4; one token block, a
-    full block, ragged second blocks; 128- and 256-token blocks."""
+    full block, ragged second blocks; every CTA shape (one band x 128 or 256
+    tokens, two bands x 240 tokens)."""
     n, k = 512, 1024
     T = (n // 128) * (k // 128)
     tmap = inputs.tile_map_fraction(T, frac, inputs.seed_of("prefill", frac))
-    _check(orc, n, k, m, tmap, f"prefill_f{frac}", bt=bt)
+    _check(orc, n, k, m, tmap, f"prefill_f{frac}", block=block)
 
 
-@pytest.mark.parametrize("bt", [128, 256])
+@pytest.mark.parametrize("block", SHAPES)
 @pytest.mark.parametrize("m", [1, 129, 1000])
-def test_prefill_ragged_tokens(orc, m, bt):
+def test_prefill_ragged_tokens(orc, m, block):
     """Token counts that leave most of a block empty (rows past m read as
-    zeros and are never stored)."""
+    zeros and are never stored); 3 bands, so the two-band shape's last CTA
+    has one."""
     n, k = 384, 768
     T = (n // 128) * (k // 128)
     tmap = inputs.tile_map_bernoulli(T, 0.5, inputs.seed_of("prefill_ragged", m))
-    _check(orc, n, k, m, tmap, "prefill_ragged", bt=bt)
+    _check(orc, n, k, m, tmap, "prefill_ragged", block=block)
 
 
-@pytest.mark.parametrize("bt", [128, 256])
-def test_prefill_4096_tokens(orc, bt):
-    """The long end of prefill: 4096 tokens (32 or 16 token blocks) on a small
-    weight, every output checked."""
+@pytest.mark.parametrize("block", SHAPES)
+def test_prefill_4096_tokens(orc, block):
+    """The long end of prefill: 4096 tokens on a small weight, every output
+    checked."""
     n, k, m = 256, 1024, 4096
     T = (n // 128) * (k // 128)
     tmap = inputs.tile_map_bernoulli(T, 0.5, inputs.seed_of("prefill_4096"))
-    _check(orc, n, k, m, tmap, "prefill_4096", bt=bt)
+    _check(orc, n, k, m, tmap, "prefill_4096", block=block)
 
 
 @pytest.mark.parametrize("frac", [0.0, 0.5, 1.0])
-def test_prefill_token_blocks_agree(frac):
-    """128- and 256-token blocks add the same products in the same order:
+def test_prefill_shapes_agree(frac):
+    """Every CTA shape adds the same products in the same order:
     bit-identical Y (the documented contract of the choice)."""
     n, k, m = 384, 1536, 700
     T = (n // 128) * (k // 128)
@@ -72,29 +77,33 @@ def test_prefill_token_blocks_agree(frac):
     W, tmap, X, _ = case(n, k, 128, 128, tmap, batch=m, name="prefill_blocks")
     P = hyb.pack(W.to(dev()), tmap, 128, 128)
     Xd = X.to(dev())
-    Y1 = hyb.spmm_prefill(P, Xd, block_tokens=128)
-    Y2 = hyb.spmm_prefill(P, Xd, block_tokens=256)
-    Y0 = hyb.spmm_prefill(P, Xd)
+    Ys = [hyb.spmm_prefill(P, Xd, block=b) for b in SHAPES] + [hyb.spmm_prefill(P, Xd)]
     torch.cuda.synchronize()
-    assert torch.equal(Y1, Y2)
-    assert torch.equal(Y0, Y1)
+    for Y in Ys[1:]:
+        assert torch.equal(Ys[0], Y)
 
 
 def test_prefill_block_choice():
-    """256 tokens per CTA only when that grid still covers every SM."""
+    """The CTA shape with the fewest modelled bytes per SM: short prompts one
+    band x 128 tokens, long ones two bands x 240 tokens (one wave of 144 CTAs
+    for the 4096-row FFN at 2048 tokens on 148 SMs)."""
     sms = torch.cuda.get_device_properties(dev()).multi_processor_count
-    bands = -(-sms // 8)  # 8 token blocks of 256 give >= sms CTAs
-    assert hyb.prefill_block_tokens(128 * bands, 2048) == 256
-    assert hyb.prefill_block_tokens(4096, 512) == 128   # 32 x 2 CTAs
-    assert hyb.prefill_block_tokens(4096, 2048) == (256 if 32 * 8 >= sms else 128)
-    assert hyb.prefill_block_tokens(0, 16) == 0
+    for n, m in ((128, 16), (4096, 512), (4096, 2048), (14336, 2048), (384, 700)):
+        assert hyb.prefill_block_shape(n, m) in SHAPES
+    assert hyb.prefill_block_shape(128, 4096)[0] == 128  # one band: no two-band CTA
+    if sms == 148:
+        assert hyb.prefill_block_shape(4096, 512) == (128, 128)
+        assert hyb.prefill_block_shape(4096, 2048) == (256, 240)
+        assert hyb.prefill_block_shape(14336, 2048) == (256, 240)
+    with pytest.raises(hyb.HybError):
+        hyb.prefill_block_shape(0, 16)
 
 
 @pytest.mark.parametrize("frac,m", [(0.0, 512), (0.5, 512), (1.0, 512), (0.5, 2048)])
 def test_prefill_ffn_full_size(orc, frac, m):
     """The 4096 x 14336 down projection at 512 tokens (128-token blocks) and
-    2048 tokens (256-token blocks, the bench's prefill case): sampled rows
-    (every token) against the oracle."""
+    2048 tokens (two bands x 240 tokens, the bench's prefill case): sampled
+    rows (every token) against the oracle."""
     n, k = 4096, 14336
     T = (n // 128) * (k // 128)
     tmap = inputs.tile_map_fraction(T, frac, inputs.seed_of("prefill_ffn", frac))
@@ -119,13 +128,14 @@ def test_prefill_matches_the_dense_path(orc):
         assert torch.equal(Y, Y2)
 
 
-def test_prefill_rejects_bad_block():
-    """A token block other than 0, 128 or 256: an argument error."""
+@pytest.mark.parametrize("block", [(128, 64), (256, 256), (256, 0), (0, 128)])
+def test_prefill_rejects_bad_block(block):
+    """A CTA shape the kernel is not built for: an argument error."""
     W = torch.zeros(128, 128, dtype=torch.bfloat16, device=dev())
     P = hyb.pack(W, np.zeros(1, np.uint8), 128, 128)
     X = torch.zeros(4, 128, dtype=torch.bfloat16, device=dev())
     with pytest.raises(hyb.HybError) as e:
-        hyb.spmm_prefill(P, X, block_tokens=64)
+        hyb.spmm_prefill(P, X, block=block)
     assert e.value.status == hyb.HYB_ERR_INVALID_ARG
 
 
