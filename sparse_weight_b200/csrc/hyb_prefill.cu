@@ -237,7 +237,11 @@ __global__ void __launch_bounds__(kPThreads, 1)
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int r0 = blockIdx.x * NB;                  // first tile-row band
-  const int nb = min(NB, p.bands - r0);            // bands present (the last CTA may have one)
+  // A CTA always runs NB bands: past the last band (an odd band count, two
+  // bands per CTA) the second one repeats the last band's loads and products
+  // and stores nothing, so that no loop below tests how many bands there are.
+  const int rlast = p.bands - 1;
+  auto band_of = [&](int b) { return min(r0 + b, rlast); };
   const int64_t m0 = (int64_t)blockIdx.y * PN;     // first token
   const int tpr = p.tpr;
   // ring slots at a 1024-byte boundary (the swizzle pattern repeats every 1024)
@@ -260,8 +264,8 @@ __global__ void __launch_bounds__(kPThreads, 1)
     const int b = i / tpr, j = i - b * tpr;
     uint8_t sp = 0;
     uint32_t mo16 = kNoMeta;
-    if (b < nb) {
-      const int64_t t = (int64_t)(r0 + b) * tpr + j;
+    {
+      const int64_t t = (int64_t)band_of(b) * tpr + j;
       sp = p.map[t];
       const int64_t mo = p.meta_off[t];
       if (mo >= 0 && mo % 16 == 0 && mo + kSMetaBytes <= p.nmb && mo / 16 < (int64_t)kNoMeta)
@@ -290,8 +294,7 @@ __global__ void __launch_bounds__(kPThreads, 1)
     auto load = [&](int w0, int64_t (&vo)[NB]) {
 #pragma unroll
       for (int b = 0; b < NB; ++b)
-        vo[b] = (b < nb && w0 + lane < tpr) ? __ldg(p.val_off + (int64_t)(r0 + b) * tpr + w0 + lane)
-                                            : 0;
+        vo[b] = w0 + lane < tpr ? __ldg(p.val_off + (int64_t)band_of(b) * tpr + w0 + lane) : 0;
     };
     int64_t vo[NB], nvo[NB];
     load(0, vo);
@@ -304,51 +307,75 @@ __global__ void __launch_bounds__(kPThreads, 1)
 #pragma unroll
         for (int b = 0; b < NB; ++b) tvo[b] = __shfl_sync(0xffffffffu, vo[b], l);
         if (lane == 0) {
-          bool sp[NB], fits[NB];
-#pragma unroll
-          for (int b = 0; b < NB; ++b) {
-            sp[b] = b < nb && s_map[b][j] == 1;
-            // a range outside the buffers (a corrupted matrix) is not copied
-            fits[b] = b < nb && (sp[b] ? (tvo[b] >= 0 && 2 * tvo[b] + kSValBytes <= p.nvb &&
-                                          tvo[b] % (kPK / 2) == 0 && s_mo[b][j] != kNoMeta)
-                                       : (tvo[b] >= 0 && 2 * tvo[b] + 2 * kAtomBytes <= p.nvb &&
-                                          tvo[b] % kPK == 0));
-            if (b < nb && !fits[b]) atomicOr(p.status, kStatusBadMap);
-          }
-          for (int h0 = 0; h0 < 2 && ok; h0 += HS) {
-            const int idx = (2 * j + h0) / HS;  // ring position of halves h0 .. h0 + HS - 1
-            const int s = idx % NS;
-            if (!ring_wait(&empty_bar[s], ((uint32_t)(idx / NS) & 1u) ^ 1u)) {
+          if constexpr (HS == 2) {
+            // one band, a whole tile per slot: both halves of A and of X
+            const int s = j % NS;
+            if (!ring_wait(&empty_bar[s], ((uint32_t)(j / NS) & 1u) ^ 1u)) {
               ok = false;
-              break;
+            } else {
+              uint8_t *st = smem + (size_t)s * Sh::kSlotBytes;
+              const bool sp = s_map[0][j] == 1;
+              // a range outside the buffers (a corrupted matrix) is not copied
+              const bool fits = sp ? (tvo[0] >= 0 && 2 * tvo[0] + kSValBytes <= p.nvb &&
+                                      tvo[0] % (kPK / 2) == 0 && s_mo[0][j] != kNoMeta)
+                                   : (tvo[0] >= 0 && 2 * tvo[0] + 2 * kAtomBytes <= p.nvb &&
+                                      tvo[0] % kPK == 0);
+              if (!fits) atomicOr(p.status, kStatusBadMap);
+              const uint32_t abytes = !fits ? 0u : (sp ? (uint32_t)kAtomBytes : 2u * kAtomBytes);
+              mbar_arrive_expect_tx(&full_bar[s], 2u * Sh::kXHalfBytes + abytes);
+              // X: tokens m0 .. m0 + PN - 1 (rows past M read as zeros), tile j's columns
+              tma_load_2d(st + kAtomBytes, &xmap, j * kPK, (int)m0, &full_bar[s]);
+              tma_load_2d(st + Sh::kHalfBytes + kAtomBytes, &xmap, j * kPK + 64, (int)m0,
+                          &full_bar[s]);
+              if (fits && !sp) {  // the tile's first row in the 128-wide view of the values
+                tma_load_2d(st, &wmap, 0, (int)(tvo[0] / kPK), &full_bar[s]);
+                tma_load_2d(st + Sh::kHalfBytes, &wmap, 64, (int)(tvo[0] / kPK), &full_bar[s]);
+              } else if (fits) {  // 64 kept values x 128 rows (128-byte swizzle)
+                tma_load_2d(st, &spmap, 0, (int)(tvo[0] / (kPK / 2)), &full_bar[s]);
+              }
             }
-            uint8_t *st = smem + (size_t)s * Sh::kSlotBytes;
-            // A's bytes in this slot: a dense tile's halves, or a 2:4 tile's
-            // whole compressed operand with its first half
-            uint32_t bytes = (uint32_t)(HS * Sh::kXHalfBytes);
+          } else {
+            // half a tile per slot
+            bool sp[NB], fits[NB];
 #pragma unroll
-            for (int b = 0; b < NB; ++b)
-              if (fits[b])
-                bytes += sp[b] ? (h0 == 0 ? (uint32_t)kAtomBytes : 0u) : (uint32_t)(HS * kAtomBytes);
-            mbar_arrive_expect_tx(&full_bar[s], bytes);
-            for (int hh = 0; hh < HS; ++hh) {
-              const int h = h0 + hh;
-              uint8_t *hb = st + (size_t)hh * Sh::kHalfBytes;
-              // X: tokens m0 .. m0 + PN - 1 (rows past M read as zeros),
-              // columns 64 h .. 64 h + 63 of tile j
-              tma_load_2d(hb + NB * kAtomBytes, &xmap, j * kPK + 64 * h, (int)m0, &full_bar[s]);
+            for (int b = 0; b < NB; ++b) {
+              sp[b] = s_map[b][j] == 1;
+              // a range outside the buffers (a corrupted matrix) is not copied
+              fits[b] = sp[b] ? (tvo[b] >= 0 && 2 * tvo[b] + kSValBytes <= p.nvb &&
+                                 tvo[b] % (kPK / 2) == 0 && s_mo[b][j] != kNoMeta)
+                              : (tvo[b] >= 0 && 2 * tvo[b] + 2 * kAtomBytes <= p.nvb &&
+                                 tvo[b] % kPK == 0);
+              if (!fits[b]) atomicOr(p.status, kStatusBadMap);
+            }
+            for (int h0 = 0; h0 < 2 && ok; ++h0) {
+              const int idx = 2 * j + h0;  // ring position of half h0
+              const int s = idx % NS;
+              if (!ring_wait(&empty_bar[s], ((uint32_t)(idx / NS) & 1u) ^ 1u)) {
+                ok = false;
+                break;
+              }
+              uint8_t *st = smem + (size_t)s * Sh::kSlotBytes;
+              // A's bytes in this slot: a dense tile's half, or a 2:4 tile's
+              // whole compressed operand with its first half
+              uint32_t bytes = (uint32_t)Sh::kXHalfBytes;
+#pragma unroll
+              for (int b = 0; b < NB; ++b)
+                if (fits[b]) bytes += sp[b] ? (h0 == 0 ? (uint32_t)kAtomBytes : 0u) : (uint32_t)kAtomBytes;
+              mbar_arrive_expect_tx(&full_bar[s], bytes);
+              // X: tokens m0 .. m0 + PN - 1 (rows past M read as zeros), columns
+              // 64 h0 .. 64 h0 + 63 of tile j
+              tma_load_2d(st + NB * kAtomBytes, &xmap, j * kPK + 64 * h0, (int)m0, &full_bar[s]);
 #pragma unroll
               for (int b = 0; b < NB; ++b)
                 if (fits[b] && !sp[b])  // the tile's first row in the 128-wide view of the values
-                  tma_load_2d(hb + b * kAtomBytes, &wmap, 64 * h, (int)(tvo[b] / kPK),
-                              &full_bar[s]);
-            }
-            if (h0 == 0) {
+                  tma_load_2d(st + b * kAtomBytes, &wmap, 64 * h0, (int)(tvo[b] / kPK), &full_bar[s]);
+              if (h0 == 0) {
 #pragma unroll
-              for (int b = 0; b < NB; ++b)
-                if (fits[b] && sp[b])  // 64 kept values x 128 rows (128-byte swizzle)
-                  tma_load_2d(st + b * kAtomBytes, &spmap, 0, (int)(tvo[b] / (kPK / 2)),
-                              &full_bar[s]);
+                for (int b = 0; b < NB; ++b)
+                  if (fits[b] && sp[b])  // 64 kept values x 128 rows (128-byte swizzle)
+                    tma_load_2d(st + b * kAtomBytes, &spmap, 0, (int)(tvo[b] / (kPK / 2)),
+                                &full_bar[s]);
+              }
             }
           }
         }
@@ -364,33 +391,76 @@ __global__ void __launch_bounds__(kPThreads, 1)
     uint32_t nsp = 0;  // 2:4 tiles multiplied so far
     const uint32_t eb0 = smem_u32(smem + (size_t)kRingBytes);  // metadata ring
     for (int j = 0; j < tpr && ok; ++j) {
-      if (lane == 0) {
+      if constexpr (HS == 2) {
+        // one band, a whole tile per slot: 8 dense products, or the metadata
+        // copy and 4 sparse ones
+        if (lane == 0) {
+          const int s = j % NS;
+          const bool sp = s_map[0][j] == 1;
+          const uint32_t q = nsp % Sh::kEsl;
+          ok = ring_wait(&full_bar[s], (uint32_t)(j / NS) & 1u);
+          if (ok && sp) ok = ring_wait(&efull_bar[q], (nsp / Sh::kEsl) & 1u);
+          if (ok) {
+            tc_fence_after();
+            const uint32_t st = smem_u32(smem + (size_t)s * Sh::kSlotBytes);
+            if (sp) {
+              // A advancing 16 stored values (32 B) per K = 32 product, B 32
+              // columns (64 B) of the product's half
+              const uint32_t te = tmem + Sh::kTmemE + 4 * q;
+              tmem_cp_128x128b(te, e_desc(eb0 + q * kEBytes));
+#pragma unroll
+              for (int kb = 0; kb < 4; ++kb) {
+                const uint32_t ecol = te + kb;
+                umma_sp_bf16(tmem, sw128_desc(st + kb * 32),
+                             sw128_desc(st + (kb >> 1) * Sh::kHalfBytes + kAtomBytes + (kb & 1) * 64),
+                             ecol & ~1u, ecol & 1u, (j | kb) != 0 ? 1u : 0u, kIdesc);
+              }
+            } else {
+#pragma unroll
+              for (int h = 0; h < 2; ++h)
+#pragma unroll
+                for (int kk = 0; kk < 4; ++kk) {
+                  // K = 16 columns (32 bytes) at a time inside the 128-byte row
+                  const uint32_t hb = st + h * Sh::kHalfBytes;
+                  umma_bf16(tmem, sw128_desc(hb + kk * 32), sw128_desc(hb + kAtomBytes + kk * 32),
+                            (j | h | kk) != 0 ? 1u : 0u, kIdesc);
+                }
+            }
+            umma_commit(&empty_bar[s]);
+            if (sp) {
+              umma_commit(&eempty_bar[q]);  // the metadata slot is free once these completed
+              ++nsp;
+            }
+          }
+        }
+      } else if (lane == 0) {
+        // half a tile per slot, every band's products for that half
         bool sp[NB];
         uint32_t qn[NB];  // metadata ring positions of the 2:4 bands
         uint32_t c = nsp;
         bool any_sp = false;
 #pragma unroll
         for (int b = 0; b < NB; ++b) {
-          sp[b] = b < nb && s_map[b][j] == 1;
+          sp[b] = s_map[b][j] == 1;
           qn[b] = sp[b] ? c++ : 0u;
           any_sp = any_sp || sp[b];
         }
         uint32_t a_sp = 0;  // the 2:4 bands' compressed A (in the first half's slot)
         int s_first = 0;
-        for (int h0 = 0; h0 < 2 && ok; h0 += HS) {
-          const int idx = (2 * j + h0) / HS;
+        for (int h = 0; h < 2 && ok; ++h) {
+          const int idx = 2 * j + h;
           const int s = idx % NS;
           ok = ring_wait(&full_bar[s], (uint32_t)(idx / NS) & 1u);
-          if (h0 == 0) {
+          if (h == 0) {
 #pragma unroll
             for (int b = 0; b < NB; ++b)
-              if (ok && sp[b])
-                ok = ring_wait(&efull_bar[qn[b] % Sh::kEsl], (qn[b] / Sh::kEsl) & 1u);
+              if (ok && sp[b]) ok = ring_wait(&efull_bar[qn[b] % Sh::kEsl], (qn[b] / Sh::kEsl) & 1u);
           }
           if (!ok) break;
           tc_fence_after();
           const uint32_t st = smem_u32(smem + (size_t)s * Sh::kSlotBytes);
-          if (h0 == 0) {
+          const uint32_t b0 = st + NB * kAtomBytes;  // X of this half
+          if (h == 0) {
             // metadata to tensor memory (4 columns: one per K = 32 product)
 #pragma unroll
             for (int b = 0; b < NB; ++b)
@@ -401,44 +471,36 @@ __global__ void __launch_bounds__(kPThreads, 1)
             s_first = s;
           }
 #pragma unroll
-          for (int hh = 0; hh < HS; ++hh) {
-            const int h = h0 + hh;
-            const uint32_t hb = st + hh * Sh::kHalfBytes;
-            const uint32_t b0 = hb + NB * kAtomBytes;  // X of this half
+          for (int b = 0; b < NB; ++b) {
+            const uint32_t d = tmem + b * Sh::kAccStride;  // band b's accumulator
+            if (sp[b]) {
+              // products 2h, 2h + 1: A advancing 16 stored values (32 B), B 32
+              // columns (64 B) of this half each
+              const uint32_t te = tmem + Sh::kTmemE + 4 * (qn[b] % Sh::kEsl);
 #pragma unroll
-            for (int b = 0; b < NB; ++b) {
-              if (b >= nb) continue;
-              const uint32_t d = tmem + b * Sh::kAccStride;  // band b's accumulator
-              if (sp[b]) {
-                // products 2h, 2h + 1: A advancing 16 stored values (32 B), B
-                // 32 columns (64 B) of this half each
-                const uint32_t te = tmem + Sh::kTmemE + 4 * (qn[b] % Sh::kEsl);
-#pragma unroll
-                for (int kk = 0; kk < 2; ++kk) {
-                  const int kb = 2 * h + kk;
-                  const uint32_t ecol = te + kb;
-                  umma_sp_bf16(d, sw128_desc(a_sp + b * kAtomBytes + kb * 32),
-                               sw128_desc(b0 + kk * 64), ecol & ~1u, ecol & 1u,
-                               (j | kb) != 0 ? 1u : 0u, kIdesc);
-                }
-              } else {
-#pragma unroll
-                for (int kk = 0; kk < 4; ++kk)
-                  // K = 16 columns (32 bytes) at a time inside the 128-byte row
-                  umma_bf16(d, sw128_desc(hb + b * kAtomBytes + kk * 32), sw128_desc(b0 + kk * 32),
-                            (j | h | kk) != 0 ? 1u : 0u, kIdesc);
+              for (int kk = 0; kk < 2; ++kk) {
+                const int kb = 2 * h + kk;
+                const uint32_t ecol = te + kb;
+                umma_sp_bf16(d, sw128_desc(a_sp + b * kAtomBytes + kb * 32), sw128_desc(b0 + kk * 64),
+                             ecol & ~1u, ecol & 1u, (j | kb) != 0 ? 1u : 0u, kIdesc);
               }
+            } else {
+#pragma unroll
+              for (int kk = 0; kk < 4; ++kk)
+                // K = 16 columns (32 bytes) at a time inside the 128-byte row
+                umma_bf16(d, sw128_desc(st + b * kAtomBytes + kk * 32), sw128_desc(b0 + kk * 32),
+                          (j | h | kk) != 0 ? 1u : 0u, kIdesc);
             }
           }
           // a slot is free once its products completed; with a 2:4 band, the
           // first half's slot holds that band's A for the second half too
-          if (!any_sp || HS == 2) {
+          if (!any_sp) {
             umma_commit(&empty_bar[s]);
-          } else if (h0 == 1) {
+          } else if (h == 1) {
             umma_commit(&empty_bar[s_first]);
             umma_commit(&empty_bar[s]);
           }
-          if (h0 + HS == 2) {
+          if (h == 1) {
 #pragma unroll
             for (int b = 0; b < NB; ++b)
               if (sp[b]) umma_commit(&eempty_bar[qn[b] % Sh::kEsl]);  // metadata slot free
@@ -487,7 +549,7 @@ __global__ void __launch_bounds__(kPThreads, 1)
     const int npos = NB * tpr;
     auto next_sparse = [&](int pos) {
       int q = pos + 1;
-      while (q < npos && !(q % NB < nb && s_map[q % NB][q / NB] == 1)) ++q;
+      while (q < npos && s_map[q % NB][q / NB] != 1) ++q;
       return q;
     };
     int pos = next_sparse(-1);
@@ -533,7 +595,7 @@ __global__ void __launch_bounds__(kPThreads, 1)
       const int b = NB == 2 && warp >= 8 ? 1 : 0;
       const int cb = NB == 1 && warp >= 8 ? PN / 2 : 0;
       const int ce = NB == 1 ? cb + PN / 2 : PN;
-      if (b < nb) {
+      if (r0 + b < p.bands) {
         const int64_t yrow = (int64_t)(r0 + b) * kPM + 32 * qw + lane;
 #pragma unroll 1
         for (int c0 = cb; c0 < ce; c0 += 16) {
