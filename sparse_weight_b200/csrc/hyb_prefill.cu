@@ -121,6 +121,17 @@ __device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr) {
   return d;
 }
 
+// The same for the 64-byte swizzle layout: rows 64 bytes apart, 8-row groups
+// 512 bytes apart, layout type 4 (a 2:4 tile's half: 32 kept values per row).
+__device__ __forceinline__ uint64_t sw64_desc(uint32_t saddr) {
+  uint64_t d = (uint64_t)((saddr >> 4) & 0x3FFFu);
+  d |= (uint64_t)1 << 16;             // leading byte offset (unused by swizzled K-major)
+  d |= (uint64_t)(512 >> 4) << 32;    // stride byte offset
+  d |= (uint64_t)1 << 46;             // version
+  d |= (uint64_t)4 << 61;             // 64-byte swizzle
+  return d;
+}
+
 __device__ __forceinline__ void umma_bf16(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc,
                                           uint32_t accumulate, uint32_t idesc) {
   asm volatile(
@@ -355,26 +366,24 @@ __global__ void __launch_bounds__(kPThreads, 1)
                 break;
               }
               uint8_t *st = smem + (size_t)s * Sh::kSlotBytes;
-              // A's bytes in this slot: a dense tile's half, or a 2:4 tile's
-              // whole compressed operand with its first half
+              // A's bytes in this slot: each band's half tile, 16 KB dense or
+              // 8 KB of kept values
               uint32_t bytes = (uint32_t)Sh::kXHalfBytes;
 #pragma unroll
               for (int b = 0; b < NB; ++b)
-                if (fits[b]) bytes += sp[b] ? (h0 == 0 ? (uint32_t)kAtomBytes : 0u) : (uint32_t)kAtomBytes;
+                if (fits[b]) bytes += sp[b] ? (uint32_t)(kAtomBytes / 2) : (uint32_t)kAtomBytes;
               mbar_arrive_expect_tx(&full_bar[s], bytes);
               // X: tokens m0 .. m0 + PN - 1 (rows past M read as zeros), columns
               // 64 h0 .. 64 h0 + 63 of tile j
               tma_load_2d(st + NB * kAtomBytes, &xmap, j * kPK + 64 * h0, (int)m0, &full_bar[s]);
 #pragma unroll
-              for (int b = 0; b < NB; ++b)
-                if (fits[b] && !sp[b])  // the tile's first row in the 128-wide view of the values
+              for (int b = 0; b < NB; ++b) {
+                if (!fits[b]) continue;
+                if (sp[b])  // kept values 32 h0 .. 32 h0 + 31 of 128 rows (64-byte swizzle)
+                  tma_load_2d(st + b * kAtomBytes, &spmap, 32 * h0, (int)(tvo[b] / (kPK / 2)),
+                              &full_bar[s]);
+                else        // the tile's first row in the 128-wide view of the values
                   tma_load_2d(st + b * kAtomBytes, &wmap, 64 * h0, (int)(tvo[b] / kPK), &full_bar[s]);
-              if (h0 == 0) {
-#pragma unroll
-                for (int b = 0; b < NB; ++b)
-                  if (fits[b] && sp[b])  // 64 kept values x 128 rows (128-byte swizzle)
-                    tma_load_2d(st + b * kAtomBytes, &spmap, 0, (int)(tvo[b] / (kPK / 2)),
-                                &full_bar[s]);
               }
             }
           }
@@ -438,15 +447,11 @@ __global__ void __launch_bounds__(kPThreads, 1)
         bool sp[NB];
         uint32_t qn[NB];  // metadata ring positions of the 2:4 bands
         uint32_t c = nsp;
-        bool any_sp = false;
 #pragma unroll
         for (int b = 0; b < NB; ++b) {
           sp[b] = s_map[b][j] == 1;
           qn[b] = sp[b] ? c++ : 0u;
-          any_sp = any_sp || sp[b];
         }
-        uint32_t a_sp = 0;  // the 2:4 bands' compressed A (in the first half's slot)
-        int s_first = 0;
         for (int h = 0; h < 2 && ok; ++h) {
           const int idx = 2 * j + h;
           const int s = idx % NS;
@@ -467,21 +472,19 @@ __global__ void __launch_bounds__(kPThreads, 1)
               if (sp[b])
                 tmem_cp_128x128b(tmem + Sh::kTmemE + 4 * (qn[b] % Sh::kEsl),
                                  e_desc(eb0 + (qn[b] % Sh::kEsl) * kEBytes));
-            a_sp = st;
-            s_first = s;
           }
 #pragma unroll
           for (int b = 0; b < NB; ++b) {
             const uint32_t d = tmem + b * Sh::kAccStride;  // band b's accumulator
             if (sp[b]) {
-              // products 2h, 2h + 1: A advancing 16 stored values (32 B), B 32
-              // columns (64 B) of this half each
+              // products 2h, 2h + 1: A (this half's 32 kept values per row)
+              // advancing 16 stored values (32 B), B 32 columns (64 B) each
               const uint32_t te = tmem + Sh::kTmemE + 4 * (qn[b] % Sh::kEsl);
 #pragma unroll
               for (int kk = 0; kk < 2; ++kk) {
                 const int kb = 2 * h + kk;
                 const uint32_t ecol = te + kb;
-                umma_sp_bf16(d, sw128_desc(a_sp + b * kAtomBytes + kb * 32), sw128_desc(b0 + kk * 64),
+                umma_sp_bf16(d, sw64_desc(st + b * kAtomBytes + kk * 32), sw128_desc(b0 + kk * 64),
                              ecol & ~1u, ecol & 1u, (j | kb) != 0 ? 1u : 0u, kIdesc);
               }
             } else {
@@ -492,14 +495,7 @@ __global__ void __launch_bounds__(kPThreads, 1)
                           (j | h | kk) != 0 ? 1u : 0u, kIdesc);
             }
           }
-          // a slot is free once its products completed; with a 2:4 band, the
-          // first half's slot holds that band's A for the second half too
-          if (!any_sp) {
-            umma_commit(&empty_bar[s]);
-          } else if (h == 1) {
-            umma_commit(&empty_bar[s_first]);
-            umma_commit(&empty_bar[s]);
-          }
+          umma_commit(&empty_bar[s]);  // the slot is free once its products completed
           if (h == 1) {
 #pragma unroll
             for (int b = 0; b < NB; ++b)
@@ -548,15 +544,19 @@ __global__ void __launch_bounds__(kPThreads, 1)
                               (0xDull << 40) | (0xEull << 48);
     const int npos = NB * tpr;
     auto next_sparse = [&](int pos) {
-      int q = pos + 1;
+      int q = pos < npos ? pos + 1 : npos;
       while (q < npos && s_map[q % NB][q / NB] != 1) ++q;
       return q;
     };
+    auto masks_at = [&](int pos) { return pos < npos ? load_masks(pos) : make_uint2(0, 0); };
+    // the masks of the next four 2:4 tiles are in flight (a load from global
+    // memory takes about as long as a tile's products)
     int pos = next_sparse(-1);
-    uint2 cur = pos < npos ? load_masks(pos) : make_uint2(0, 0);
+    int pos1 = next_sparse(pos), pos2 = next_sparse(pos1), pos3 = next_sparse(pos2);
+    uint2 cur = masks_at(pos), m1 = masks_at(pos1), m2 = masks_at(pos2), m3 = masks_at(pos3);
     while (pos < npos) {
-      const int pn = next_sparse(pos);
-      const uint2 nxt = pn < npos ? load_masks(pn) : make_uint2(0, 0);
+      const int pn = next_sparse(pos3);
+      const uint2 mn = masks_at(pn);
       const int q = (int)(nsp % Sh::kEsl);
       // the slot's previous tile has been multiplied
       if (!ring_wait(&eempty_bar[q], ((nsp / Sh::kEsl) & 1u) ^ 1u)) {
@@ -582,8 +582,14 @@ __global__ void __launch_bounds__(kPThreads, 1)
       // generic-proxy writes, read next by tcgen05.cp (async proxy)
       asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
       mbar_arrive(&efull_bar[q]);
-      cur = nxt;
-      pos = pn;
+      cur = m1;
+      m1 = m2;
+      m2 = m3;
+      m3 = mn;
+      pos = pos1;
+      pos1 = pos2;
+      pos2 = pos3;
+      pos3 = pn;
     }
     if (!ok && lane == 0) atomicOr(p.status, kStatusTimeout);
     // epilogue: TMEM lanes 32 (warp % 4) .. + 31 are this warp's weight rows;
@@ -622,19 +628,21 @@ __global__ void __launch_bounds__(kPThreads, 1)
   }
 }
 
-// 2-D tensor map, bf16, 128-byte swizzle, box 64 columns x box_rows rows.
-int encode_sw128(const void *base, uint64_t cols, uint64_t rows, uint64_t row_bytes,
-                 uint32_t box_rows, CUtensorMap *map) {
+// 2-D tensor map, bf16, box box_cols x box_rows, 128- or 64-byte swizzle
+// (box_cols 64 or 32).
+int encode_swz(const void *base, uint64_t cols, uint64_t rows, uint64_t row_bytes,
+               uint32_t box_cols, uint32_t box_rows, CUtensorMap *map) {
   PFN_cuTensorMapEncodeTiled_v12000 encode = tensor_map_encoder();
   if (!encode) return HYB_ERR_CUDA;
   const cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
   const cuuint64_t strides[1] = {(cuuint64_t)row_bytes};
-  const cuuint32_t box[2] = {64, box_rows};
+  const cuuint32_t box[2] = {box_cols, box_rows};
   const cuuint32_t estr[2] = {1, 1};
-  const CUresult res =
-      encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides,
-             box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  const CUresult res = encode(
+      map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides, box, estr,
+      CU_TENSOR_MAP_INTERLEAVE_NONE,
+      box_cols == 64 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B,
+      CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return res == CUDA_SUCCESS ? HYB_OK : HYB_ERR_CUDA;
 }
 
@@ -724,18 +732,21 @@ int hyb_spmm_prefill_blocked(const hyb_matrix *A, int64_t m, const uint16_t *X, 
   alignas(64) CUtensorMap xmap{};
   alignas(64) CUtensorMap wmap{};
   // X: a box of 64 columns x one token block
-  int rc = encode_sw128(X, (uint64_t)A->k, (uint64_t)m, (uint64_t)ldx * 2, (uint32_t)pn, &xmap);
+  int rc = encode_swz(X, (uint64_t)A->k, (uint64_t)m, (uint64_t)ldx * 2, 64, (uint32_t)pn, &xmap);
   if (rc != HYB_OK) return rc;
   // the value buffer seen as rows of 128 bf16: a dense tile at element offset
   // vo is rows vo / 128 .. + 127
-  rc = encode_sw128(A->vals, (uint64_t)kPK, (uint64_t)(A->n_vals / kPK), (uint64_t)kPK * 2,
-                    (uint32_t)kPM, &wmap);
+  rc = encode_swz(A->vals, (uint64_t)kPK, (uint64_t)(A->n_vals / kPK), (uint64_t)kPK * 2, 64,
+                  (uint32_t)kPM, &wmap);
   if (rc != HYB_OK) return rc;
   // and as rows of 64 bf16: a 2:4 tile's 128 rows of kept values at element
-  // offset vo are rows vo / 64 .. + 127
+  // offset vo are rows vo / 64 .. + 127, loaded whole (a box of 64 values,
+  // 128-byte swizzle) where a ring slot holds a whole tile, else by halves (a
+  // box of 32 values, 64-byte swizzle)
   alignas(64) CUtensorMap spmap{};
-  rc = encode_sw128(A->vals, (uint64_t)(kPK / 2), (uint64_t)(A->n_vals / (kPK / 2)),
-                    (uint64_t)kPK, (uint32_t)kPM, &spmap);
+  const bool whole_tiles = rows == 128 && pn == 128;
+  rc = encode_swz(A->vals, (uint64_t)(kPK / 2), (uint64_t)(A->n_vals / (kPK / 2)), (uint64_t)kPK,
+                  whole_tiles ? 64u : 32u, (uint32_t)kPM, &spmap);
   if (rc != HYB_OK) return rc;
 
   PrefillParams prm{};
