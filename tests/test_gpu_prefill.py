@@ -128,6 +128,35 @@ def test_prefill_matches_the_dense_path(orc):
         assert torch.equal(Y, Y2)
 
 
+@pytest.mark.parametrize("block", SHAPES)
+@pytest.mark.parametrize("field", ["val_off", "meta_off"])
+def test_prefill_bad_offsets_are_flagged(block, field):
+    """Corrupted offsets (past the value or mask buffer) of a dense and a 2:4
+    tile are not copied and are reported through the status word; the launch
+    completes and nothing is read out of bounds."""
+    n, k, m = 384, 1024, 200
+    T = (n // 128) * (k // 128)
+    tmap = inputs.tile_map_fraction(T, 0.5, inputs.seed_of("prefill_bad"))
+    W = inputs.weight(n, k, 0.02, inputs.seed_of("prefill_bad", "W")).to(dev())
+    P = hyb.pack(W, tmap, 128, 128)
+    t_dense = int(np.flatnonzero(tmap == 0)[0])
+    t_sparse = int(np.flatnonzero(tmap == 1)[-1])
+    if field == "val_off":
+        P.val_off[t_dense] = P.n_vals + 128 * 128
+        P.val_off[t_sparse] = P.n_vals + 64 * 128
+    else:  # only a 2:4 tile reads masks
+        P.meta_off[t_sparse] = P.n_meta + 4096
+    ws = hyb.new_workspace(hyb.lib().hyb_prefill_workspace_bytes(), dev())
+    X = torch.ones(m, k, dtype=torch.bfloat16, device=dev())
+    hyb.spmm_prefill(P, X, ws=ws, block=block)
+    with pytest.raises(hyb.HybError) as e:
+        hyb.check_status(ws)
+    assert e.value.status == hyb.HYB_ERR_DEVICE_CHECK
+    assert e.value.flags & hyb.STATUS_BAD_MAP
+    assert not e.value.flags & hyb.STATUS_TIMEOUT
+    hyb.check_status(ws)  # cleared
+
+
 @pytest.mark.parametrize("block", [(128, 64), (256, 256), (256, 0), (0, 128)])
 def test_prefill_rejects_bad_block(block):
     """A CTA shape the kernel is not built for: an argument error."""
