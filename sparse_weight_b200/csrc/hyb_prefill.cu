@@ -245,6 +245,7 @@ __global__ void __launch_bounds__(kPThreads, 1)
   __shared__ uint32_t s_tmem;
   __shared__ uint8_t s_map[NB][kMaxBandTiles];
   __shared__ uint32_t s_mo[NB][kMaxBandTiles];  // the bands' mask offsets / 16, or kNoMeta
+  __shared__ int64_t s_vo[NB][32];               // the producer's window of value offsets
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int r0 = blockIdx.x * NB;                  // first tile-row band
@@ -299,25 +300,30 @@ __global__ void __launch_bounds__(kPThreads, 1)
 
   if (warp == 0) {
     // ------------------------------ producer ------------------------------
-    // lane l holds the value offsets of tile w0 + l of each band (a window of
-    // 32, the next window loaded while this one is issued)
+    // Windows of 32 tiles: lane l loads the value offsets of tile w0 + l of
+    // each band (the next window's loads stay in flight while this one is
+    // issued) and leaves them in shared memory, where lane 0 alone takes them
+    // tile by tile (the warp meets once per window, not once per tile).
     bool ok = true;
     auto load = [&](int w0, int64_t (&vo)[NB]) {
 #pragma unroll
       for (int b = 0; b < NB; ++b)
         vo[b] = w0 + lane < tpr ? __ldg(p.val_off + (int64_t)band_of(b) * tpr + w0 + lane) : 0;
     };
-    int64_t vo[NB], nvo[NB];
-    load(0, vo);
+    int64_t nvo[NB];
+    load(0, nvo);
     for (int w0 = 0; w0 < tpr && ok; w0 += 32) {
+#pragma unroll
+      for (int b = 0; b < NB; ++b) s_vo[b][lane] = nvo[b];
+      __syncwarp();
       load(w0 + 32, nvo);
       const int nw = min(32, tpr - w0);
-      for (int l = 0; l < nw && ok; ++l) {
+      for (int l = 0; l < nw && ok && lane == 0; ++l) {
         const int j = w0 + l;
         int64_t tvo[NB];
 #pragma unroll
-        for (int b = 0; b < NB; ++b) tvo[b] = __shfl_sync(0xffffffffu, vo[b], l);
-        if (lane == 0) {
+        for (int b = 0; b < NB; ++b) tvo[b] = s_vo[b][l];
+        {
           if constexpr (HS == 2) {
             // one band, a whole tile per slot: both halves of A and of X
             const int s = j % NS;
@@ -392,10 +398,9 @@ __global__ void __launch_bounds__(kPThreads, 1)
             }
           }
         }
-        ok = __shfl_sync(0xffffffffu, ok, 0);
       }
-#pragma unroll
-      for (int b = 0; b < NB; ++b) vo[b] = nvo[b];
+      ok = __shfl_sync(0xffffffffu, ok, 0);
+      __syncwarp();  // lane 0 is done with this window's offsets
     }
     if (!ok && lane == 0) atomicOr(p.status, kStatusTimeout);
   } else if (warp == 1) {
@@ -403,7 +408,9 @@ __global__ void __launch_bounds__(kPThreads, 1)
     bool ok = true;
     uint32_t nsp = 0;  // 2:4 tiles multiplied so far
     const uint32_t eb0 = smem_u32(smem + (size_t)kRingBytes);  // metadata ring
-    for (int j = 0; j < tpr && ok; ++j) {
+    // lane 0 alone walks the tiles (the other lanes wait at the end: no warp
+    // convergence per tile, measured faster)
+    for (int j = 0; j < tpr && ok && lane == 0; ++j) {
       if constexpr (HS == 2) {
         // one band, a whole tile per slot: 8 dense products, or the metadata
         // copy and 4 sparse ones
@@ -510,7 +517,6 @@ __global__ void __launch_bounds__(kPThreads, 1)
           }
         }
       }
-      ok = __shfl_sync(0xffffffffu, ok, 0);
     }
     if (lane == 0) {
       if (!ok) atomicOr(p.status, kStatusTimeout);
