@@ -714,8 +714,9 @@ def sweep(device, steps=200, warmup=10):
 
 
 def _sweep_prefill(device, emit, steps=20, warmup=3):
-    """Prefill on the tensor cores (hyb_spmm_prefill): the FFN shapes at 512
-    and 2048 tokens and three 2:4-tile fractions, against torch.matmul (cuBLAS
+    """Prefill on the tensor cores (hyb_spmm_prefill): the FFN shapes at 512,
+    1024, 2048 and 4096 tokens, every CTA shape and three 2:4-tile fractions,
+    against torch.matmul (cuBLAS
     bf16, the dense weight) on the same inputs.  Tokens x weight bytes exceed
     L2, so back-to-back calls are timed (CUDA events, mean of `steps`)."""
     try:
@@ -726,7 +727,7 @@ def _sweep_prefill(device, emit, steps=20, warmup=3):
     for n, k in ((4096, 14336), (14336, 4096)):
         W = inputs.weight(n, k, 0.02, inputs.seed_of("prefill_sweep", n, k)).to(device)
         T = (n // 128) * (k // 128)
-        for m in (512, 2048):
+        for m in (512, 1024, 2048, 4096):
             X = inputs.activations(m, k, inputs.seed_of("prefill_sweep", "X", m, k)).to(device)
             Y = torch.empty(m, n, dtype=torch.float32, device=device)
             stream = torch.cuda.current_stream(device)
