@@ -129,6 +129,25 @@ def test_prefill_matches_the_dense_path(orc):
 
 
 @pytest.mark.parametrize("block", SHAPES)
+def test_prefill_strided_x_and_y(orc, block):
+    """X and Y as views with row strides above k and n (ldx, ldy): the same
+    values as contiguous buffers, and Y's padding columns untouched."""
+    n, k, m = 384, 768, 300
+    T = (n // 128) * (k // 128)
+    tmap = inputs.tile_map_fraction(T, 0.5, inputs.seed_of("prefill_strided"))
+    W, tmap, X, _ = case(n, k, 128, 128, tmap, batch=m, name="prefill_strided")
+    P = hyb.pack(W.to(dev()), tmap, 128, 128)
+    Xbig = torch.zeros(m, k + 64, dtype=torch.bfloat16, device=dev())
+    Xbig[:, :k] = X.to(dev())
+    Ybig = torch.full((m, n + 32), -7.0, dtype=torch.float32, device=dev())
+    hyb.spmm_prefill(P, Xbig[:, :k], Y=Ybig[:, :n], block=block)
+    Y0 = hyb.spmm_prefill(P, X.to(dev()), block=block)
+    torch.cuda.synchronize()
+    assert torch.equal(Ybig[:, :n], Y0)
+    assert bool((Ybig[:, n:] == -7.0).all())
+
+
+@pytest.mark.parametrize("block", SHAPES)
 @pytest.mark.parametrize("field", ["val_off", "meta_off"])
 def test_prefill_bad_offsets_are_flagged(block, field):
     """Corrupted offsets (past the value or mask buffer) of a dense and a 2:4
