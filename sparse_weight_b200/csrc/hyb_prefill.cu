@@ -9,37 +9,41 @@
 // both kinds of tile feed one tcgen05 pipeline, dense tiles through
 // tcgen05.mma and 2:4 tiles through tcgen05.mma.sp:
 //
-//   * CTA (band r, token block mb) owns Y[PN mb .. +PN][128 r .. +128]: a
-//     128 x PN fp32 accumulator in tensor memory (TMEM), M = 128 weight rows,
-//     N = PN tokens (128 or 256), K looped over the band's tiles (128 columns
-//     each), every tile in two halves of 64 columns.
-//   * warp 0 (one lane) moves the operands with TMA into a ring of 192 KB
-//     (3 slots of a whole tile at N = 128, 4 slots of a half-tile at N =
-//     256): a dense tile's half as a 2-D box of 64 columns x 128 rows with
-//     128-byte swizzle (the K-major layout tcgen05.mma reads), a 2:4 tile's
-//     kept values with its first half as one box of 64 values x 128 rows
-//     (already the sparse MMA's compressed A operand: 2 kept values per group
-//     of 4, ascending), X as a box of 64 columns x PN tokens per half.
+//   * A CTA owns NB 128-row bands (1 or 2) and PN tokens (128 or 256 for one
+//     band, 240 for two): one 128 x PN fp32 accumulator per band in tensor
+//     memory (TMEM, band b from column 256 b), M = 128 weight rows per MMA,
+//     N = PN tokens, K looped over the bands' tiles (128 columns each, in two
+//     halves of 64).  hyb_prefill_block_shape picks the shape per call.
+//   * warp 0 moves the operands with TMA into a ring of 192 KB: 3 slots of a
+//     whole tile (one band, 128 tokens), else slots of a half-tile (4 x 48 KB
+//     for one band and 256 tokens, 3 x 62 KB for two bands): a dense tile's
+//     half as a 2-D box of 64 columns x 128 rows with the 128-byte swizzle
+//     (the K-major layout tcgen05.mma reads), a 2:4 tile's kept values (already
+//     the sparse MMA's compressed A operand: 2 kept values per group of 4,
+//     ascending) as a box of 64 values x 128 rows, or of 32 values x 128 rows
+//     in the 64-byte swizzle per half in the half-tile rings, X as a box of 64
+//     columns x PN tokens per half.  Its lanes load a window of 32 tiles'
+//     value offsets into shared memory; lane 0 alone walks the tiles.
 //   * warps 4-11 turn each 2:4 tile's masks into the sparse MMA's metadata
 //     (the two kept positions of a group as a nibble, laid out by tensor-
 //     memory lane and column), fence it for the async proxy and signal the
 //     MMA warp.
-//   * warp 1 owns the TMEM allocation; one lane issues per half-tile 4
-//     tcgen05.mma (dense: kind::f16, bf16 x bf16 -> fp32, K = 16 each) or, for
-//     a 2:4 tile, a tcgen05.cp of the metadata and 2 tcgen05.mma.sp (K = 32
-//     each) per half, and frees each ring slot with tcgen05.commit (a 2:4
-//     tile's first half-tile slot only after its second half's products: it
-//     holds A).
-//   * warps 4-11 then read the accumulator with tcgen05.ld (warp w: TMEM lanes
-//     32 (w % 4) .., half of the token columns each) and store Y (a warp
-//     writes 32 consecutive rows of one token: 128 contiguous bytes).
+//   * warp 1 owns the TMEM allocation; its lane 0 issues per band and half-tile
+//     4 tcgen05.mma (dense: kind::f16, bf16 x bf16 -> fp32, K = 16 each) or,
+//     for a 2:4 tile, a tcgen05.cp of the metadata and 2 tcgen05.mma.sp (K =
+//     32 each) per half, and frees each ring slot with tcgen05.commit.
+//   * warps 4-11 then read the accumulators with tcgen05.ld (warp w: TMEM
+//     lanes 32 (w % 4) .., half of the token columns of one band, or every
+//     column of band w / 8 - 1) and store Y (a warp writes 32 consecutive
+//     rows of one token: 128 contiguous bytes).
 //
-// Every half-tile moves 16 KB of A and PN x 128 bytes of X into shared
-// memory for PN x 128 x 64 multiply-adds, so N = 256 halves the operand bytes
-// per product of N = 128; it is taken when the grid still fills the SMs.
-// A 2:4 tile moves the hybrid format's bytes and costs half a dense tile's
-// tensor work.  Every wait is bounded; one that runs out sets kStatusTimeout
-// in the status word and the CTA leaves its pipeline.
+// A CTA's operand bytes per tile are its bands' A (16 KB per band and half)
+// and PN x 256 bytes of X, against NB x PN x 128 x 128 multiply-adds: the
+// two-band shape moves the fewest bytes per product, one band x 128 tokens
+// the most; the choice weighs that against the number of CTA waves.  A 2:4
+// tile moves the hybrid format's bytes and costs half a dense tile's tensor
+// work.  Every wait is bounded; one that runs out sets kStatusTimeout in the
+// status word and the CTA leaves its pipeline.
 #include "hyb_internal.cuh"
 
 namespace hyb {
