@@ -504,6 +504,11 @@ __global__ void __launch_bounds__(TmaCfg<BP, B1, B2, LR, PAT>::kThreads, 1)
         s_range[1] = ((int64_t)(c + 1) * p.T + G - 1) / G;
       }
     }
+    // this warp's entries of the 4:8 selector table (the other warps fill
+    // theirs below); like the barriers, they are published by bar.arrive 1
+    if constexpr (PAT == 1) {
+      for (int m = tid; m < 256; m += blockDim.x) lut48[m] = lut48_entry((uint32_t)m);
+    }
     __syncwarp();
     asm volatile("bar.arrive 1, %0;" ::"r"(C::kThreads) : "memory");
   } else {

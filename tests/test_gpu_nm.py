@@ -113,6 +113,41 @@ def test_spmm_nm_strided_operands(orc):
     assert bool((Ys[:, :4] == 7.0).all()) and bool((Ys[:, 4 + n:] == 7.0).all())
 
 
+_FRESH = """
+import sys, numpy as np, torch
+sys.path.insert(0, sys.argv[1])
+from sparse_weight_b200 import hyb, inputs
+n, k, b1, b2, batch = 512, 512, 64, 64, 3
+tmap = inputs.tile_map_fraction((n // b1) * (k // b2), 0.5, inputs.seed_of("nm_fresh"))
+W = inputs.weight(n, k, 0.02, inputs.seed_of("nm_fresh", "W")).to("cuda")
+X = inputs.activations(batch, k, inputs.seed_of("nm_fresh", "X")).to("cuda")
+P = hyb.pack_nm(W, tmap, b1, b2, 4, 8)
+Y = hyb.spmm_skinny_nm(P, X, 4, 8)
+torch.cuda.synchronize()
+np.save(sys.argv[2], Y.cpu().numpy())
+"""
+
+
+def test_spmm_nm_4of8_first_product_of_a_process(orc, tmp_path):
+    """The 4:8 selector table in shared memory is whole in every CTA: with
+    64-row tiles the producer warp's threads own table entries too.  Run as
+    the first product of a fresh process (no earlier kernel has left a table
+    in shared memory), a 64 x 64-tile 4:8 product matches the oracle."""
+    import os
+    import subprocess
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    out = str(tmp_path / "y.npy")
+    subprocess.run([sys.executable, "-c", _FRESH, root, out], check=True, timeout=300)
+    n, k, b1, b2, batch = 512, 512, 64, 64, 3
+    tmap = inputs.tile_map_fraction((n // b1) * (k // b2), 0.5, inputs.seed_of("nm_fresh"))
+    W = inputs.weight(n, k, 0.02, inputs.seed_of("nm_fresh", "W"))
+    X = inputs.activations(batch, k, inputs.seed_of("nm_fresh", "X"))
+    ref = orc.pack_nm(inputs.bits(W), b1, b2, tmap, 4, 8)
+    y_ref, env = orc.spmv_nm(n, k, b1, b2, 4, 8, tmap, ref, inputs.bits(X))
+    assert_within(np.load(out), y_ref, env, what="4:8 64x64 fresh process")
+
+
 @pytest.mark.parametrize("nk,m", [(4, 8), (2, 8)])
 def test_spmm_nm_bad_offsets_are_flagged(nk, m):
     """A corrupted offset (past the value buffer) is skipped and reported
