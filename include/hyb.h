@@ -259,12 +259,12 @@ HYB_API int hyb_shard_bands(int64_t n, int64_t k, int b1, int b2,
  *      clears it).  Nothing is allocated.  Asynchronous on `stream`.
  * hyb_spmm_prefill takes the CTA shape hyb_prefill_block_shape(n, m)
  * returns; hyb_spmm_prefill_blocked takes it from (block_rows, block_tokens):
- * (128, 128), (128, 256) or (256, 240) (two bands sharing each X tile); (0, 0)
- * = the same choice; anything else is HYB_ERR_INVALID_ARG.  Every shape adds
- * the same products in the same order: Y is bit-identical. */
+ * (128, 128), (128, 256), (256, 240) or (256, 208) (two bands sharing each X
+ * tile); (0, 0) = the same choice; anything else is HYB_ERR_INVALID_ARG.  Every
+ * shape adds the same products in the same order: Y is bit-identical. */
 HYB_API size_t hyb_prefill_workspace_bytes(void);
 /* The CTA shape for an n-row weight and m tokens on the current device: of
- * the three above, the one with the fewest modelled bytes per SM (CTAs
+ * the four above, the one with the fewest modelled bytes per SM (CTAs
  * stream their operands from L2 at about the same rate, so a launch takes
  * its waves of CTAs times the bytes one CTA moves per tile).  Writes
  * *block_rows and *block_tokens; HYB_ERR_INVALID_ARG for n < 128, m < 1 or a

@@ -10,7 +10,7 @@
 // tcgen05.mma and 2:4 tiles through tcgen05.mma.sp:
 //
 //   * A CTA owns NB 128-row bands (1 or 2) and PN tokens (128 or 256 for one
-//     band, 240 for two): one 128 x PN fp32 accumulator per band in tensor
+//     band, 240 or 208 for two): one 128 x PN fp32 accumulator per band in tensor
 //     memory (TMEM, band b from column 256 b), M = 128 weight rows per MMA,
 //     N = PN tokens, K looped over the bands' tiles (128 columns each, in two
 //     halves of 64).  hyb_prefill_block_shape picks the shape per call.
@@ -68,7 +68,7 @@ static_assert(kSValBytes == kAtomBytes, "a 2:4 tile's kept values fill one swizz
 // being the bands' A halves (16 KB each) and then X's (PN x 128 bytes): a
 // whole tile per slot for one band and 128 tokens (3 slots of 64 KB), a half
 // per slot otherwise (4 slots of 48 KB for one band and 256 tokens, 3 slots of
-// 62 KB for two bands and 240 tokens).  TMEM holds the bands' PN-column fp32
+// 62 or 58 KB for two bands and 240 or 208 tokens).  TMEM holds the bands' PN-column fp32
 // accumulators (band b from column 256 b), then 4 metadata columns per
 // metadata slot (8 slots for one band, 4 in the last 16 columns for two).
 template <int PN, int NB>
@@ -675,7 +675,7 @@ int launch_prefill(const PrefillParams &prm, const CUtensorMap &xmap, const CUte
 }
 
 // The CTA shapes (rows, tokens) the kernel is built for.
-constexpr int kShapes[3][2] = {{128, 128}, {128, 256}, {256, 240}};
+constexpr int kShapes[4][2] = {{128, 128}, {128, 256}, {256, 240}, {256, 208}};
 
 }  // namespace
 }  // namespace hyb
@@ -783,7 +783,9 @@ int hyb_spmm_prefill_blocked(const hyb_matrix *A, int64_t m, const uint16_t *X, 
   prm.status = static_cast<uint32_t *>(ws);
 
   cudaStream_t st = (cudaStream_t)stream;
-  if (rows == 256) return launch_prefill<240, 2>(prm, xmap, wmap, spmap, m, st);
+  if (rows == 256)
+    return pn == 240 ? launch_prefill<240, 2>(prm, xmap, wmap, spmap, m, st)
+                     : launch_prefill<208, 2>(prm, xmap, wmap, spmap, m, st);
   return pn == 256 ? launch_prefill<256, 1>(prm, xmap, wmap, spmap, m, st)
                    : launch_prefill<128, 1>(prm, xmap, wmap, spmap, m, st);
 }

@@ -493,7 +493,7 @@ def spmm_prefill(A: Packed, X: torch.Tensor, Y: torch.Tensor = None, ws: torch.T
     return Y
 
 
-PREFILL_SHAPES = ((128, 128), (128, 256), (256, 240))
+PREFILL_SHAPES = ((128, 128), (128, 256), (256, 240), (256, 208))
 
 
 def prefill_block_shape(n: int, m: int):

@@ -86,7 +86,8 @@ def test_prefill_shapes_agree(frac):
 def test_prefill_block_choice():
     """The CTA shape with the fewest modelled bytes per SM: short prompts one
     band x 128 tokens, long ones two bands x 240 tokens (one wave of 144 CTAs
-    for the 4096-row FFN at 2048 tokens on 148 SMs)."""
+    for the 4096-row FFN at 2048 tokens on 148 SMs) or x 208 tokens (the
+    14336-row FFN at 2048 tokens: as many waves as 240, fewer bytes each)."""
     sms = torch.cuda.get_device_properties(dev()).multi_processor_count
     for n, m in ((128, 16), (4096, 512), (4096, 2048), (14336, 2048), (384, 700)):
         assert hyb.prefill_block_shape(n, m) in SHAPES
@@ -94,7 +95,7 @@ def test_prefill_block_choice():
     if sms == 148:
         assert hyb.prefill_block_shape(4096, 512) == (128, 128)
         assert hyb.prefill_block_shape(4096, 2048) == (256, 240)
-        assert hyb.prefill_block_shape(14336, 2048) == (256, 240)
+        assert hyb.prefill_block_shape(14336, 2048) == (256, 208)  # 560 CTAs, 4 waves
     with pytest.raises(hyb.HybError):
         hyb.prefill_block_shape(0, 16)
 
